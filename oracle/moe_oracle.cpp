@@ -1,0 +1,293 @@
+// Oracle for the DeepSeekMoE layer forward — TEST INFRASTRUCTURE ONLY.
+//
+// A plain, slow, obviously correct CPU restatement of what one DeepSeekMoE
+// layer computes, used to check the CUDA path. Only tests/, the package's
+// smoke() entry and bench.py's CPU-baseline leg may load it. It shares no code,
+// header, table or helper with the CUDA library and includes no CUDA header.
+//
+// Sources (the pages this follows):
+//  [V3-notes]  DeepSeek-V3 model.py notes (73biji.xyz/llm_pp_dsv3):
+//              - "DeepSeekMoE 三改进" passage and its total-output equation
+//                h'_t = u_t + FFN_share(u_t) + sum_r g_{i,t} FFN_r(u_t);
+//              - "V3 改进①：无辅助损失负载均衡" (s_{i,t} + b_i enters top-k only);
+//              - "Gate 选专家流程（model.py，五步）" (the five gate steps);
+//              - "MoE 前向四步" (gate -> y[idx] += expert(x[idx]) * w -> + z).
+//  [V2-card]   DeepSeek-V2 model card (aigallery), "架构简图" (160 routed, top-6,
+//              2 shared).
+// The expert body is SwiGLU, W2 (silu(W1 v) * W3 v), with silu(g) = g*sigmoid(g)
+// (the pages only say "FFN"; SwiGLU is the stated reading).
+//
+// Precision: dot products and the FFN are accumulated in double; logits and
+// scores are rounded to fp32; the selection arithmetic of gate steps 2-5
+// (s + b, group score, renormalisation, route_scale) runs in fp32, in the order
+// written below, so that a GPU gate fed the same fp32 scores can be compared
+// index for index.
+//
+// Readings where the pages are silent (each listed in the design doc):
+//  - ties in both top-k's go to the lower index (groups and experts);
+//  - idx is returned in descending key order;
+//  - renormalisation is a config switch (on for sigmoid, off for softmax);
+//  - the group score is the max of the group's keys (AMAX) or the fp32 sum of
+//    its two largest keys (TOP2SUM);
+//  - the bias enters only the selection; the weights gather raw scores.
+//
+// Parity pins for every function here are in tests/test_oracle_pins.py.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+extern "C" {
+
+// Mirrors the fields a caller fixes for one layer. All "auto" choices are
+// resolved by the Python wrapper before the call.
+typedef struct {
+  int32_t n_experts;    // E, routed experts
+  int32_t n_groups;     // G
+  int32_t topk_groups;  // TG
+  int32_t topk;         // k
+  float route_scale;
+  int32_t score_func;   // 0 sigmoid, 1 softmax
+  int32_t dim;          // d
+  int32_t inter;        // I, per-expert SwiGLU hidden size
+  int32_t n_shared;     // S
+  int32_t norm_topk;    // 0/1: divide gathered scores by their sum
+  int32_t group_score;  // 1 AMAX, 2 TOP2SUM (ignored when n_groups == 1)
+  int32_t add_residual; // 0/1: add u_t to the output
+} oracle_cfg;
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+}  // extern "C"
+
+namespace {
+
+// bf16 -> fp32 is exact: the 16 stored bits are the top half of an fp32.
+inline double load_elem(const void* base, int dtype, int64_t i) {
+  if (dtype == 0) return (double)((const float*)base)[i];
+  uint32_t bits = (uint32_t)((const uint16_t*)base)[i] << 16;
+  float f;
+  std::memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+const float kNegInf = -std::numeric_limits<float>::infinity();
+
+// Order used by both top-k's: larger key first, lower index on equal keys.
+struct KeyIdx {
+  float key;
+  int idx;
+};
+inline bool before(const KeyIdx& a, const KeyIdx& b) {
+  if (a.key != b.key) return a.key > b.key;
+  return a.idx < b.idx;
+}
+
+// Gate steps 2-5 for one token, from its fp32 scores s[E] (post score function).
+// Outputs: key[E] (s + b, -inf outside the kept groups), gsc[G], idx[k], w[k],
+// and the two selection margins.
+void select_one(const oracle_cfg& c, const float* s, const float* bias, float* key,
+                float* gsc, int32_t* idx, float* w, float* kth_margin,
+                float* grp_margin) {
+  const int E = c.n_experts, G = c.n_groups, TG = c.topk_groups, k = c.topk;
+  const int gs = E / G;
+
+  // s_{i,t} + b_i takes part in the selection only ("V3 改进①").
+  for (int e = 0; e < E; ++e) key[e] = bias ? (float)(s[e] + bias[e]) : s[e];
+
+  // Group-limited routing ("Gate 选专家流程", steps 2-3).
+  *grp_margin = std::numeric_limits<float>::infinity();
+  if (G > 1) {
+    std::vector<float> grp(gs);
+    for (int g = 0; g < G; ++g) {
+      for (int i = 0; i < gs; ++i) grp[i] = key[g * gs + i];
+      std::sort(grp.begin(), grp.end(), [](float a, float b) { return a > b; });
+      gsc[g] = (c.group_score == 2) ? (float)(grp[0] + grp[1]) : grp[0];
+    }
+    std::vector<KeyIdx> order(G);
+    for (int g = 0; g < G; ++g) order[g] = {gsc[g], g};
+    std::sort(order.begin(), order.end(), before);
+    std::vector<char> keep(G, 0);
+    for (int r = 0; r < TG; ++r) keep[order[r].idx] = 1;
+    if (TG < G) *grp_margin = order[TG - 1].key - order[TG].key;
+    for (int e = 0; e < E; ++e)
+      if (!keep[e / gs]) key[e] = kNegInf;
+  } else if (gsc) {
+    gsc[0] = 0.f;
+  }
+
+  // Global top-k over the masked keys (step 4).
+  std::vector<KeyIdx> order(E);
+  for (int e = 0; e < E; ++e) order[e] = {key[e], e};
+  std::sort(order.begin(), order.end(), before);
+  for (int j = 0; j < k; ++j) idx[j] = order[j].idx;
+  *kth_margin = std::numeric_limits<float>::infinity();
+  if (k < E && order[k].key != kNegInf) *kth_margin = order[k - 1].key - order[k].key;
+
+  // Gather the raw scores, renormalise, times route_scale (step 5).
+  float sum = 0.f;
+  for (int j = 0; j < k; ++j) sum = sum + s[idx[j]];
+  for (int j = 0; j < k; ++j) {
+    float v = s[idx[j]];
+    if (c.norm_topk) v = v / sum;
+    w[j] = v * c.route_scale;
+  }
+}
+
+// One SwiGLU expert on one token, accumulating weight * FFN(u) into acc[d].
+void expert_ffn_acc(const oracle_cfg& c, int dtype, const double* u, const void* w1,
+                    const void* w3, const void* w2, double weight, double* acc) {
+  const int d = c.dim, I = c.inter;
+  std::vector<double> h(I);
+  for (int f = 0; f < I; ++f) {
+    double g = 0.0, v = 0.0;
+    for (int i = 0; i < d; ++i) {
+      g += load_elem(w1, dtype, (int64_t)f * d + i) * u[i];
+      v += load_elem(w3, dtype, (int64_t)f * d + i) * u[i];
+    }
+    double silu = g / (1.0 + std::exp(-g));
+    h[f] = silu * v;
+  }
+  for (int o = 0; o < d; ++o) {
+    double y = 0.0;
+    for (int f = 0; f < I; ++f) y += load_elem(w2, dtype, (int64_t)o * I + f) * h[f];
+    acc[o] += weight * y;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+// Gate logits l = u W_g^T ("DeepSeekMoE 三改进": W_g u_t), double accumulate,
+// rounded to fp32. x [T, d], w_gate [E, d], both row-major in `dtype`.
+int oracle_gate_logits(const oracle_cfg* c, int64_t T, int dtype, const void* x,
+                       const void* w_gate, float* logits) {
+  const int E = c->n_experts, d = c->dim;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t t = 0; t < T; ++t) {
+    std::vector<double> u(d);
+    for (int i = 0; i < d; ++i) u[i] = load_elem(x, dtype, t * d + i);
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int i = 0; i < d; ++i) acc += load_elem(w_gate, dtype, (int64_t)e * d + i) * u[i];
+      logits[t * E + e] = (float)acc;
+    }
+  }
+  return 0;
+}
+
+// Score function ("三改进" item 3 for sigmoid; the traditional-MoE softmax).
+// Computed in double from the fp32 logits, rounded to fp32.
+int oracle_scores(const oracle_cfg* c, int64_t T, const float* logits, float* scores) {
+  const int E = c->n_experts;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    const float* l = logits + t * E;
+    float* s = scores + t * E;
+    if (c->score_func == 0) {
+      for (int e = 0; e < E; ++e) s[e] = (float)(1.0 / (1.0 + std::exp(-(double)l[e])));
+    } else {
+      double m = -std::numeric_limits<double>::infinity();
+      for (int e = 0; e < E; ++e) m = std::max(m, (double)l[e]);
+      double z = 0.0;
+      for (int e = 0; e < E; ++e) z += std::exp((double)l[e] - m);
+      for (int e = 0; e < E; ++e) s[e] = (float)(std::exp((double)l[e] - m) / z);
+    }
+  }
+  return 0;
+}
+
+// Gate steps 2-5 for T tokens from fp32 scores [T, E]. Any output pointer
+// except idx/w may be NULL. gsc is [T, G]; margins are [T].
+int oracle_select(const oracle_cfg* c, int64_t T, const float* scores, const float* bias,
+                  float* keys, float* gsc, int32_t* idx, float* w, float* kth_margin,
+                  float* grp_margin) {
+  const int E = c->n_experts, G = c->n_groups, k = c->topk;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    std::vector<float> key(E), g(G);
+    float km, gm;
+    select_one(*c, scores + t * E, bias, key.data(), g.data(), idx + t * k, w + t * k, &km, &gm);
+    if (keys) std::copy(key.begin(), key.end(), keys + t * E);
+    if (gsc) std::copy(g.begin(), g.end(), gsc + t * G);
+    if (kth_margin) kth_margin[t] = km;
+    if (grp_margin) grp_margin[t] = gm;
+  }
+  return 0;
+}
+
+// The literal MoE forward ("MoE 前向四步", single card) for n_tok selected
+// tokens: y = sum_shared FFN_s(u) + sum_j w_j FFN_{idx_j}(u) [+ u].
+// w1/w3/w2 are arrays of E+S per-expert pointers (routed 0..E-1, shared
+// E..E+S-1); W1/W3 are [I, d], W2 is [d, I]. An expert a token needs must not
+// be NULL (returns -1 otherwise). idx/w are the gate's [T, k] outputs. y is
+// [n_tok, d] double.
+int oracle_forward(const oracle_cfg* c, int64_t T, int dtype, const void* x,
+                   const int32_t* idx, const float* w, const void* const* w1,
+                   const void* const* w3, const void* const* w2, int64_t n_tok,
+                   const int64_t* tok_ids, double* y) {
+  const int d = c->dim, k = c->topk, E = c->n_experts, S = c->n_shared;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t n = 0; n < n_tok; ++n) {
+    const int64_t t = tok_ids[n];
+    if (t < 0 || t >= T) { bad |= 1; continue; }
+    std::vector<double> u(d), acc(d, 0.0);
+    for (int i = 0; i < d; ++i) u[i] = load_elem(x, dtype, t * d + i);
+    for (int s = 0; s < S; ++s) {
+      const int e = E + s;
+      if (!w1[e] || !w3[e] || !w2[e]) { bad |= 1; continue; }
+      expert_ffn_acc(*c, dtype, u.data(), w1[e], w3[e], w2[e], 1.0, acc.data());
+    }
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[t * k + j];
+      if (e < 0 || e >= E || !w1[e] || !w3[e] || !w2[e]) { bad |= 1; continue; }
+      expert_ffn_acc(*c, dtype, u.data(), w1[e], w3[e], w2[e], (double)w[t * k + j], acc.data());
+    }
+    if (c->add_residual)
+      for (int i = 0; i < d; ++i) acc[i] += u[i];
+    std::copy(acc.begin(), acc.end(), y + n * d);
+  }
+  return bad ? -1 : 0;
+}
+
+// One expert's SwiGLU hidden vector h = silu(W1 u) * W3 u for n_tok tokens,
+// double. h is [n_tok, I]. Used to localise a mismatch to the first GEMM.
+int oracle_expert_hidden(const oracle_cfg* c, int64_t T, int dtype, const void* x,
+                         const void* w1, const void* w3, int64_t n_tok,
+                         const int64_t* tok_ids, double* h) {
+  const int d = c->dim, I = c->inter;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t n = 0; n < n_tok; ++n) {
+    const int64_t t = tok_ids[n];
+    if (t < 0 || t >= T) { bad |= 1; continue; }
+    std::vector<double> u(d);
+    for (int i = 0; i < d; ++i) u[i] = load_elem(x, dtype, t * d + i);
+    for (int f = 0; f < I; ++f) {
+      double g = 0.0, v = 0.0;
+      for (int i = 0; i < d; ++i) {
+        g += load_elem(w1, dtype, (int64_t)f * d + i) * u[i];
+        v += load_elem(w3, dtype, (int64_t)f * d + i) * u[i];
+      }
+      h[n * I + f] = g / (1.0 + std::exp(-g)) * v;
+    }
+  }
+  return bad ? -1 : 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,223 @@
+"""Oracle for the DeepSeekMoE layer forward — TEST INFRASTRUCTURE ONLY.
+
+Thin ctypes wrapper around ``moe_oracle.cpp`` (plain C++17, fp64, OpenMP).
+Only ``tests/``, the package's ``smoke()`` entry and ``bench.py``'s CPU-baseline
+leg may import this module. It imports nothing from the CUDA package and the
+CUDA package imports nothing from here; the two meet only through the seeded
+input generators, which hold none of the method's arithmetic.
+
+What each function computes, and the page passage it follows, is stated in the
+C++ source. Parity pins for every function are in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.cpp")
+_LIB = os.path.join(_HERE, "libmoe_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+SIGMOID, SOFTMAX = 0, 1
+AMAX, TOP2SUM = 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (IEEE arithmetic: no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["g++", "-std=c++17", "-O2", "-fopenmp", "-fPIC", "-shared",
+               "-ffp-contract=off", "-fno-fast-math", "-o", tmp, _SRC]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("n_experts", ctypes.c_int32), ("n_groups", ctypes.c_int32),
+                ("topk_groups", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("route_scale", ctypes.c_float), ("score_func", ctypes.c_int32),
+                ("dim", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32), ("norm_topk", ctypes.c_int32),
+                ("group_score", ctypes.c_int32), ("add_residual", ctypes.c_int32)]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64 = ctypes.c_int64
+            CP = ctypes.POINTER(_Cfg)
+            lib.oracle_gate_logits.argtypes = [CP, I64, ctypes.c_int, P, P, P]
+            lib.oracle_scores.argtypes = [CP, I64, P, P]
+            lib.oracle_select.argtypes = [CP, I64, P, P, P, P, P, P, P, P]
+            lib.oracle_forward.argtypes = [CP, I64, ctypes.c_int, P, P, P, P, P, P, I64, P, P]
+            lib.oracle_expert_hidden.argtypes = [CP, I64, ctypes.c_int, P, P, P, I64, P, P]
+            lib.oracle_num_threads.argtypes = []
+            lib.oracle_num_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def resolve(cfg: dict, has_bias: bool) -> dict:
+    """Resolve the config's automatic choices.
+
+    norm_topk = -1: renormalise iff sigmoid scoring (the V3 gate renormalises;
+    the V2-style softmax configs do not). group_score = 0 (auto): the sum of the
+    top-2 keys when a bias exists, else the group max ("Gate 选专家流程", step 2).
+    """
+    out = dict(cfg)
+    if out.get("norm_topk", -1) < 0:
+        out["norm_topk"] = 1 if out["score_func"] == SIGMOID else 0
+    if out.get("group_score", 0) == 0:
+        out["group_score"] = TOP2SUM if has_bias else AMAX
+    out.setdefault("add_residual", 0)
+    return out
+
+
+def _cfg_struct(cfg: dict) -> _Cfg:
+    return _Cfg(int(cfg["n_experts"]), int(cfg["n_groups"]), int(cfg["topk_groups"]),
+                int(cfg["topk"]), float(cfg["route_scale"]), int(cfg["score_func"]),
+                int(cfg["dim"]), int(cfg["inter"]), int(cfg["n_shared"]),
+                int(cfg["norm_topk"]), int(cfg["group_score"]), int(cfg.get("add_residual", 0)))
+
+
+def _as_raw(a):
+    """Return (contiguous numpy array, dtype code): 0 = fp32, 1 = bf16 bits."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach()
+            if a.device.type != "cpu":
+                a = a.cpu()
+            a = a.contiguous()
+            if a.dtype == torch.bfloat16:
+                return a.view(torch.int16).numpy().view(np.uint16), 1
+            if a.dtype == torch.float32:
+                return a.numpy(), 0
+            raise TypeError(f"unsupported dtype {a.dtype}")
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a, 0
+    if a.dtype == np.uint16:
+        return a, 1
+    raise TypeError(f"unsupported dtype {a.dtype}")
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def gate_logits(cfg: dict, x, w_gate) -> np.ndarray:
+    """fp32 logits [T, E] = x W_g^T, accumulated in double."""
+    xa, dt = _as_raw(x)
+    wa, dt2 = _as_raw(w_gate)
+    assert dt == dt2
+    T = xa.shape[0]
+    out = np.empty((T, cfg["n_experts"]), np.float32)
+    c = _cfg_struct(resolve(cfg, False))
+    _load().oracle_gate_logits(ctypes.byref(c), T, dt, _ptr(xa), _ptr(wa), _ptr(out))
+    return out
+
+
+def scores(cfg: dict, logits: np.ndarray) -> np.ndarray:
+    logits = np.ascontiguousarray(logits, np.float32)
+    out = np.empty_like(logits)
+    c = _cfg_struct(resolve(cfg, False))
+    _load().oracle_scores(ctypes.byref(c), logits.shape[0], _ptr(logits), _ptr(out))
+    return out
+
+
+def select(cfg: dict, s: np.ndarray, bias=None) -> dict:
+    """Gate steps 2-5 from fp32 scores [T, E]; bias [E] fp32 or None."""
+    s = np.ascontiguousarray(s, np.float32)
+    T, E = s.shape
+    rc = resolve(cfg, bias is not None)
+    G, k = rc["n_groups"], rc["topk"]
+    b = None if bias is None else np.ascontiguousarray(_as_raw(bias)[0], np.float32)
+    out = dict(keys=np.empty((T, E), np.float32), gsc=np.empty((T, G), np.float32),
+               idx=np.empty((T, k), np.int32), w=np.empty((T, k), np.float32),
+               kth_margin=np.empty(T, np.float32), grp_margin=np.empty(T, np.float32))
+    c = _cfg_struct(rc)
+    _load().oracle_select(ctypes.byref(c), T, _ptr(s), _ptr(b), _ptr(out["keys"]),
+                          _ptr(out["gsc"]), _ptr(out["idx"]), _ptr(out["w"]),
+                          _ptr(out["kth_margin"]), _ptr(out["grp_margin"]))
+    return out
+
+
+def gate(cfg: dict, x, w_gate, bias=None) -> dict:
+    """The whole gate: logits, scores, keys, group scores, idx, w and margins."""
+    l = gate_logits(cfg, x, w_gate)
+    s = scores(cfg, l)
+    out = select(cfg, s, bias)
+    out["logits"] = l
+    out["scores"] = s
+    return out
+
+
+def forward(cfg: dict, x, idx: np.ndarray, w: np.ndarray, w1, w3, w2, tok_ids,
+            has_bias: bool) -> np.ndarray:
+    """Literal loop for the tokens in ``tok_ids``; returns y [n, d] float64.
+
+    w1/w3/w2 are sequences of E+S per-expert weights (None where unused) or
+    stacked [E+S, ...] tensors.
+    """
+    xa, dt = _as_raw(x)
+    T = xa.shape[0]
+    rc = resolve(cfg, has_bias)
+    n_all = rc["n_experts"] + rc["n_shared"]
+    keep = []
+
+    def ptrs(ws):
+        arr = (ctypes.c_void_p * n_all)()
+        for e in range(n_all):
+            we = ws[e]
+            if we is None:
+                arr[e] = None
+                continue
+            a, d2 = _as_raw(we)
+            assert d2 == dt, "weights and activations must share a dtype"
+            keep.append(a)
+            arr[e] = a.ctypes.data
+        return arr
+
+    p1, p3, p2 = ptrs(w1), ptrs(w3), ptrs(w2)
+    idx = np.ascontiguousarray(idx, np.int32)
+    w = np.ascontiguousarray(w, np.float32)
+    tok = np.ascontiguousarray(np.asarray(tok_ids, np.int64))
+    y = np.empty((tok.shape[0], rc["dim"]), np.float64)
+    c = _cfg_struct(rc)
+    rcode = _load().oracle_forward(ctypes.byref(c), T, dt, _ptr(xa), _ptr(idx), _ptr(w),
+                                   p1, p3, p2, tok.shape[0], _ptr(tok), _ptr(y))
+    if rcode != 0:
+        raise ValueError("oracle_forward: bad token id or missing expert weights")
+    return y
+
+
+def expert_hidden(cfg: dict, x, w1_e, w3_e, tok_ids) -> np.ndarray:
+    """h = silu(W1 u) * W3 u for one expert, [n, I] float64."""
+    xa, dt = _as_raw(x)
+    a1, _ = _as_raw(w1_e)
+    a3, _ = _as_raw(w3_e)
+    tok = np.ascontiguousarray(np.asarray(tok_ids, np.int64))
+    h = np.empty((tok.shape[0], cfg["inter"]), np.float64)
+    c = _cfg_struct(resolve(cfg, False))
+    rcode = _load().oracle_expert_hidden(ctypes.byref(c), xa.shape[0], dt, _ptr(xa), _ptr(a1),
+                                         _ptr(a3), tok.shape[0], _ptr(tok), _ptr(h))
+    if rcode != 0:
+        raise ValueError("oracle_expert_hidden: bad token id")
+    return h
