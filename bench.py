@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Throughput of the DeepSeekMoE layer forward on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one kt_moe_forward of the V3-shaped prefill layer (T = 8192 tokens,
+Zipf(1.1) expert load, bf16) with inputs resident in HBM; the same run also
+measures the V3-shaped decode step (T = 8) and prints it under "decode". With N
+GPUs every rank runs its own replica on its own tokens (data parallel over
+tokens, no collective on the data path): weak scaling, timed on the device as
+the max over ranks.
+
+Rank 0 prints one JSON line. `value` is tokens/s of the whole job; `e2e` is the
+same metric with host buffers (pinned x copied in and y copied out every step);
+`roofline` is the dominant kernel (the gate/up expert GEMM) against the measured
+bf16 tensor peak; `cpu_baseline` is the CPU oracle timed on a sample of the
+same workload on this host's cores. `--impl reference` times the oracle alone
+(rank 0 only) in the same JSON form.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_34_b200 import workloads as W  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+LAUNCHES_PER_FORWARD = 7   # logits, select, scan, scatter, up GEMM, down GEMM, combine
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=W.V3_PREFILL.name)
+    ap.add_argument("--decode-workload", default=W.V3_DECODE.name, help="'none' to skip")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target wall time of the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+# ---------------------------------------------------------------------------
+# Process group (only for barriers and the max-over-ranks of device times)
+# ---------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=300))
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_tokens_seed(layer, rank: int) -> int:
+    """Each rank routes its own tokens; weights and bias are the same everywhere."""
+    return layer.seed * 1000 + rank
+
+
+# ---------------------------------------------------------------------------
+# Peaks, clocks
+# ---------------------------------------------------------------------------
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 100 ms while the timed work runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        power = [float(r[3]) if r[3].replace(".", "").isdigit() else 0.0 for r in rows]
+        loaded = [s for s, p in zip(sm, power) if p > 0.3 * max(power)] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work (per launch), stated in the design doc
+# ---------------------------------------------------------------------------
+def algorithmic(layer, idx: np.ndarray) -> dict:
+    T, d, I, k, S, E = layer.T, layer.dim, layer.inter, layer.topk, layer.n_shared, layer.n_experts
+    es = 4 if layer.dtype == "f32" else 2
+    R = T * (k + S)
+    active = int((np.bincount(idx.ravel(), minlength=E) > 0).sum()) + S
+    return {
+        "rows": R,
+        "active_experts": active,
+        "flops_layer": W.flops_per_token(layer) * T,
+        "flops_up": 4 * d * I * R,
+        "flops_down": 2 * d * I * R,
+        # bytes the method must move: activated experts' weights, W_gate, x, y
+        "bytes_layer": active * 3 * d * I * es + E * d * es + 2 * T * d * es,
+        # gate/up GEMM: W1, W3 of active experts, the token rows in, hidden rows out
+        "bytes_up": active * 2 * d * I * es + R * d * es + R * I * es,
+    }
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps):
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    inp = W.make_layer(layer, dev)
+    if rank > 0:
+        g = torch.Generator(device="cpu").manual_seed(rank_tokens_seed(layer, rank))
+        inp["x"] = torch.randn(inp["x"].shape, generator=g).to(inp["x"].dtype).to(dev)
+    cfg = K.config_for(layer)
+    T = layer.T
+    ws = K.alloc_workspace(cfg, T, dev)
+    y = torch.empty((T, layer.dim), dtype=inp["x"].dtype, device=dev)
+    idx = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
+    w = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
+    args = (cfg, T, inp["x"], inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], y, idx, w, ws)
+
+    for _ in range(warmup):
+        K.kt_moe_forward(*args)
+    rc = K.kt_moe_check(ws)
+    if rc != K.KT_OK:
+        raise RuntimeError(f"device error after warm-up: {K.strerror(rc)}")
+
+    # Stage events, created (recorded once) before the timed region.
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(K.KT_STAGE_EVENTS)]
+          for _ in range(steps)]
+    for row in ev:
+        for e in row:
+            e.record()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record()
+    for s in range(steps):
+        K.kt_moe_forward_profiled(*args, ev[s])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = t0.elapsed_time(t1)
+    rc = K.kt_moe_check(ws)
+    if rc != K.KT_OK:
+        raise RuntimeError(f"device error in the timed region: {K.strerror(rc)}")
+    stage_ms = {name: statistics.fmean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps))
+                for i, name in enumerate(K.STAGES)}
+    ms_max = max_over_ranks(ms, world, dev)
+
+    # End to end through the same C ABI call, host buffers: pinned x in, y out.
+    x_h = inp["x"].cpu().pin_memory()
+    y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    x_d = torch.empty_like(inp["x"])
+    eargs = list(args)
+    eargs[2] = x_d
+    for _ in range(3):
+        x_d.copy_(x_h, non_blocking=True)
+        K.kt_moe_forward(*eargs)
+        y_h.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(e2e_steps):
+        x_d.copy_(x_h, non_blocking=True)
+        K.kt_moe_forward(*eargs)
+        y_h.copy_(y, non_blocking=True)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+
+    work = algorithmic(layer, idx.cpu().numpy())
+    out = dict(inp=inp, idx=idx.cpu().numpy(), ms=ms_max, stage_ms=stage_ms, e2e_ms=e2e_ms,
+               work=work, h2d=inp["x"].numel() * inp["x"].element_size(),
+               d2h=y.numel() * y.element_size())
+    del ws, y
+    return out
+
+
+def cpu_oracle_sample(layer, inp, idx_all, target_s: float) -> dict:
+    """Time the CPU oracle (gate + literal expert loop) on the first n tokens."""
+    import oracle.oracle as O
+    kf = layer.kernel_fields()
+    threads = O.num_threads()
+    x_h = inp["x"].cpu()
+    wg_h = inp["w_gate"].cpu()
+    bias = None if inp["bias"] is None else inp["bias"].float().cpu().numpy()
+    E, S = layer.n_experts, layer.n_shared
+    host_w = {}
+
+    def run(n):
+        need = set(range(E, E + S)) | set(int(e) for e in idx_all[:n].ravel())
+        for e in need - set(host_w):
+            host_w[e] = (inp["w1"][e].cpu(), inp["w3"][e].cpu(), inp["w2"][e].cpu())
+        w1 = [host_w[e][0] if e in host_w else None for e in range(E + S)]
+        w3 = [host_w[e][1] if e in host_w else None for e in range(E + S)]
+        w2 = [host_w[e][2] if e in host_w else None for e in range(E + S)]
+        xs = x_h[:n].contiguous()
+        t = time.perf_counter()
+        g = O.gate(kf, xs, wg_h, bias)
+        O.forward(kf, xs, g["idx"], g["w"], w1, w3, w2, range(n), bias is not None)
+        return time.perf_counter() - t
+
+    n = max(1, min(layer.T, threads))
+    dt = run(n)
+    if dt < 0.5 * target_s and n < layer.T:
+        n = int(min(layer.T, max(n + 1, n * target_s / max(dt, 1e-3)), 16 * threads))
+        dt = run(n)
+    return {"value": n / dt, "unit": "tokens/s", "cores": min(threads, n), "kind": "oracle",
+            "sample": f"first {n} tokens of {layer.name}: fp64 gate + literal expert loop "
+                      f"({dt:.1f} s)"}
+
+
+def run_ours(a):
+    rank, world, local = dist_env()
+    if world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    K.lib()   # fail loudly if the CUDA library is missing
+    peaks = load_peaks()
+    layer = W.BY_NAME[a.workload]
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    pre = time_layer(layer, dev, rank, world, a.steps, a.warmup, a.e2e_steps)
+    dec = None
+    if a.decode_workload != "none":
+        dlayer = W.BY_NAME[a.decode_workload]
+        dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps)
+    clk = clocks.stop()
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_oracle_sample(layer, pre["inp"], pre["idx"], a.cpu_seconds)
+    pre.pop("inp")
+    if dec:
+        dec.pop("inp")
+    torch.cuda.empty_cache()
+
+    if rank == 0:
+        T, K_ = layer.T, a.steps
+        tokens = world * T * K_
+        value = tokens / (pre["ms"] / 1e3)
+        up_ms = pre["stage_ms"]["up_gemm"]
+        achieved = pre["work"]["flops_up"] / (up_ms / 1e3) / 1e12
+        line = {
+            "metric": "MoE layer tokens/s (prefill T=8192, decode T=8) + % of HBM/tensor roofline",
+            "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K_,
+            "warmup": a.warmup, "ms_per_step": round(pre["ms"] / K_, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init weights of the V3 layer shape)",
+            "impl": "ours",
+            "config": {"workload": layer.name, "T": T, "dim": layer.dim, "experts": layer.n_experts,
+                       "groups": f"{layer.n_groups}/{layer.topk_groups}", "topk": layer.topk,
+                       "shared": layer.n_shared, "inter": layer.inter,
+                       "load": "Zipf(1.1)", "parallelism": f"dp{world} (replicas, no collective)",
+                       "l2": "inputs larger than L2: ~22 GB of expert weights read per step"},
+            "stage_ms": {k: round(v, 4) for k, v in pre["stage_ms"].items()},
+            "layer_tflops": round(pre["work"]["flops_layer"] / (pre["ms"] / K_ / 1e3) / 1e12, 1),
+            "roofline": {"kernel": "grouped gate/up GEMM (tcgen05)", "bound": "tensor",
+                         "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                         "traffic": None, "peak_source": peaks["source"] + " (burst)"},
+            "e2e": {"value": round(world * T * a.e2e_steps / (pre["e2e_ms"] / 1e3), 1),
+                    "unit": "tokens/s", "h2d_bytes_per_step": pre["h2d"],
+                    "d2h_bytes_per_step": pre["d2h"]},
+            "gpu_launches": LAUNCHES_PER_FORWARD * K_,
+            "cpu_baseline": cpu,
+            "clocks": clk,
+        }
+        if dec:
+            dl = W.BY_NAME[a.decode_workload]
+            dms = dec["ms"] / a.steps
+            up_bytes = dec["work"]["bytes_up"]
+            up_gbs = up_bytes / (dec["stage_ms"]["up_gemm"] / 1e3) / 1e9
+            layer_gbs = dec["work"]["bytes_layer"] / (dms / 1e3) / 1e9
+            line["decode"] = {
+                "workload": dl.name, "value": round(world * dl.T / (dms / 1e3), 1),
+                "unit": "tokens/s", "ms_per_step": round(dms, 4),
+                "active_experts": dec["work"]["active_experts"],
+                "stage_ms": {k: round(v, 4) for k, v in dec["stage_ms"].items()},
+                "layer_hbm_gbs": round(layer_gbs, 1),
+                "layer_hbm_frac": round(layer_gbs / peaks["hbm_gbs"], 4),
+                "roofline": {"kernel": "grouped gate/up GEMM (tcgen05)", "bound": "hbm",
+                             "achieved": round(up_gbs, 1), "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(up_gbs / peaks["hbm_gbs"], 4),
+                             "traffic": None},
+                "e2e": {"value": round(world * dl.T * a.e2e_steps / (dec["e2e_ms"] / 1e3), 1),
+                        "unit": "tokens/s"},
+            }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the CPU oracle, rank 0 only
+# ---------------------------------------------------------------------------
+def run_reference(a):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    import oracle.oracle as O
+    layer = W.BY_NAME[a.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    threads = O.num_threads()
+    n = max(1, min(layer.T, threads))
+    gi = W.make_gate_inputs(layer)
+    kf = layer.kernel_fields()
+    bias = None if gi["bias"] is None else gi["bias"].numpy()
+    xs = gi["x"][:n].contiguous()
+    g = O.gate(kf, xs, gi["w_gate"], bias)
+    need = set(range(layer.n_experts, layer.n_experts + layer.n_shared)) | set(g["idx"].ravel().tolist())
+    full = W.make_layer(layer, dev)
+    nall = layer.n_experts + layer.n_shared
+    w1 = [full["w1"][e].cpu() if e in need else None for e in range(nall)]
+    w3 = [full["w3"][e].cpu() if e in need else None for e in range(nall)]
+    w2 = [full["w2"][e].cpu() if e in need else None for e in range(nall)]
+    del full
+
+    def step():
+        gg = O.gate(kf, xs, gi["w_gate"], bias)
+        O.forward(kf, xs, gg["idx"], gg["w"], w1, w3, w2, range(n), bias is not None)
+
+    for _ in range(a.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(a.steps):
+        step()
+    dt = time.perf_counter() - t
+    value = n * a.steps / dt
+    sample = f"first {n} tokens of {layer.name} per step: fp64 gate + literal expert loop"
+    print(json.dumps({
+        "metric": "MoE layer tokens/s (prefill T=8192, decode T=8) + % of HBM/tensor roofline",
+        "value": round(value, 3), "unit": "tokens/s", "n_gpus": a.gpus, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(dt / a.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": layer.name, "T": layer.T, "sample_tokens_per_step": n},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": min(threads, n),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    a = parse_args(argv)
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+/*
+ * ktmoe.h — C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ *
+ * One DeepSeekMoE layer computes, per token u_t (the total-output equation of
+ * the "DeepSeekMoE 三改进" passage of the DeepSeek-V3 model.py notes,
+ * 73biji.xyz/llm_pp_dsv3):
+ *
+ *     h'_t = [u_t +] sum_{shared s} FFN_s(u_t) + sum_{j<k} g_{j,t} FFN_{idx_j}(u_t)
+ *
+ * with FFN(v) = W2 (silu(W1 v) * W3 v) (SwiGLU; the pages only say "FFN") and
+ * the routing (idx, g) of the same page's "Gate 选专家流程（model.py，五步）":
+ *   1. s = sigmoid(W_g u) (or softmax over all experts), kept raw;
+ *   2. keys s + b (bias b only where the layer has one, "V3 改进①"); group score
+ *      = max of the group's keys (no bias) or the sum of its two largest keys
+ *      (with bias);
+ *   3. keep the topk_groups best groups, other experts' keys := -inf;
+ *   4. global top-k over the keys;
+ *   5. gather the raw s at the chosen experts, renormalise, times route_scale.
+ * Ties in both top-k's go to the lower index; idx is in descending key order.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named "device" are caller-owned CUDA device memory; the library
+ *    never allocates, frees or retains them. Host pointers are read only during
+ *    the call.
+ *  - `stream` is a cudaStream_t (0 = legacy default stream). Calls only enqueue
+ *    work on it and return without synchronising, except kt_moe_check.
+ *  - Layouts are row-major. Activations and expert weights share one dtype
+ *    (kt_moe_config.dtype); the bias and routing weights are always fp32.
+ *  - Expert weights are stacked, routed experts 0..E-1 then shared experts
+ *    E..E+S-1, each in nn.Linear [out, in] order:
+ *        w1, w3 : [E+S, inter, dim]   (gate and up projections)
+ *        w2     : [E+S, dim, inter]   (down projection)
+ *  - Return value: KT_OK (0) or a negative KT_ERR_* code. Host-side checks run
+ *    before anything is enqueued; on an error return nothing was enqueued.
+ *  - The library keeps no state between calls; a call's scratch lives in the
+ *    caller's workspace, so concurrent calls need distinct workspaces.
+ */
+#ifndef KTMOE_H
+#define KTMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Score function of gate step 1. */
+enum { KT_SCORE_SIGMOID = 0, KT_SCORE_SOFTMAX = 1 };
+/* Group score of gate step 2. AUTO = TOP2SUM when a bias is given, else AMAX. */
+enum { KT_GROUP_AUTO = 0, KT_GROUP_AMAX = 1, KT_GROUP_TOP2SUM = 2 };
+/* Activation / expert-weight dtype. */
+enum { KT_DTYPE_F32 = 0, KT_DTYPE_BF16 = 1 };
+
+enum {
+  KT_OK = 0,
+  KT_ERR_INVALID_CONFIG = -1, /* inconsistent config or token count               */
+  KT_ERR_NULL = -2,           /* a required pointer is NULL                         */
+  KT_ERR_WORKSPACE = -3,      /* workspace NULL or smaller than kt_moe_workspace_size */
+  KT_ERR_ALIGN = -4,          /* a pointer is not 16-byte aligned (workspace: 256)  */
+  KT_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed               */
+  KT_ERR_TIMEOUT = -6,        /* a bounded device-side wait gave up (kt_moe_check)  */
+  KT_ERR_UNSUPPORTED = -7     /* no sm_100 device, or a size beyond a kernel limit  */
+};
+
+/*
+ * Layer description. The first six fields are the gate's parameters named by
+ * the "Gate 选专家流程" passage (n_groups, topk_groups, topk, route_scale and
+ * the sigmoid/softmax score); the rest are shapes and switches.
+ *
+ * Limits (KT_ERR_INVALID_CONFIG otherwise): 1 <= n_experts <= 512;
+ * n_experts % n_groups == 0; 1 <= topk_groups <= n_groups <= 32;
+ * 1 <= topk <= min(32, topk_groups * n_experts / n_groups); n_groups == 1
+ * implies topk_groups == 1; TOP2SUM needs >= 2 experts per group;
+ * 0 <= n_shared <= 8; route_scale finite and > 0; dim, inter >= 8 and
+ * multiples of 8 (bf16) or 4 (fp32), so rows are 16-byte multiples.
+ */
+typedef struct {
+  int32_t n_experts;    /* E: routed experts                                      */
+  int32_t n_groups;     /* G: expert groups (1 = no group limit)                   */
+  int32_t topk_groups;  /* TG: groups kept per token                              */
+  int32_t topk;         /* k: routed experts per token                            */
+  float route_scale;    /* multiplies the routing weights (2.5 in DeepSeek-V3)     */
+  int32_t score_func;   /* KT_SCORE_SIGMOID or KT_SCORE_SOFTMAX                    */
+  int32_t dim;          /* d: hidden size                                         */
+  int32_t inter;        /* I: SwiGLU hidden size of one expert                     */
+  int32_t n_shared;     /* S: always-on shared experts (weight 1)                  */
+  int32_t norm_topk;    /* -1 auto (renormalise iff sigmoid), 0 off, 1 on          */
+  int32_t group_score;  /* KT_GROUP_*                                              */
+  int32_t dtype;        /* KT_DTYPE_*                                              */
+  int32_t add_residual; /* 1: add u_t to the output (h'_t); 0: MoE-module output   */
+} kt_moe_config;
+
+/* Host-only validation of a config for T tokens (T >= 1, T <= 2^20). No CUDA
+ * call. `has_bias` says whether a bias will be passed (it decides AUTO group
+ * scoring). Returns KT_OK or KT_ERR_INVALID_CONFIG. */
+int kt_moe_validate(const kt_moe_config* cfg, int64_t T, int has_bias);
+
+/* Bytes of device workspace kt_moe_gate / kt_moe_forward need for T tokens
+ * (0 if the config is invalid). No CUDA call. */
+size_t kt_moe_workspace_size(const kt_moe_config* cfg, int64_t T);
+
+/*
+ * Gate only (steps 1-5 above).
+ *   x        device [T, dim] (dtype)           tokens u_t
+ *   w_gate   device [E, dim] (dtype)           gate weights W_g
+ *   bias     device [E] fp32 or NULL           per-expert selection bias b
+ *   scores_in device [T, E] fp32 or NULL       if given, used as the scores s
+ *            (post score function) and x / w_gate are not read (may be NULL):
+ *            the selection steps 2-5 alone, for index-exact comparisons
+ *   topk_idx device [T, k] int32  (out)        chosen experts, descending key
+ *   topk_w   device [T, k] fp32   (out)        routing weights g
+ *   workspace device, ws_bytes >= kt_moe_workspace_size(cfg, T), 256-B aligned
+ * Logits accumulate in fp32; the selection arithmetic is fp32 in the order of
+ * steps 2-5 (s + b; group max or top-2 sum; sum of gathered scores in slot
+ * order; division; times route_scale).
+ */
+int kt_moe_gate(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                const float* bias, const float* scores_in, int32_t* topk_idx,
+                float* topk_w, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The whole layer forward.
+ *   x, w_gate, bias    as for kt_moe_gate
+ *   w1, w3             device [E+S, inter, dim] (dtype)
+ *   w2                 device [E+S, dim, inter] (dtype)
+ *   y                  device [T, dim] (dtype) (out); must not alias x
+ *   topk_idx_out       device [T, k] int32 or NULL: the routing, if wanted
+ *   topk_w_out         device [T, k] fp32 or NULL
+ * The output sum runs in a fixed order per token (shared experts in index
+ * order, then the k routed slots in key order, then u_t if add_residual) in
+ * fp32, so repeated calls give bitwise-equal y. bf16 layers keep the SwiGLU
+ * hidden vectors and the weighted expert outputs in bf16 between kernels.
+ */
+int kt_moe_forward(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                   const float* bias, const void* w1, const void* w3, const void* w2,
+                   void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                   size_t ws_bytes, void* stream);
+
+/* kt_moe_forward plus stage timing: `stage_events` points to KT_STAGE_EVENTS
+ * cudaEvent_t handles (entries may be NULL) that are recorded on `stream` at
+ * the stage boundaries, in this order: start, after the gate (logits and
+ * selection), after the token permutation, after the gate/up expert GEMM,
+ * after the down expert GEMM, after the combine. cudaEventElapsedTime between
+ * consecutive events gives each stage's device time. Same arguments, errors
+ * and results as kt_moe_forward otherwise. */
+enum { KT_STAGE_EVENTS = 6 };
+int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
+                            const void* w_gate, const float* bias, const void* w1,
+                            const void* w3, const void* w2, void* y, int32_t* topk_idx_out,
+                            float* topk_w_out, void* workspace, size_t ws_bytes, void* stream,
+                            void* const* stage_events);
+
+/* Synchronise `stream`, then read the device error word the last call on this
+ * workspace left (a bounded wait inside a kernel that gave up sets it).
+ * Returns KT_OK, KT_ERR_TIMEOUT, or KT_ERR_CUDA if the stream reports an error. */
+int kt_moe_check(const void* workspace, void* stream);
+
+/* Byte offsets of the internal buffers inside the workspace, for tests and
+ * debugging (all -1 if the config is invalid). Counts: per-group row counts
+ * [E+S]; offsets: exclusive prefix [E+S+1]; row_of: [T, k] row of (t, j) in the
+ * expert-sorted order; tok_of: [T*k] token of each sorted row; hidden: SwiGLU
+ * hidden rows [T*(k+S), inter] (dtype); expert_out: weighted expert outputs
+ * [T*(k+S), dim] (dtype). Rows T*k + s*T + t belong to shared expert s. */
+typedef struct {
+  int64_t error_word;
+  int64_t logits;
+  int64_t counts;
+  int64_t offsets;
+  int64_t row_of;
+  int64_t tok_of;
+  int64_t row_weight;
+  int64_t hidden;
+  int64_t expert_out;
+  int64_t total;
+} kt_moe_ws_layout;
+
+int kt_moe_workspace_layout(const kt_moe_config* cfg, int64_t T, kt_moe_ws_layout* out);
+
+/* Static description of an error code. */
+const char* kt_moe_strerror(int code);
+
+/* Library version: (major << 16) | minor. */
+int kt_moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KTMOE_H */

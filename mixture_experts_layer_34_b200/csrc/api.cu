@@ -1,0 +1,278 @@
+// C ABI of the B200 DeepSeekMoE layer library: config checks, workspace layout
+// and the launch sequence of one layer forward on the caller's stream.
+//
+//   gate_logits -> gate_select (+ per-chunk expert counts) -> permute_scan ->
+//   permute_scatter (+ permuted x) -> up GEMM -> down GEMM -> combine
+//
+// No host synchronisation happens between the kernels: the per-expert token
+// counts stay on the device, where the scan turns them into the chunk lists
+// the persistent GEMM kernels walk.
+#include <cmath>
+#include <cstring>
+
+#include "ktmoe_internal.cuh"
+
+namespace ktmoe {
+namespace {
+
+constexpr int64_t kMaxTokens = int64_t(1) << 20;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int device_info(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KT_ERR_CUDA;
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return KT_ERR_CUDA;
+  if (major != 10 || minor != 0) return KT_ERR_UNSUPPORTED;   // built for sm_100a only
+  *num_sms = sms;
+  return KT_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+}  // namespace
+
+int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
+  if (!c || !r) return KT_ERR_NULL;
+  if (T < 1 || T > kMaxTokens) return KT_ERR_INVALID_CONFIG;
+  const int E = c->n_experts, G = c->n_groups, TG = c->topk_groups, k = c->topk;
+  if (E < 1 || E > kMaxExperts) return KT_ERR_INVALID_CONFIG;
+  if (G < 1 || G > kMaxGroups || E % G != 0) return KT_ERR_INVALID_CONFIG;
+  if (TG < 1 || TG > G || (G == 1 && TG != 1)) return KT_ERR_INVALID_CONFIG;
+  const int gs = E / G;
+  if (k < 1 || k > kMaxTopk || k > TG * gs) return KT_ERR_INVALID_CONFIG;
+  if (c->n_shared < 0 || c->n_shared > kMaxShared) return KT_ERR_INVALID_CONFIG;
+  if (!std::isfinite(c->route_scale) || !(c->route_scale > 0.f)) return KT_ERR_INVALID_CONFIG;
+  if (c->score_func != KT_SCORE_SIGMOID && c->score_func != KT_SCORE_SOFTMAX)
+    return KT_ERR_INVALID_CONFIG;
+  if (c->dtype != KT_DTYPE_F32 && c->dtype != KT_DTYPE_BF16) return KT_ERR_INVALID_CONFIG;
+  const int align = c->dtype == KT_DTYPE_BF16 ? 8 : 4;
+  if (c->dim < 8 || c->inter < 8 || c->dim % align || c->inter % align) return KT_ERR_INVALID_CONFIG;
+  if (c->dim > (1 << 16) || c->inter > (1 << 16)) return KT_ERR_INVALID_CONFIG;
+  if (c->norm_topk < -1 || c->norm_topk > 1) return KT_ERR_INVALID_CONFIG;
+  if (c->group_score < KT_GROUP_AUTO || c->group_score > KT_GROUP_TOP2SUM) return KT_ERR_INVALID_CONFIG;
+  if (c->add_residual != 0 && c->add_residual != 1) return KT_ERR_INVALID_CONFIG;
+  r->E = E;
+  r->G = G;
+  r->TG = TG;
+  r->k = k;
+  r->S = c->n_shared;
+  r->d = c->dim;
+  r->I = c->inter;
+  r->gs = gs;
+  r->route_scale = c->route_scale;
+  r->score_func = c->score_func;
+  r->norm = c->norm_topk < 0 ? (c->score_func == KT_SCORE_SIGMOID ? 1 : 0) : c->norm_topk;
+  r->group_score = c->group_score == KT_GROUP_AUTO ? (has_bias ? KT_GROUP_TOP2SUM : KT_GROUP_AMAX)
+                                                   : c->group_score;
+  if (G > 1 && r->group_score == KT_GROUP_TOP2SUM && gs < 2) return KT_ERR_INVALID_CONFIG;
+  r->dtype = c->dtype;
+  r->add_residual = c->add_residual;
+  r->has_bias = has_bias ? 1 : 0;
+  return KT_OK;
+}
+
+Layout make_layout(const Resolved& r, int64_t T) {
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes, size_t align) {
+    off = round_up(off, align);
+    const size_t o = off;
+    off += bytes;
+    return o;
+  };
+  const size_t NG = (size_t)(r.E + r.S);
+  const size_t Tk = (size_t)T * r.k;
+  const size_t R = (size_t)T * (r.k + r.S);
+  const size_t es = r.dtype == KT_DTYPE_BF16 ? 2 : 4;
+  L.nperm = (T + kPermChunk - 1) / kPermChunk;
+  L.max_up = (int64_t)(R / kUpChunk + NG + 1);
+  L.max_down = (int64_t)(R / kDownChunk + NG + 1);
+  L.err = take(256, 256);
+  L.meta = take(64, 256);
+  L.logits = take((size_t)T * r.E * 4, 256);
+  L.idx = take(Tk * 4, 256);
+  L.w = take(Tk * 4, 256);
+  L.chunk_counts = take((size_t)L.nperm * r.E * 4, 256);
+  L.chunk_base = take((size_t)L.nperm * r.E * 4, 256);
+  L.counts = take(NG * 4, 256);
+  L.offsets = take((NG + 1) * 4, 256);
+  L.row_of = take(Tk * 4, 256);
+  L.tok_of = take(Tk * 4, 256);
+  L.row_weight = take(Tk * 4, 256);
+  L.up_chunks = take((size_t)L.max_up * sizeof(Chunk), 256);
+  L.down_chunks = take((size_t)L.max_down * sizeof(Chunk), 256);
+  L.xperm = take(r.dtype == KT_DTYPE_BF16 ? Tk * r.d * es : 0, 1024);
+  L.hidden = take(R * r.I * es, 1024);
+  L.expert_out = take(R * r.d * es, 1024);
+  L.total = round_up(off, 1024);
+  return L;
+}
+
+}  // namespace ktmoe
+
+using namespace ktmoe;
+
+extern "C" {
+
+int kt_moe_validate(const kt_moe_config* cfg, int64_t T, int has_bias) {
+  Resolved r;
+  const int rc = resolve(cfg, T, has_bias, &r);
+  return rc == KT_ERR_NULL ? KT_ERR_NULL : (rc == KT_OK ? KT_OK : KT_ERR_INVALID_CONFIG);
+}
+
+size_t kt_moe_workspace_size(const kt_moe_config* cfg, int64_t T) {
+  Resolved r;
+  if (resolve(cfg, T, 0, &r) != KT_OK && resolve(cfg, T, 1, &r) != KT_OK) return 0;
+  return make_layout(r, T).total;
+}
+
+int kt_moe_workspace_layout(const kt_moe_config* cfg, int64_t T, kt_moe_ws_layout* out) {
+  if (!out) return KT_ERR_NULL;
+  Resolved r;
+  if (resolve(cfg, T, 0, &r) != KT_OK && resolve(cfg, T, 1, &r) != KT_OK) {
+    std::memset(out, 0xff, sizeof(*out));
+    return KT_ERR_INVALID_CONFIG;
+  }
+  const Layout L = make_layout(r, T);
+  out->error_word = (int64_t)L.err;
+  out->logits = (int64_t)L.logits;
+  out->counts = (int64_t)L.counts;
+  out->offsets = (int64_t)L.offsets;
+  out->row_of = (int64_t)L.row_of;
+  out->tok_of = (int64_t)L.tok_of;
+  out->row_weight = (int64_t)L.row_weight;
+  out->hidden = (int64_t)L.hidden;
+  out->expert_out = (int64_t)L.expert_out;
+  out->total = (int64_t)L.total;
+  return KT_OK;
+}
+
+int kt_moe_gate(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                const float* bias, const float* scores_in, int32_t* topk_idx, float* topk_w,
+                void* workspace, size_t ws_bytes, void* stream) {
+  Resolved r;
+  int rc = resolve(cfg, T, bias != nullptr, &r);
+  if (rc != KT_OK) return rc;
+  if (!topk_idx || !topk_w) return KT_ERR_NULL;
+  if (!scores_in && (!x || !w_gate)) return KT_ERR_NULL;
+  if (!workspace) return KT_ERR_WORKSPACE;
+  const Layout L = make_layout(r, T);
+  if (ws_bytes < L.total) return KT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
+      (bias && !aligned(bias, 4)) || (scores_in && !aligned(scores_in, 4)) ||
+      (x && !aligned(x, 16)) || (w_gate && !aligned(w_gate, 16)))
+    return KT_ERR_ALIGN;
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+  if (!scores_in) {
+    if (launch_gate_logits(r, T, x, w_gate, logits, err, st) != cudaSuccess) return KT_ERR_CUDA;
+    err = nullptr;   // already reset by the first kernel
+  }
+  if (launch_gate_select(r, T, logits, scores_in, bias, topk_idx, topk_w,
+                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), err, st) != cudaSuccess)
+    return KT_ERR_CUDA;
+  return KT_OK;
+}
+
+int kt_moe_forward(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                   const float* bias, const void* w1, const void* w3, const void* w2, void* y,
+                   int32_t* topk_idx_out, float* topk_w_out, void* workspace, size_t ws_bytes,
+                   void* stream) {
+  return kt_moe_forward_profiled(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                                 workspace, ws_bytes, stream, nullptr);
+}
+
+int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
+                            const void* w_gate, const float* bias, const void* w1,
+                            const void* w3, const void* w2, void* y, int32_t* topk_idx_out,
+                            float* topk_w_out, void* workspace, size_t ws_bytes, void* stream,
+                            void* const* stage_events) {
+  Resolved r;
+  int rc = resolve(cfg, T, bias != nullptr, &r);
+  if (rc != KT_OK) return rc;
+  if (!x || !w_gate || !w1 || !w3 || !w2 || !y) return KT_ERR_NULL;
+  if (!workspace) return KT_ERR_WORKSPACE;
+  const Layout L = make_layout(r, T);
+  if (ws_bytes < L.total) return KT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256) || !aligned(x, 16) || !aligned(w_gate, 16) || !aligned(w1, 16) ||
+      !aligned(w3, 16) || !aligned(w2, 16) || !aligned(y, 16) || (bias && !aligned(bias, 4)) ||
+      (topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
+    return KT_ERR_ALIGN;
+  const size_t es = r.dtype == KT_DTYPE_BF16 ? 2 : 4;
+  const size_t act_bytes = (size_t)T * r.d * es;
+  if (overlaps(x, act_bytes, y, act_bytes) || overlaps(workspace, L.total, y, act_bytes))
+    return KT_ERR_INVALID_CONFIG;
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(ws + L.w);
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+
+  auto mark = [&](int i) {
+    if (stage_events && stage_events[i])
+      return cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st) == cudaSuccess;
+    return true;
+  };
+  if (!mark(0)) return KT_ERR_CUDA;
+  if (launch_gate_logits(r, T, x, w_gate, logits, err, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_gate_select(r, T, logits, nullptr, bias, idx, w,
+                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), nullptr, st) != cudaSuccess)
+    return KT_ERR_CUDA;
+  if (!mark(1)) return KT_ERR_CUDA;
+  if (launch_permute(r, T, L, ws, idx, w, x, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (!mark(2)) return KT_ERR_CUDA;
+  cudaError_t e = r.dtype == KT_DTYPE_BF16
+                      ? launch_experts_bf16(r, T, L, ws, x, w1, w3, sms, st, /*up=*/true)
+                      : launch_experts_f32(r, T, L, ws, x, w1, w3, w2, sms, st, /*up=*/true);
+  if (e != cudaSuccess || !mark(3)) return KT_ERR_CUDA;
+  e = r.dtype == KT_DTYPE_BF16 ? launch_experts_bf16(r, T, L, ws, x, w2, nullptr, sms, st, false)
+                               : launch_experts_f32(r, T, L, ws, x, w1, w3, w2, sms, st, false);
+  if (e != cudaSuccess || !mark(4)) return KT_ERR_CUDA;
+  if (launch_combine(r, T, L, ws, x, y, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (!mark(5)) return KT_ERR_CUDA;
+  return KT_OK;
+}
+
+int kt_moe_check(const void* workspace, void* stream) {
+  if (!workspace) return KT_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KT_ERR_CUDA;
+  int err[2] = {0, 0};
+  if (cudaMemcpy(err, workspace, sizeof err, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KT_ERR_CUDA;
+  return err[0] == 0 ? KT_OK : KT_ERR_TIMEOUT;
+}
+
+const char* kt_moe_strerror(int code) {
+  switch (code) {
+    case KT_OK: return "ok";
+    case KT_ERR_INVALID_CONFIG: return "invalid layer config or token count";
+    case KT_ERR_NULL: return "a required pointer is NULL";
+    case KT_ERR_WORKSPACE: return "workspace missing or too small";
+    case KT_ERR_ALIGN: return "pointer not aligned (16 B for tensors, 256 B for the workspace)";
+    case KT_ERR_CUDA: return "CUDA runtime error or failed launch";
+    case KT_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case KT_ERR_UNSUPPORTED: return "unsupported device (needs compute capability 10.0, sm_100a)";
+    default: return "unknown error code";
+  }
+}
+
+int kt_moe_version(void) { return (0 << 16) | 1; }
+
+}  // extern "C"

@@ -1,0 +1,330 @@
+// Gate of the DeepSeekMoE layer: logits, score function and the group-limited
+// top-k selection. Follows "Gate 选专家流程（model.py，五步）" of the DeepSeek-V3
+// model.py notes (73biji.xyz/llm_pp_dsv3) and the bias rule of its
+// "V3 改进①：无辅助损失负载均衡" section.
+//
+//   gate_logits_kernel : l = u W_g^T, fp32 FMA accumulation, register-tiled.
+//   gate_select_kernel : one warp per token; scores, keys s + b, group scores,
+//                        top topk_groups groups, top-k experts, weights. Each
+//                        CTA covers one 32-token chunk and also writes that
+//                        chunk's per-expert counts for the token permutation.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "ktmoe_internal.cuh"
+
+namespace ktmoe {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Logits: CTA tile 64 tokens x 128 experts, 128 threads, 8x8 outputs per
+// thread (rows ty*4+{0..3} and 32+ty*4+{0..3}; experts tx*4+{0..3} and
+// 64+tx*4+{0..3}), K slab of 32 staged in shared memory k-major.
+// ---------------------------------------------------------------------------
+constexpr int kLT = 64, kLE = 128, kLK = 32, kLThreads = 128;
+
+template <typename T>
+struct Vec16;  // 16-byte chunk of T
+template <>
+struct Vec16<float> {
+  static constexpr int n = 4;
+  __device__ static void load(const float* p, float* out) {
+    float4 v = *reinterpret_cast<const float4*>(p);
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+  }
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ static void load(const __nv_bfloat16* p, float* out) {
+    uint4 v = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      out[2 * i] = __uint_as_float(w[i] << 16);
+      out[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+
+// Load a [rows x kLK] slab (row-major source, leading dim ld) into s[k][row]
+// (k-major), zero-filling rows >= nrows and columns >= ncols.
+template <typename T, int ROWS>
+__device__ __forceinline__ void load_slab(const T* src, int64_t ld, int nrows, int ncols, int k0,
+                                          float (*s)[ROWS + 4]) {
+  constexpr int VN = Vec16<T>::n;
+  constexpr int chunks_per_row = kLK / VN;
+  constexpr int total = ROWS * chunks_per_row;
+  for (int c = threadIdx.x; c < total; c += kLThreads) {
+    const int row = c / chunks_per_row;
+    const int kk = (c % chunks_per_row) * VN;
+    float v[VN];
+    if (row < nrows && k0 + kk < ncols) {
+      Vec16<T>::load(src + (int64_t)row * ld + k0 + kk, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < VN; ++i) v[i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < VN; ++i) s[kk + i][row] = v[i];
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kLThreads)
+gate_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg, float* __restrict__ logits,
+                   int T_, int E, int d, int* err_reset) {
+  __shared__ float xs[kLK][kLT + 4];
+  __shared__ float ws[kLK][kLE + 4];
+  if (err_reset && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    err_reset[0] = 0;
+    err_reset[1] = 0;
+  }
+  const int e0 = blockIdx.x * kLE;
+  const int t0 = blockIdx.y * kLT;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  const T* xb = x + (int64_t)t0 * d;
+  const T* wb = wg + (int64_t)e0 * d;
+  for (int k0 = 0; k0 < d; k0 += kLK) {
+    load_slab<T, kLT>(xb, d, T_ - t0, d, k0, xs);
+    load_slab<T, kLE>(wb, d, E - e0, d, k0, ws);
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kLK; ++kk) {
+      float a[8], b[8];
+      *reinterpret_cast<float4*>(a) = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      *reinterpret_cast<float4*>(a + 4) = *reinterpret_cast<const float4*>(&xs[kk][32 + ty * 4]);
+      *reinterpret_cast<float4*>(b) = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+      *reinterpret_cast<float4*>(b + 4) = *reinterpret_cast<const float4*>(&ws[kk][64 + tx * 4]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + (i < 4 ? ty * 4 + i : 32 + ty * 4 + (i - 4));
+    if (t >= T_) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = e0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
+      if (e < E) logits[(int64_t)t * E + e] = acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Selection: 8 warps per CTA, 4 tokens per warp, 32 tokens per CTA.
+// Lane l holds experts e = i*32 + l, i < ceil(E/32) (at most 16).
+// ---------------------------------------------------------------------------
+constexpr int kSelWarps = 8;
+constexpr int kNPer = kMaxExperts / 32;
+constexpr unsigned kFull = 0xffffffffu;
+
+struct Best {
+  float key;
+  int idx;
+};
+// Larger key wins; lower index wins a tie.
+__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
+  return ka > kb || (ka == kb && ia < ib);
+}
+__device__ __forceinline__ Best warp_argmax(Best b) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ok = __shfl_xor_sync(kFull, b.key, off);
+    const int oi = __shfl_xor_sync(kFull, b.idx, off);
+    if (better(ok, oi, b.key, b.idx)) {
+      b.key = ok;
+      b.idx = oi;
+    }
+  }
+  return b;
+}
+
+__global__ void __launch_bounds__(kSelWarps * 32)
+gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
+                   const float* __restrict__ scores_in, const float* __restrict__ bias,
+                   int32_t* __restrict__ out_idx, float* __restrict__ out_w,
+                   int32_t* __restrict__ chunk_counts, int* err_reset) {
+  __shared__ int scount[kMaxExperts];
+  __shared__ float skey[kSelWarps][kMaxExperts];
+  if (err_reset && blockIdx.x == 0 && threadIdx.x == 0) {
+    err_reset[0] = 0;
+    err_reset[1] = 0;
+  }
+  const int E = r.E, k = r.k, G = r.G, gs = r.gs;
+  const int nper = (E + 31) / 32;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) scount[e] = 0;
+  __syncthreads();
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const float NEG_INF = -INFINITY;
+  for (int tt = 0; tt < kPermChunk / kSelWarps; ++tt) {
+    const int t = blockIdx.x * kPermChunk + warp * (kPermChunk / kSelWarps) + tt;
+    if (t >= T_) break;
+    // Step 1: scores (kept raw for step 5).
+    float s[kNPer], key[kNPer];
+    const float* row = (scores_in ? scores_in : logits) + (int64_t)t * E;
+#pragma unroll
+    for (int i = 0; i < kNPer; ++i) {
+      const int e = i * 32 + lane;
+      s[i] = (i < nper && e < E) ? row[e] : NEG_INF;
+    }
+    if (!scores_in) {
+      if (r.score_func == KT_SCORE_SIGMOID) {
+#pragma unroll
+        for (int i = 0; i < kNPer; ++i)
+          if (i < nper) s[i] = 1.0f / (1.0f + expf(-s[i]));
+      } else {
+        float m = NEG_INF;
+#pragma unroll
+        for (int i = 0; i < kNPer; ++i)
+          if (i < nper) m = fmaxf(m, s[i]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+        float z = 0.f;
+#pragma unroll
+        for (int i = 0; i < kNPer; ++i)
+          if (i < nper) {
+            s[i] = (i * 32 + lane < E) ? expf(s[i] - m) : 0.f;
+            z += s[i];
+          }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFull, z, off);
+#pragma unroll
+        for (int i = 0; i < kNPer; ++i)
+          if (i < nper) s[i] = __fdiv_rn(s[i], z);
+      }
+    }
+    // Step 2a: selection keys s + b (the bias takes part in the selection only).
+#pragma unroll
+    for (int i = 0; i < kNPer; ++i) {
+      const int e = i * 32 + lane;
+      if (i < nper && e < E) {
+        key[i] = r.has_bias ? __fadd_rn(s[i], bias[e]) : s[i];
+        if (key[i] != key[i]) key[i] = NEG_INF;   // NaN input: keep indices valid
+      } else {
+        key[i] = NEG_INF;
+      }
+    }
+    // Steps 2b-3: group scores, keep topk_groups groups, mask the rest.
+    if (G > 1) {
+#pragma unroll
+      for (int i = 0; i < kNPer; ++i) {
+        const int e = i * 32 + lane;
+        if (i < nper && e < E) skey[warp][e] = key[i];
+      }
+      __syncwarp();
+      float gsc = NEG_INF;
+      if (lane < G) {
+        const float* kg = &skey[warp][lane * gs];
+        if (r.group_score == KT_GROUP_TOP2SUM) {
+          float b1 = NEG_INF, b2 = NEG_INF;
+          for (int i = 0; i < gs; ++i) {
+            const float v = kg[i];
+            if (v > b1) {
+              b2 = b1;
+              b1 = v;
+            } else if (v > b2) {
+              b2 = v;
+            }
+          }
+          gsc = __fadd_rn(b1, b2);
+        } else {
+          for (int i = 0; i < gs; ++i) gsc = fmaxf(gsc, kg[i]);
+        }
+      }
+      __syncwarp();
+      unsigned kept = 0;
+      bool taken = lane >= G;
+      for (int rr = 0; rr < r.TG; ++rr) {
+        Best b = warp_argmax(Best{taken ? NEG_INF : gsc, taken ? 0x7fffffff : lane});
+        kept |= 1u << b.idx;
+        if (lane == b.idx) taken = true;
+      }
+#pragma unroll
+      for (int i = 0; i < kNPer; ++i) {
+        const int e = i * 32 + lane;
+        if (i < nper && e < E && !((kept >> (e / gs)) & 1u)) key[i] = NEG_INF;
+      }
+    }
+    // Step 4: global top-k over the masked keys; lane j keeps slot j.
+    int my_e = 0;
+    float my_s = 0.f;
+    for (int j = 0; j < k; ++j) {
+      Best lb{NEG_INF, 0x7fffffff};
+#pragma unroll
+      for (int i = 0; i < kNPer; ++i) {
+        const int e = i * 32 + lane;
+        if (i < nper && e < E && better(key[i], e, lb.key, lb.idx)) {
+          lb.key = key[i];
+          lb.idx = e;
+        }
+      }
+      const Best b = warp_argmax(lb);
+      float won_s = 0.f;
+      if (lane == (b.idx & 31)) {
+#pragma unroll
+        for (int i = 0; i < kNPer; ++i)
+          if (i == (b.idx >> 5)) {
+            won_s = s[i];
+            key[i] = __int_as_float(0x7fffffff);  // NaN: never wins again
+          }
+      }
+      won_s = __shfl_sync(kFull, won_s, b.idx & 31);
+      if (lane == j) {
+        my_e = b.idx;
+        my_s = won_s;
+      }
+    }
+    // Step 5: gather raw scores, renormalise (slot order), times route_scale.
+    float sum = 0.f;
+    for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(kFull, my_s, j));
+    if (lane < k) {
+      float wv = r.norm ? __fdiv_rn(my_s, sum) : my_s;
+      wv = __fmul_rn(wv, r.route_scale);
+      out_idx[(int64_t)t * k + lane] = my_e;
+      out_w[(int64_t)t * k + lane] = wv;
+      atomicAdd(&scount[my_e], 1);
+    }
+  }
+  __syncthreads();
+  if (chunk_counts)
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      chunk_counts[(int64_t)blockIdx.x * E + e] = scount[e];
+}
+
+}  // namespace
+
+cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, const void* w_gate,
+                               float* logits, int* err_reset, cudaStream_t st) {
+  dim3 grid((r.E + kLE - 1) / kLE, (unsigned)((T + kLT - 1) / kLT));
+  if (r.dtype == KT_DTYPE_BF16)
+    gate_logits_kernel<__nv_bfloat16><<<grid, kLThreads, 0, st>>>(
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d, err_reset);
+  else
+    gate_logits_kernel<float><<<grid, kLThreads, 0, st>>>((const float*)x, (const float*)w_gate,
+                                                          logits, (int)T, r.E, r.d, err_reset);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits,
+                               const float* scores_in, const float* bias, int32_t* idx, float* w,
+                               int32_t* chunk_counts, int* err_reset, cudaStream_t st) {
+  const unsigned grid = (unsigned)((T + kPermChunk - 1) / kPermChunk);
+  gate_select_kernel<<<grid, kSelWarps * 32, 0, st>>>(r, (int)T, logits, scores_in, bias, idx, w,
+                                                     chunk_counts, err_reset);
+  return cudaGetLastError();
+}
+
+}  // namespace ktmoe

@@ -1,0 +1,105 @@
+// Internal declarations shared by the kernels and the host orchestrator of the
+// B200 DeepSeekMoE layer library. Not part of the public ABI (include/ktmoe.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "ktmoe.h"
+
+namespace ktmoe {
+
+// ---------------------------------------------------------------------------
+// Tiling constants
+// ---------------------------------------------------------------------------
+constexpr int kPermChunk = 32;      // tokens per gate-select / scatter CTA
+constexpr int kUpChunk = 128;       // token rows per gate/up GEMM tile (MMA N <= 128)
+constexpr int kDownChunk = 256;     // token rows per down GEMM tile (MMA N <= 256)
+constexpr int kWRows = 128;         // weight rows per GEMM tile (MMA M)
+constexpr int kMaxExperts = 512;
+constexpr int kMaxGroups = 32;
+constexpr int kMaxTopk = 32;
+constexpr int kMaxShared = 8;
+
+// Device error word codes (workspace offset 0). The second int holds a detail.
+constexpr int kDevErrTimeout = 1;
+
+// ---------------------------------------------------------------------------
+// Config with every automatic choice resolved
+// ---------------------------------------------------------------------------
+struct Resolved {
+  int E, G, TG, k, S, d, I, gs;
+  float route_scale;
+  int score_func;   // KT_SCORE_*
+  int norm;         // 0/1
+  int group_score;  // KT_GROUP_AMAX / KT_GROUP_TOP2SUM (G == 1: unused)
+  int dtype;        // KT_DTYPE_*
+  int add_residual;
+  int has_bias;
+};
+
+// One token chunk of one expert group, as scheduled on the grouped GEMMs.
+// Rows live in the "hidden-row" space: routed rows 0..T*k-1 sorted by expert,
+// then shared expert s at T*k + s*T + t.
+struct Chunk {
+  int32_t group;    // 0..E-1 routed, E..E+S-1 shared
+  int32_t row0;     // first hidden row of the chunk
+  int32_t nrows;    // rows in the chunk (<= chunk size)
+  int32_t src_row0; // first activation row: permuted-x row (routed) or token (shared)
+};
+
+// Byte offsets of the workspace's internal buffers.
+struct Layout {
+  size_t err;          // int32[2]
+  size_t meta;         // int32[16]: [0] up chunks, [1] down chunks
+  size_t logits;       // fp32 [T, E]
+  size_t idx;          // int32 [T, k] (when the caller gives no output buffer)
+  size_t w;            // fp32 [T, k]
+  size_t chunk_counts; // int32 [nperm, E]
+  size_t chunk_base;   // int32 [nperm, E]
+  size_t counts;       // int32 [E+S]
+  size_t offsets;      // int32 [E+S+1]
+  size_t row_of;       // int32 [T*k]
+  size_t tok_of;       // int32 [T*k]
+  size_t row_weight;   // fp32 [T*k]
+  size_t up_chunks;    // Chunk [max_up]
+  size_t down_chunks;  // Chunk [max_down]
+  size_t xperm;        // dtype [T*k, d] (bf16 layers only)
+  size_t hidden;       // dtype [T*(k+S), I]
+  size_t expert_out;   // dtype [T*(k+S), d]
+  size_t total;
+  int64_t nperm, max_up, max_down;
+};
+
+int resolve(const kt_moe_config* cfg, int64_t T, int has_bias, Resolved* r);
+Layout make_layout(const Resolved& r, int64_t T);
+
+// ---------------------------------------------------------------------------
+// Kernel launchers (each returns the cudaError_t of its launch)
+// ---------------------------------------------------------------------------
+cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, const void* w_gate,
+                               float* logits, int* err_reset, cudaStream_t st);
+cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits,
+                               const float* scores_in, const float* bias, int32_t* idx,
+                               float* w, int32_t* chunk_counts, int* err_reset, cudaStream_t st);
+cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                           const int32_t* idx, const float* w, const void* x, cudaStream_t st);
+// up = true: the gate/up GEMM (wa = W1, wb = W3); up = false: the down GEMM
+// (wa = W2, wb unused).
+cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                                const void* x, const void* wa, const void* wb, int num_sms,
+                                cudaStream_t st, bool up);
+cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                               const void* x, const void* w1, const void* w3, const void* w2,
+                               int num_sms, cudaStream_t st, bool up);
+cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                           const void* x, void* y, cudaStream_t st);
+
+// Device-side helpers used by several kernels.
+__device__ __forceinline__ void set_error(int* err, int code, int detail) {
+  if (atomicCAS(err, 0, code) == 0) err[1] = detail;
+}
+
+}  // namespace ktmoe

@@ -1,0 +1,185 @@
+// Token permutation: from the gate's (idx, w) to expert-contiguous rows.
+//
+// The expert loop of "MoE 前向四步" in the DeepSeek-V3 model.py notes
+// (73biji.xyz/llm_pp_dsv3) runs each expert on x[idx]: the tokens that chose it.
+// Here those gathers become one deterministic counting sort:
+//   counts   per 32-token chunk and expert (written by the gate-select CTAs),
+//   scan     per expert over chunks, then over experts -> row offsets, plus the
+//            chunk lists the grouped GEMMs walk (shared experts appended as
+//            always-selected groups of all T tokens),
+//   scatter  rank of (t, j) inside its expert = number of earlier tokens of the
+//            same chunk that chose that expert (bit mask + popc), so rows of one
+//            expert are in ascending token order; bf16 layers also copy x into
+//            the permuted activation buffer.
+#include <cuda_bf16.h>
+
+#include "ktmoe_internal.cuh"
+
+namespace ktmoe {
+namespace {
+
+constexpr int kScanThreads = 1024;
+
+// Exclusive scan over n <= kScanThreads ints in shared memory; returns total.
+__device__ int block_exclusive_scan(int* buf, int n) {
+  __shared__ int warp_tot[kScanThreads / 32];
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int v = tid < n ? buf[tid] : 0;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int wv = lane < (int)(blockDim.x / 32) ? warp_tot[lane] : 0;
+    int wi = wv;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += o;
+    }
+    warp_tot[lane] = wi - wv;  // exclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = incl - v + warp_tot[warp];
+  __syncthreads();
+  if (tid < n) buf[tid] = excl;
+  __shared__ int total;
+  if (tid == n - 1) total = excl + v;
+  __syncthreads();
+  return total;
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+permute_scan_kernel(int E, int S, int T_, int k, int nperm, const int32_t* __restrict__ chunk_counts,
+                    int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
+                    int32_t* __restrict__ offsets, Chunk* __restrict__ up, Chunk* __restrict__ down,
+                    int32_t* __restrict__ meta) {
+  __shared__ int tot[kMaxExperts + kMaxShared];
+  __shared__ int nup[kMaxExperts + kMaxShared];
+  __shared__ int ndn[kMaxExperts + kMaxShared];
+  const int tid = threadIdx.x;
+  const int NG = E + S;
+  // Per-expert totals over the chunks.
+  if (tid < NG) {
+    int run = 0;
+    if (tid < E)
+      for (int c = 0; c < nperm; ++c) run += chunk_counts[(int64_t)c * E + tid];
+    else
+      run = T_;
+    tot[tid] = run;
+    counts[tid] = run;
+  }
+  __syncthreads();
+  // Routed experts: rows [0, T*k); shared expert s: rows T*k + s*T.
+  const int ntot = block_exclusive_scan(tot, E);
+  (void)ntot;
+  if (tid >= E && tid < NG) tot[tid] = T_ * k + (tid - E) * T_;
+  __syncthreads();
+  if (tid < NG) offsets[tid] = tot[tid];
+  if (tid == 0) offsets[NG] = T_ * k + S * T_;
+  // Chunk bases (global row of each chunk's first row for each expert).
+  if (tid < E) {
+    int run = tot[tid];
+    for (int c = 0; c < nperm; ++c) {
+      chunk_base[(int64_t)c * E + tid] = run;
+      run += chunk_counts[(int64_t)c * E + tid];
+    }
+  }
+  // Chunk lists for the two GEMMs.
+  if (tid < NG) {
+    const int n = tid < E ? counts[tid] : T_;
+    nup[tid] = (n + kUpChunk - 1) / kUpChunk;
+    ndn[tid] = (n + kDownChunk - 1) / kDownChunk;
+  }
+  __syncthreads();
+  const int total_up = block_exclusive_scan(nup, NG);
+  const int total_dn = block_exclusive_scan(ndn, NG);
+  if (tid < NG) {
+    const int n = tid < E ? counts[tid] : T_;
+    const int row0 = tot[tid];
+    const int src0 = tid < E ? row0 : 0;
+    for (int c = 0, r = 0; r < n; ++c, r += kUpChunk)
+      up[nup[tid] + c] = Chunk{tid, row0 + r, min(kUpChunk, n - r), src0 + r};
+    for (int c = 0, r = 0; r < n; ++c, r += kDownChunk)
+      down[ndn[tid] + c] = Chunk{tid, row0 + r, min(kDownChunk, n - r), src0 + r};
+  }
+  if (tid == 0) {
+    meta[0] = total_up;
+    meta[1] = total_dn;
+  }
+}
+
+template <bool kCopyX>
+__global__ void __launch_bounds__(256)
+permute_scatter_kernel(int E, int T_, int k, int d, const int32_t* __restrict__ idx,
+                       const float* __restrict__ w, const int32_t* __restrict__ chunk_base,
+                       int32_t* __restrict__ row_of, int32_t* __restrict__ tok_of,
+                       float* __restrict__ row_weight, const uint4* __restrict__ x,
+                       uint4* __restrict__ xperm) {
+  __shared__ uint32_t mask[kMaxExperts];
+  __shared__ int srow[kPermChunk * kMaxTopk];
+  const int c = blockIdx.x;
+  const int t0 = c * kPermChunk;
+  const int nt = min(kPermChunk, T_ - t0);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) mask[e] = 0u;
+  __syncthreads();
+  const int nent = nt * k;
+  for (int q = threadIdx.x; q < nent; q += blockDim.x) {
+    const int tl = q / k;
+    const int e = idx[(int64_t)t0 * k + q];
+    atomicOr(&mask[e], 1u << tl);
+  }
+  __syncthreads();
+  for (int q = threadIdx.x; q < nent; q += blockDim.x) {
+    const int tl = q / k;
+    const int e = idx[(int64_t)t0 * k + q];
+    const int rank = __popc(mask[e] & ((1u << tl) - 1u));
+    const int row = chunk_base[(int64_t)c * E + e] + rank;
+    row_of[(int64_t)t0 * k + q] = row;
+    tok_of[row] = t0 + tl;
+    row_weight[row] = w[(int64_t)t0 * k + q];
+    srow[q] = row;
+  }
+  if (!kCopyX) return;
+  __syncthreads();
+  // Copy each token's row of x to its k permuted rows (16-byte chunks).
+  const int nchunk = d / 8;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int tl = warp; tl < nt; tl += blockDim.x / 32) {
+    const uint4* src = x + (int64_t)(t0 + tl) * nchunk;
+    for (int q = lane; q < nchunk; q += 32) {
+      const uint4 v = src[q];
+      for (int j = 0; j < k; ++j) xperm[(int64_t)srow[tl * k + j] * nchunk + q] = v;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                           const int32_t* idx, const float* w, const void* x, cudaStream_t st) {
+  auto I32 = [&](size_t off) { return reinterpret_cast<int32_t*>(ws + off); };
+  permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
+      r.E, r.S, (int)T, r.k, (int)L.nperm, I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts),
+      I32(L.offsets), reinterpret_cast<Chunk*>(ws + L.up_chunks),
+      reinterpret_cast<Chunk*>(ws + L.down_chunks), I32(L.meta));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)L.nperm;
+  float* rw = reinterpret_cast<float*>(ws + L.row_weight);
+  if (r.dtype == KT_DTYPE_BF16)
+    permute_scatter_kernel<true><<<grid, 256, 0, st>>>(
+        r.E, (int)T, r.k, r.d, idx, w, I32(L.chunk_base), I32(L.row_of), I32(L.tok_of), rw,
+        reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(ws + L.xperm));
+  else
+    permute_scatter_kernel<false><<<grid, 256, 0, st>>>(
+        r.E, (int)T, r.k, r.d, idx, w, I32(L.chunk_base), I32(L.row_of), I32(L.tok_of), rw,
+        nullptr, nullptr);
+  return cudaGetLastError();
+}
+
+}  // namespace ktmoe

@@ -1,0 +1,196 @@
+"""Python binding of libktmoe.so (include/ktmoe.h): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; this module only
+turns torch tensors into pointers, picks the current CUDA stream, and raises on
+error codes. There is no fallback: if the library is missing or fails to load,
+importing the entry points raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libktmoe.so")
+
+KT_SCORE_SIGMOID, KT_SCORE_SOFTMAX = 0, 1
+KT_GROUP_AUTO, KT_GROUP_AMAX, KT_GROUP_TOP2SUM = 0, 1, 2
+KT_DTYPE_F32, KT_DTYPE_BF16 = 0, 1
+KT_OK = 0
+KT_ERR_INVALID_CONFIG, KT_ERR_NULL, KT_ERR_WORKSPACE, KT_ERR_ALIGN = -1, -2, -3, -4
+KT_ERR_CUDA, KT_ERR_TIMEOUT, KT_ERR_UNSUPPORTED = -5, -6, -7
+
+# Every symbol include/ktmoe.h declares.
+EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_forward",
+           "kt_moe_forward_profiled", "kt_moe_check", "kt_moe_workspace_layout", "kt_moe_strerror", "kt_moe_version")
+
+
+class kt_moe_config(ctypes.Structure):
+    _fields_ = [("n_experts", ctypes.c_int32), ("n_groups", ctypes.c_int32),
+                ("topk_groups", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("route_scale", ctypes.c_float), ("score_func", ctypes.c_int32),
+                ("dim", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32), ("norm_topk", ctypes.c_int32),
+                ("group_score", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("add_residual", ctypes.c_int32)]
+
+
+class kt_moe_ws_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("error_word", "logits", "counts", "offsets",
+                                              "row_of", "tok_of", "row_weight", "hidden",
+                                              "expert_out", "total")]
+
+
+class KtMoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {strerror(code)} (code {code})")
+        self.code = code
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libktmoe.so (raises OSError if it is missing: no fallback path)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise OSError(f"{LIB_PATH} not found: build it with "
+                              "`python -m mixture_experts_layer_34_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I64, CP = ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(kt_moe_config)
+            L.kt_moe_validate.argtypes = [CP, I64, ctypes.c_int]
+            L.kt_moe_validate.restype = ctypes.c_int
+            L.kt_moe_workspace_size.argtypes = [CP, I64]
+            L.kt_moe_workspace_size.restype = ctypes.c_size_t
+            L.kt_moe_gate.argtypes = [CP, I64, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+            L.kt_moe_gate.restype = ctypes.c_int
+            L.kt_moe_forward.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+            L.kt_moe_forward.restype = ctypes.c_int
+            L.kt_moe_forward_profiled.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P,
+                                                  ctypes.c_size_t, P, ctypes.POINTER(P)]
+            L.kt_moe_forward_profiled.restype = ctypes.c_int
+            L.kt_moe_check.argtypes = [P, P]
+            L.kt_moe_check.restype = ctypes.c_int
+            L.kt_moe_workspace_layout.argtypes = [CP, I64, ctypes.POINTER(kt_moe_ws_layout)]
+            L.kt_moe_workspace_layout.restype = ctypes.c_int
+            L.kt_moe_strerror.argtypes = [ctypes.c_int]
+            L.kt_moe_strerror.restype = ctypes.c_char_p
+            L.kt_moe_version.argtypes = []
+            L.kt_moe_version.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().kt_moe_strerror(int(code)).decode()
+
+
+def make_config(n_experts, n_groups, topk_groups, topk, route_scale, score_func, dim, inter,
+                n_shared, norm_topk=-1, group_score=KT_GROUP_AUTO, dtype=KT_DTYPE_BF16,
+                add_residual=0) -> kt_moe_config:
+    return kt_moe_config(int(n_experts), int(n_groups), int(topk_groups), int(topk),
+                         float(route_scale), int(score_func), int(dim), int(inter), int(n_shared),
+                         int(norm_topk), int(group_score), int(dtype), int(add_residual))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def kt_moe_validate(cfg: kt_moe_config, T: int, has_bias: bool) -> int:
+    return lib().kt_moe_validate(ctypes.byref(cfg), int(T), int(bool(has_bias)))
+
+
+def kt_moe_workspace_size(cfg: kt_moe_config, T: int) -> int:
+    return int(lib().kt_moe_workspace_size(ctypes.byref(cfg), int(T)))
+
+
+def kt_moe_workspace_layout(cfg: kt_moe_config, T: int) -> dict:
+    out = kt_moe_ws_layout()
+    rc = lib().kt_moe_workspace_layout(ctypes.byref(cfg), int(T), ctypes.byref(out))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_workspace_layout", rc)
+    return {n: getattr(out, n) for n, _ in kt_moe_ws_layout._fields_}
+
+
+def kt_moe_gate(cfg, T, x, w_gate, bias, scores_in, topk_idx, topk_w, workspace, stream=None):
+    rc = lib().kt_moe_gate(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias),
+                           _ptr(scores_in), _ptr(topk_idx), _ptr(topk_w), _ptr(workspace),
+                           _nbytes(workspace), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_gate", rc)
+
+
+def kt_moe_forward(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out, workspace,
+                   stream=None):
+    rc = lib().kt_moe_forward(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias),
+                              _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y), _ptr(topk_idx_out),
+                              _ptr(topk_w_out), _ptr(workspace), _nbytes(workspace),
+                              _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_forward", rc)
+
+
+KT_STAGE_EVENTS = 6
+STAGES = ("gate", "permute", "up_gemm", "down_gemm", "combine")
+
+
+def kt_moe_forward_profiled(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                            workspace, events, stream=None):
+    """kt_moe_forward recording `events` (6 torch.cuda.Event, created with
+    enable_timing=True) at the stage boundaries on the launch stream."""
+    if len(events) != KT_STAGE_EVENTS:
+        raise ValueError(f"need {KT_STAGE_EVENTS} events")
+    arr = (ctypes.c_void_p * KT_STAGE_EVENTS)(*[ctypes.c_void_p(e.cuda_event) if e is not None
+                                                 else None for e in events])
+    rc = lib().kt_moe_forward_profiled(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias),
+                                       _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y), _ptr(topk_idx_out),
+                                       _ptr(topk_w_out), _ptr(workspace), _nbytes(workspace),
+                                       _stream(stream), arr)
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_forward_profiled", rc)
+
+
+def kt_moe_check(workspace, stream=None) -> int:
+    """Synchronise the stream and read the workspace's device error word."""
+    return lib().kt_moe_check(_ptr(workspace), _stream(stream))
+
+
+def kt_moe_version() -> int:
+    return lib().kt_moe_version()
+
+
+def config_for(layer) -> kt_moe_config:
+    """kt_moe_config of a workloads.LayerConfig."""
+    return make_config(dtype=KT_DTYPE_F32 if layer.dtype == "f32" else KT_DTYPE_BF16,
+                       **layer.kernel_fields())
+
+
+def alloc_workspace(cfg: kt_moe_config, T: int, device="cuda"):
+    """A byte tensor of kt_moe_workspace_size bytes (torch's allocator aligns to 512 B)."""
+    import torch
+    n = kt_moe_workspace_size(cfg, T)
+    if n == 0:
+        raise KtMoeError("kt_moe_workspace_size", KT_ERR_INVALID_CONFIG)
+    return torch.empty(n, dtype=torch.uint8, device=device)

@@ -1,0 +1,66 @@
+"""Helpers for comparing the CUDA library with the oracle (test code only)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle.oracle as O
+from mixture_experts_layer_34_b200 import ktmoe as K
+from mixture_experts_layer_34_b200 import workloads as W
+
+NEAR_TIE = 1e-5
+TOL_BF16 = 2e-2     # max |dy| <= TOL * RMS(y_ref), bf16 layers
+TOL_F32 = 1e-4      # same form, fp32 layers
+
+
+def tolerance(layer) -> float:
+    return TOL_F32 if layer.dtype == "f32" else TOL_BF16
+
+
+def run_forward(layer, inp, T=None, ws=None):
+    """One kt_moe_forward on the current stream; returns y, idx, w, workspace."""
+    T = layer.T if T is None else T
+    cfg = K.config_for(layer)
+    dev = inp["x"].device
+    ws = K.alloc_workspace(cfg, T, dev) if ws is None else ws
+    y = torch.empty((T, layer.dim), dtype=inp["x"].dtype, device=dev)
+    idx = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
+    w = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
+    K.kt_moe_forward(cfg, T, inp["x"], inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                     y, idx, w, ws)
+    rc = K.kt_moe_check(ws)
+    assert rc == K.KT_OK, K.strerror(rc)
+    return dict(y=y, idx=idx, w=w, ws=ws)
+
+
+def oracle_gate(layer, inp):
+    bias = inp["bias"]
+    return O.gate(layer.kernel_fields(), inp["x"], inp["w_gate"],
+                  None if bias is None else bias.float().cpu().numpy())
+
+
+def routing_agreement(layer, og, idx_gpu: np.ndarray):
+    """Tokens whose routing differs, and whether each difference is a near tie."""
+    diff = np.where((og["idx"] != idx_gpu).any(1))[0]
+    near = (og["kth_margin"] <= NEAR_TIE) | (og["grp_margin"] <= NEAR_TIE)
+    return diff, near
+
+
+def oracle_outputs(layer, inp, og, tok_ids) -> np.ndarray:
+    """The oracle's y for tok_ids, copying only the experts those tokens use."""
+    E, S = layer.n_experts, layer.n_shared
+    need = set(range(E, E + S))
+    for t in tok_ids:
+        need.update(int(e) for e in og["idx"][t])
+    w1 = [inp["w1"][e].cpu() if e in need else None for e in range(E + S)]
+    w3 = [inp["w3"][e].cpu() if e in need else None for e in range(E + S)]
+    w2 = [inp["w2"][e].cpu() if e in need else None for e in range(E + S)]
+    return O.forward(layer.kernel_fields(), inp["x"].cpu(), og["idx"], og["w"], w1, w3, w2,
+                     tok_ids, inp["bias"] is not None)
+
+
+def compare_outputs(layer, y_gpu: torch.Tensor, y_ref: np.ndarray, tok_ids) -> dict:
+    yg = y_gpu[torch.as_tensor(np.asarray(tok_ids), device=y_gpu.device)].float().cpu().numpy()
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    err = float(np.abs(yg - y_ref).max())
+    return dict(max_abs=err, rms=rms, rel=err / rms if rms > 0 else float("inf"))

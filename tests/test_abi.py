@@ -1,0 +1,155 @@
+"""The C-ABI library: loads, exports what include/ktmoe.h declares, and rejects bad
+calls on the host before any CUDA call (CPU; safe on a GPU machine too)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from mixture_experts_layer_34_b200 import ktmoe as K
+from mixture_experts_layer_34_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "ktmoe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kt_moe_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = K.lib()
+    declared = _declared_functions()
+    assert declared, "no declarations found"
+    assert set(declared) == set(K.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_library_links_no_torch():
+    # The library is plain C ABI: it must not need libtorch / libc10 to load.
+    import subprocess
+    out = subprocess.run(["ldd", K.LIB_PATH], capture_output=True, text=True).stdout
+    assert "torch" not in out and "c10" not in out
+
+
+def test_config_struct_layout_matches_header():
+    assert ctypes.sizeof(K.kt_moe_config) == 13 * 4
+    assert ctypes.sizeof(K.kt_moe_ws_layout) == 10 * 8
+
+
+@pytest.mark.parametrize("layer", W.NAMED + W.SMALL, ids=lambda c: c.name)
+def test_named_configs_validate(layer):
+    cfg = K.config_for(layer)
+    assert K.kt_moe_validate(cfg, layer.T, layer.bias != "none") == K.KT_OK
+    ws = K.kt_moe_workspace_size(cfg, layer.T)
+    assert ws > 0 and ws % 1024 == 0
+    lay = K.kt_moe_workspace_layout(cfg, layer.T)
+    assert lay["total"] == ws and lay["error_word"] == 0
+    for key in ("hidden", "expert_out"):
+        assert lay[key] % 1024 == 0
+    # workspace grows with T
+    assert K.kt_moe_workspace_size(cfg, layer.T * 2) > ws
+
+
+BAD = [
+    dict(n_experts=0), dict(n_experts=513), dict(n_groups=3),            # E % G != 0 for E=16
+    dict(topk_groups=5), dict(n_groups=1, topk_groups=2), dict(topk=0),
+    dict(topk=9),                                                         # > TG * E/G = 8
+    dict(n_shared=-1), dict(n_shared=9), dict(route_scale=0.0), dict(route_scale=float("inf")),
+    dict(route_scale=float("nan")), dict(score_func=2), dict(dtype=3), dict(dim=12),
+    dict(inter=4), dict(norm_topk=2), dict(group_score=3), dict(add_residual=2),
+    dict(n_experts=16, n_groups=16, topk_groups=4, topk=4, group_score=2),  # top-2 of 1 expert
+]
+
+
+@pytest.mark.parametrize("bad", BAD)
+def test_invalid_configs_rejected(bad):
+    base = dict(n_experts=16, n_groups=4, topk_groups=2, topk=4, route_scale=2.5, score_func=0,
+                dim=256, inter=128, n_shared=1, norm_topk=-1, group_score=0, dtype=K.KT_DTYPE_BF16,
+                add_residual=0)
+    base.update(bad)
+    cfg = K.make_config(**base)
+    assert K.kt_moe_validate(cfg, 64, True) == K.KT_ERR_INVALID_CONFIG
+    assert K.kt_moe_workspace_size(cfg, 64) == 0
+
+
+def test_token_count_limits():
+    cfg = K.config_for(W.TINY)
+    assert K.kt_moe_validate(cfg, 0, True) == K.KT_ERR_INVALID_CONFIG
+    assert K.kt_moe_validate(cfg, 1, True) == K.KT_OK
+    assert K.kt_moe_validate(cfg, 1 << 20, True) == K.KT_OK
+    assert K.kt_moe_validate(cfg, (1 << 20) + 1, True) == K.KT_ERR_INVALID_CONFIG
+
+
+def _call_forward(cfg, T, ptrs, ws_ptr, ws_bytes):
+    L = K.lib()
+    return L.kt_moe_forward(ctypes.byref(cfg), T, *[ctypes.c_void_p(p) if p else None for p in ptrs],
+                            ctypes.c_void_p(ws_ptr) if ws_ptr else None, ws_bytes, None)
+
+
+def test_host_side_errors_return_before_any_device_work():
+    """Fake (never dereferenced) pointer values: every case must be rejected on
+    the host, so this is safe with or without a GPU."""
+    cfg = K.config_for(W.BY_NAME["small_sig_bias"])
+    T = 300
+    need = K.kt_moe_workspace_size(cfg, T)
+    good = [0x10000 * (i + 1) for i in range(9)]   # x wg bias w1 w3 w2 y idx w, 16-B aligned
+    ws = 0x7000000
+    # NULL required pointer
+    p = list(good)
+    p[0] = 0
+    assert _call_forward(cfg, T, p, ws, need) == K.KT_ERR_NULL
+    # workspace missing / too small
+    assert _call_forward(cfg, T, good, 0, need) == K.KT_ERR_WORKSPACE
+    assert _call_forward(cfg, T, good, ws, need - 1) == K.KT_ERR_WORKSPACE
+    # misaligned tensor and workspace
+    p = list(good)
+    p[3] += 8
+    assert _call_forward(cfg, T, p, ws, need) == K.KT_ERR_ALIGN
+    assert _call_forward(cfg, T, good, ws + 128, need) == K.KT_ERR_ALIGN
+    # output aliasing the input
+    p = list(good)
+    p[6] = p[0]
+    assert _call_forward(cfg, T, p, ws, need) == K.KT_ERR_INVALID_CONFIG
+    # invalid config
+    bad = K.make_config(**{**{f: getattr(cfg, f) for f, _ in K.kt_moe_config._fields_}, "topk": 0})
+    assert _call_forward(bad, T, good, ws, need) == K.KT_ERR_INVALID_CONFIG
+
+
+def test_gate_host_side_errors():
+    cfg = K.config_for(W.BY_NAME["small_sig_bias"])
+    L = K.lib()
+    need = K.kt_moe_workspace_size(cfg, 300)
+    V = ctypes.c_void_p
+    # scores_in absent and x missing
+    rc = L.kt_moe_gate(ctypes.byref(cfg), 300, None, V(0x10000), None, None, V(0x20000),
+                       V(0x30000), V(0x7000000), need, None)
+    assert rc == K.KT_ERR_NULL
+    # outputs missing
+    rc = L.kt_moe_gate(ctypes.byref(cfg), 300, V(0x10000), V(0x20000), None, None, None,
+                       V(0x30000), V(0x7000000), need, None)
+    assert rc == K.KT_ERR_NULL
+
+
+def test_strerror_covers_codes():
+    for code in range(-7, 1):
+        assert K.strerror(code) and K.strerror(code) != "unknown error code"
+    assert K.strerror(-99) == "unknown error code"
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_reports_cuda_error():
+    cfg = K.config_for(W.TINY)
+    n = K.kt_moe_workspace_size(cfg, 64)
+    buf = torch.empty(n + 256, dtype=torch.uint8)
+    ws_ptr = (buf.data_ptr() + 255) // 256 * 256
+    x = torch.empty(64, 256)
+    # Valid host-side arguments; the first CUDA call fails without a device.
+    ptrs = [x.data_ptr()] * 6 + [x.data_ptr() + (1 << 20)] + [0, 0]
+    rc = _call_forward(cfg, 64, ptrs, ws_ptr, n)
+    assert rc in (K.KT_ERR_CUDA, K.KT_ERR_UNSUPPORTED)

@@ -1,0 +1,183 @@
+"""Layer-forward parity on the GPU, through the C ABI (kt_moe_forward).
+
+Outputs must match the oracle within max|dy| <= 2e-2 * RMS(y_ref) for bf16
+layers and 1e-4 * RMS(y_ref) for fp32 ones; tokens whose routing differs from
+the oracle's (allowed only at near ties) are excluded and counted. The
+permutation buffers are compared exactly.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.oracle as O
+from mixture_experts_layer_34_b200 import ktmoe as K
+from mixture_experts_layer_34_b200 import workloads as W
+
+from parity import (compare_outputs, oracle_gate, oracle_outputs, routing_agreement, run_forward,
+                    tolerance)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_layer(layer, inp, tok_ids, out=None):
+    out = out or run_forward(layer, inp)
+    og = oracle_gate(layer, inp)
+    idx = out["idx"].cpu().numpy()
+    diff, near = routing_agreement(layer, og, idx)
+    assert near[diff].all(), f"routing differs away from near ties: {diff[~near[diff]]}"
+    keep = [t for t in tok_ids if t not in set(diff.tolist())]
+    y_ref = oracle_outputs(layer, inp, og, keep)
+    res = compare_outputs(layer, out["y"], y_ref, keep)
+    print(f"{layer.name}: rel err {res['rel']:.3e} over {len(keep)} tokens "
+          f"({len(diff)} near-tie routing differences excluded)")
+    assert res["rel"] <= tolerance(layer), res
+    return out, og
+
+
+@pytest.mark.parametrize("layer", W.SMALL + [W.TINY], ids=lambda c: c.name)
+def test_small_layers_every_token(layer):
+    inp = W.make_layer(layer, "cuda")
+    _check_layer(layer, inp, list(range(layer.T)))
+
+
+@pytest.mark.parametrize("layer", [W.V2_LITE, W.V2, W.V3_DECODE], ids=lambda c: c.name)
+def test_named_layers_sampled_tokens(layer):
+    inp = W.make_layer(layer, "cuda")
+    rng = np.random.default_rng(layer.seed)
+    n = min(layer.T, 24)
+    tok = sorted(rng.choice(layer.T, n, replace=False).tolist())
+    _check_layer(layer, inp, tok)
+
+
+def test_v3_prefill_zipf_sampled_tokens():
+    layer = W.V3_PREFILL
+    inp = W.make_layer(layer, "cuda")
+    out = run_forward(layer, inp)
+    og = oracle_gate(layer, inp)
+    # include the first/last token and tokens routed to the lightest experts
+    load = np.bincount(og["idx"].ravel(), minlength=layer.n_experts)
+    light = [e for e in np.argsort(load) if load[e] > 0][:3]
+    tok = {0, layer.T - 1}
+    for e in light:
+        tok.add(int(np.where((og["idx"] == e).any(1))[0][0]))
+    rng = np.random.default_rng(1)
+    tok.update(rng.choice(layer.T, 5, replace=False).tolist())
+    _check_layer(layer, inp, sorted(tok), out=out)
+
+
+def _ws_array(ws, off, n, dtype):
+    nbytes = n * torch.tensor([], dtype=dtype).element_size()
+    return ws[off: off + nbytes].view(dtype).cpu().numpy()
+
+
+@pytest.mark.parametrize("layer", [W.BY_NAME["small_sig_bias"], W.V3_DECODE, W.TINY],
+                         ids=lambda c: c.name)
+def test_permutation_buffers_exact(layer):
+    """counts, offsets, row_of and tok_of are the counting sort of the routing:
+    rows grouped by expert, tokens ascending within an expert."""
+    inp = W.make_layer(layer, "cuda")
+    out = run_forward(layer, inp)
+    T, k, E, S = layer.T, layer.topk, layer.n_experts, layer.n_shared
+    idx = out["idx"].cpu().numpy()
+    lay = K.kt_moe_workspace_layout(K.config_for(layer), T)
+    ws = out["ws"]
+    counts = _ws_array(ws, lay["counts"], E + S, torch.int32)
+    offsets = _ws_array(ws, lay["offsets"], E + S + 1, torch.int32)
+    row_of = _ws_array(ws, lay["row_of"], T * k, torch.int32).reshape(T, k)
+    tok_of = _ws_array(ws, lay["tok_of"], T * k, torch.int32)
+    rw = _ws_array(ws, lay["row_weight"], T * k, torch.float32)
+    ref_counts = np.bincount(idx.ravel(), minlength=E)
+    assert np.array_equal(counts[:E], ref_counts)
+    assert (counts[E:] == T).all()
+    ref_off = np.concatenate([[0], np.cumsum(ref_counts)])
+    assert np.array_equal(offsets[:E + 1], ref_off)
+    for s in range(S):
+        assert offsets[E + s] == T * k + s * T
+    assert offsets[E + S] == T * k + S * T
+    w = out["w"].cpu().numpy()
+    for e in range(E):
+        toks = np.where((idx == e).any(1))[0]          # ascending token order
+        rows = np.arange(ref_off[e], ref_off[e + 1])
+        assert np.array_equal(tok_of[rows], toks)
+        for r, t in zip(rows, toks):
+            j = int(np.where(idx[t] == e)[0][0])
+            assert row_of[t, j] == r and rw[r] == w[t, j]
+
+
+def test_hidden_rows_match_oracle_expert_hidden():
+    """The up GEMM alone: SwiGLU hidden rows of a few (expert, token) pairs."""
+    layer = W.BY_NAME["small_sig_bias"]
+    inp = W.make_layer(layer, "cuda")
+    out = run_forward(layer, inp)
+    T, k, E, I = layer.T, layer.topk, layer.n_experts, layer.inter
+    lay = K.kt_moe_workspace_layout(K.config_for(layer), T)
+    R = T * (k + layer.n_shared)
+    hidden = out["ws"][lay["hidden"]: lay["hidden"] + R * I * 2].view(torch.bfloat16)
+    hidden = hidden.view(R, I).float().cpu().numpy()
+    row_of = _ws_array(out["ws"], lay["row_of"], T * k, torch.int32).reshape(T, k)
+    idx = out["idx"].cpu().numpy()
+    xc = inp["x"].cpu()
+    for t in (0, 1, 150, T - 1):
+        for j in range(k):
+            e = int(idx[t, j])
+            h = O.expert_hidden(layer.kernel_fields(), xc, inp["w1"][e].cpu(), inp["w3"][e].cpu(), [t])[0]
+            got = hidden[row_of[t, j]]
+            assert np.abs(got - h).max() <= 2e-2 * np.sqrt(np.mean(h ** 2)) + 1e-6
+        h = O.expert_hidden(layer.kernel_fields(), xc, inp["w1"][E].cpu(), inp["w3"][E].cpu(), [t])[0]
+        got = hidden[T * k + t]
+        assert np.abs(got - h).max() <= 2e-2 * np.sqrt(np.mean(h ** 2)) + 1e-6
+
+
+@pytest.mark.parametrize("T", [1, 15, 16, 17, 127, 128, 129, 255, 256, 257])
+def test_every_token_to_the_same_experts(T):
+    """W_gate = 0: every score is sigmoid(0) = 0.5, so the bias alone picks the
+    same k experts for all tokens; each chosen expert holds all T rows (per-expert
+    M = T across the 16/128/256 tile boundaries) and the others hold none."""
+    layer = W.BY_NAME["small_sig_bias"].with_(T=T, seed=3000 + T)
+    inp = W.make_layer(layer, "cuda")
+    inp["w_gate"].zero_()
+    inp["bias"] = torch.linspace(-0.5, 0.5, layer.n_experts, device="cuda").flip(0).contiguous()
+    out, og = _check_layer(layer, inp, list(range(T)))
+    idx = out["idx"].cpu().numpy()
+    assert (idx == np.arange(layer.topk)[None, :]).all()
+
+
+def test_residual_layer_adds_tokens():
+    layer = W.BY_NAME["small_odd_dims"]
+    assert layer.add_residual == 1
+    inp = W.make_layer(layer, "cuda")
+    _check_layer(layer, inp, list(range(layer.T)))
+
+
+def test_forward_is_deterministic():
+    layer = W.BY_NAME["small_sig_bias"]
+    inp = W.make_layer(layer, "cuda")
+    a = run_forward(layer, inp)
+    b = run_forward(layer, inp)
+    assert torch.equal(a["y"], b["y"]) and torch.equal(a["idx"], b["idx"])
+
+
+def test_token_permutation_permutes_routing():
+    layer = W.BY_NAME["small_sig_bias"]
+    inp = W.make_layer(layer, "cuda")
+    a = run_forward(layer, inp)
+    perm = torch.randperm(layer.T, generator=torch.Generator().manual_seed(5)).cuda()
+    inp2 = dict(inp, x=inp["x"][perm].contiguous())
+    b = run_forward(layer, inp2)
+    assert torch.equal(b["idx"], a["idx"][perm]) and torch.equal(b["w"], a["w"][perm])
+    ya, yb = a["y"][perm].float(), b["y"].float()
+    rms = ya.pow(2).mean().sqrt()
+    assert (ya - yb).abs().max() <= 1e-2 * rms
+
+
+def test_workspace_reuse_across_layers():
+    """One workspace sized for the larger layer serves a smaller one afterwards."""
+    big = W.BY_NAME["small_sig_bias"]
+    small = W.BY_NAME["small_softmax_ragged"]
+    ws = K.alloc_workspace(K.config_for(big), big.T)
+    assert ws.numel() >= K.kt_moe_workspace_size(K.config_for(small), small.T)
+    inp = W.make_layer(small, "cuda")
+    out = run_forward(small, inp, ws=ws)
+    _check_layer(small, inp, list(range(0, small.T, 7)), out=out)
