@@ -89,6 +89,8 @@ typedef struct {
   int32_t group_score;  /* KT_GROUP_*                                              */
   int32_t dtype;        /* KT_DTYPE_*                                              */
   int32_t add_residual; /* 1: add u_t to the output (h'_t); 0: MoE-module output   */
+  int32_t y_fp32;       /* 1: y is fp32 even for bf16 layers (the fp32 sum before   */
+                        /*    its final rounding); 0: y in `dtype`                 */
 } kt_moe_config;
 
 /* Host-only validation of a config for T tokens (T >= 1, T <= 2^20). No CUDA
@@ -124,13 +126,15 @@ int kt_moe_gate(const kt_moe_config* cfg, int64_t T, const void* x, const void* 
  *   x, w_gate, bias    as for kt_moe_gate
  *   w1, w3             device [E+S, inter, dim] (dtype)
  *   w2                 device [E+S, dim, inter] (dtype)
- *   y                  device [T, dim] (dtype) (out); must not alias x
+ *   y                  device [T, dim] (out): dtype, or fp32 if cfg->y_fp32;
+ *                      must not overlap x or the workspace
  *   topk_idx_out       device [T, k] int32 or NULL: the routing, if wanted
  *   topk_w_out         device [T, k] fp32 or NULL
  * The output sum runs in a fixed order per token (shared experts in index
  * order, then the k routed slots in key order, then u_t if add_residual) in
  * fp32, so repeated calls give bitwise-equal y. bf16 layers keep the SwiGLU
- * hidden vectors and the weighted expert outputs in bf16 between kernels.
+ * hidden vectors in bf16 (the down GEMM's tensor-core operand) and the weighted
+ * expert outputs in fp32 between kernels.
  */
 int kt_moe_forward(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
                    const float* bias, const void* w1, const void* w3, const void* w2,
@@ -161,7 +165,7 @@ int kt_moe_check(const void* workspace, void* stream);
  * [E+S]; offsets: exclusive prefix [E+S+1]; row_of: [T, k] row of (t, j) in the
  * expert-sorted order; tok_of: [T*k] token of each sorted row; hidden: SwiGLU
  * hidden rows [T*(k+S), inter] (dtype); expert_out: weighted expert outputs
- * [T*(k+S), dim] (dtype). Rows T*k + s*T + t belong to shared expert s. */
+ * [T*(k+S), dim] (fp32). Rows T*k + s*T + t belong to shared expert s. */
 typedef struct {
   int64_t error_word;
   int64_t logits;

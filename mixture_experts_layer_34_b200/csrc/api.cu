@@ -61,6 +61,7 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
   if (c->norm_topk < -1 || c->norm_topk > 1) return KT_ERR_INVALID_CONFIG;
   if (c->group_score < KT_GROUP_AUTO || c->group_score > KT_GROUP_TOP2SUM) return KT_ERR_INVALID_CONFIG;
   if (c->add_residual != 0 && c->add_residual != 1) return KT_ERR_INVALID_CONFIG;
+  if (c->y_fp32 != 0 && c->y_fp32 != 1) return KT_ERR_INVALID_CONFIG;
   r->E = E;
   r->G = G;
   r->TG = TG;
@@ -77,6 +78,7 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
   if (G > 1 && r->group_score == KT_GROUP_TOP2SUM && gs < 2) return KT_ERR_INVALID_CONFIG;
   r->dtype = c->dtype;
   r->add_residual = c->add_residual;
+  r->y_fp32 = c->dtype == KT_DTYPE_F32 ? 1 : c->y_fp32;
   r->has_bias = has_bias ? 1 : 0;
   return KT_OK;
 }
@@ -113,7 +115,7 @@ Layout make_layout(const Resolved& r, int64_t T) {
   L.down_chunks = take((size_t)L.max_down * sizeof(Chunk), 256);
   L.xperm = take(r.dtype == KT_DTYPE_BF16 ? Tk * r.d * es : 0, 1024);
   L.hidden = take(R * r.I * es, 1024);
-  L.expert_out = take(R * r.d * es, 1024);
+  L.expert_out = take(R * r.d * 4, 1024);   // fp32 for every dtype
   L.total = round_up(off, 1024);
   return L;
 }
@@ -178,12 +180,11 @@ int kt_moe_gate(const kt_moe_config* cfg, int64_t T, const void* x, const void* 
   char* ws = static_cast<char*>(workspace);
   int* err = reinterpret_cast<int*>(ws + L.err);
   float* logits = reinterpret_cast<float*>(ws + L.logits);
-  if (!scores_in) {
-    if (launch_gate_logits(r, T, x, w_gate, logits, err, st) != cudaSuccess) return KT_ERR_CUDA;
-    err = nullptr;   // already reset by the first kernel
-  }
+  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  if (!scores_in && launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess)
+    return KT_ERR_CUDA;
   if (launch_gate_select(r, T, logits, scores_in, bias, topk_idx, topk_w,
-                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), err, st) != cudaSuccess)
+                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), st) != cudaSuccess)
     return KT_ERR_CUDA;
   return KT_OK;
 }
@@ -213,8 +214,9 @@ int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
       (topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
     return KT_ERR_ALIGN;
   const size_t es = r.dtype == KT_DTYPE_BF16 ? 2 : 4;
-  const size_t act_bytes = (size_t)T * r.d * es;
-  if (overlaps(x, act_bytes, y, act_bytes) || overlaps(workspace, L.total, y, act_bytes))
+  const size_t x_bytes = (size_t)T * r.d * es;
+  const size_t y_bytes = (size_t)T * r.d * (r.y_fp32 ? 4 : es);
+  if (overlaps(x, x_bytes, y, y_bytes) || overlaps(workspace, L.total, y, y_bytes))
     return KT_ERR_INVALID_CONFIG;
   int sms = 0;
   if ((rc = device_info(&sms)) != KT_OK) return rc;
@@ -231,9 +233,10 @@ int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
     return true;
   };
   if (!mark(0)) return KT_ERR_CUDA;
-  if (launch_gate_logits(r, T, x, w_gate, logits, err, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
   if (launch_gate_select(r, T, logits, nullptr, bias, idx, w,
-                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), nullptr, st) != cudaSuccess)
+                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), st) != cudaSuccess)
     return KT_ERR_CUDA;
   if (!mark(1)) return KT_ERR_CUDA;
   if (launch_permute(r, T, L, ws, idx, w, x, st) != cudaSuccess) return KT_ERR_CUDA;

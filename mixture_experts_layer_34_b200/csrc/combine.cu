@@ -2,7 +2,7 @@
 // "DeepSeekMoE 三改进" passage (DeepSeek-V3 model.py notes,
 // 73biji.xyz/llm_pp_dsv3) and the "加共享专家 z" step of "MoE 前向四步":
 //     y_t = sum_s out[shared row of (s, t)] + sum_j out[row_of[t, j]]  (+ u_t)
-// The weighted expert outputs were written per row by the down GEMM. The sum
+// The weighted expert outputs (fp32) were written per row by the down GEMM. The sum
 // runs in fp32 in a fixed order (shared experts, then the routed slots in key
 // order, then the residual), so the result does not depend on scheduling.
 // One CTA per token; 16-byte loads along the hidden dimension.
@@ -13,32 +13,37 @@
 namespace ktmoe {
 namespace {
 
-template <bool kBF16>
+// 8 (bf16 input) or 4 (fp32) elements per thread per iteration; y in bf16 or
+// fp32 (kF32Out).
+template <bool kBF16, bool kF32Out>
 __global__ void __launch_bounds__(128)
 combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __restrict__ row_of,
-               const void* __restrict__ expert_out, const void* __restrict__ x, void* __restrict__ y) {
+               const float* __restrict__ expert_out, const void* __restrict__ x,
+               void* __restrict__ y) {
+  constexpr int V = kBF16 ? 8 : 4;
   __shared__ int rows[kMaxShared + kMaxTopk];
   const int t = blockIdx.x;
   if (threadIdx.x < S) rows[threadIdx.x] = T_ * k + threadIdx.x * T_ + t;
   if (threadIdx.x < k) rows[S + threadIdx.x] = row_of[(int64_t)t * k + threadIdx.x];
   __syncthreads();
   const int nrow = S + k;
-  if (kBF16) {
-    const int nq = d / 8;
-    const uint4* src = static_cast<const uint4*>(expert_out);
-    for (int q = threadIdx.x; q < nq; q += blockDim.x) {
-      float acc[8];
+  const int nq = d / V;
+  for (int q = threadIdx.x; q < nq; q += blockDim.x) {
+    float acc[V];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      for (int j = 0; j < nrow; ++j) {
-        const uint4 v = src[(int64_t)rows[j] * nq + q];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < V; ++i) acc[i] = 0.f;
+    for (int j = 0; j < nrow; ++j) {
+      const float4* src = reinterpret_cast<const float4*>(expert_out + (int64_t)rows[j] * d) + q * (V / 4);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[2 * i] += __uint_as_float(w[i] << 16);
-          acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
-        }
+      for (int h = 0; h < V / 4; ++h) {
+        const float4 v = src[h];
+        acc[4 * h] += v.x;
+        acc[4 * h + 1] += v.y;
+        acc[4 * h + 2] += v.z;
+        acc[4 * h + 3] += v.w;
       }
+    }
+    if (kBF16) {
       if (add_residual) {
         const uint4 v = static_cast<const uint4*>(x)[(int64_t)t * nq + q];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -48,35 +53,29 @@ combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __r
           acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
         }
       }
-      uint4 o;
-      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+      if (kF32Out) {
+        float4* yo = static_cast<float4*>(y) + ((int64_t)t * nq + q) * 2;
+        yo[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        yo[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      } else {
+        uint4 o;
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-        ow[i] = *reinterpret_cast<const uint32_t*>(&p);
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+          ow[i] = *reinterpret_cast<const uint32_t*>(&p);
+        }
+        static_cast<uint4*>(y)[(int64_t)t * nq + q] = o;
       }
-      static_cast<uint4*>(y)[(int64_t)t * nq + q] = o;
-    }
-  } else {
-    const int nq = d / 4;
-    const float4* src = static_cast<const float4*>(expert_out);
-    for (int q = threadIdx.x; q < nq; q += blockDim.x) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int j = 0; j < nrow; ++j) {
-        const float4 v = src[(int64_t)rows[j] * nq + q];
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
+    } else {
       if (add_residual) {
         const float4 v = static_cast<const float4*>(x)[(int64_t)t * nq + q];
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+        acc[0] += v.x;
+        acc[1] += v.y;
+        acc[2] += v.z;
+        acc[3] += v.w;
       }
-      static_cast<float4*>(y)[(int64_t)t * nq + q] = acc;
+      static_cast<float4*>(y)[(int64_t)t * nq + q] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
   }
 }
@@ -86,12 +85,16 @@ combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __r
 cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* ws, const void* x,
                            void* y, cudaStream_t st) {
   const int32_t* row_of = reinterpret_cast<const int32_t*>(ws + L.row_of);
-  if (r.dtype == KT_DTYPE_BF16)
-    combine_kernel<true><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual, row_of,
-                                                      ws + L.expert_out, x, y);
+  const float* eo = reinterpret_cast<const float*>(ws + L.expert_out);
+  if (r.dtype == KT_DTYPE_BF16 && !r.y_fp32)
+    combine_kernel<true, false><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+                                                             row_of, eo, x, y);
+  else if (r.dtype == KT_DTYPE_BF16)
+    combine_kernel<true, true><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+                                                            row_of, eo, x, y);
   else
-    combine_kernel<false><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual, row_of,
-                                                       ws + L.expert_out, x, y);
+    combine_kernel<false, true><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+                                                             row_of, eo, x, y);
   return cudaGetLastError();
 }
 

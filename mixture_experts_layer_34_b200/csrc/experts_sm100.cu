@@ -5,7 +5,8 @@
 //     FFN_e(u) = W2_e (silu(W1_e u) * W3_e u),
 // runs as two grouped GEMMs over the expert-sorted token rows:
 //   up   : hidden[r, f]     = silu(<W1_e[f], u_r>) * <W3_e[f], u_r>
-//   down : expert_out[r, o] = w_r * <W2_e[o], hidden[r]>
+//   down : expert_out[r, o] = w_r * <W2_e[o], hidden[r]>   (fp32, so the
+//          combine sums unrounded terms)
 // with w_r the routing weight of row r (1 for shared-expert rows), as in the
 // "y[idx] += expert(x[idx]) * w" loop of "MoE 前向四步".
 //
@@ -15,7 +16,7 @@
 //   warp 1     allocates 512 TMEM columns; lane 0 issues tcgen05.mma
 //              (kind::f16, bf16 in, fp32 accumulate) and tcgen05.commit;
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator, SwiGLU (up) or the
-//              routing weight (down), bf16 store through a shared staging tile.
+//              routing weight (down), store through a shared staging tile.
 // Operands are swapped relative to the math (D^T = W X^T): the weight tile is
 // the M = 128 operand and the tokens of the chunk are N (a multiple of 16 up to
 // 128 for up, 256 for down), so an expert with few tokens costs an MMA of
@@ -41,27 +42,35 @@ constexpr int kBoxRows = 16;                 // token rows per TMA box
 constexpr int kThreads = 192;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-template <bool kUp>
+// Epilogue kinds of the grouped GEMM.
+constexpr int kKindUp = 0;      // hidden = silu(W1 u) * W3 u          (bf16 out)
+constexpr int kKindDown = 1;    // expert_out = w_r * W2 h             (fp32 out)
+constexpr int kKindLogits = 2;  // logits = W_g u, one group, implicit token chunks (fp32 out)
+
+template <int kKind>
 struct Cfg {
+  static constexpr bool kUp = kKind == kKindUp;
   static constexpr int kNumA = kUp ? 2 : 1;
-  static constexpr int kMaxN = kUp ? kUpChunk : kDownChunk;
+  static constexpr int kMaxN = kKind == kKindDown ? kDownChunk : kUpChunk;
   static constexpr int kBBytes = kMaxN * kBK * 2;
   static constexpr int kStageBytes = kNumA * kATileBytes + kBBytes;
   static constexpr int kAccCols = 256;       // TMEM columns per accumulator buffer
-  static constexpr int kStagingBytes = 4 * 16 * 32 * 2;
+  static constexpr int kOutBytes = kUp ? 2 : 4;   // bf16 hidden rows / fp32 expert outputs
+  static constexpr int kStagingBytes = 4 * 16 * 32 * 4;
   static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 256 + 1024;
 };
 
 struct GemmArgs {
   const Chunk* chunks;
   const int32_t* n_chunks;   // device: number of chunks
+  int implicit_rows;         // > 0: no chunk list; chunks of kMaxN rows over this many rows of group 0
   int n_ftiles;              // weight-row tiles per group
   int rows_per_group;        // weight rows per expert (I for up, d for down)
   int K;                     // reduction length (d for up, I for down)
   int E;                     // routed experts (up: groups >= E read x directly)
   int out_cols;              // valid output columns (I or d)
   int ldo;                   // output row stride in elements
-  __nv_bfloat16* out;
+  void* out;                 // up: bf16 hidden rows; down: fp32 weighted expert outputs
   const float* row_weight;   // down: weight of routed rows
   int n_routed_rows;         // T * k
   int* err;
@@ -193,23 +202,32 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
+template <int kKind>
+__device__ __forceinline__ Chunk get_chunk(const GemmArgs& a, int ci) {
+  if (a.implicit_rows > 0) {
+    constexpr int n = Cfg<kKind>::kMaxN;
+    return Chunk{0, ci * n, min(n, a.implicit_rows - ci * n), ci * n};
+  }
+  return a.chunks[ci];
+}
+
 // ---------------------------------------------------------------------------
 // The grouped GEMM kernel
 // ---------------------------------------------------------------------------
-template <bool kUp>
+template <int kKind>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2 (down)
                     const __grid_constant__ CUtensorMap tmA1,   // W3 (up)
                     const __grid_constant__ CUtensorMap tmB0,   // permuted x (up) or hidden (down)
                     const __grid_constant__ CUtensorMap tmB1,   // x (up, shared experts)
                     const GemmArgs args) {
-  using C = Cfg<kUp>;
+  using C = Cfg<kKind>;
+  constexpr bool kUp = C::kUp;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* stage_base = smem;
-  __nv_bfloat16* staging =
-      reinterpret_cast<__nv_bfloat16*>(smem + kStages * C::kStageBytes);
+  uint8_t* staging = smem + kStages * C::kStageBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes + C::kStagingBytes);
   uint64_t* full_bar = bars;                    // [kStages]
   uint64_t* empty_bar = bars + kStages;         // [kStages]
@@ -243,7 +261,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int n_chunks = *args.n_chunks;
+  const int n_chunks = args.implicit_rows > 0 ? (args.implicit_rows + C::kMaxN - 1) / C::kMaxN
+                                              : *args.n_chunks;
   const int n_tiles = n_chunks * args.n_ftiles;
   const int nk = (args.K + kBK - 1) / kBK;
   int* err = args.err;
@@ -256,7 +275,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
       bool ok = true;
       int issued = 0;   // loads issued and not yet known complete (drained on error)
       for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-        const Chunk ch = args.chunks[tile / args.n_ftiles];
+        const Chunk ch = get_chunk<kKind>(args, tile / args.n_ftiles);
         const int ft = tile % args.n_ftiles;
         const int nb = (ch.nrows + kBoxRows - 1) & ~(kBoxRows - 1);
         const int a_row = ch.group * args.rows_per_group + ft * kWRows;
@@ -268,7 +287,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
         }
         const uint32_t tx = C::kNumA * kATileBytes + nb * kBK * 2;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, err, 1)) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, err, 1 + 8 * kKind)) {
             ok = false;
             break;
           }
@@ -312,9 +331,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
       bool ok = true;
       bool issued_any = false;
       for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-        const Chunk ch = args.chunks[tile / args.n_ftiles];
+        const Chunk ch = get_chunk<kKind>(args, tile / args.n_ftiles);
         const int nb = (ch.nrows + kBoxRows - 1) & ~(kBoxRows - 1);
-        if (!mbar_wait(&tempty_bar[buf], bphase ^ 1u, err, 2)) {
+        if (!mbar_wait(&tempty_bar[buf], bphase ^ 1u, err, 2 + 8 * kKind)) {
           ok = false;
           break;
         }
@@ -322,7 +341,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
         const uint32_t idesc = idesc_bf16(kWRows, nb);
         const uint32_t d0 = tmem_base + buf * C::kAccCols;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, err, 3)) {
+          if (!mbar_wait(&full_bar[stage], phase, err, 3 + 8 * kKind)) {
             ok = false;
             break;
           }
@@ -362,15 +381,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
   } else {
     // ---------------- Epilogue (warps 2..5) ----------------
     const int q = warp & 3;              // TMEM lane quarter this warp may access
-    __nv_bfloat16* stg = staging + (warp - 2) * 16 * 32;
+    uint8_t* stg = staging + (warp - 2) * 16 * 32 * 4;
     int buf = 0;
     uint32_t bphase = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-      const Chunk ch = args.chunks[tile / args.n_ftiles];
+      const Chunk ch = get_chunk<kKind>(args, tile / args.n_ftiles);
       const int ft = tile % args.n_ftiles;
       const int nb = (ch.nrows + kBoxRows - 1) & ~(kBoxRows - 1);
       // The outcome must be warp-uniform: tcgen05.ld below is .sync.aligned.
-      const bool ready = mbar_wait(&tfull_bar[buf], bphase, err, 4);
+      const bool ready = mbar_wait(&tfull_bar[buf], bphase, err, 4 + 8 * kKind);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
@@ -387,26 +406,39 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
         } else {
           tmem_ld16(tbase + c0, h);
           tmem_ld_wait();
+          if (kKind == kKindDown) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int row = ch.row0 + c0 + i;
-            const float wr = row < args.n_routed_rows ? args.row_weight[row] : 1.0f;
-            h[i] *= wr;
+            for (int i = 0; i < 16; ++i) {
+              const int row = ch.row0 + c0 + i;
+              const float wr = row < args.n_routed_rows ? args.row_weight[row] : 1.0f;
+              h[i] *= wr;
+            }
           }
         }
-        // Transpose through shared memory: stg[token][feature].
+        // Transpose through shared memory: stg[token][feature], then 16-byte
+        // stores along each output row (32 features = 64 B bf16 / 128 B fp32).
+        if (kUp) {
+          __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) stg[i * 32 + lane] = __float2bfloat16_rn(h[i]);
+          for (int i = 0; i < 16; ++i) sb[i * 32 + lane] = __float2bfloat16_rn(h[i]);
+        } else {
+          float* sf = reinterpret_cast<float*>(stg);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) sf[i * 32 + lane] = h[i];
+        }
         __syncwarp();
+        constexpr int kChunksPerRow = 32 * C::kOutBytes / 16;
+        constexpr int kElemsPerChunk = 16 / C::kOutBytes;
 #pragma unroll
-        for (int it = 0; it < 2; ++it) {
-          const int idx = lane + it * 32;     // 16 rows x 4 chunks of 16 B
-          const int rr = idx >> 2, part = idx & 3;
+        for (int it = 0; it < 16 * kChunksPerRow / 32; ++it) {
+          const int idx = lane + it * 32;
+          const int rr = idx / kChunksPerRow, part = idx % kChunksPerRow;
           const int c = c0 + rr;
-          const int col = col0 + part * 8;
+          const int col = col0 + part * kElemsPerChunk;
           if (c < ch.nrows && col < args.out_cols) {
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 32 + part * 8);
-            *reinterpret_cast<uint4*>(args.out + (int64_t)(ch.row0 + c) * args.ldo + col) = v;
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 32 * C::kOutBytes + part * 16);
+            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
+                                      ((int64_t)(ch.row0 + c) * args.ldo + col) * C::kOutBytes) = v;
           }
         }
         __syncwarp();
@@ -465,10 +497,10 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
          CUDA_SUCCESS;
 }
 
-template <bool kUp>
+template <int kKind>
 cudaError_t set_smem_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Cfg<kUp>::kSmemBytes);
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kKind>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<kKind>::kSmemBytes);
 }
 
 }  // namespace
@@ -491,7 +523,7 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
         !make_map(&mW3, wb, (uint64_t)NG * r.I, r.d, kWRows) ||
         !make_map(&mXp, ws + L.xperm, Rr, r.d, kBoxRows) || !make_map(&mX, x, T, r.d, kBoxRows))
       return cudaErrorInvalidValue;
-    cudaError_t e = set_smem_attr<true>();
+    cudaError_t e = set_smem_attr<kKindUp>();
     if (e != cudaSuccess) return e;
     a.chunks = reinterpret_cast<const Chunk*>(ws + L.up_chunks);
     a.n_chunks = meta + 0;
@@ -500,15 +532,15 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
     a.K = r.d;
     a.out_cols = r.I;
     a.ldo = r.I;
-    a.out = reinterpret_cast<__nv_bfloat16*>(ws + L.hidden);
+    a.out = ws + L.hidden;
     a.row_weight = nullptr;
-    grouped_gemm_kernel<true><<<num_sms, kThreads, Cfg<true>::kSmemBytes, st>>>(mW1, mW3, mXp, mX, a);
+    grouped_gemm_kernel<kKindUp><<<num_sms, kThreads, Cfg<kKindUp>::kSmemBytes, st>>>(mW1, mW3, mXp, mX, a);
   } else {
     CUtensorMap mW2, mH;
     if (!make_map(&mW2, wa, (uint64_t)NG * r.d, r.I, kWRows) ||
         !make_map(&mH, ws + L.hidden, R, r.I, kBoxRows))
       return cudaErrorInvalidValue;
-    cudaError_t e = set_smem_attr<false>();
+    cudaError_t e = set_smem_attr<kKindDown>();
     if (e != cudaSuccess) return e;
     a.chunks = reinterpret_cast<const Chunk*>(ws + L.down_chunks);
     a.n_chunks = meta + 1;
@@ -517,10 +549,38 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
     a.K = r.I;
     a.out_cols = r.d;
     a.ldo = r.d;
-    a.out = reinterpret_cast<__nv_bfloat16*>(ws + L.expert_out);
+    a.out = ws + L.expert_out;
     a.row_weight = reinterpret_cast<const float*>(ws + L.row_weight);
-    grouped_gemm_kernel<false><<<num_sms, kThreads, Cfg<false>::kSmemBytes, st>>>(mW2, mW2, mH, mH, a);
+    grouped_gemm_kernel<kKindDown><<<num_sms, kThreads, Cfg<kKindDown>::kSmemBytes, st>>>(mW2, mW2, mH, mH, a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, const void* w_gate,
+                                  float* logits, int* err, int num_sms, cudaStream_t st) {
+  CUtensorMap mWg, mX;
+  if (!make_map(&mWg, w_gate, (uint64_t)r.E, r.d, kWRows) || !make_map(&mX, x, T, r.d, kBoxRows))
+    return cudaErrorInvalidValue;
+  cudaError_t e = set_smem_attr<kKindLogits>();
+  if (e != cudaSuccess) return e;
+  GemmArgs a{};
+  a.chunks = nullptr;
+  a.n_chunks = nullptr;
+  a.implicit_rows = (int)T;
+  a.n_ftiles = (r.E + kWRows - 1) / kWRows;
+  a.rows_per_group = r.E;
+  a.K = r.d;
+  a.E = 1;                  // every chunk reads its token rows from the first B map
+  a.out_cols = r.E;
+  a.ldo = r.E;
+  a.out = logits;
+  a.row_weight = nullptr;
+  a.n_routed_rows = 0;
+  a.err = err;
+  const int tiles = (int)((T + kUpChunk - 1) / kUpChunk) * a.n_ftiles;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  grouped_gemm_kernel<kKindLogits><<<grid, kThreads, Cfg<kKindLogits>::kSmemBytes, st>>>(
+      mWg, mWg, mX, mX, a);
   return cudaGetLastError();
 }
 

@@ -3,7 +3,11 @@
 // model.py notes (73biji.xyz/llm_pp_dsv3) and the bias rule of its
 // "V3 改进①：无辅助损失负载均衡" section.
 //
-//   gate_logits_kernel : l = u W_g^T, fp32 FMA accumulation, register-tiled.
+//   logits             : l = u W_g^T with fp32 accumulation. bf16 layers with
+//                        more than 64 tokens use the tcgen05 grouped GEMM
+//                        (experts_sm100.cu); otherwise gate_logits_small_kernel
+//                        (one warp per expert, for few tokens) or the
+//                        register-tiled gate_logits_kernel (fp32 layers).
 //   gate_select_kernel : one warp per token; scores, keys s + b, group scores,
 //                        top topk_groups groups, top-k experts, weights. Each
 //                        CTA covers one 32-token chunk and also writes that
@@ -74,13 +78,9 @@ __device__ __forceinline__ void load_slab(const T* src, int64_t ld, int nrows, i
 template <typename T>
 __global__ void __launch_bounds__(kLThreads)
 gate_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg, float* __restrict__ logits,
-                   int T_, int E, int d, int* err_reset) {
+                   int T_, int E, int d) {
   __shared__ float xs[kLK][kLT + 4];
   __shared__ float ws[kLK][kLE + 4];
-  if (err_reset && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    err_reset[0] = 0;
-    err_reset[1] = 0;
-  }
   const int e0 = blockIdx.x * kLE;
   const int t0 = blockIdx.y * kLT;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -123,6 +123,49 @@ gate_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg, float* __r
 }
 
 // ---------------------------------------------------------------------------
+// Logits for few tokens: one warp per expert streams its W_g row once (16-byte
+// loads split over the lanes) against up to 8 token rows at a time, then
+// reduces across the lanes.
+// ---------------------------------------------------------------------------
+constexpr int kSmallWarps = 4, kSmallTok = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kSmallWarps * 32)
+gate_logits_small_kernel(const T* __restrict__ x, const T* __restrict__ wg,
+                         float* __restrict__ logits, int T_, int E, int d) {
+  constexpr int VN = Vec16<T>::n;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int e = blockIdx.x * kSmallWarps + warp;
+  if (e >= E) return;
+  const int nc = d / VN;
+  const T* wrow = wg + (int64_t)e * d;
+  for (int t0 = 0; t0 < T_; t0 += kSmallTok) {
+    float acc[kSmallTok];
+#pragma unroll
+    for (int j = 0; j < kSmallTok; ++j) acc[j] = 0.f;
+    for (int c = lane; c < nc; c += 32) {
+      float wv[VN];
+      Vec16<T>::load(wrow + c * VN, wv);
+#pragma unroll
+      for (int j = 0; j < kSmallTok; ++j) {
+        if (t0 + j < T_) {
+          float xv[VN];
+          Vec16<T>::load(x + (int64_t)(t0 + j) * d + c * VN, xv);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[j] = fmaf(wv[i], xv[i], acc[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kSmallTok; ++j) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+      if (lane == 0 && t0 + j < T_) logits[(int64_t)(t0 + j) * E + e] = acc[j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Selection: 8 warps per CTA, 4 tokens per warp, 32 tokens per CTA.
 // Lane l holds experts e = i*32 + l, i < ceil(E/32) (at most 16).
 // ---------------------------------------------------------------------------
@@ -155,13 +198,9 @@ __global__ void __launch_bounds__(kSelWarps * 32)
 gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
                    const float* __restrict__ scores_in, const float* __restrict__ bias,
                    int32_t* __restrict__ out_idx, float* __restrict__ out_w,
-                   int32_t* __restrict__ chunk_counts, int* err_reset) {
+                   int32_t* __restrict__ chunk_counts) {
   __shared__ int scount[kMaxExperts];
   __shared__ float skey[kSelWarps][kMaxExperts];
-  if (err_reset && blockIdx.x == 0 && threadIdx.x == 0) {
-    err_reset[0] = 0;
-    err_reset[1] = 0;
-  }
   const int E = r.E, k = r.k, G = r.G, gs = r.gs;
   const int nper = (E + 31) / 32;
   for (int e = threadIdx.x; e < E; e += blockDim.x) scount[e] = 0;
@@ -307,23 +346,36 @@ gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
 }  // namespace
 
 cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, const void* w_gate,
-                               float* logits, int* err_reset, cudaStream_t st) {
+                               float* logits, int* err, int num_sms, cudaStream_t st) {
+  const bool bf16 = r.dtype == KT_DTYPE_BF16;
+  if (T <= 64) {
+    const unsigned grid = (unsigned)((r.E + kSmallWarps - 1) / kSmallWarps);
+    if (bf16)
+      gate_logits_small_kernel<__nv_bfloat16><<<grid, kSmallWarps * 32, 0, st>>>(
+          (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d);
+    else
+      gate_logits_small_kernel<float><<<grid, kSmallWarps * 32, 0, st>>>(
+          (const float*)x, (const float*)w_gate, logits, (int)T, r.E, r.d);
+    return cudaGetLastError();
+  }
+  // Tensor-core logits write 16-byte chunks of fp32 rows of E entries.
+  if (bf16 && r.E % 4 == 0) return launch_gate_logits_tc(r, T, x, w_gate, logits, err, num_sms, st);
   dim3 grid((r.E + kLE - 1) / kLE, (unsigned)((T + kLT - 1) / kLT));
-  if (r.dtype == KT_DTYPE_BF16)
+  if (bf16)
     gate_logits_kernel<__nv_bfloat16><<<grid, kLThreads, 0, st>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d, err_reset);
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d);
   else
     gate_logits_kernel<float><<<grid, kLThreads, 0, st>>>((const float*)x, (const float*)w_gate,
-                                                          logits, (int)T, r.E, r.d, err_reset);
+                                                          logits, (int)T, r.E, r.d);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits,
                                const float* scores_in, const float* bias, int32_t* idx, float* w,
-                               int32_t* chunk_counts, int* err_reset, cudaStream_t st) {
+                               int32_t* chunk_counts, cudaStream_t st) {
   const unsigned grid = (unsigned)((T + kPermChunk - 1) / kPermChunk);
   gate_select_kernel<<<grid, kSelWarps * 32, 0, st>>>(r, (int)T, logits, scores_in, bias, idx, w,
-                                                     chunk_counts, err_reset);
+                                                     chunk_counts);
   return cudaGetLastError();
 }
 

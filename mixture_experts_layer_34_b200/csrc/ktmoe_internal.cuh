@@ -37,6 +37,7 @@ struct Resolved {
   int group_score;  // KT_GROUP_AMAX / KT_GROUP_TOP2SUM (G == 1: unused)
   int dtype;        // KT_DTYPE_*
   int add_residual;
+  int y_fp32;       // y in fp32 (else in dtype)
   int has_bias;
 };
 
@@ -68,7 +69,7 @@ struct Layout {
   size_t down_chunks;  // Chunk [max_down]
   size_t xperm;        // dtype [T*k, d] (bf16 layers only)
   size_t hidden;       // dtype [T*(k+S), I]
-  size_t expert_out;   // dtype [T*(k+S), d]
+  size_t expert_out;   // fp32 [T*(k+S), d]
   size_t total;
   int64_t nperm, max_up, max_down;
 };
@@ -80,10 +81,13 @@ Layout make_layout(const Resolved& r, int64_t T);
 // Kernel launchers (each returns the cudaError_t of its launch)
 // ---------------------------------------------------------------------------
 cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, const void* w_gate,
-                               float* logits, int* err_reset, cudaStream_t st);
+                               float* logits, int* err, int num_sms, cudaStream_t st);
+// bf16 logits on the tensor cores (the grouped GEMM with one group); E % 4 == 0.
+cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, const void* w_gate,
+                                  float* logits, int* err, int num_sms, cudaStream_t st);
 cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits,
                                const float* scores_in, const float* bias, int32_t* idx,
-                               float* w, int32_t* chunk_counts, int* err_reset, cudaStream_t st);
+                               float* w, int32_t* chunk_counts, cudaStream_t st);
 cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* ws,
                            const int32_t* idx, const float* w, const void* x, cudaStream_t st);
 // up = true: the gate/up GEMM (wa = W1, wb = W3); up = false: the down GEMM

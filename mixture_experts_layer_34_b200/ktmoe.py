@@ -33,7 +33,7 @@ class kt_moe_config(ctypes.Structure):
                 ("dim", ctypes.c_int32), ("inter", ctypes.c_int32),
                 ("n_shared", ctypes.c_int32), ("norm_topk", ctypes.c_int32),
                 ("group_score", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("add_residual", ctypes.c_int32)]
+                ("add_residual", ctypes.c_int32), ("y_fp32", ctypes.c_int32)]
 
 
 class kt_moe_ws_layout(ctypes.Structure):
@@ -91,10 +91,11 @@ def strerror(code: int) -> str:
 
 def make_config(n_experts, n_groups, topk_groups, topk, route_scale, score_func, dim, inter,
                 n_shared, norm_topk=-1, group_score=KT_GROUP_AUTO, dtype=KT_DTYPE_BF16,
-                add_residual=0) -> kt_moe_config:
+                add_residual=0, y_fp32=0) -> kt_moe_config:
     return kt_moe_config(int(n_experts), int(n_groups), int(topk_groups), int(topk),
                          float(route_scale), int(score_func), int(dim), int(inter), int(n_shared),
-                         int(norm_topk), int(group_score), int(dtype), int(add_residual))
+                         int(norm_topk), int(group_score), int(dtype), int(add_residual),
+                         int(y_fp32))
 
 
 def _ptr(t):
@@ -181,10 +182,10 @@ def kt_moe_version() -> int:
     return lib().kt_moe_version()
 
 
-def config_for(layer) -> kt_moe_config:
+def config_for(layer, y_fp32: bool = False) -> kt_moe_config:
     """kt_moe_config of a workloads.LayerConfig."""
     return make_config(dtype=KT_DTYPE_F32 if layer.dtype == "f32" else KT_DTYPE_BF16,
-                       **layer.kernel_fields())
+                       y_fp32=int(y_fp32), **layer.kernel_fields())
 
 
 def alloc_workspace(cfg: kt_moe_config, T: int, device="cuda"):

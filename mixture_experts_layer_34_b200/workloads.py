@@ -134,6 +134,16 @@ SMALL = [
 ]
 BY_NAME.update({c.name: c for c in SMALL})
 
+# Reduced V3-shaped layer (d, I, k, S, groups of the V3 layer; 32 experts, about
+# 3 GB of weights) for full ncu captures, which must stay a few GB on the device.
+PROFILE = [
+    LayerConfig("v3_shape_T2048_E32_profile", T=2048, dim=7168, n_experts=32, n_groups=8,
+                topk_groups=4, topk=8, n_shared=1, inter=2048, score_func=SIGMOID,
+                route_scale=2.5, norm_topk=-1, group_score=GROUP_TOP2SUM, dtype="bf16",
+                bias="normal", seed=2101),
+]
+BY_NAME.update({c.name: c for c in PROFILE})
+
 
 def torch_dtype(cfg: LayerConfig) -> torch.dtype:
     return torch.float32 if cfg.dtype == "f32" else torch.bfloat16

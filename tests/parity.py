@@ -17,13 +17,14 @@ def tolerance(layer) -> float:
     return TOL_F32 if layer.dtype == "f32" else TOL_BF16
 
 
-def run_forward(layer, inp, T=None, ws=None):
+def run_forward(layer, inp, T=None, ws=None, y_fp32=False):
     """One kt_moe_forward on the current stream; returns y, idx, w, workspace."""
     T = layer.T if T is None else T
-    cfg = K.config_for(layer)
+    cfg = K.config_for(layer, y_fp32=y_fp32)
     dev = inp["x"].device
     ws = K.alloc_workspace(cfg, T, dev) if ws is None else ws
-    y = torch.empty((T, layer.dim), dtype=inp["x"].dtype, device=dev)
+    ydt = torch.float32 if y_fp32 else inp["x"].dtype
+    y = torch.empty((T, layer.dim), dtype=ydt, device=dev)
     idx = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
     w = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
     K.kt_moe_forward(cfg, T, inp["x"], inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],

@@ -38,7 +38,7 @@ def test_library_links_no_torch():
 
 
 def test_config_struct_layout_matches_header():
-    assert ctypes.sizeof(K.kt_moe_config) == 13 * 4
+    assert ctypes.sizeof(K.kt_moe_config) == 14 * 4
     assert ctypes.sizeof(K.kt_moe_ws_layout) == 10 * 8
 
 
@@ -62,7 +62,7 @@ BAD = [
     dict(topk=9),                                                         # > TG * E/G = 8
     dict(n_shared=-1), dict(n_shared=9), dict(route_scale=0.0), dict(route_scale=float("inf")),
     dict(route_scale=float("nan")), dict(score_func=2), dict(dtype=3), dict(dim=12),
-    dict(inter=4), dict(norm_topk=2), dict(group_score=3), dict(add_residual=2),
+    dict(inter=4), dict(norm_topk=2), dict(group_score=3), dict(add_residual=2), dict(y_fp32=2),
     dict(n_experts=16, n_groups=16, topk_groups=4, topk=4, group_score=2),  # top-2 of 1 expert
 ]
 

@@ -2,8 +2,16 @@
 
 Outputs must match the oracle within max|dy| <= 2e-2 * RMS(y_ref) for bf16
 layers and 1e-4 * RMS(y_ref) for fp32 ones; tokens whose routing differs from
-the oracle's (allowed only at near ties) are excluded and counted. The
-permutation buffers are compared exactly.
+the oracle's (allowed only at near ties) are excluded and counted.
+
+For bf16 layers the tolerance is checked on the fp32 form of the output (the
+config's y_fp32 switch: the fp32 sum before its final rounding), and the bf16
+output is checked to be exactly that sum rounded to nearest-even. A bf16 output
+cannot be closer to the exact value than half a bf16 ulp, up to 2^-8 |y|, which
+at the largest elements is already about 2% of the RMS; splitting the check
+keeps the 2e-2 bound on the arithmetic the kernels do.
+
+The permutation buffers are compared exactly.
 """
 from __future__ import annotations
 
@@ -22,7 +30,12 @@ pytestmark = pytest.mark.gpu
 
 
 def _check_layer(layer, inp, tok_ids, out=None):
-    out = out or run_forward(layer, inp)
+    out = out or run_forward(layer, inp, y_fp32=True)
+    if layer.dtype == "bf16":
+        assert out["y"].dtype == torch.float32
+        out16 = run_forward(layer, inp)
+        assert torch.equal(out16["idx"], out["idx"])
+        assert torch.equal(out16["y"], out["y"].to(torch.bfloat16)), "bf16 y is not round(fp32 y)"
     og = oracle_gate(layer, inp)
     idx = out["idx"].cpu().numpy()
     diff, near = routing_agreement(layer, og, idx)
@@ -54,7 +67,7 @@ def test_named_layers_sampled_tokens(layer):
 def test_v3_prefill_zipf_sampled_tokens():
     layer = W.V3_PREFILL
     inp = W.make_layer(layer, "cuda")
-    out = run_forward(layer, inp)
+    out = run_forward(layer, inp, y_fp32=True)
     og = oracle_gate(layer, inp)
     # include the first/last token and tokens routed to the lightest experts
     load = np.bincount(og["idx"].ravel(), minlength=layer.n_experts)
@@ -176,8 +189,8 @@ def test_workspace_reuse_across_layers():
     """One workspace sized for the larger layer serves a smaller one afterwards."""
     big = W.BY_NAME["small_sig_bias"]
     small = W.BY_NAME["small_softmax_ragged"]
-    ws = K.alloc_workspace(K.config_for(big), big.T)
-    assert ws.numel() >= K.kt_moe_workspace_size(K.config_for(small), small.T)
+    ws = K.alloc_workspace(K.config_for(big, y_fp32=True), 2 * big.T)
+    assert ws.numel() >= K.kt_moe_workspace_size(K.config_for(small, y_fp32=True), small.T)
     inp = W.make_layer(small, "cuda")
-    out = run_forward(small, inp, ws=ws)
+    out = run_forward(small, inp, ws=ws, y_fp32=True)
     _check_layer(small, inp, list(range(0, small.T, 7)), out=out)

@@ -18,7 +18,9 @@ from parity import NEAR_TIE, oracle_gate
 
 pytestmark = pytest.mark.gpu
 
-LAYERS = W.NAMED + W.SMALL
+# bf16 with E % 4 != 0 and T > 64: the register-tiled SIMT logits path.
+ODD_E = W.BY_NAME["small_sig_bias"].with_(name="small_E30_simt_logits", n_experts=30, n_groups=3)
+LAYERS = W.NAMED + W.SMALL + [ODD_E]
 
 
 def _gpu_gate(layer, inp, scores_in=None):
@@ -56,7 +58,9 @@ def test_gate_from_tokens_matches_up_to_near_ties(layer):
     near = (og["kth_margin"] <= NEAR_TIE) | (og["grp_margin"] <= NEAR_TIE)
     assert near[diff].all(), f"routing differs away from a near tie at tokens {diff[~near[diff]]}"
     same = np.setdiff1d(np.arange(layer.T), diff)
-    np.testing.assert_allclose(w[same], og["w"][same], rtol=2e-6, atol=1e-7)
+    # The weights inherit the fp32 logits' accumulation error (about 1e-5 at
+    # d = 7168) through the score function.
+    np.testing.assert_allclose(w[same], og["w"][same], rtol=1e-4, atol=1e-6)
     print(f"{layer.name}: {len(diff)} near-tie routing differences, {near.sum()} near ties")
 
 
