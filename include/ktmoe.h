@@ -165,7 +165,11 @@ int kt_moe_check(const void* workspace, void* stream);
  * [E+S]; offsets: exclusive prefix [E+S+1]; row_of: [T, k] row of (t, j) in the
  * expert-sorted order; tok_of: [T*k] token of each sorted row; hidden: SwiGLU
  * hidden rows [T*(k+S), inter] (dtype); expert_out: weighted expert outputs
- * [T*(k+S), dim] (fp32). Rows T*k + s*T + t belong to shared expert s. */
+ * [T*(k+S), dim] (fp32). Rows T*k + s*T + t belong to shared expert s.
+ * meta: int32 [3] = number of GEMM chunks, gate/up tiles, down tiles; chunks:
+ * int32 [n][4] = (group, first row, rows, first activation row) of chunks of at
+ * most 256 rows; tiles_up / tiles_down: int32 [n][2] = (chunk, feature tile)
+ * in schedule order (feature tiles of 128 / 256 rows). */
 typedef struct {
   int64_t error_word;
   int64_t logits;
@@ -176,6 +180,10 @@ typedef struct {
   int64_t row_weight;
   int64_t hidden;
   int64_t expert_out;
+  int64_t meta;
+  int64_t chunks;
+  int64_t tiles_up;
+  int64_t tiles_down;
   int64_t total;
 } kt_moe_ws_layout;
 

@@ -97,8 +97,7 @@ Layout make_layout(const Resolved& r, int64_t T) {
   const size_t R = (size_t)T * (r.k + r.S);
   const size_t es = r.dtype == KT_DTYPE_BF16 ? 2 : 4;
   L.nperm = (T + kPermChunk - 1) / kPermChunk;
-  L.max_up = (int64_t)(R / kUpChunk + NG + 1);
-  L.max_down = (int64_t)(R / kDownChunk + NG + 1);
+  L.max_chunks = (int64_t)(R / kChunkRows + NG + 1);
   L.err = take(256, 256);
   L.meta = take(64, 256);
   L.logits = take((size_t)T * r.E * 4, 256);
@@ -111,8 +110,9 @@ Layout make_layout(const Resolved& r, int64_t T) {
   L.row_of = take(Tk * 4, 256);
   L.tok_of = take(Tk * 4, 256);
   L.row_weight = take(Tk * 4, 256);
-  L.up_chunks = take((size_t)L.max_up * sizeof(Chunk), 256);
-  L.down_chunks = take((size_t)L.max_down * sizeof(Chunk), 256);
+  L.chunks = take((size_t)L.max_chunks * sizeof(Chunk), 256);
+  L.tiles_up = take((size_t)L.max_chunks * ((r.I + 127) / 128) * 8, 256);
+  L.tiles_down = take((size_t)L.max_chunks * ((r.d + 255) / 256) * 8, 256);
   L.xperm = take(r.dtype == KT_DTYPE_BF16 ? Tk * r.d * es : 0, 1024);
   L.hidden = take(R * r.I * es, 1024);
   L.expert_out = take(R * r.d * 4, 1024);   // fp32 for every dtype
@@ -155,6 +155,10 @@ int kt_moe_workspace_layout(const kt_moe_config* cfg, int64_t T, kt_moe_ws_layou
   out->row_weight = (int64_t)L.row_weight;
   out->hidden = (int64_t)L.hidden;
   out->expert_out = (int64_t)L.expert_out;
+  out->meta = (int64_t)L.meta;
+  out->chunks = (int64_t)L.chunks;
+  out->tiles_up = (int64_t)L.tiles_up;
+  out->tiles_down = (int64_t)L.tiles_down;
   out->total = (int64_t)L.total;
   return KT_OK;
 }

@@ -28,7 +28,7 @@ up_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_ch
   __shared__ float bs[kTB][kTK + 1];
   __shared__ int tok[kTB];
   const int n_chunks = *n_chunks_p;
-  const int rblocks = kUpChunk / kTB;
+  const int rblocks = kChunkRows / kTB;
   const int fblocks = (I + kTB - 1) / kTB;
   const int ntiles = n_chunks * rblocks * fblocks;
   const int ty = threadIdx.x / 8, tx = threadIdx.x % 8;   // row ty, columns tx*4..+3
@@ -90,7 +90,7 @@ down_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_
   __shared__ float hs[kTB][kTK + 1];
   __shared__ float ws[kTB][kTK + 1];
   const int n_chunks = *n_chunks_p;
-  const int rblocks = kDownChunk / kTB;
+  const int rblocks = kChunkRows / kTB;
   const int oblocks = (d + kTB - 1) / kTB;
   const int ntiles = n_chunks * rblocks * oblocks;
   const int ty = threadIdx.x / 8, tx = threadIdx.x % 8;
@@ -143,13 +143,13 @@ cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, ch
   const int grid = num_sms * 4;
   if (up) {
     up_f32_kernel<<<grid, 256, 0, st>>>(
-        reinterpret_cast<const Chunk*>(ws + L.up_chunks), meta + 0, r.E, r.d, r.I,
+        reinterpret_cast<const Chunk*>(ws + L.chunks), meta + 0, r.E, r.d, r.I,
         static_cast<const float*>(x), static_cast<const float*>(w1), static_cast<const float*>(w3),
         reinterpret_cast<const int32_t*>(ws + L.tok_of), reinterpret_cast<float*>(ws + L.hidden));
     return cudaGetLastError();
   }
   down_f32_kernel<<<grid, 256, 0, st>>>(
-      reinterpret_cast<const Chunk*>(ws + L.down_chunks), meta + 1, r.d, r.I, (int)(T * r.k),
+      reinterpret_cast<const Chunk*>(ws + L.chunks), meta + 0, r.d, r.I, (int)(T * r.k),
       reinterpret_cast<const float*>(ws + L.hidden), static_cast<const float*>(w2),
       reinterpret_cast<const float*>(ws + L.row_weight),
       reinterpret_cast<float*>(ws + L.expert_out));

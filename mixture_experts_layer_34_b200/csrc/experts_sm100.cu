@@ -1,28 +1,43 @@
-// Routed + shared expert SwiGLU FFNs on the sm_100a tensor cores.
+// Routed + shared expert SwiGLU FFNs (and the bf16 gate logits) on the sm_100a
+// tensor cores.
 //
 // The expert FFN of the total-output equation in the "DeepSeekMoE 三改进"
 // passage of the DeepSeek-V3 model.py notes (73biji.xyz/llm_pp_dsv3),
 //     FFN_e(u) = W2_e (silu(W1_e u) * W3_e u),
 // runs as two grouped GEMMs over the expert-sorted token rows:
-//   up   : hidden[r, f]     = silu(<W1_e[f], u_r>) * <W3_e[f], u_r>
-//   down : expert_out[r, o] = w_r * <W2_e[o], hidden[r]>   (fp32, so the
-//          combine sums unrounded terms)
+//   up   : hidden[r, f]     = silu(<W1_e[f], u_r>) * <W3_e[f], u_r>      (bf16)
+//   down : expert_out[r, o] = w_r * <W2_e[o], hidden[r]>                 (fp32)
 // with w_r the routing weight of row r (1 for shared-expert rows), as in the
-// "y[idx] += expert(x[idx]) * w" loop of "MoE 前向四步".
+// "y[idx] += expert(x[idx]) * w" loop of "MoE 前向四步". The same kernel with a
+// plain epilogue computes the gate logits W_g u (one group).
 //
-// Design (one persistent CTA per SM, 192 threads):
-//   warp 0     TMA producer: weight tile (128 rows x 64 K) and the token-row
-//              tile (N rows x 64 K, in 16-row boxes) into a 4-stage ring;
-//   warp 1     allocates 512 TMEM columns; lane 0 issues tcgen05.mma
-//              (kind::f16, bf16 in, fp32 accumulate) and tcgen05.commit;
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, SwiGLU (up) or the
-//              routing weight (down), store through a shared staging tile.
-// Operands are swapped relative to the math (D^T = W X^T): the weight tile is
-// the M = 128 operand and the tokens of the chunk are N (a multiple of 16 up to
-// 128 for up, 256 for down), so an expert with few tokens costs an MMA of
-// matching width instead of a 128-row tile of padding. Two accumulators (gate
-// and up) per tile for the up GEMM; two TMEM buffers so the epilogue of one tile
-// overlaps the main loop of the next.
+// Design: persistent CTA pairs (a 2-CTA cluster per pair of SMs), 192 threads
+// per CTA, tcgen05 with cta_group::2.
+//   - Operands are swapped relative to the math (D^T = W X^T): weights are the
+//     M = 256 operand (128 rows in each CTA of the pair) and the tokens of one
+//     chunk are N (a multiple of 32, at most 256; each CTA loads N/2 rows). An
+//     expert with 37 tokens runs an N = 64 MMA instead of a 128-row tile of
+//     padding, and decode streams weights at N = 32.
+//   - Gate/up: each CTA's 128 weight rows are [64 rows of W1 | the same 64 rows
+//     of W3] (two TMA boxes), so TMEM lanes 0-63 hold gate and 64-127 hold up of
+//     the same 64 features; the "up" epilogue warps hand their values to the
+//     "gate" warps through a double-buffered shared-memory exchange. One pair
+//     tile covers 128 features; down and logits tiles cover 256 rows.
+//   - Few, large TMA boxes per stage (TMA cost grows with the box count): the
+//     weight tile in one or two boxes, the token rows in one 128-row box for a
+//     full chunk, else in 32-row boxes.
+//   - warp 0: TMA producer (6-stage ring of 32 KB per CTA); warp 1: TMEM owner,
+//     and in the even CTA the single thread issuing tcgen05.mma for the pair;
+//     warps 2-5: epilogue (tcgen05.ld, SwiGLU / routing weight / none, staging
+//     through shared memory for 16-byte row stores).
+//   - Both CTAs' TMA loads signal the even CTA's "full" barrier; the MMA thread
+//     commits to the "empty" and "accumulator full" barriers of both CTAs; both
+//     epilogues arrive on the even CTA's "accumulator empty" barrier. Two TMEM
+//     accumulator buffers of 256 columns overlap the epilogue with the next tile.
+//   - The tile schedule (chunk, feature tile) is built on the device: within an
+//     expert, blocks of 8 token chunks run feature-tile-major, so the pairs that
+//     read one weight tile run together and share it through L2.
+// No TMA multicast is used.
 //
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the
 // kernel records KT_ERR_TIMEOUT in the workspace error word, drains what it
@@ -35,42 +50,46 @@
 namespace ktmoe {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kBK = 64;                      // K elements per stage (128 B of bf16)
-constexpr int kATileBytes = kWRows * kBK * 2;  // 16 KB
-constexpr int kBoxRows = 16;                 // token rows per TMA box
+constexpr int kStages = 6;
+constexpr int kBK = 64;                          // K elements per stage (128 B of bf16)
+constexpr int kARowsCta = 128;                   // weight rows per CTA (MMA M = 256 per pair)
+constexpr int kATileBytes = kARowsCta * kBK * 2;   // 16 KB
+constexpr int kBHalfMax = kChunkRows / 2;        // token rows per CTA
+constexpr int kBTileBytes = kBHalfMax * kBK * 2;   // 16 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kBoxRows = 32;                     // token-row TMA box for partial chunks
+constexpr int kBoxBytes = kBoxRows * kBK * 2;    // 4 KB
 constexpr int kThreads = 192;
+constexpr int kStagingBytes = 4 * 16 * 32 * 4;   // 4 epilogue warps x [16 tokens][32 x 4 B]
+constexpr int kXchgBytes = 2 * 2 * 16 * 32 * 4;  // up -> gate: 2 warp pairs x 2 buffers
+constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + kXchgBytes + 256 + 1024;
+constexpr int kAccCols = 256;                    // TMEM columns per accumulator buffer
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Epilogue kinds of the grouped GEMM.
-constexpr int kKindUp = 0;      // hidden = silu(W1 u) * W3 u          (bf16 out)
-constexpr int kKindDown = 1;    // expert_out = w_r * W2 h             (fp32 out)
-constexpr int kKindLogits = 2;  // logits = W_g u, one group, implicit token chunks (fp32 out)
+// Epilogue kinds.
+constexpr int kKindUp = 0;      // hidden = silu(W1 u) * W3 u            (bf16 out)
+constexpr int kKindDown = 1;    // expert_out = w_r * W2 h               (fp32 out)
+constexpr int kKindLogits = 2;  // logits = W_g u, implicit token chunks (fp32 out)
 
 template <int kKind>
-struct Cfg {
+struct Kind {
   static constexpr bool kUp = kKind == kKindUp;
-  static constexpr int kNumA = kUp ? 2 : 1;
-  static constexpr int kMaxN = kKind == kKindDown ? kDownChunk : kUpChunk;
-  static constexpr int kBBytes = kMaxN * kBK * 2;
-  static constexpr int kStageBytes = kNumA * kATileBytes + kBBytes;
-  static constexpr int kAccCols = 256;       // TMEM columns per accumulator buffer
-  static constexpr int kOutBytes = kUp ? 2 : 4;   // bf16 hidden rows / fp32 expert outputs
-  static constexpr int kStagingBytes = 4 * 16 * 32 * 4;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 256 + 1024;
+  static constexpr int kOutBytes = kUp ? 2 : 4;
+  static constexpr int kRowsPerPair = kUp ? 128 : 256;   // output features per pair tile
 };
 
 struct GemmArgs {
   const Chunk* chunks;
-  const int32_t* n_chunks;   // device: number of chunks
-  int implicit_rows;         // > 0: no chunk list; chunks of kMaxN rows over this many rows of group 0
-  int n_ftiles;              // weight-row tiles per group
-  int rows_per_group;        // weight rows per expert (I for up, d for down)
-  int K;                     // reduction length (d for up, I for down)
+  const int2* tiles;         // (chunk index, feature tile) in schedule order
+  const int32_t* n_tiles;    // device count of tiles
+  int implicit_rows;         // > 0: logits; chunks of kChunkRows over this many token rows
+  int n_ftiles;              // feature tiles per group
+  int rows_per_group;        // weight rows per group (I for up, d for down, E for logits)
+  int K;                     // reduction length
   int E;                     // routed experts (up: groups >= E read x directly)
-  int out_cols;              // valid output columns (I or d)
+  int out_cols;              // valid output columns
   int ldo;                   // output row stride in elements
-  void* out;                 // up: bf16 hidden rows; down: fp32 weighted expert outputs
+  void* out;
   const float* row_weight;   // down: weight of routed rows
   int n_routed_rows;         // T * k
   int* err;
@@ -81,6 +100,20 @@ struct GemmArgs {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -95,14 +128,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Arrive on a barrier given by its shared::cluster address (own or peer CTA).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
+               : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -125,12 +160,14 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
     }
   }
 }
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int c0, int c1) {
+// 2-D tiled TMA load into this CTA's shared memory, completing on the barrier
+// at shared::cluster address `bar` (the even CTA's, for the pair).
+__device__ __forceinline__ void tma_load_pair(void* dst, const CUtensorMap* map, uint32_t bar, int c0,
+                                              int c1) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -142,15 +179,15 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(slot)),
                "r"(ncols)
                : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
@@ -169,20 +206,21 @@ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accumulate) {
+__device__ __forceinline__ void mma_pair_bf16(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                              uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
+// Arrive once on the barrier at shared::cluster address `bar` when every MMA
+// this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
@@ -202,41 +240,55 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
-template <int kKind>
-__device__ __forceinline__ Chunk get_chunk(const GemmArgs& a, int ci) {
+__device__ __forceinline__ void get_tile(const GemmArgs& a, int t, Chunk& ch, int& ft) {
   if (a.implicit_rows > 0) {
-    constexpr int n = Cfg<kKind>::kMaxN;
-    return Chunk{0, ci * n, min(n, a.implicit_rows - ci * n), ci * n};
+    const int ci = t / a.n_ftiles;
+    ft = t % a.n_ftiles;
+    ch = Chunk{0, ci * kChunkRows, min(kChunkRows, a.implicit_rows - ci * kChunkRows),
+               ci * kChunkRows};
+  } else {
+    const int2 e = a.tiles[t];
+    ch = a.chunks[e.x];
+    ft = e.y;
   }
-  return a.chunks[ci];
 }
+
+// Token columns of a chunk rounded up so that each CTA of the pair gets a
+// multiple of 16 rows (the MMA N is then a multiple of 32).
+__device__ __forceinline__ int pair_cols(int nrows) { return (nrows + 31) & ~31; }
 
 // ---------------------------------------------------------------------------
 // The grouped GEMM kernel
 // ---------------------------------------------------------------------------
 template <int kKind>
-__global__ void __launch_bounds__(kThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2 (down)
-                    const __grid_constant__ CUtensorMap tmA1,   // W3 (up)
-                    const __grid_constant__ CUtensorMap tmB0,   // permuted x (up) or hidden (down)
-                    const __grid_constant__ CUtensorMap tmB1,   // x (up, shared experts)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_g
+                    const __grid_constant__ CUtensorMap tmA1,    // W3 (up)
+                    const __grid_constant__ CUtensorMap tmB0s,   // token rows, 32-row box
+                    const __grid_constant__ CUtensorMap tmB0l,   // token rows, 128-row box
+                    const __grid_constant__ CUtensorMap tmB1s,   // x (up, shared experts), 32-row box
+                    const __grid_constant__ CUtensorMap tmB1l,   // x, 128-row box
                     const GemmArgs args) {
-  using C = Cfg<kKind>;
-  constexpr bool kUp = C::kUp;
+  using KD = Kind<kKind>;
+  constexpr bool kUp = KD::kUp;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* stage_base = smem;
-  uint8_t* staging = smem + kStages * C::kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes + C::kStagingBytes);
-  uint64_t* full_bar = bars;                    // [kStages]
-  uint64_t* empty_bar = bars + kStages;         // [kStages]
-  uint64_t* tfull_bar = bars + 2 * kStages;     // [2]
-  uint64_t* tempty_bar = bars + 2 * kStages + 2;  // [2]
-  uint64_t* drain_bar = bars + 2 * kStages + 4;   // [1]
+  uint8_t* staging = smem + kStages * kStageBytes;
+  float* xchg = reinterpret_cast<float*>(smem + kStages * kStageBytes + kStagingBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kStagingBytes +
+                                               kXchgBytes);
+  uint64_t* full_bar = bars;                        // [kStages]  (even CTA's are used)
+  uint64_t* empty_bar = bars + kStages;             // [kStages]
+  uint64_t* tfull_bar = bars + 2 * kStages;         // [2]
+  uint64_t* tempty_bar = bars + 2 * kStages + 2;    // [2]        (even CTA's are used)
+  uint64_t* drain_bar = bars + 2 * kStages + 4;     // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank();             // 0: even (MMA-issuing) CTA, 1: odd
+  const bool leader = rank == 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -244,60 +296,86 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 4);
+      mbar_init(&tempty_bar[b], 8);     // 4 epilogue warps x 2 CTAs
     }
     mbar_init(drain_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmA0);
-    prefetch_tmap(&tmB0);
+    prefetch_tmap(&tmB0s);
+    prefetch_tmap(&tmB0l);
     if (kUp) {
       prefetch_tmap(&tmA1);
-      prefetch_tmap(&tmB1);
+      prefetch_tmap(&tmB1s);
+      prefetch_tmap(&tmB1l);
     }
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int n_chunks = args.implicit_rows > 0 ? (args.implicit_rows + C::kMaxN - 1) / C::kMaxN
-                                              : *args.n_chunks;
-  const int n_tiles = n_chunks * args.n_ftiles;
+  const int n_tiles = args.implicit_rows > 0
+                          ? ((args.implicit_rows + kChunkRows - 1) / kChunkRows) * args.n_ftiles
+                          : *args.n_tiles;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   const int nk = (args.K + kBK - 1) / kBK;
   int* err = args.err;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
+      // ---------------- TMA producer (both CTAs) ----------------
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int issued = 0;   // loads issued and not yet known complete (drained on error)
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-        const Chunk ch = get_chunk<kKind>(args, tile / args.n_ftiles);
-        const int ft = tile % args.n_ftiles;
-        const int nb = (ch.nrows + kBoxRows - 1) & ~(kBoxRows - 1);
-        const int a_row = ch.group * args.rows_per_group + ft * kWRows;
-        const CUtensorMap* bmap = &tmB0;
+      int issued = 0;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+        Chunk ch;
+        int ft;
+        get_tile(args, t, ch, ft);
+        const int half = pair_cols(ch.nrows) / 2;
+        // First weight row of this CTA's half of the pair tile.
+        const int a_row = ch.group * args.rows_per_group + ft * KD::kRowsPerPair +
+                          (kUp ? 64 : 128) * (int)rank;
+        const CUtensorMap* bs = &tmB0s;
+        const CUtensorMap* bl = &tmB0l;
         int b_row = ch.row0;
         if (kUp) {
           b_row = ch.src_row0;
-          if (ch.group >= args.E) bmap = &tmB1;
+          if (ch.group >= args.E) {
+            bs = &tmB1s;
+            bl = &tmB1l;
+          }
         }
-        const uint32_t tx = C::kNumA * kATileBytes + nb * kBK * 2;
+        b_row += half * (int)rank;
+        // Token rows: one 128-row box for a full half, else 32-row boxes (the
+        // last may run up to 16 rows past the chunk; those columns are unused).
+        const int nbox = half == kBHalfMax ? 0 : (half + kBoxRows - 1) / kBoxRows;
+        const uint32_t bbytes = nbox == 0 ? kBTileBytes : nbox * kBoxBytes;
+        const uint32_t tx = 2u * (kATileBytes + bbytes);   // both CTAs' bytes
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, err, 1 + 8 * kKind)) {
             ok = false;
             break;
           }
-          uint8_t* sb = stage_base + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&full_bar[stage], tx);
-          tma_load_2d(sb, &tmA0, &full_bar[stage], kb * kBK, a_row);
-          if (kUp) tma_load_2d(sb + kATileBytes, &tmA1, &full_bar[stage], kb * kBK, a_row);
-          uint8_t* sB = sb + C::kNumA * kATileBytes;
-          for (int rr = 0; rr < nb; rr += kBoxRows)
-            tma_load_2d(sB + rr * kBK * 2, bmap, &full_bar[stage], kb * kBK, b_row + rr);
+          const uint32_t fbar = map_to_cta(smem_u32(&full_bar[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
+          uint8_t* sA = stage_base + stage * kStageBytes;
+          uint8_t* sB = sA + kATileBytes;
+          const int kc = kb * kBK;
+          if (kUp) {
+            // [64 rows of W1 | the same 64 rows of W3]
+            tma_load_pair(sA, &tmA0, fbar, kc, a_row);
+            tma_load_pair(sA + 64 * 128, &tmA1, fbar, kc, a_row);
+          } else {
+            tma_load_pair(sA, &tmA0, fbar, kc, a_row);
+          }
+          if (nbox == 0) {
+            tma_load_pair(sB, bl, fbar, kc, b_row);
+          } else {
+            for (int i = 0; i < nbox; ++i)
+              tma_load_pair(sB + i * kBoxBytes, bs, fbar, kc, b_row + i * kBoxRows);
+          }
           issued = issued < kStages ? issued + 1 : kStages;
           if (++stage == kStages) {
             stage = 0;
@@ -305,9 +383,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
           }
         }
       }
-      if (!ok) {
-        // Let the copies already in flight land before the CTA can exit: wait
-        // (bounded) on the full barrier of each of the last `issued` stages.
+      if (!ok && leader) {
+        // Let the copies already in flight land before the CTA can exit.
         int s = stage;
         uint32_t ph = phase;
         for (int i = 0; i < issued; ++i) {
@@ -322,40 +399,42 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (even CTA, for the pair) ----------------
+      const uint32_t peer = 1;
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
       uint32_t bphase = 0;
       bool ok = true;
       bool issued_any = false;
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-        const Chunk ch = get_chunk<kKind>(args, tile / args.n_ftiles);
-        const int nb = (ch.nrows + kBoxRows - 1) & ~(kBoxRows - 1);
+      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+        Chunk ch;
+        int ft;
+        get_tile(args, t, ch, ft);
+        const int n = pair_cols(ch.nrows);
         if (!mbar_wait(&tempty_bar[buf], bphase ^ 1u, err, 2 + 8 * kKind)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(kWRows, nb);
-        const uint32_t d0 = tmem_base + buf * C::kAccCols;
+        const uint32_t idesc = idesc_bf16(256, n);
+        const uint32_t d0 = tmem_base + buf * kAccCols;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, err, 3 + 8 * kKind)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sb = smem_u32(stage_base + stage * C::kStageBytes);
-          const uint32_t sB = sb + C::kNumA * kATileBytes;
+          const uint32_t sA = smem_u32(stage_base + stage * kStageBytes);
+          const uint32_t sB = sA + kATileBytes;
 #pragma unroll
-          for (int ks = 0; ks < kBK / 16; ++ks) {
-            const uint64_t bdesc = sw128_desc(sB + ks * 32);
-            const uint32_t acc = (kb | ks) != 0;
-            mma_bf16(d0, sw128_desc(sb + ks * 32), bdesc, idesc, acc);
-            if (kUp) mma_bf16(d0 + 128, sw128_desc(sb + kATileBytes + ks * 32), bdesc, idesc, acc);
-          }
-          mma_commit(&empty_bar[stage]);
+          for (int ks = 0; ks < kBK / 16; ++ks)
+            mma_pair_bf16(d0, sw128_desc(sA + ks * 32), sw128_desc(sB + ks * 32), idesc,
+                          (kb | ks) != 0);
+          const uint32_t eb = smem_u32(&empty_bar[stage]);
+          mma_commit_pair(eb);
+          mma_commit_pair(map_to_cta(eb, peer));
           issued_any = true;
           if (++stage == kStages) {
             stage = 0;
@@ -363,89 +442,120 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
           }
         }
         if (!ok) break;
-        mma_commit(&tfull_bar[buf]);
+        const uint32_t fb = smem_u32(&tfull_bar[buf]);
+        mma_commit_pair(fb);
+        mma_commit_pair(map_to_cta(fb, peer));
         if (++buf == 2) {
           buf = 0;
           bphase ^= 1u;
         }
       }
-      // Wait (bounded) until every MMA this thread issued has completed, so TMEM
-      // and shared memory can be released.
+      // Wait (bounded) until every MMA issued has completed, so TMEM and shared
+      // memory can be released.
       if (issued_any) {
-        mma_commit(drain_bar);
+        mma_commit_pair(smem_u32(drain_bar));
         const uint64_t t0 = globaltimer();
         while (!mbar_try_wait(drain_bar, 0) && globaltimer() - t0 < kWaitLimitNs) {
         }
       }
     }
   } else {
-    // ---------------- Epilogue (warps 2..5) ----------------
+    // ---------------- Epilogue (warps 2..5, both CTAs) ----------------
     const int q = warp & 3;              // TMEM lane quarter this warp may access
     uint8_t* stg = staging + (warp - 2) * 16 * 32 * 4;
+    // Gate/up: quarters 0,1 hold gate of features 0-31 / 32-63, quarters 2,3
+    // hold up of the same features; warp pair p = q & 1 meets on named barrier
+    // 1 + p (64 threads).
+    const int pr = q & 1;
+    const bool gate_warp = q < 2;
+    const uint32_t tempty_leader0 = map_to_cta(smem_u32(&tempty_bar[0]), 0);
+    const uint32_t tempty_leader1 = map_to_cta(smem_u32(&tempty_bar[1]), 0);
     int buf = 0;
     uint32_t bphase = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-      const Chunk ch = get_chunk<kKind>(args, tile / args.n_ftiles);
-      const int ft = tile % args.n_ftiles;
-      const int nb = (ch.nrows + kBoxRows - 1) & ~(kBoxRows - 1);
-      // The outcome must be warp-uniform: tcgen05.ld below is .sync.aligned.
+    int xb = 0;                          // exchange buffer in use (up pairs)
+    for (int t = pair; t < n_tiles; t += n_pairs) {
+      Chunk ch;
+      int ft;
+      get_tile(args, t, ch, ft);
+      const int n = pair_cols(ch.nrows);
       const bool ready = mbar_wait(&tfull_bar[buf], bphase, err, 4 + 8 * kKind);
-      if (!__all_sync(0xffffffffu, ready)) break;
+      // The outcome must be uniform over the threads that go on together:
+      // tcgen05.ld is .sync.aligned, and up pairs meet on named barriers.
+      if (kUp) {
+        uint32_t all_ok;
+        asm volatile(
+            "{\n\t.reg .pred p, r;\n\t"
+            "setp.ne.u32 p, %1, 0;\n\t"
+            "bar.red.and.pred r, %2, 64, p;\n\t"
+            "selp.u32 %0, 1, 0, r;\n\t}"
+            : "=r"(all_ok)
+            : "r"(ready ? 1u : 0u), "r"(1 + pr)
+            : "memory");
+        if (!all_ok) break;
+      } else if (!__all_sync(0xffffffffu, ready)) {
+        break;
+      }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
-      const int col0 = ft * kWRows + q * 32;   // first output column of this warp
-      for (int c0 = 0; c0 < nb; c0 += 16) {
-        float h[16];
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
+      // First output column of this warp.
+      const int col0 = kUp ? ft * 128 + 64 * (int)rank + 32 * pr
+                           : ft * 256 + 128 * (int)rank + 32 * q;
+      for (int c0 = 0; c0 < n; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+        tmem_ld_wait();
         if (kUp) {
-          float g[16], u[16];
-          tmem_ld16(tbase + c0, g);
-          tmem_ld16(tbase + 128 + c0, u);
-          tmem_ld_wait();
+          float* xc = xchg + (pr * 2 + xb) * 16 * 32;
+          if (!gate_warp) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) h[i] = silu(g[i]) * u[i];
+            for (int i = 0; i < 16; ++i) xc[i * 32 + lane] = v[i];
+          }
+          asm volatile("bar.sync %0, 64;" ::"r"(1 + pr) : "memory");
+          xb ^= 1;
+          if (gate_warp) {
+            __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              sb[i * 32 + lane] = __float2bfloat16_rn(silu(v[i]) * xc[i * 32 + lane]);
+          }
         } else {
-          tmem_ld16(tbase + c0, h);
-          tmem_ld_wait();
           if (kKind == kKindDown) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int row = ch.row0 + c0 + i;
-              const float wr = row < args.n_routed_rows ? args.row_weight[row] : 1.0f;
-              h[i] *= wr;
+              v[i] *= row < args.n_routed_rows ? args.row_weight[row] : 1.0f;
             }
           }
-        }
-        // Transpose through shared memory: stg[token][feature], then 16-byte
-        // stores along each output row (32 features = 64 B bf16 / 128 B fp32).
-        if (kUp) {
-          __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) sb[i * 32 + lane] = __float2bfloat16_rn(h[i]);
-        } else {
           float* sf = reinterpret_cast<float*>(stg);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) sf[i * 32 + lane] = h[i];
+          for (int i = 0; i < 16; ++i) sf[i * 32 + lane] = v[i];
         }
-        __syncwarp();
-        constexpr int kChunksPerRow = 32 * C::kOutBytes / 16;
-        constexpr int kElemsPerChunk = 16 / C::kOutBytes;
+        if (!kUp || gate_warp) {
+          __syncwarp();
+          // 16 token rows of this warp's 32 output columns in 16-byte chunks:
+          // 64 B per row (bf16 hidden) or 128 B per row (fp32).
+          constexpr int kRowBytes = 32 * KD::kOutBytes;
+          constexpr int kChunksPerRow = kRowBytes / 16;
+          constexpr int kElemsPerChunk = 16 / KD::kOutBytes;
 #pragma unroll
-        for (int it = 0; it < 16 * kChunksPerRow / 32; ++it) {
-          const int idx = lane + it * 32;
-          const int rr = idx / kChunksPerRow, part = idx % kChunksPerRow;
-          const int c = c0 + rr;
-          const int col = col0 + part * kElemsPerChunk;
-          if (c < ch.nrows && col < args.out_cols) {
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 32 * C::kOutBytes + part * 16);
-            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
-                                      ((int64_t)(ch.row0 + c) * args.ldo + col) * C::kOutBytes) = v;
+          for (int it = 0; it < 16 * kChunksPerRow / 32; ++it) {
+            const int idx = lane + it * 32;
+            const int rr = idx / kChunksPerRow, part = idx % kChunksPerRow;
+            const int c = c0 + rr;
+            const int col = col0 + part * kElemsPerChunk;
+            if (c < ch.nrows && col < args.out_cols) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * kRowBytes + part * 16);
+              *reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
+                                        ((int64_t)(ch.row0 + c) * args.ldo + col) *
+                                            KD::kOutBytes) = val;
+            }
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+      if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
       if (++buf == 2) {
         buf = 0;
         bphase ^= 1u;
@@ -454,11 +564,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,   // W1 (up) or W2
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc_pair(tmem_base, 512);
   }
 }
 
@@ -498,9 +608,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 template <int kKind>
-cudaError_t set_smem_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kKind>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<kKind>::kSmemBytes);
+cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0s,
+                   const CUtensorMap& b0l, const CUtensorMap& b1s, const CUtensorMap& b1l,
+                   const GemmArgs& args, int grid, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kKind>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  grouped_gemm_kernel<kKind><<<grid, kThreads, kSmemBytes, st>>>(a0, a1, b0s, b0l, b1s, b1l, args);
+  return cudaGetLastError();
+}
+
+// Grid of whole CTA pairs: at most one pair per two SMs, at most max_pairs.
+int pair_grid(int num_sms, int max_pairs) {
+  int pairs = num_sms / 2;
+  if (max_pairs > 0 && max_pairs < pairs) pairs = max_pairs;
+  return 2 * (pairs > 0 ? pairs : 1);
 }
 
 }  // namespace
@@ -511,77 +633,73 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
   const int NG = r.E + r.S;
   const int64_t R = T * (r.k + r.S);     // hidden rows
   const int64_t Rr = T * r.k;            // routed rows
-  int32_t* meta = reinterpret_cast<int32_t*>(ws + L.meta);
-  int* err = reinterpret_cast<int*>(ws + L.err);
+  const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.meta);
   GemmArgs a{};
+  a.chunks = reinterpret_cast<const Chunk*>(ws + L.chunks);
+  a.implicit_rows = 0;
   a.n_routed_rows = (int)Rr;
-  a.err = err;
+  a.err = reinterpret_cast<int*>(ws + L.err);
   a.E = r.E;
+  const int grid = pair_grid(num_sms, 0);
   if (up) {
-    CUtensorMap mW1, mW3, mXp, mX;
-    if (!make_map(&mW1, wa, (uint64_t)NG * r.I, r.d, kWRows) ||
-        !make_map(&mW3, wb, (uint64_t)NG * r.I, r.d, kWRows) ||
-        !make_map(&mXp, ws + L.xperm, Rr, r.d, kBoxRows) || !make_map(&mX, x, T, r.d, kBoxRows))
+    CUtensorMap mW1, mW3, mXps, mXpl, mXs, mXl;
+    if (!make_map(&mW1, wa, (uint64_t)NG * r.I, r.d, 64) ||
+        !make_map(&mW3, wb, (uint64_t)NG * r.I, r.d, 64) ||
+        !make_map(&mXps, ws + L.xperm, Rr, r.d, kBoxRows) ||
+        !make_map(&mXpl, ws + L.xperm, Rr, r.d, kBHalfMax) ||
+        !make_map(&mXs, x, T, r.d, kBoxRows) || !make_map(&mXl, x, T, r.d, kBHalfMax))
       return cudaErrorInvalidValue;
-    cudaError_t e = set_smem_attr<kKindUp>();
-    if (e != cudaSuccess) return e;
-    a.chunks = reinterpret_cast<const Chunk*>(ws + L.up_chunks);
-    a.n_chunks = meta + 0;
-    a.n_ftiles = (r.I + kWRows - 1) / kWRows;
+    a.tiles = reinterpret_cast<const int2*>(ws + L.tiles_up);
+    a.n_tiles = meta + 1;
+    a.n_ftiles = (r.I + 127) / 128;
     a.rows_per_group = r.I;
     a.K = r.d;
     a.out_cols = r.I;
     a.ldo = r.I;
     a.out = ws + L.hidden;
     a.row_weight = nullptr;
-    grouped_gemm_kernel<kKindUp><<<num_sms, kThreads, Cfg<kKindUp>::kSmemBytes, st>>>(mW1, mW3, mXp, mX, a);
-  } else {
-    CUtensorMap mW2, mH;
-    if (!make_map(&mW2, wa, (uint64_t)NG * r.d, r.I, kWRows) ||
-        !make_map(&mH, ws + L.hidden, R, r.I, kBoxRows))
-      return cudaErrorInvalidValue;
-    cudaError_t e = set_smem_attr<kKindDown>();
-    if (e != cudaSuccess) return e;
-    a.chunks = reinterpret_cast<const Chunk*>(ws + L.down_chunks);
-    a.n_chunks = meta + 1;
-    a.n_ftiles = (r.d + kWRows - 1) / kWRows;
-    a.rows_per_group = r.d;
-    a.K = r.I;
-    a.out_cols = r.d;
-    a.ldo = r.d;
-    a.out = ws + L.expert_out;
-    a.row_weight = reinterpret_cast<const float*>(ws + L.row_weight);
-    grouped_gemm_kernel<kKindDown><<<num_sms, kThreads, Cfg<kKindDown>::kSmemBytes, st>>>(mW2, mW2, mH, mH, a);
+    return launch<kKindUp>(mW1, mW3, mXps, mXpl, mXs, mXl, a, grid, st);
   }
-  return cudaGetLastError();
+  CUtensorMap mW2, mHs, mHl;
+  if (!make_map(&mW2, wa, (uint64_t)NG * r.d, r.I, kARowsCta) ||
+      !make_map(&mHs, ws + L.hidden, R, r.I, kBoxRows) ||
+      !make_map(&mHl, ws + L.hidden, R, r.I, kBHalfMax))
+    return cudaErrorInvalidValue;
+  a.tiles = reinterpret_cast<const int2*>(ws + L.tiles_down);
+  a.n_tiles = meta + 2;
+  a.n_ftiles = (r.d + 255) / 256;
+  a.rows_per_group = r.d;
+  a.K = r.I;
+  a.out_cols = r.d;
+  a.ldo = r.d;
+  a.out = ws + L.expert_out;
+  a.row_weight = reinterpret_cast<const float*>(ws + L.row_weight);
+  return launch<kKindDown>(mW2, mW2, mHs, mHl, mHs, mHl, a, grid, st);
 }
 
 cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, const void* w_gate,
                                   float* logits, int* err, int num_sms, cudaStream_t st) {
-  CUtensorMap mWg, mX;
-  if (!make_map(&mWg, w_gate, (uint64_t)r.E, r.d, kWRows) || !make_map(&mX, x, T, r.d, kBoxRows))
+  CUtensorMap mWg, mXs, mXl;
+  if (!make_map(&mWg, w_gate, (uint64_t)r.E, r.d, kARowsCta) ||
+      !make_map(&mXs, x, T, r.d, kBoxRows) || !make_map(&mXl, x, T, r.d, kBHalfMax))
     return cudaErrorInvalidValue;
-  cudaError_t e = set_smem_attr<kKindLogits>();
-  if (e != cudaSuccess) return e;
   GemmArgs a{};
   a.chunks = nullptr;
-  a.n_chunks = nullptr;
+  a.tiles = nullptr;
+  a.n_tiles = nullptr;
   a.implicit_rows = (int)T;
-  a.n_ftiles = (r.E + kWRows - 1) / kWRows;
+  a.n_ftiles = (r.E + 255) / 256;
   a.rows_per_group = r.E;
   a.K = r.d;
-  a.E = 1;                  // every chunk reads its token rows from the first B map
+  a.E = 1;                  // every chunk reads its token rows from the first B maps
   a.out_cols = r.E;
   a.ldo = r.E;
   a.out = logits;
   a.row_weight = nullptr;
   a.n_routed_rows = 0;
   a.err = err;
-  const int tiles = (int)((T + kUpChunk - 1) / kUpChunk) * a.n_ftiles;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  grouped_gemm_kernel<kKindLogits><<<grid, kThreads, Cfg<kKindLogits>::kSmemBytes, st>>>(
-      mWg, mWg, mX, mX, a);
-  return cudaGetLastError();
+  const int tiles = (int)((T + kChunkRows - 1) / kChunkRows) * a.n_ftiles;
+  return launch<kKindLogits>(mWg, mWg, mXs, mXl, mXs, mXl, a, pair_grid(num_sms, tiles), st);
 }
 
 }  // namespace ktmoe

@@ -15,9 +15,8 @@ namespace ktmoe {
 // Tiling constants
 // ---------------------------------------------------------------------------
 constexpr int kPermChunk = 32;      // tokens per gate-select / scatter CTA
-constexpr int kUpChunk = 128;       // token rows per gate/up GEMM tile (MMA N <= 128)
-constexpr int kDownChunk = 256;     // token rows per down GEMM tile (MMA N <= 256)
-constexpr int kWRows = 128;         // weight rows per GEMM tile (MMA M)
+constexpr int kChunkRows = 256;     // token rows per GEMM chunk (MMA N <= 256)
+constexpr int kTileBlock = 8;       // chunks per schedule block (feature-tile-major inside)
 constexpr int kMaxExperts = 512;
 constexpr int kMaxGroups = 32;
 constexpr int kMaxTopk = 32;
@@ -54,7 +53,7 @@ struct Chunk {
 // Byte offsets of the workspace's internal buffers.
 struct Layout {
   size_t err;          // int32[2]
-  size_t meta;         // int32[16]: [0] up chunks, [1] down chunks
+  size_t meta;         // int32[16]: [0] chunks, [1] up tiles, [2] down tiles
   size_t logits;       // fp32 [T, E]
   size_t idx;          // int32 [T, k] (when the caller gives no output buffer)
   size_t w;            // fp32 [T, k]
@@ -65,13 +64,14 @@ struct Layout {
   size_t row_of;       // int32 [T*k]
   size_t tok_of;       // int32 [T*k]
   size_t row_weight;   // fp32 [T*k]
-  size_t up_chunks;    // Chunk [max_up]
-  size_t down_chunks;  // Chunk [max_down]
+  size_t chunks;       // Chunk [max_chunks]
+  size_t tiles_up;     // int2 (chunk, feature tile) [max_chunks * ceil(I/128)]
+  size_t tiles_down;   // int2 [max_chunks * ceil(d/256)]
   size_t xperm;        // dtype [T*k, d] (bf16 layers only)
   size_t hidden;       // dtype [T*(k+S), I]
   size_t expert_out;   // fp32 [T*(k+S), d]
   size_t total;
-  int64_t nperm, max_up, max_down;
+  int64_t nperm, max_chunks;
 };
 
 int resolve(const kt_moe_config* cfg, int64_t T, int has_bias, Resolved* r);

@@ -53,17 +53,41 @@ __device__ int block_exclusive_scan(int* buf, int n) {
   return total;
 }
 
+// Largest i with base[i] <= v, for a non-decreasing base[0..n] with base[0] = 0.
+__device__ __forceinline__ int find_group(const int* base, int n, int v) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (base[mid] <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Tile t of a group with nc chunks and F feature tiles: blocks of kTileBlock
+// chunks, feature-tile-major inside a block, so the pairs that run one weight
+// tile over several token chunks run together.
+__device__ __forceinline__ int2 tile_of(int local, int nc, int F, int chunk0) {
+  const int b = local / (kTileBlock * F);
+  const int bs = min(kTileBlock, nc - b * kTileBlock);
+  const int rem = local - b * kTileBlock * F;
+  return make_int2(chunk0 + b * kTileBlock + rem % bs, rem / bs);
+}
+
 __global__ void __launch_bounds__(kScanThreads)
-permute_scan_kernel(int E, int S, int T_, int k, int nperm, const int32_t* __restrict__ chunk_counts,
-                    int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
-                    int32_t* __restrict__ offsets, Chunk* __restrict__ up, Chunk* __restrict__ down,
-                    int32_t* __restrict__ meta) {
-  __shared__ int tot[kMaxExperts + kMaxShared];
-  __shared__ int nup[kMaxExperts + kMaxShared];
-  __shared__ int ndn[kMaxExperts + kMaxShared];
+permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd,
+                    const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base,
+                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                    Chunk* __restrict__ chunks, int2* __restrict__ tiles_up,
+                    int2* __restrict__ tiles_dn, int32_t* __restrict__ meta) {
+  constexpr int NGMAX = kMaxExperts + kMaxShared;
+  __shared__ int tot[NGMAX];
+  __shared__ int rows0[NGMAX];
+  __shared__ int cb[NGMAX + 1];
+  __shared__ int tub[NGMAX + 1];
+  __shared__ int tdb[NGMAX + 1];
   const int tid = threadIdx.x;
   const int NG = E + S;
-  // Per-expert totals over the chunks.
+  // Per-expert totals over the chunks; shared experts hold all T tokens.
   if (tid < NG) {
     int run = 0;
     if (tid < E)
@@ -71,45 +95,57 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, const int32_t* __res
     else
       run = T_;
     tot[tid] = run;
+    rows0[tid] = run;
     counts[tid] = run;
   }
   __syncthreads();
   // Routed experts: rows [0, T*k); shared expert s: rows T*k + s*T.
-  const int ntot = block_exclusive_scan(tot, E);
-  (void)ntot;
-  if (tid >= E && tid < NG) tot[tid] = T_ * k + (tid - E) * T_;
+  block_exclusive_scan(rows0, E);
+  if (tid >= E && tid < NG) rows0[tid] = T_ * k + (tid - E) * T_;
   __syncthreads();
-  if (tid < NG) offsets[tid] = tot[tid];
+  if (tid < NG) offsets[tid] = rows0[tid];
   if (tid == 0) offsets[NG] = T_ * k + S * T_;
-  // Chunk bases (global row of each chunk's first row for each expert).
+  // Chunk bases (global row of each permutation chunk's first row per expert).
   if (tid < E) {
-    int run = tot[tid];
+    int run = rows0[tid];
     for (int c = 0; c < nperm; ++c) {
       chunk_base[(int64_t)c * E + tid] = run;
       run += chunk_counts[(int64_t)c * E + tid];
     }
   }
-  // Chunk lists for the two GEMMs.
+  // GEMM chunks of kChunkRows rows and the two tile schedules.
   if (tid < NG) {
-    const int n = tid < E ? counts[tid] : T_;
-    nup[tid] = (n + kUpChunk - 1) / kUpChunk;
-    ndn[tid] = (n + kDownChunk - 1) / kDownChunk;
+    const int nc = (tot[tid] + kChunkRows - 1) / kChunkRows;
+    cb[tid] = nc;
+    tub[tid] = nc * Fu;
+    tdb[tid] = nc * Fd;
   }
   __syncthreads();
-  const int total_up = block_exclusive_scan(nup, NG);
-  const int total_dn = block_exclusive_scan(ndn, NG);
-  if (tid < NG) {
-    const int n = tid < E ? counts[tid] : T_;
-    const int row0 = tot[tid];
-    const int src0 = tid < E ? row0 : 0;
-    for (int c = 0, r = 0; r < n; ++c, r += kUpChunk)
-      up[nup[tid] + c] = Chunk{tid, row0 + r, min(kUpChunk, n - r), src0 + r};
-    for (int c = 0, r = 0; r < n; ++c, r += kDownChunk)
-      down[ndn[tid] + c] = Chunk{tid, row0 + r, min(kDownChunk, n - r), src0 + r};
-  }
+  const int n_chunks = block_exclusive_scan(cb, NG);
+  const int n_up = block_exclusive_scan(tub, NG);
+  const int n_dn = block_exclusive_scan(tdb, NG);
   if (tid == 0) {
-    meta[0] = total_up;
-    meta[1] = total_dn;
+    cb[NG] = n_chunks;
+    tub[NG] = n_up;
+    tdb[NG] = n_dn;
+    meta[0] = n_chunks;
+    meta[1] = n_up;
+    meta[2] = n_dn;
+  }
+  __syncthreads();
+  for (int i = tid; i < n_chunks; i += blockDim.x) {
+    const int g = find_group(cb, NG, i);
+    const int r = (i - cb[g]) * kChunkRows;
+    const int src0 = g < E ? rows0[g] : 0;
+    chunks[i] = Chunk{g, rows0[g] + r, min(kChunkRows, tot[g] - r), src0 + r};
+  }
+  for (int t = tid; t < n_up; t += blockDim.x) {
+    const int g = find_group(tub, NG, t);
+    tiles_up[t] = tile_of(t - tub[g], cb[g + 1] - cb[g], Fu, cb[g]);
+  }
+  for (int t = tid; t < n_dn; t += blockDim.x) {
+    const int g = find_group(tdb, NG, t);
+    tiles_dn[t] = tile_of(t - tdb[g], cb[g + 1] - cb[g], Fd, cb[g]);
   }
 }
 
@@ -164,9 +200,10 @@ cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* 
                            const int32_t* idx, const float* w, const void* x, cudaStream_t st) {
   auto I32 = [&](size_t off) { return reinterpret_cast<int32_t*>(ws + off); };
   permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
-      r.E, r.S, (int)T, r.k, (int)L.nperm, I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts),
-      I32(L.offsets), reinterpret_cast<Chunk*>(ws + L.up_chunks),
-      reinterpret_cast<Chunk*>(ws + L.down_chunks), I32(L.meta));
+      r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256,
+      I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts), I32(L.offsets),
+      reinterpret_cast<Chunk*>(ws + L.chunks), reinterpret_cast<int2*>(ws + L.tiles_up),
+      reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)L.nperm;

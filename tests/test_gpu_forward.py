@@ -119,6 +119,34 @@ def test_permutation_buffers_exact(layer):
             assert row_of[t, j] == r and rw[r] == w[t, j]
 
 
+@pytest.mark.parametrize("layer", [W.BY_NAME["small_sig_bias"], W.V3_DECODE, W.V3_PREFILL],
+                         ids=lambda c: c.name)
+def test_gemm_schedule_covers_every_tile_once(layer):
+    """The device-built chunk list tiles each expert's rows exactly, and each
+    GEMM schedule names every (chunk, feature tile) pair exactly once."""
+    inp = W.make_layer(layer, "cuda")
+    out = run_forward(layer, inp)
+    T, k, E, S = layer.T, layer.topk, layer.n_experts, layer.n_shared
+    lay = K.kt_moe_workspace_layout(K.config_for(layer), T)
+    ws = out["ws"]
+    n_chunks, n_up, n_dn = _ws_array(ws, lay["meta"], 3, torch.int32).tolist()
+    chunks = _ws_array(ws, lay["chunks"], 4 * n_chunks, torch.int32).reshape(-1, 4)
+    counts = np.bincount(out["idx"].cpu().numpy().ravel(), minlength=E).tolist() + [T] * S
+    offsets = np.concatenate([[0], np.cumsum(counts[:E])]).tolist() + \
+        [T * k + s * T for s in range(S)]
+    for g in range(E + S):
+        mine = chunks[chunks[:, 0] == g]
+        rows = np.concatenate([np.arange(r0, r0 + n) for _, r0, n, _ in mine]) if len(mine) else []
+        assert np.array_equal(rows, np.arange(offsets[g], offsets[g] + counts[g]))
+        assert all(1 <= n <= 256 for n in mine[:, 2])
+    for key, n, F in (("tiles_up", n_up, -(-layer.inter // 128)),
+                      ("tiles_down", n_dn, -(-layer.dim // 256))):
+        tiles = _ws_array(ws, lay[key], 2 * n, torch.int32).reshape(-1, 2)
+        assert n == n_chunks * F
+        seen = set(map(tuple, tiles.tolist()))
+        assert len(seen) == n and seen == {(c, f) for c in range(n_chunks) for f in range(F)}
+
+
 def test_hidden_rows_match_oracle_expert_hidden():
     """The up GEMM alone: SwiGLU hidden rows of a few (expert, token) pairs."""
     layer = W.BY_NAME["small_sig_bias"]
