@@ -34,9 +34,13 @@
 //     commits to the "empty" and "accumulator full" barriers of both CTAs; both
 //     epilogues arrive on the even CTA's "accumulator empty" barrier. Two TMEM
 //     accumulator buffers of 256 columns overlap the epilogue with the next tile.
-//   - The tile schedule (chunk, feature tile) is built on the device: within an
-//     expert, blocks of 8 token chunks run feature-tile-major, so the pairs that
-//     read one weight tile run together and share it through L2.
+//   - The tile list (chunk, feature tile) is built on the device: within an
+//     expert, blocks of 8 token chunks run feature-tile-major, so that tiles
+//     reading one weight tile are neighbours in the list. Pairs take tiles from
+//     a device counter (the even CTA's producer fetches and publishes each tile
+//     to both CTAs through a 4-slot ring of mbarrier-guarded slots), so tiles
+//     start in list order and neighbours run together and share the weight
+//     tile through L2, however long earlier tiles took.
 // No TMA multicast is used.
 //
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the
@@ -50,7 +54,10 @@
 namespace ktmoe {
 namespace {
 
-constexpr int kStages = 6;
+#ifndef KT_STAGES
+#define KT_STAGES 6
+#endif
+constexpr int kStages = KT_STAGES;
 constexpr int kBK = 64;                          // K elements per stage (128 B of bf16)
 constexpr int kARowsCta = 128;                   // weight rows per CTA (MMA M = 256 per pair)
 constexpr int kATileBytes = kARowsCta * kBK * 2;   // 16 KB
@@ -62,9 +69,14 @@ constexpr int kBoxBytes = kBoxRows * kBK * 2;    // 4 KB
 constexpr int kThreads = 192;
 constexpr int kStagingBytes = 4 * 16 * 32 * 4;   // 4 epilogue warps x [16 tokens][32 x 4 B]
 constexpr int kXchgBytes = 2 * 2 * 16 * 32 * 4;  // up -> gate: 2 warp pairs x 2 buffers
-constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + kXchgBytes + 256 + 1024;
+constexpr int kCtrlBytes = 512;                  // mbarriers, TMEM address, schedule slots
+constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + kXchgBytes + kCtrlBytes + 1024;
 constexpr int kAccCols = 256;                    // TMEM columns per accumulator buffer
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kSched = 4;                        // tile schedule ring slots
+// Consumers of a schedule slot: the MMA thread and 4 epilogue warps of the even
+// CTA, the producer and 4 epilogue warps of the odd CTA.
+constexpr int kSchedConsumers = 10;
 
 // Epilogue kinds.
 constexpr int kKindUp = 0;      // hidden = silu(W1 u) * W3 u            (bf16 out)
@@ -82,6 +94,8 @@ struct GemmArgs {
   const Chunk* chunks;
   const int2* tiles;         // (chunk index, feature tile) in schedule order
   const int32_t* n_tiles;    // device count of tiles
+  int* counter;              // device tile counter (zeroed before the launch), or null:
+                             // then pair p takes tiles p, p + pairs, ...
   int implicit_rows;         // > 0: logits; chunks of kChunkRows over this many token rows
   int n_ftiles;              // feature tiles per group
   int rows_per_group;        // weight rows per group (I for up, d for down, E for logits)
@@ -146,8 +160,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Bounded wait. Returns false (after recording the timeout) if the phase did not
 // complete within kWaitLimitNs, or if another CTA already recorded an error.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int where) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait, out of line so the issuing loops stay short.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int* err, int where) {
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -160,15 +174,35 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
     }
   }
 }
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int where) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, err, where);
+}
 // 2-D tiled TMA load into this CTA's shared memory, completing on the barrier
-// at shared::cluster address `bar` (the even CTA's, for the pair).
+// at shared::cluster address `bar` (the even CTA's, for the pair), with an L2
+// eviction-priority policy.
 __device__ __forceinline__ void tma_load_pair(void* dst, const CUtensorMap* map, uint32_t bar, int c0,
-                                              int c1) {
+                                              int c1, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
       : "memory");
+}
+// L2 policies: data read once soon (evict first) and data re-read later (evict last).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -222,6 +256,16 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
                    bar)
                : "memory");
 }
+// The same arrival on the barrier at this shared::cta offset in both CTAs of
+// the pair (CTA mask 0b11).
+__device__ __forceinline__ void mma_commit_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
   asm volatile(
@@ -239,6 +283,35 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+
+__device__ __forceinline__ void st_cluster_s32(uint32_t caddr, int v) {
+  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void read_slot(const int* slot, Chunk& ch, int& ft) {
+  const volatile int* v = slot;
+  ch = Chunk{v[0], v[1], v[2], v[3]};
+  ft = v[4];
+}
+
+// True iff `v` holds on every thread that continues together: the warp, or the
+// 64 threads of an up-epilogue warp pair (named barrier `bar_id`).
+template <bool kPair>
+__device__ __forceinline__ bool uniform_ok(bool v, int bar_id) {
+  if (kPair) {
+    uint32_t all_ok;
+    asm volatile(
+        "{\n\t.reg .pred p, r;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred r, %2, 64, p;\n\t"
+        "selp.u32 %0, 1, 0, r;\n\t}"
+        : "=r"(all_ok)
+        : "r"(v ? 1u : 0u), "r"(bar_id)
+        : "memory");
+    return all_ok != 0;
+  }
+  return __all_sync(0xffffffffu, v);
+}
 
 __device__ __forceinline__ void get_tile(const GemmArgs& a, int t, Chunk& ch, int& ft) {
   if (a.implicit_rows > 0) {
@@ -284,7 +357,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
   uint64_t* tfull_bar = bars + 2 * kStages;         // [2]
   uint64_t* tempty_bar = bars + 2 * kStages + 2;    // [2]        (even CTA's are used)
   uint64_t* drain_bar = bars + 2 * kStages + 4;     // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  uint64_t* sched_full = bars + 2 * kStages + 5;    // [kSched] tile published (each CTA)
+  uint64_t* sched_empty = sched_full + kSched;      // [kSched] slot consumed (even CTA's)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sched_empty + kSched);
+  // Schedule slots: {group, row0, nrows, src_row0, feature tile, -, -, -}; group
+  // -1 ends the schedule.
+  int* sched_info = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 256);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_rank();             // 0: even (MMA-issuing) CTA, 1: odd
@@ -299,6 +377,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
       mbar_init(&tempty_bar[b], 8);     // 4 epilogue warps x 2 CTAs
     }
     mbar_init(drain_bar, 1);
+    for (int i = 0; i < kSched; ++i) {
+      mbar_init(&sched_full[i], 1);     // one arrival: the even CTA's producer
+      mbar_init(&sched_empty[i], kSchedConsumers);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmA0);
     prefetch_tmap(&tmB0s);
@@ -318,21 +400,71 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
   const int n_tiles = args.implicit_rows > 0
                           ? ((args.implicit_rows + kChunkRows - 1) / kChunkRows) * args.n_ftiles
                           : *args.n_tiles;
-  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;   // static schedule only
   const int nk = (args.K + kBK - 1) / kBK;
   int* err = args.err;
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs) ----------------
+      // The even CTA's producer also schedules: it takes the pair's next tile and
+      // publishes it to both CTAs' schedule slots; the odd CTA's producer reads it.
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int issued = 0;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+      int sslot = 0, iter = 0;
+      uint32_t sphase = 0;
+      // Expert weights stream through once per tile group (evict first); token
+      // rows are re-read by every feature tile of their chunk (evict last). The
+      // gate logits re-read W_g for every token chunk instead.
+#if KT_L2_HINTS
+      const uint64_t pol_a = kKind == kKindLogits ? policy_evict_last() : policy_evict_first();
+      const uint64_t pol_b = kKind == kKindLogits ? policy_evict_first() : policy_evict_last();
+#else
+      const uint64_t pol_a = policy_evict_normal(), pol_b = pol_a;
+#endif
+      for (;;) {
+        int t;
+        if (leader) {
+          if (!mbar_wait(&sched_empty[sslot], sphase ^ 1u, err, 5 + 8 * kKind)) {
+            ok = false;
+            break;
+          }
+          t = args.counter ? atomicAdd(args.counter, 1) : pair + iter * n_pairs;
+          ++iter;
+          Chunk c{-1, 0, 0, 0};
+          int f = 0;
+          if (t < n_tiles) get_tile(args, t, c, f);
+          int* slot = sched_info + 8 * sslot;
+          slot[0] = c.group;
+          slot[1] = c.row0;
+          slot[2] = c.nrows;
+          slot[3] = c.src_row0;
+          slot[4] = f;
+          const uint32_t peer_slot = map_to_cta(smem_u32(slot), 1);
+          st_cluster_s32(peer_slot, c.group);
+          st_cluster_s32(peer_slot + 4, c.row0);
+          st_cluster_s32(peer_slot + 8, c.nrows);
+          st_cluster_s32(peer_slot + 12, c.src_row0);
+          st_cluster_s32(peer_slot + 16, f);
+          mbar_arrive_cluster(map_to_cta(smem_u32(&sched_full[sslot]), 0));
+          mbar_arrive_cluster(map_to_cta(smem_u32(&sched_full[sslot]), 1));
+        } else {
+          if (!mbar_wait(&sched_full[sslot], sphase, err, 6 + 8 * kKind)) {
+            ok = false;
+            break;
+          }
+        }
         Chunk ch;
         int ft;
-        get_tile(args, t, ch, ft);
+        read_slot(sched_info + 8 * sslot, ch, ft);
+        if (!leader) mbar_arrive_cluster(map_to_cta(smem_u32(&sched_empty[sslot]), 0));
+        if (++sslot == kSched) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
+        if (ch.group < 0) break;
         const int half = pair_cols(ch.nrows) / 2;
         // First weight row of this CTA's half of the pair tile.
         const int a_row = ch.group * args.rows_per_group + ft * KD::kRowsPerPair +
@@ -365,16 +497,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
           const int kc = kb * kBK;
           if (kUp) {
             // [64 rows of W1 | the same 64 rows of W3]
-            tma_load_pair(sA, &tmA0, fbar, kc, a_row);
-            tma_load_pair(sA + 64 * 128, &tmA1, fbar, kc, a_row);
+            tma_load_pair(sA, &tmA0, fbar, kc, a_row, pol_a);
+            tma_load_pair(sA + 64 * 128, &tmA1, fbar, kc, a_row, pol_a);
           } else {
-            tma_load_pair(sA, &tmA0, fbar, kc, a_row);
+            tma_load_pair(sA, &tmA0, fbar, kc, a_row, pol_a);
           }
           if (nbox == 0) {
-            tma_load_pair(sB, bl, fbar, kc, b_row);
+            tma_load_pair(sB, bl, fbar, kc, b_row, pol_b);
           } else {
             for (int i = 0; i < nbox; ++i)
-              tma_load_pair(sB + i * kBoxBytes, bs, fbar, kc, b_row + i * kBoxRows);
+              tma_load_pair(sB + i * kBoxBytes, bs, fbar, kc, b_row + i * kBoxRows, pol_b);
           }
           issued = issued < kStages ? issued + 1 : kStages;
           if (++stage == kStages) {
@@ -382,6 +514,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
             phase ^= 1u;
           }
         }
+        if (!ok) break;
       }
       if (!ok && leader) {
         // Let the copies already in flight land before the CTA can exit.
@@ -401,17 +534,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer (even CTA, for the pair) ----------------
-      const uint32_t peer = 1;
+      const uint64_t desc_a0 = sw128_desc(smem_u32(stage_base));
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
       uint32_t bphase = 0;
       bool ok = true;
       bool issued_any = false;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+      int sslot = 0;
+      uint32_t sphase = 0;
+      for (;;) {
+        if (!mbar_wait(&sched_full[sslot], sphase, err, 7 + 8 * kKind)) break;
         Chunk ch;
         int ft;
-        get_tile(args, t, ch, ft);
+        read_slot(sched_info + 8 * sslot, ch, ft);
+        mbar_arrive_cluster(smem_u32(&sched_empty[sslot]));
+        if (++sslot == kSched) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
+        if (ch.group < 0) break;
         const int n = pair_cols(ch.nrows);
         if (!mbar_wait(&tempty_bar[buf], bphase ^ 1u, err, 2 + 8 * kKind)) {
           ok = false;
@@ -425,16 +567,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t sA = smem_u32(stage_base + stage * kStageBytes);
-          const uint32_t sB = sA + kATileBytes;
+          // Descriptors of this stage: the start-address field counts 16-byte
+          // units, so the 32-byte step between K sub-blocks adds 2.
+          const uint64_t da = desc_a0 + (uint64_t)(stage * (kStageBytes >> 4));
+          const uint64_t db = da + (kATileBytes >> 4);
 #pragma unroll
           for (int ks = 0; ks < kBK / 16; ++ks)
-            mma_pair_bf16(d0, sw128_desc(sA + ks * 32), sw128_desc(sB + ks * 32), idesc,
-                          (kb | ks) != 0);
-          const uint32_t eb = smem_u32(&empty_bar[stage]);
-          mma_commit_pair(eb);
-          mma_commit_pair(map_to_cta(eb, peer));
+            mma_pair_bf16(d0, da + 2 * ks, db + 2 * ks, idesc, (kb | ks) != 0);
+          mma_commit_both(smem_u32(&empty_bar[stage]));
           issued_any = true;
           if (++stage == kStages) {
             stage = 0;
@@ -442,9 +582,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
           }
         }
         if (!ok) break;
-        const uint32_t fb = smem_u32(&tfull_bar[buf]);
-        mma_commit_pair(fb);
-        mma_commit_pair(map_to_cta(fb, peer));
+        mma_commit_both(smem_u32(&tfull_bar[buf]));
         if (++buf == 2) {
           buf = 0;
           bphase ^= 1u;
@@ -473,28 +611,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
     int buf = 0;
     uint32_t bphase = 0;
     int xb = 0;                          // exchange buffer in use (up pairs)
-    for (int t = pair; t < n_tiles; t += n_pairs) {
+    int sslot = 0;
+    uint32_t sphase = 0;
+    const uint32_t sched_empty_leader = map_to_cta(smem_u32(&sched_empty[0]), 0);
+    for (;;) {
+      // Wait outcomes must be uniform over the threads that go on together:
+      // tcgen05.ld is .sync.aligned, and up pairs meet on named barriers.
+      const bool got = mbar_wait(&sched_full[sslot], sphase, err, 8 + 8 * kKind);
+      if (!uniform_ok<kUp>(got, 1 + pr)) break;
       Chunk ch;
       int ft;
-      get_tile(args, t, ch, ft);
+      read_slot(sched_info + 8 * sslot, ch, ft);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(sched_empty_leader + sslot * 8);
+      if (++sslot == kSched) {
+        sslot = 0;
+        sphase ^= 1u;
+      }
+      if (ch.group < 0) break;
       const int n = pair_cols(ch.nrows);
       const bool ready = mbar_wait(&tfull_bar[buf], bphase, err, 4 + 8 * kKind);
-      // The outcome must be uniform over the threads that go on together:
-      // tcgen05.ld is .sync.aligned, and up pairs meet on named barriers.
-      if (kUp) {
-        uint32_t all_ok;
-        asm volatile(
-            "{\n\t.reg .pred p, r;\n\t"
-            "setp.ne.u32 p, %1, 0;\n\t"
-            "bar.red.and.pred r, %2, 64, p;\n\t"
-            "selp.u32 %0, 1, 0, r;\n\t}"
-            : "=r"(all_ok)
-            : "r"(ready ? 1u : 0u), "r"(1 + pr)
-            : "memory");
-        if (!all_ok) break;
-      } else if (!__all_sync(0xffffffffu, ready)) {
-        break;
-      }
+      if (!uniform_ok<kUp>(ready, 1 + pr)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
       // First output column of this warp.
@@ -651,6 +788,7 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
       return cudaErrorInvalidValue;
     a.tiles = reinterpret_cast<const int2*>(ws + L.tiles_up);
     a.n_tiles = meta + 1;
+    a.counter = const_cast<int32_t*>(meta) + 3;
     a.n_ftiles = (r.I + 127) / 128;
     a.rows_per_group = r.I;
     a.K = r.d;
@@ -667,6 +805,7 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
     return cudaErrorInvalidValue;
   a.tiles = reinterpret_cast<const int2*>(ws + L.tiles_down);
   a.n_tiles = meta + 2;
+  a.counter = const_cast<int32_t*>(meta) + 4;
   a.n_ftiles = (r.d + 255) / 256;
   a.rows_per_group = r.d;
   a.K = r.I;
@@ -687,6 +826,7 @@ cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, c
   a.chunks = nullptr;
   a.tiles = nullptr;
   a.n_tiles = nullptr;
+  a.counter = nullptr;
   a.implicit_rows = (int)T;
   a.n_ftiles = (r.E + 255) / 256;
   a.rows_per_group = r.E;

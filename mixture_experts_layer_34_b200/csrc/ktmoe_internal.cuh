@@ -16,7 +16,18 @@ namespace ktmoe {
 // ---------------------------------------------------------------------------
 constexpr int kPermChunk = 32;      // tokens per gate-select / scatter CTA
 constexpr int kChunkRows = 256;     // token rows per GEMM chunk (MMA N <= 256)
-constexpr int kTileBlock = 8;       // chunks per schedule block (feature-tile-major inside)
+// Schedule tuning (compile-time; -D overrides are for tuning sweeps).
+#ifndef KT_TILE_BLOCK
+#define KT_TILE_BLOCK 8
+#endif
+#ifndef KT_HEAVY_ROWS
+#define KT_HEAVY_ROWS 192
+#endif
+#ifndef KT_L2_HINTS
+#define KT_L2_HINTS 1
+#endif
+constexpr int kTileBlock = KT_TILE_BLOCK;   // chunks per schedule block (feature-tile-major inside)
+constexpr int kHeavyRows = KT_HEAVY_ROWS;   // experts with at least this many rows are compute-bound
 constexpr int kMaxExperts = 512;
 constexpr int kMaxGroups = 32;
 constexpr int kMaxTopk = 32;
@@ -53,7 +64,8 @@ struct Chunk {
 // Byte offsets of the workspace's internal buffers.
 struct Layout {
   size_t err;          // int32[2]
-  size_t meta;         // int32[16]: [0] chunks, [1] up tiles, [2] down tiles
+  size_t meta;         // int32[16]: [0] chunks, [1] up tiles, [2] down tiles,
+                       // [3] / [4] up / down GEMM tile counters
   size_t logits;       // fp32 [T, E]
   size_t idx;          // int32 [T, k] (when the caller gives no output buffer)
   size_t w;            // fp32 [T, k]

@@ -73,6 +73,54 @@ __device__ __forceinline__ int2 tile_of(int local, int nc, int F, int chunk0) {
   return make_int2(chunk0 + b * kTileBlock + rem % bs, rem / bs);
 }
 
+// Positions of a proportional merge of two tile streams, H (nh tiles) and L
+// (nl tiles): element i of a stream of n has key (2i+1)/(2n); keys ascend, H
+// first on equal keys. Integer arithmetic, so the positions form a permutation.
+__device__ __forceinline__ int merged_pos_h(int i, int nh, int nl) {
+  const int64_t A = (int64_t)(2 * i + 1) * nl;           // L tiles with (2j+1)*nh < A go first
+  const int64_t M = A > 0 ? (A - 1) / nh : 0;
+  const int64_t c = (M + 1) / 2;
+  return i + (int)(c < nl ? c : nl);
+}
+__device__ __forceinline__ int merged_pos_l(int j, int nh, int nl) {
+  const int64_t B = (int64_t)(2 * j + 1) * nh;           // H tiles with (2i+1)*nl <= B go first
+  const int64_t M = B / nl;
+  const int64_t c = (M + 1) / 2;
+  return j + (int)(c < nh ? c : nh);
+}
+
+// Fill one GEMM's tile list: experts with at least kHeavyRows rows (compute-
+// bound) form stream H, the others (weight-streaming) stream L; each stream is
+// ordered per group by tile_of, and the two are merged proportionally so that
+// the pairs running at any moment mix both kinds.
+__device__ void fill_tiles(int2* __restrict__ tiles, int F, int NG, const int* cb, int* hb,
+                           int* lb, const int* tot) {
+  const int tid = threadIdx.x;
+  if (tid < NG) {
+    const int nt = (cb[tid + 1] - cb[tid]) * F;
+    const bool heavy = tot[tid] >= kHeavyRows;
+    hb[tid] = heavy ? nt : 0;
+    lb[tid] = heavy ? 0 : nt;
+  }
+  __syncthreads();
+  const int nh = block_exclusive_scan(hb, NG);
+  const int nl = block_exclusive_scan(lb, NG);
+  if (tid == 0) {
+    hb[NG] = nh;
+    lb[NG] = nl;
+  }
+  __syncthreads();
+  for (int i = tid; i < nh; i += blockDim.x) {
+    const int g = find_group(hb, NG, i);
+    tiles[merged_pos_h(i, nh, nl)] = tile_of(i - hb[g], cb[g + 1] - cb[g], F, cb[g]);
+  }
+  for (int j = tid; j < nl; j += blockDim.x) {
+    const int g = find_group(lb, NG, j);
+    tiles[merged_pos_l(j, nh, nl)] = tile_of(j - lb[g], cb[g + 1] - cb[g], F, cb[g]);
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kScanThreads)
 permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd,
                     const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base,
@@ -83,8 +131,8 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd,
   __shared__ int tot[NGMAX];
   __shared__ int rows0[NGMAX];
   __shared__ int cb[NGMAX + 1];
-  __shared__ int tub[NGMAX + 1];
-  __shared__ int tdb[NGMAX + 1];
+  __shared__ int hb[NGMAX + 1];
+  __shared__ int lb[NGMAX + 1];
   const int tid = threadIdx.x;
   const int NG = E + S;
   // Per-expert totals over the chunks; shared experts hold all T tokens.
@@ -113,24 +161,17 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd,
       run += chunk_counts[(int64_t)c * E + tid];
     }
   }
-  // GEMM chunks of kChunkRows rows and the two tile schedules.
-  if (tid < NG) {
-    const int nc = (tot[tid] + kChunkRows - 1) / kChunkRows;
-    cb[tid] = nc;
-    tub[tid] = nc * Fu;
-    tdb[tid] = nc * Fd;
-  }
+  // GEMM chunks of kChunkRows rows and the two tile lists.
+  if (tid < NG) cb[tid] = (tot[tid] + kChunkRows - 1) / kChunkRows;
   __syncthreads();
   const int n_chunks = block_exclusive_scan(cb, NG);
-  const int n_up = block_exclusive_scan(tub, NG);
-  const int n_dn = block_exclusive_scan(tdb, NG);
   if (tid == 0) {
     cb[NG] = n_chunks;
-    tub[NG] = n_up;
-    tdb[NG] = n_dn;
     meta[0] = n_chunks;
-    meta[1] = n_up;
-    meta[2] = n_dn;
+    meta[1] = n_chunks * Fu;
+    meta[2] = n_chunks * Fd;
+    meta[3] = 0;   // gate/up GEMM tile counter
+    meta[4] = 0;   // down GEMM tile counter
   }
   __syncthreads();
   for (int i = tid; i < n_chunks; i += blockDim.x) {
@@ -139,14 +180,8 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd,
     const int src0 = g < E ? rows0[g] : 0;
     chunks[i] = Chunk{g, rows0[g] + r, min(kChunkRows, tot[g] - r), src0 + r};
   }
-  for (int t = tid; t < n_up; t += blockDim.x) {
-    const int g = find_group(tub, NG, t);
-    tiles_up[t] = tile_of(t - tub[g], cb[g + 1] - cb[g], Fu, cb[g]);
-  }
-  for (int t = tid; t < n_dn; t += blockDim.x) {
-    const int g = find_group(tdb, NG, t);
-    tiles_dn[t] = tile_of(t - tdb[g], cb[g + 1] - cb[g], Fd, cb[g]);
-  }
+  fill_tiles(tiles_up, Fu, NG, cb, hb, lb, tot);
+  fill_tiles(tiles_dn, Fd, NG, cb, hb, lb, tot);
 }
 
 template <bool kCopyX>

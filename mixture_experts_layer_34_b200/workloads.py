@@ -141,6 +141,13 @@ PROFILE = [
                 topk_groups=4, topk=8, n_shared=1, inter=2048, score_func=SIGMOID,
                 route_scale=2.5, norm_topk=-1, group_score=GROUP_TOP2SUM, dtype="bf16",
                 bias="normal", seed=2101),
+    # One routed expert, every token routed to it: the two expert GEMMs become
+    # dense 8192 x 4096 x 7168 and 8192 x 7168 x 2048 GEMMs (main-loop efficiency
+    # without the grouped structure).
+    LayerConfig("dense_T8192_E1_profile", T=8192, dim=7168, n_experts=1, n_groups=1,
+                topk_groups=1, topk=1, n_shared=0, inter=2048, score_func=SIGMOID,
+                route_scale=1.0, norm_topk=-1, group_score=GROUP_AUTO, dtype="bf16",
+                bias="none", seed=2102),
 ]
 BY_NAME.update({c.name: c for c in PROFILE})
 
