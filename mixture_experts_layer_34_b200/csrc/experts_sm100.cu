@@ -26,7 +26,8 @@
 //   - Few, large TMA boxes per stage (TMA cost grows with the box count): the
 //     weight tile in one or two boxes, the token rows in one 128-row box for a
 //     full chunk, else in 32-row boxes.
-//   - warp 0: TMA producer (6-stage ring of 32 KB per CTA); warp 1: TMEM owner,
+//   - warp 0: TMA producer (3-stage ring of 64 KB per CTA, each stage two K
+//     slabs of 64 so one wait and one commit serve 8 MMAs); warp 1: TMEM owner,
 //     and in the even CTA the single thread issuing tcgen05.mma for the pair;
 //     warps 2-5: epilogue (tcgen05.ld, SwiGLU / routing weight / none, staging
 //     through shared memory for 16-byte row stores).
@@ -54,16 +55,23 @@
 namespace ktmoe {
 namespace {
 
-#ifndef KT_STAGES
-#define KT_STAGES 6
+// A pipeline stage holds kSlabs K-slabs of 64 (each [weight tile | token tile]),
+// so the MMA thread's per-stage wait and commit are shared by 4 * kSlabs MMAs.
+#ifndef KT_SLABS
+#define KT_SLABS 2
 #endif
+#ifndef KT_STAGES
+#define KT_STAGES (6 / KT_SLABS)
+#endif
+constexpr int kSlabs = KT_SLABS;
 constexpr int kStages = KT_STAGES;
 constexpr int kBK = 64;                          // K elements per stage (128 B of bf16)
 constexpr int kARowsCta = 128;                   // weight rows per CTA (MMA M = 256 per pair)
 constexpr int kATileBytes = kARowsCta * kBK * 2;   // 16 KB
 constexpr int kBHalfMax = kChunkRows / 2;        // token rows per CTA
 constexpr int kBTileBytes = kBHalfMax * kBK * 2;   // 16 KB
-constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kSlabBytes = kATileBytes + kBTileBytes;   // 32 KB
+constexpr int kStageBytes = kSlabs * kSlabBytes;
 constexpr int kBoxRows = 32;                     // token-row TMA box for partial chunks
 constexpr int kBoxBytes = kBoxRows * kBK * 2;    // 4 KB
 constexpr int kThreads = 192;
@@ -401,7 +409,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
                           ? ((args.implicit_rows + kChunkRows - 1) / kChunkRows) * args.n_ftiles
                           : *args.n_tiles;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;   // static schedule only
-  const int nk = (args.K + kBK - 1) / kBK;
+  // Stages per tile; slabs past K read as zeros (TMA fills out-of-range boxes).
+  const int nk = (args.K + kBK * kSlabs - 1) / (kBK * kSlabs);
   int* err = args.err;
 
   if (warp == 0) {
@@ -484,7 +493,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
         // last may run up to 16 rows past the chunk; those columns are unused).
         const int nbox = half == kBHalfMax ? 0 : (half + kBoxRows - 1) / kBoxRows;
         const uint32_t bbytes = nbox == 0 ? kBTileBytes : nbox * kBoxBytes;
-        const uint32_t tx = 2u * (kATileBytes + bbytes);   // both CTAs' bytes
+        const uint32_t tx = 2u * kSlabs * (kATileBytes + bbytes);   // both CTAs' bytes
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, err, 1 + 8 * kKind)) {
             ok = false;
@@ -492,21 +501,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
           }
           const uint32_t fbar = map_to_cta(smem_u32(&full_bar[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
-          uint8_t* sA = stage_base + stage * kStageBytes;
-          uint8_t* sB = sA + kATileBytes;
-          const int kc = kb * kBK;
-          if (kUp) {
-            // [64 rows of W1 | the same 64 rows of W3]
-            tma_load_pair(sA, &tmA0, fbar, kc, a_row, pol_a);
-            tma_load_pair(sA + 64 * 128, &tmA1, fbar, kc, a_row, pol_a);
-          } else {
-            tma_load_pair(sA, &tmA0, fbar, kc, a_row, pol_a);
-          }
-          if (nbox == 0) {
-            tma_load_pair(sB, bl, fbar, kc, b_row, pol_b);
-          } else {
-            for (int i = 0; i < nbox; ++i)
-              tma_load_pair(sB + i * kBoxBytes, bs, fbar, kc, b_row + i * kBoxRows, pol_b);
+#pragma unroll
+          for (int j = 0; j < kSlabs; ++j) {
+            uint8_t* sA = stage_base + stage * kStageBytes + j * kSlabBytes;
+            uint8_t* sB = sA + kATileBytes;
+            const int kc = (kb * kSlabs + j) * kBK;
+            if (kUp) {
+              // [64 rows of W1 | the same 64 rows of W3]
+              tma_load_pair(sA, &tmA0, fbar, kc, a_row, pol_a);
+              tma_load_pair(sA + 64 * 128, &tmA1, fbar, kc, a_row, pol_a);
+            } else {
+              tma_load_pair(sA, &tmA0, fbar, kc, a_row, pol_a);
+            }
+            if (nbox == 0) {
+              tma_load_pair(sB, bl, fbar, kc, b_row, pol_b);
+            } else {
+              for (int i = 0; i < nbox; ++i)
+                tma_load_pair(sB + i * kBoxBytes, bs, fbar, kc, b_row + i * kBoxRows, pol_b);
+            }
           }
           issued = issued < kStages ? issued + 1 : kStages;
           if (++stage == kStages) {
@@ -569,11 +581,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
           }
           // Descriptors of this stage: the start-address field counts 16-byte
           // units, so the 32-byte step between K sub-blocks adds 2.
-          const uint64_t da = desc_a0 + (uint64_t)(stage * (kStageBytes >> 4));
-          const uint64_t db = da + (kATileBytes >> 4);
 #pragma unroll
-          for (int ks = 0; ks < kBK / 16; ++ks)
-            mma_pair_bf16(d0, da + 2 * ks, db + 2 * ks, idesc, (kb | ks) != 0);
+          for (int j = 0; j < kSlabs; ++j) {
+            const uint64_t da = desc_a0 + (uint64_t)((stage * kStageBytes + j * kSlabBytes) >> 4);
+            const uint64_t db = da + (kATileBytes >> 4);
+#pragma unroll
+            for (int ks = 0; ks < kBK / 16; ++ks)
+              mma_pair_bf16(d0, da + 2 * ks, db + 2 * ks, idesc, (kb | j | ks) != 0);
+          }
           mma_commit_both(smem_u32(&empty_bar[stage]));
           issued_any = true;
           if (++stage == kStages) {
