@@ -60,7 +60,8 @@ enum {
   KT_ERR_ALIGN = -4,          /* a pointer is not 16-byte aligned (workspace: 256)  */
   KT_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed               */
   KT_ERR_TIMEOUT = -6,        /* a bounded device-side wait gave up (kt_moe_check)  */
-  KT_ERR_UNSUPPORTED = -7     /* no sm_100 device, or a size beyond a kernel limit  */
+  KT_ERR_UNSUPPORTED = -7,    /* no sm_100 device, or a size beyond a kernel limit  */
+  KT_ERR_SCRATCH_LIMIT = -8   /* call needs more than the static scratch holds       */
 };
 
 /*
@@ -154,6 +155,41 @@ int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
                             const void* w3, const void* w2, void* y, int32_t* topk_idx_out,
                             float* topk_w_out, void* workspace, size_t ws_bytes, void* stream,
                             void* const* stage_events);
+
+/*
+ * kt_moe_forward for callers that cannot allocate device memory. There is no
+ * counterpart on the pages: this entry point exists for the calling code, not
+ * for the method.
+ *
+ * Some callers cannot call cudaMalloc or any allocator: code that runs while a
+ * stream is being captured into a CUDA graph (an allocation there breaks the
+ * capture), engines whose device memory is entirely owned by their own pool,
+ * and plugin hosts that hand out no workspace. They pass only inputs and
+ * outputs; the scratch comes from a fixed 32 MiB device array inside this
+ * library (KT_STATIC_SCRATCH_BYTES), reserved on every GPU that loads the
+ * library until the process exits. A call whose scratch need
+ * (kt_moe_workspace_size) exceeds that returns KT_ERR_SCRATCH_LIMIT before
+ * anything is enqueued — about 78 tokens of a DeepSeek-V3-shaped layer, so
+ * decode-sized batches.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture. Every call on a device shares the one array, which keeps
+ * the previous call's contents (each call resets what must start at zero);
+ * calls whose work overlaps on the GPU — concurrent streams, or host threads
+ * without ordering — race on it and must be serialised by the caller.
+ * Arguments, layouts, results and errors are otherwise those of
+ * kt_moe_forward; kt_moe_check takes kt_moe_static_scratch() as its workspace.
+ */
+enum { KT_STATIC_SCRATCH_BYTES = 32 << 20 };
+int kt_moe_forward_static(const kt_moe_config* cfg, int64_t T, const void* x,
+                          const void* w_gate, const float* bias, const void* w1,
+                          const void* w3, const void* w2, void* y, int32_t* topk_idx_out,
+                          float* topk_w_out, void* stream);
+
+/* Device address of the current device's static scratch (NULL on error); for
+ * kt_moe_check and for reading its buffers after kt_moe_forward_static. */
+void* kt_moe_static_scratch(void);
 
 /* Synchronise `stream`, then read the device error word the last call on this
  * workspace left (a bounded wait inside a kernel that gave up sets it).

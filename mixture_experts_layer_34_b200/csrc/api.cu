@@ -9,6 +9,7 @@
 // the persistent GEMM kernels walk.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "ktmoe_internal.cuh"
 
@@ -257,6 +258,55 @@ int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
   return KT_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Static scratch for kt_moe_forward_static (callers that cannot allocate).
+// A file-scope device array; host code must use the address that
+// cudaGetSymbolAddress returns for the current device, never the array name.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_scratch[KT_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the current device's scratch, looked up once per device.
+void* static_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int kt_moe_forward_static(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                          const float* bias, const void* w1, const void* w3, const void* w2,
+                          void* y, int32_t* topk_idx_out, float* topk_w_out, void* stream) {
+  Resolved r;
+  const int rc = resolve(cfg, T, bias != nullptr, &r);
+  if (rc != KT_OK) return rc;
+  if (make_layout(r, T).total > (size_t)KT_STATIC_SCRATCH_BYTES) return KT_ERR_SCRATCH_LIMIT;
+  void* scratch = static_scratch_ptr();
+  if (!scratch) return KT_ERR_CUDA;
+  // The error word is reset and the tile counters are rewritten inside every
+  // forward; nothing else in the scratch is read before it is written.
+  return kt_moe_forward_profiled(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                                 scratch, KT_STATIC_SCRATCH_BYTES, stream, nullptr);
+}
+
+void* kt_moe_static_scratch(void) { return static_scratch_ptr(); }
+
 int kt_moe_check(const void* workspace, void* stream) {
   if (!workspace) return KT_ERR_WORKSPACE;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KT_ERR_CUDA;
@@ -276,6 +326,8 @@ const char* kt_moe_strerror(int code) {
     case KT_ERR_CUDA: return "CUDA runtime error or failed launch";
     case KT_ERR_TIMEOUT: return "a bounded device-side wait gave up";
     case KT_ERR_UNSUPPORTED: return "unsupported device (needs compute capability 10.0, sm_100a)";
+    case KT_ERR_SCRATCH_LIMIT:
+      return "kt_moe_forward_static: the call needs more scratch than the 32 MiB static array";
     default: return "unknown error code";
   }
 }

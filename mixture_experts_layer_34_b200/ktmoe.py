@@ -19,11 +19,13 @@ KT_GROUP_AUTO, KT_GROUP_AMAX, KT_GROUP_TOP2SUM = 0, 1, 2
 KT_DTYPE_F32, KT_DTYPE_BF16 = 0, 1
 KT_OK = 0
 KT_ERR_INVALID_CONFIG, KT_ERR_NULL, KT_ERR_WORKSPACE, KT_ERR_ALIGN = -1, -2, -3, -4
-KT_ERR_CUDA, KT_ERR_TIMEOUT, KT_ERR_UNSUPPORTED = -5, -6, -7
+KT_ERR_CUDA, KT_ERR_TIMEOUT, KT_ERR_UNSUPPORTED, KT_ERR_SCRATCH_LIMIT = -5, -6, -7, -8
+KT_STATIC_SCRATCH_BYTES = 32 << 20
 
 # Every symbol include/ktmoe.h declares.
 EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_forward",
-           "kt_moe_forward_profiled", "kt_moe_check", "kt_moe_workspace_layout", "kt_moe_strerror", "kt_moe_version")
+           "kt_moe_forward_profiled", "kt_moe_forward_static", "kt_moe_static_scratch",
+           "kt_moe_check", "kt_moe_workspace_layout", "kt_moe_strerror", "kt_moe_version")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -74,6 +76,10 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_forward_profiled.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P,
                                                   ctypes.c_size_t, P, ctypes.POINTER(P)]
             L.kt_moe_forward_profiled.restype = ctypes.c_int
+            L.kt_moe_forward_static.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P]
+            L.kt_moe_forward_static.restype = ctypes.c_int
+            L.kt_moe_static_scratch.argtypes = []
+            L.kt_moe_static_scratch.restype = ctypes.c_void_p
             L.kt_moe_check.argtypes = [P, P]
             L.kt_moe_check.restype = ctypes.c_int
             L.kt_moe_workspace_layout.argtypes = [CP, I64, ctypes.POINTER(kt_moe_ws_layout)]
@@ -172,6 +178,22 @@ def kt_moe_forward_profiled(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out
                                        _stream(stream), arr)
     if rc != KT_OK:
         raise KtMoeError("kt_moe_forward_profiled", rc)
+
+
+def kt_moe_forward_static(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                          stream=None):
+    """kt_moe_forward with the library's static device scratch: no workspace,
+    no allocation (see include/ktmoe.h for its limit and sharing rules)."""
+    rc = lib().kt_moe_forward_static(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias),
+                                     _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y), _ptr(topk_idx_out),
+                                     _ptr(topk_w_out), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_forward_static", rc)
+
+
+def kt_moe_static_scratch() -> int:
+    """Device address of the current device's static scratch (0 on error)."""
+    return lib().kt_moe_static_scratch() or 0
 
 
 def kt_moe_check(workspace, stream=None) -> int:

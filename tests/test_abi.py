@@ -137,7 +137,7 @@ def test_gate_host_side_errors():
 
 
 def test_strerror_covers_codes():
-    for code in range(-7, 1):
+    for code in range(-8, 1):
         assert K.strerror(code) and K.strerror(code) != "unknown error code"
     assert K.strerror(-99) == "unknown error code"
 
