@@ -208,7 +208,8 @@ int kt_moe_check(const void* workspace, void* stream);
  * in schedule order (feature tiles of 128 / 256 rows). */
 typedef struct {
   int64_t error_word;
-  int64_t logits;
+  int64_t logits;         /* fp32 [logits_splits][T][E]: partial sums over K, added in order */
+  int64_t logits_splits;
   int64_t counts;
   int64_t offsets;
   int64_t row_of;

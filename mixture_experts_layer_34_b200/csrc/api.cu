@@ -101,7 +101,7 @@ Layout make_layout(const Resolved& r, int64_t T) {
   L.max_chunks = (int64_t)(R / kChunkRows + NG + 1);
   L.err = take(256, 256);
   L.meta = take(64, 256);
-  L.logits = take((size_t)T * r.E * 4, 256);
+  L.logits = take((size_t)gate_logit_splits(r, T) * T * r.E * 4, 256);
   L.idx = take(Tk * 4, 256);
   L.w = take(Tk * 4, 256);
   L.chunk_counts = take((size_t)L.nperm * r.E * 4, 256);
@@ -149,6 +149,7 @@ int kt_moe_workspace_layout(const kt_moe_config* cfg, int64_t T, kt_moe_ws_layou
   const Layout L = make_layout(r, T);
   out->error_word = (int64_t)L.err;
   out->logits = (int64_t)L.logits;
+  out->logits_splits = gate_logit_splits(r, T);
   out->counts = (int64_t)L.counts;
   out->offsets = (int64_t)L.offsets;
   out->row_of = (int64_t)L.row_of;

@@ -123,44 +123,50 @@ gate_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg, float* __r
 }
 
 // ---------------------------------------------------------------------------
-// Logits for few tokens: one warp per expert streams its W_g row once (16-byte
-// loads split over the lanes) against up to 8 token rows at a time, then
-// reduces across the lanes.
+// Logits for few tokens (T <= 64), split over K: CTA (eb, ks) computes the
+// partial dot products of 32 experts over the ks-th K range for all tokens
+// (one warp per 4 experts, 16-byte loads along K split over the lanes, 8 tokens
+// at a time) and writes them to part[ks][t][e]. The selection kernel adds the
+// kSplitK partials in ks order, so the result does not depend on scheduling.
 // ---------------------------------------------------------------------------
-constexpr int kSmallWarps = 4, kSmallTok = 8;
+constexpr int kSmallWarps = 8, kSmallTok = 8, kSplitK = kGateSplitK;
 
 template <typename T>
 __global__ void __launch_bounds__(kSmallWarps * 32)
-gate_logits_small_kernel(const T* __restrict__ x, const T* __restrict__ wg,
-                         float* __restrict__ logits, int T_, int E, int d) {
+gate_logits_splitk_kernel(const T* __restrict__ x, const T* __restrict__ wg,
+                          float* __restrict__ part, int T_, int E, int d, int kc) {
   constexpr int VN = Vec16<T>::n;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int e = blockIdx.x * kSmallWarps + warp;
-  if (e >= E) return;
-  const int nc = d / VN;
-  const T* wrow = wg + (int64_t)e * d;
-  for (int t0 = 0; t0 < T_; t0 += kSmallTok) {
-    float acc[kSmallTok];
+  const int ks = blockIdx.y;
+  const int k0 = ks * kc, k1 = min(d, k0 + kc);
+  const int nc = k1 > k0 ? (k1 - k0) / VN : 0;
+  for (int ei = 0; ei < 4; ++ei) {
+    const int e = blockIdx.x * 32 + warp * 4 + ei;
+    if (e >= E) break;
+    const T* wrow = wg + (int64_t)e * d + k0;
+    for (int t0 = 0; t0 < T_; t0 += kSmallTok) {
+      float acc[kSmallTok];
 #pragma unroll
-    for (int j = 0; j < kSmallTok; ++j) acc[j] = 0.f;
-    for (int c = lane; c < nc; c += 32) {
-      float wv[VN];
-      Vec16<T>::load(wrow + c * VN, wv);
+      for (int j = 0; j < kSmallTok; ++j) acc[j] = 0.f;
+      for (int c = lane; c < nc; c += 32) {
+        float wv[VN];
+        Vec16<T>::load(wrow + c * VN, wv);
 #pragma unroll
-      for (int j = 0; j < kSmallTok; ++j) {
-        if (t0 + j < T_) {
-          float xv[VN];
-          Vec16<T>::load(x + (int64_t)(t0 + j) * d + c * VN, xv);
+        for (int j = 0; j < kSmallTok; ++j) {
+          if (t0 + j < T_) {
+            float xv[VN];
+            Vec16<T>::load(x + (int64_t)(t0 + j) * d + k0 + c * VN, xv);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[j] = fmaf(wv[i], xv[i], acc[j]);
+            for (int i = 0; i < VN; ++i) acc[j] = fmaf(wv[i], xv[i], acc[j]);
+          }
         }
       }
-    }
 #pragma unroll
-    for (int j = 0; j < kSmallTok; ++j) {
+      for (int j = 0; j < kSmallTok; ++j) {
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
-      if (lane == 0 && t0 + j < T_) logits[(int64_t)(t0 + j) * E + e] = acc[j];
+        for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+        if (lane == 0 && t0 + j < T_) part[((int64_t)ks * T_ + t0 + j) * E + e] = acc[j];
+      }
     }
   }
 }
@@ -170,7 +176,6 @@ gate_logits_small_kernel(const T* __restrict__ x, const T* __restrict__ wg,
 // Lane l holds experts e = i*32 + l, i < ceil(E/32) (at most 16).
 // ---------------------------------------------------------------------------
 constexpr int kSelWarps = 8;
-constexpr int kNPer = kMaxExperts / 32;
 constexpr unsigned kFull = 0xffffffffu;
 
 struct Best {
@@ -194,15 +199,18 @@ __device__ __forceinline__ Best warp_argmax(Best b) {
   return b;
 }
 
+// NP = experts per lane (E <= 32 * NP), a compile-time bound so the per-lane
+// arrays stay in registers. ksplit > 1: `logits` holds ksplit partial sums
+// [ksplit][T][E], added here in order.
+template <int NP>
 __global__ void __launch_bounds__(kSelWarps * 32)
-gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
+gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ logits,
                    const float* __restrict__ scores_in, const float* __restrict__ bias,
                    int32_t* __restrict__ out_idx, float* __restrict__ out_w,
                    int32_t* __restrict__ chunk_counts) {
   __shared__ int scount[kMaxExperts];
   __shared__ float skey[kSelWarps][kMaxExperts];
   const int E = r.E, k = r.k, G = r.G, gs = r.gs;
-  const int nper = (E + 31) / 32;
   for (int e = threadIdx.x; e < E; e += blockDim.x) scount[e] = 0;
   __syncthreads();
 
@@ -212,44 +220,52 @@ gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
     const int t = blockIdx.x * kPermChunk + warp * (kPermChunk / kSelWarps) + tt;
     if (t >= T_) break;
     // Step 1: scores (kept raw for step 5).
-    float s[kNPer], key[kNPer];
+    float s[NP], key[NP];
     const float* row = (scores_in ? scores_in : logits) + (int64_t)t * E;
 #pragma unroll
-    for (int i = 0; i < kNPer; ++i) {
+    for (int i = 0; i < NP; ++i) {
       const int e = i * 32 + lane;
-      s[i] = (i < nper && e < E) ? row[e] : NEG_INF;
+      s[i] = e < E ? row[e] : NEG_INF;
+    }
+    if (!scores_in && ksplit > 1) {
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const int e = i * 32 + lane;
+        if (e < E)
+          for (int k = 1; k < ksplit; ++k) s[i] += logits[((int64_t)k * T_ + t) * E + e];
+      }
     }
     if (!scores_in) {
       if (r.score_func == KT_SCORE_SIGMOID) {
 #pragma unroll
-        for (int i = 0; i < kNPer; ++i)
-          if (i < nper) s[i] = 1.0f / (1.0f + expf(-s[i]));
+        for (int i = 0; i < NP; ++i)
+          s[i] = 1.0f / (1.0f + expf(-s[i]));
       } else {
         float m = NEG_INF;
 #pragma unroll
-        for (int i = 0; i < kNPer; ++i)
-          if (i < nper) m = fmaxf(m, s[i]);
+        for (int i = 0; i < NP; ++i)
+          m = fmaxf(m, s[i]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
         float z = 0.f;
 #pragma unroll
-        for (int i = 0; i < kNPer; ++i)
-          if (i < nper) {
+        for (int i = 0; i < NP; ++i)
+          {
             s[i] = (i * 32 + lane < E) ? expf(s[i] - m) : 0.f;
             z += s[i];
           }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFull, z, off);
 #pragma unroll
-        for (int i = 0; i < kNPer; ++i)
-          if (i < nper) s[i] = __fdiv_rn(s[i], z);
+        for (int i = 0; i < NP; ++i)
+          s[i] = __fdiv_rn(s[i], z);
       }
     }
     // Step 2a: selection keys s + b (the bias takes part in the selection only).
 #pragma unroll
-    for (int i = 0; i < kNPer; ++i) {
+    for (int i = 0; i < NP; ++i) {
       const int e = i * 32 + lane;
-      if (i < nper && e < E) {
+      if (e < E) {
         key[i] = r.has_bias ? __fadd_rn(s[i], bias[e]) : s[i];
         if (key[i] != key[i]) key[i] = NEG_INF;   // NaN input: keep indices valid
       } else {
@@ -259,9 +275,9 @@ gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
     // Steps 2b-3: group scores, keep topk_groups groups, mask the rest.
     if (G > 1) {
 #pragma unroll
-      for (int i = 0; i < kNPer; ++i) {
+      for (int i = 0; i < NP; ++i) {
         const int e = i * 32 + lane;
-        if (i < nper && e < E) skey[warp][e] = key[i];
+        if (e < E) skey[warp][e] = key[i];
       }
       __syncwarp();
       float gsc = NEG_INF;
@@ -292,9 +308,9 @@ gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
         if (lane == b.idx) taken = true;
       }
 #pragma unroll
-      for (int i = 0; i < kNPer; ++i) {
+      for (int i = 0; i < NP; ++i) {
         const int e = i * 32 + lane;
-        if (i < nper && e < E && !((kept >> (e / gs)) & 1u)) key[i] = NEG_INF;
+        if (e < E && !((kept >> (e / gs)) & 1u)) key[i] = NEG_INF;
       }
     }
     // Step 4: global top-k over the masked keys; lane j keeps slot j.
@@ -303,9 +319,9 @@ gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
     for (int j = 0; j < k; ++j) {
       Best lb{NEG_INF, 0x7fffffff};
 #pragma unroll
-      for (int i = 0; i < kNPer; ++i) {
+      for (int i = 0; i < NP; ++i) {
         const int e = i * 32 + lane;
-        if (i < nper && e < E && better(key[i], e, lb.key, lb.idx)) {
+        if (e < E && better(key[i], e, lb.key, lb.idx)) {
           lb.key = key[i];
           lb.idx = e;
         }
@@ -314,7 +330,7 @@ gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
       float won_s = 0.f;
       if (lane == (b.idx & 31)) {
 #pragma unroll
-        for (int i = 0; i < kNPer; ++i)
+        for (int i = 0; i < NP; ++i)
           if (i == (b.idx >> 5)) {
             won_s = s[i];
             key[i] = __int_as_float(0x7fffffff);  // NaN: never wins again
@@ -345,17 +361,21 @@ gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
 
 }  // namespace
 
+int gate_logit_splits(const Resolved& r, int64_t T) { return T <= kSmallTokens ? kSplitK : 1; }
+
 cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, const void* w_gate,
                                float* logits, int* err, int num_sms, cudaStream_t st) {
   const bool bf16 = r.dtype == KT_DTYPE_BF16;
-  if (T <= 64) {
-    const unsigned grid = (unsigned)((r.E + kSmallWarps - 1) / kSmallWarps);
+  if (T <= kSmallTokens) {
+    const int vn = bf16 ? 8 : 4;
+    const int kc = ((r.d + kSplitK - 1) / kSplitK + vn - 1) / vn * vn;
+    const dim3 grid((unsigned)((r.E + 31) / 32), kSplitK);
     if (bf16)
-      gate_logits_small_kernel<__nv_bfloat16><<<grid, kSmallWarps * 32, 0, st>>>(
-          (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d);
+      gate_logits_splitk_kernel<__nv_bfloat16><<<grid, kSmallWarps * 32, 0, st>>>(
+          (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d, kc);
     else
-      gate_logits_small_kernel<float><<<grid, kSmallWarps * 32, 0, st>>>(
-          (const float*)x, (const float*)w_gate, logits, (int)T, r.E, r.d);
+      gate_logits_splitk_kernel<float><<<grid, kSmallWarps * 32, 0, st>>>(
+          (const float*)x, (const float*)w_gate, logits, (int)T, r.E, r.d, kc);
     return cudaGetLastError();
   }
   // Tensor-core logits write 16-byte chunks of fp32 rows of E entries.
@@ -374,8 +394,17 @@ cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits
                                const float* scores_in, const float* bias, int32_t* idx, float* w,
                                int32_t* chunk_counts, cudaStream_t st) {
   const unsigned grid = (unsigned)((T + kPermChunk - 1) / kPermChunk);
-  gate_select_kernel<<<grid, kSelWarps * 32, 0, st>>>(r, (int)T, logits, scores_in, bias, idx, w,
-                                                     chunk_counts);
+  const int ks = scores_in ? 1 : gate_logit_splits(r, T);
+  const int np = (r.E + 31) / 32;
+#define KT_SELECT(NPV)                                                                        \
+  gate_select_kernel<NPV><<<grid, kSelWarps * 32, 0, st>>>(r, (int)T, ks, logits, scores_in, \
+                                                           bias, idx, w, chunk_counts)
+  if (np <= 1) KT_SELECT(1);
+  else if (np <= 2) KT_SELECT(2);
+  else if (np <= 4) KT_SELECT(4);
+  else if (np <= 8) KT_SELECT(8);
+  else KT_SELECT(16);
+#undef KT_SELECT
   return cudaGetLastError();
 }
 

@@ -32,6 +32,8 @@ constexpr int kMaxExperts = 512;
 constexpr int kMaxGroups = 32;
 constexpr int kMaxTopk = 32;
 constexpr int kMaxShared = 8;
+constexpr int kSmallTokens = 64;    // up to this many tokens the gate logits are split over K
+constexpr int kGateSplitK = 16;     // ... into this many partial sums
 
 // Device error word codes (workspace offset 0). The second int holds a detail.
 constexpr int kDevErrTimeout = 1;
@@ -92,6 +94,9 @@ Layout make_layout(const Resolved& r, int64_t T);
 // ---------------------------------------------------------------------------
 // Kernel launchers (each returns the cudaError_t of its launch)
 // ---------------------------------------------------------------------------
+// Number of partial-sum blocks the logits region holds (1, or kGateSplitK for
+// calls of at most kSmallTokens tokens).
+int gate_logit_splits(const Resolved& r, int64_t T);
 cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, const void* w_gate,
                                float* logits, int* err, int num_sms, cudaStream_t st);
 // bf16 logits on the tensor cores (the grouped GEMM with one group); E % 4 == 0.

@@ -39,7 +39,7 @@ class kt_moe_config(ctypes.Structure):
 
 
 class kt_moe_ws_layout(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int64) for n in ("error_word", "logits", "counts", "offsets",
+    _fields_ = [(n, ctypes.c_int64) for n in ("error_word", "logits", "logits_splits", "counts", "offsets",
                                               "row_of", "tok_of", "row_weight", "hidden",
                                               "expert_out", "meta", "chunks", "tiles_up",
                                               "tiles_down", "total")]
