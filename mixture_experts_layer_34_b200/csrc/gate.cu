@@ -125,8 +125,8 @@ gate_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg, float* __r
 // ---------------------------------------------------------------------------
 // Logits for few tokens (T <= 64), split over K: CTA (eb, ks) computes the
 // partial dot products of 32 experts over the ks-th K range for all tokens
-// (one warp per 4 experts, 16-byte loads along K split over the lanes, 8 tokens
-// at a time) and writes them to part[ks][t][e]. The selection kernel adds the
+// (one warp per 4 experts computed together, 16-byte loads along K split over
+// the lanes, 8 tokens at a time) and writes them to part[ks][t][e]. The selection kernel adds the
 // kSplitK partials in ks order, so the result does not depend on scheduling.
 // ---------------------------------------------------------------------------
 constexpr int kSmallWarps = 8, kSmallTok = 8, kSplitK = kGateSplitK;
@@ -135,39 +135,52 @@ template <typename T>
 __global__ void __launch_bounds__(kSmallWarps * 32)
 gate_logits_splitk_kernel(const T* __restrict__ x, const T* __restrict__ wg,
                           float* __restrict__ part, int T_, int E, int d, int kc) {
-  constexpr int VN = Vec16<T>::n;
+  constexpr int VN = Vec16<T>::n, EW = 4;  // experts per warp, computed together
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ks = blockIdx.y;
   const int k0 = ks * kc, k1 = min(d, k0 + kc);
   const int nc = k1 > k0 ? (k1 - k0) / VN : 0;
-  for (int ei = 0; ei < 4; ++ei) {
-    const int e = blockIdx.x * 32 + warp * 4 + ei;
-    if (e >= E) break;
-    const T* wrow = wg + (int64_t)e * d + k0;
-    for (int t0 = 0; t0 < T_; t0 += kSmallTok) {
-      float acc[kSmallTok];
+  const int e0 = blockIdx.x * 32 + warp * EW;
+  if (e0 >= E) return;
+  for (int t0 = 0; t0 < T_; t0 += kSmallTok) {
+    float acc[EW][kSmallTok];
 #pragma unroll
-      for (int j = 0; j < kSmallTok; ++j) acc[j] = 0.f;
-      for (int c = lane; c < nc; c += 32) {
-        float wv[VN];
-        Vec16<T>::load(wrow + c * VN, wv);
+    for (int ei = 0; ei < EW; ++ei)
 #pragma unroll
-        for (int j = 0; j < kSmallTok; ++j) {
-          if (t0 + j < T_) {
-            float xv[VN];
-            Vec16<T>::load(x + (int64_t)(t0 + j) * d + k0 + c * VN, xv);
+      for (int j = 0; j < kSmallTok; ++j) acc[ei][j] = 0.f;
+    for (int c = lane; c < nc; c += 32) {
+      float wv[EW][VN];
 #pragma unroll
-            for (int i = 0; i < VN; ++i) acc[j] = fmaf(wv[i], xv[i], acc[j]);
-          }
+      for (int ei = 0; ei < EW; ++ei) {
+        if (e0 + ei < E) {
+          Vec16<T>::load(wg + (int64_t)(e0 + ei) * d + k0 + c * VN, wv[ei]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < VN; ++i) wv[ei][i] = 0.f;
         }
       }
 #pragma unroll
       for (int j = 0; j < kSmallTok; ++j) {
+        if (t0 + j < T_) {
+          float xv[VN];
+          Vec16<T>::load(x + (int64_t)(t0 + j) * d + k0 + c * VN, xv);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
-        if (lane == 0 && t0 + j < T_) part[((int64_t)ks * T_ + t0 + j) * E + e] = acc[j];
+          for (int ei = 0; ei < EW; ++ei)
+#pragma unroll
+            for (int i = 0; i < VN; ++i) acc[ei][j] = fmaf(wv[ei][i], xv[i], acc[ei][j]);
+        }
       }
     }
+#pragma unroll
+    for (int ei = 0; ei < EW; ++ei)
+#pragma unroll
+      for (int j = 0; j < kSmallTok; ++j) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          acc[ei][j] += __shfl_xor_sync(0xffffffffu, acc[ei][j], off);
+        if (lane == 0 && t0 + j < T_ && e0 + ei < E)
+          part[((int64_t)ks * T_ + t0 + j) * E + e0 + ei] = acc[ei][j];
+      }
   }
 }
 
@@ -216,8 +229,10 @@ gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const float NEG_INF = -INFINITY;
+  // Tokens interleave over the warps, so a chunk of fewer than 32 tokens (a
+  // decode step) still keeps every warp busy.
   for (int tt = 0; tt < kPermChunk / kSelWarps; ++tt) {
-    const int t = blockIdx.x * kPermChunk + warp * (kPermChunk / kSelWarps) + tt;
+    const int t = blockIdx.x * kPermChunk + tt * kSelWarps + warp;
     if (t >= T_) break;
     // Step 1: scores (kept raw for step 5).
     float s[NP], key[NP];
@@ -228,11 +243,18 @@ gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
       s[i] = e < E ? row[e] : NEG_INF;
     }
     if (!scores_in && ksplit > 1) {
+      // Unrolled so that all partial loads are in flight at once; the adds
+      // still run in ks order.
 #pragma unroll
       for (int i = 0; i < NP; ++i) {
         const int e = i * 32 + lane;
-        if (e < E)
-          for (int k = 1; k < ksplit; ++k) s[i] += logits[((int64_t)k * T_ + t) * E + e];
+        float p[kSplitK - 1];
+#pragma unroll
+        for (int q = 1; q < kSplitK; ++q)
+          p[q - 1] = (e < E && q < ksplit) ? logits[((int64_t)q * T_ + t) * E + e] : 0.f;
+#pragma unroll
+        for (int q = 1; q < kSplitK; ++q)
+          if (q < ksplit) s[i] += p[q - 1];
       }
     }
     if (!scores_in) {

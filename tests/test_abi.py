@@ -33,8 +33,9 @@ def test_library_exports_every_declared_symbol():
 def test_library_links_no_torch():
     # The library is plain C ABI: it must not need libtorch / libc10 to load.
     import subprocess
-    out = subprocess.run(["ldd", K.LIB_PATH], capture_output=True, text=True).stdout
-    assert "torch" not in out and "c10" not in out
+    r = subprocess.run(["ldd", K.LIB_PATH], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert "torch" not in r.stdout and "c10" not in r.stdout, r.stdout
 
 
 def test_config_struct_layout_matches_header():
