@@ -48,6 +48,7 @@
 // kernel records KT_ERR_TIMEOUT in the workspace error word, drains what it
 // issued, frees TMEM and returns.
 #include <cuda.h>
+#include <cstring>
 #include <cuda_bf16.h>
 
 #include "ktmoe_internal.cuh"
@@ -78,6 +79,14 @@ constexpr int kThreads = 192;
 constexpr int kStagingBytes = 4 * 16 * 32 * 4;   // 4 epilogue warps x [16 tokens][32 x 4 B]
 constexpr int kXchgBytes = 2 * 2 * 16 * 32 * 4;  // up -> gate: 2 warp pairs x 2 buffers
 constexpr int kCtrlBytes = 512;                  // mbarriers, TMEM address, schedule slots
+// Stage layout: [weight tiles of the stage's K slabs | token tiles of the same
+// slabs], each slab's weight tile 128 rows x 64 (16 KB) and its token tile
+// hb x 32 rows x 64, hb = ceil(token rows per CTA / 32). A tile with hb = 1 (a
+// pair N of at most 64) carries three K slabs per stage, others two.
+constexpr int kSlabsLight = 3;
+static_assert(kSlabsLight * (kATileBytes + kBoxBytes) <= kStageBytes, "3-slab stage layout");
+static_assert(kSlabs * (kATileBytes + kBTileBytes) <= kStageBytes, "2-slab stage layout");
+__device__ __forceinline__ int stage_slabs(int hb) { return hb == 1 ? kSlabsLight : kSlabs; }
 constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + kXchgBytes + kCtrlBytes + 1024;
 constexpr int kAccCols = 256;                    // TMEM columns per accumulator buffer
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -115,6 +124,23 @@ struct GemmArgs {
   const float* row_weight;   // down: weight of routed rows
   int n_routed_rows;         // T * k
   int* err;
+  int tma3d;                 // 1: one box per stage from the 3-D/4-D maps (K % 64 == 0)
+  int gate_hi;               // up, 3-D maps: W3 precedes W1 in memory, so the upper 64
+                             // rows of each CTA's weight tile are W1 (gate)
+};
+
+// Tensor maps of one launch (bf16, 128-byte swizzle). Token-row sources: up: 0
+// the permuted rows, 1 x (shared experts); down: the hidden rows; logits: x.
+//   2-D maps (K a multiple of 8): one K slab per box.
+//   3-D/4-D maps (K a multiple of 64): K split as [K / 64][64], so one box
+//   covers all K slabs of a stage; the gate/up weight map has a fourth
+//   dimension that steps from one of W1, W3 to the other, so one box yields
+//   [64 rows of one | the same 64 rows of the other] for every slab.
+struct TmaMaps {
+  CUtensorMap a2[2];      // weights, one slab: W1 | W2 | W_g, and W3 (up)
+  CUtensorMap b2[2][2];   // [source][32-row box, 128-row box], one slab
+  CUtensorMap a3[2];      // weights of a [2-slab, 3-slab] stage
+  CUtensorMap b3[2][5];   // [source][2-slab stage of 32/64/96/128 rows, 3-slab stage of 32]
 };
 
 // ---------------------------------------------------------------------------
@@ -194,6 +220,23 @@ __device__ __forceinline__ void tma_load_pair(void* dst, const CUtensorMap* map,
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load3_pair(void* dst, const CUtensorMap* map, uint32_t bar,
+                                               int c0, int c1, int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load4_pair(void* dst, const CUtensorMap* map, uint32_t bar,
+                                               int c0, int c1, int c2, int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "l"(policy)
       : "memory");
 }
 // L2 policies: data read once soon (evict first) and data re-read later (evict last).
@@ -343,13 +386,7 @@ __device__ __forceinline__ int pair_cols(int nrows) { return (nrows + 31) & ~31;
 // ---------------------------------------------------------------------------
 template <int kKind>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_g
-                    const __grid_constant__ CUtensorMap tmA1,    // W3 (up)
-                    const __grid_constant__ CUtensorMap tmB0s,   // token rows, 32-row box
-                    const __grid_constant__ CUtensorMap tmB0l,   // token rows, 128-row box
-                    const __grid_constant__ CUtensorMap tmB1s,   // x (up, shared experts), 32-row box
-                    const __grid_constant__ CUtensorMap tmB1l,   // x, 128-row box
-                    const GemmArgs args) {
+grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
   using KD = Kind<kKind>;
   constexpr bool kUp = KD::kUp;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -390,13 +427,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
       mbar_init(&sched_empty[i], kSchedConsumers);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    prefetch_tmap(&tmA0);
-    prefetch_tmap(&tmB0s);
-    prefetch_tmap(&tmB0l);
-    if (kUp) {
-      prefetch_tmap(&tmA1);
-      prefetch_tmap(&tmB1s);
-      prefetch_tmap(&tmB1l);
+    if (args.tma3d) {
+      for (int i = 0; i < 2; ++i) prefetch_tmap(&maps.a3[i]);
+      for (int i = 0; i < (kUp ? 2 : 1); ++i)
+        for (int j = 0; j < 5; ++j) prefetch_tmap(&maps.b3[i][j]);
+    } else {
+      for (int i = 0; i < (kUp ? 2 : 1); ++i) {
+        prefetch_tmap(&maps.a2[i]);
+        prefetch_tmap(&maps.b2[i][0]);
+        prefetch_tmap(&maps.b2[i][1]);
+      }
     }
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
@@ -409,8 +449,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
                           ? ((args.implicit_rows + kChunkRows - 1) / kChunkRows) * args.n_ftiles
                           : *args.n_tiles;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;   // static schedule only
-  // Stages per tile; slabs past K read as zeros (TMA fills out-of-range boxes).
-  const int nk = (args.K + kBK * kSlabs - 1) / (kBK * kSlabs);
+  // K slabs per tile (the last may run past K: TMA fills those columns with zeros).
+  const int n_slabs = (args.K + kBK - 1) / kBK;
   int* err = args.err;
 
   if (warp == 0) {
@@ -478,46 +518,55 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
         // First weight row of this CTA's half of the pair tile.
         const int a_row = ch.group * args.rows_per_group + ft * KD::kRowsPerPair +
                           (kUp ? 64 : 128) * (int)rank;
-        const CUtensorMap* bs = &tmB0s;
-        const CUtensorMap* bl = &tmB0l;
-        int b_row = ch.row0;
-        if (kUp) {
-          b_row = ch.src_row0;
-          if (ch.group >= args.E) {
-            bs = &tmB1s;
-            bl = &tmB1l;
-          }
-        }
-        b_row += half * (int)rank;
-        // Token rows: one 128-row box for a full half, else 32-row boxes (the
-        // last may run up to 16 rows past the chunk; those columns are unused).
-        const int nbox = half == kBHalfMax ? 0 : (half + kBoxRows - 1) / kBoxRows;
-        const uint32_t bbytes = nbox == 0 ? kBTileBytes : nbox * kBoxBytes;
-        const uint32_t tx = 2u * kSlabs * (kATileBytes + bbytes);   // both CTAs' bytes
+        const int src = (kUp && ch.group >= args.E) ? 1 : 0;
+        int b_row = (kUp ? ch.src_row0 : ch.row0) + half * (int)rank;
+        // Token rows in 32-row blocks (the last may run up to 16 rows past the
+        // chunk; those columns are unused).
+        const int hb = (half + kBoxRows - 1) / kBoxRows;
+        const int slabs = stage_slabs(hb);
+        const int nk = (n_slabs + slabs - 1) / slabs;
+        const uint32_t b_slab = hb * kBoxBytes;   // token-tile bytes of one slab
+        const CUtensorMap* a3 = &maps.a3[slabs == kSlabsLight ? 1 : 0];
+        const CUtensorMap* b3 = &maps.b3[src][slabs == kSlabsLight ? 4 : hb - 1];
         for (int kb = 0; kb < nk; ++kb) {
+          const int s0 = kb * slabs;
+          const int valid = min(slabs, n_slabs - s0);
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, err, 1 + 8 * kKind)) {
             ok = false;
             break;
           }
           const uint32_t fbar = map_to_cta(smem_u32(&full_bar[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
-#pragma unroll
-          for (int j = 0; j < kSlabs; ++j) {
-            uint8_t* sA = stage_base + stage * kStageBytes + j * kSlabBytes;
-            uint8_t* sB = sA + kATileBytes;
-            const int kc = (kb * kSlabs + j) * kBK;
-            if (kUp) {
-              // [64 rows of W1 | the same 64 rows of W3]
-              tma_load_pair(sA, &tmA0, fbar, kc, a_row, pol_a);
-              tma_load_pair(sA + 64 * 128, &tmA1, fbar, kc, a_row, pol_a);
-            } else {
-              tma_load_pair(sA, &tmA0, fbar, kc, a_row, pol_a);
-            }
-            if (nbox == 0) {
-              tma_load_pair(sB, bl, fbar, kc, b_row, pol_b);
-            } else {
-              for (int i = 0; i < nbox; ++i)
-                tma_load_pair(sB + i * kBoxBytes, bs, fbar, kc, b_row + i * kBoxRows, pol_b);
+          uint8_t* sA = stage_base + stage * kStageBytes;
+          uint8_t* sB = sA + slabs * kATileBytes;
+          if (args.tma3d) {
+            // Two boxes for the whole stage; slabs past K are filled with zeros
+            // and counted in the transaction bytes.
+            if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * slabs * (kATileBytes + b_slab));
+            if (kUp)
+              tma_load4_pair(sA, a3, fbar, 0, a_row, 0, s0, pol_a);
+            else
+              tma_load3_pair(sA, a3, fbar, 0, a_row, s0, pol_a);
+            tma_load3_pair(sB, b3, fbar, 0, b_row, s0, pol_b);
+          } else {
+            if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * valid * (kATileBytes + b_slab));
+            for (int j = 0; j < valid; ++j) {
+              const int kc = (s0 + j) * kBK;
+              uint8_t* a = sA + j * kATileBytes;
+              uint8_t* b = sB + j * b_slab;
+              if (kUp) {
+                // [64 rows of W1 | the same 64 rows of W3]
+                tma_load_pair(a, &maps.a2[0], fbar, kc, a_row, pol_a);
+                tma_load_pair(a + 64 * 128, &maps.a2[1], fbar, kc, a_row, pol_a);
+              } else {
+                tma_load_pair(a, &maps.a2[0], fbar, kc, a_row, pol_a);
+              }
+              if (half == kBHalfMax) {
+                tma_load_pair(b, &maps.b2[src][1], fbar, kc, b_row, pol_b);
+              } else {
+                for (int i = 0; i < hb; ++i)
+                  tma_load_pair(b + i * kBoxBytes, &maps.b2[src][0], fbar, kc,
+                                b_row + i * kBoxRows, pol_b);
+              }
             }
           }
           issued = issued < kStages ? issued + 1 : kStages;
@@ -574,7 +623,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
         tc_fence_after();
         const uint32_t idesc = idesc_bf16(256, n);
         const uint32_t d0 = tmem_base + buf * kAccCols;
+        const int hb = (n / 2 + kBoxRows - 1) / kBoxRows;
+        const int slabs = stage_slabs(hb);
+        const int nk = (n_slabs + slabs - 1) / slabs;
+        const uint32_t b_off = slabs * kATileBytes, b_slab = hb * kBoxBytes;
         for (int kb = 0; kb < nk; ++kb) {
+          const int valid = min(slabs, n_slabs - kb * slabs);
           if (!mbar_wait(&full_bar[stage], phase, err, 3 + 8 * kKind)) {
             ok = false;
             break;
@@ -582,9 +636,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
           // Descriptors of this stage: the start-address field counts 16-byte
           // units, so the 32-byte step between K sub-blocks adds 2.
 #pragma unroll
-          for (int j = 0; j < kSlabs; ++j) {
-            const uint64_t da = desc_a0 + (uint64_t)((stage * kStageBytes + j * kSlabBytes) >> 4);
-            const uint64_t db = da + (kATileBytes >> 4);
+          for (int j = 0; j < kSlabsLight; ++j) {
+            if (j >= valid) break;
+            const uint64_t da = desc_a0 + (uint64_t)((stage * kStageBytes + j * kATileBytes) >> 4);
+            const uint64_t db =
+                desc_a0 + (uint64_t)((stage * kStageBytes + b_off + j * b_slab) >> 4);
 #pragma unroll
             for (int ks = 0; ks < kBK / 16; ++ks)
               mma_pair_bf16(d0, da + 2 * ks, db + 2 * ks, idesc, (kb | j | ks) != 0);
@@ -620,7 +676,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,    // W1 / W2 / W_
     // hold up of the same features; warp pair p = q & 1 meets on named barrier
     // 1 + p (64 threads).
     const int pr = q & 1;
-    const bool gate_warp = q < 2;
+    const bool gate_warp = (q < 2) != (args.gate_hi != 0);
     const uint32_t tempty_leader0 = map_to_cta(smem_u32(&tempty_bar[0]), 0);
     const uint32_t tempty_leader1 = map_to_cta(smem_u32(&tempty_bar[1]), 0);
     int buf = 0;
@@ -759,14 +815,64 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
          CUDA_SUCCESS;
 }
 
+// 3-D view [cols / 64][rows][64] of a row-major [rows, cols] bf16 matrix (cols a
+// multiple of 64); box = box_slabs x box_rows x 64, landing slab-major.
+bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+               uint32_t box_slabs) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc || cols % kBK != 0) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kBK), rows, cols / kBK};
+  const cuuint64_t strides[2] = {cols * 2, static_cast<cuuint64_t>(kBK) * 2};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), box_rows, box_slabs};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// 4-D view [cols / 64][2][rows][64] of two equally shaped row-major bf16
+// matrices p and q (cols a multiple of 64): the second index steps from the one
+// at the lower address to the other. box = box_slabs x 2 x box_rows x 64, i.e.
+// per slab [box_rows rows of the first | the same rows of the second].
+// *q_first tells whether q is the first.
+bool make_map4_pair(CUtensorMap* m, const void* p, const void* q, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows, uint32_t box_slabs, bool* q_first) {
+  EncodeTiledFn enc = get_encode_fn();
+  const uint64_t up = reinterpret_cast<uint64_t>(p), uq = reinterpret_cast<uint64_t>(q);
+  const uint64_t lo = up < uq ? up : uq, hi = up < uq ? uq : up;
+  *q_first = uq < up;
+  if (!enc || cols % kBK != 0 || hi == lo || (hi - lo) % 16 != 0 || (hi - lo) >= (1ull << 40))
+    return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kBK), rows, 2, cols / kBK};
+  const cuuint64_t strides[3] = {cols * 2, hi - lo, static_cast<cuuint64_t>(kBK) * 2};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(kBK), box_rows, 2, box_slabs};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, reinterpret_cast<void*>(lo), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Token-row maps of one source: 2-D boxes of 32 and 128 rows; 3-D boxes of
+// 2-slab stages (32, 64, 96, 128 rows) and of 3-slab stages (32 rows).
+bool make_token_maps(TmaMaps* M, int src, const void* base, uint64_t rows, uint64_t cols,
+                     bool three_d) {
+  if (!make_map(&M->b2[src][0], base, rows, cols, kBoxRows) ||
+      !make_map(&M->b2[src][1], base, rows, cols, kBHalfMax))
+    return false;
+  if (!three_d) return true;
+  for (int hb = 1; hb <= 4; ++hb)
+    if (!make_map3(&M->b3[src][hb - 1], base, rows, cols, hb * kBoxRows, kSlabs)) return false;
+  return make_map3(&M->b3[src][4], base, rows, cols, kBoxRows, kSlabsLight);
+}
+
 template <int kKind>
-cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0s,
-                   const CUtensorMap& b0l, const CUtensorMap& b1s, const CUtensorMap& b1l,
-                   const GemmArgs& args, int grid, cudaStream_t st) {
+cudaError_t launch(const TmaMaps& maps, const GemmArgs& args, int grid, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kKind>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<kKind><<<grid, kThreads, kSmemBytes, st>>>(a0, a1, b0s, b0l, b1s, b1l, args);
+  grouped_gemm_kernel<kKind><<<grid, kThreads, kSmemBytes, st>>>(maps, args);
   return cudaGetLastError();
 }
 
@@ -793,14 +899,20 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
   a.err = reinterpret_cast<int*>(ws + L.err);
   a.E = r.E;
   const int grid = pair_grid(num_sms, 0);
+  TmaMaps M;
+  memset(&M, 0, sizeof(M));
   if (up) {
-    CUtensorMap mW1, mW3, mXps, mXpl, mXs, mXl;
-    if (!make_map(&mW1, wa, (uint64_t)NG * r.I, r.d, 64) ||
-        !make_map(&mW3, wb, (uint64_t)NG * r.I, r.d, 64) ||
-        !make_map(&mXps, ws + L.xperm, Rr, r.d, kBoxRows) ||
-        !make_map(&mXpl, ws + L.xperm, Rr, r.d, kBHalfMax) ||
-        !make_map(&mXs, x, T, r.d, kBoxRows) || !make_map(&mXl, x, T, r.d, kBHalfMax))
+    const uint64_t rows = (uint64_t)NG * r.I;
+    if (!make_map(&M.a2[0], wa, rows, r.d, 64) || !make_map(&M.a2[1], wb, rows, r.d, 64) ||
+        !make_token_maps(&M, 0, ws + L.xperm, Rr, r.d, false) ||
+        !make_token_maps(&M, 1, x, T, r.d, false))
       return cudaErrorInvalidValue;
+    bool w3_first = false;
+    a.tma3d = make_map4_pair(&M.a3[0], wa, wb, rows, r.d, 64, kSlabs, &w3_first) &&
+              make_map4_pair(&M.a3[1], wa, wb, rows, r.d, 64, kSlabsLight, &w3_first) &&
+              make_token_maps(&M, 0, ws + L.xperm, Rr, r.d, true) &&
+              make_token_maps(&M, 1, x, T, r.d, true);
+    a.gate_hi = a.tma3d && w3_first;
     a.tiles = reinterpret_cast<const int2*>(ws + L.tiles_up);
     a.n_tiles = meta + 1;
     a.counter = const_cast<int32_t*>(meta) + 3;
@@ -811,13 +923,16 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
     a.ldo = r.I;
     a.out = ws + L.hidden;
     a.row_weight = nullptr;
-    return launch<kKindUp>(mW1, mW3, mXps, mXpl, mXs, mXl, a, grid, st);
+    return launch<kKindUp>(M, a, grid, st);
   }
-  CUtensorMap mW2, mHs, mHl;
-  if (!make_map(&mW2, wa, (uint64_t)NG * r.d, r.I, kARowsCta) ||
-      !make_map(&mHs, ws + L.hidden, R, r.I, kBoxRows) ||
-      !make_map(&mHl, ws + L.hidden, R, r.I, kBHalfMax))
+  const uint64_t rows = (uint64_t)NG * r.d;
+  if (!make_map(&M.a2[0], wa, rows, r.I, kARowsCta) ||
+      !make_token_maps(&M, 0, ws + L.hidden, R, r.I, false))
     return cudaErrorInvalidValue;
+  a.tma3d = make_map3(&M.a3[0], wa, rows, r.I, kARowsCta, kSlabs) &&
+            make_map3(&M.a3[1], wa, rows, r.I, kARowsCta, kSlabsLight) &&
+            make_token_maps(&M, 0, ws + L.hidden, R, r.I, true);
+  a.gate_hi = 0;
   a.tiles = reinterpret_cast<const int2*>(ws + L.tiles_down);
   a.n_tiles = meta + 2;
   a.counter = const_cast<int32_t*>(meta) + 4;
@@ -828,16 +943,21 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
   a.ldo = r.d;
   a.out = ws + L.expert_out;
   a.row_weight = reinterpret_cast<const float*>(ws + L.row_weight);
-  return launch<kKindDown>(mW2, mW2, mHs, mHl, mHs, mHl, a, grid, st);
+  return launch<kKindDown>(M, a, grid, st);
 }
 
 cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, const void* w_gate,
                                   float* logits, int* err, int num_sms, cudaStream_t st) {
-  CUtensorMap mWg, mXs, mXl;
-  if (!make_map(&mWg, w_gate, (uint64_t)r.E, r.d, kARowsCta) ||
-      !make_map(&mXs, x, T, r.d, kBoxRows) || !make_map(&mXl, x, T, r.d, kBHalfMax))
+  TmaMaps M;
+  memset(&M, 0, sizeof(M));
+  if (!make_map(&M.a2[0], w_gate, (uint64_t)r.E, r.d, kARowsCta) ||
+      !make_token_maps(&M, 0, x, T, r.d, false))
     return cudaErrorInvalidValue;
   GemmArgs a{};
+  a.tma3d = make_map3(&M.a3[0], w_gate, (uint64_t)r.E, r.d, kARowsCta, kSlabs) &&
+            make_map3(&M.a3[1], w_gate, (uint64_t)r.E, r.d, kARowsCta, kSlabsLight) &&
+            make_token_maps(&M, 0, x, T, r.d, true);
+  a.gate_hi = 0;
   a.chunks = nullptr;
   a.tiles = nullptr;
   a.n_tiles = nullptr;
@@ -846,7 +966,7 @@ cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, c
   a.n_ftiles = (r.E + 255) / 256;
   a.rows_per_group = r.E;
   a.K = r.d;
-  a.E = 1;                  // every chunk reads its token rows from the first B maps
+  a.E = 1;                  // every chunk reads its token rows from source 0
   a.out_cols = r.E;
   a.ldo = r.E;
   a.out = logits;
@@ -854,7 +974,7 @@ cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, c
   a.n_routed_rows = 0;
   a.err = err;
   const int tiles = (int)((T + kChunkRows - 1) / kChunkRows) * a.n_ftiles;
-  return launch<kKindLogits>(mWg, mWg, mXs, mXl, mXs, mXl, a, pair_grid(num_sms, tiles), st);
+  return launch<kKindLogits>(M, a, pair_grid(num_sms, tiles), st);
 }
 
 }  // namespace ktmoe

@@ -222,3 +222,21 @@ def test_workspace_reuse_across_layers():
     inp = W.make_layer(small, "cuda")
     out = run_forward(small, inp, ws=ws, y_fp32=True)
     _check_layer(small, inp, list(range(0, small.T, 7)), out=out)
+
+
+def test_w3_below_w1_in_memory_gives_the_same_output():
+    """The gate/up weight loads read W1 and W3 rows in one box whose extra
+    dimension steps from the lower of the two addresses to the higher; with W3
+    placed below W1 the kernel must still take gate from W1. Same arithmetic in
+    the same order, so the output is bitwise the same."""
+    layer = W.BY_NAME["small_sig_bias"]
+    inp = W.make_layer(layer, "cuda")
+    a = run_forward(layer, inp, y_fp32=True)
+    both = torch.empty((2,) + tuple(inp["w1"].shape), dtype=inp["w1"].dtype, device="cuda")
+    both[0].copy_(inp["w3"])
+    both[1].copy_(inp["w1"])
+    inp2 = dict(inp, w1=both[1], w3=both[0])
+    assert inp2["w3"].data_ptr() < inp2["w1"].data_ptr()
+    b = run_forward(layer, inp2, y_fp32=True)
+    assert torch.equal(a["idx"], b["idx"])
+    assert torch.equal(a["y"], b["y"])
