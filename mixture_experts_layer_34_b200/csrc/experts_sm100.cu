@@ -464,15 +464,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
       int issued = 0;
       int sslot = 0, iter = 0;
       uint32_t sphase = 0;
-      // Expert weights stream through once per tile group (evict first); token
-      // rows are re-read by every feature tile of their chunk (evict last). The
-      // gate logits re-read W_g for every token chunk instead.
-#if KT_L2_HINTS
-      const uint64_t pol_a = kKind == kKindLogits ? policy_evict_last() : policy_evict_first();
-      const uint64_t pol_b = kKind == kKindLogits ? policy_evict_first() : policy_evict_last();
-#else
-      const uint64_t pol_a = policy_evict_normal(), pol_b = pol_a;
-#endif
+      const uint64_t p_first = policy_evict_first(), p_normal = policy_evict_normal(),
+                     p_last = policy_evict_last();
       for (;;) {
         int t;
         if (leader) {
@@ -518,6 +511,24 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
         // First weight row of this CTA's half of the pair tile.
         const int a_row = ch.group * args.rows_per_group + ft * KD::kRowsPerPair +
                           (kUp ? 64 : 128) * (int)rank;
+        // L2 priorities (KT_L2_HINTS): 0 none; 1 weights evict-first, token rows
+        // evict-last; 2 as 1 for partial chunks, while a full chunk's weights
+        // (re-read by the expert's other chunks) stay normal; 3 as 2 with
+        // normal token rows. The gate logits re-read W_g for every chunk.
+        uint64_t pol_a = p_normal, pol_b = p_normal;
+        if (KT_L2_HINTS != 0) {
+          const bool full = ch.nrows == kChunkRows;
+          if (kKind == kKindLogits) {
+            pol_a = p_last;
+            pol_b = p_first;
+          } else if (KT_L2_HINTS == 1) {
+            pol_a = p_first;
+            pol_b = p_last;
+          } else {
+            pol_a = full ? p_normal : p_first;
+            pol_b = (KT_L2_HINTS == 2 && full) ? p_last : p_normal;
+          }
+        }
         const int src = (kUp && ch.group >= args.E) ? 1 : 0;
         int b_row = (kUp ? ch.src_row0 : ch.row0) + half * (int)rank;
         // Token rows in 32-row blocks (the last may run up to 16 rows past the

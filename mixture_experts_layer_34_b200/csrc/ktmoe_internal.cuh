@@ -24,7 +24,7 @@ constexpr int kChunkRows = 256;     // token rows per GEMM chunk (MMA N <= 256)
 #define KT_HEAVY_ROWS 192
 #endif
 #ifndef KT_L2_HINTS
-#define KT_L2_HINTS 1
+#define KT_L2_HINTS 2
 #endif
 constexpr int kTileBlock = KT_TILE_BLOCK;   // chunks per schedule block (feature-tile-major inside)
 constexpr int kHeavyRows = KT_HEAVY_ROWS;   // experts with at least this many rows are compute-bound
