@@ -51,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=W.V3_PREFILL.name)
     ap.add_argument("--decode-workload", default=W.V3_DECODE.name, help="'none' to skip")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall time of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args(argv)
@@ -294,7 +294,7 @@ def cpu_oracle_sample(layer, inp, idx_all, target_s: float) -> dict:
     n = max(1, min(layer.T, threads))
     dt = run(n)
     if dt < 0.5 * target_s and n < layer.T:
-        n = int(min(layer.T, max(n + 1, n * target_s / max(dt, 1e-3)), 16 * threads))
+        n = int(min(layer.T, max(n + 1, n * target_s / max(dt, 1e-3)), 64 * threads))
         dt = run(n)
     return {"value": n / dt, "unit": "tokens/s", "cores": min(threads, n), "kind": "oracle",
             "sample": f"first {n} tokens of {layer.name}: fp64 gate + literal expert loop "
