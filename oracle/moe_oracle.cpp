@@ -265,6 +265,74 @@ int oracle_forward(const oracle_cfg* c, int64_t T, int dtype, const void* x,
   return bad ? -1 : 0;
 }
 
+// Expert load: how many (token, slot) picks each routed expert received, i.e.
+// the histogram of idx [T, k]. counts is [E]. Returns -1 if an index is out of
+// range (and counts only the valid ones).
+int oracle_expert_load(const oracle_cfg* c, int64_t T, const int32_t* idx, int64_t* counts) {
+  const int E = c->n_experts, k = c->topk;
+  int bad = 0;
+  for (int e = 0; e < E; ++e) counts[e] = 0;
+  for (int64_t i = 0; i < T * k; ++i) {
+    if (idx[i] < 0 || idx[i] >= E) {
+      bad = 1;
+      continue;
+    }
+    ++counts[idx[i]];
+  }
+  return bad ? -1 : 0;
+}
+
+// Aux-loss-free bias update ("V3 改进①：无辅助损失负载均衡": the bias follows the
+// expert's load, at a speed set by gamma). Reading of the rule: the mean load is
+// T*k/E picks per expert; an expert above it is overloaded and its bias drops
+// by gamma, one below it is underloaded and its bias rises by gamma, one exactly
+// at it keeps its bias. The comparison load_i > T*k/E is done in integers
+// (load_i * E > T * k); the update is one fp32 addition. bias [E] is in-out.
+int oracle_bias_update(const oracle_cfg* c, int64_t T, const int32_t* idx, float gamma,
+                       float* bias) {
+  const int E = c->n_experts, k = c->topk;
+  std::vector<int64_t> load(E);
+  const int rc = oracle_expert_load(c, T, idx, load.data());
+  const int64_t total = T * (int64_t)k;
+  for (int e = 0; e < E; ++e) {
+    const int64_t scaled = load[e] * (int64_t)E;
+    if (scaled > total)
+      bias[e] = bias[e] - gamma;
+    else if (scaled < total)
+      bias[e] = bias[e] + gamma;
+  }
+  return rc;
+}
+
+// Sequence-wise balance statistics ("V3 改进②：序列级平衡损失",
+// L_Bal = alpha * sum_i f_i * P_i) over the T tokens given:
+//   f_i = (1/T) * #{t : i is among idx_t}      (top-k activation frequency),
+//   P_i = (1/T) * sum_t s_{i,t} / sum_j s_{j,t} (time mean of the normalised
+//                                                affinity s'),
+// with s the fp32 scores [T, E] (after the score function, before any bias).
+// Everything in double; f, P are [E], loss is one value.
+int oracle_balance_stats(const oracle_cfg* c, int64_t T, const float* scores,
+                         const int32_t* idx, double alpha, double* f, double* P,
+                         double* loss) {
+  const int E = c->n_experts;
+  std::vector<int64_t> load(E);
+  const int rc = oracle_expert_load(c, T, idx, load.data());
+  for (int e = 0; e < E; ++e) P[e] = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    double z = 0.0;
+    for (int e = 0; e < E; ++e) z += (double)scores[t * E + e];
+    for (int e = 0; e < E; ++e) P[e] += (double)scores[t * E + e] / z;
+  }
+  double l = 0.0;
+  for (int e = 0; e < E; ++e) {
+    f[e] = (double)load[e] / (double)T;
+    P[e] = P[e] / (double)T;
+    l += f[e] * P[e];
+  }
+  *loss = alpha * l;
+  return rc;
+}
+
 // One expert's SwiGLU hidden vector h = silu(W1 u) * W3 u for n_tok tokens,
 // double. h is [n_tok, I]. Used to localise a mismatch to the first GEMM.
 int oracle_expert_hidden(const oracle_cfg* c, int64_t T, int dtype, const void* x,

@@ -61,6 +61,9 @@ def _load():
             lib.oracle_select.argtypes = [CP, I64, P, P, P, P, P, P, P, P]
             lib.oracle_forward.argtypes = [CP, I64, ctypes.c_int, P, P, P, P, P, P, I64, P, P]
             lib.oracle_expert_hidden.argtypes = [CP, I64, ctypes.c_int, P, P, P, I64, P, P]
+            lib.oracle_expert_load.argtypes = [CP, I64, P, P]
+            lib.oracle_bias_update.argtypes = [CP, I64, P, ctypes.c_float, P]
+            lib.oracle_balance_stats.argtypes = [CP, I64, P, P, ctypes.c_double, P, P, P]
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -221,3 +224,37 @@ def expert_hidden(cfg: dict, x, w1_e, w3_e, tok_ids) -> np.ndarray:
     if rcode != 0:
         raise ValueError("oracle_expert_hidden: bad token id")
     return h
+
+
+def expert_load(cfg: dict, idx: np.ndarray) -> np.ndarray:
+    """Picks per routed expert (histogram of idx [T, k]), int64 [E]."""
+    idx = np.ascontiguousarray(idx, np.int32)
+    out = np.empty(cfg["n_experts"], np.int64)
+    c = _cfg_struct(resolve(dict(cfg, topk=idx.shape[1]), False))
+    if _load().oracle_expert_load(ctypes.byref(c), idx.shape[0], _ptr(idx), _ptr(out)) != 0:
+        raise ValueError("oracle_expert_load: expert index out of range")
+    return out
+
+
+def bias_update(cfg: dict, idx: np.ndarray, gamma: float, bias) -> np.ndarray:
+    """Aux-loss-free bias update: returns the new fp32 bias [E]."""
+    idx = np.ascontiguousarray(idx, np.int32)
+    b = np.array(_as_raw(bias)[0], np.float32, copy=True)
+    c = _cfg_struct(resolve(dict(cfg, topk=idx.shape[1]), False))
+    if _load().oracle_bias_update(ctypes.byref(c), idx.shape[0], _ptr(idx), ctypes.c_float(gamma),
+                                  _ptr(b)) != 0:
+        raise ValueError("oracle_bias_update: expert index out of range")
+    return b
+
+
+def balance_stats(cfg: dict, s: np.ndarray, idx: np.ndarray, alpha: float) -> dict:
+    """f [E], P [E] and L_Bal = alpha * sum f P, float64, from fp32 scores [T, E]."""
+    s = np.ascontiguousarray(s, np.float32)
+    idx = np.ascontiguousarray(idx, np.int32)
+    E = s.shape[1]
+    f, P, loss = np.empty(E, np.float64), np.empty(E, np.float64), np.empty(1, np.float64)
+    c = _cfg_struct(resolve(dict(cfg, n_experts=E, topk=idx.shape[1]), False))
+    if _load().oracle_balance_stats(ctypes.byref(c), s.shape[0], _ptr(s), _ptr(idx),
+                                    ctypes.c_double(alpha), _ptr(f), _ptr(P), _ptr(loss)) != 0:
+        raise ValueError("oracle_balance_stats: expert index out of range")
+    return dict(f=f, P=P, loss=float(loss[0]))
