@@ -191,6 +191,61 @@ int kt_moe_forward_static(const kt_moe_config* cfg, int64_t T, const void* x,
  * kt_moe_check and for reading its buffers after kt_moe_forward_static. */
 void* kt_moe_static_scratch(void);
 
+/*
+ * Scores alone: s = the score function of the gate logits, gate step 1 of the
+ * "Gate 选专家流程（model.py，五步）" passage of the DeepSeek-V3 model.py notes
+ * (sigmoid, or softmax over all experts), for the balance statistics below or
+ * for the caller's own use.
+ *   x, w_gate   as for kt_moe_gate
+ *   scores_out  device [T, E] fp32 (out)
+ *   workspace   device, ws_bytes >= kt_moe_workspace_size(cfg, T), 256-B aligned
+ * Computed by the same code as kt_moe_gate's selection, so kt_moe_gate with
+ * scores_in = scores_out gives exactly the routing kt_moe_gate computes from x.
+ */
+int kt_moe_scores(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                  float* scores_out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Aux-loss-free bias update ("V3 改进①：无辅助损失负载均衡" of the DeepSeek-V3
+ * model.py notes: the selection bias follows each expert's load, at a speed
+ * gamma). The load of expert i is the number of its picks among the T*k
+ * (token, slot) pairs of topk_idx; the mean load is T*k/E. An expert above the
+ * mean has its bias lowered by gamma, one below it raised by gamma, one exactly
+ * at it keeps its bias (compared in integers; one fp32 addition per expert).
+ *   topk_idx  device [T, k] int32: a routing (kt_moe_gate / kt_moe_forward);
+ *             indices outside [0, E) are not counted
+ *   bias      device [E] fp32, updated in place
+ *   gamma     finite, >= 0
+ *   load_out  device [E] int32 or NULL (out): the loads
+ * One kernel on `stream`, no workspace. Errors: KT_ERR_INVALID_CONFIG (config,
+ * T or gamma), KT_ERR_NULL, KT_ERR_ALIGN (4-B alignment), KT_ERR_CUDA.
+ */
+int kt_moe_bias_update(const kt_moe_config* cfg, int64_t T, const int32_t* topk_idx,
+                       float* bias, float gamma, int32_t* load_out, void* stream);
+
+/*
+ * Sequence-wise balance statistics ("V3 改进②：序列级平衡损失" of the DeepSeek-V3
+ * model.py notes, L_Bal = alpha * sum_i f_i * P_i) over T tokens:
+ *   f_i = load_i / T                          (top-k activation frequency)
+ *   P_i = (1/T) * sum_t s_{i,t} / sum_j s_{j,t} (time mean of the normalised
+ *                                               affinity)
+ *   scores    device [T, E] fp32: s after the score function (kt_moe_scores)
+ *   topk_idx  device [T, k] int32 (indices outside [0, E) are not counted)
+ *   alpha     finite
+ *   f_out, P_out  device [E] fp32 (out); loss_out device [1] fp32 (out)
+ *   workspace device, ws_bytes >= kt_moe_balance_workspace_size(cfg, T),
+ *             256-B aligned
+ * fp32 sums in a fixed order (per token, per chunk of tokens, then over the
+ * chunks), so repeated calls give bitwise-equal results; the loss sums the E
+ * products in double. The page gives f_i only as the activation frequency: any
+ * constant factor on it (the paper's experts / top-k normalisation) is a
+ * factor on alpha.
+ */
+size_t kt_moe_balance_workspace_size(const kt_moe_config* cfg, int64_t T);
+int kt_moe_balance_stats(const kt_moe_config* cfg, int64_t T, const float* scores,
+                         const int32_t* topk_idx, float alpha, float* f_out, float* P_out,
+                         float* loss_out, void* workspace, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, then read the device error word the last call on this
  * workspace left (a bounded wait inside a kernel that gave up sets it).
  * Returns KT_OK, KT_ERR_TIMEOUT, or KT_ERR_CUDA if the stream reports an error. */

@@ -195,6 +195,75 @@ int kt_moe_gate(const kt_moe_config* cfg, int64_t T, const void* x, const void* 
   return KT_OK;
 }
 
+int kt_moe_scores(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                  float* scores_out, void* workspace, size_t ws_bytes, void* stream) {
+  Resolved r;
+  int rc = resolve(cfg, T, 0, &r);
+  if (rc != KT_OK) return rc;
+  if (!x || !w_gate || !scores_out) return KT_ERR_NULL;
+  if (!workspace) return KT_ERR_WORKSPACE;
+  const Layout L = make_layout(r, T);
+  if (ws_bytes < L.total) return KT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256) || !aligned(scores_out, 4) || !aligned(x, 16) ||
+      !aligned(w_gate, 16))
+    return KT_ERR_ALIGN;
+  if (overlaps(scores_out, (size_t)T * r.E * 4, workspace, ws_bytes)) return KT_ERR_INVALID_CONFIG;
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_gate_scores(r, T, logits, scores_out, st) != cudaSuccess) return KT_ERR_CUDA;
+  return KT_OK;
+}
+
+int kt_moe_bias_update(const kt_moe_config* cfg, int64_t T, const int32_t* topk_idx,
+                       float* bias, float gamma, int32_t* load_out, void* stream) {
+  Resolved r;
+  int rc = resolve(cfg, T, 1, &r);
+  if (rc != KT_OK) return rc;
+  if (!std::isfinite(gamma) || gamma < 0.f) return KT_ERR_INVALID_CONFIG;
+  if (!topk_idx || !bias) return KT_ERR_NULL;
+  if (!aligned(topk_idx, 4) || !aligned(bias, 4) || (load_out && !aligned(load_out, 4)))
+    return KT_ERR_ALIGN;
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  if (launch_bias_update(r, T, topk_idx, bias, gamma, load_out,
+                         static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KT_ERR_CUDA;
+  return KT_OK;
+}
+
+size_t kt_moe_balance_workspace_size(const kt_moe_config* cfg, int64_t T) {
+  Resolved r;
+  if (resolve(cfg, T, 0, &r) != KT_OK) return 0;
+  return balance_scratch_bytes(r, T);
+}
+
+int kt_moe_balance_stats(const kt_moe_config* cfg, int64_t T, const float* scores,
+                         const int32_t* topk_idx, float alpha, float* f_out, float* P_out,
+                         float* loss_out, void* workspace, size_t ws_bytes, void* stream) {
+  Resolved r;
+  int rc = resolve(cfg, T, 0, &r);
+  if (rc != KT_OK) return rc;
+  if (!std::isfinite(alpha)) return KT_ERR_INVALID_CONFIG;
+  if (!scores || !topk_idx || !f_out || !P_out || !loss_out) return KT_ERR_NULL;
+  if (!workspace) return KT_ERR_WORKSPACE;
+  if (ws_bytes < balance_scratch_bytes(r, T)) return KT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256) || !aligned(scores, 4) || !aligned(topk_idx, 4) ||
+      !aligned(f_out, 4) || !aligned(P_out, 4) || !aligned(loss_out, 4))
+    return KT_ERR_ALIGN;
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  if (launch_balance_stats(r, T, scores, topk_idx, alpha, f_out, P_out, loss_out, workspace,
+                           static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KT_ERR_CUDA;
+  return KT_OK;
+}
+
 int kt_moe_forward(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
                    const float* bias, const void* w1, const void* w3, const void* w2, void* y,
                    int32_t* topk_idx_out, float* topk_w_out, void* workspace, size_t ws_bytes,

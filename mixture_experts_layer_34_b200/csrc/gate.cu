@@ -212,6 +212,66 @@ __device__ __forceinline__ Best warp_argmax(Best b) {
   return b;
 }
 
+// Gate step 1 and the score function for token t, one warp: lane l gets the
+// scores of experts i * 32 + l in s[i]. `logits` holds `ksplit` partial sums
+// [ksplit][T][E], added in ks order; if `scores_in` is given it is used as is.
+// Lanes past E hold -inf (scores_in), 0 (sigmoid of -inf) or 0 (softmax).
+template <int NP>
+__device__ __forceinline__ void token_scores(const Resolved& r, int T_, int ksplit,
+                                             const float* __restrict__ logits,
+                                             const float* __restrict__ scores_in, int t, int lane,
+                                             float (&s)[NP]) {
+  const int E = r.E;
+  const float NEG_INF = -INFINITY;
+  const float* row = (scores_in ? scores_in : logits) + (int64_t)t * E;
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    const int e = i * 32 + lane;
+    s[i] = e < E ? row[e] : NEG_INF;
+  }
+  if (!scores_in && ksplit > 1) {
+    // Unrolled so that all partial loads are in flight at once; the adds
+    // still run in ks order.
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const int e = i * 32 + lane;
+      float p[kSplitK - 1];
+#pragma unroll
+      for (int q = 1; q < kSplitK; ++q)
+        p[q - 1] = (e < E && q < ksplit) ? logits[((int64_t)q * T_ + t) * E + e] : 0.f;
+#pragma unroll
+      for (int q = 1; q < kSplitK; ++q)
+        if (q < ksplit) s[i] += p[q - 1];
+    }
+  }
+  if (!scores_in) {
+    if (r.score_func == KT_SCORE_SIGMOID) {
+#pragma unroll
+      for (int i = 0; i < NP; ++i)
+        s[i] = 1.0f / (1.0f + expf(-s[i]));
+    } else {
+      float m = NEG_INF;
+#pragma unroll
+      for (int i = 0; i < NP; ++i)
+        m = fmaxf(m, s[i]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+      float z = 0.f;
+#pragma unroll
+      for (int i = 0; i < NP; ++i)
+        {
+          s[i] = (i * 32 + lane < E) ? expf(s[i] - m) : 0.f;
+          z += s[i];
+        }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFull, z, off);
+#pragma unroll
+      for (int i = 0; i < NP; ++i)
+        s[i] = __fdiv_rn(s[i], z);
+    }
+  }
+}
+
 // NP = experts per lane (E <= 32 * NP), a compile-time bound so the per-lane
 // arrays stay in registers. ksplit > 1: `logits` holds ksplit partial sums
 // [ksplit][T][E], added here in order.
@@ -236,53 +296,7 @@ gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
     if (t >= T_) break;
     // Step 1: scores (kept raw for step 5).
     float s[NP], key[NP];
-    const float* row = (scores_in ? scores_in : logits) + (int64_t)t * E;
-#pragma unroll
-    for (int i = 0; i < NP; ++i) {
-      const int e = i * 32 + lane;
-      s[i] = e < E ? row[e] : NEG_INF;
-    }
-    if (!scores_in && ksplit > 1) {
-      // Unrolled so that all partial loads are in flight at once; the adds
-      // still run in ks order.
-#pragma unroll
-      for (int i = 0; i < NP; ++i) {
-        const int e = i * 32 + lane;
-        float p[kSplitK - 1];
-#pragma unroll
-        for (int q = 1; q < kSplitK; ++q)
-          p[q - 1] = (e < E && q < ksplit) ? logits[((int64_t)q * T_ + t) * E + e] : 0.f;
-#pragma unroll
-        for (int q = 1; q < kSplitK; ++q)
-          if (q < ksplit) s[i] += p[q - 1];
-      }
-    }
-    if (!scores_in) {
-      if (r.score_func == KT_SCORE_SIGMOID) {
-#pragma unroll
-        for (int i = 0; i < NP; ++i)
-          s[i] = 1.0f / (1.0f + expf(-s[i]));
-      } else {
-        float m = NEG_INF;
-#pragma unroll
-        for (int i = 0; i < NP; ++i)
-          m = fmaxf(m, s[i]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-        float z = 0.f;
-#pragma unroll
-        for (int i = 0; i < NP; ++i)
-          {
-            s[i] = (i * 32 + lane < E) ? expf(s[i] - m) : 0.f;
-            z += s[i];
-          }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFull, z, off);
-#pragma unroll
-        for (int i = 0; i < NP; ++i)
-          s[i] = __fdiv_rn(s[i], z);
-      }
-    }
+    token_scores<NP>(r, T_, ksplit, logits, scores_in, t, lane, s);
     // Step 2a: selection keys s + b (the bias takes part in the selection only).
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
@@ -381,6 +395,27 @@ gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
       chunk_counts[(int64_t)blockIdx.x * E + e] = scount[e];
 }
 
+// Scores alone: s [T, E] fp32, the score function of the logits, computed by
+// the same token_scores as the selection (so selecting from these scores gives
+// the selection's result bit for bit). Same token-to-warp mapping.
+template <int NP>
+__global__ void __launch_bounds__(kSelWarps * 32)
+gate_scores_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ logits,
+                   float* __restrict__ out) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int tt = 0; tt < kPermChunk / kSelWarps; ++tt) {
+    const int t = blockIdx.x * kPermChunk + tt * kSelWarps + warp;
+    if (t >= T_) break;
+    float s[NP];
+    token_scores<NP>(r, T_, ksplit, logits, nullptr, t, lane, s);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const int e = i * 32 + lane;
+      if (e < r.E) out[(int64_t)t * r.E + e] = s[i];
+    }
+  }
+}
+
 }  // namespace
 
 int gate_logit_splits(const Resolved& r, int64_t T) { return T <= kSmallTokens ? kSplitK : 1; }
@@ -427,6 +462,26 @@ cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits
   else if (np <= 8) KT_SELECT(8);
   else KT_SELECT(16);
 #undef KT_SELECT
+  return cudaGetLastError();
+}
+
+}  // namespace ktmoe
+
+namespace ktmoe {
+
+cudaError_t launch_gate_scores(const Resolved& r, int64_t T, const float* logits, float* scores,
+                               cudaStream_t st) {
+  const unsigned grid = (unsigned)((T + kPermChunk - 1) / kPermChunk);
+  const int ks = gate_logit_splits(r, T);
+  const int np = (r.E + 31) / 32;
+#define KT_SCORES(NPV) \
+  gate_scores_kernel<NPV><<<grid, kSelWarps * 32, 0, st>>>(r, (int)T, ks, logits, scores)
+  if (np <= 1) KT_SCORES(1);
+  else if (np <= 2) KT_SCORES(2);
+  else if (np <= 4) KT_SCORES(4);
+  else if (np <= 8) KT_SCORES(8);
+  else KT_SCORES(16);
+#undef KT_SCORES
   return cudaGetLastError();
 }
 

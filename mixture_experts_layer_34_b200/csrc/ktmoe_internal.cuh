@@ -105,6 +105,18 @@ cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, c
 cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits,
                                const float* scores_in, const float* bias, int32_t* idx,
                                float* w, int32_t* chunk_counts, cudaStream_t st);
+// Scores s [T, E] fp32 from the logits region (gate step 1's score function).
+cudaError_t launch_gate_scores(const Resolved& r, int64_t T, const float* logits, float* scores,
+                               cudaStream_t st);
+// Load statistics (balance.cu).
+cudaError_t launch_bias_update(const Resolved& r, int64_t T, const int32_t* idx, float* bias,
+                               float gamma, int32_t* load_out, cudaStream_t st);
+// Token chunks of the balance statistics and the scratch bytes they need.
+int balance_chunks(int64_t T, int* tokens_per_chunk);
+size_t balance_scratch_bytes(const Resolved& r, int64_t T);
+cudaError_t launch_balance_stats(const Resolved& r, int64_t T, const float* scores,
+                                 const int32_t* idx, float alpha, float* f, float* P, float* loss,
+                                 void* scratch, cudaStream_t st);
 cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* ws,
                            const int32_t* idx, const float* w, const void* x, cudaStream_t st);
 // up = true: the gate/up GEMM (wa = W1, wb = W3); up = false: the down GEMM

@@ -25,7 +25,9 @@ KT_STATIC_SCRATCH_BYTES = 32 << 20
 # Every symbol include/ktmoe.h declares.
 EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_forward",
            "kt_moe_forward_profiled", "kt_moe_forward_static", "kt_moe_static_scratch",
-           "kt_moe_check", "kt_moe_workspace_layout", "kt_moe_strerror", "kt_moe_version")
+           "kt_moe_check", "kt_moe_workspace_layout", "kt_moe_strerror", "kt_moe_version",
+           "kt_moe_scores", "kt_moe_bias_update", "kt_moe_balance_workspace_size",
+           "kt_moe_balance_stats")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -86,6 +88,15 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_workspace_layout.restype = ctypes.c_int
             L.kt_moe_strerror.argtypes = [ctypes.c_int]
             L.kt_moe_strerror.restype = ctypes.c_char_p
+            L.kt_moe_scores.argtypes = [CP, I64, P, P, P, P, ctypes.c_size_t, P]
+            L.kt_moe_scores.restype = ctypes.c_int
+            L.kt_moe_bias_update.argtypes = [CP, I64, P, P, ctypes.c_float, P, P]
+            L.kt_moe_bias_update.restype = ctypes.c_int
+            L.kt_moe_balance_workspace_size.argtypes = [CP, I64]
+            L.kt_moe_balance_workspace_size.restype = ctypes.c_size_t
+            L.kt_moe_balance_stats.argtypes = [CP, I64, P, P, ctypes.c_float, P, P, P, P,
+                                               ctypes.c_size_t, P]
+            L.kt_moe_balance_stats.restype = ctypes.c_int
             L.kt_moe_version.argtypes = []
             L.kt_moe_version.restype = ctypes.c_int
             _lib = L
@@ -148,6 +159,34 @@ def kt_moe_gate(cfg, T, x, w_gate, bias, scores_in, topk_idx, topk_w, workspace,
                            _nbytes(workspace), _stream(stream))
     if rc != KT_OK:
         raise KtMoeError("kt_moe_gate", rc)
+
+
+def kt_moe_scores(cfg, T, x, w_gate, scores_out, workspace, stream=None):
+    rc = lib().kt_moe_scores(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(scores_out),
+                             _ptr(workspace), _nbytes(workspace), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_scores", rc)
+
+
+def kt_moe_bias_update(cfg, T, topk_idx, bias, gamma, load_out=None, stream=None):
+    rc = lib().kt_moe_bias_update(ctypes.byref(cfg), int(T), _ptr(topk_idx), _ptr(bias),
+                                  ctypes.c_float(gamma), _ptr(load_out), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_bias_update", rc)
+
+
+def kt_moe_balance_workspace_size(cfg: kt_moe_config, T: int) -> int:
+    return int(lib().kt_moe_balance_workspace_size(ctypes.byref(cfg), int(T)))
+
+
+def kt_moe_balance_stats(cfg, T, scores, topk_idx, alpha, f_out, P_out, loss_out, workspace,
+                         stream=None):
+    rc = lib().kt_moe_balance_stats(ctypes.byref(cfg), int(T), _ptr(scores), _ptr(topk_idx),
+                                    ctypes.c_float(alpha), _ptr(f_out), _ptr(P_out),
+                                    _ptr(loss_out), _ptr(workspace), _nbytes(workspace),
+                                    _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_balance_stats", rc)
 
 
 def kt_moe_forward(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out, workspace,

@@ -137,6 +137,48 @@ def test_gate_host_side_errors():
     assert rc == K.KT_ERR_NULL
 
 
+def test_load_statistics_host_side_errors():
+    """kt_moe_scores / kt_moe_bias_update / kt_moe_balance_stats reject bad
+    arguments on the host (fake pointers, never dereferenced)."""
+    cfg = K.config_for(W.BY_NAME["small_sig_bias"])
+    L = K.lib()
+    V = ctypes.c_void_p
+    T = 300
+    f32 = ctypes.c_float
+    # bias update: gamma must be finite and >= 0; idx and bias are required
+    for g in (float("nan"), float("inf"), -1e-3):
+        rc = L.kt_moe_bias_update(ctypes.byref(cfg), T, V(0x10000), V(0x20000), f32(g), None, None)
+        assert rc == K.KT_ERR_INVALID_CONFIG, g
+    assert L.kt_moe_bias_update(ctypes.byref(cfg), T, None, V(0x20000), f32(1e-3), None,
+                                None) == K.KT_ERR_NULL
+    assert L.kt_moe_bias_update(ctypes.byref(cfg), T, V(0x10002), V(0x20000), f32(1e-3), None,
+                                None) == K.KT_ERR_ALIGN
+    # balance statistics: workspace size, alpha, pointers
+    need = K.kt_moe_balance_workspace_size(cfg, T)
+    assert need > 0
+    bad = K.make_config(**{**{f: getattr(cfg, f) for f, _ in K.kt_moe_config._fields_}, "topk": 0})
+    assert K.kt_moe_balance_workspace_size(bad, T) == 0
+    args = [V(0x10000), V(0x20000), f32(1.0), V(0x30000), V(0x40000), V(0x50000)]
+    assert L.kt_moe_balance_stats(ctypes.byref(cfg), T, *args, V(0x7000000), need - 1,
+                                  None) == K.KT_ERR_WORKSPACE
+    a2 = list(args)
+    a2[2] = f32(float("inf"))
+    assert L.kt_moe_balance_stats(ctypes.byref(cfg), T, *a2, V(0x7000000), need,
+                                  None) == K.KT_ERR_INVALID_CONFIG
+    a2 = list(args)
+    a2[0] = None
+    assert L.kt_moe_balance_stats(ctypes.byref(cfg), T, *a2, V(0x7000000), need,
+                                  None) == K.KT_ERR_NULL
+    assert L.kt_moe_balance_stats(ctypes.byref(cfg), T, *args, V(0x7000080), need,
+                                  None) == K.KT_ERR_ALIGN
+    # scores: x required, workspace of the forward's size
+    wneed = K.kt_moe_workspace_size(cfg, T)
+    assert L.kt_moe_scores(ctypes.byref(cfg), T, None, V(0x20000), V(0x30000), V(0x7000000),
+                           wneed, None) == K.KT_ERR_NULL
+    assert L.kt_moe_scores(ctypes.byref(cfg), T, V(0x10000), V(0x20000), V(0x30000),
+                           V(0x7000000), wneed - 1, None) == K.KT_ERR_WORKSPACE
+
+
 def test_strerror_covers_codes():
     for code in range(-8, 1):
         assert K.strerror(code) and K.strerror(code) != "unknown error code"
@@ -150,7 +192,8 @@ def test_no_device_reports_cuda_error():
     buf = torch.empty(n + 256, dtype=torch.uint8)
     ws_ptr = (buf.data_ptr() + 255) // 256 * 256
     x = torch.empty(64, 256)
+    y = torch.empty(64, 256)      # its own allocation: must overlap neither x nor the workspace
     # Valid host-side arguments; the first CUDA call fails without a device.
-    ptrs = [x.data_ptr()] * 6 + [x.data_ptr() + (1 << 20)] + [0, 0]
+    ptrs = [x.data_ptr()] * 6 + [y.data_ptr()] + [0, 0]
     rc = _call_forward(cfg, 64, ptrs, ws_ptr, n)
     assert rc in (K.KT_ERR_CUDA, K.KT_ERR_UNSUPPORTED)
