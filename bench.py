@@ -192,7 +192,7 @@ def algorithmic(layer, idx: np.ndarray) -> dict:
 # ---------------------------------------------------------------------------
 # Our arm
 # ---------------------------------------------------------------------------
-def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps):
+def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
     from mixture_experts_layer_34_b200 import ktmoe as K
     inp = W.make_layer(layer, dev)
     if rank > 0:
@@ -236,6 +236,27 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps):
                 for i, name in enumerate(K.STAGES)}
     ms_max = max_over_ranks(ms, world, dev)
 
+    # The same forward replayed as one CUDA graph (kt_moe_graph_*), same buffers.
+    graph_ms = None
+    if graph:
+        gr = K.KtMoeGraph(*args)
+        for _ in range(warmup):
+            gr.launch()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record()
+        for _ in range(steps):
+            gr.launch()
+        t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        graph_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+        gr.destroy()
+        rc = K.kt_moe_check(ws)
+        if rc != K.KT_OK:
+            raise RuntimeError(f"device error in the graph launches: {K.strerror(rc)}")
+
     # End to end through the same C ABI call, host buffers: pinned x in, y out.
     x_h = inp["x"].cpu().pin_memory()
     y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
@@ -261,6 +282,7 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps):
 
     work = algorithmic(layer, idx.cpu().numpy())
     out = dict(inp=inp, idx=idx.cpu().numpy(), ms=ms_max, stage_ms=stage_ms, e2e_ms=e2e_ms,
+               graph_ms=graph_ms,
                work=work, h2d=inp["x"].numel() * inp["x"].element_size(),
                d2h=y.numel() * y.element_size())
     del ws, y
@@ -319,7 +341,7 @@ def run_ours(a):
     dec = None
     if a.decode_workload != "none":
         dlayer = W.BY_NAME[a.decode_workload]
-        dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps)
+        dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, graph=True)
     clk = clocks.stop()
 
     cpu = None
@@ -386,6 +408,10 @@ def run_ours(a):
                              "traffic": traffic("up", dl.name)},
                 "e2e": {"value": round(world * dl.T * a.e2e_steps / (dec["e2e_ms"] / 1e3), 1),
                         "unit": "tokens/s"},
+                # the same steps replayed as one CUDA graph per step (kt_moe_graph_launch)
+                "graph": {"ms_per_step": round(dec["graph_ms"] / a.steps, 4),
+                          "value": round(world * dl.T * a.steps / (dec["graph_ms"] / 1e3), 1),
+                          "unit": "tokens/s"},
             }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -192,6 +192,32 @@ int kt_moe_forward_static(const kt_moe_config* cfg, int64_t T, const void* x,
 void* kt_moe_static_scratch(void);
 
 /*
+ * The layer forward as a replayable CUDA graph, for decode steps where the
+ * launch gaps of the eight stream operations are a visible share of a step of
+ * well under a millisecond. There is no counterpart on the pages (their engine
+ * runs without graphs); this serves the calling code.
+ *
+ * kt_moe_graph_create captures one kt_moe_forward with exactly these arguments
+ * (checked on the host first; same errors) on a private stream and instantiates
+ * it. Every pointer is bound into the graph: each kt_moe_graph_launch runs the
+ * whole forward on `stream` reading x, w_gate, bias and the weights as they are
+ * then, writing y (and topk_idx_out / topk_w_out if given) and using the
+ * workspace, which must stay allocated and unshared while launches are pending.
+ * Results are bitwise those of kt_moe_forward on the same inputs.
+ * kt_moe_graph_destroy frees the graph (NULL is ignored); the caller must not
+ * destroy it while a launch is pending. The graph object and the driver's
+ * graph resources are the only things allocated; kt_moe_check(workspace,
+ * stream) reads the error word as for kt_moe_forward.
+ */
+typedef struct kt_moe_graph kt_moe_graph;
+int kt_moe_graph_create(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                        const float* bias, const void* w1, const void* w3, const void* w2,
+                        void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                        size_t ws_bytes, kt_moe_graph** graph_out);
+int kt_moe_graph_launch(kt_moe_graph* graph, void* stream);
+void kt_moe_graph_destroy(kt_moe_graph* graph);
+
+/*
  * Scores alone: s = the score function of the gate logits, gate step 1 of the
  * "Gate 选专家流程（model.py，五步）" passage of the DeepSeek-V3 model.py notes
  * (sigmoid, or softmax over all experts), for the balance statistics below or

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include "ktmoe_internal.cuh"
 
@@ -272,27 +273,48 @@ int kt_moe_forward(const kt_moe_config* cfg, int64_t T, const void* x, const voi
                                  workspace, ws_bytes, stream, nullptr);
 }
 
+}  // extern "C"
+
+namespace {
+
+// The forward's host-side checks (no CUDA call): config, NULLs, workspace size,
+// alignment, and y overlapping x or the workspace.
+int check_forward_args(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                       const float* bias, const void* w1, const void* w3, const void* w2,
+                       const void* y, const int32_t* topk_idx_out, const float* topk_w_out,
+                       const void* workspace, size_t ws_bytes, Resolved* r) {
+  int rc = resolve(cfg, T, bias != nullptr, r);
+  if (rc != KT_OK) return rc;
+  if (!x || !w_gate || !w1 || !w3 || !w2 || !y) return KT_ERR_NULL;
+  if (!workspace) return KT_ERR_WORKSPACE;
+  const Layout L = make_layout(*r, T);
+  if (ws_bytes < L.total) return KT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256) || !aligned(x, 16) || !aligned(w_gate, 16) || !aligned(w1, 16) ||
+      !aligned(w3, 16) || !aligned(w2, 16) || !aligned(y, 16) || (bias && !aligned(bias, 4)) ||
+      (topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
+    return KT_ERR_ALIGN;
+  const size_t es = r->dtype == KT_DTYPE_BF16 ? 2 : 4;
+  const size_t x_bytes = (size_t)T * r->d * es;
+  const size_t y_bytes = (size_t)T * r->d * (r->y_fp32 ? 4 : es);
+  if (overlaps(x, x_bytes, y, y_bytes) || overlaps(workspace, L.total, y, y_bytes))
+    return KT_ERR_INVALID_CONFIG;
+  return KT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
                             const void* w_gate, const float* bias, const void* w1,
                             const void* w3, const void* w2, void* y, int32_t* topk_idx_out,
                             float* topk_w_out, void* workspace, size_t ws_bytes, void* stream,
                             void* const* stage_events) {
   Resolved r;
-  int rc = resolve(cfg, T, bias != nullptr, &r);
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                              workspace, ws_bytes, &r);
   if (rc != KT_OK) return rc;
-  if (!x || !w_gate || !w1 || !w3 || !w2 || !y) return KT_ERR_NULL;
-  if (!workspace) return KT_ERR_WORKSPACE;
   const Layout L = make_layout(r, T);
-  if (ws_bytes < L.total) return KT_ERR_WORKSPACE;
-  if (!aligned(workspace, 256) || !aligned(x, 16) || !aligned(w_gate, 16) || !aligned(w1, 16) ||
-      !aligned(w3, 16) || !aligned(w2, 16) || !aligned(y, 16) || (bias && !aligned(bias, 4)) ||
-      (topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
-    return KT_ERR_ALIGN;
-  const size_t es = r.dtype == KT_DTYPE_BF16 ? 2 : 4;
-  const size_t x_bytes = (size_t)T * r.d * es;
-  const size_t y_bytes = (size_t)T * r.d * (r.y_fp32 ? 4 : es);
-  if (overlaps(x, x_bytes, y, y_bytes) || overlaps(workspace, L.total, y, y_bytes))
-    return KT_ERR_INVALID_CONFIG;
   int sms = 0;
   if ((rc = device_info(&sms)) != KT_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -376,6 +398,75 @@ int kt_moe_forward_static(const kt_moe_config* cfg, int64_t T, const void* x, co
 }
 
 void* kt_moe_static_scratch(void) { return static_scratch_ptr(); }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Graph form of the forward.
+// ---------------------------------------------------------------------------
+struct kt_moe_graph {
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+};
+
+extern "C" {
+
+int kt_moe_graph_create(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                        const float* bias, const void* w1, const void* w3, const void* w2,
+                        void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                        size_t ws_bytes, kt_moe_graph** graph_out) {
+  if (!graph_out) return KT_ERR_NULL;
+  *graph_out = nullptr;
+  Resolved r;
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                              workspace, ws_bytes, &r);
+  if (rc != KT_OK) return rc;
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  if (prepare_grouped_gemm() != cudaSuccess) return KT_ERR_CUDA;
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return KT_ERR_CUDA;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return KT_ERR_CUDA;
+  }
+  rc = kt_moe_forward_profiled(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                               workspace, ws_bytes, cs, nullptr);
+  cudaGraph_t g = nullptr;
+  const cudaError_t ec = cudaStreamEndCapture(cs, &g);
+  cudaStreamDestroy(cs);
+  if (rc != KT_OK || ec != cudaSuccess || !g) {
+    if (g) cudaGraphDestroy(g);
+    return rc != KT_OK ? rc : KT_ERR_CUDA;
+  }
+  cudaGraphExec_t ex = nullptr;
+  if (cudaGraphInstantiate(&ex, g, 0) != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return KT_ERR_CUDA;
+  }
+  kt_moe_graph* h = new (std::nothrow) kt_moe_graph{g, ex};
+  if (!h) {
+    cudaGraphExecDestroy(ex);
+    cudaGraphDestroy(g);
+    return KT_ERR_CUDA;
+  }
+  *graph_out = h;
+  return KT_OK;
+}
+
+int kt_moe_graph_launch(kt_moe_graph* graph, void* stream) {
+  if (!graph) return KT_ERR_NULL;
+  return cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KT_OK
+             : KT_ERR_CUDA;
+}
+
+void kt_moe_graph_destroy(kt_moe_graph* graph) {
+  if (!graph) return;
+  cudaGraphExecDestroy(graph->exec);
+  cudaGraphDestroy(graph->graph);
+  delete graph;
+}
 
 int kt_moe_check(const void* workspace, void* stream) {
   if (!workspace) return KT_ERR_WORKSPACE;

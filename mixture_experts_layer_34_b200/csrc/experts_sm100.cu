@@ -48,6 +48,7 @@
 // kernel records KT_ERR_TIMEOUT in the workspace error word, drains what it
 // issued, frees TMEM and returns.
 #include <cuda.h>
+#include <atomic>
 #include <cstring>
 #include <cuda_bf16.h>
 
@@ -878,10 +879,25 @@ bool make_token_maps(TmaMaps* M, int src, const void* base, uint64_t rows, uint6
   return make_map3(&M->b3[src][4], base, rows, cols, kBoxRows, kSlabsLight);
 }
 
+// The dynamic shared-memory limit of each kernel kind, raised once per device
+// (a plain host call, kept out of stream capture after the first time).
+template <int kKind>
+cudaError_t ensure_smem_attr() {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev >= 0 && dev < 64 ? 1ull << dev : 0;
+  if (bit && (done.load() & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit);
+  return e;
+}
+
 template <int kKind>
 cudaError_t launch(const TmaMaps& maps, const GemmArgs& args, int grid, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kKind>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = ensure_smem_attr<kKind>();
   if (e != cudaSuccess) return e;
   grouped_gemm_kernel<kKind><<<grid, kThreads, kSmemBytes, st>>>(maps, args);
   return cudaGetLastError();
@@ -895,6 +911,14 @@ int pair_grid(int num_sms, int max_pairs) {
 }
 
 }  // namespace
+
+cudaError_t prepare_grouped_gemm() {
+  cudaError_t e = ensure_smem_attr<kKindUp>();
+  if (e == cudaSuccess) e = ensure_smem_attr<kKindDown>();
+  if (e == cudaSuccess) e = ensure_smem_attr<kKindLogits>();
+  if (e == cudaSuccess && !get_encode_fn()) e = cudaErrorNotSupported;
+  return e;
+}
 
 cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                 const void* x, const void* wa, const void* wb, int num_sms,

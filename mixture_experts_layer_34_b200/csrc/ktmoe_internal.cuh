@@ -124,6 +124,10 @@ cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* 
 cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                 const void* x, const void* wa, const void* wb, int num_sms,
                                 cudaStream_t st, bool up);
+// Host-side setup of the grouped GEMM (shared-memory limits, the tensor-map
+// encoder), done before a stream capture so that the capture holds only
+// stream work.
+cudaError_t prepare_grouped_gemm();
 cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                const void* x, const void* w1, const void* w3, const void* w2,
                                int num_sms, cudaStream_t st, bool up);

@@ -27,7 +27,8 @@ EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_fo
            "kt_moe_forward_profiled", "kt_moe_forward_static", "kt_moe_static_scratch",
            "kt_moe_check", "kt_moe_workspace_layout", "kt_moe_strerror", "kt_moe_version",
            "kt_moe_scores", "kt_moe_bias_update", "kt_moe_balance_workspace_size",
-           "kt_moe_balance_stats")
+           "kt_moe_balance_stats", "kt_moe_graph_create", "kt_moe_graph_launch",
+           "kt_moe_graph_destroy")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -97,6 +98,13 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_balance_stats.argtypes = [CP, I64, P, P, ctypes.c_float, P, P, P, P,
                                                ctypes.c_size_t, P]
             L.kt_moe_balance_stats.restype = ctypes.c_int
+            L.kt_moe_graph_create.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P,
+                                              ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]
+            L.kt_moe_graph_create.restype = ctypes.c_int
+            L.kt_moe_graph_launch.argtypes = [P, P]
+            L.kt_moe_graph_launch.restype = ctypes.c_int
+            L.kt_moe_graph_destroy.argtypes = [P]
+            L.kt_moe_graph_destroy.restype = None
             L.kt_moe_version.argtypes = []
             L.kt_moe_version.restype = ctypes.c_int
             _lib = L
@@ -197,6 +205,42 @@ def kt_moe_forward(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_
                               _stream(stream))
     if rc != KT_OK:
         raise KtMoeError("kt_moe_forward", rc)
+
+
+class KtMoeGraph:
+    """A captured kt_moe_forward (kt_moe_graph_create); launch() replays it.
+
+    Holds references to every tensor bound into the graph so that none is freed
+    while the graph exists."""
+
+    def __init__(self, cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                 workspace):
+        self._keep = (x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out, workspace)
+        h = ctypes.c_void_p(0)
+        rc = lib().kt_moe_graph_create(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate),
+                                       _ptr(bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
+                                       _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
+                                       _nbytes(workspace), ctypes.byref(h))
+        if rc != KT_OK:
+            raise KtMoeError("kt_moe_graph_create", rc)
+        self._h = h
+
+    def launch(self, stream=None):
+        rc = lib().kt_moe_graph_launch(self._h, _stream(stream))
+        if rc != KT_OK:
+            raise KtMoeError("kt_moe_graph_launch", rc)
+
+    def destroy(self):
+        if self._h:
+            lib().kt_moe_graph_destroy(self._h)
+            self._h = ctypes.c_void_p(0)
+            self._keep = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
 
 
 KT_STAGE_EVENTS = 6

@@ -179,6 +179,29 @@ def test_load_statistics_host_side_errors():
                            V(0x7000000), wneed - 1, None) == K.KT_ERR_WORKSPACE
 
 
+def test_graph_create_host_side_errors():
+    """kt_moe_graph_create runs the forward's host checks before any CUDA call
+    and leaves the output handle NULL on failure."""
+    cfg = K.config_for(W.BY_NAME["small_sig_bias"])
+    L = K.lib()
+    V = ctypes.c_void_p
+    T = 300
+    need = K.kt_moe_workspace_size(cfg, T)
+    good = [V(0x10000 * (i + 1)) for i in range(9)]
+    h = V(0x1234)
+    rc = L.kt_moe_graph_create(ctypes.byref(cfg), T, *good, V(0x7000000), need - 1, ctypes.byref(h))
+    assert rc == K.KT_ERR_WORKSPACE and not h.value
+    p = list(good)
+    p[0] = None
+    h = V(0x1234)
+    rc = L.kt_moe_graph_create(ctypes.byref(cfg), T, *p, V(0x7000000), need, ctypes.byref(h))
+    assert rc == K.KT_ERR_NULL and not h.value
+    assert L.kt_moe_graph_create(ctypes.byref(cfg), T, *good, V(0x7000000), need,
+                                 None) == K.KT_ERR_NULL
+    assert L.kt_moe_graph_launch(None, None) == K.KT_ERR_NULL
+    L.kt_moe_graph_destroy(None)
+
+
 def test_strerror_covers_codes():
     for code in range(-8, 1):
         assert K.strerror(code) and K.strerror(code) != "unknown error code"
