@@ -359,3 +359,188 @@ int oracle_expert_hidden(const oracle_cfg* c, int64_t T, int dtype, const void* 
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// MXFP8 expert weights (the FP8 form of the layer).
+//
+// Format: MX FP8 E4M3. Blocks of 32 consecutive elements along the reduction
+// dimension (K) share one power-of-two scale 2^e, stored as an 8-bit biased
+// exponent (e + 127); each element is FP8 E4M3 (1 sign bit, 4 exponent bits
+// with bias 7, 3 mantissa bits, subnormals, no infinities, largest finite
+// value 448 = 1.75 * 2^8, code 0x7F / 0xFF is NaN). The pages name the family
+// (the DeepSeek-V3 notes' "FP8 混合精度训练" and the KTransformers page's native
+// MXFP4 routed experts) but give no quantisation rule; the rule taken here:
+//   scale : e = the smallest integer with amax <= 448 * 2^e, so that no element
+//           of the block saturates; for amax = m * 2^E with m in [1, 2) that is
+//           e = E - 8 + (m > 1.75); amax = 0 gives e = -127; e is clamped to
+//           [-127, 127];
+//   element: code = E4M3 round-to-nearest-even of v / 2^e (exact division).
+// The FP8 forward quantises each token's u (blocks of 32 along d) and each
+// SwiGLU hidden vector (blocks of 32 along I) by the same rule and runs the
+// literal loop in double on the dequantised values.
+// ===========================================================================
+namespace {
+
+uint8_t e4m3_from_double(double v) {
+  if (std::isnan(v)) return 0x7F;
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(v);
+  if (a < std::ldexp(1.0, -6)) {
+    // Subnormal range: multiples of 2^-9; 8 * 2^-9 is the smallest normal.
+    const double q = std::nearbyint(std::ldexp(a, 9));
+    return (uint8_t)(sign | (q >= 8.0 ? 0x08 : (uint8_t)q));
+  }
+  int E = 0;
+  std::frexp(a, &E);            // a = f * 2^E, f in [0.5, 1)
+  int ex = E - 1;               // a in [2^ex, 2^(ex+1))
+  double q = std::nearbyint(std::ldexp(a, 3 - ex));   // 1.mmm as an integer in [8, 16]
+  if (q == 16.0) {
+    ex += 1;
+    q = 8.0;
+  }
+  if (ex > 8 || (ex == 8 && q > 14.0)) return (uint8_t)(sign | 0x7E);   // saturate at 448
+  return (uint8_t)(sign | ((ex + 7) << 3) | ((int)q - 8));
+}
+
+double e4m3_to_double(uint8_t c) {
+  const int ex = (c >> 3) & 15, man = c & 7;
+  if (ex == 15 && man == 7) return std::numeric_limits<double>::quiet_NaN();
+  const double mag = ex == 0 ? std::ldexp((double)man, -9) : std::ldexp((double)(8 + man), ex - 10);
+  return (c & 0x80) ? -mag : mag;
+}
+
+int mx_exponent(double amax) {
+  if (!(amax > 0.0)) return -127;
+  int E = 0;
+  const double f = std::frexp(amax, &E);   // amax = (2f) * 2^(E-1), 2f in [1, 2)
+  int e = (E - 1) - 8 + (2.0 * f > 1.75 ? 1 : 0);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// One row of K values (K a multiple of 32) to codes and biased scale bytes.
+void mx_quantize_row(const double* v, int64_t K, uint8_t* codes, uint8_t* scales) {
+  for (int64_t b = 0; b < K / 32; ++b) {
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i) amax = std::max(amax, std::fabs(v[b * 32 + i]));
+    const int e = mx_exponent(amax);
+    scales[b] = (uint8_t)(e + 127);
+    for (int i = 0; i < 32; ++i) codes[b * 32 + i] = e4m3_from_double(std::ldexp(v[b * 32 + i], -e));
+  }
+}
+
+double mx_value(const uint8_t* codes, const uint8_t* scales, int64_t i) {
+  return std::ldexp(e4m3_to_double(codes[i]), (int)scales[i / 32] - 127);
+}
+
+double load_any(const void* src, int dtype, int64_t i) {
+  if (dtype == 2) return ((const double*)src)[i];
+  return load_elem(src, dtype, i);
+}
+
+}  // namespace
+
+extern "C" {
+
+// E4M3 round-to-nearest-even of n doubles (saturating at +-448) and back.
+int oracle_e4m3_encode(int64_t n, const double* v, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_from_double(v[i]);
+  return 0;
+}
+int oracle_e4m3_decode(int64_t n, const uint8_t* c, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_double(c[i]);
+  return 0;
+}
+
+// MX quantisation of a row-major [rows, K] matrix (K a multiple of 32) held as
+// fp32 (dtype 0), bf16 (1) or double (2): codes [rows, K], scales [rows, K/32]
+// (biased exponents). Returns -1 if K is not a multiple of 32.
+int oracle_mx_quantize(int64_t rows, int64_t K, int dtype, const void* src, uint8_t* codes,
+                       uint8_t* scales) {
+  if (K % 32 != 0) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    std::vector<double> v(K);
+    for (int64_t i = 0; i < K; ++i) v[i] = load_any(src, dtype, r * K + i);
+    mx_quantize_row(v.data(), K, codes + r * K, scales + r * (K / 32));
+  }
+  return 0;
+}
+
+// codes * 2^(scale - 127), double [rows, K].
+int oracle_mx_dequantize(int64_t rows, int64_t K, const uint8_t* codes, const uint8_t* scales,
+                         double* out) {
+  if (K % 32 != 0) return -1;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t i = 0; i < K; ++i) out[r * K + i] = mx_value(codes + r * K, scales + r * (K / 32), i);
+  return 0;
+}
+
+// The literal forward ("MoE 前向四步") with MXFP8 expert weights: per token, u
+// is quantised (blocks of 32 along d); every expert computes, in double on the
+// dequantised values, h = silu(W1 u) * W3 u, quantises h (blocks of 32 along I;
+// skipped if quantize_hidden == 0) and returns W2 h. x is bf16 [T, d]. w1q/w3q
+// are per-expert code arrays [I, d] with scales [I, d/32]; w2q codes [d, I]
+// with scales [d, I/32]; E+S entries each (NULL where unused). y [n_tok, d].
+int oracle_forward_mxfp8(const oracle_cfg* c, int64_t T, const void* x, const int32_t* idx,
+                         const float* w, const uint8_t* const* w1q, const uint8_t* const* w1s,
+                         const uint8_t* const* w3q, const uint8_t* const* w3s,
+                         const uint8_t* const* w2q, const uint8_t* const* w2s,
+                         int quantize_hidden, int64_t n_tok, const int64_t* tok_ids, double* y) {
+  const int d = c->dim, I = c->inter, k = c->topk, E = c->n_experts, S = c->n_shared;
+  if (d % 32 != 0 || I % 32 != 0) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t n = 0; n < n_tok; ++n) {
+    const int64_t t = tok_ids[n];
+    if (t < 0 || t >= T) {
+      bad |= 1;
+      continue;
+    }
+    std::vector<double> u(d), uq(d), acc(d, 0.0), h(I), hq(I);
+    std::vector<uint8_t> cu(d), su(d / 32), ch(I), sh(I / 32);
+    for (int i = 0; i < d; ++i) u[i] = load_elem(x, 1, t * d + i);
+    mx_quantize_row(u.data(), d, cu.data(), su.data());
+    for (int i = 0; i < d; ++i) uq[i] = mx_value(cu.data(), su.data(), i);
+    auto run_expert = [&](int e, double weight) {
+      if (!w1q[e] || !w1s[e] || !w3q[e] || !w3s[e] || !w2q[e] || !w2s[e]) {
+        bad |= 1;
+        return;
+      }
+      for (int f = 0; f < I; ++f) {
+        double g = 0.0, v = 0.0;
+        for (int i = 0; i < d; ++i) {
+          const int64_t j = (int64_t)f * d + i;
+          g += mx_value(w1q[e], w1s[e], j) * uq[i];
+          v += mx_value(w3q[e], w3s[e], j) * uq[i];
+        }
+        h[f] = g / (1.0 + std::exp(-g)) * v;
+      }
+      if (quantize_hidden) {
+        mx_quantize_row(h.data(), I, ch.data(), sh.data());
+        for (int f = 0; f < I; ++f) hq[f] = mx_value(ch.data(), sh.data(), f);
+      } else {
+        hq = h;
+      }
+      for (int o = 0; o < d; ++o) {
+        double s = 0.0;
+        for (int f = 0; f < I; ++f) s += mx_value(w2q[e], w2s[e], (int64_t)o * I + f) * hq[f];
+        acc[o] += weight * s;
+      }
+    };
+    for (int s = 0; s < S; ++s) run_expert(E + s, 1.0);
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[t * k + j];
+      if (e < 0 || e >= E) {
+        bad |= 1;
+        continue;
+      }
+      run_expert(e, (double)w[t * k + j]);
+    }
+    if (c->add_residual)
+      for (int i = 0; i < d; ++i) acc[i] += u[i];
+    std::copy(acc.begin(), acc.end(), y + n * d);
+  }
+  return bad ? -1 : 0;
+}
+
+}  // extern "C"

@@ -64,6 +64,12 @@ def _load():
             lib.oracle_expert_load.argtypes = [CP, I64, P, P]
             lib.oracle_bias_update.argtypes = [CP, I64, P, ctypes.c_float, P]
             lib.oracle_balance_stats.argtypes = [CP, I64, P, P, ctypes.c_double, P, P, P]
+            lib.oracle_e4m3_encode.argtypes = [I64, P, P]
+            lib.oracle_e4m3_decode.argtypes = [I64, P, P]
+            lib.oracle_mx_quantize.argtypes = [I64, I64, ctypes.c_int, P, P, P]
+            lib.oracle_mx_dequantize.argtypes = [I64, I64, P, P, P]
+            lib.oracle_forward_mxfp8.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                                 I64, P, P]
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -258,3 +264,81 @@ def balance_stats(cfg: dict, s: np.ndarray, idx: np.ndarray, alpha: float) -> di
                                     ctypes.c_double(alpha), _ptr(f), _ptr(P), _ptr(loss)) != 0:
         raise ValueError("oracle_balance_stats: expert index out of range")
     return dict(f=f, P=P, loss=float(loss[0]))
+
+
+# ----------------------------------------------------------------------------
+# MXFP8 (E4M3 elements, one power-of-two scale per 32 along K)
+# ----------------------------------------------------------------------------
+def e4m3_encode(v) -> np.ndarray:
+    """E4M3 codes (uint8) of float64 values, round to nearest even, saturating at 448."""
+    v = np.ascontiguousarray(np.asarray(v, np.float64))
+    out = np.empty(v.shape, np.uint8)
+    _load().oracle_e4m3_encode(v.size, _ptr(v), _ptr(out))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(c, np.uint8))
+    out = np.empty(c.shape, np.float64)
+    _load().oracle_e4m3_decode(c.size, _ptr(c), _ptr(out))
+    return out
+
+
+def mx_quantize(a) -> tuple[np.ndarray, np.ndarray]:
+    """[rows, K] (fp32, bf16 tensor or float64) -> (codes [rows, K] uint8,
+    biased scale exponents [rows, K/32] uint8)."""
+    if isinstance(a, np.ndarray) and a.dtype == np.float64:
+        raw, dt = np.ascontiguousarray(a), 2
+    else:
+        raw, dt = _as_raw(a)
+    rows, K = raw.shape
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, K // 32), np.uint8)
+    if _load().oracle_mx_quantize(rows, K, dt, _ptr(raw), _ptr(codes), _ptr(scales)) != 0:
+        raise ValueError("mx_quantize: K must be a multiple of 32")
+    return codes, scales
+
+
+def mx_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, K = codes.shape
+    out = np.empty((rows, K), np.float64)
+    _load().oracle_mx_dequantize(rows, K, _ptr(codes), _ptr(scales), _ptr(out))
+    return out
+
+
+def forward_mxfp8(cfg: dict, x, idx, w, w1, w3, w2, tok_ids, has_bias: bool,
+                  quantize_hidden: bool = True) -> np.ndarray:
+    """The literal loop with MXFP8 expert weights. w1/w3/w2: sequences of E+S
+    (codes, scales) pairs (None where unused); x bf16 [T, d]. Returns y [n, d]."""
+    xa, dt = _as_raw(x)
+    assert dt == 1, "the FP8 form takes bf16 tokens"
+    T = xa.shape[0]
+    rc = resolve(cfg, has_bias)
+    n_all = rc["n_experts"] + rc["n_shared"]
+    keep = []
+
+    def ptrs(ws, part):
+        arr = (ctypes.c_void_p * n_all)()
+        for e in range(n_all):
+            if ws[e] is None:
+                arr[e] = None
+                continue
+            a = np.ascontiguousarray(ws[e][part], np.uint8)
+            keep.append(a)
+            arr[e] = a.ctypes.data
+        return arr
+
+    tok = np.ascontiguousarray(np.asarray(tok_ids, np.int64))
+    y = np.empty((tok.shape[0], rc["dim"]), np.float64)
+    idx = np.ascontiguousarray(idx, np.int32)
+    w = np.ascontiguousarray(w, np.float32)
+    c = _cfg_struct(rc)
+    code = _load().oracle_forward_mxfp8(
+        ctypes.byref(c), T, _ptr(xa), _ptr(idx), _ptr(w), ptrs(w1, 0), ptrs(w1, 1), ptrs(w3, 0),
+        ptrs(w3, 1), ptrs(w2, 0), ptrs(w2, 1), int(bool(quantize_hidden)), tok.shape[0], _ptr(tok),
+        _ptr(y))
+    if code != 0:
+        raise ValueError("oracle_forward_mxfp8: bad token id, missing weights or dims not multiples of 32")
+    return y
