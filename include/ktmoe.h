@@ -49,8 +49,9 @@ extern "C" {
 enum { KT_SCORE_SIGMOID = 0, KT_SCORE_SOFTMAX = 1 };
 /* Group score of gate step 2. AUTO = TOP2SUM when a bias is given, else AMAX. */
 enum { KT_GROUP_AUTO = 0, KT_GROUP_AMAX = 1, KT_GROUP_TOP2SUM = 2 };
-/* Activation / expert-weight dtype. */
-enum { KT_DTYPE_F32 = 0, KT_DTYPE_BF16 = 1 };
+/* Activation / expert-weight dtype. KT_DTYPE_MXFP8: bf16 tokens, gate weights
+ * and output (as KT_DTYPE_BF16); expert weights in MXFP8 (kt_moe_forward_mxfp8). */
+enum { KT_DTYPE_F32 = 0, KT_DTYPE_BF16 = 1, KT_DTYPE_MXFP8 = 2 };
 
 enum {
   KT_OK = 0,
@@ -74,7 +75,8 @@ enum {
  * 1 <= topk <= min(32, topk_groups * n_experts / n_groups); n_groups == 1
  * implies topk_groups == 1; TOP2SUM needs >= 2 experts per group;
  * 0 <= n_shared <= 8; route_scale finite and > 0; dim, inter >= 8 and
- * multiples of 8 (bf16) or 4 (fp32), so rows are 16-byte multiples.
+ * multiples of 8 (bf16) or 4 (fp32), so rows are 16-byte multiples; for
+ * KT_DTYPE_MXFP8 multiples of 128 (one 128-byte K slab of FP8).
  */
 typedef struct {
   int32_t n_experts;    /* E: routed experts                                      */
@@ -218,6 +220,58 @@ int kt_moe_graph_launch(kt_moe_graph* graph, void* stream);
 void kt_moe_graph_destroy(kt_moe_graph* graph);
 
 /*
+ * MXFP8 expert weights: the FP8 form of the layer (cfg->dtype = KT_DTYPE_MXFP8).
+ * The pages name the format family (the DeepSeek-V3 notes' FP8 mixed precision,
+ * the KTransformers page's native MXFP4 routed experts) but no rule. Format:
+ * E4M3 elements (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest
+ * finite 448), one power-of-two scale 2^e per 32 consecutive elements along K,
+ * stored as the byte e + 127. Rule: e is the smallest integer with
+ * amax <= 448 * 2^e (amax = the block's largest magnitude; 0 gives e = -127),
+ * each element the E4M3 round-to-nearest-even of v * 2^-e.
+ *
+ * kt_moe_mxfp8_quantize: row-major [rows, K] bf16 (K % 32 == 0) -> codes
+ *   [rows, K] and scale bytes [rows, K/32], row-major; device pointers, 16-B
+ *   aligned src and codes.
+ *
+ * kt_moe_mxfp8_pack: stacked bf16 expert weights (w1, w3 [E+S, inter, dim],
+ *   w2 [E+S, dim, inter]) -> codes in the same layout (w1q, w3q, w2q, one byte
+ *   each) and the scales packed as the grouped GEMM reads them:
+ *   sf_up   (kt_moe_mxfp8_scale_bytes(cfg, 0) bytes): a 512-byte block per
+ *           (group g, feature tile ft of 128, half h, K slab s of 128 along dim)
+ *           at block index ((g * inter/128 + ft) * 2 + h) * dim/128 + s; in it
+ *           the scale of tile row m (m < 64: W1 row 128 ft + 64 h + m; m >= 64:
+ *           W3 row 128 ft + 64 h + m - 64) and K block 4 s + k1 sits at byte
+ *           16 * (m % 32) + 4 * (m / 32) + k1;
+ *   sf_down (kt_moe_mxfp8_scale_bytes(cfg, 1) bytes): the same for W2 with
+ *           feature tiles of 256 output rows (nft = ceil(dim/256)) and K slabs
+ *           along inter: block ((g * nft + ft) * 2 + h) * inter/128 + s, tile row
+ *           m = W2 row 256 ft + 128 h + m (rows past dim hold 0).
+ *   dim and inter must be multiples of 128.
+ *
+ * kt_moe_forward_mxfp8: the layer forward with packed MXFP8 weights. x, w_gate,
+ *   bias, y, topk outputs, workspace (kt_moe_workspace_size with the MXFP8
+ *   config) and errors as for kt_moe_forward; w3q must lie above w1q in memory
+ *   (e.g. the two halves of one [2, E+S, inter, dim] buffer: the kernel reads
+ *   the codes of both in one box, in address order, and the packed scales list
+ *   W1 first), else KT_ERR_INVALID_CONFIG; stage_events as for
+ *   kt_moe_forward_profiled (NULL for none). The gate runs in bf16 / fp32 as in
+ *   the bf16 form; the tokens and the SwiGLU hidden rows are quantised to MXFP8
+ *   by the rule above; the expert GEMMs accumulate in fp32 on the tensor cores
+ *   (block-scaled E4M3); the output sum is the fixed-order fp32 combine.
+ */
+int kt_moe_mxfp8_quantize(int64_t rows, int64_t K, const void* src, uint8_t* codes,
+                          uint8_t* scales, void* stream);
+size_t kt_moe_mxfp8_scale_bytes(const kt_moe_config* cfg, int down);
+int kt_moe_mxfp8_pack(const kt_moe_config* cfg, const void* w1, const void* w3, const void* w2,
+                      uint8_t* w1q, uint8_t* w3q, uint8_t* w2q, uint8_t* sf_up, uint8_t* sf_down,
+                      void* stream);
+int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                         const float* bias, const uint8_t* w1q, const uint8_t* w3q,
+                         const uint8_t* w2q, const uint8_t* sf_up, const uint8_t* sf_down,
+                         void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                         size_t ws_bytes, void* stream, void* const* stage_events);
+
+/*
  * Scores alone: s = the score function of the gate logits, gate step 1 of the
  * "Gate 选专家流程（model.py，五步）" passage of the DeepSeek-V3 model.py notes
  * (sigmoid, or softmax over all experts), for the balance statistics below or
@@ -303,6 +357,17 @@ typedef struct {
   int64_t tiles_up;
   int64_t tiles_down;
   int64_t total;
+  /* MXFP8 layers (else -1): xq, xs = E4M3 codes [T, dim] and scale bytes
+   * [T, dim/32] of x; xperm = codes of the permuted routed rows [T*k, dim];
+   * tok_sf / hid_sf = the scales of each GEMM chunk's token / hidden rows,
+   * [chunk][K/128][1024 B] (two 512-byte halves of 128 rows, scale of row m and
+   * K block b at 512 (m / 128) + 16 (m % 32) + 4 (m / 32 % 4) + b % 4); hidden
+   * holds E4M3 codes; chunks have at most 224 rows. */
+  int64_t xq;
+  int64_t xs;
+  int64_t xperm;
+  int64_t tok_sf;
+  int64_t hid_sf;
 } kt_moe_ws_layout;
 
 int kt_moe_workspace_layout(const kt_moe_config* cfg, int64_t T, kt_moe_ws_layout* out);

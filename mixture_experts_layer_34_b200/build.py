@@ -24,7 +24,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libktmoe.so")
 
 SOURCES = ["api.cu", "gate.cu", "permute.cu", "experts_sm100.cu", "experts_f32.cu", "combine.cu",
-           "balance.cu"]
+           "balance.cu", "mxfp8.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

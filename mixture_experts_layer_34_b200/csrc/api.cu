@@ -56,8 +56,9 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
   if (!std::isfinite(c->route_scale) || !(c->route_scale > 0.f)) return KT_ERR_INVALID_CONFIG;
   if (c->score_func != KT_SCORE_SIGMOID && c->score_func != KT_SCORE_SOFTMAX)
     return KT_ERR_INVALID_CONFIG;
-  if (c->dtype != KT_DTYPE_F32 && c->dtype != KT_DTYPE_BF16) return KT_ERR_INVALID_CONFIG;
-  const int align = c->dtype == KT_DTYPE_BF16 ? 8 : 4;
+  if (c->dtype != KT_DTYPE_F32 && c->dtype != KT_DTYPE_BF16 && c->dtype != KT_DTYPE_MXFP8)
+    return KT_ERR_INVALID_CONFIG;
+  const int align = c->dtype == KT_DTYPE_MXFP8 ? 128 : (c->dtype == KT_DTYPE_BF16 ? 8 : 4);
   if (c->dim < 8 || c->inter < 8 || c->dim % align || c->inter % align) return KT_ERR_INVALID_CONFIG;
   if (c->dim > (1 << 16) || c->inter > (1 << 16)) return KT_ERR_INVALID_CONFIG;
   if (c->norm_topk < -1 || c->norm_topk > 1) return KT_ERR_INVALID_CONFIG;
@@ -79,6 +80,9 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
                                                    : c->group_score;
   if (G > 1 && r->group_score == KT_GROUP_TOP2SUM && gs < 2) return KT_ERR_INVALID_CONFIG;
   r->dtype = c->dtype;
+  r->act_bf16 = c->dtype != KT_DTYPE_F32;
+  r->fp8 = c->dtype == KT_DTYPE_MXFP8;
+  r->chunk_rows = r->fp8 ? kChunkRowsF8 : kChunkRows;
   r->add_residual = c->add_residual;
   r->y_fp32 = c->dtype == KT_DTYPE_F32 ? 1 : c->y_fp32;
   r->has_bias = has_bias ? 1 : 0;
@@ -97,9 +101,10 @@ Layout make_layout(const Resolved& r, int64_t T) {
   const size_t NG = (size_t)(r.E + r.S);
   const size_t Tk = (size_t)T * r.k;
   const size_t R = (size_t)T * (r.k + r.S);
-  const size_t es = r.dtype == KT_DTYPE_BF16 ? 2 : 4;
+  const size_t es = r.act_bf16 ? 2 : 4;          // token / output element bytes
+  const size_t hs = r.fp8 ? 1 : es;              // hidden-row element bytes
   L.nperm = (T + kPermChunk - 1) / kPermChunk;
-  L.max_chunks = (int64_t)(R / kChunkRows + NG + 1);
+  L.max_chunks = (int64_t)(R / r.chunk_rows + NG + 1);
   L.err = take(256, 256);
   L.meta = take(64, 256);
   L.logits = take((size_t)gate_logit_splits(r, T) * T * r.E * 4, 256);
@@ -115,8 +120,14 @@ Layout make_layout(const Resolved& r, int64_t T) {
   L.chunks = take((size_t)L.max_chunks * sizeof(Chunk), 256);
   L.tiles_up = take((size_t)L.max_chunks * ((r.I + 127) / 128) * 8, 256);
   L.tiles_down = take((size_t)L.max_chunks * ((r.d + 255) / 256) * 8, 256);
-  L.xperm = take(r.dtype == KT_DTYPE_BF16 ? Tk * r.d * es : 0, 1024);
-  L.hidden = take(R * r.I * es, 1024);
+  L.xperm = take(r.dtype == KT_DTYPE_BF16 ? Tk * r.d * es : (r.fp8 ? Tk * r.d : 0), 1024);
+  L.hidden = take(R * r.I * hs, 1024);
+  const size_t fp8 = r.fp8 ? 1 : 0;
+  L.xq = take(fp8 * (size_t)T * r.d, 1024);
+  L.xs = take(fp8 * (size_t)T * (r.d / 32), 256);
+  L.tok_sf = take(fp8 * (size_t)L.max_chunks * (r.d / 128) * 1024, 1024);
+  L.hid_sf = take(fp8 * (size_t)L.max_chunks * (r.I / 128) * 1024, 1024);
+  L.gchunk0 = take(NG * 4, 256);
   L.expert_out = take(R * r.d * 4, 1024);   // fp32 for every dtype
   L.total = round_up(off, 1024);
   return L;
@@ -163,6 +174,11 @@ int kt_moe_workspace_layout(const kt_moe_config* cfg, int64_t T, kt_moe_ws_layou
   out->tiles_up = (int64_t)L.tiles_up;
   out->tiles_down = (int64_t)L.tiles_down;
   out->total = (int64_t)L.total;
+  out->xq = r.fp8 ? (int64_t)L.xq : -1;
+  out->xs = r.fp8 ? (int64_t)L.xs : -1;
+  out->xperm = r.fp8 ? (int64_t)L.xperm : -1;
+  out->tok_sf = r.fp8 ? (int64_t)L.tok_sf : -1;
+  out->hid_sf = r.fp8 ? (int64_t)L.hid_sf : -1;
   return KT_OK;
 }
 
@@ -293,7 +309,7 @@ int check_forward_args(const kt_moe_config* cfg, int64_t T, const void* x, const
       !aligned(w3, 16) || !aligned(w2, 16) || !aligned(y, 16) || (bias && !aligned(bias, 4)) ||
       (topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
     return KT_ERR_ALIGN;
-  const size_t es = r->dtype == KT_DTYPE_BF16 ? 2 : 4;
+  const size_t es = r->act_bf16 ? 2 : 4;
   const size_t x_bytes = (size_t)T * r->d * es;
   const size_t y_bytes = (size_t)T * r->d * (r->y_fp32 ? 4 : es);
   if (overlaps(x, x_bytes, y, y_bytes) || overlaps(workspace, L.total, y, y_bytes))
@@ -314,6 +330,7 @@ int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
   int rc = check_forward_args(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
                               workspace, ws_bytes, &r);
   if (rc != KT_OK) return rc;
+  if (r.fp8) return KT_ERR_INVALID_CONFIG;   // MXFP8 weights: kt_moe_forward_mxfp8
   const Layout L = make_layout(r, T);
   int sms = 0;
   if ((rc = device_info(&sms)) != KT_OK) return rc;
@@ -395,6 +412,100 @@ int kt_moe_forward_static(const kt_moe_config* cfg, int64_t T, const void* x, co
   // forward; nothing else in the scratch is read before it is written.
   return kt_moe_forward_profiled(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
                                  scratch, KT_STATIC_SCRATCH_BYTES, stream, nullptr);
+}
+
+int kt_moe_mxfp8_quantize(int64_t rows, int64_t K, const void* src, uint8_t* codes,
+                          uint8_t* scales, void* stream) {
+  if (rows < 0 || K <= 0 || K % 32 != 0) return KT_ERR_INVALID_CONFIG;
+  if (!src || !codes || !scales) return KT_ERR_NULL;
+  if (!aligned(src, 16) || !aligned(codes, 16)) return KT_ERR_ALIGN;
+  int sms = 0;
+  const int rc = device_info(&sms);
+  if (rc != KT_OK) return rc;
+  return launch_mx_quantize(src, rows, K, codes, scales, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? KT_OK
+             : KT_ERR_CUDA;
+}
+
+size_t kt_moe_mxfp8_scale_bytes(const kt_moe_config* cfg, int down) {
+  Resolved r;
+  if (resolve(cfg, 1, 0, &r) != KT_OK || !r.fp8) return 0;
+  return mx_packed_bytes(r, down != 0);
+}
+
+int kt_moe_mxfp8_pack(const kt_moe_config* cfg, const void* w1, const void* w3, const void* w2,
+                      uint8_t* w1q, uint8_t* w3q, uint8_t* w2q, uint8_t* sf_up, uint8_t* sf_down,
+                      void* stream) {
+  Resolved r;
+  int rc = resolve(cfg, 1, 0, &r);
+  if (rc != KT_OK) return rc;
+  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
+  if (!w1 || !w3 || !w2 || !w1q || !w3q || !w2q || !sf_up || !sf_down) return KT_ERR_NULL;
+  if (!aligned(w1, 16) || !aligned(w3, 16) || !aligned(w2, 16) || !aligned(w1q, 16) ||
+      !aligned(w3q, 16) || !aligned(w2q, 16) || !aligned(sf_up, 16) || !aligned(sf_down, 16))
+    return KT_ERR_ALIGN;
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  return launch_mx_pack(r, w1, w3, w2, w1q, w3q, w2q, sf_up, sf_down,
+                        static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KT_OK
+             : KT_ERR_CUDA;
+}
+
+int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                         const float* bias, const uint8_t* w1q, const uint8_t* w3q,
+                         const uint8_t* w2q, const uint8_t* sf_up, const uint8_t* sf_down,
+                         void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                         size_t ws_bytes, void* stream, void* const* stage_events) {
+  Resolved r;
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y, topk_idx_out,
+                              topk_w_out, workspace, ws_bytes, &r);
+  if (rc != KT_OK) return rc;
+  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
+  if (!sf_up || !sf_down) return KT_ERR_NULL;
+  // The packed gate/up scales list W1's rows before W3's; the kernel loads the
+  // codes of both in one box in address order, so W1's must come first.
+  if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
+    return KT_ERR_INVALID_CONFIG;
+  if (!aligned(sf_up, 16) || !aligned(sf_down, 16)) return KT_ERR_ALIGN;
+  const Layout L = make_layout(r, T);
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(ws + L.w);
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+  auto mark = [&](int i) {
+    if (stage_events && stage_events[i])
+      return cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st) == cudaSuccess;
+    return true;
+  };
+  if (!mark(0)) return KT_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_gate_select(r, T, logits, nullptr, bias, idx, w,
+                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), st) != cudaSuccess)
+    return KT_ERR_CUDA;
+  if (!mark(1)) return KT_ERR_CUDA;
+  // Tokens to MXFP8 (codes and scales of x), then the permutation, which copies
+  // the codes into expert order and the scales into each GEMM chunk's blocks.
+  if (launch_mx_quantize(x, T, r.d, reinterpret_cast<uint8_t*>(ws + L.xq),
+                         reinterpret_cast<uint8_t*>(ws + L.xs), st) != cudaSuccess)
+    return KT_ERR_CUDA;
+  if (launch_permute(r, T, L, ws, idx, w, x, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (!mark(2)) return KT_ERR_CUDA;
+  if (launch_experts_mxfp8(r, T, L, ws, w1q, w3q, sf_up, sms, st, true) != cudaSuccess ||
+      !mark(3))
+    return KT_ERR_CUDA;
+  if (launch_experts_mxfp8(r, T, L, ws, w2q, nullptr, sf_down, sms, st, false) != cudaSuccess ||
+      !mark(4))
+    return KT_ERR_CUDA;
+  if (launch_combine(r, T, L, ws, x, y, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (!mark(5)) return KT_ERR_CUDA;
+  return KT_OK;
 }
 
 void* kt_moe_static_scratch(void) { return static_scratch_ptr(); }

@@ -86,10 +86,10 @@ cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* 
                            void* y, cudaStream_t st) {
   const int32_t* row_of = reinterpret_cast<const int32_t*>(ws + L.row_of);
   const float* eo = reinterpret_cast<const float*>(ws + L.expert_out);
-  if (r.dtype == KT_DTYPE_BF16 && !r.y_fp32)
+  if (r.act_bf16 && !r.y_fp32)
     combine_kernel<true, false><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
                                                              row_of, eo, x, y);
-  else if (r.dtype == KT_DTYPE_BF16)
+  else if (r.act_bf16)
     combine_kernel<true, true><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
                                                             row_of, eo, x, y);
   else

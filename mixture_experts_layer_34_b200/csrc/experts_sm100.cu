@@ -88,8 +88,15 @@ constexpr int kSlabsLight = 3;
 static_assert(kSlabsLight * (kATileBytes + kBoxBytes) <= kStageBytes, "3-slab stage layout");
 static_assert(kSlabs * (kATileBytes + kBTileBytes) <= kStageBytes, "2-slab stage layout");
 __device__ __forceinline__ int stage_slabs(int hb) { return hb == 1 ? kSlabsLight : kSlabs; }
-constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + kXchgBytes + kCtrlBytes + 1024;
-constexpr int kAccCols = 256;                    // TMEM columns per accumulator buffer
+// MXFP8 kinds: the block scales of each stage's slabs (per slab: 512 B for the
+// CTA's 128 weight rows, 1 KB for the pair tile's up to 256 token rows).
+constexpr int kSfaSlabBytes = 512, kSfbSlabBytes = 1024;
+constexpr int kScaleStageBytes = kSlabsLight * (kSfaSlabBytes + kSfbSlabBytes);
+constexpr int kSmemBase = kStages * kStageBytes + kStagingBytes + kXchgBytes + kCtrlBytes + 1024;
+constexpr int kAccColsF8 = kChunkRowsF8;         // MXFP8 accumulator buffers (2 x 224 columns)
+constexpr int kSfaCol = 2 * kAccColsF8;          // TMEM columns of the A scales (4)
+constexpr int kSfbCol = kSfaCol + 4;             // and of the B scales (8)
+static_assert(kSfbCol + 8 <= 512, "MXFP8 TMEM budget");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kSched = 4;                        // tile schedule ring slots
 // Consumers of a schedule slot: the MMA thread and 4 epilogue warps of the even
@@ -100,12 +107,18 @@ constexpr int kSchedConsumers = 10;
 constexpr int kKindUp = 0;      // hidden = silu(W1 u) * W3 u            (bf16 out)
 constexpr int kKindDown = 1;    // expert_out = w_r * W2 h               (fp32 out)
 constexpr int kKindLogits = 2;  // logits = W_g u, implicit token chunks (fp32 out)
+constexpr int kKindUpF8 = 3;    // MXFP8 weights and tokens: hidden as MXFP8 codes + scales
+constexpr int kKindDownF8 = 4;  // MXFP8 weights and hidden rows: expert_out (fp32 out)
 
 template <int kKind>
 struct Kind {
-  static constexpr bool kUp = kKind == kKindUp;
-  static constexpr int kOutBytes = kUp ? 2 : 4;
+  static constexpr bool kF8 = kKind == kKindUpF8 || kKind == kKindDownF8;
+  static constexpr bool kUp = kKind == kKindUp || kKind == kKindUpF8;
+  static constexpr int kOutBytes = kKind == kKindUpF8 ? 1 : (kUp ? 2 : 4);
   static constexpr int kRowsPerPair = kUp ? 128 : 256;   // output features per pair tile
+  static constexpr int kSlabK = kF8 ? 128 : kBK;         // K elements per 128-byte slab
+  static constexpr int kAccCols = kF8 ? kAccColsF8 : 256;  // TMEM columns per accumulator
+  static constexpr int kSmem = kSmemBase + (kF8 ? kStages * kScaleStageBytes : 0);
 };
 
 struct GemmArgs {
@@ -128,6 +141,10 @@ struct GemmArgs {
   int tma3d;                 // 1: one box per stage from the 3-D/4-D maps (K % 64 == 0)
   int gate_hi;               // up, 3-D maps: W3 precedes W1 in memory, so the upper 64
                              // rows of each CTA's weight tile are W1 (gate)
+  // MXFP8 kinds:
+  int n_kslabs;              // K / 128
+  int n_ftiles_sf;           // feature tiles per group in the packed weight scales
+  uint8_t* hid_sf;           // up: hidden-row scale blocks [chunk][I / 128][1 KB]
 };
 
 // Tensor maps of one launch (bf16, 128-byte swizzle). Token-row sources: up: 0
@@ -142,6 +159,10 @@ struct TmaMaps {
   CUtensorMap b2[2][2];   // [source][32-row box, 128-row box], one slab
   CUtensorMap a3[2];      // weights of a [2-slab, 3-slab] stage
   CUtensorMap b3[2][5];   // [source][2-slab stage of 32/64/96/128 rows, 3-slab stage of 32]
+  // MXFP8 kinds: the packed weight scales and the token chunks' scales, as
+  // rows of 256 bytes; boxes of [2-slab, 3-slab] stages.
+  CUtensorMap sfa[2];
+  CUtensorMap sfb[2];
 };
 
 // ---------------------------------------------------------------------------
@@ -292,6 +313,41 @@ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
+// MXFP8: E4M3 A and B, E8M0 block scales (one per 32 along K) read from TMEM;
+// the scale byte used by this K = 32 MMA is selected by sf_id (bits 29-30 for A,
+// 4-5 for B). Accumulation is fp32.
+__device__ __forceinline__ uint32_t idesc_mxf8(int M, int N, int sf_id) {
+  return (static_cast<uint32_t>(sf_id) << 4) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) |
+         (static_cast<uint32_t>(sf_id) << 29);
+}
+__device__ __forceinline__ void mma_pair_mxf8(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                              uint32_t idesc, uint32_t sfa_tmem,
+                                              uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// Shared-memory descriptor of a block of 32 rows x 16 bytes (no swizzle,
+// K-major, 8-row core matrices 128 bytes apart), the source of a scale copy.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;      // LBO
+  d |= static_cast<uint64_t>(128u >> 4) << 32;      // SBO
+  d |= static_cast<uint64_t>(1u) << 46;             // version
+  return d;
+}
+// 512 bytes of block scales (128 rows x 4 K blocks) into 4 TMEM columns of all
+// 128 lanes of both CTAs of the pair, each from its own shared memory.
+__device__ __forceinline__ void sf_copy_pair(uint32_t tmem_col, uint32_t saddr) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(tmem_col),
+               "l"(sf_desc(saddr))
+               : "memory");
+}
 __device__ __forceinline__ void mma_pair_bf16(uint32_t d_tmem, uint64_t a, uint64_t b,
                                               uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -340,10 +396,11 @@ __device__ __forceinline__ void st_cluster_s32(uint32_t caddr, int v) {
   asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void read_slot(const int* slot, Chunk& ch, int& ft) {
+__device__ __forceinline__ void read_slot(const int* slot, Chunk& ch, int& ft, int& ci) {
   const volatile int* v = slot;
   ch = Chunk{v[0], v[1], v[2], v[3]};
   ft = v[4];
+  ci = v[5];
 }
 
 // True iff `v` holds on every thread that continues together: the warp, or the
@@ -365,14 +422,15 @@ __device__ __forceinline__ bool uniform_ok(bool v, int bar_id) {
   return __all_sync(0xffffffffu, v);
 }
 
-__device__ __forceinline__ void get_tile(const GemmArgs& a, int t, Chunk& ch, int& ft) {
+__device__ __forceinline__ void get_tile(const GemmArgs& a, int t, Chunk& ch, int& ft, int& ci) {
   if (a.implicit_rows > 0) {
-    const int ci = t / a.n_ftiles;
+    ci = t / a.n_ftiles;
     ft = t % a.n_ftiles;
     ch = Chunk{0, ci * kChunkRows, min(kChunkRows, a.implicit_rows - ci * kChunkRows),
                ci * kChunkRows};
   } else {
     const int2 e = a.tiles[t];
+    ci = e.x;
     ch = a.chunks[e.x];
     ft = e.y;
   }
@@ -406,6 +464,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
   uint64_t* sched_full = bars + 2 * kStages + 5;    // [kSched] tile published (each CTA)
   uint64_t* sched_empty = sched_full + kSched;      // [kSched] slot consumed (even CTA's)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sched_empty + kSched);
+  // MXFP8: per stage [A scales of up to 3 slabs | B scales of up to 3 slabs].
+  uint8_t* sf_base = smem + kSmemBase - 1024;
   // Schedule slots: {group, row0, nrows, src_row0, feature tile, -, -, -}; group
   // -1 ends the schedule.
   int* sched_info = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 256);
@@ -428,6 +488,11 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
       mbar_init(&sched_empty[i], kSchedConsumers);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (KD::kF8)
+      for (int i = 0; i < 2; ++i) {
+        prefetch_tmap(&maps.sfa[i]);
+        prefetch_tmap(&maps.sfb[i]);
+      }
     if (args.tma3d) {
       for (int i = 0; i < 2; ++i) prefetch_tmap(&maps.a3[i]);
       for (int i = 0; i < (kUp ? 2 : 1); ++i)
@@ -451,7 +516,7 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
                           : *args.n_tiles;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;   // static schedule only
   // K slabs per tile (the last may run past K: TMA fills those columns with zeros).
-  const int n_slabs = (args.K + kBK - 1) / kBK;
+  const int n_slabs = (args.K + KD::kSlabK - 1) / KD::kSlabK;
   int* err = args.err;
 
   if (warp == 0) {
@@ -477,20 +542,22 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           t = args.counter ? atomicAdd(args.counter, 1) : pair + iter * n_pairs;
           ++iter;
           Chunk c{-1, 0, 0, 0};
-          int f = 0;
-          if (t < n_tiles) get_tile(args, t, c, f);
+          int f = 0, cidx = 0;
+          if (t < n_tiles) get_tile(args, t, c, f, cidx);
           int* slot = sched_info + 8 * sslot;
           slot[0] = c.group;
           slot[1] = c.row0;
           slot[2] = c.nrows;
           slot[3] = c.src_row0;
           slot[4] = f;
+          slot[5] = cidx;
           const uint32_t peer_slot = map_to_cta(smem_u32(slot), 1);
           st_cluster_s32(peer_slot, c.group);
           st_cluster_s32(peer_slot + 4, c.row0);
           st_cluster_s32(peer_slot + 8, c.nrows);
           st_cluster_s32(peer_slot + 12, c.src_row0);
           st_cluster_s32(peer_slot + 16, f);
+          st_cluster_s32(peer_slot + 20, cidx);
           mbar_arrive_cluster(map_to_cta(smem_u32(&sched_full[sslot]), 0));
           mbar_arrive_cluster(map_to_cta(smem_u32(&sched_full[sslot]), 1));
         } else {
@@ -500,8 +567,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           }
         }
         Chunk ch;
-        int ft;
-        read_slot(sched_info + 8 * sslot, ch, ft);
+        int ft, ci;
+        read_slot(sched_info + 8 * sslot, ch, ft, ci);
         if (!leader) mbar_arrive_cluster(map_to_cta(smem_u32(&sched_empty[sslot]), 0));
         if (++sslot == kSched) {
           sslot = 0;
@@ -518,7 +585,7 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
         // normal token rows. The gate logits re-read W_g for every chunk.
         uint64_t pol_a = p_normal, pol_b = p_normal;
         if (KT_L2_HINTS != 0) {
-          const bool full = ch.nrows == kChunkRows;
+          const bool full = ch.nrows == (KD::kF8 ? kChunkRowsF8 : kChunkRows);
           if (kKind == kKindLogits) {
             pol_a = p_last;
             pol_b = p_first;
@@ -553,16 +620,30 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           if (args.tma3d) {
             // Two boxes for the whole stage; slabs past K are filled with zeros
             // and counted in the transaction bytes.
-            if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * slabs * (kATileBytes + b_slab));
+            const uint32_t sf_bytes = KD::kF8 ? slabs * (kSfaSlabBytes + kSfbSlabBytes) : 0;
+            if (leader)
+              mbar_arrive_expect_tx(&full_bar[stage], 2u * (slabs * (kATileBytes + b_slab) + sf_bytes));
             if (kUp)
               tma_load4_pair(sA, a3, fbar, 0, a_row, 0, s0, pol_a);
             else
               tma_load3_pair(sA, a3, fbar, 0, a_row, s0, pol_a);
             tma_load3_pair(sB, b3, fbar, 0, b_row, s0, pol_b);
+            if (KD::kF8) {
+              // Scales: this CTA's 128 weight rows (packed, 512 B per slab) and all
+              // token rows of the pair tile (1 KB per slab of the chunk's blocks),
+              // as rows of 256 bytes.
+              uint8_t* sS = sf_base + stage * kScaleStageBytes;
+              const int li = slabs == kSlabsLight ? 1 : 0;
+              const int64_t ablk =
+                  ((int64_t)(ch.group * args.n_ftiles_sf + ft) * 2 + rank) * args.n_kslabs + s0;
+              tma_load_pair(sS, &maps.sfa[li], fbar, 0, (int)(2 * ablk), pol_a);
+              tma_load_pair(sS + kSlabsLight * kSfaSlabBytes, &maps.sfb[li], fbar, 0,
+                            (int)(((int64_t)ci * args.n_kslabs + s0) * 4), pol_b);
+            }
           } else {
             if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * valid * (kATileBytes + b_slab));
             for (int j = 0; j < valid; ++j) {
-              const int kc = (s0 + j) * kBK;
+              const int kc = (s0 + j) * KD::kSlabK;
               uint8_t* a = sA + j * kATileBytes;
               uint8_t* b = sB + j * b_slab;
               if (kUp) {
@@ -619,8 +700,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
       for (;;) {
         if (!mbar_wait(&sched_full[sslot], sphase, err, 7 + 8 * kKind)) break;
         Chunk ch;
-        int ft;
-        read_slot(sched_info + 8 * sslot, ch, ft);
+        int ft, ci;
+        read_slot(sched_info + 8 * sslot, ch, ft, ci);
         mbar_arrive_cluster(smem_u32(&sched_empty[sslot]));
         if (++sslot == kSched) {
           sslot = 0;
@@ -634,7 +715,7 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
         }
         tc_fence_after();
         const uint32_t idesc = idesc_bf16(256, n);
-        const uint32_t d0 = tmem_base + buf * kAccCols;
+        const uint32_t d0 = tmem_base + buf * KD::kAccCols;
         const int hb = (n / 2 + kBoxRows - 1) / kBoxRows;
         const int slabs = stage_slabs(hb);
         const int nk = (n_slabs + slabs - 1) / slabs;
@@ -653,9 +734,24 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
             const uint64_t da = desc_a0 + (uint64_t)((stage * kStageBytes + j * kATileBytes) >> 4);
             const uint64_t db =
                 desc_a0 + (uint64_t)((stage * kStageBytes + b_off + j * b_slab) >> 4);
+            if (KD::kF8) {
+              // This slab's block scales into TMEM (in issue order with the MMAs
+              // that read them and with the previous slab's MMAs), then four
+              // K = 32 MMAs, each reading its K block's scale byte.
+              const uint32_t sS = smem_u32(sf_base + stage * kScaleStageBytes);
+              const uint32_t sB = sS + kSlabsLight * kSfaSlabBytes + j * kSfbSlabBytes;
+              sf_copy_pair(tmem_base + kSfaCol, sS + j * kSfaSlabBytes);
+              sf_copy_pair(tmem_base + kSfbCol, sB);
+              sf_copy_pair(tmem_base + kSfbCol + 4, sB + kSfbSlabBytes / 2);
 #pragma unroll
-            for (int ks = 0; ks < kBK / 16; ++ks)
-              mma_pair_bf16(d0, da + 2 * ks, db + 2 * ks, idesc, (kb | j | ks) != 0);
+              for (int ks = 0; ks < 4; ++ks)
+                mma_pair_mxf8(d0, da + 2 * ks, db + 2 * ks, idesc_mxf8(256, n, ks),
+                              tmem_base + kSfaCol, tmem_base + kSfbCol, (kb | j | ks) != 0);
+            } else {
+#pragma unroll
+              for (int ks = 0; ks < kBK / 16; ++ks)
+                mma_pair_bf16(d0, da + 2 * ks, db + 2 * ks, idesc, (kb | j | ks) != 0);
+            }
           }
           mma_commit_both(smem_u32(&empty_bar[stage]));
           issued_any = true;
@@ -703,8 +799,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
       const bool got = mbar_wait(&sched_full[sslot], sphase, err, 8 + 8 * kKind);
       if (!uniform_ok<kUp>(got, 1 + pr)) break;
       Chunk ch;
-      int ft;
-      read_slot(sched_info + 8 * sslot, ch, ft);
+      int ft, ci;
+      read_slot(sched_info + 8 * sslot, ch, ft, ci);
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(sched_empty_leader + sslot * 8);
       if (++sslot == kSched) {
@@ -716,7 +812,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
       const bool ready = mbar_wait(&tfull_bar[buf], bphase, err, 4 + 8 * kKind);
       if (!uniform_ok<kUp>(ready, 1 + pr)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * KD::kAccCols;
       // First output column of this warp.
       const int col0 = kUp ? ft * 128 + 64 * (int)rank + 32 * pr
                            : ft * 256 + 128 * (int)rank + 32 * q;
@@ -732,14 +829,35 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           }
           asm volatile("bar.sync %0, 64;" ::"r"(1 + pr) : "memory");
           xb ^= 1;
-          if (gate_warp) {
+          if (gate_warp && KD::kF8) {
+            // MXFP8 hidden rows: the warp's 32 features of one token are one
+            // block; its scale is the rule's exponent of the block's absolute
+            // maximum (a warp reduction), written into the down GEMM's scale
+            // blocks of this chunk by lane i for token row c0 + i.
+            uint8_t* s8 = stg;
+            uint8_t my_scale = 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h = silu(v[i]) * xc[i * 32 + lane];
+              float a = fabsf(h);
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1)
+                a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+              const int e = mx_scale_exp(a);
+              s8[i * 32 + lane] = mx_code(h, mx_inv_scale(e));
+              if (lane == i) my_scale = (uint8_t)(e + 127);
+            }
+            if (lane < 16 && c0 + lane < ch.nrows)
+              args.hid_sf[chunk_scale_offset(ci, args.out_cols / 128, c0 + lane, col0 / 32)] =
+                  my_scale;
+          } else if (gate_warp) {
             __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               sb[i * 32 + lane] = __float2bfloat16_rn(silu(v[i]) * xc[i * 32 + lane]);
           }
         } else {
-          if (kKind == kKindDown) {
+          if (kKind == kKindDown || kKind == kKindDownF8) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int row = ch.row0 + c0 + i;
@@ -753,7 +871,7 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
         if (!kUp || gate_warp) {
           __syncwarp();
           // 16 token rows of this warp's 32 output columns in 16-byte chunks:
-          // 64 B per row (bf16 hidden) or 128 B per row (fp32).
+          // 32 B per row (MXFP8 hidden codes), 64 B (bf16 hidden) or 128 B (fp32).
           constexpr int kRowBytes = 32 * KD::kOutBytes;
           constexpr int kChunksPerRow = kRowBytes / 16;
           constexpr int kElemsPerChunk = 16 / KD::kOutBytes;
@@ -827,17 +945,20 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
          CUDA_SUCCESS;
 }
 
-// 3-D view [cols / 64][rows][64] of a row-major [rows, cols] bf16 matrix (cols a
-// multiple of 64); box = box_slabs x box_rows x 64, landing slab-major.
+// 3-D view [cols / slab][rows][slab] of a row-major [rows, cols] matrix of bf16
+// (slab 64) or one-byte E4M3 codes (u8: slab 128) with cols a multiple of the
+// slab; box = box_slabs x box_rows x slab (128 bytes wide), landing slab-major.
 bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
-               uint32_t box_slabs) {
+               uint32_t box_slabs, bool u8 = false) {
   EncodeTiledFn enc = get_encode_fn();
-  if (!enc || cols % kBK != 0) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kBK), rows, cols / kBK};
-  const cuuint64_t strides[2] = {cols * 2, static_cast<cuuint64_t>(kBK) * 2};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), box_rows, box_slabs};
+  const uint64_t es = u8 ? 1 : 2, slab = 128 / es;
+  if (!enc || cols % slab != 0) return false;
+  const cuuint64_t dims[3] = {slab, rows, cols / slab};
+  const cuuint64_t strides[2] = {cols * es, 128};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(slab), box_rows, box_slabs};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
@@ -849,18 +970,20 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
 // per slab [box_rows rows of the first | the same rows of the second].
 // *q_first tells whether q is the first.
 bool make_map4_pair(CUtensorMap* m, const void* p, const void* q, uint64_t rows, uint64_t cols,
-                    uint32_t box_rows, uint32_t box_slabs, bool* q_first) {
+                    uint32_t box_rows, uint32_t box_slabs, bool* q_first, bool u8 = false) {
   EncodeTiledFn enc = get_encode_fn();
   const uint64_t up = reinterpret_cast<uint64_t>(p), uq = reinterpret_cast<uint64_t>(q);
   const uint64_t lo = up < uq ? up : uq, hi = up < uq ? uq : up;
+  const uint64_t es = u8 ? 1 : 2, slab = 128 / es;
   *q_first = uq < up;
-  if (!enc || cols % kBK != 0 || hi == lo || (hi - lo) % 16 != 0 || (hi - lo) >= (1ull << 40))
+  if (!enc || cols % slab != 0 || hi == lo || (hi - lo) % 16 != 0 || (hi - lo) >= (1ull << 40))
     return false;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kBK), rows, 2, cols / kBK};
-  const cuuint64_t strides[3] = {cols * 2, hi - lo, static_cast<cuuint64_t>(kBK) * 2};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(kBK), box_rows, 2, box_slabs};
+  const cuuint64_t dims[4] = {slab, rows, 2, cols / slab};
+  const cuuint64_t strides[3] = {cols * es, hi - lo, 128};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(slab), box_rows, 2, box_slabs};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, reinterpret_cast<void*>(lo), dims, strides,
+  return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+             reinterpret_cast<void*>(lo), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
@@ -868,6 +991,28 @@ bool make_map4_pair(CUtensorMap* m, const void* p, const void* q, uint64_t rows,
 
 // Token-row maps of one source: 2-D boxes of 32 and 128 rows; 3-D boxes of
 // 2-slab stages (32, 64, 96, 128 rows) and of 3-slab stages (32 rows).
+// Rows of 256 bytes over a byte array of n_rows * 256 bytes (block scales);
+// box = 256 bytes x box_rows, no swizzle.
+bool make_map_rows256(CUtensorMap* m, const void* base, uint64_t n_rows, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {256, n_rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {256, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// E4M3 token-row maps of one source (3-D only).
+bool make_token_maps_u8(TmaMaps* M, int src, const void* base, uint64_t rows, uint64_t cols) {
+  for (int hb = 1; hb <= 4; ++hb)
+    if (!make_map3(&M->b3[src][hb - 1], base, rows, cols, hb * kBoxRows, kSlabs, true))
+      return false;
+  return make_map3(&M->b3[src][4], base, rows, cols, kBoxRows, kSlabsLight, true);
+}
+
 bool make_token_maps(TmaMaps* M, int src, const void* base, uint64_t rows, uint64_t cols,
                      bool three_d) {
   if (!make_map(&M->b2[src][0], base, rows, cols, kBoxRows) ||
@@ -890,7 +1035,7 @@ cudaError_t ensure_smem_attr() {
   const uint64_t bit = dev >= 0 && dev < 64 ? 1ull << dev : 0;
   if (bit && (done.load() & bit)) return cudaSuccess;
   e = cudaFuncSetAttribute(grouped_gemm_kernel<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmemBytes);
+                           Kind<kKind>::kSmem);
   if (e == cudaSuccess && bit) done.fetch_or(bit);
   return e;
 }
@@ -899,7 +1044,7 @@ template <int kKind>
 cudaError_t launch(const TmaMaps& maps, const GemmArgs& args, int grid, cudaStream_t st) {
   cudaError_t e = ensure_smem_attr<kKind>();
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<kKind><<<grid, kThreads, kSmemBytes, st>>>(maps, args);
+  grouped_gemm_kernel<kKind><<<grid, kThreads, Kind<kKind>::kSmem, st>>>(maps, args);
   return cudaGetLastError();
 }
 
@@ -916,6 +1061,8 @@ cudaError_t prepare_grouped_gemm() {
   cudaError_t e = ensure_smem_attr<kKindUp>();
   if (e == cudaSuccess) e = ensure_smem_attr<kKindDown>();
   if (e == cudaSuccess) e = ensure_smem_attr<kKindLogits>();
+  if (e == cudaSuccess) e = ensure_smem_attr<kKindUpF8>();
+  if (e == cudaSuccess) e = ensure_smem_attr<kKindDownF8>();
   if (e == cudaSuccess && !get_encode_fn()) e = cudaErrorNotSupported;
   return e;
 }
@@ -979,6 +1126,80 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
   a.out = ws + L.expert_out;
   a.row_weight = reinterpret_cast<const float*>(ws + L.row_weight);
   return launch<kKindDown>(M, a, grid, st);
+}
+
+cudaError_t launch_experts_mxfp8(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                                 const void* wa, const void* wb, const uint8_t* sf, int num_sms,
+                                 cudaStream_t st, bool up) {
+  const int NG = r.E + r.S;
+  const int64_t R = T * (r.k + r.S);     // hidden rows
+  const int64_t Rr = T * r.k;            // routed rows
+  const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.meta);
+  GemmArgs a{};
+  a.chunks = reinterpret_cast<const Chunk*>(ws + L.chunks);
+  a.implicit_rows = 0;
+  a.n_routed_rows = (int)Rr;
+  a.err = reinterpret_cast<int*>(ws + L.err);
+  a.E = r.E;
+  a.tma3d = 1;
+  const int grid = pair_grid(num_sms, 0);
+  TmaMaps M;
+  memset(&M, 0, sizeof(M));
+  if (up) {
+    const uint64_t rows = (uint64_t)NG * r.I;
+    const uint64_t sfb_rows = (uint64_t)L.max_chunks * (r.d / 128) * 4;
+    bool w3_first = false;
+    if (!make_map4_pair(&M.a3[0], wa, wb, rows, r.d, 64, kSlabs, &w3_first, true) ||
+        !make_map4_pair(&M.a3[1], wa, wb, rows, r.d, 64, kSlabsLight, &w3_first, true) ||
+        !make_token_maps_u8(&M, 0, ws + L.xperm, Rr, r.d) ||
+        !make_token_maps_u8(&M, 1, ws + L.xq, T, r.d) ||
+        !make_map_rows256(&M.sfa[0], sf, mx_packed_bytes(r, false) / 256, 2 * kSlabs) ||
+        !make_map_rows256(&M.sfa[1], sf, mx_packed_bytes(r, false) / 256, 2 * kSlabsLight) ||
+        !make_map_rows256(&M.sfb[0], ws + L.tok_sf, sfb_rows, 4 * kSlabs) ||
+        !make_map_rows256(&M.sfb[1], ws + L.tok_sf, sfb_rows, 4 * kSlabsLight))
+      return cudaErrorInvalidValue;
+    if (w3_first) return cudaErrorInvalidValue;   // the packed scales list W1 first
+    a.gate_hi = 0;
+    a.n_kslabs = r.d / 128;
+    a.n_ftiles_sf = r.I / 128;
+    a.hid_sf = reinterpret_cast<uint8_t*>(ws + L.hid_sf);
+    a.tiles = reinterpret_cast<const int2*>(ws + L.tiles_up);
+    a.n_tiles = meta + 1;
+    a.counter = const_cast<int32_t*>(meta) + 3;
+    a.n_ftiles = r.I / 128;
+    a.rows_per_group = r.I;
+    a.K = r.d;
+    a.out_cols = r.I;
+    a.ldo = r.I;
+    a.out = ws + L.hidden;
+    a.row_weight = nullptr;
+    return launch<kKindUpF8>(M, a, grid, st);
+  }
+  const uint64_t rows = (uint64_t)NG * r.d;
+  const uint64_t sfb_rows = (uint64_t)L.max_chunks * (r.I / 128) * 4;
+  if (!make_map3(&M.a3[0], wa, rows, r.I, kARowsCta, kSlabs, true) ||
+      !make_map3(&M.a3[1], wa, rows, r.I, kARowsCta, kSlabsLight, true) ||
+      !make_token_maps_u8(&M, 0, ws + L.hidden, R, r.I) ||
+      !make_map_rows256(&M.sfa[0], sf, mx_packed_bytes(r, true) / 256, 2 * kSlabs) ||
+      !make_map_rows256(&M.sfa[1], sf, mx_packed_bytes(r, true) / 256, 2 * kSlabsLight) ||
+      !make_map_rows256(&M.sfb[0], ws + L.hid_sf, sfb_rows, 4 * kSlabs) ||
+      !make_map_rows256(&M.sfb[1], ws + L.hid_sf, sfb_rows, 4 * kSlabsLight))
+    return cudaErrorInvalidValue;
+  a.gate_hi = 0;
+  a.n_kslabs = r.I / 128;
+  a.n_ftiles_sf = (r.d + 255) / 256;
+  a.hid_sf = nullptr;
+  a.tiles = reinterpret_cast<const int2*>(ws + L.tiles_down);
+  a.n_tiles = meta + 2;
+  a.counter = const_cast<int32_t*>(meta) + 4;
+  a.n_ftiles = (r.d + 255) / 256;
+  a.rows_per_group = r.d;
+  a.K = r.I;
+  a.out_cols = r.d;
+  a.ldo = r.d;
+  a.out = ws + L.expert_out;
+  a.row_weight = reinterpret_cast<const float*>(ws + L.row_weight);
+  return launch<kKindDownF8>(M, a, grid, st);
 }
 
 cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, const void* w_gate,

@@ -422,7 +422,7 @@ int gate_logit_splits(const Resolved& r, int64_t T) { return T <= kSmallTokens ?
 
 cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, const void* w_gate,
                                float* logits, int* err, int num_sms, cudaStream_t st) {
-  const bool bf16 = r.dtype == KT_DTYPE_BF16;
+  const bool bf16 = r.act_bf16 != 0;
   if (T <= kSmallTokens) {
     const int vn = bf16 ? 8 : 4;
     const int kc = ((r.d + kSplitK - 1) / kSplitK + vn - 1) / vn * vn;

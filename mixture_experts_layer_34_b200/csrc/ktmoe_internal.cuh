@@ -5,6 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "ktmoe.h"
@@ -15,6 +16,7 @@ namespace ktmoe {
 // Tiling constants
 // ---------------------------------------------------------------------------
 constexpr int kPermChunk = 32;      // tokens per gate-select / scatter CTA
+constexpr int kChunkRowsF8 = 224;  // MXFP8 layers: two 224-column accumulators + scales in TMEM
 constexpr int kChunkRows = 256;     // token rows per GEMM chunk (MMA N <= 256)
 // Schedule tuning (compile-time; -D overrides are for tuning sweeps).
 #ifndef KT_TILE_BLOCK
@@ -48,6 +50,9 @@ struct Resolved {
   int norm;         // 0/1
   int group_score;  // KT_GROUP_AMAX / KT_GROUP_TOP2SUM (G == 1: unused)
   int dtype;        // KT_DTYPE_*
+  int act_bf16;     // tokens, gate weights and output in bf16 (KT_DTYPE_BF16 / MXFP8)
+  int fp8;          // expert weights in MXFP8
+  int chunk_rows;   // token rows per GEMM chunk: kChunkRows, or kChunkRowsF8 for MXFP8
   int add_residual;
   int y_fp32;       // y in fp32 (else in dtype)
   int has_bias;
@@ -81,8 +86,14 @@ struct Layout {
   size_t chunks;       // Chunk [max_chunks]
   size_t tiles_up;     // int2 (chunk, feature tile) [max_chunks * ceil(I/128)]
   size_t tiles_down;   // int2 [max_chunks * ceil(d/256)]
-  size_t xperm;        // dtype [T*k, d] (bf16 layers only)
-  size_t hidden;       // dtype [T*(k+S), I]
+  size_t xperm;        // [T*k, d]: bf16 (bf16 layers) or E4M3 codes (MXFP8 layers)
+  size_t hidden;       // [T*(k+S), I]: dtype, or E4M3 codes (MXFP8)
+  // MXFP8 layers only (else empty):
+  size_t xq;           // E4M3 codes of x [T, d]
+  size_t xs;           // their scale bytes [T, d/32] (row-major)
+  size_t tok_sf;       // token scales per GEMM chunk and 128-wide K slab: [chunks][d/128][1 KB]
+  size_t hid_sf;       // hidden-row scales, same form: [chunks][I/128][1 KB]
+  size_t gchunk0;      // int32 [E+S]: index of each group's first GEMM chunk
   size_t expert_out;   // fp32 [T*(k+S), d]
   size_t total;
   int64_t nperm, max_chunks;
@@ -133,6 +144,47 @@ cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, ch
                                int num_sms, cudaStream_t st, bool up);
 cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* ws,
                            const void* x, void* y, cudaStream_t st);
+
+// MXFP8 (mxfp8.cu).
+cudaError_t launch_mx_quantize(const void* src, int64_t rows, int64_t K, uint8_t* codes,
+                               uint8_t* scales, cudaStream_t st);
+size_t mx_packed_bytes(const Resolved& r, bool down);
+cudaError_t launch_mx_pack(const Resolved& r, const void* w1, const void* w3, const void* w2,
+                           uint8_t* w1q, uint8_t* w3q, uint8_t* w2q, uint8_t* sf_up,
+                           uint8_t* sf_down, cudaStream_t st);
+// The grouped GEMMs with MXFP8 weights (up: wa/wb = W1/W3 codes, sf = packed
+// gate/up scales; down: wa = W2 codes, sf = packed down scales).
+cudaError_t launch_experts_mxfp8(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                                 const void* wa, const void* wb, const uint8_t* sf, int num_sms,
+                                 cudaStream_t st, bool up);
+
+// MX block scale of a block with absolute maximum amax (>= 0): the smallest e
+// with amax <= 448 * 2^e, from the fp32 bits (amax = 1.m * 2^E: e = E - 8 +
+// (1.m > 1.75)); zero or subnormal amax gives -127; clamped to [-127, 127].
+__device__ __forceinline__ int mx_scale_exp(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ef = (int)((b >> 23) & 0xFF);
+  if (ef == 0) return -127;
+  const int e = ef - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+// 2^-e as an fp32 (e <= 126 for every finite amax).
+__device__ __forceinline__ float mx_inv_scale(int e) {
+  return e >= 127 ? 0x1p-127f : __uint_as_float((uint32_t)(127 - e) << 23);
+}
+// E4M3 code of v * inv, round to nearest even (|v * inv| <= 448 by the scale rule).
+__device__ __forceinline__ uint8_t mx_code(float v, float inv) {
+  return (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(v, inv), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Byte offset of the scale of (row m of a GEMM chunk, K block b) in the chunk
+// scale blocks [chunk][K / 128][1 KB]: two 512-byte halves of 128 rows, each in
+// the order the tensor cores read block scales (16 * (m % 32) + 4 * (m / 32 % 4)
+// + b % 4).
+__device__ __forceinline__ int64_t chunk_scale_offset(int64_t chunk, int nslab, int m, int b) {
+  return (chunk * nslab + b / 4) * 1024 + (m / 128) * 512 + 16 * (m % 32) + 4 * ((m / 32) % 4) +
+         (b % 4);
+}
 
 // Device-side helpers used by several kernels.
 __device__ __forceinline__ void set_error(int* err, int code, int detail) {

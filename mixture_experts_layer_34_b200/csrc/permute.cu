@@ -122,11 +122,12 @@ __device__ void fill_tiles(int2* __restrict__ tiles, int F, int NG, const int* c
 }
 
 __global__ void __launch_bounds__(kScanThreads)
-permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd,
+permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int chunk_rows,
                     const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base,
                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                     Chunk* __restrict__ chunks, int2* __restrict__ tiles_up,
-                    int2* __restrict__ tiles_dn, int32_t* __restrict__ meta) {
+                    int2* __restrict__ tiles_dn, int32_t* __restrict__ meta,
+                    int32_t* __restrict__ gchunk0) {
   constexpr int NGMAX = kMaxExperts + kMaxShared;
   __shared__ int tot[NGMAX];
   __shared__ int rows0[NGMAX];
@@ -161,10 +162,11 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd,
       run += chunk_counts[(int64_t)c * E + tid];
     }
   }
-  // GEMM chunks of kChunkRows rows and the two tile lists.
-  if (tid < NG) cb[tid] = (tot[tid] + kChunkRows - 1) / kChunkRows;
+  // GEMM chunks of chunk_rows rows and the two tile lists.
+  if (tid < NG) cb[tid] = (tot[tid] + chunk_rows - 1) / chunk_rows;
   __syncthreads();
   const int n_chunks = block_exclusive_scan(cb, NG);
+  if (tid < NG) gchunk0[tid] = cb[tid];
   if (tid == 0) {
     cb[NG] = n_chunks;
     meta[0] = n_chunks;
@@ -176,21 +178,26 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd,
   __syncthreads();
   for (int i = tid; i < n_chunks; i += blockDim.x) {
     const int g = find_group(cb, NG, i);
-    const int r = (i - cb[g]) * kChunkRows;
+    const int r = (i - cb[g]) * chunk_rows;
     const int src0 = g < E ? rows0[g] : 0;
-    chunks[i] = Chunk{g, rows0[g] + r, min(kChunkRows, tot[g] - r), src0 + r};
+    chunks[i] = Chunk{g, rows0[g] + r, min(chunk_rows, tot[g] - r), src0 + r};
   }
   fill_tiles(tiles_up, Fu, NG, cb, hb, lb, tot);
   fill_tiles(tiles_dn, Fd, NG, cb, hb, lb, tot);
 }
 
-template <bool kCopyX>
+// Copy modes of the scatter.
+enum { kNoCopy = 0, kCopyBf16 = 1, kCopyF8 = 2 };
+
+template <int kMode>
 __global__ void __launch_bounds__(256)
-permute_scatter_kernel(int E, int T_, int k, int d, const int32_t* __restrict__ idx,
-                       const float* __restrict__ w, const int32_t* __restrict__ chunk_base,
-                       int32_t* __restrict__ row_of, int32_t* __restrict__ tok_of,
-                       float* __restrict__ row_weight, const uint4* __restrict__ x,
-                       uint4* __restrict__ xperm) {
+permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
+                       const int32_t* __restrict__ idx, const float* __restrict__ w,
+                       const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
+                       const int32_t* __restrict__ gchunk0, int32_t* __restrict__ row_of,
+                       int32_t* __restrict__ tok_of, float* __restrict__ row_weight,
+                       const uint4* __restrict__ x, uint4* __restrict__ xperm,
+                       const uint8_t* __restrict__ xs, uint8_t* __restrict__ tok_sf) {
   __shared__ uint32_t mask[kMaxExperts];
   __shared__ int srow[kPermChunk * kMaxTopk];
   const int c = blockIdx.x;
@@ -215,10 +222,11 @@ permute_scatter_kernel(int E, int T_, int k, int d, const int32_t* __restrict__ 
     row_weight[row] = w[(int64_t)t0 * k + q];
     srow[q] = row;
   }
-  if (!kCopyX) return;
+  if (kMode == kNoCopy) return;
   __syncthreads();
-  // Copy each token's row of x to its k permuted rows (16-byte chunks).
-  const int nchunk = d / 8;
+  // Copy each token's row of x (bf16), or of its E4M3 codes, to its k permuted
+  // rows in 16-byte chunks.
+  const int nchunk = kMode == kCopyF8 ? d / 16 : d / 8;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int tl = warp; tl < nt; tl += blockDim.x / 32) {
     const uint4* src = x + (int64_t)(t0 + tl) * nchunk;
@@ -226,6 +234,28 @@ permute_scatter_kernel(int E, int T_, int k, int d, const int32_t* __restrict__ 
       const uint4 v = src[q];
       for (int j = 0; j < k; ++j) xperm[(int64_t)srow[tl * k + j] * nchunk + q] = v;
     }
+  }
+  if (kMode != kCopyF8) return;
+  // MXFP8: each routed row's and each shared-expert row's scale bytes into its
+  // GEMM chunk's scale blocks (4 K blocks per 32-bit word).
+  const int nslab = d / 128;
+  const int nent_all = nt * (k + S);
+  for (int q = warp; q < nent_all; q += blockDim.x / 32) {
+    const int tl = q / (k + S), j = q % (k + S);
+    int g, rel;
+    if (j < k) {
+      g = idx[(int64_t)(t0 + tl) * k + j];
+      rel = srow[tl * k + j] - offsets[g];
+    } else {
+      g = E + (j - k);
+      rel = t0 + tl;
+    }
+    const int64_t chunk = gchunk0[g] + rel / chunk_rows;
+    const int m = rel % chunk_rows;
+    const uint32_t* srcs = reinterpret_cast<const uint32_t*>(xs + (int64_t)(t0 + tl) * (d / 32));
+    for (int s4 = lane; s4 < nslab; s4 += 32)
+      *reinterpret_cast<uint32_t*>(tok_sf + chunk_scale_offset(chunk, nslab, m, 4 * s4)) =
+          srcs[s4];
   }
 }
 
@@ -235,22 +265,30 @@ cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* 
                            const int32_t* idx, const float* w, const void* x, cudaStream_t st) {
   auto I32 = [&](size_t off) { return reinterpret_cast<int32_t*>(ws + off); };
   permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
-      r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256,
+      r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows,
       I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts), I32(L.offsets),
       reinterpret_cast<Chunk*>(ws + L.chunks), reinterpret_cast<int2*>(ws + L.tiles_up),
-      reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta));
+      reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)L.nperm;
   float* rw = reinterpret_cast<float*>(ws + L.row_weight);
-  if (r.dtype == KT_DTYPE_BF16)
-    permute_scatter_kernel<true><<<grid, 256, 0, st>>>(
-        r.E, (int)T, r.k, r.d, idx, w, I32(L.chunk_base), I32(L.row_of), I32(L.tok_of), rw,
-        reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(ws + L.xperm));
+  const int32_t* base = I32(L.chunk_base);
+  if (r.fp8)
+    permute_scatter_kernel<kCopyF8><<<grid, 256, 0, st>>>(
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(ws + L.xq),
+        reinterpret_cast<uint4*>(ws + L.xperm), reinterpret_cast<const uint8_t*>(ws + L.xs),
+        reinterpret_cast<uint8_t*>(ws + L.tok_sf));
+  else if (r.dtype == KT_DTYPE_BF16)
+    permute_scatter_kernel<kCopyBf16><<<grid, 256, 0, st>>>(
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(x),
+        reinterpret_cast<uint4*>(ws + L.xperm), nullptr, nullptr);
   else
-    permute_scatter_kernel<false><<<grid, 256, 0, st>>>(
-        r.E, (int)T, r.k, r.d, idx, w, I32(L.chunk_base), I32(L.row_of), I32(L.tok_of), rw,
-        nullptr, nullptr);
+    permute_scatter_kernel<kNoCopy><<<grid, 256, 0, st>>>(
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr, nullptr);
   return cudaGetLastError();
 }
 

@@ -16,11 +16,11 @@ LIB_PATH = os.path.join(HERE, "libktmoe.so")
 
 KT_SCORE_SIGMOID, KT_SCORE_SOFTMAX = 0, 1
 KT_GROUP_AUTO, KT_GROUP_AMAX, KT_GROUP_TOP2SUM = 0, 1, 2
-KT_DTYPE_F32, KT_DTYPE_BF16 = 0, 1
 KT_OK = 0
 KT_ERR_INVALID_CONFIG, KT_ERR_NULL, KT_ERR_WORKSPACE, KT_ERR_ALIGN = -1, -2, -3, -4
 KT_ERR_CUDA, KT_ERR_TIMEOUT, KT_ERR_UNSUPPORTED, KT_ERR_SCRATCH_LIMIT = -5, -6, -7, -8
 KT_STATIC_SCRATCH_BYTES = 32 << 20
+KT_DTYPE_F32, KT_DTYPE_BF16, KT_DTYPE_MXFP8 = 0, 1, 2
 
 # Every symbol include/ktmoe.h declares.
 EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_forward",
@@ -28,7 +28,8 @@ EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_fo
            "kt_moe_check", "kt_moe_workspace_layout", "kt_moe_strerror", "kt_moe_version",
            "kt_moe_scores", "kt_moe_bias_update", "kt_moe_balance_workspace_size",
            "kt_moe_balance_stats", "kt_moe_graph_create", "kt_moe_graph_launch",
-           "kt_moe_graph_destroy")
+           "kt_moe_graph_destroy", "kt_moe_mxfp8_quantize", "kt_moe_mxfp8_scale_bytes",
+           "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -45,7 +46,8 @@ class kt_moe_ws_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in ("error_word", "logits", "logits_splits", "counts", "offsets",
                                               "row_of", "tok_of", "row_weight", "hidden",
                                               "expert_out", "meta", "chunks", "tiles_up",
-                                              "tiles_down", "total")]
+                                              "tiles_down", "total", "xq", "xs", "xperm",
+                                              "tok_sf", "hid_sf")]
 
 
 class KtMoeError(RuntimeError):
@@ -105,6 +107,15 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_graph_launch.restype = ctypes.c_int
             L.kt_moe_graph_destroy.argtypes = [P]
             L.kt_moe_graph_destroy.restype = None
+            L.kt_moe_mxfp8_quantize.argtypes = [I64, I64, P, P, P, P]
+            L.kt_moe_mxfp8_quantize.restype = ctypes.c_int
+            L.kt_moe_mxfp8_scale_bytes.argtypes = [CP, ctypes.c_int]
+            L.kt_moe_mxfp8_scale_bytes.restype = ctypes.c_size_t
+            L.kt_moe_mxfp8_pack.argtypes = [CP, P, P, P, P, P, P, P, P, P]
+            L.kt_moe_mxfp8_pack.restype = ctypes.c_int
+            L.kt_moe_forward_mxfp8.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P, P, P,
+                                               ctypes.c_size_t, P, P]
+            L.kt_moe_forward_mxfp8.restype = ctypes.c_int
             L.kt_moe_version.argtypes = []
             L.kt_moe_version.restype = ctypes.c_int
             _lib = L
@@ -243,6 +254,55 @@ class KtMoeGraph:
             pass
 
 
+def kt_moe_mxfp8_quantize(rows, K, src, codes, scales, stream=None):
+    rc = lib().kt_moe_mxfp8_quantize(int(rows), int(K), _ptr(src), _ptr(codes), _ptr(scales),
+                                     _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_mxfp8_quantize", rc)
+
+
+def kt_moe_mxfp8_scale_bytes(cfg: kt_moe_config, down: bool) -> int:
+    return int(lib().kt_moe_mxfp8_scale_bytes(ctypes.byref(cfg), int(bool(down))))
+
+
+def kt_moe_mxfp8_pack(cfg, w1, w3, w2, w1q, w3q, w2q, sf_up, sf_down, stream=None):
+    rc = lib().kt_moe_mxfp8_pack(ctypes.byref(cfg), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(w1q),
+                                 _ptr(w3q), _ptr(w2q), _ptr(sf_up), _ptr(sf_down), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_mxfp8_pack", rc)
+
+
+def pack_mxfp8(cfg, w1, w3, w2, stream=None) -> dict:
+    """Allocate the MXFP8 codes (W1 and W3 as the two halves of one buffer) and
+    the packed scales for bf16 weights, and pack them."""
+    import torch
+    w13 = torch.empty((2,) + tuple(w1.shape), dtype=torch.uint8, device=w1.device)
+    out = dict(w1q=w13[0], w3q=w13[1],      # W1's codes below W3's, as the forward needs
+               w2q=torch.empty(w2.shape, dtype=torch.uint8, device=w2.device),
+               sf_up=torch.empty(kt_moe_mxfp8_scale_bytes(cfg, False), dtype=torch.uint8,
+                                 device=w1.device),
+               sf_down=torch.empty(kt_moe_mxfp8_scale_bytes(cfg, True), dtype=torch.uint8,
+                                   device=w1.device))
+    kt_moe_mxfp8_pack(cfg, w1, w3, w2, out["w1q"], out["w3q"], out["w2q"], out["sf_up"],
+                      out["sf_down"], stream)
+    return out
+
+
+def kt_moe_forward_mxfp8(cfg, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y, topk_idx_out,
+                         topk_w_out, workspace, stream=None, stage_events=None):
+    ev = None
+    if stage_events is not None:
+        ev = (ctypes.c_void_p * KT_STAGE_EVENTS)(*[ctypes.c_void_p(e.cuda_event)
+                                                   if e is not None else None
+                                                   for e in stage_events])
+    rc = lib().kt_moe_forward_mxfp8(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias),
+                                    _ptr(w1q), _ptr(w3q), _ptr(w2q), _ptr(sf_up), _ptr(sf_down),
+                                    _ptr(y), _ptr(topk_idx_out), _ptr(topk_w_out),
+                                    _ptr(workspace), _nbytes(workspace), _stream(stream), ev)
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_forward_mxfp8", rc)
+
+
 KT_STAGE_EVENTS = 6
 STAGES = ("gate", "permute", "up_gemm", "down_gemm", "combine")
 
@@ -290,8 +350,8 @@ def kt_moe_version() -> int:
 
 def config_for(layer, y_fp32: bool = False) -> kt_moe_config:
     """kt_moe_config of a workloads.LayerConfig."""
-    return make_config(dtype=KT_DTYPE_F32 if layer.dtype == "f32" else KT_DTYPE_BF16,
-                       y_fp32=int(y_fp32), **layer.kernel_fields())
+    dt = {"f32": KT_DTYPE_F32, "bf16": KT_DTYPE_BF16, "mxfp8": KT_DTYPE_MXFP8}[layer.dtype]
+    return make_config(dtype=dt, y_fp32=int(y_fp32), **layer.kernel_fields())
 
 
 def alloc_workspace(cfg: kt_moe_config, T: int, device="cuda"):

@@ -59,7 +59,7 @@ class LayerConfig:
     route_scale: float
     norm_topk: int          # -1 auto (renormalise iff sigmoid), 0, 1
     group_score: int        # 0 auto, 1 amax, 2 top-2 sum
-    dtype: str              # "f32" or "bf16"
+    dtype: str              # "f32", "bf16" or "mxfp8" (bf16 tokens, MXFP8 expert weights)
     bias: str               # "none", "normal", "zipf"
     seed: int
     init: str = "std002"    # "std002" or "fan_in"
@@ -150,6 +150,22 @@ PROFILE = [
                 bias="none", seed=2102),
 ]
 BY_NAME.update({c.name: c for c in PROFILE})
+
+# MXFP8-expert forms (bf16 tokens and gate, expert weights packed to MXFP8 from
+# the same seeded bf16 weights): the V3-shaped layers and two small parity
+# layers (dims multiples of 128; ragged token counts; chunks of 224 rows).
+MXFP8 = [
+    V3_PREFILL.with_(name="v3_prefill_T8192_zipf_mxfp8", dtype="mxfp8"),
+    V3_DECODE.with_(name="v3_decode_T8_mxfp8", dtype="mxfp8"),
+    LayerConfig("small_sig_bias_mxfp8", T=300, dim=512, n_experts=32, n_groups=4, topk_groups=2,
+                topk=4, n_shared=1, inter=256, score_func=SIGMOID, route_scale=2.5,
+                norm_topk=-1, group_score=GROUP_AUTO, dtype="mxfp8", bias="normal", seed=2301),
+    LayerConfig("small_softmax_mxfp8", T=500, dim=384, n_experts=16, n_groups=1, topk_groups=1,
+                topk=3, n_shared=2, inter=384, score_func=SOFTMAX, route_scale=1.0,
+                norm_topk=0, group_score=GROUP_AUTO, dtype="mxfp8", bias="none", seed=2302),
+    PROFILE[0].with_(name="v3_shape_T2048_E32_profile_mxfp8", dtype="mxfp8"),
+]
+BY_NAME.update({c.name: c for c in MXFP8})
 
 
 def torch_dtype(cfg: LayerConfig) -> torch.dtype:

@@ -40,7 +40,7 @@ def test_library_links_no_torch():
 
 def test_config_struct_layout_matches_header():
     assert ctypes.sizeof(K.kt_moe_config) == 14 * 4
-    assert ctypes.sizeof(K.kt_moe_ws_layout) == 15 * 8
+    assert ctypes.sizeof(K.kt_moe_ws_layout) == 20 * 8
 
 
 @pytest.mark.parametrize("layer", W.NAMED + W.SMALL, ids=lambda c: c.name)

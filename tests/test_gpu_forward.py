@@ -240,3 +240,19 @@ def test_w3_below_w1_in_memory_gives_the_same_output():
     b = run_forward(layer, inp2, y_fp32=True)
     assert torch.equal(a["idx"], b["idx"])
     assert torch.equal(a["y"], b["y"])
+
+
+@pytest.mark.parametrize("name", ["small_sig_bias", "small_odd_dims"])
+def test_output_does_not_depend_on_workspace_contents(name):
+    """A forward that read any workspace byte it did not write first would change
+    (or turn NaN: 0xFF bytes are NaN in fp32) with this fill."""
+    layer = W.BY_NAME[name]
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer, y_fp32=True)
+    outs = []
+    for fill in (0x00, 0xFF):
+        ws = K.alloc_workspace(cfg, layer.T)
+        ws.fill_(fill)
+        outs.append(run_forward(layer, inp, ws=ws, y_fp32=True)["y"])
+    assert not torch.isnan(outs[1]).any()
+    assert torch.equal(outs[0], outs[1])
