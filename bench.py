@@ -54,6 +54,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall time of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8-weight lines")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -174,6 +175,8 @@ class ClockSampler:
 def algorithmic(layer, idx: np.ndarray) -> dict:
     T, d, I, k, S, E = layer.T, layer.dim, layer.inter, layer.topk, layer.n_shared, layer.n_experts
     es = 4 if layer.dtype == "f32" else 2
+    # expert-weight bytes per element (MXFP8: one byte plus one scale byte per 32)
+    ew = 1 + 1 / 32 if layer.dtype == "mxfp8" else es
     R = T * (k + S)
     active = int((np.bincount(idx.ravel(), minlength=E) > 0).sum()) + S
     return {
@@ -183,9 +186,9 @@ def algorithmic(layer, idx: np.ndarray) -> dict:
         "flops_up": 4 * d * I * R,
         "flops_down": 2 * d * I * R,
         # bytes the method must move: activated experts' weights, W_gate, x, y
-        "bytes_layer": active * 3 * d * I * es + E * d * es + 2 * T * d * es,
+        "bytes_layer": active * 3 * d * I * ew + E * d * es + 2 * T * d * es,
         # gate/up GEMM: W1, W3 of active experts, the token rows in, hidden rows out
-        "bytes_up": active * 2 * d * I * es + R * d * es + R * I * es,
+        "bytes_up": active * 2 * d * I * ew + R * d * es + R * I * es,
     }
 
 
@@ -205,9 +208,26 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
     idx = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
     w = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
     args = (cfg, T, inp["x"], inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], y, idx, w, ws)
+    fp8 = layer.dtype == "mxfp8"
+    if fp8:
+        # MXFP8 form: pack the seeded bf16 expert weights once, then drop them.
+        q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+        torch.cuda.synchronize()
+        inp["w1"] = inp["w3"] = inp["w2"] = None
+        torch.cuda.empty_cache()
+
+    def fwd(x, events=None):
+        if fp8:
+            K.kt_moe_forward_mxfp8(cfg, T, x, inp["w_gate"], inp["bias"], q["w1q"], q["w3q"],
+                                   q["w2q"], q["sf_up"], q["sf_down"], y, idx, w, ws,
+                                   stage_events=events)
+        elif events is not None:
+            K.kt_moe_forward_profiled(cfg, T, x, *args[3:], events)
+        else:
+            K.kt_moe_forward(cfg, T, x, *args[3:])
 
     for _ in range(warmup):
-        K.kt_moe_forward(*args)
+        fwd(inp["x"])
     rc = K.kt_moe_check(ws)
     if rc != K.KT_OK:
         raise RuntimeError(f"device error after warm-up: {K.strerror(rc)}")
@@ -224,7 +244,7 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
     torch.cuda.synchronize()
     t0.record()
     for s in range(steps):
-        K.kt_moe_forward_profiled(*args, ev[s])
+        fwd(inp["x"], ev[s])
     t1.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -238,7 +258,7 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
 
     # The same forward replayed as one CUDA graph (kt_moe_graph_*), same buffers.
     graph_ms = None
-    if graph:
+    if graph and not fp8:
         gr = K.KtMoeGraph(*args)
         for _ in range(warmup):
             gr.launch()
@@ -261,11 +281,9 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
     x_h = inp["x"].cpu().pin_memory()
     y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
     x_d = torch.empty_like(inp["x"])
-    eargs = list(args)
-    eargs[2] = x_d
     for _ in range(3):
         x_d.copy_(x_h, non_blocking=True)
-        K.kt_moe_forward(*eargs)
+        fwd(x_d)
         y_h.copy_(y, non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
@@ -273,7 +291,7 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
     t0.record()
     for _ in range(e2e_steps):
         x_d.copy_(x_h, non_blocking=True)
-        K.kt_moe_forward(*eargs)
+        fwd(x_d)
         y_h.copy_(y, non_blocking=True)
     t1.record()
     torch.cuda.synchronize()
@@ -342,6 +360,15 @@ def run_ours(a):
     if a.decode_workload != "none":
         dlayer = W.BY_NAME[a.decode_workload]
         dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, graph=True)
+    # The same layers with MXFP8 expert weights (same shapes, seeds and tokens).
+    f8 = {}
+    if not a.no_mxfp8:
+        for key, base in (("prefill", layer.name), ("decode", a.decode_workload)):
+            name = base + "_mxfp8"
+            if name in W.BY_NAME:
+                f8[key] = (W.BY_NAME[name], time_layer(W.BY_NAME[name], dev, rank, world, a.steps,
+                                                       a.warmup, a.e2e_steps))
+                f8[key][1].pop("inp")
     clk = clocks.stop()
 
     cpu = None
@@ -413,6 +440,38 @@ def run_ours(a):
                           "value": round(world * dl.T * a.steps / (dec["graph_ms"] / 1e3), 1),
                           "unit": "tokens/s"},
             }
+        if f8:
+            line["mxfp8"] = {"note": "MXFP8 expert weights (E4M3, power-of-two scale per 32 "
+                                     "along K); bf16 tokens, gate and output"}
+            f8_peak = 2 * peaks["bf16_tflops_sustained"]
+            for key, (fl, res) in f8.items():
+                ms = res["ms"] / K_
+                ent = {"workload": fl.name, "value": round(world * fl.T / (ms / 1e3), 1),
+                       "unit": "tokens/s", "ms_per_step": round(ms, 4),
+                       "stage_ms": {k: round(v, 4) for k, v in res["stage_ms"].items()},
+                       "e2e": {"value": round(world * fl.T * a.e2e_steps / (res["e2e_ms"] / 1e3), 1),
+                               "unit": "tokens/s"}}
+                up_s = res["stage_ms"]["up_gemm"] / 1e3
+                if key == "prefill":
+                    ach = res["work"]["flops_up"] / up_s / 1e12
+                    ent["roofline"] = {"kernel": "grouped gate/up GEMM (tcgen05 kind::mxf8f6f4)",
+                                       "bound": "tensor", "achieved": round(ach, 1),
+                                       "peak": f8_peak, "unit": "TFLOP/s",
+                                       "frac": round(ach / f8_peak, 4),
+                                       "traffic": traffic("up", fl.name),
+                                       "peak_source": peaks["source"] + " bf16 (sustained) x 2, "
+                                                      "the nominal fp8 / bf16 ratio"}
+                else:
+                    gbs = res["work"]["bytes_up"] / up_s / 1e9
+                    lgbs = res["work"]["bytes_layer"] / (ms / 1e3) / 1e9
+                    ent["layer_hbm_gbs"] = round(lgbs, 1)
+                    ent["layer_hbm_frac"] = round(lgbs / peaks["hbm_gbs"], 4)
+                    ent["roofline"] = {"kernel": "grouped gate/up GEMM (tcgen05 kind::mxf8f6f4)",
+                                       "bound": "hbm", "achieved": round(gbs, 1),
+                                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                       "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                       "traffic": traffic("up", fl.name)}
+                line["mxfp8"][key] = ent
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
