@@ -821,6 +821,48 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
         float v[16];
         tmem_ld16(tbase + c0, v);
         tmem_ld_wait();
+        if (KD::kF8 && kUp) {
+          // MXFP8 hidden rows. The two warps of a pair split the 16 columns: each
+          // sends the other the 8 values it lacks (gate or up), then computes,
+          // quantises and stores its own 8 token rows. The warp's 32 features of
+          // one token are one block: its scale is the rule's exponent of the
+          // block's absolute maximum (one integer warp reduction over |h| bits),
+          // written into the down GEMM's scale blocks of this chunk.
+          float* xc = xchg + (pr * 2 + xb) * 16 * 32;
+          const int mine0 = gate_warp ? 0 : 8, other0 = 8 - mine0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) xc[(other0 + i) * 32 + lane] = v[other0 + i];
+          asm volatile("bar.sync %0, 64;" ::"r"(1 + pr) : "memory");
+          xb ^= 1;
+          uint8_t* s8 = stg;
+          uint8_t my_scale = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float mv = v[mine0 + i], ov = xc[(mine0 + i) * 32 + lane];
+            const float h = gate_warp ? silu(mv) * ov : silu(ov) * mv;
+            const uint32_t amax =
+                __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7fffffffu);
+            const int e = mx_scale_exp(__uint_as_float(amax));
+            s8[i * 32 + lane] = mx_code(h, mx_inv_scale(e));
+            if (lane == i) my_scale = (uint8_t)(e + 127);
+          }
+          const int cr = c0 + mine0;
+          if (lane < 8 && cr + lane < ch.nrows)
+            args.hid_sf[chunk_scale_offset(ci, args.out_cols / 128, cr + lane, col0 / 32)] =
+                my_scale;
+          __syncwarp();
+          // 8 token rows x 32 code bytes: 16 chunks of 16 bytes.
+          if (lane < 16) {
+            const int rr = lane / 2, part = lane % 2;
+            if (cr + rr < ch.nrows)
+              *reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
+                                        (int64_t)(ch.row0 + cr + rr) * args.ldo + col0 +
+                                        part * 16) =
+                  *reinterpret_cast<const uint4*>(s8 + rr * 32 + part * 16);
+          }
+          __syncwarp();
+          continue;
+        }
         if (kUp) {
           float* xc = xchg + (pr * 2 + xb) * 16 * 32;
           if (!gate_warp) {
@@ -829,28 +871,7 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           }
           asm volatile("bar.sync %0, 64;" ::"r"(1 + pr) : "memory");
           xb ^= 1;
-          if (gate_warp && KD::kF8) {
-            // MXFP8 hidden rows: the warp's 32 features of one token are one
-            // block; its scale is the rule's exponent of the block's absolute
-            // maximum (a warp reduction), written into the down GEMM's scale
-            // blocks of this chunk by lane i for token row c0 + i.
-            uint8_t* s8 = stg;
-            uint8_t my_scale = 0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h = silu(v[i]) * xc[i * 32 + lane];
-              float a = fabsf(h);
-#pragma unroll
-              for (int off = 16; off > 0; off >>= 1)
-                a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-              const int e = mx_scale_exp(a);
-              s8[i * 32 + lane] = mx_code(h, mx_inv_scale(e));
-              if (lane == i) my_scale = (uint8_t)(e + 127);
-            }
-            if (lane < 16 && c0 + lane < ch.nrows)
-              args.hid_sf[chunk_scale_offset(ci, args.out_cols / 128, c0 + lane, col0 / 32)] =
-                  my_scale;
-          } else if (gate_warp) {
+          if (gate_warp) {
             __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(stg);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
