@@ -216,6 +216,14 @@ int kt_moe_graph_create(const kt_moe_config* cfg, int64_t T, const void* x, cons
                         const float* bias, const void* w1, const void* w3, const void* w2,
                         void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                         size_t ws_bytes, kt_moe_graph** graph_out);
+/* The same for the MXFP8 form: captures one kt_moe_forward_mxfp8 with these
+ * arguments (host checks and errors as for kt_moe_forward_mxfp8). */
+int kt_moe_graph_create_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x,
+                              const void* w_gate, const float* bias, const uint8_t* w1q,
+                              const uint8_t* w3q, const uint8_t* w2q, const uint8_t* sf_up,
+                              const uint8_t* sf_down, void* y, int32_t* topk_idx_out,
+                              float* topk_w_out, void* workspace, size_t ws_bytes,
+                              kt_moe_graph** graph_out);
 int kt_moe_graph_launch(kt_moe_graph* graph, void* stream);
 void kt_moe_graph_destroy(kt_moe_graph* graph);
 

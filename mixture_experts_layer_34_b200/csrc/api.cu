@@ -522,18 +522,17 @@ struct kt_moe_graph {
 
 extern "C" {
 
-int kt_moe_graph_create(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
-                        const float* bias, const void* w1, const void* w3, const void* w2,
-                        void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
-                        size_t ws_bytes, kt_moe_graph** graph_out) {
-  if (!graph_out) return KT_ERR_NULL;
-  *graph_out = nullptr;
-  Resolved r;
-  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
-                              workspace, ws_bytes, &r);
-  if (rc != KT_OK) return rc;
+}  // extern "C"
+
+namespace {
+
+// Capture one forward (`fwd`, enqueued on the given stream) on a private stream
+// and instantiate it.
+template <class Fwd>
+int capture_graph(Fwd fwd, kt_moe_graph** graph_out) {
   int sms = 0;
-  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  int rc = device_info(&sms);
+  if (rc != KT_OK) return rc;
   if (prepare_grouped_gemm() != cudaSuccess) return KT_ERR_CUDA;
   cudaStream_t cs = nullptr;
   if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return KT_ERR_CUDA;
@@ -541,8 +540,7 @@ int kt_moe_graph_create(const kt_moe_config* cfg, int64_t T, const void* x, cons
     cudaStreamDestroy(cs);
     return KT_ERR_CUDA;
   }
-  rc = kt_moe_forward_profiled(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
-                               workspace, ws_bytes, cs, nullptr);
+  rc = fwd(cs);
   cudaGraph_t g = nullptr;
   const cudaError_t ec = cudaStreamEndCapture(cs, &g);
   cudaStreamDestroy(cs);
@@ -563,6 +561,53 @@ int kt_moe_graph_create(const kt_moe_config* cfg, int64_t T, const void* x, cons
   }
   *graph_out = h;
   return KT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kt_moe_graph_create(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                        const float* bias, const void* w1, const void* w3, const void* w2,
+                        void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                        size_t ws_bytes, kt_moe_graph** graph_out) {
+  if (!graph_out) return KT_ERR_NULL;
+  *graph_out = nullptr;
+  Resolved r;
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out, topk_w_out,
+                              workspace, ws_bytes, &r);
+  if (rc != KT_OK) return rc;
+  if (r.fp8) return KT_ERR_INVALID_CONFIG;
+  return capture_graph(
+      [&](cudaStream_t cs) {
+        return kt_moe_forward_profiled(cfg, T, x, w_gate, bias, w1, w3, w2, y, topk_idx_out,
+                                       topk_w_out, workspace, ws_bytes, cs, nullptr);
+      },
+      graph_out);
+}
+
+int kt_moe_graph_create_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x,
+                              const void* w_gate, const float* bias, const uint8_t* w1q,
+                              const uint8_t* w3q, const uint8_t* w2q, const uint8_t* sf_up,
+                              const uint8_t* sf_down, void* y, int32_t* topk_idx_out,
+                              float* topk_w_out, void* workspace, size_t ws_bytes,
+                              kt_moe_graph** graph_out) {
+  if (!graph_out) return KT_ERR_NULL;
+  *graph_out = nullptr;
+  Resolved r;
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y, topk_idx_out,
+                              topk_w_out, workspace, ws_bytes, &r);
+  if (rc != KT_OK) return rc;
+  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
+  if (!sf_up || !sf_down) return KT_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
+    return KT_ERR_INVALID_CONFIG;
+  return capture_graph(
+      [&](cudaStream_t cs) {
+        return kt_moe_forward_mxfp8(cfg, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y,
+                                    topk_idx_out, topk_w_out, workspace, ws_bytes, cs, nullptr);
+      },
+      graph_out);
 }
 
 int kt_moe_graph_launch(kt_moe_graph* graph, void* stream) {

@@ -29,7 +29,7 @@ EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_fo
            "kt_moe_scores", "kt_moe_bias_update", "kt_moe_balance_workspace_size",
            "kt_moe_balance_stats", "kt_moe_graph_create", "kt_moe_graph_launch",
            "kt_moe_graph_destroy", "kt_moe_mxfp8_quantize", "kt_moe_mxfp8_scale_bytes",
-           "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8")
+           "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8", "kt_moe_graph_create_mxfp8")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -103,6 +103,10 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_graph_create.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P,
                                               ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]
             L.kt_moe_graph_create.restype = ctypes.c_int
+            L.kt_moe_graph_create_mxfp8.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P, P, P,
+                                                    ctypes.c_size_t,
+                                                    ctypes.POINTER(ctypes.c_void_p)]
+            L.kt_moe_graph_create_mxfp8.restype = ctypes.c_int
             L.kt_moe_graph_launch.argtypes = [P, P]
             L.kt_moe_graph_launch.restype = ctypes.c_int
             L.kt_moe_graph_destroy.argtypes = [P]
@@ -235,6 +239,22 @@ class KtMoeGraph:
         if rc != KT_OK:
             raise KtMoeError("kt_moe_graph_create", rc)
         self._h = h
+
+    @classmethod
+    def mxfp8(cls, cfg, T, x, w_gate, bias, q, y, topk_idx_out, topk_w_out, workspace):
+        """A captured kt_moe_forward_mxfp8; q holds the packed weights (pack_mxfp8)."""
+        self = cls.__new__(cls)
+        self._keep = (x, w_gate, bias, q, y, topk_idx_out, topk_w_out, workspace)
+        h = ctypes.c_void_p(0)
+        rc = lib().kt_moe_graph_create_mxfp8(
+            ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias), _ptr(q["w1q"]),
+            _ptr(q["w3q"]), _ptr(q["w2q"]), _ptr(q["sf_up"]), _ptr(q["sf_down"]), _ptr(y),
+            _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace), _nbytes(workspace),
+            ctypes.byref(h))
+        if rc != KT_OK:
+            raise KtMoeError("kt_moe_graph_create_mxfp8", rc)
+        self._h = h
+        return self
 
     def launch(self, stream=None):
         rc = lib().kt_moe_graph_launch(self._h, _stream(stream))

@@ -57,3 +57,33 @@ def test_graph_create_rejects_bad_arguments_without_leaving_a_handle():
     with pytest.raises(K.KtMoeError):
         K.KtMoeGraph(cfg, layer.T, inp["x"], inp["w_gate"], inp["bias"], inp["w1"], inp["w3"],
                      inp["w2"], y, None, None, ws[:-1])
+
+
+@pytest.mark.parametrize("name", ["v3_decode_T8_mxfp8", "small_sig_bias_mxfp8"])
+def test_mxfp8_graph_launches_match_the_direct_forward(name):
+    layer = W.BY_NAME[name]
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer)
+    T = layer.T
+    q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+    ws = K.alloc_workspace(cfg, T)
+    y = torch.full((T, layer.dim), float("nan"), dtype=torch.bfloat16, device="cuda")
+    idx = torch.full((T, layer.topk), -1, dtype=torch.int32, device="cuda")
+    w = torch.full((T, layer.topk), float("nan"), device="cuda")
+    x = inp["x"].clone()
+    g = K.KtMoeGraph.mxfp8(cfg, T, x, inp["w_gate"], inp["bias"], q, y, idx, w, ws)
+    try:
+        for step in range(2):
+            gen = torch.Generator(device="cpu").manual_seed(91 + step)
+            x.copy_(torch.randn(x.shape, generator=gen).to(x.dtype))
+            g.launch()
+            assert K.kt_moe_check(ws) == K.KT_OK
+            ws2 = K.alloc_workspace(cfg, T)
+            y2 = torch.empty_like(y)
+            idx2, w2 = torch.empty_like(idx), torch.empty_like(w)
+            K.kt_moe_forward_mxfp8(cfg, T, x, inp["w_gate"], inp["bias"], q["w1q"], q["w3q"],
+                                   q["w2q"], q["sf_up"], q["sf_down"], y2, idx2, w2, ws2)
+            torch.cuda.synchronize()
+            assert torch.equal(idx, idx2) and torch.equal(w, w2) and torch.equal(y, y2), step
+    finally:
+        g.destroy()
