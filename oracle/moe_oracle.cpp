@@ -333,6 +333,55 @@ int oracle_balance_stats(const oracle_cfg* c, int64_t T, const float* scores,
   return rc;
 }
 
+// One rank's part of the expert-parallel forward ("MoE 前向四步": each rank
+// loops over its own experts [expert_begin, expert_end), y is all-reduced over
+// the ranks, and the shared experts' z is added after the reduction):
+//   y_routed = sum over slots j with expert_begin <= idx_j < expert_end of
+//              w_j FFN_{idx_j}(u)                    (slot order, double);
+//   y_shared = sum_s FFN_s(u)                        (if y_shared is not NULL).
+// Weights as for oracle_forward (E+S per-expert pointers; unused ones may be
+// NULL). Both outputs are [n_tok, d] double.
+int oracle_forward_part(const oracle_cfg* c, int64_t T, int dtype, const void* x,
+                        const int32_t* idx, const float* w, const void* const* w1,
+                        const void* const* w3, const void* const* w2, int expert_begin,
+                        int expert_end, int64_t n_tok, const int64_t* tok_ids, double* y_routed,
+                        double* y_shared) {
+  const int d = c->dim, k = c->topk, E = c->n_experts, S = c->n_shared;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t n = 0; n < n_tok; ++n) {
+    const int64_t t = tok_ids[n];
+    if (t < 0 || t >= T) {
+      bad |= 1;
+      continue;
+    }
+    std::vector<double> u(d), acc(d, 0.0), sh(d, 0.0);
+    for (int i = 0; i < d; ++i) u[i] = load_elem(x, dtype, t * d + i);
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[t * k + j];
+      if (e < expert_begin || e >= expert_end) continue;
+      if (e < 0 || e >= E || !w1[e] || !w3[e] || !w2[e]) {
+        bad |= 1;
+        continue;
+      }
+      expert_ffn_acc(*c, dtype, u.data(), w1[e], w3[e], w2[e], (double)w[t * k + j], acc.data());
+    }
+    std::copy(acc.begin(), acc.end(), y_routed + n * d);
+    if (y_shared) {
+      for (int s = 0; s < S; ++s) {
+        const int e = E + s;
+        if (!w1[e] || !w3[e] || !w2[e]) {
+          bad |= 1;
+          continue;
+        }
+        expert_ffn_acc(*c, dtype, u.data(), w1[e], w3[e], w2[e], 1.0, sh.data());
+      }
+      std::copy(sh.begin(), sh.end(), y_shared + n * d);
+    }
+  }
+  return bad ? -1 : 0;
+}
+
 // One expert's SwiGLU hidden vector h = silu(W1 u) * W3 u for n_tok tokens,
 // double. h is [n_tok, I]. Used to localise a mismatch to the first GEMM.
 int oracle_expert_hidden(const oracle_cfg* c, int64_t T, int dtype, const void* x,

@@ -70,6 +70,8 @@ def _load():
             lib.oracle_mx_dequantize.argtypes = [I64, I64, P, P, P]
             lib.oracle_forward_mxfp8.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, ctypes.c_int,
                                                  I64, P, P]
+            lib.oracle_forward_part.argtypes = [CP, I64, ctypes.c_int, P, P, P, P, P, P,
+                                                ctypes.c_int, ctypes.c_int, I64, P, P, P]
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -342,3 +344,38 @@ def forward_mxfp8(cfg: dict, x, idx, w, w1, w3, w2, tok_ids, has_bias: bool,
     if code != 0:
         raise ValueError("oracle_forward_mxfp8: bad token id, missing weights or dims not multiples of 32")
     return y
+
+
+def forward_part(cfg: dict, x, idx, w, w1, w3, w2, tok_ids, has_bias: bool, expert_begin: int,
+                 expert_end: int, shared: bool = True) -> tuple[np.ndarray, np.ndarray | None]:
+    """One rank's part of the expert-parallel forward: (y_routed over experts
+    [expert_begin, expert_end), y_shared or None), each [n, d] float64."""
+    xa, dt = _as_raw(x)
+    T = xa.shape[0]
+    rc = resolve(cfg, has_bias)
+    n_all = rc["n_experts"] + rc["n_shared"]
+    keep = []
+
+    def ptrs(ws):
+        arr = (ctypes.c_void_p * n_all)()
+        for e in range(n_all):
+            if ws[e] is None:
+                arr[e] = None
+                continue
+            a, d2 = _as_raw(ws[e])
+            assert d2 == dt
+            keep.append(a)
+            arr[e] = a.ctypes.data
+        return arr
+
+    tok = np.ascontiguousarray(np.asarray(tok_ids, np.int64))
+    yr = np.empty((tok.shape[0], rc["dim"]), np.float64)
+    ys = np.empty((tok.shape[0], rc["dim"]), np.float64) if shared else None
+    c = _cfg_struct(rc)
+    code = _load().oracle_forward_part(
+        ctypes.byref(c), T, dt, _ptr(xa), _ptr(np.ascontiguousarray(idx, np.int32)),
+        _ptr(np.ascontiguousarray(w, np.float32)), ptrs(w1), ptrs(w3), ptrs(w2),
+        int(expert_begin), int(expert_end), tok.shape[0], _ptr(tok), _ptr(yr), _ptr(ys))
+    if code != 0:
+        raise ValueError("oracle_forward_part: bad token id or missing expert weights")
+    return yr, ys
