@@ -280,6 +280,63 @@ int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, con
                          size_t ws_bytes, void* stream, void* const* stage_events);
 
 /*
+ * Expert-parallel form: the multi-card steps of "MoE 前向四步" in the DeepSeek-V3
+ * model.py notes (each card loops over its own experts only, y is all-reduced
+ * over the cards, the shared experts' z is added); the number of cards is the
+ * expert_parallel_degree setting of the tuning section ("性能调优策略") of the
+ * DeepSeek model-family article (cloud.baidu.com/article/3606489). Per rank:
+ *
+ * kt_moe_forward_local: the gate on all T tokens (every rank computes the same
+ *   routing from the same x, w_gate, bias), then
+ *     y_part[t] = [shared_begin <= t < shared_end] * sum_s FFN_s(u_t)
+ *               + sum over slots j with expert_begin <= idx[t,j] < expert_end
+ *                 of w[t,j] * FFN_idx[t,j](u_t)
+ *   in fp32, without the residual. The shared experts' tokens are split over
+ *   the ranks (the sum over ranks is the same as adding z once after the
+ *   all-reduce, in one message instead of two).
+ *     expert_begin, expert_end   routed experts of this rank, 0 <= b <= e <= E
+ *     shared_begin, shared_end   its tokens of the shared experts, 0 <= b <= e <= T
+ *     w1, w3 [ (expert_end - expert_begin) + S, inter, dim ], w2 [ ..., dim,
+ *       inter ]: slot i < expert_end - expert_begin holds routed expert
+ *       expert_begin + i, the last S slots the shared experts (dtype of cfg)
+ *     y_part  device [T, dim] fp32 (out), 16-B aligned, not overlapping x or the
+ *             workspace; every row is written (zeros for a token with no local
+ *             work)
+ *   x, w_gate, bias, topk outputs, workspace (kt_moe_workspace_size of the full
+ *   config) and errors as for kt_moe_forward; a range outside its bounds:
+ *   KT_ERR_INVALID_CONFIG; an MXFP8 config: KT_ERR_INVALID_CONFIG (use
+ *   kt_moe_forward_local_mxfp8, with codes and scales from
+ *   kt_moe_mxfp8_pack_local on the same local stacks, sized by
+ *   kt_moe_mxfp8_scale_bytes_local: the layouts of kt_moe_mxfp8_pack with the
+ *   group index g running over the local slots).
+ *
+ * kt_moe_ep_finish: after the caller's sum of y_part over the ranks into y_sum
+ *   (an all-reduce; fp32 [T, dim], device), y = y_sum (+ x if add_residual) in
+ *   y's type (as kt_moe_forward). y may be y_sum itself when y is fp32; any
+ *   other overlap: KT_ERR_INVALID_CONFIG. x may be NULL without the residual.
+ */
+int kt_moe_forward_local(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                         const float* bias, int expert_begin, int expert_end,
+                         int64_t shared_begin, int64_t shared_end, const void* w1, const void* w3,
+                         const void* w2, float* y_part, int32_t* topk_idx_out, float* topk_w_out,
+                         void* workspace, size_t ws_bytes, void* stream);
+int kt_moe_forward_local_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x,
+                               const void* w_gate, const float* bias, int expert_begin,
+                               int expert_end, int64_t shared_begin, int64_t shared_end,
+                               const uint8_t* w1q, const uint8_t* w3q, const uint8_t* w2q,
+                               const uint8_t* sf_up, const uint8_t* sf_down, float* y_part,
+                               int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                               size_t ws_bytes, void* stream);
+int kt_moe_ep_finish(const kt_moe_config* cfg, int64_t T, const float* y_sum, const void* x,
+                     void* y, void* stream);
+size_t kt_moe_mxfp8_scale_bytes_local(const kt_moe_config* cfg, int expert_begin, int expert_end,
+                                      int down);
+int kt_moe_mxfp8_pack_local(const kt_moe_config* cfg, int expert_begin, int expert_end,
+                            const void* w1, const void* w3, const void* w2, uint8_t* w1q,
+                            uint8_t* w3q, uint8_t* w2q, uint8_t* sf_up, uint8_t* sf_down,
+                            void* stream);
+
+/*
  * Scores alone: s = the score function of the gate logits, gate step 1 of the
  * "Gate 选专家流程（model.py，五步）" passage of the DeepSeek-V3 model.py notes
  * (sigmoid, or softmax over all experts), for the balance statistics below or

@@ -83,6 +83,10 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
   r->act_bf16 = c->dtype != KT_DTYPE_F32;
   r->fp8 = c->dtype == KT_DTYPE_MXFP8;
   r->chunk_rows = r->fp8 ? kChunkRowsF8 : kChunkRows;
+  r->eb = 0;
+  r->ee = E;
+  r->sb = 0;
+  r->se = (int)T;
   r->add_residual = c->add_residual;
   r->y_fp32 = c->dtype == KT_DTYPE_F32 ? 1 : c->y_fp32;
   r->has_bias = has_bias ? 1 : 0;
@@ -298,7 +302,8 @@ namespace {
 int check_forward_args(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
                        const float* bias, const void* w1, const void* w3, const void* w2,
                        const void* y, const int32_t* topk_idx_out, const float* topk_w_out,
-                       const void* workspace, size_t ws_bytes, Resolved* r) {
+                       const void* workspace, size_t ws_bytes, Resolved* r,
+                       bool y_partial = false) {
   int rc = resolve(cfg, T, bias != nullptr, r);
   if (rc != KT_OK) return rc;
   if (!x || !w_gate || !w1 || !w3 || !w2 || !y) return KT_ERR_NULL;
@@ -311,9 +316,68 @@ int check_forward_args(const kt_moe_config* cfg, int64_t T, const void* x, const
     return KT_ERR_ALIGN;
   const size_t es = r->act_bf16 ? 2 : 4;
   const size_t x_bytes = (size_t)T * r->d * es;
-  const size_t y_bytes = (size_t)T * r->d * (r->y_fp32 ? 4 : es);
+  const size_t y_bytes = (size_t)T * r->d * (r->y_fp32 || y_partial ? 4 : es);
   if (overlaps(x, x_bytes, y, y_bytes) || overlaps(workspace, L.total, y, y_bytes))
     return KT_ERR_INVALID_CONFIG;
+  return KT_OK;
+}
+
+// The forward's launches for a checked config: gate logits and selection, the
+// permutation (after the token quantisation for MXFP8), the two grouped GEMMs,
+// then the combine into y, or (partial) the fp32 sum of this launch's experts.
+// wa/wb/wc: W1, W3, W2 (bf16/fp32) or their codes (MXFP8, with sf_up/sf_down).
+int run_forward(const Resolved& r, int64_t T, const void* x, const void* w_gate,
+                const float* bias, const void* wa, const void* wb, const void* wc,
+                const uint8_t* sf_up, const uint8_t* sf_down, void* y, bool partial,
+                int32_t* topk_idx_out, float* topk_w_out, void* workspace, void* stream,
+                void* const* stage_events) {
+  const Layout L = make_layout(r, T);
+  int sms = 0;
+  int rc = device_info(&sms);
+  if (rc != KT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(ws + L.w);
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+  auto mark = [&](int i) {
+    if (stage_events && stage_events[i])
+      return cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st) == cudaSuccess;
+    return true;
+  };
+  if (!mark(0)) return KT_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_gate_select(r, T, logits, nullptr, bias, idx, w,
+                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), st) != cudaSuccess)
+    return KT_ERR_CUDA;
+  if (!mark(1)) return KT_ERR_CUDA;
+  // MXFP8: tokens to codes and scales first; the permutation copies the codes
+  // into expert order and the scales into each GEMM chunk's blocks.
+  if (r.fp8 && launch_mx_quantize(x, T, r.d, reinterpret_cast<uint8_t*>(ws + L.xq),
+                                  reinterpret_cast<uint8_t*>(ws + L.xs), st) != cudaSuccess)
+    return KT_ERR_CUDA;
+  if (launch_permute(r, T, L, ws, idx, w, x, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (!mark(2)) return KT_ERR_CUDA;
+  cudaError_t e;
+  if (r.fp8)
+    e = launch_experts_mxfp8(r, T, L, ws, wa, wb, sf_up, sms, st, /*up=*/true);
+  else if (r.dtype == KT_DTYPE_BF16)
+    e = launch_experts_bf16(r, T, L, ws, x, wa, wb, sms, st, /*up=*/true);
+  else
+    e = launch_experts_f32(r, T, L, ws, x, wa, wb, wc, sms, st, /*up=*/true);
+  if (e != cudaSuccess || !mark(3)) return KT_ERR_CUDA;
+  if (r.fp8)
+    e = launch_experts_mxfp8(r, T, L, ws, wc, nullptr, sf_down, sms, st, false);
+  else if (r.dtype == KT_DTYPE_BF16)
+    e = launch_experts_bf16(r, T, L, ws, x, wc, nullptr, sms, st, false);
+  else
+    e = launch_experts_f32(r, T, L, ws, x, wa, wb, wc, sms, st, false);
+  if (e != cudaSuccess || !mark(4)) return KT_ERR_CUDA;
+  e = partial ? launch_combine_partial(r, T, L, ws, static_cast<float*>(y), st)
+              : launch_combine(r, T, L, ws, x, y, st);
+  if (e != cudaSuccess || !mark(5)) return KT_ERR_CUDA;
   return KT_OK;
 }
 
@@ -331,40 +395,8 @@ int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
                               workspace, ws_bytes, &r);
   if (rc != KT_OK) return rc;
   if (r.fp8) return KT_ERR_INVALID_CONFIG;   // MXFP8 weights: kt_moe_forward_mxfp8
-  const Layout L = make_layout(r, T);
-  int sms = 0;
-  if ((rc = device_info(&sms)) != KT_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  char* ws = static_cast<char*>(workspace);
-  int* err = reinterpret_cast<int*>(ws + L.err);
-  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
-  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(ws + L.w);
-  float* logits = reinterpret_cast<float*>(ws + L.logits);
-
-  auto mark = [&](int i) {
-    if (stage_events && stage_events[i])
-      return cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st) == cudaSuccess;
-    return true;
-  };
-  if (!mark(0)) return KT_ERR_CUDA;
-  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
-  if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
-  if (launch_gate_select(r, T, logits, nullptr, bias, idx, w,
-                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), st) != cudaSuccess)
-    return KT_ERR_CUDA;
-  if (!mark(1)) return KT_ERR_CUDA;
-  if (launch_permute(r, T, L, ws, idx, w, x, st) != cudaSuccess) return KT_ERR_CUDA;
-  if (!mark(2)) return KT_ERR_CUDA;
-  cudaError_t e = r.dtype == KT_DTYPE_BF16
-                      ? launch_experts_bf16(r, T, L, ws, x, w1, w3, sms, st, /*up=*/true)
-                      : launch_experts_f32(r, T, L, ws, x, w1, w3, w2, sms, st, /*up=*/true);
-  if (e != cudaSuccess || !mark(3)) return KT_ERR_CUDA;
-  e = r.dtype == KT_DTYPE_BF16 ? launch_experts_bf16(r, T, L, ws, x, w2, nullptr, sms, st, false)
-                               : launch_experts_f32(r, T, L, ws, x, w1, w3, w2, sms, st, false);
-  if (e != cudaSuccess || !mark(4)) return KT_ERR_CUDA;
-  if (launch_combine(r, T, L, ws, x, y, st) != cudaSuccess) return KT_ERR_CUDA;
-  if (!mark(5)) return KT_ERR_CUDA;
-  return KT_OK;
+  return run_forward(r, T, x, w_gate, bias, w1, w3, w2, nullptr, nullptr, y, false, topk_idx_out,
+                     topk_w_out, workspace, stream, stage_events);
 }
 
 }  // extern "C"
@@ -469,43 +501,114 @@ int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, con
   if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
     return KT_ERR_INVALID_CONFIG;
   if (!aligned(sf_up, 16) || !aligned(sf_down, 16)) return KT_ERR_ALIGN;
-  const Layout L = make_layout(r, T);
+  return run_forward(r, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y, false, topk_idx_out,
+                     topk_w_out, workspace, stream, stage_events);
+}
+
+// ---------------------------------------------------------------------------
+// Expert-parallel form ("MoE 前向四步"): each rank runs the gate on all tokens,
+// its own routed experts [expert_begin, expert_end) and the shared experts on
+// its share of the tokens [shared_begin, shared_end), into an fp32 partial; the
+// caller sums the partials over the ranks (all-reduce) and kt_moe_ep_finish
+// adds the residual and rounds.
+// ---------------------------------------------------------------------------
+
+static int set_ep_range(Resolved* r, int64_t T, int expert_begin, int expert_end,
+                        int64_t shared_begin, int64_t shared_end) {
+  if (expert_begin < 0 || expert_begin > expert_end || expert_end > r->E)
+    return KT_ERR_INVALID_CONFIG;
+  if (shared_begin < 0 || shared_begin > shared_end || shared_end > T) return KT_ERR_INVALID_CONFIG;
+  r->eb = expert_begin;
+  r->ee = expert_end;
+  r->sb = (int)shared_begin;
+  r->se = (int)shared_end;
+  return KT_OK;
+}
+
+int kt_moe_forward_local(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                         const float* bias, int expert_begin, int expert_end,
+                         int64_t shared_begin, int64_t shared_end, const void* w1, const void* w3,
+                         const void* w2, float* y_part, int32_t* topk_idx_out, float* topk_w_out,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  Resolved r;
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1, w3, w2, y_part, topk_idx_out,
+                              topk_w_out, workspace, ws_bytes, &r, /*y_partial=*/true);
+  if (rc != KT_OK) return rc;
+  if (r.fp8) return KT_ERR_INVALID_CONFIG;   // MXFP8 weights: kt_moe_forward_local_mxfp8
+  if ((rc = set_ep_range(&r, T, expert_begin, expert_end, shared_begin, shared_end)) != KT_OK)
+    return rc;
+  return run_forward(r, T, x, w_gate, bias, w1, w3, w2, nullptr, nullptr, y_part, true,
+                     topk_idx_out, topk_w_out, workspace, stream, nullptr);
+}
+
+int kt_moe_forward_local_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x,
+                               const void* w_gate, const float* bias, int expert_begin,
+                               int expert_end, int64_t shared_begin, int64_t shared_end,
+                               const uint8_t* w1q, const uint8_t* w3q, const uint8_t* w2q,
+                               const uint8_t* sf_up, const uint8_t* sf_down, float* y_part,
+                               int32_t* topk_idx_out, float* topk_w_out, void* workspace,
+                               size_t ws_bytes, void* stream) {
+  Resolved r;
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y_part, topk_idx_out,
+                              topk_w_out, workspace, ws_bytes, &r, /*y_partial=*/true);
+  if (rc != KT_OK) return rc;
+  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
+  if (!sf_up || !sf_down) return KT_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
+    return KT_ERR_INVALID_CONFIG;
+  if (!aligned(sf_up, 16) || !aligned(sf_down, 16)) return KT_ERR_ALIGN;
+  if ((rc = set_ep_range(&r, T, expert_begin, expert_end, shared_begin, shared_end)) != KT_OK)
+    return rc;
+  return run_forward(r, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y_part, true,
+                     topk_idx_out, topk_w_out, workspace, stream, nullptr);
+}
+
+int kt_moe_ep_finish(const kt_moe_config* cfg, int64_t T, const float* y_sum, const void* x,
+                     void* y, void* stream) {
+  Resolved r;
+  int rc = resolve(cfg, T, 0, &r);
+  if (rc != KT_OK) return rc;
+  if (!y_sum || !y || (r.add_residual && !x)) return KT_ERR_NULL;
+  if (!aligned(y_sum, 16) || !aligned(y, 16) || (x && !aligned(x, 16))) return KT_ERR_ALIGN;
+  const size_t y_bytes = (size_t)T * r.d * (r.y_fp32 ? 4 : 2);
+  // In place only where every element is read and written by one thread at the
+  // same address (fp32 y).
+  if (overlaps(y_sum, (size_t)T * r.d * 4, y, y_bytes) && !(y_sum == y && r.y_fp32))
+    return KT_ERR_INVALID_CONFIG;
   int sms = 0;
   if ((rc = device_info(&sms)) != KT_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  char* ws = static_cast<char*>(workspace);
-  int* err = reinterpret_cast<int*>(ws + L.err);
-  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
-  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(ws + L.w);
-  float* logits = reinterpret_cast<float*>(ws + L.logits);
-  auto mark = [&](int i) {
-    if (stage_events && stage_events[i])
-      return cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st) == cudaSuccess;
-    return true;
-  };
-  if (!mark(0)) return KT_ERR_CUDA;
-  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
-  if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
-  if (launch_gate_select(r, T, logits, nullptr, bias, idx, w,
-                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), st) != cudaSuccess)
-    return KT_ERR_CUDA;
-  if (!mark(1)) return KT_ERR_CUDA;
-  // Tokens to MXFP8 (codes and scales of x), then the permutation, which copies
-  // the codes into expert order and the scales into each GEMM chunk's blocks.
-  if (launch_mx_quantize(x, T, r.d, reinterpret_cast<uint8_t*>(ws + L.xq),
-                         reinterpret_cast<uint8_t*>(ws + L.xs), st) != cudaSuccess)
-    return KT_ERR_CUDA;
-  if (launch_permute(r, T, L, ws, idx, w, x, st) != cudaSuccess) return KT_ERR_CUDA;
-  if (!mark(2)) return KT_ERR_CUDA;
-  if (launch_experts_mxfp8(r, T, L, ws, w1q, w3q, sf_up, sms, st, true) != cudaSuccess ||
-      !mark(3))
-    return KT_ERR_CUDA;
-  if (launch_experts_mxfp8(r, T, L, ws, w2q, nullptr, sf_down, sms, st, false) != cudaSuccess ||
-      !mark(4))
-    return KT_ERR_CUDA;
-  if (launch_combine(r, T, L, ws, x, y, st) != cudaSuccess) return KT_ERR_CUDA;
-  if (!mark(5)) return KT_ERR_CUDA;
-  return KT_OK;
+  return launch_ep_finish(r, T, y_sum, x, y, sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KT_OK
+             : KT_ERR_CUDA;
+}
+
+size_t kt_moe_mxfp8_scale_bytes_local(const kt_moe_config* cfg, int expert_begin, int expert_end,
+                                      int down) {
+  Resolved r;
+  if (resolve(cfg, 1, 0, &r) != KT_OK || !r.fp8) return 0;
+  if (set_ep_range(&r, 1, expert_begin, expert_end, 0, 0) != KT_OK) return 0;
+  return mx_packed_bytes(r, down != 0);
+}
+
+int kt_moe_mxfp8_pack_local(const kt_moe_config* cfg, int expert_begin, int expert_end,
+                            const void* w1, const void* w3, const void* w2, uint8_t* w1q,
+                            uint8_t* w3q, uint8_t* w2q, uint8_t* sf_up, uint8_t* sf_down,
+                            void* stream) {
+  Resolved r;
+  int rc = resolve(cfg, 1, 0, &r);
+  if (rc != KT_OK) return rc;
+  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
+  if ((rc = set_ep_range(&r, 1, expert_begin, expert_end, 0, 0)) != KT_OK) return rc;
+  if (!w1 || !w3 || !w2 || !w1q || !w3q || !w2q || !sf_up || !sf_down) return KT_ERR_NULL;
+  if (!aligned(w1, 16) || !aligned(w3, 16) || !aligned(w2, 16) || !aligned(w1q, 16) ||
+      !aligned(w3q, 16) || !aligned(w2q, 16) || !aligned(sf_up, 16) || !aligned(sf_down, 16))
+    return KT_ERR_ALIGN;
+  int sms = 0;
+  if ((rc = device_info(&sms)) != KT_OK) return rc;
+  return launch_mx_pack(r, w1, w3, w2, w1q, w3q, w2q, sf_up, sf_down,
+                        static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KT_OK
+             : KT_ERR_CUDA;
 }
 
 void* kt_moe_static_scratch(void) { return static_scratch_ptr(); }

@@ -8,6 +8,8 @@
 // One CTA per token; 16-byte loads along the hidden dimension.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "ktmoe_internal.cuh"
 
 namespace ktmoe {
@@ -80,7 +82,99 @@ combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __r
   }
 }
 
+// Expert-parallel partial sum (the local expert loop of "MoE 前向四步"): per
+// token, the shared experts if the token is in [sb, se), then the routed slots
+// whose expert is computed here (row_of >= 0), in fp32; no residual.
+__global__ void __launch_bounds__(128)
+combine_partial_kernel(int T_, int k, int S, int d, int sb, int se,
+                       const int32_t* __restrict__ row_of, const float* __restrict__ expert_out,
+                       float4* __restrict__ y) {
+  __shared__ int rows[kMaxShared + kMaxTopk];
+  __shared__ int nrow;
+  const int t = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    if (t >= sb && t < se)
+      for (int s = 0; s < S; ++s) rows[n++] = T_ * k + s * T_ + t;
+    for (int j = 0; j < k; ++j) {
+      const int row = row_of[(int64_t)t * k + j];
+      if (row >= 0) rows[n++] = row;
+    }
+    nrow = n;
+  }
+  __syncthreads();
+  const int nq = d / 4;
+  for (int q = threadIdx.x; q < nq; q += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < nrow; ++j) {
+      const float4 v = reinterpret_cast<const float4*>(expert_out + (int64_t)rows[j] * d)[q];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    y[(int64_t)t * nq + q] = acc;
+  }
+}
+
+// After the sum over ranks ("all_reduce(y)" of "MoE 前向四步", the shared
+// experts' z already inside it): y = y_sum (+ u), in y's type.
+template <bool kBF16X, bool kF32Out>
+__global__ void __launch_bounds__(256)
+ep_finish_kernel(int64_t n4, int add_residual, const float4* __restrict__ y_sum,
+                 const void* __restrict__ x, void* __restrict__ y) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 v = y_sum[i];
+    if (add_residual) {
+      if (kBF16X) {
+        const uint2 u = static_cast<const uint2*>(x)[i];
+        v.x += __uint_as_float(u.x << 16);
+        v.y += __uint_as_float(u.x & 0xffff0000u);
+        v.z += __uint_as_float(u.y << 16);
+        v.w += __uint_as_float(u.y & 0xffff0000u);
+      } else {
+        const float4 u = static_cast<const float4*>(x)[i];
+        v.x += u.x;
+        v.y += u.y;
+        v.z += u.z;
+        v.w += u.w;
+      }
+    }
+    if (kF32Out) {
+      static_cast<float4*>(y)[i] = v;
+    } else {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+      static_cast<uint2*>(y)[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                             *reinterpret_cast<const uint32_t*>(&hi));
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_combine_partial(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                                   float* y_part, cudaStream_t st) {
+  combine_partial_kernel<<<(unsigned)T, 128, 0, st>>>(
+      (int)T, r.k, r.S, r.d, r.sb, r.se, reinterpret_cast<const int32_t*>(ws + L.row_of),
+      reinterpret_cast<const float*>(ws + L.expert_out), reinterpret_cast<float4*>(y_part));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_finish(const Resolved& r, int64_t T, const float* y_sum, const void* x,
+                             void* y, int num_sms, cudaStream_t st) {
+  const int64_t n4 = T * r.d / 4;
+  const unsigned grid = (unsigned)std::min<int64_t>((n4 + 255) / 256, (int64_t)num_sms * 8);
+  const float4* ys = reinterpret_cast<const float4*>(y_sum);
+  if (r.act_bf16 && !r.y_fp32)
+    ep_finish_kernel<true, false><<<grid, 256, 0, st>>>(n4, r.add_residual, ys, x, y);
+  else if (r.act_bf16)
+    ep_finish_kernel<true, true><<<grid, 256, 0, st>>>(n4, r.add_residual, ys, x, y);
+  else
+    ep_finish_kernel<false, true><<<grid, 256, 0, st>>>(n4, r.add_residual, ys, x, y);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* ws, const void* x,
                            void* y, cudaStream_t st) {

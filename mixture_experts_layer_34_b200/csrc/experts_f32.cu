@@ -5,7 +5,8 @@
 // notes), in fp32 FMA arithmetic: TF32 tensor cores would not meet a 1e-4
 // relative tolerance. Tiles of 32 rows x 32 output columns, K slabs of 32 in
 // shared memory; token rows are gathered from x through tok_of (routed) or
-// taken in order (shared experts), so no permuted copy of x is needed.
+// taken in order (shared experts), so no permuted copy of x is needed. Chunks
+// name weight slots; slots below E (the routed-slot count passed in) are routed.
 #include <cmath>
 
 #include "ktmoe_internal.cuh"
@@ -143,7 +144,7 @@ cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, ch
   const int grid = num_sms * 4;
   if (up) {
     up_f32_kernel<<<grid, 256, 0, st>>>(
-        reinterpret_cast<const Chunk*>(ws + L.chunks), meta + 0, r.E, r.d, r.I,
+        reinterpret_cast<const Chunk*>(ws + L.chunks), meta + 0, routed_slots(r), r.d, r.I,
         static_cast<const float*>(x), static_cast<const float*>(w1), static_cast<const float*>(w3),
         reinterpret_cast<const int32_t*>(ws + L.tok_of), reinterpret_cast<float*>(ws + L.hidden));
     return cudaGetLastError();

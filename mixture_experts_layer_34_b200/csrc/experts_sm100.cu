@@ -1091,7 +1091,7 @@ cudaError_t prepare_grouped_gemm() {
 cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                 const void* x, const void* wa, const void* wb, int num_sms,
                                 cudaStream_t st, bool up) {
-  const int NG = r.E + r.S;
+  const int NG = weight_slots(r);
   const int64_t R = T * (r.k + r.S);     // hidden rows
   const int64_t Rr = T * r.k;            // routed rows
   const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.meta);
@@ -1100,7 +1100,7 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
   a.implicit_rows = 0;
   a.n_routed_rows = (int)Rr;
   a.err = reinterpret_cast<int*>(ws + L.err);
-  a.E = r.E;
+  a.E = routed_slots(r);
   const int grid = pair_grid(num_sms, 0);
   TmaMaps M;
   memset(&M, 0, sizeof(M));
@@ -1152,7 +1152,7 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
 cudaError_t launch_experts_mxfp8(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                  const void* wa, const void* wb, const uint8_t* sf, int num_sms,
                                  cudaStream_t st, bool up) {
-  const int NG = r.E + r.S;
+  const int NG = weight_slots(r);
   const int64_t R = T * (r.k + r.S);     // hidden rows
   const int64_t Rr = T * r.k;            // routed rows
   const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.meta);
@@ -1161,7 +1161,7 @@ cudaError_t launch_experts_mxfp8(const Resolved& r, int64_t T, const Layout& L, 
   a.implicit_rows = 0;
   a.n_routed_rows = (int)Rr;
   a.err = reinterpret_cast<int*>(ws + L.err);
-  a.E = r.E;
+  a.E = routed_slots(r);
   a.tma3d = 1;
   const int grid = pair_grid(num_sms, 0);
   TmaMaps M;

@@ -53,6 +53,9 @@ struct Resolved {
   int act_bf16;     // tokens, gate weights and output in bf16 (KT_DTYPE_BF16 / MXFP8)
   int fp8;          // expert weights in MXFP8
   int chunk_rows;   // token rows per GEMM chunk: kChunkRows, or kChunkRowsF8 for MXFP8
+  int eb, ee;       // routed experts computed here: [eb, ee) (all: [0, E)); their weights
+                    // are the first ee - eb slots of w1/w3/w2, the shared ones follow
+  int sb, se;       // tokens the shared experts run on here: [sb, se) (all: [0, T))
   int add_residual;
   int y_fp32;       // y in fp32 (else in dtype)
   int has_bias;
@@ -62,11 +65,15 @@ struct Resolved {
 // Rows live in the "hidden-row" space: routed rows 0..T*k-1 sorted by expert,
 // then shared expert s at T*k + s*T + t.
 struct Chunk {
-  int32_t group;    // 0..E-1 routed, E..E+S-1 shared
+  int32_t group;    // weight slot: 0..ee-eb-1 routed expert eb + slot, then the shared ones
   int32_t row0;     // first hidden row of the chunk
   int32_t nrows;    // rows in the chunk (<= chunk size)
   int32_t src_row0; // first activation row: permuted-x row (routed) or token (shared)
 };
+
+// Weight slots of a launch: the routed experts computed here, then the shared ones.
+inline int routed_slots(const Resolved& r) { return r.ee - r.eb; }
+inline int weight_slots(const Resolved& r) { return r.ee - r.eb + r.S; }
 
 // Byte offsets of the workspace's internal buffers.
 struct Layout {
@@ -144,6 +151,12 @@ cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, ch
                                int num_sms, cudaStream_t st, bool up);
 cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* ws,
                            const void* x, void* y, cudaStream_t st);
+// Expert-parallel forms: this launch's experts summed per token in fp32 (no
+// residual), and the finish after the sum over ranks.
+cudaError_t launch_combine_partial(const Resolved& r, int64_t T, const Layout& L, char* ws,
+                                   float* y_part, cudaStream_t st);
+cudaError_t launch_ep_finish(const Resolved& r, int64_t T, const float* y_sum, const void* x,
+                             void* y, int num_sms, cudaStream_t st);
 
 // MXFP8 (mxfp8.cu).
 cudaError_t launch_mx_quantize(const void* src, int64_t rows, int64_t K, uint8_t* codes,

@@ -107,7 +107,7 @@ cudaError_t launch_mx_quantize(const void* src, int64_t rows, int64_t K, uint8_t
 }
 
 size_t mx_packed_bytes(const Resolved& r, bool down) {
-  const size_t NG = (size_t)(r.E + r.S);
+  const size_t NG = (size_t)weight_slots(r);
   if (down) return NG * ((r.d + 255) / 256) * 2 * (r.I / 128) * 512;
   return NG * (r.I / 128) * 2 * (r.d / 128) * 512;
 }
@@ -115,7 +115,7 @@ size_t mx_packed_bytes(const Resolved& r, bool down) {
 cudaError_t launch_mx_pack(const Resolved& r, const void* w1, const void* w3, const void* w2,
                            uint8_t* w1q, uint8_t* w3q, uint8_t* w2q, uint8_t* sf_up,
                            uint8_t* sf_down, cudaStream_t st) {
-  const int64_t NG = r.E + r.S;
+  const int64_t NG = weight_slots(r);
   // Blocks of packed rows past d (a last down feature tile of 128 rows) stay 0.
   cudaError_t e = cudaMemsetAsync(sf_down, 0, mx_packed_bytes(r, true), st);
   if (e != cudaSuccess) return e;

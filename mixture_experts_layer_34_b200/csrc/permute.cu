@@ -122,7 +122,8 @@ __device__ void fill_tiles(int2* __restrict__ tiles, int F, int NG, const int* c
 }
 
 __global__ void __launch_bounds__(kScanThreads)
-permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int chunk_rows,
+permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int chunk_rows, int eb,
+                    int ee, int sb, int se,
                     const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base,
                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                     Chunk* __restrict__ chunks, int2* __restrict__ tiles_up,
@@ -136,19 +137,21 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
   __shared__ int lb[NGMAX + 1];
   const int tid = threadIdx.x;
   const int NG = E + S;
-  // Per-expert totals over the chunks; shared experts hold all T tokens.
+  // Per-expert totals over the chunks; shared experts hold tokens [sb, se) (all
+  // T unless the caller splits them); routed experts outside [eb, ee) are
+  // computed elsewhere and hold none.
   if (tid < NG) {
     int run = 0;
-    if (tid < E)
+    if (tid >= E)
+      run = se - sb;
+    else if (tid >= eb && tid < ee)
       for (int c = 0; c < nperm; ++c) run += chunk_counts[(int64_t)c * E + tid];
-    else
-      run = T_;
     tot[tid] = run;
     rows0[tid] = run;
     counts[tid] = run;
   }
   __syncthreads();
-  // Routed experts: rows [0, T*k); shared expert s: rows T*k + s*T.
+  // Routed experts: rows [0, T*k); shared expert s: rows T*k + s*T + t.
   block_exclusive_scan(rows0, E);
   if (tid >= E && tid < NG) rows0[tid] = T_ * k + (tid - E) * T_;
   __syncthreads();
@@ -176,11 +179,15 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
     meta[4] = 0;   // down GEMM tile counter
   }
   __syncthreads();
+  // The chunks name weight slots: routed expert g in slot g - eb, shared expert
+  // E + s in slot ee - eb + s.
   for (int i = tid; i < n_chunks; i += blockDim.x) {
     const int g = find_group(cb, NG, i);
     const int r = (i - cb[g]) * chunk_rows;
-    const int src0 = g < E ? rows0[g] : 0;
-    chunks[i] = Chunk{g, rows0[g] + r, min(chunk_rows, tot[g] - r), src0 + r};
+    const int slot = g < E ? g - eb : ee - eb + (g - E);
+    const int row0 = g < E ? rows0[g] : rows0[g] + sb;
+    const int src0 = g < E ? rows0[g] : sb;
+    chunks[i] = Chunk{slot, row0 + r, min(chunk_rows, tot[g] - r), src0 + r};
   }
   fill_tiles(tiles_up, Fu, NG, cb, hb, lb, tot);
   fill_tiles(tiles_dn, Fd, NG, cb, hb, lb, tot);
@@ -191,7 +198,8 @@ enum { kNoCopy = 0, kCopyBf16 = 1, kCopyF8 = 2 };
 
 template <int kMode>
 __global__ void __launch_bounds__(256)
-permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
+permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int eb, int ee, int sb,
+                       int se,
                        const int32_t* __restrict__ idx, const float* __restrict__ w,
                        const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
                        const int32_t* __restrict__ gchunk0, int32_t* __restrict__ row_of,
@@ -215,6 +223,11 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
   for (int q = threadIdx.x; q < nent; q += blockDim.x) {
     const int tl = q / k;
     const int e = idx[(int64_t)t0 * k + q];
+    if (e < eb || e >= ee) {   // an expert computed elsewhere: no row here
+      row_of[(int64_t)t0 * k + q] = -1;
+      srow[q] = -1;
+      continue;
+    }
     const int rank = __popc(mask[e] & ((1u << tl) - 1u));
     const int row = chunk_base[(int64_t)c * E + e] + rank;
     row_of[(int64_t)t0 * k + q] = row;
@@ -232,7 +245,10 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
     const uint4* src = x + (int64_t)(t0 + tl) * nchunk;
     for (int q = lane; q < nchunk; q += 32) {
       const uint4 v = src[q];
-      for (int j = 0; j < k; ++j) xperm[(int64_t)srow[tl * k + j] * nchunk + q] = v;
+      for (int j = 0; j < k; ++j) {
+        const int row = srow[tl * k + j];
+        if (row >= 0) xperm[(int64_t)row * nchunk + q] = v;
+      }
     }
   }
   if (kMode != kCopyF8) return;
@@ -245,10 +261,12 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
     int g, rel;
     if (j < k) {
       g = idx[(int64_t)(t0 + tl) * k + j];
+      if (srow[tl * k + j] < 0) continue;
       rel = srow[tl * k + j] - offsets[g];
     } else {
+      if (t0 + tl < sb || t0 + tl >= se) continue;
       g = E + (j - k);
-      rel = t0 + tl;
+      rel = t0 + tl - sb;
     }
     const int64_t chunk = gchunk0[g] + rel / chunk_rows;
     const int m = rel % chunk_rows;
@@ -265,7 +283,8 @@ cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* 
                            const int32_t* idx, const float* w, const void* x, cudaStream_t st) {
   auto I32 = [&](size_t off) { return reinterpret_cast<int32_t*>(ws + off); };
   permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
-      r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows,
+      r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows, r.eb,
+      r.ee, r.sb, r.se,
       I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts), I32(L.offsets),
       reinterpret_cast<Chunk*>(ws + L.chunks), reinterpret_cast<int2*>(ws + L.tiles_up),
       reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0));
@@ -276,18 +295,18 @@ cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* 
   const int32_t* base = I32(L.chunk_base);
   if (r.fp8)
     permute_scatter_kernel<kCopyF8><<<grid, 256, 0, st>>>(
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(ws + L.xq),
         reinterpret_cast<uint4*>(ws + L.xperm), reinterpret_cast<const uint8_t*>(ws + L.xs),
         reinterpret_cast<uint8_t*>(ws + L.tok_sf));
   else if (r.dtype == KT_DTYPE_BF16)
     permute_scatter_kernel<kCopyBf16><<<grid, 256, 0, st>>>(
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(x),
         reinterpret_cast<uint4*>(ws + L.xperm), nullptr, nullptr);
   else
     permute_scatter_kernel<kNoCopy><<<grid, 256, 0, st>>>(
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr, nullptr);
   return cudaGetLastError();
 }

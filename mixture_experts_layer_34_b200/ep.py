@@ -1,0 +1,125 @@
+"""Expert-parallel MoE layer over a torch.distributed process group.
+
+The multi-card form of "MoE 前向四步" in the DeepSeek-V3 model.py notes
+(73biji.xyz/llm_pp_dsv3): each card loops over its own experts only, the
+partial outputs are all-reduced, and the shared experts' z is added. The number
+of cards is the expert_parallel_degree setting of the tuning section of the
+DeepSeek model-family article (cloud.baidu.com/article/3606489).
+
+Per rank:
+  * the routed experts of one contiguous range (``expert_range``), held as a
+    local weight stack: those experts, then the shared ones (``local_stack``);
+  * the gate on all tokens (every rank routes the same tokens identically), the
+    local experts on their tokens, and the shared experts on this rank's share
+    of the tokens (``token_range``), summed in fp32 by ``kt_moe_forward_local``;
+  * one all-reduce of that fp32 [T, dim] partial (NCCL over NVLink/NVSwitch on
+    GPUs), which sums routed outputs and z in one message;
+  * ``kt_moe_ep_finish``: the residual and the rounding to y's type.
+
+Every arithmetic step runs in libktmoe.so's kernels; this module holds the
+partition, the local weight stacks, the buffers and the collective.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import ktmoe as K
+
+
+def split_range(n: int, world: int, rank: int) -> tuple[int, int]:
+    """[begin, end) of rank's share of n items in world contiguous parts; the
+    first n % world parts hold one more item."""
+    if world < 1 or not 0 <= rank < world or n < 0:
+        raise ValueError(f"bad split: n={n} world={world} rank={rank}")
+    base, extra = divmod(n, world)
+    begin = rank * base + min(rank, extra)
+    return begin, begin + base + (1 if rank < extra else 0)
+
+
+def expert_range(n_experts: int, world: int, rank: int) -> tuple[int, int]:
+    """Routed experts of one rank."""
+    return split_range(n_experts, world, rank)
+
+
+def token_range(T: int, world: int, rank: int) -> tuple[int, int]:
+    """Tokens one rank runs the shared experts on."""
+    return split_range(T, world, rank)
+
+
+def local_stack(w, n_experts: int, n_shared: int, begin: int, end: int):
+    """A rank's weight slots from a stacked [E + S, ...] weight: routed experts
+    [begin, end), then the S shared experts, as one contiguous tensor."""
+    return torch.cat([w[begin:end], w[n_experts:n_experts + n_shared]]).contiguous()
+
+
+class ExpertParallelMoE:
+    """One rank of the expert-parallel layer.
+
+    cfg: the full layer's kt_moe_config (all E routed experts). w1/w3/w2: the
+    full stacked weights [E + S, ...] (sliced here), or, with
+    ``weights_are_local``, this rank's stack already. With an MXFP8 config the
+    local stacks (bf16) are packed once here.
+    """
+
+    def __init__(self, cfg, w_gate, bias, w1, w3, w2, rank: int, world: int, group=None,
+                 weights_are_local: bool = False):
+        self.cfg, self.rank, self.world, self.group = cfg, rank, world, group
+        E, S = cfg.n_experts, cfg.n_shared
+        self.eb, self.ee = expert_range(E, world, rank)
+        if not weights_are_local:
+            w1, w3, w2 = (local_stack(w, E, S, self.eb, self.ee) for w in (w1, w3, w2))
+        n_slots = self.ee - self.eb + S
+        for w in (w1, w3, w2):
+            if w.shape[0] != n_slots:
+                raise ValueError(f"local stack has {w.shape[0]} slots, expected {n_slots}")
+        self.w_gate, self.bias = w_gate, bias
+        self.mxfp8 = cfg.dtype == K.KT_DTYPE_MXFP8
+        if self.mxfp8:
+            self.q = K.pack_mxfp8_local(cfg, self.eb, self.ee, w1, w3, w2)
+            self.w1 = self.w3 = self.w2 = None
+        else:
+            self.q = None
+            self.w1, self.w3, self.w2 = w1, w3, w2
+        self._ws: dict[int, torch.Tensor] = {}
+        self._part: dict[int, torch.Tensor] = {}
+
+    def shared_range(self, T: int) -> tuple[int, int]:
+        return token_range(T, self.world, self.rank)
+
+    def buffers(self, T: int, device) -> tuple[torch.Tensor, torch.Tensor]:
+        """The workspace and the fp32 partial for T tokens (allocated once per T)."""
+        if T not in self._ws:
+            self._ws[T] = K.alloc_workspace(self.cfg, T, device)
+            self._part[T] = torch.empty((T, self.cfg.dim), dtype=torch.float32, device=device)
+        return self._ws[T], self._part[T]
+
+    def local(self, x, part, topk_idx=None, topk_w=None):
+        """This rank's fp32 partial into ``part`` (every row written)."""
+        T = x.shape[0]
+        ws, _ = self.buffers(T, x.device)
+        sb, se = self.shared_range(T)
+        if self.mxfp8:
+            q = self.q
+            K.kt_moe_forward_local_mxfp8(self.cfg, T, x, self.w_gate, self.bias, self.eb, self.ee,
+                                         sb, se, q["w1q"], q["w3q"], q["w2q"], q["sf_up"],
+                                         q["sf_down"], part, topk_idx, topk_w, ws)
+        else:
+            K.kt_moe_forward_local(self.cfg, T, x, self.w_gate, self.bias, self.eb, self.ee, sb,
+                                   se, self.w1, self.w3, self.w2, part, topk_idx, topk_w, ws)
+
+    def reduce(self, part):
+        """Sum of the partials over the ranks, in place."""
+        if self.world > 1:
+            dist.all_reduce(part, op=dist.ReduceOp.SUM, group=self.group)
+
+    def finish(self, part, x, y):
+        K.kt_moe_ep_finish(self.cfg, x.shape[0], part, x, y)
+
+    def forward(self, x, y, topk_idx=None, topk_w=None):
+        """y = the layer's output for tokens x (the same x on every rank)."""
+        _, part = self.buffers(x.shape[0], x.device)
+        self.local(x, part, topk_idx, topk_w)
+        self.reduce(part)
+        self.finish(part, x, y)
+        return y

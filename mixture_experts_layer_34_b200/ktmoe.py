@@ -29,7 +29,9 @@ EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_fo
            "kt_moe_scores", "kt_moe_bias_update", "kt_moe_balance_workspace_size",
            "kt_moe_balance_stats", "kt_moe_graph_create", "kt_moe_graph_launch",
            "kt_moe_graph_destroy", "kt_moe_mxfp8_quantize", "kt_moe_mxfp8_scale_bytes",
-           "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8", "kt_moe_graph_create_mxfp8")
+           "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8", "kt_moe_graph_create_mxfp8",
+           "kt_moe_forward_local", "kt_moe_forward_local_mxfp8", "kt_moe_ep_finish",
+           "kt_moe_mxfp8_scale_bytes_local", "kt_moe_mxfp8_pack_local")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -120,6 +122,19 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_forward_mxfp8.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, P, P, P,
                                                ctypes.c_size_t, P, P]
             L.kt_moe_forward_mxfp8.restype = ctypes.c_int
+            C = ctypes.c_int
+            L.kt_moe_forward_local.argtypes = [CP, I64, P, P, P, C, C, I64, I64, P, P, P, P, P, P,
+                                               P, ctypes.c_size_t, P]
+            L.kt_moe_forward_local.restype = ctypes.c_int
+            L.kt_moe_forward_local_mxfp8.argtypes = [CP, I64, P, P, P, C, C, I64, I64, P, P, P, P,
+                                                     P, P, P, P, P, ctypes.c_size_t, P]
+            L.kt_moe_forward_local_mxfp8.restype = ctypes.c_int
+            L.kt_moe_ep_finish.argtypes = [CP, I64, P, P, P, P]
+            L.kt_moe_ep_finish.restype = ctypes.c_int
+            L.kt_moe_mxfp8_scale_bytes_local.argtypes = [CP, C, C, C]
+            L.kt_moe_mxfp8_scale_bytes_local.restype = ctypes.c_size_t
+            L.kt_moe_mxfp8_pack_local.argtypes = [CP, C, C, P, P, P, P, P, P, P, P, P]
+            L.kt_moe_mxfp8_pack_local.restype = ctypes.c_int
             L.kt_moe_version.argtypes = []
             L.kt_moe_version.restype = ctypes.c_int
             _lib = L
@@ -321,6 +336,70 @@ def kt_moe_forward_mxfp8(cfg, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down,
                                     _ptr(workspace), _nbytes(workspace), _stream(stream), ev)
     if rc != KT_OK:
         raise KtMoeError("kt_moe_forward_mxfp8", rc)
+
+
+def kt_moe_forward_local(cfg, T, x, w_gate, bias, expert_begin, expert_end, shared_begin,
+                         shared_end, w1, w3, w2, y_part, topk_idx_out, topk_w_out, workspace,
+                         stream=None):
+    """One rank's part of the expert-parallel forward: fp32 y_part from routed
+    experts [expert_begin, expert_end) (local weight slots, then the shared
+    experts) and the shared experts on tokens [shared_begin, shared_end)."""
+    rc = lib().kt_moe_forward_local(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias),
+                                    int(expert_begin), int(expert_end), int(shared_begin),
+                                    int(shared_end), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y_part),
+                                    _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
+                                    _nbytes(workspace), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_forward_local", rc)
+
+
+def kt_moe_forward_local_mxfp8(cfg, T, x, w_gate, bias, expert_begin, expert_end, shared_begin,
+                               shared_end, w1q, w3q, w2q, sf_up, sf_down, y_part, topk_idx_out,
+                               topk_w_out, workspace, stream=None):
+    rc = lib().kt_moe_forward_local_mxfp8(
+        ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias), int(expert_begin),
+        int(expert_end), int(shared_begin), int(shared_end), _ptr(w1q), _ptr(w3q), _ptr(w2q),
+        _ptr(sf_up), _ptr(sf_down), _ptr(y_part), _ptr(topk_idx_out), _ptr(topk_w_out),
+        _ptr(workspace), _nbytes(workspace), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_forward_local_mxfp8", rc)
+
+
+def kt_moe_ep_finish(cfg, T, y_sum, x, y, stream=None):
+    """y = y_sum (+ x with the residual) in y's type, after the sum over ranks."""
+    rc = lib().kt_moe_ep_finish(ctypes.byref(cfg), int(T), _ptr(y_sum), _ptr(x), _ptr(y),
+                                _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_ep_finish", rc)
+
+
+def kt_moe_mxfp8_scale_bytes_local(cfg, expert_begin, expert_end, down) -> int:
+    return int(lib().kt_moe_mxfp8_scale_bytes_local(ctypes.byref(cfg), int(expert_begin),
+                                                    int(expert_end), int(bool(down))))
+
+
+def kt_moe_mxfp8_pack_local(cfg, expert_begin, expert_end, w1, w3, w2, w1q, w3q, w2q, sf_up,
+                            sf_down, stream=None):
+    rc = lib().kt_moe_mxfp8_pack_local(ctypes.byref(cfg), int(expert_begin), int(expert_end),
+                                       _ptr(w1), _ptr(w3), _ptr(w2), _ptr(w1q), _ptr(w3q),
+                                       _ptr(w2q), _ptr(sf_up), _ptr(sf_down), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_mxfp8_pack_local", rc)
+
+
+def pack_mxfp8_local(cfg, expert_begin, expert_end, w1, w3, w2, stream=None) -> dict:
+    """pack_mxfp8 for one rank's local stacks (routed experts [expert_begin,
+    expert_end), then the shared ones)."""
+    import torch
+    w13 = torch.empty((2,) + tuple(w1.shape), dtype=torch.uint8, device=w1.device)
+    sb = lambda down: kt_moe_mxfp8_scale_bytes_local(cfg, expert_begin, expert_end, down)
+    out = dict(w1q=w13[0], w3q=w13[1],
+               w2q=torch.empty(w2.shape, dtype=torch.uint8, device=w2.device),
+               sf_up=torch.empty(sb(False), dtype=torch.uint8, device=w1.device),
+               sf_down=torch.empty(sb(True), dtype=torch.uint8, device=w1.device))
+    kt_moe_mxfp8_pack_local(cfg, expert_begin, expert_end, w1, w3, w2, out["w1q"], out["w3q"],
+                            out["w2q"], out["sf_up"], out["sf_down"], stream)
+    return out
 
 
 KT_STAGE_EVENTS = 6

@@ -202,6 +202,62 @@ def test_graph_create_host_side_errors():
     L.kt_moe_graph_destroy(None)
 
 
+def test_expert_parallel_host_side_errors():
+    """kt_moe_forward_local / _mxfp8, kt_moe_ep_finish and the local pack check
+    ranges, pointers and dtypes on the host (fake pointers, never dereferenced)."""
+    layer = W.BY_NAME["small_sig_bias"]
+    cfg = K.config_for(layer)
+    L = K.lib()
+    V = ctypes.c_void_p
+    T, E = layer.T, layer.n_experts
+    need = K.kt_moe_workspace_size(cfg, T)
+    ptr = lambda i: V(0x10000 * (i + 1))
+
+    def local(eb, ee, sb, se, ws_bytes=need, y=ptr(7), x=ptr(0)):
+        return L.kt_moe_forward_local(ctypes.byref(cfg), T, x, ptr(1), ptr(2), eb, ee, sb, se,
+                                      ptr(3), ptr(4), ptr(5), y, None, None, V(0x7000000),
+                                      ws_bytes, None)
+
+    for eb, ee, sb, se in ((-1, 4, 0, T), (5, 4, 0, T), (0, E + 1, 0, T), (0, E, -1, T),
+                           (0, E, 10, 9), (0, E, 0, T + 1)):
+        assert local(eb, ee, sb, se) == K.KT_ERR_INVALID_CONFIG, (eb, ee, sb, se)
+    assert local(0, E, 0, T, ws_bytes=need - 1) == K.KT_ERR_WORKSPACE
+    assert local(0, E, 0, T, y=None) == K.KT_ERR_NULL
+    assert local(0, E, 0, T, x=None) == K.KT_ERR_NULL
+    assert local(0, E, 0, T, y=V(0x80008)) == K.KT_ERR_ALIGN
+    # y_part is fp32 [T, dim]: overlapping x over that size is rejected
+    assert local(0, E, 0, T, y=V(0x10000 + 16)) == K.KT_ERR_INVALID_CONFIG
+    # the bf16 entry rejects an MXFP8 config and the MXFP8 entry a bf16 one
+    cf8 = K.config_for(W.BY_NAME["small_sig_bias_mxfp8"])
+    need8 = K.kt_moe_workspace_size(cf8, 300)
+    assert L.kt_moe_forward_local(ctypes.byref(cf8), 300, ptr(0), ptr(1), ptr(2), 0, 4, 0, 300,
+                                  ptr(3), ptr(4), ptr(5), ptr(7), None, None, V(0x7000000),
+                                  need8, None) == K.KT_ERR_INVALID_CONFIG
+    f8 = lambda c, w1q, w3q: L.kt_moe_forward_local_mxfp8(
+        ctypes.byref(c), 300, ptr(0), ptr(1), ptr(2), 0, 4, 0, 300, w1q, w3q, ptr(5), ptr(8),
+        ptr(9), ptr(7), None, None, V(0x7000000), max(need, need8), None)
+    assert f8(cfg, ptr(3), ptr(4)) == K.KT_ERR_INVALID_CONFIG
+    assert f8(cf8, ptr(4), ptr(3)) == K.KT_ERR_INVALID_CONFIG     # W3 codes below W1's
+    # finish: NULLs, alignment, overlap (in place only for fp32 y)
+    fin = lambda c, ys, x, y: L.kt_moe_ep_finish(ctypes.byref(c), T, ys, x, y, None)
+    assert fin(cfg, None, ptr(0), ptr(1)) == K.KT_ERR_NULL
+    assert fin(cfg, ptr(2), ptr(0), V(0x30008)) == K.KT_ERR_ALIGN
+    assert fin(cfg, ptr(2), ptr(0), ptr(2)) == K.KT_ERR_INVALID_CONFIG      # bf16 y in place
+    res = K.config_for(W.BY_NAME["small_odd_dims"])                        # with the residual
+    assert L.kt_moe_ep_finish(ctypes.byref(res), 77, ptr(2), None, ptr(1), None) == K.KT_ERR_NULL
+    # local pack sizes follow the slot count; bad ranges give 0 / an error
+    full = K.kt_moe_mxfp8_scale_bytes(cf8, False)
+    n_all = 32 + 1
+    assert K.kt_moe_mxfp8_scale_bytes_local(cf8, 0, 32, False) == full
+    assert K.kt_moe_mxfp8_scale_bytes_local(cf8, 8, 16, False) == full // n_all * 9
+    assert K.kt_moe_mxfp8_scale_bytes_local(cf8, 8, 16, True) == \
+        K.kt_moe_mxfp8_scale_bytes(cf8, True) // n_all * 9
+    assert K.kt_moe_mxfp8_scale_bytes_local(cf8, 16, 8, False) == 0
+    assert K.kt_moe_mxfp8_scale_bytes_local(cfg, 0, 8, False) == 0
+    assert L.kt_moe_mxfp8_pack_local(ctypes.byref(cf8), 0, 33, *[ptr(i) for i in range(8)],
+                                     None) == K.KT_ERR_INVALID_CONFIG
+
+
 def test_strerror_covers_codes():
     for code in range(-8, 1):
         assert K.strerror(code) and K.strerror(code) != "unknown error code"

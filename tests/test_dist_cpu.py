@@ -1,9 +1,17 @@
-"""Multi-rank host logic of bench.py on CPU (gloo, world size 2).
+"""Multi-rank host logic on CPU (gloo, world size 2).
 
-The layer shards as data-parallel replicas over tokens: no collective on the
-data path. What the ranks share is host logic: barriers, the max over ranks of
-the device times, per-rank token seeds, and the reference arm running on rank 0
-only. These run as two gloo processes on 127.0.0.1.
+bench.py shards the layer as data-parallel replicas over tokens: no collective
+on the data path. What the ranks share there is host logic: barriers, the max
+over ranks of the device times, per-rank token seeds, and the reference arm
+running on rank 0 only.
+
+The expert-parallel layer (mixture_experts_layer_34_b200.ep) has one exchange,
+the all-reduce of the fp32 partials. Its host logic (the expert and token
+splits, the local weight stacks, the reduction and the finish order) runs here
+over gloo with the oracle standing in for the two kernels, and the sum must be
+the oracle's full forward.
+
+These run as two gloo processes on 127.0.0.1.
 """
 from __future__ import annotations
 
@@ -45,11 +53,12 @@ def _worker(rank, world, port, q):
         q.put((rank, repr(e), None))
 
 
-def _run(world=2):
+def _run(world=2, target=None):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    target = target or _worker
+    procs = [ctx.Process(target=target, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     out = [q.get(timeout=120) for _ in range(world)]
@@ -78,3 +87,104 @@ def test_bench_rejects_too_few_warmup_steps():
     import bench
     with pytest.raises(SystemExit):
         bench.parse_args(["--warmup", "2"])
+
+
+# ----------------------------------------------------------------------------
+# Expert-parallel layer
+# ----------------------------------------------------------------------------
+
+def test_splits_cover_every_item_once():
+    from mixture_experts_layer_34_b200 import ep
+    for n in (0, 1, 7, 16, 256, 257):
+        for world in range(1, 10):
+            parts = [ep.split_range(n, world, r) for r in range(world)]
+            assert parts[0][0] == 0 and parts[-1][1] == n
+            for (b0, e0), (b1, e1) in zip(parts, parts[1:]):
+                assert e0 == b1
+            sizes = [e - b for b, e in parts]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        ep.split_range(8, 2, 2)
+
+
+def test_local_stack_slots():
+    from mixture_experts_layer_34_b200 import ep
+    w = torch.arange(10).view(10, 1)            # E = 8 routed + S = 2 shared
+    assert ep.local_stack(w, 8, 2, 3, 6).view(-1).tolist() == [3, 4, 5, 8, 9]
+    assert ep.local_stack(w, 8, 2, 4, 4).view(-1).tolist() == [8, 9]
+
+
+def _ep_layer():
+    from mixture_experts_layer_34_b200 import workloads as W
+    layer = W.BY_NAME["small_sig_bias"]
+    return layer, W.make_layer(layer, "cpu")
+
+
+def _ep_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import numpy as np
+    import oracle.oracle as O
+    from mixture_experts_layer_34_b200 import ep
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        layer, inp = _ep_layer()
+        fields = layer.kernel_fields()
+        E, S = layer.n_experts, layer.n_shared
+        toks = list(range(0, layer.T, 5))
+        x = inp["x"][toks].contiguous()
+        og = O.gate(fields, inp["x"], inp["w_gate"], inp["bias"])
+        idx, w = og["idx"][toks], og["w"][toks]
+
+        class OracleRank(ep.ExpertParallelMoE):
+            """The two kernels replaced by the oracle, on this rank's local stacks."""
+
+            def local(self, x, part, topk_idx=None, topk_w=None):
+                n_local = self.ee - self.eb
+                lists = []
+                for stack in (self.w1, self.w3, self.w2):
+                    full = [None] * (E + S)
+                    for i in range(n_local):
+                        full[self.eb + i] = stack[i]
+                    for s in range(S):
+                        full[E + s] = stack[n_local + s]
+                    lists.append(full)
+                T = x.shape[0]
+                yr, _ = O.forward_part(fields, x, idx, w, *lists, range(T), True, self.eb,
+                                       self.ee, shared=False)
+                sb, se = self.shared_range(T)
+                part.copy_(torch.from_numpy(yr))
+                if se > sb:
+                    _, ys = O.forward_part(fields, x, idx, w, *lists, range(sb, se), True,
+                                           self.eb, self.ee)
+                    part[sb:se] += torch.from_numpy(ys)
+
+            def buffers(self, T, device):
+                return None, self._part.setdefault(T, torch.empty(T, layer.dim,
+                                                                  dtype=torch.float64))
+
+            def finish(self, part, x, y):
+                y.copy_(part + (x.to(torch.float64) if layer.add_residual else 0))
+
+        cfg = K.config_for(layer)
+        m = OracleRank(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], rank,
+                       world)
+        y = torch.empty(x.shape[0], layer.dim, dtype=torch.float64)
+        m.forward(x, y)
+        dist.destroy_process_group()
+        ref = O.forward(fields, x, idx, w, inp["w1"], inp["w3"], inp["w2"], range(x.shape[0]),
+                        True)
+        err = float(np.abs(y.numpy() - ref).max() / np.abs(ref).max())
+        q.put((rank, (m.eb, m.ee), err))
+    except Exception as e:  # pragma: no cover - reported to the parent
+        import traceback
+        q.put((rank, None, traceback.format_exc()))
+
+
+def test_expert_parallel_sum_is_the_forward_gloo():
+    out = _run(2, _ep_worker)
+    assert [r[1] for r in out] == [(0, 16), (16, 32)], out
+    for rank, rng, err in out:
+        assert isinstance(err, float), err
+        assert err < 1e-12, (rank, err)
