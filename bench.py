@@ -16,6 +16,13 @@ same metric with host buffers (pinned x copied in and y copied out every step);
 bf16 tensor peak; `cpu_baseline` is the CPU oracle timed on a sample of the
 same workload on this host's cores. `--impl reference` times the oracle alone
 (rank 0 only) in the same JSON form.
+
+"expert_parallel" (N = 1) times each rank's local step of the expert-parallel
+layer over --ep-ranks ranks (its experts, all tokens through the gate, its
+share of the shared experts' tokens) one rank after another on this GPU, plus
+the finish kernel; the all-reduce between them is projected, not measured.
+With N > 1, `--parallel ep` runs that layer for real over NCCL (the same T
+tokens on every rank, strong scaling).
 """
 from __future__ import annotations
 
@@ -55,6 +62,12 @@ def parse_args(argv=None):
                     help="target wall time of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8-weight lines")
+    ap.add_argument("--ep-ranks", type=int, default=8,
+                    help="N=1: time each rank's local step of the expert-parallel layer over "
+                         "this many ranks, one after another (0 to skip)")
+    ap.add_argument("--parallel", choices=("dp", "ep"), default="dp",
+                    help="N>1: dp = replicas on their own tokens (default); ep = experts "
+                         "split over the ranks, one all-reduce per step")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -195,6 +208,97 @@ def algorithmic(layer, idx: np.ndarray) -> dict:
 # ---------------------------------------------------------------------------
 # Our arm
 # ---------------------------------------------------------------------------
+# All-reduce bus bandwidth of 8 B200s over NVSwitch at 1 GiB messages, measured
+# on this pool (NCCL); used only to project the expert-parallel step's
+# collective from one GPU.
+ALLREDUCE_BUS_GBS = 725.0
+
+
+def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
+    """The expert-parallel layer's per-rank local step (kt_moe_forward_local:
+    gate on all tokens, the rank's experts, its share of the shared experts'
+    tokens), each rank timed on this GPU in turn, and the finish kernel."""
+    from mixture_experts_layer_34_b200 import ep
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    cfg = K.config_for(layer)
+    T, E, S = layer.T, layer.n_experts, layer.n_shared
+    ws = K.alloc_workspace(cfg, T, dev)
+    part = torch.empty((T, layer.dim), dtype=torch.float32, device=dev)
+    y = torch.empty((T, layer.dim), dtype=inp["x"].dtype, device=dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    rank_ms = []
+    for r in range(ranks):
+        eb, ee = ep.expert_range(E, ranks, r)
+        sb, se = ep.token_range(T, ranks, r)
+        w1, w3, w2 = (ep.local_stack(inp[k], E, S, eb, ee) for k in ("w1", "w3", "w2"))
+        run = lambda: K.kt_moe_forward_local(cfg, T, inp["x"], inp["w_gate"], inp["bias"], eb, ee,
+                                             sb, se, w1, w3, w2, part, None, None, ws)
+        for _ in range(warmup):
+            run()
+        torch.cuda.synchronize()
+        t0.record()
+        for _ in range(steps):
+            run()
+        t1.record()
+        torch.cuda.synchronize()
+        rank_ms.append(t0.elapsed_time(t1) / steps)
+        del w1, w3, w2
+    for _ in range(warmup):
+        K.kt_moe_ep_finish(cfg, T, part, inp["x"], y)
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(steps):
+        K.kt_moe_ep_finish(cfg, T, part, inp["x"], y)
+    t1.record()
+    torch.cuda.synchronize()
+    rc = K.kt_moe_check(ws)
+    if rc != K.KT_OK:
+        raise RuntimeError(f"device error in the expert-parallel steps: {K.strerror(rc)}")
+    finish_ms = t0.elapsed_time(t1) / steps
+    msg = T * layer.dim * 4
+    ar_ms = 2 * (ranks - 1) / ranks * msg / (ALLREDUCE_BUS_GBS * 1e9) * 1e3
+    step_ms = max(rank_ms) + ar_ms + finish_ms
+    torch.cuda.empty_cache()
+    return {"ranks": ranks, "workload": layer.name,
+            "rank_local_ms": [round(v, 4) for v in rank_ms],
+            "max_rank_local_ms": round(max(rank_ms), 4), "finish_ms": round(finish_ms, 4),
+            "allreduce_bytes": msg,
+            "allreduce_ms_projected": round(ar_ms, 4),
+            "step_ms_projected": round(step_ms, 4),
+            "value_projected": round(T / (step_ms / 1e3), 1), "unit": "tokens/s",
+            "note": "local steps and finish measured here, one rank after another on this GPU; "
+                    "the fp32 all-reduce is projected at the measured 8-GPU NCCL bus bandwidth "
+                    f"({ALLREDUCE_BUS_GBS:.0f} GB/s), not measured (one GPU)"}
+
+
+def time_ep_layer(layer, dev, rank, world, steps, warmup):
+    """N > 1, --parallel ep: the expert-parallel layer over the process group
+    (NCCL all-reduce of the fp32 partials); the same T tokens on every rank."""
+    from mixture_experts_layer_34_b200 import ep
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    inp = W.make_layer(layer, dev)
+    cfg = K.config_for(layer)
+    m = ep.ExpertParallelMoE(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                             rank, world)
+    inp["w1"] = inp["w3"] = inp["w2"] = None
+    torch.cuda.empty_cache()
+    y = torch.empty((layer.T, layer.dim), dtype=inp["x"].dtype, device=dev)
+    for _ in range(warmup):
+        m.forward(inp["x"], y)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(steps):
+        m.forward(inp["x"], y)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    rc = K.kt_moe_check(m.buffers(layer.T, dev)[0])
+    if rc != K.KT_OK:
+        raise RuntimeError(f"device error in the expert-parallel steps: {K.strerror(rc)}")
+    return max_over_ranks(t0.elapsed_time(t1), world, dev)
 def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
     from mixture_experts_layer_34_b200 import ktmoe as K
     inp = W.make_layer(layer, dev)
@@ -354,9 +458,14 @@ def run_ours(a):
     peaks = load_peaks()
     layer = W.BY_NAME[a.workload]
 
+    if world > 1 and a.parallel == "ep":
+        return run_ep(a, layer, dev, rank, world, local, peaks)
     clocks = ClockSampler(local)
     clocks.start()
     pre = time_layer(layer, dev, rank, world, a.steps, a.warmup, a.e2e_steps)
+    epr = None
+    if world == 1 and a.ep_ranks > 1:
+        epr = time_ep_ranks(layer, pre["inp"], dev, a.ep_ranks, a.steps, a.warmup)
     dec = None
     if a.decode_workload != "none":
         dlayer = W.BY_NAME[a.decode_workload]
@@ -478,9 +587,35 @@ def run_ours(a):
                                     "value": round(world * fl.T * K_ / (res["graph_ms"] / 1e3), 1),
                                     "unit": "tokens/s"}
                 line["mxfp8"][key] = ent
+        if epr:
+            line["expert_parallel"] = epr
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+def run_ep(a, layer, dev, rank, world, local, peaks):
+    """--parallel ep with N > 1: one JSON line for the expert-parallel layer."""
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = time_ep_layer(layer, dev, rank, world, a.steps, a.warmup)
+    clk = clocks.stop()
+    if rank == 0:
+        T = layer.T
+        print(json.dumps({
+            "metric": "MoE layer tokens/s (prefill T=8192, decode T=8) + % of HBM/tensor roofline",
+            "value": round(T * a.steps / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms / a.steps, 4),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init weights of the V3 layer shape)",
+            "impl": "ours",
+            "config": {"workload": layer.name, "T": T, "parallelism": f"ep{world} "
+                       "(experts split, fp32 partials all-reduced over NCCL)",
+                       "l2": "inputs larger than L2"},
+            "gpu_launches": (LAUNCHES_PER_FORWARD + 1) * a.steps,
+            "clocks": clk,
+        }), flush=True)
+    torch.distributed.destroy_process_group()
 
 
 # ---------------------------------------------------------------------------
