@@ -214,6 +214,48 @@ def algorithmic(layer, idx: np.ndarray) -> dict:
 ALLREDUCE_BUS_GBS = 725.0
 
 
+def routing_stats(layer, inp, idx: np.ndarray, dev) -> dict:
+    """Expert-load histogram summary of the timed routing, and the number of
+    near-tie tokens: those whose k-th and (k+1)-th selection keys, or TG-th and
+    (TG+1)-th group scores, differ by at most 1e-5 (from the library's scores,
+    kt_moe_scores, plus the bias, on the host)."""
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    T, E, G, TG, k = layer.T, layer.n_experts, layer.n_groups, layer.topk_groups, layer.topk
+    cfg = K.config_for(layer)
+    ws = K.alloc_workspace(cfg, T, dev)
+    sc = torch.empty((T, E), dtype=torch.float32, device=dev)
+    K.kt_moe_scores(cfg, T, inp["x"], inp["w_gate"], sc, ws)
+    key = sc.cpu().numpy()
+    has_bias = inp["bias"] is not None
+    if has_bias:
+        key = (key + inp["bias"].float().cpu().numpy()[None, :]).astype(np.float32)
+    margin_g = np.full(T, np.inf, np.float32)
+    if G > 1:
+        gk = key.reshape(T, G, E // G)
+        top2 = layer.group_score == W.GROUP_TOP2SUM or (layer.group_score == W.GROUP_AUTO
+                                                       and has_bias)
+        if top2:
+            two = -np.sort(-gk, axis=2)[:, :, :2]
+            gsc = (two[:, :, 0] + two[:, :, 1]).astype(np.float32)
+        else:
+            gsc = gk.max(axis=2)
+        order = np.argsort(-gsc, axis=1, kind="stable")
+        gs_sorted = np.take_along_axis(gsc, order, axis=1)
+        margin_g = gs_sorted[:, TG - 1] - gs_sorted[:, TG]
+        keep = np.zeros((T, G), bool)
+        np.put_along_axis(keep, order[:, :TG], True, axis=1)
+        key = np.where(np.repeat(keep, E // G, axis=1), key, -np.inf)
+    ks = -np.sort(-key, axis=1)
+    margin_k = np.where(np.isfinite(ks[:, k]), ks[:, k - 1] - ks[:, k], np.inf)
+    near = (margin_k <= 1e-5) | (margin_g <= 1e-5)
+    load = np.bincount(idx.ravel(), minlength=E)
+    return {"load_max": int(load.max()), "load_mean": round(float(load.mean()), 2),
+            "max_over_mean": round(float(load.max() / load.mean()), 2),
+            "active_experts": int((load > 0).sum()), "zero_load_experts": int((load == 0).sum()),
+            "load_top8": np.sort(load)[::-1][:8].tolist(),
+            "near_tie_tokens": int(near.sum()), "near_tie_threshold": 1e-5}
+
+
 def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
     """The expert-parallel layer's per-rank local step (kt_moe_forward_local:
     gate on all tokens, the rank's experts, its share of the shared experts'
@@ -466,10 +508,12 @@ def run_ours(a):
     epr = None
     if world == 1 and a.ep_ranks > 1:
         epr = time_ep_ranks(layer, pre["inp"], dev, a.ep_ranks, a.steps, a.warmup)
+    pre["routing"] = routing_stats(layer, pre["inp"], pre["idx"], dev)
     dec = None
     if a.decode_workload != "none":
         dlayer = W.BY_NAME[a.decode_workload]
         dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, graph=True)
+        dec["routing"] = routing_stats(dlayer, dec["inp"], dec["idx"], dev)
     # The same layers with MXFP8 expert weights (same shapes, seeds and tokens).
     f8 = {}
     if not a.no_mxfp8:
@@ -509,6 +553,7 @@ def run_ours(a):
                        "load": "Zipf(1.1)", "parallelism": f"dp{world} (replicas, no collective)",
                        "l2": "inputs larger than L2: ~22 GB of expert weights read per step"},
             "stage_ms": {k: round(v, 4) for k, v in pre["stage_ms"].items()},
+            "routing": pre["routing"],
             "layer_tflops": round(pre["work"]["flops_layer"] / (pre["ms"] / K_ / 1e3) / 1e12, 1),
             # The gate/up GEMM runs inside back-to-back steps under the 1 kW power
             # cap, so its denominator is the sustained bf16 figure; the burst
@@ -537,6 +582,7 @@ def run_ours(a):
                 "workload": dl.name, "value": round(world * dl.T / (dms / 1e3), 1),
                 "unit": "tokens/s", "ms_per_step": round(dms, 4),
                 "active_experts": dec["work"]["active_experts"],
+                "routing": dec["routing"],
                 "stage_ms": {k: round(v, 4) for k, v in dec["stage_ms"].items()},
                 "layer_hbm_gbs": round(layer_gbs, 1),
                 "layer_hbm_frac": round(layer_gbs / peaks["hbm_gbs"], 4),

@@ -30,7 +30,10 @@ combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __r
   __syncthreads();
   const int nrow = S + k;
   const int nq = d / V;
-  for (int q = threadIdx.x; q < nq; q += blockDim.x) {
+  // blockIdx.y: a slice of the columns (few tokens: several CTAs per token).
+  const int per = (nq + gridDim.y - 1) / gridDim.y;
+  const int q1 = min(nq, (int)(blockIdx.y + 1) * per);
+  for (int q = blockIdx.y * per + threadIdx.x; q < q1; q += blockDim.x) {
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
@@ -104,7 +107,9 @@ combine_partial_kernel(int T_, int k, int S, int d, int sb, int se,
   }
   __syncthreads();
   const int nq = d / 4;
-  for (int q = threadIdx.x; q < nq; q += blockDim.x) {
+  const int per = (nq + gridDim.y - 1) / gridDim.y;
+  const int q1 = min(nq, (int)(blockIdx.y + 1) * per);
+  for (int q = blockIdx.y * per + threadIdx.x; q < q1; q += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < nrow; ++j) {
       const float4 v = reinterpret_cast<const float4*>(expert_out + (int64_t)rows[j] * d)[q];
@@ -154,9 +159,16 @@ ep_finish_kernel(int64_t n4, int add_residual, const float4* __restrict__ y_sum,
 
 }  // namespace
 
+// Column slices per token: one CTA per token when there are many, several when
+// few (a decode step), each slice at least 128 columns of 16-byte vectors.
+dim3 combine_grid(int64_t T, int d) {
+  const int64_t most = std::max<int64_t>(1, d / (128 * 8));
+  return dim3((unsigned)T, (unsigned)std::max<int64_t>(1, std::min<int64_t>(most, 296 / T)));
+}
+
 cudaError_t launch_combine_partial(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                    float* y_part, cudaStream_t st) {
-  combine_partial_kernel<<<(unsigned)T, 128, 0, st>>>(
+  combine_partial_kernel<<<combine_grid(T, r.d), 128, 0, st>>>(
       (int)T, r.k, r.S, r.d, r.sb, r.se, reinterpret_cast<const int32_t*>(ws + L.row_of),
       reinterpret_cast<const float*>(ws + L.expert_out), reinterpret_cast<float4*>(y_part));
   return cudaGetLastError();
@@ -181,13 +193,13 @@ cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* 
   const int32_t* row_of = reinterpret_cast<const int32_t*>(ws + L.row_of);
   const float* eo = reinterpret_cast<const float*>(ws + L.expert_out);
   if (r.act_bf16 && !r.y_fp32)
-    combine_kernel<true, false><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+    combine_kernel<true, false><<<combine_grid(T, r.d), 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
                                                              row_of, eo, x, y);
   else if (r.act_bf16)
-    combine_kernel<true, true><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+    combine_kernel<true, true><<<combine_grid(T, r.d), 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
                                                             row_of, eo, x, y);
   else
-    combine_kernel<false, true><<<(unsigned)T, 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+    combine_kernel<false, true><<<combine_grid(T, r.d), 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
                                                              row_of, eo, x, y);
   return cudaGetLastError();
 }

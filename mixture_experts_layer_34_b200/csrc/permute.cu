@@ -13,6 +13,8 @@
 //            the permuted activation buffer.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "ktmoe_internal.cuh"
 
 namespace ktmoe {
@@ -220,19 +222,24 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int e
     atomicOr(&mask[e], 1u << tl);
   }
   __syncthreads();
+  // blockIdx.y: a column slice of the copies (few tokens: several CTAs share a
+  // chunk's copy); slice 0 also writes the row maps and the scales.
+  const bool lead = blockIdx.y == 0;
   for (int q = threadIdx.x; q < nent; q += blockDim.x) {
     const int tl = q / k;
     const int e = idx[(int64_t)t0 * k + q];
     if (e < eb || e >= ee) {   // an expert computed elsewhere: no row here
-      row_of[(int64_t)t0 * k + q] = -1;
+      if (lead) row_of[(int64_t)t0 * k + q] = -1;
       srow[q] = -1;
       continue;
     }
     const int rank = __popc(mask[e] & ((1u << tl) - 1u));
     const int row = chunk_base[(int64_t)c * E + e] + rank;
-    row_of[(int64_t)t0 * k + q] = row;
-    tok_of[row] = t0 + tl;
-    row_weight[row] = w[(int64_t)t0 * k + q];
+    if (lead) {
+      row_of[(int64_t)t0 * k + q] = row;
+      tok_of[row] = t0 + tl;
+      row_weight[row] = w[(int64_t)t0 * k + q];
+    }
     srow[q] = row;
   }
   if (kMode == kNoCopy) return;
@@ -240,10 +247,12 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int e
   // Copy each token's row of x (bf16), or of its E4M3 codes, to its k permuted
   // rows in 16-byte chunks.
   const int nchunk = kMode == kCopyF8 ? d / 16 : d / 8;
+  const int per = (nchunk + gridDim.y - 1) / gridDim.y;
+  const int q0 = blockIdx.y * per, q1 = min(nchunk, q0 + per);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int tl = warp; tl < nt; tl += blockDim.x / 32) {
     const uint4* src = x + (int64_t)(t0 + tl) * nchunk;
-    for (int q = lane; q < nchunk; q += 32) {
+    for (int q = q0 + lane; q < q1; q += 32) {
       const uint4 v = src[q];
       for (int j = 0; j < k; ++j) {
         const int row = srow[tl * k + j];
@@ -251,7 +260,7 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int e
       }
     }
   }
-  if (kMode != kCopyF8) return;
+  if (kMode != kCopyF8 || !lead) return;
   // MXFP8: each routed row's and each shared-expert row's scale bytes into its
   // GEMM chunk's scale blocks (4 K blocks per 32-bit word).
   const int nslab = d / 128;
@@ -290,7 +299,10 @@ cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* 
       reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)L.nperm;
+  // Few chunks (a decode step): split each chunk's row copies over column
+  // slices so that about two CTAs per SM copy.
+  const int slices = r.act_bf16 ? (int)std::max<int64_t>(1, std::min<int64_t>(16, (296 + L.nperm - 1) / L.nperm)) : 1;
+  const dim3 grid((unsigned)L.nperm, (unsigned)slices);
   float* rw = reinterpret_cast<float*>(ws + L.row_weight);
   const int32_t* base = I32(L.chunk_base);
   if (r.fp8)
