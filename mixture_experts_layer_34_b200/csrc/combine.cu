@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(128)
 combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __restrict__ row_of,
                const float* __restrict__ expert_out, const void* __restrict__ x,
                void* __restrict__ y) {
+  pdl_wait();
   constexpr int V = kBF16 ? 8 : 4;
   __shared__ int rows[kMaxShared + kMaxTopk];
   const int t = blockIdx.x;
@@ -92,6 +93,7 @@ __global__ void __launch_bounds__(128)
 combine_partial_kernel(int T_, int k, int S, int d, int sb, int se,
                        const int32_t* __restrict__ row_of, const float* __restrict__ expert_out,
                        float4* __restrict__ y) {
+  pdl_wait();
   __shared__ int rows[kMaxShared + kMaxTopk];
   __shared__ int nrow;
   const int t = blockIdx.x;
@@ -128,6 +130,7 @@ template <bool kBF16X, bool kF32Out>
 __global__ void __launch_bounds__(256)
 ep_finish_kernel(int64_t n4, int add_residual, const float4* __restrict__ y_sum,
                  const void* __restrict__ x, void* __restrict__ y) {
+  pdl_wait();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (int64_t)gridDim.x * blockDim.x) {
     float4 v = y_sum[i];
@@ -168,7 +171,7 @@ dim3 combine_grid(int64_t T, int d) {
 
 cudaError_t launch_combine_partial(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                    float* y_part, cudaStream_t st) {
-  combine_partial_kernel<<<combine_grid(T, r.d), 128, 0, st>>>(
+  (void)launch_pdl(combine_partial_kernel, dim3(combine_grid(T, r.d)), dim3(128), 0, st,
       (int)T, r.k, r.S, r.d, r.sb, r.se, reinterpret_cast<const int32_t*>(ws + L.row_of),
       reinterpret_cast<const float*>(ws + L.expert_out), reinterpret_cast<float4*>(y_part));
   return cudaGetLastError();
@@ -180,11 +183,11 @@ cudaError_t launch_ep_finish(const Resolved& r, int64_t T, const float* y_sum, c
   const unsigned grid = (unsigned)std::min<int64_t>((n4 + 255) / 256, (int64_t)num_sms * 8);
   const float4* ys = reinterpret_cast<const float4*>(y_sum);
   if (r.act_bf16 && !r.y_fp32)
-    ep_finish_kernel<true, false><<<grid, 256, 0, st>>>(n4, r.add_residual, ys, x, y);
+    (void)launch_pdl(ep_finish_kernel<true, false>, dim3(grid), dim3(256), 0, st, n4, r.add_residual, ys, x, y);
   else if (r.act_bf16)
-    ep_finish_kernel<true, true><<<grid, 256, 0, st>>>(n4, r.add_residual, ys, x, y);
+    (void)launch_pdl(ep_finish_kernel<true, true>, dim3(grid), dim3(256), 0, st, n4, r.add_residual, ys, x, y);
   else
-    ep_finish_kernel<false, true><<<grid, 256, 0, st>>>(n4, r.add_residual, ys, x, y);
+    (void)launch_pdl(ep_finish_kernel<false, true>, dim3(grid), dim3(256), 0, st, n4, r.add_residual, ys, x, y);
   return cudaGetLastError();
 }
 
@@ -193,13 +196,13 @@ cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* 
   const int32_t* row_of = reinterpret_cast<const int32_t*>(ws + L.row_of);
   const float* eo = reinterpret_cast<const float*>(ws + L.expert_out);
   if (r.act_bf16 && !r.y_fp32)
-    combine_kernel<true, false><<<combine_grid(T, r.d), 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+    (void)launch_pdl(combine_kernel<true, false>, dim3(combine_grid(T, r.d)), dim3(128), 0, st, (int)T, r.k, r.S, r.d, r.add_residual,
                                                              row_of, eo, x, y);
   else if (r.act_bf16)
-    combine_kernel<true, true><<<combine_grid(T, r.d), 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+    (void)launch_pdl(combine_kernel<true, true>, dim3(combine_grid(T, r.d)), dim3(128), 0, st, (int)T, r.k, r.S, r.d, r.add_residual,
                                                             row_of, eo, x, y);
   else
-    combine_kernel<false, true><<<combine_grid(T, r.d), 128, 0, st>>>((int)T, r.k, r.S, r.d, r.add_residual,
+    (void)launch_pdl(combine_kernel<false, true>, dim3(combine_grid(T, r.d)), dim3(128), 0, st, (int)T, r.k, r.S, r.d, r.add_residual,
                                                              row_of, eo, x, y);
   return cudaGetLastError();
 }

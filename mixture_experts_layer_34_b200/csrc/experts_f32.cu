@@ -24,6 +24,7 @@ up_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_ch
               int d, int I, const float* __restrict__ x, const float* __restrict__ w1,
               const float* __restrict__ w3, const int32_t* __restrict__ tok_of,
               float* __restrict__ hidden) {
+  pdl_wait();
   __shared__ float xs[kTB][kTK + 1];
   __shared__ float as[kTB][kTK + 1];
   __shared__ float bs[kTB][kTK + 1];
@@ -88,6 +89,7 @@ down_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_
                 int I, int n_routed_rows, const float* __restrict__ hidden,
                 const float* __restrict__ w2, const float* __restrict__ row_weight,
                 float* __restrict__ out) {
+  pdl_wait();
   __shared__ float hs[kTB][kTK + 1];
   __shared__ float ws[kTB][kTK + 1];
   const int n_chunks = *n_chunks_p;
@@ -143,13 +145,13 @@ cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, ch
   const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.meta);
   const int grid = num_sms * 4;
   if (up) {
-    up_f32_kernel<<<grid, 256, 0, st>>>(
+    (void)launch_pdl(up_f32_kernel, dim3(grid), dim3(256), 0, st,
         reinterpret_cast<const Chunk*>(ws + L.chunks), meta + 0, routed_slots(r), r.d, r.I,
         static_cast<const float*>(x), static_cast<const float*>(w1), static_cast<const float*>(w3),
         reinterpret_cast<const int32_t*>(ws + L.tok_of), reinterpret_cast<float*>(ws + L.hidden));
     return cudaGetLastError();
   }
-  down_f32_kernel<<<grid, 256, 0, st>>>(
+  (void)launch_pdl(down_f32_kernel, dim3(grid), dim3(256), 0, st,
       reinterpret_cast<const Chunk*>(ws + L.chunks), meta + 0, r.d, r.I, (int)(T * r.k),
       reinterpret_cast<const float*>(ws + L.hidden), static_cast<const float*>(w2),
       reinterpret_cast<const float*>(ws + L.row_weight),

@@ -510,6 +510,9 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touches only this CTA pair's shared memory, TMEM and the
+  // kernel parameters; the previous kernel's outputs are read after this.
+  pdl_wait();
 
   const int n_tiles = args.implicit_rows > 0
                           ? ((args.implicit_rows + kChunkRows - 1) / kChunkRows) * args.n_ftiles
@@ -1065,8 +1068,8 @@ template <int kKind>
 cudaError_t launch(const TmaMaps& maps, const GemmArgs& args, int grid, cudaStream_t st) {
   cudaError_t e = ensure_smem_attr<kKind>();
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<kKind><<<grid, kThreads, Kind<kKind>::kSmem, st>>>(maps, args);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<kKind>, dim3(grid), dim3(kThreads), Kind<kKind>::kSmem, st,
+                    maps, args);
 }
 
 // Grid of whole CTA pairs: at most one pair per two SMs, at most max_pairs.

@@ -79,6 +79,7 @@ template <typename T>
 __global__ void __launch_bounds__(kLThreads)
 gate_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg, float* __restrict__ logits,
                    int T_, int E, int d) {
+  pdl_wait();
   __shared__ float xs[kLK][kLT + 4];
   __shared__ float ws[kLK][kLE + 4];
   const int e0 = blockIdx.x * kLE;
@@ -135,6 +136,7 @@ template <typename T>
 __global__ void __launch_bounds__(kSmallWarps * 32)
 gate_logits_splitk_kernel(const T* __restrict__ x, const T* __restrict__ wg,
                           float* __restrict__ part, int T_, int E, int d, int kc) {
+  pdl_wait();
   constexpr int VN = Vec16<T>::n, EW = 4;  // experts per warp, computed together
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ks = blockIdx.y;
@@ -281,6 +283,7 @@ gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
                    const float* __restrict__ scores_in, const float* __restrict__ bias,
                    int32_t* __restrict__ out_idx, float* __restrict__ out_w,
                    int32_t* __restrict__ chunk_counts) {
+  pdl_wait();
   __shared__ int scount[kMaxExperts];
   __shared__ float skey[kSelWarps][kMaxExperts];
   const int E = r.E, k = r.k, G = r.G, gs = r.gs;
@@ -402,6 +405,7 @@ template <int NP>
 __global__ void __launch_bounds__(kSelWarps * 32)
 gate_scores_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ logits,
                    float* __restrict__ out) {
+  pdl_wait();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int tt = 0; tt < kPermChunk / kSelWarps; ++tt) {
     const int t = blockIdx.x * kPermChunk + tt * kSelWarps + warp;
@@ -428,10 +432,10 @@ cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, cons
     const int kc = ((r.d + kSplitK - 1) / kSplitK + vn - 1) / vn * vn;
     const dim3 grid((unsigned)((r.E + 31) / 32), kSplitK);
     if (bf16)
-      gate_logits_splitk_kernel<__nv_bfloat16><<<grid, kSmallWarps * 32, 0, st>>>(
+      (void)launch_pdl(gate_logits_splitk_kernel<__nv_bfloat16>, dim3(grid), dim3(kSmallWarps * 32), 0, st,
           (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d, kc);
     else
-      gate_logits_splitk_kernel<float><<<grid, kSmallWarps * 32, 0, st>>>(
+      (void)launch_pdl(gate_logits_splitk_kernel<float>, dim3(grid), dim3(kSmallWarps * 32), 0, st,
           (const float*)x, (const float*)w_gate, logits, (int)T, r.E, r.d, kc);
     return cudaGetLastError();
   }
@@ -439,10 +443,10 @@ cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, cons
   if (bf16 && r.E % 4 == 0) return launch_gate_logits_tc(r, T, x, w_gate, logits, err, num_sms, st);
   dim3 grid((r.E + kLE - 1) / kLE, (unsigned)((T + kLT - 1) / kLT));
   if (bf16)
-    gate_logits_kernel<__nv_bfloat16><<<grid, kLThreads, 0, st>>>(
+    (void)launch_pdl(gate_logits_kernel<__nv_bfloat16>, dim3(grid), dim3(kLThreads), 0, st,
         (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d);
   else
-    gate_logits_kernel<float><<<grid, kLThreads, 0, st>>>((const float*)x, (const float*)w_gate,
+    (void)launch_pdl(gate_logits_kernel<float>, dim3(grid), dim3(kLThreads), 0, st, (const float*)x, (const float*)w_gate,
                                                           logits, (int)T, r.E, r.d);
   return cudaGetLastError();
 }
@@ -454,7 +458,7 @@ cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits
   const int ks = scores_in ? 1 : gate_logit_splits(r, T);
   const int np = (r.E + 31) / 32;
 #define KT_SELECT(NPV)                                                                        \
-  gate_select_kernel<NPV><<<grid, kSelWarps * 32, 0, st>>>(r, (int)T, ks, logits, scores_in, \
+  (void)launch_pdl(gate_select_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, ks, logits, scores_in, \
                                                            bias, idx, w, chunk_counts)
   if (np <= 1) KT_SELECT(1);
   else if (np <= 2) KT_SELECT(2);
@@ -475,7 +479,7 @@ cudaError_t launch_gate_scores(const Resolved& r, int64_t T, const float* logits
   const int ks = gate_logit_splits(r, T);
   const int np = (r.E + 31) / 32;
 #define KT_SCORES(NPV) \
-  gate_scores_kernel<NPV><<<grid, kSelWarps * 32, 0, st>>>(r, (int)T, ks, logits, scores)
+  (void)launch_pdl(gate_scores_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, ks, logits, scores)
   if (np <= 1) KT_SCORES(1);
   else if (np <= 2) KT_SCORES(2);
   else if (np <= 4) KT_SCORES(4);

@@ -56,6 +56,7 @@ __device__ __forceinline__ uint8_t mx_block_bf16(const uint4* __restrict__ src,
 __global__ void __launch_bounds__(256)
 mx_quantize_kernel(const uint4* __restrict__ src, int64_t nblocks, uint4* __restrict__ codes,
                    uint8_t* __restrict__ scales) {
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nblocks) return;
   scales[i] = mx_block_bf16(src + i * 4, codes + i * 2);
@@ -101,7 +102,7 @@ cudaError_t launch_mx_quantize(const void* src, int64_t rows, int64_t K, uint8_t
                                uint8_t* scales, cudaStream_t st) {
   const int64_t nb = rows * (K / 32);
   if (nb == 0) return cudaSuccess;
-  mx_quantize_kernel<<<(unsigned)((nb + 255) / 256), 256, 0, st>>>(
+  (void)launch_pdl(mx_quantize_kernel, dim3((unsigned)((nb + 255) / 256)), dim3(256), 0, st,
       static_cast<const uint4*>(src), nb, reinterpret_cast<uint4*>(codes), scales);
   return cudaGetLastError();
 }

@@ -131,6 +131,7 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
                     Chunk* __restrict__ chunks, int2* __restrict__ tiles_up,
                     int2* __restrict__ tiles_dn, int32_t* __restrict__ meta,
                     int32_t* __restrict__ gchunk0) {
+  pdl_wait();
   constexpr int NGMAX = kMaxExperts + kMaxShared;
   __shared__ int tot[NGMAX];
   __shared__ int rows0[NGMAX];
@@ -208,6 +209,7 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int e
                        int32_t* __restrict__ tok_of, float* __restrict__ row_weight,
                        const uint4* __restrict__ x, uint4* __restrict__ xperm,
                        const uint8_t* __restrict__ xs, uint8_t* __restrict__ tok_sf) {
+  pdl_wait();
   __shared__ uint32_t mask[kMaxExperts];
   __shared__ int srow[kPermChunk * kMaxTopk];
   const int c = blockIdx.x;
@@ -291,7 +293,7 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int e
 cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* ws,
                            const int32_t* idx, const float* w, const void* x, cudaStream_t st) {
   auto I32 = [&](size_t off) { return reinterpret_cast<int32_t*>(ws + off); };
-  permute_scan_kernel<<<1, kScanThreads, 0, st>>>(
+  (void)launch_pdl(permute_scan_kernel, dim3(1), dim3(kScanThreads), 0, st,
       r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows, r.eb,
       r.ee, r.sb, r.se,
       I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts), I32(L.offsets),
@@ -306,18 +308,18 @@ cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* 
   float* rw = reinterpret_cast<float*>(ws + L.row_weight);
   const int32_t* base = I32(L.chunk_base);
   if (r.fp8)
-    permute_scatter_kernel<kCopyF8><<<grid, 256, 0, st>>>(
+    (void)launch_pdl(permute_scatter_kernel<kCopyF8>, dim3(grid), dim3(256), 0, st,
         r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(ws + L.xq),
         reinterpret_cast<uint4*>(ws + L.xperm), reinterpret_cast<const uint8_t*>(ws + L.xs),
         reinterpret_cast<uint8_t*>(ws + L.tok_sf));
   else if (r.dtype == KT_DTYPE_BF16)
-    permute_scatter_kernel<kCopyBf16><<<grid, 256, 0, st>>>(
+    (void)launch_pdl(permute_scatter_kernel<kCopyBf16>, dim3(grid), dim3(256), 0, st,
         r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(x),
         reinterpret_cast<uint4*>(ws + L.xperm), nullptr, nullptr);
   else
-    permute_scatter_kernel<kNoCopy><<<grid, 256, 0, st>>>(
+    (void)launch_pdl(permute_scatter_kernel<kNoCopy>, dim3(grid), dim3(256), 0, st,
         r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr, nullptr);
   return cudaGetLastError();
