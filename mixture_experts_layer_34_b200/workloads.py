@@ -167,6 +167,33 @@ MXFP8 = [
 ]
 BY_NAME.update({c.name: c for c in MXFP8})
 
+# The library's limits and degenerate sizes: the most experts, groups, top-k and
+# shared experts a config may have (512, 32, 32, 8), a single token, top-1 over
+# 512 experts, and a large token count (int32 row arithmetic over 589,824 rows).
+LIMITS = [
+    LayerConfig("limits_E512_k32_S8", T=67, dim=256, n_experts=512, n_groups=32, topk_groups=8,
+                topk=32, n_shared=8, inter=128, score_func=SIGMOID, route_scale=2.5,
+                norm_topk=-1, group_score=GROUP_AUTO, dtype="bf16", bias="normal", seed=2401),
+    LayerConfig("limits_T1", T=1, dim=512, n_experts=64, n_groups=8, topk_groups=4, topk=8,
+                n_shared=1, inter=256, score_func=SIGMOID, route_scale=2.5, norm_topk=-1,
+                group_score=GROUP_AUTO, dtype="bf16", bias="normal", seed=2402),
+    LayerConfig("limits_E512_k1_softmax", T=40, dim=128, n_experts=512, n_groups=1,
+                topk_groups=1, topk=1, n_shared=0, inter=64, score_func=SOFTMAX, route_scale=1.0,
+                norm_topk=0, group_score=GROUP_AUTO, dtype="bf16", bias="none", seed=2403),
+    LayerConfig("limits_T65536", T=65536, dim=256, n_experts=64, n_groups=8, topk_groups=4,
+                topk=8, n_shared=1, inter=128, score_func=SIGMOID, route_scale=2.5,
+                norm_topk=-1, group_score=GROUP_AUTO, dtype="bf16", bias="normal", seed=2404),
+    LayerConfig("limits_E512_k32_S8_f32", T=67, dim=256, n_experts=512, n_groups=32,
+                topk_groups=8, topk=32, n_shared=8, inter=128, score_func=SIGMOID,
+                route_scale=2.5, norm_topk=-1, group_score=GROUP_AUTO, dtype="f32",
+                bias="normal", seed=2405, init="fan_in"),
+    LayerConfig("limits_E512_k32_S8_mxfp8", T=67, dim=256, n_experts=512, n_groups=32,
+                topk_groups=8, topk=32, n_shared=8, inter=128, score_func=SIGMOID,
+                route_scale=2.5, norm_topk=-1, group_score=GROUP_AUTO, dtype="mxfp8",
+                bias="normal", seed=2406),
+]
+BY_NAME.update({c.name: c for c in LIMITS})
+
 
 def torch_dtype(cfg: LayerConfig) -> torch.dtype:
     return torch.float32 if cfg.dtype == "f32" else torch.bfloat16
