@@ -527,6 +527,10 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
       // ---------------- TMA producer (both CTAs) ----------------
       // The even CTA's producer also schedules: it takes the pair's next tile and
       // publishes it to both CTAs' schedule slots; the odd CTA's producer reads it.
+      // The next tile is claimed halfway through the current tile's stages and
+      // read after its last stage is issued, so the claim (a global atomic) and
+      // the reads of the tile list overlap the copies in flight instead of
+      // stalling the pipeline between tiles.
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -535,18 +539,31 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
       uint32_t sphase = 0;
       const uint64_t p_first = policy_evict_first(), p_normal = policy_evict_normal(),
                      p_last = policy_evict_last();
+      int t_next = 0;
+      Chunk c_next{-1, 0, 0, 0};
+      int f_next = 0, ci_next = 0;
+      auto claim = [&]() {
+        t_next = args.counter ? atomicAdd(args.counter, 1) : pair + iter * n_pairs;
+        ++iter;
+      };
+      auto fetch = [&]() {
+        c_next = Chunk{-1, 0, 0, 0};
+        f_next = 0;
+        ci_next = 0;
+        if (t_next < n_tiles) get_tile(args, t_next, c_next, f_next, ci_next);
+      };
+      if (leader) {
+        claim();
+        fetch();
+      }
       for (;;) {
-        int t;
         if (leader) {
           if (!mbar_wait(&sched_empty[sslot], sphase ^ 1u, err, 5 + 8 * kKind)) {
             ok = false;
             break;
           }
-          t = args.counter ? atomicAdd(args.counter, 1) : pair + iter * n_pairs;
-          ++iter;
-          Chunk c{-1, 0, 0, 0};
-          int f = 0, cidx = 0;
-          if (t < n_tiles) get_tile(args, t, c, f, cidx);
+          const Chunk c = c_next;
+          const int f = f_next, cidx = ci_next;
           int* slot = sched_info + 8 * sslot;
           slot[0] = c.group;
           slot[1] = c.row0;
@@ -666,6 +683,10 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
             }
           }
           issued = issued < kStages ? issued + 1 : kStages;
+          if (leader) {
+            if (kb == nk / 2) claim();
+            if (kb == nk - 1) fetch();
+          }
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
