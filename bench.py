@@ -257,9 +257,12 @@ def routing_stats(layer, inp, idx: np.ndarray, dev) -> dict:
 
 
 def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
-    """The expert-parallel layer's per-rank local step (kt_moe_forward_local:
-    gate on all tokens, the rank's experts, its share of the shared experts'
-    tokens), each rank timed on this GPU in turn, and the finish kernel."""
+    """The expert-parallel layer's per-rank local step (the gate on all tokens,
+    the rank's experts, its share of the shared experts' tokens), each rank
+    timed on this GPU in turn, for two placements of the routed experts:
+    contiguous ranges (kt_moe_forward_local) and a placement balanced on the
+    expert load of another batch of the same workload (kt_moe_forward_placed);
+    and the finish kernel."""
     from mixture_experts_layer_34_b200 import ep
     from mixture_experts_layer_34_b200 import ktmoe as K
     cfg = K.config_for(layer)
@@ -268,13 +271,8 @@ def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
     part = torch.empty((T, layer.dim), dtype=torch.float32, device=dev)
     y = torch.empty((T, layer.dim), dtype=inp["x"].dtype, device=dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    rank_ms = []
-    for r in range(ranks):
-        eb, ee = ep.expert_range(E, ranks, r)
-        sb, se = ep.token_range(T, ranks, r)
-        w1, w3, w2 = (ep.local_stack(inp[k], E, S, eb, ee) for k in ("w1", "w3", "w2"))
-        run = lambda: K.kt_moe_forward_local(cfg, T, inp["x"], inp["w_gate"], inp["bias"], eb, ee,
-                                             sb, se, w1, w3, w2, part, None, None, ws)
+
+    def timed(run):
         for _ in range(warmup):
             run()
         torch.cuda.synchronize()
@@ -283,34 +281,58 @@ def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
             run()
         t1.record()
         torch.cuda.synchronize()
-        rank_ms.append(t0.elapsed_time(t1) / steps)
-        del w1, w3, w2
-    for _ in range(warmup):
-        K.kt_moe_ep_finish(cfg, T, part, inp["x"], y)
-    torch.cuda.synchronize()
-    t0.record()
-    for _ in range(steps):
-        K.kt_moe_ep_finish(cfg, T, part, inp["x"], y)
-    t1.record()
-    torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / steps
+
+    # Expected load: the routing of another seeded batch (rank 1's tokens).
+    g = torch.Generator(device="cpu").manual_seed(rank_tokens_seed(layer, 1))
+    x2 = torch.randn(inp["x"].shape, generator=g).to(inp["x"].dtype).to(dev)
+    idx2 = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
+    w2_ = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
+    K.kt_moe_gate(cfg, T, x2, inp["w_gate"], inp["bias"], None, idx2, w2_, ws)
+    load2 = np.bincount(idx2.cpu().numpy().ravel(), minlength=E)
+    del x2
+    placements = {"contiguous": ep.contiguous_placement(E, ranks),
+                  "balanced": ep.balanced_placement(load2, ranks)}
+    out = {}
+    for name, placement in placements.items():
+        rank_ms = []
+        for r in range(ranks):
+            sb, se = ep.token_range(T, ranks, r)
+            experts = placement[r]
+            w1, w3, w2 = (ep.local_stack_of(inp[k], E, S, experts) for k in ("w1", "w3", "w2"))
+            if name == "contiguous":
+                eb, ee = experts[0], experts[-1] + 1
+                run = lambda: K.kt_moe_forward_local(cfg, T, inp["x"], inp["w_gate"], inp["bias"],
+                                                     eb, ee, sb, se, w1, w3, w2, part, None, None,
+                                                     ws)
+            else:
+                tab = ep.slot_table(experts, E)
+                run = lambda: K.kt_moe_forward_placed(cfg, T, inp["x"], inp["w_gate"],
+                                                      inp["bias"], tab, sb, se, w1, w3, w2, part,
+                                                      None, None, ws)
+            rank_ms.append(timed(run))
+            del w1, w3, w2
+        out[name] = rank_ms
+    finish_ms = timed(lambda: K.kt_moe_ep_finish(cfg, T, part, inp["x"], y))
     rc = K.kt_moe_check(ws)
     if rc != K.KT_OK:
         raise RuntimeError(f"device error in the expert-parallel steps: {K.strerror(rc)}")
-    finish_ms = t0.elapsed_time(t1) / steps
     msg = T * layer.dim * 4
     ar_ms = 2 * (ranks - 1) / ranks * msg / (ALLREDUCE_BUS_GBS * 1e9) * 1e3
-    step_ms = max(rank_ms) + ar_ms + finish_ms
     torch.cuda.empty_cache()
-    return {"ranks": ranks, "workload": layer.name,
-            "rank_local_ms": [round(v, 4) for v in rank_ms],
-            "max_rank_local_ms": round(max(rank_ms), 4), "finish_ms": round(finish_ms, 4),
-            "allreduce_bytes": msg,
-            "allreduce_ms_projected": round(ar_ms, 4),
-            "step_ms_projected": round(step_ms, 4),
-            "value_projected": round(T / (step_ms / 1e3), 1), "unit": "tokens/s",
-            "note": "local steps and finish measured here, one rank after another on this GPU; "
-                    "the fp32 all-reduce is projected at the measured 8-GPU NCCL bus bandwidth "
-                    f"({ALLREDUCE_BUS_GBS:.0f} GB/s), not measured (one GPU)"}
+    res = {"ranks": ranks, "workload": layer.name, "finish_ms": round(finish_ms, 4),
+           "allreduce_bytes": msg, "allreduce_ms_projected": round(ar_ms, 4), "unit": "tokens/s"}
+    for name, rank_ms in out.items():
+        step_ms = max(rank_ms) + ar_ms + finish_ms
+        res[name] = {"rank_local_ms": [round(v, 4) for v in rank_ms],
+                     "max_rank_local_ms": round(max(rank_ms), 4),
+                     "step_ms_projected": round(step_ms, 4),
+                     "value_projected": round(T / (step_ms / 1e3), 1)}
+    res["note"] = ("local steps and finish measured here, one rank after another on this GPU; "
+                   "the fp32 all-reduce is projected at the measured 8-GPU NCCL bus bandwidth "
+                   f"({ALLREDUCE_BUS_GBS:.0f} GB/s), not measured (one GPU); the balanced "
+                   "placement is computed from the expert load of another seeded batch")
+    return res
 
 
 def time_ep_layer(layer, dev, rank, world, steps, warmup):

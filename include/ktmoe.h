@@ -310,6 +310,17 @@ int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, con
  *   kt_moe_mxfp8_scale_bytes_local: the layouts of kt_moe_mxfp8_pack with the
  *   group index g running over the local slots).
  *
+ * kt_moe_forward_placed (and _mxfp8): the same with any placement of the routed
+ *   experts instead of a range. expert_slot: host array of E entries, the weight
+ *   slot of routed expert e on this rank or -1 if it runs elsewhere; the slots
+ *   used must be exactly 0 .. n_local - 1, each once (n_local = the number of
+ *   entries >= 0), else KT_ERR_INVALID_CONFIG; NULL: KT_ERR_NULL. The local
+ *   stacks hold n_local routed slots, then the S shared experts; MXFP8 stacks
+ *   are packed by kt_moe_mxfp8_pack_local(cfg, 0, n_local, ...). A placement by
+ *   expected load (several heavy experts on different ranks) evens out the
+ *   ranks' work, which a contiguous range does not under a skewed load. The
+ *   table is read on the host during the call.
+ *
  * kt_moe_ep_finish: after the caller's sum of y_part over the ranks into y_sum
  *   (an all-reduce; fp32 [T, dim], device), y = y_sum (+ x if add_residual) in
  *   y's type (as kt_moe_forward). y may be y_sum itself when y is fp32; any
@@ -327,6 +338,18 @@ int kt_moe_forward_local_mxfp8(const kt_moe_config* cfg, int64_t T, const void* 
                                const uint8_t* sf_up, const uint8_t* sf_down, float* y_part,
                                int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                                size_t ws_bytes, void* stream);
+int kt_moe_forward_placed(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                          const float* bias, const int32_t* expert_slot, int64_t shared_begin,
+                          int64_t shared_end, const void* w1, const void* w3, const void* w2,
+                          float* y_part, int32_t* topk_idx_out, float* topk_w_out,
+                          void* workspace, size_t ws_bytes, void* stream);
+int kt_moe_forward_placed_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x,
+                                const void* w_gate, const float* bias, const int32_t* expert_slot,
+                                int64_t shared_begin, int64_t shared_end, const uint8_t* w1q,
+                                const uint8_t* w3q, const uint8_t* w2q, const uint8_t* sf_up,
+                                const uint8_t* sf_down, float* y_part, int32_t* topk_idx_out,
+                                float* topk_w_out, void* workspace, size_t ws_bytes,
+                                void* stream);
 int kt_moe_ep_finish(const kt_moe_config* cfg, int64_t T, const float* y_sum, const void* x,
                      void* y, void* stream);
 size_t kt_moe_mxfp8_scale_bytes_local(const kt_moe_config* cfg, int expert_begin, int expert_end,

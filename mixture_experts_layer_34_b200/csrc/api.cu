@@ -83,8 +83,7 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
   r->act_bf16 = c->dtype != KT_DTYPE_F32;
   r->fp8 = c->dtype == KT_DTYPE_MXFP8;
   r->chunk_rows = r->fp8 ? kChunkRowsF8 : kChunkRows;
-  r->eb = 0;
-  r->ee = E;
+  r->n_local = E;
   r->sb = 0;
   r->se = (int)T;
   r->add_residual = c->add_residual;
@@ -326,7 +325,15 @@ int check_forward_args(const kt_moe_config* cfg, int64_t T, const void* x, const
 // permutation (after the token quantisation for MXFP8), the two grouped GEMMs,
 // then the combine into y, or (partial) the fp32 sum of this launch's experts.
 // wa/wb/wc: W1, W3, W2 (bf16/fp32) or their codes (MXFP8, with sf_up/sf_down).
-int run_forward(const Resolved& r, int64_t T, const void* x, const void* w_gate,
+// The plain forward's placement: routed expert e in weight slot e.
+SlotTable identity_table(const Resolved& r) {
+  SlotTable t;
+  for (int e = 0; e < kMaxExperts; ++e) t.slot[e] = (int16_t)(e < r.E ? e : -1);
+  return t;
+}
+
+int run_forward(const Resolved& r, const SlotTable& tab, int64_t T, const void* x,
+                const void* w_gate,
                 const float* bias, const void* wa, const void* wb, const void* wc,
                 const uint8_t* sf_up, const uint8_t* sf_down, void* y, bool partial,
                 int32_t* topk_idx_out, float* topk_w_out, void* workspace, void* stream,
@@ -358,7 +365,7 @@ int run_forward(const Resolved& r, int64_t T, const void* x, const void* w_gate,
   if (r.fp8 && launch_mx_quantize(x, T, r.d, reinterpret_cast<uint8_t*>(ws + L.xq),
                                   reinterpret_cast<uint8_t*>(ws + L.xs), st) != cudaSuccess)
     return KT_ERR_CUDA;
-  if (launch_permute(r, T, L, ws, idx, w, x, st) != cudaSuccess) return KT_ERR_CUDA;
+  if (launch_permute(r, tab, T, L, ws, idx, w, x, st) != cudaSuccess) return KT_ERR_CUDA;
   if (!mark(2)) return KT_ERR_CUDA;
   cudaError_t e;
   if (r.fp8)
@@ -395,7 +402,8 @@ int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
                               workspace, ws_bytes, &r);
   if (rc != KT_OK) return rc;
   if (r.fp8) return KT_ERR_INVALID_CONFIG;   // MXFP8 weights: kt_moe_forward_mxfp8
-  return run_forward(r, T, x, w_gate, bias, w1, w3, w2, nullptr, nullptr, y, false, topk_idx_out,
+  return run_forward(r, identity_table(r), T, x, w_gate, bias, w1, w3, w2, nullptr, nullptr, y,
+                     false, topk_idx_out,
                      topk_w_out, workspace, stream, stage_events);
 }
 
@@ -501,27 +509,65 @@ int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, con
   if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
     return KT_ERR_INVALID_CONFIG;
   if (!aligned(sf_up, 16) || !aligned(sf_down, 16)) return KT_ERR_ALIGN;
-  return run_forward(r, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y, false, topk_idx_out,
+  return run_forward(r, identity_table(r), T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y,
+                     false, topk_idx_out,
                      topk_w_out, workspace, stream, stage_events);
 }
 
 // ---------------------------------------------------------------------------
 // Expert-parallel form ("MoE 前向四步"): each rank runs the gate on all tokens,
-// its own routed experts [expert_begin, expert_end) and the shared experts on
-// its share of the tokens [shared_begin, shared_end), into an fp32 partial; the
-// caller sums the partials over the ranks (all-reduce) and kt_moe_ep_finish
-// adds the residual and rounds.
+// its own routed experts (a range, or any placement given as a slot table) and
+// the shared experts on its share of the tokens [shared_begin, shared_end),
+// into an fp32 partial; the caller sums the partials over the ranks
+// (all-reduce) and kt_moe_ep_finish adds the residual and rounds.
 // ---------------------------------------------------------------------------
 
-static int set_ep_range(Resolved* r, int64_t T, int expert_begin, int expert_end,
-                        int64_t shared_begin, int64_t shared_end) {
-  if (expert_begin < 0 || expert_begin > expert_end || expert_end > r->E)
-    return KT_ERR_INVALID_CONFIG;
+static int set_shared_range(Resolved* r, int64_t T, int64_t shared_begin, int64_t shared_end) {
   if (shared_begin < 0 || shared_begin > shared_end || shared_end > T) return KT_ERR_INVALID_CONFIG;
-  r->eb = expert_begin;
-  r->ee = expert_end;
   r->sb = (int)shared_begin;
   r->se = (int)shared_end;
+  return KT_OK;
+}
+
+// Routed experts [expert_begin, expert_end) in slots 0, 1, ...
+static int range_table(Resolved* r, int expert_begin, int expert_end, SlotTable* tab) {
+  if (expert_begin < 0 || expert_begin > expert_end || expert_end > r->E)
+    return KT_ERR_INVALID_CONFIG;
+  for (int e = 0; e < kMaxExperts; ++e)
+    tab->slot[e] = (int16_t)(e >= expert_begin && e < expert_end ? e - expert_begin : -1);
+  r->n_local = expert_end - expert_begin;
+  return KT_OK;
+}
+
+// expert_slot[e] (host, E entries): the weight slot of routed expert e, or -1;
+// the slots used must be exactly 0 .. n_local - 1, each once.
+static int placed_table(Resolved* r, const int32_t* expert_slot, SlotTable* tab) {
+  if (!expert_slot) return KT_ERR_NULL;
+  int n = 0;
+  for (int e = 0; e < r->E; ++e) {
+    if (expert_slot[e] < -1 || expert_slot[e] >= r->E) return KT_ERR_INVALID_CONFIG;
+    n += expert_slot[e] >= 0;
+  }
+  bool seen[kMaxExperts] = {};
+  for (int e = 0; e < kMaxExperts; ++e) tab->slot[e] = -1;
+  for (int e = 0; e < r->E; ++e) {
+    const int s = expert_slot[e];
+    if (s < 0) continue;
+    if (s >= n || seen[s]) return KT_ERR_INVALID_CONFIG;
+    seen[s] = true;
+    tab->slot[e] = (int16_t)s;
+  }
+  r->n_local = n;
+  return KT_OK;
+}
+
+static int mxfp8_weight_args(const Resolved& r, const uint8_t* w1q, const uint8_t* w3q,
+                             const uint8_t* sf_up, const uint8_t* sf_down) {
+  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
+  if (!sf_up || !sf_down) return KT_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
+    return KT_ERR_INVALID_CONFIG;
+  if (!aligned(sf_up, 16) || !aligned(sf_down, 16)) return KT_ERR_ALIGN;
   return KT_OK;
 }
 
@@ -531,13 +577,14 @@ int kt_moe_forward_local(const kt_moe_config* cfg, int64_t T, const void* x, con
                          const void* w2, float* y_part, int32_t* topk_idx_out, float* topk_w_out,
                          void* workspace, size_t ws_bytes, void* stream) {
   Resolved r;
+  SlotTable tab;
   int rc = check_forward_args(cfg, T, x, w_gate, bias, w1, w3, w2, y_part, topk_idx_out,
                               topk_w_out, workspace, ws_bytes, &r, /*y_partial=*/true);
   if (rc != KT_OK) return rc;
   if (r.fp8) return KT_ERR_INVALID_CONFIG;   // MXFP8 weights: kt_moe_forward_local_mxfp8
-  if ((rc = set_ep_range(&r, T, expert_begin, expert_end, shared_begin, shared_end)) != KT_OK)
-    return rc;
-  return run_forward(r, T, x, w_gate, bias, w1, w3, w2, nullptr, nullptr, y_part, true,
+  if ((rc = range_table(&r, expert_begin, expert_end, &tab)) != KT_OK) return rc;
+  if ((rc = set_shared_range(&r, T, shared_begin, shared_end)) != KT_OK) return rc;
+  return run_forward(r, tab, T, x, w_gate, bias, w1, w3, w2, nullptr, nullptr, y_part, true,
                      topk_idx_out, topk_w_out, workspace, stream, nullptr);
 }
 
@@ -549,17 +596,50 @@ int kt_moe_forward_local_mxfp8(const kt_moe_config* cfg, int64_t T, const void* 
                                int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                                size_t ws_bytes, void* stream) {
   Resolved r;
+  SlotTable tab;
   int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y_part, topk_idx_out,
                               topk_w_out, workspace, ws_bytes, &r, /*y_partial=*/true);
   if (rc != KT_OK) return rc;
-  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
-  if (!sf_up || !sf_down) return KT_ERR_NULL;
-  if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
-    return KT_ERR_INVALID_CONFIG;
-  if (!aligned(sf_up, 16) || !aligned(sf_down, 16)) return KT_ERR_ALIGN;
-  if ((rc = set_ep_range(&r, T, expert_begin, expert_end, shared_begin, shared_end)) != KT_OK)
-    return rc;
-  return run_forward(r, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y_part, true,
+  if ((rc = mxfp8_weight_args(r, w1q, w3q, sf_up, sf_down)) != KT_OK) return rc;
+  if ((rc = range_table(&r, expert_begin, expert_end, &tab)) != KT_OK) return rc;
+  if ((rc = set_shared_range(&r, T, shared_begin, shared_end)) != KT_OK) return rc;
+  return run_forward(r, tab, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y_part, true,
+                     topk_idx_out, topk_w_out, workspace, stream, nullptr);
+}
+
+int kt_moe_forward_placed(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
+                          const float* bias, const int32_t* expert_slot, int64_t shared_begin,
+                          int64_t shared_end, const void* w1, const void* w3, const void* w2,
+                          float* y_part, int32_t* topk_idx_out, float* topk_w_out,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  Resolved r;
+  SlotTable tab;
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1, w3, w2, y_part, topk_idx_out,
+                              topk_w_out, workspace, ws_bytes, &r, /*y_partial=*/true);
+  if (rc != KT_OK) return rc;
+  if (r.fp8) return KT_ERR_INVALID_CONFIG;   // MXFP8 weights: kt_moe_forward_placed_mxfp8
+  if ((rc = placed_table(&r, expert_slot, &tab)) != KT_OK) return rc;
+  if ((rc = set_shared_range(&r, T, shared_begin, shared_end)) != KT_OK) return rc;
+  return run_forward(r, tab, T, x, w_gate, bias, w1, w3, w2, nullptr, nullptr, y_part, true,
+                     topk_idx_out, topk_w_out, workspace, stream, nullptr);
+}
+
+int kt_moe_forward_placed_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x,
+                                const void* w_gate, const float* bias, const int32_t* expert_slot,
+                                int64_t shared_begin, int64_t shared_end, const uint8_t* w1q,
+                                const uint8_t* w3q, const uint8_t* w2q, const uint8_t* sf_up,
+                                const uint8_t* sf_down, float* y_part, int32_t* topk_idx_out,
+                                float* topk_w_out, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  Resolved r;
+  SlotTable tab;
+  int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y_part, topk_idx_out,
+                              topk_w_out, workspace, ws_bytes, &r, /*y_partial=*/true);
+  if (rc != KT_OK) return rc;
+  if ((rc = mxfp8_weight_args(r, w1q, w3q, sf_up, sf_down)) != KT_OK) return rc;
+  if ((rc = placed_table(&r, expert_slot, &tab)) != KT_OK) return rc;
+  if ((rc = set_shared_range(&r, T, shared_begin, shared_end)) != KT_OK) return rc;
+  return run_forward(r, tab, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y_part, true,
                      topk_idx_out, topk_w_out, workspace, stream, nullptr);
 }
 
@@ -586,7 +666,8 @@ size_t kt_moe_mxfp8_scale_bytes_local(const kt_moe_config* cfg, int expert_begin
                                       int down) {
   Resolved r;
   if (resolve(cfg, 1, 0, &r) != KT_OK || !r.fp8) return 0;
-  if (set_ep_range(&r, 1, expert_begin, expert_end, 0, 0) != KT_OK) return 0;
+  SlotTable tab;
+  if (range_table(&r, expert_begin, expert_end, &tab) != KT_OK) return 0;
   return mx_packed_bytes(r, down != 0);
 }
 
@@ -598,7 +679,8 @@ int kt_moe_mxfp8_pack_local(const kt_moe_config* cfg, int expert_begin, int expe
   int rc = resolve(cfg, 1, 0, &r);
   if (rc != KT_OK) return rc;
   if (!r.fp8) return KT_ERR_INVALID_CONFIG;
-  if ((rc = set_ep_range(&r, 1, expert_begin, expert_end, 0, 0)) != KT_OK) return rc;
+  SlotTable tab;
+  if ((rc = range_table(&r, expert_begin, expert_end, &tab)) != KT_OK) return rc;
   if (!w1 || !w3 || !w2 || !w1q || !w3q || !w2q || !sf_up || !sf_down) return KT_ERR_NULL;
   if (!aligned(w1, 16) || !aligned(w3, 16) || !aligned(w2, 16) || !aligned(w1q, 16) ||
       !aligned(w3q, 16) || !aligned(w2q, 16) || !aligned(sf_up, 16) || !aligned(sf_down, 16))

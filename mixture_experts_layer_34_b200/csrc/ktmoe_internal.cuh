@@ -53,8 +53,8 @@ struct Resolved {
   int act_bf16;     // tokens, gate weights and output in bf16 (KT_DTYPE_BF16 / MXFP8)
   int fp8;          // expert weights in MXFP8
   int chunk_rows;   // token rows per GEMM chunk: kChunkRows, or kChunkRowsF8 for MXFP8
-  int eb, ee;       // routed experts computed here: [eb, ee) (all: [0, E)); their weights
-                    // are the first ee - eb slots of w1/w3/w2, the shared ones follow
+  int n_local;      // routed experts computed here (all: E); their weights are the first
+                    // n_local slots of w1/w3/w2 (placed by a SlotTable), the shared ones follow
   int sb, se;       // tokens the shared experts run on here: [sb, se) (all: [0, T))
   int add_residual;
   int y_fp32;       // y in fp32 (else in dtype)
@@ -72,8 +72,15 @@ struct Chunk {
 };
 
 // Weight slots of a launch: the routed experts computed here, then the shared ones.
-inline int routed_slots(const Resolved& r) { return r.ee - r.eb; }
-inline int weight_slots(const Resolved& r) { return r.ee - r.eb + r.S; }
+inline int routed_slots(const Resolved& r) { return r.n_local; }
+inline int weight_slots(const Resolved& r) { return r.n_local + r.S; }
+
+// Routed expert -> weight slot of this launch, -1 for an expert computed
+// elsewhere (passed by value to the permutation kernels). The plain forward
+// uses the identity; the expert-parallel forms a range or any placement.
+struct SlotTable {
+  int16_t slot[kMaxExperts];
+};
 
 // Byte offsets of the workspace's internal buffers.
 struct Layout {
@@ -135,8 +142,9 @@ size_t balance_scratch_bytes(const Resolved& r, int64_t T);
 cudaError_t launch_balance_stats(const Resolved& r, int64_t T, const float* scores,
                                  const int32_t* idx, float alpha, float* f, float* P, float* loss,
                                  void* scratch, cudaStream_t st);
-cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* ws,
-                           const int32_t* idx, const float* w, const void* x, cudaStream_t st);
+cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, const Layout& L,
+                           char* ws, const int32_t* idx, const float* w, const void* x,
+                           cudaStream_t st);
 // up = true: the gate/up GEMM (wa = W1, wb = W3); up = false: the down GEMM
 // (wa = W2, wb unused).
 cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, char* ws,

@@ -124,8 +124,8 @@ __device__ void fill_tiles(int2* __restrict__ tiles, int F, int NG, const int* c
 }
 
 __global__ void __launch_bounds__(kScanThreads)
-permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int chunk_rows, int eb,
-                    int ee, int sb, int se,
+permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int chunk_rows,
+                    const __grid_constant__ SlotTable tab, int n_local, int sb, int se,
                     const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base,
                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                     Chunk* __restrict__ chunks, int2* __restrict__ tiles_up,
@@ -142,12 +142,12 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
   const int NG = E + S;
   // Per-expert totals over the chunks; shared experts hold tokens [sb, se) (all
   // T unless the caller splits them); routed experts outside [eb, ee) are
-  // computed elsewhere and hold none.
+  // computed elsewhere (slot -1) hold none.
   if (tid < NG) {
     int run = 0;
     if (tid >= E)
       run = se - sb;
-    else if (tid >= eb && tid < ee)
+    else if (tab.slot[tid] >= 0)
       for (int c = 0; c < nperm; ++c) run += chunk_counts[(int64_t)c * E + tid];
     tot[tid] = run;
     rows0[tid] = run;
@@ -182,12 +182,12 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
     meta[4] = 0;   // down GEMM tile counter
   }
   __syncthreads();
-  // The chunks name weight slots: routed expert g in slot g - eb, shared expert
-  // E + s in slot ee - eb + s.
+  // The chunks name weight slots: routed expert g in slot tab.slot[g], shared
+  // expert E + s in slot n_local + s.
   for (int i = tid; i < n_chunks; i += blockDim.x) {
     const int g = find_group(cb, NG, i);
     const int r = (i - cb[g]) * chunk_rows;
-    const int slot = g < E ? g - eb : ee - eb + (g - E);
+    const int slot = g < E ? tab.slot[g] : n_local + (g - E);
     const int row0 = g < E ? rows0[g] : rows0[g] + sb;
     const int src0 = g < E ? rows0[g] : sb;
     chunks[i] = Chunk{slot, row0 + r, min(chunk_rows, tot[g] - r), src0 + r};
@@ -201,8 +201,9 @@ enum { kNoCopy = 0, kCopyBf16 = 1, kCopyF8 = 2 };
 
 template <int kMode>
 __global__ void __launch_bounds__(256)
-permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int eb, int ee, int sb,
-                       int se,
+permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
+                       const __grid_constant__ SlotTable tab,
+                       int sb, int se,
                        const int32_t* __restrict__ idx, const float* __restrict__ w,
                        const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
                        const int32_t* __restrict__ gchunk0, int32_t* __restrict__ row_of,
@@ -230,7 +231,7 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int e
   for (int q = threadIdx.x; q < nent; q += blockDim.x) {
     const int tl = q / k;
     const int e = idx[(int64_t)t0 * k + q];
-    if (e < eb || e >= ee) {   // an expert computed elsewhere: no row here
+    if (tab.slot[e] < 0) {   // an expert computed elsewhere: no row here
       if (lead) row_of[(int64_t)t0 * k + q] = -1;
       srow[q] = -1;
       continue;
@@ -254,11 +255,19 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int e
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int tl = warp; tl < nt; tl += blockDim.x / 32) {
     const uint4* src = x + (int64_t)(t0 + tl) * nchunk;
-    for (int q = q0 + lane; q < q1; q += 32) {
-      const uint4 v = src[q];
+    // Four 16-byte loads in flight per lane, then their copies.
+    for (int q = q0 + lane; q < q1; q += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (q + 32 * u < q1) v[u] = src[q + 32 * u];
       for (int j = 0; j < k; ++j) {
         const int row = srow[tl * k + j];
-        if (row >= 0) xperm[(int64_t)row * nchunk + q] = v;
+        if (row < 0) continue;
+        uint4* dst = xperm + (int64_t)row * nchunk;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (q + 32 * u < q1) dst[q + 32 * u] = v[u];
       }
     }
   }
@@ -290,12 +299,13 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows, int e
 
 }  // namespace
 
-cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* ws,
-                           const int32_t* idx, const float* w, const void* x, cudaStream_t st) {
+cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, const Layout& L,
+                           char* ws, const int32_t* idx, const float* w, const void* x,
+                           cudaStream_t st) {
   auto I32 = [&](size_t off) { return reinterpret_cast<int32_t*>(ws + off); };
   (void)launch_pdl(permute_scan_kernel, dim3(1), dim3(kScanThreads), 0, st,
-      r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows, r.eb,
-      r.ee, r.sb, r.se,
+      r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows, tab,
+      r.n_local, r.sb, r.se,
       I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts), I32(L.offsets),
       reinterpret_cast<Chunk*>(ws + L.chunks), reinterpret_cast<int2*>(ws + L.tiles_up),
       reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0));
@@ -309,18 +319,18 @@ cudaError_t launch_permute(const Resolved& r, int64_t T, const Layout& L, char* 
   const int32_t* base = I32(L.chunk_base);
   if (r.fp8)
     (void)launch_pdl(permute_scatter_kernel<kCopyF8>, dim3(grid), dim3(256), 0, st,
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(ws + L.xq),
         reinterpret_cast<uint4*>(ws + L.xperm), reinterpret_cast<const uint8_t*>(ws + L.xs),
         reinterpret_cast<uint8_t*>(ws + L.tok_sf));
   else if (r.dtype == KT_DTYPE_BF16)
     (void)launch_pdl(permute_scatter_kernel<kCopyBf16>, dim3(grid), dim3(256), 0, st,
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(x),
         reinterpret_cast<uint4*>(ws + L.xperm), nullptr, nullptr);
   else
     (void)launch_pdl(permute_scatter_kernel<kNoCopy>, dim3(grid), dim3(256), 0, st,
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, r.eb, r.ee, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
+        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
         I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr, nullptr);
   return cudaGetLastError();
 }

@@ -7,8 +7,10 @@ of cards is the expert_parallel_degree setting of the tuning section of the
 DeepSeek model-family article (cloud.baidu.com/article/3606489).
 
 Per rank:
-  * the routed experts of one contiguous range (``expert_range``), held as a
-    local weight stack: those experts, then the shared ones (``local_stack``);
+  * the routed experts of one contiguous range (``expert_range``, the pages'
+    form), or of any placement (``balanced_placement`` spreads the heavy
+    experts of a skewed load over the ranks), held as a local weight stack:
+    those experts, then the shared ones (``local_stack``);
   * the gate on all tokens (every rank routes the same tokens identically), the
     local experts on their tokens, and the shared experts on this rank's share
     of the tokens (``token_range``), summed in fp32 by ``kt_moe_forward_local``;
@@ -53,30 +55,85 @@ def local_stack(w, n_experts: int, n_shared: int, begin: int, end: int):
     return torch.cat([w[begin:end], w[n_experts:n_experts + n_shared]]).contiguous()
 
 
+def local_stack_of(w, n_experts: int, n_shared: int, experts):
+    """The same for any list of routed experts (slot i holds experts[i])."""
+    idx = torch.as_tensor(list(experts) + list(range(n_experts, n_experts + n_shared)),
+                          dtype=torch.long, device=w.device)
+    return w.index_select(0, idx).contiguous()
+
+
+def contiguous_placement(n_experts: int, world: int) -> list[list[int]]:
+    """Each rank's experts as contiguous ranges (``expert_range``)."""
+    return [list(range(*expert_range(n_experts, world, r))) for r in range(world)]
+
+
+def balanced_placement(load, world: int) -> list[list[int]]:
+    """Experts over ranks by expected load (for example a previous batch's
+    per-expert token counts): heaviest first, each to the least-loaded rank that
+    still has room, so that every rank holds as many experts as a contiguous
+    split gives it. Each rank's list is in ascending expert order."""
+    load = [float(v) for v in load]
+    E = len(load)
+    cap = [e - b for b, e in (expert_range(E, world, r) for r in range(world))]
+    total = [0.0] * world
+    count = [0] * world
+    out: list[list[int]] = [[] for _ in range(world)]
+    for e in sorted(range(E), key=lambda i: (-load[i], i)):
+        r = min((r for r in range(world) if count[r] < cap[r]), key=lambda r: (total[r], r))
+        out[r].append(e)
+        total[r] += load[e]
+        count[r] += 1
+    return [sorted(x) for x in out]
+
+
+def slot_table(experts, n_experts: int) -> list[int]:
+    """expert -> weight slot on the rank holding ``experts`` (-1 elsewhere)."""
+    tab = [-1] * n_experts
+    for i, e in enumerate(experts):
+        if not 0 <= e < n_experts or tab[e] != -1:
+            raise ValueError(f"bad expert list: {experts}")
+        tab[e] = i
+    return tab
+
+
 class ExpertParallelMoE:
     """One rank of the expert-parallel layer.
 
     cfg: the full layer's kt_moe_config (all E routed experts). w1/w3/w2: the
     full stacked weights [E + S, ...] (sliced here), or, with
-    ``weights_are_local``, this rank's stack already. With an MXFP8 config the
-    local stacks (bf16) are packed once here.
+    ``weights_are_local``, this rank's stack already. placement: None for
+    contiguous ranges, else every rank's list of routed experts (the same
+    lists on every rank). With an MXFP8 config the local stacks (bf16) are
+    packed once here.
     """
 
     def __init__(self, cfg, w_gate, bias, w1, w3, w2, rank: int, world: int, group=None,
-                 weights_are_local: bool = False):
+                 weights_are_local: bool = False, placement=None):
         self.cfg, self.rank, self.world, self.group = cfg, rank, world, group
         E, S = cfg.n_experts, cfg.n_shared
-        self.eb, self.ee = expert_range(E, world, rank)
+        if placement is None:
+            self.eb, self.ee = expert_range(E, world, rank)
+            self.experts = list(range(self.eb, self.ee))
+            self.table = None
+        else:
+            if len(placement) != world or sorted(e for p in placement for e in p) != list(range(E)):
+                raise ValueError("placement must list every routed expert exactly once")
+            self.experts = list(placement[rank])
+            self.table = slot_table(self.experts, E)
         if not weights_are_local:
-            w1, w3, w2 = (local_stack(w, E, S, self.eb, self.ee) for w in (w1, w3, w2))
-        n_slots = self.ee - self.eb + S
+            if self.table is None:
+                w1, w3, w2 = (local_stack(w, E, S, self.eb, self.ee) for w in (w1, w3, w2))
+            else:
+                w1, w3, w2 = (local_stack_of(w, E, S, self.experts) for w in (w1, w3, w2))
+        n_local = len(self.experts)
+        n_slots = n_local + S
         for w in (w1, w3, w2):
             if w.shape[0] != n_slots:
                 raise ValueError(f"local stack has {w.shape[0]} slots, expected {n_slots}")
         self.w_gate, self.bias = w_gate, bias
         self.mxfp8 = cfg.dtype == K.KT_DTYPE_MXFP8
         if self.mxfp8:
-            self.q = K.pack_mxfp8_local(cfg, self.eb, self.ee, w1, w3, w2)
+            self.q = K.pack_mxfp8_local(cfg, 0, n_local, w1, w3, w2)
             self.w1 = self.w3 = self.w2 = None
         else:
             self.q = None
@@ -99,8 +156,15 @@ class ExpertParallelMoE:
         T = x.shape[0]
         ws, _ = self.buffers(T, x.device)
         sb, se = self.shared_range(T)
-        if self.mxfp8:
-            q = self.q
+        q = self.q
+        if self.table is not None and self.mxfp8:
+            K.kt_moe_forward_placed_mxfp8(self.cfg, T, x, self.w_gate, self.bias, self.table, sb, se,
+                                          q["w1q"], q["w3q"], q["w2q"], q["sf_up"], q["sf_down"],
+                                          part, topk_idx, topk_w, ws)
+        elif self.table is not None:
+            K.kt_moe_forward_placed(self.cfg, T, x, self.w_gate, self.bias, self.table, sb, se,
+                                    self.w1, self.w3, self.w2, part, topk_idx, topk_w, ws)
+        elif self.mxfp8:
             K.kt_moe_forward_local_mxfp8(self.cfg, T, x, self.w_gate, self.bias, self.eb, self.ee,
                                          sb, se, q["w1q"], q["w3q"], q["w2q"], q["sf_up"],
                                          q["sf_down"], part, topk_idx, topk_w, ws)

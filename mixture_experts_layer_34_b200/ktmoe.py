@@ -31,7 +31,8 @@ EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_fo
            "kt_moe_graph_destroy", "kt_moe_mxfp8_quantize", "kt_moe_mxfp8_scale_bytes",
            "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8", "kt_moe_graph_create_mxfp8",
            "kt_moe_forward_local", "kt_moe_forward_local_mxfp8", "kt_moe_ep_finish",
-           "kt_moe_mxfp8_scale_bytes_local", "kt_moe_mxfp8_pack_local")
+           "kt_moe_mxfp8_scale_bytes_local", "kt_moe_mxfp8_pack_local", "kt_moe_forward_placed",
+           "kt_moe_forward_placed_mxfp8")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -129,6 +130,12 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_forward_local_mxfp8.argtypes = [CP, I64, P, P, P, C, C, I64, I64, P, P, P, P,
                                                      P, P, P, P, P, ctypes.c_size_t, P]
             L.kt_moe_forward_local_mxfp8.restype = ctypes.c_int
+            L.kt_moe_forward_placed.argtypes = [CP, I64, P, P, P, P, I64, I64, P, P, P, P, P, P,
+                                                P, ctypes.c_size_t, P]
+            L.kt_moe_forward_placed.restype = ctypes.c_int
+            L.kt_moe_forward_placed_mxfp8.argtypes = [CP, I64, P, P, P, P, I64, I64, P, P, P, P, P,
+                                                      P, P, P, P, ctypes.c_size_t, P]
+            L.kt_moe_forward_placed_mxfp8.restype = ctypes.c_int
             L.kt_moe_ep_finish.argtypes = [CP, I64, P, P, P, P]
             L.kt_moe_ep_finish.restype = ctypes.c_int
             L.kt_moe_mxfp8_scale_bytes_local.argtypes = [CP, C, C, C]
@@ -363,6 +370,38 @@ def kt_moe_forward_local_mxfp8(cfg, T, x, w_gate, bias, expert_begin, expert_end
         _ptr(workspace), _nbytes(workspace), _stream(stream))
     if rc != KT_OK:
         raise KtMoeError("kt_moe_forward_local_mxfp8", rc)
+
+
+def _slot_array(expert_slot):
+    arr = (ctypes.c_int32 * len(expert_slot))(*[int(v) for v in expert_slot])
+    return arr
+
+
+def kt_moe_forward_placed(cfg, T, x, w_gate, bias, expert_slot, shared_begin, shared_end, w1, w3,
+                          w2, y_part, topk_idx_out, topk_w_out, workspace, stream=None):
+    """kt_moe_forward_local with any placement: expert_slot[e] = the weight slot
+    of routed expert e on this rank, or -1 (a sequence of n_experts ints)."""
+    tab = _slot_array(expert_slot)
+    rc = lib().kt_moe_forward_placed(ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias),
+                                     ctypes.cast(tab, ctypes.c_void_p), int(shared_begin),
+                                     int(shared_end), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y_part),
+                                     _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
+                                     _nbytes(workspace), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_forward_placed", rc)
+
+
+def kt_moe_forward_placed_mxfp8(cfg, T, x, w_gate, bias, expert_slot, shared_begin, shared_end,
+                                w1q, w3q, w2q, sf_up, sf_down, y_part, topk_idx_out, topk_w_out,
+                                workspace, stream=None):
+    tab = _slot_array(expert_slot)
+    rc = lib().kt_moe_forward_placed_mxfp8(
+        ctypes.byref(cfg), int(T), _ptr(x), _ptr(w_gate), _ptr(bias),
+        ctypes.cast(tab, ctypes.c_void_p), int(shared_begin), int(shared_end), _ptr(w1q),
+        _ptr(w3q), _ptr(w2q), _ptr(sf_up), _ptr(sf_down), _ptr(y_part), _ptr(topk_idx_out),
+        _ptr(topk_w_out), _ptr(workspace), _nbytes(workspace), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_forward_placed_mxfp8", rc)
 
 
 def kt_moe_ep_finish(cfg, T, y_sum, x, y, stream=None):

@@ -258,6 +258,34 @@ def test_expert_parallel_host_side_errors():
                                      None) == K.KT_ERR_INVALID_CONFIG
 
 
+def test_placed_table_host_side_errors():
+    """kt_moe_forward_placed validates the slot table on the host: every slot
+    used is one of 0 .. n_local - 1, exactly once."""
+    layer = W.BY_NAME["small_sig_bias"]          # E = 32
+    cfg = K.config_for(layer)
+    L = K.lib()
+    V = ctypes.c_void_p
+    T, E = layer.T, layer.n_experts
+    need = K.kt_moe_workspace_size(cfg, T)
+    ptr = lambda i: V(0x10000 * (i + 1))
+
+    def placed(tab):
+        arr = None if tab is None else (ctypes.c_int32 * E)(*tab)
+        return L.kt_moe_forward_placed(ctypes.byref(cfg), T, ptr(0), ptr(1), ptr(2),
+                                       None if arr is None else ctypes.cast(arr, V), 0, T,
+                                       ptr(3), ptr(4), ptr(5), ptr(7), None, None, V(0x7000000),
+                                       need, None)
+
+    base = [-1] * E
+    dup = list(base); dup[3] = 0; dup[9] = 0            # slot 0 twice
+    gap = list(base); gap[3] = 0; gap[9] = 2            # slots 0 and 2: 1 missing
+    low = list(base); low[4] = -2
+    high = list(base); high[4] = E
+    for tab in (dup, gap, low, high):
+        assert placed(tab) == K.KT_ERR_INVALID_CONFIG, tab
+    assert placed(None) == K.KT_ERR_NULL
+
+
 def test_strerror_covers_codes():
     for code in range(-8, 1):
         assert K.strerror(code) and K.strerror(code) != "unknown error code"

@@ -120,7 +120,7 @@ def _ep_layer():
     return layer, W.make_layer(layer, "cpu")
 
 
-def _ep_worker(rank, world, port, q):
+def _ep_worker(rank, world, port, q, placed=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
     import numpy as np
@@ -141,23 +141,24 @@ def _ep_worker(rank, world, port, q):
             """The two kernels replaced by the oracle, on this rank's local stacks."""
 
             def local(self, x, part, topk_idx=None, topk_w=None):
-                n_local = self.ee - self.eb
+                n_local = len(self.experts)
                 lists = []
                 for stack in (self.w1, self.w3, self.w2):
                     full = [None] * (E + S)
-                    for i in range(n_local):
-                        full[self.eb + i] = stack[i]
+                    for i, e in enumerate(self.experts):
+                        full[e] = stack[i]
                     for s in range(S):
                         full[E + s] = stack[n_local + s]
                     lists.append(full)
                 T = x.shape[0]
-                yr, _ = O.forward_part(fields, x, idx, w, *lists, range(T), True, self.eb,
-                                       self.ee, shared=False)
+                part.zero_()
+                for e in self.experts:     # the rank's experts, one range each
+                    yr, _ = O.forward_part(fields, x, idx, w, *lists, range(T), True, e, e + 1,
+                                           shared=False)
+                    part += torch.from_numpy(yr)
                 sb, se = self.shared_range(T)
-                part.copy_(torch.from_numpy(yr))
                 if se > sb:
-                    _, ys = O.forward_part(fields, x, idx, w, *lists, range(sb, se), True,
-                                           self.eb, self.ee)
+                    _, ys = O.forward_part(fields, x, idx, w, *lists, range(sb, se), True, 0, 0)
                     part[sb:se] += torch.from_numpy(ys)
 
             def buffers(self, T, device):
@@ -168,15 +169,19 @@ def _ep_worker(rank, world, port, q):
                 y.copy_(part + (x.to(torch.float64) if layer.add_residual else 0))
 
         cfg = K.config_for(layer)
+        placement = None
+        if placed:   # a seeded shuffle of the experts, the same on every rank
+            perm = np.random.default_rng(5).permutation(E).tolist()
+            placement = [sorted(perm[r::world]) for r in range(world)]
         m = OracleRank(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], rank,
-                       world)
+                       world, placement=placement)
         y = torch.empty(x.shape[0], layer.dim, dtype=torch.float64)
         m.forward(x, y)
         dist.destroy_process_group()
         ref = O.forward(fields, x, idx, w, inp["w1"], inp["w3"], inp["w2"], range(x.shape[0]),
                         True)
         err = float(np.abs(y.numpy() - ref).max() / np.abs(ref).max())
-        q.put((rank, (m.eb, m.ee), err))
+        q.put((rank, (m.experts[0], m.experts[-1] + 1) if not placed else len(m.experts), err))
     except Exception as e:  # pragma: no cover - reported to the parent
         import traceback
         q.put((rank, None, traceback.format_exc()))
@@ -188,3 +193,33 @@ def test_expert_parallel_sum_is_the_forward_gloo():
     for rank, rng, err in out:
         assert isinstance(err, float), err
         assert err < 1e-12, (rank, err)
+
+
+def _ep_worker_placed(rank, world, port, q):
+    _ep_worker(rank, world, port, q, placed=True)
+
+
+def test_expert_parallel_with_a_placement_gloo():
+    out = _run(2, _ep_worker_placed)
+    assert [r[1] for r in out] == [16, 16], out
+    for rank, n, err in out:
+        assert isinstance(err, float), err
+        assert err < 1e-12, (rank, err)
+
+
+def test_balanced_placement_evens_a_skewed_load():
+    import numpy as np
+    from mixture_experts_layer_34_b200 import ep
+    load = np.random.default_rng(3).zipf(1.3, 256).astype(float)
+    for world in (2, 4, 8):
+        p = ep.balanced_placement(load, world)
+        assert sorted(e for r in p for e in r) == list(range(256))
+        assert [len(r) for r in p] == [len(r) for r in ep.contiguous_placement(256, world)]
+        per = [load[r].sum() for r in p]
+        cont = [load[r].sum() for r in ep.contiguous_placement(256, world)]
+        # The greedy bound: no rank exceeds the mean by more than the heaviest expert.
+        assert max(per) <= load.sum() / world + load.max() + 1e-9
+        assert max(per) <= max(cont)
+    assert ep.slot_table([5, 2, 7], 8) == [-1, -1, 1, -1, -1, 0, -1, 2]
+    with pytest.raises(ValueError):
+        ep.slot_table([1, 1], 4)

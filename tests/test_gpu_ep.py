@@ -239,3 +239,79 @@ def test_mxfp8_class_one_rank_is_the_forward():
     y = torch.empty_like(yf)
     m.forward(inp["x"], y)
     assert torch.equal(y, yf)
+
+
+# ----------------------------------------------------------------------------
+# Placements other than contiguous ranges (kt_moe_forward_placed)
+# ----------------------------------------------------------------------------
+
+def _shuffled_placement(E, world, seed=9):
+    perm = np.random.default_rng(seed).permutation(E).tolist()
+    return [sorted(perm[r::world]) for r in range(world)]
+
+
+def _oracle_set_part(layer, inp, og, experts, sb, se, toks):
+    """The oracle's part for a set of routed experts: one range per expert."""
+    total = np.zeros((len(toks), layer.dim))
+    for e in experts:
+        total += _oracle_part(layer, inp, og, e, e + 1, 0, 0, toks)
+    return total + _oracle_part(layer, inp, og, 0, 0, sb, se, toks)
+
+
+@pytest.mark.parametrize("name", ["small_sig_bias", "small_softmax_ragged", "small_fp32_groups"])
+def test_placed_ranks_match_the_oracle(name):
+    layer = W.BY_NAME[name]
+    world = 3
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer, y_fp32=True)
+    full = run_forward(layer, inp, y_fp32=True)
+    og = oracle_gate(layer, inp)
+    diff, near = routing_agreement(layer, og, full["idx"].cpu().numpy())
+    assert near[diff].all()
+    toks = [t for t in range(layer.T) if t not in set(diff.tolist())]
+    sel = torch.as_tensor(toks, device="cuda")
+    y_ref = oracle_outputs(layer, inp, og, toks)
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    placement = _shuffled_placement(layer.n_experts, world)
+    y_sum = torch.zeros((layer.T, layer.dim), device="cuda")
+    for rank in range(world):
+        m = ep.ExpertParallelMoE(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                                 rank, world, placement=placement)
+        ws, part = m.buffers(layer.T, inp["x"].device)
+        part.fill_(float("nan"))
+        idx = torch.empty_like(full["idx"])
+        m.local(inp["x"], part, idx)
+        assert K.kt_moe_check(ws) == K.KT_OK
+        assert torch.equal(idx, full["idx"])
+        sb, se = m.shared_range(layer.T)
+        ref = _oracle_set_part(layer, inp, og, m.experts, sb, se, toks)
+        err = float(np.abs(part[sel].cpu().numpy() - ref).max())
+        assert err <= tolerance(layer) * rms, (rank, err / rms)
+        y_sum += part
+    y = _finish(layer, inp, y_sum, True)
+    assert float(np.abs(y[sel].cpu().numpy() - y_ref).max()) <= tolerance(layer) * rms
+    frms = float(full["y"].square().mean().sqrt())
+    assert float((y - full["y"]).abs().max()) <= SUM_ORDER_TOL * frms
+
+
+def test_mxfp8_placed_ranks_sum_to_the_forward():
+    layer = W.BY_NAME["small_sig_bias_mxfp8"]
+    world = 4
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer, y_fp32=True)
+    qf = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+    ws = K.alloc_workspace(cfg, layer.T)
+    yf = torch.empty((layer.T, layer.dim), device="cuda")
+    K.kt_moe_forward_mxfp8(cfg, layer.T, inp["x"], inp["w_gate"], inp["bias"], qf["w1q"],
+                           qf["w3q"], qf["w2q"], qf["sf_up"], qf["sf_down"], yf, None, None, ws)
+    placement = _shuffled_placement(layer.n_experts, world, seed=4)
+    y_sum = torch.zeros((layer.T, layer.dim), device="cuda")
+    for rank in range(world):
+        m = ep.ExpertParallelMoE(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                                 rank, world, placement=placement)
+        _, part = m.buffers(layer.T, inp["x"].device)
+        m.local(inp["x"], part)
+        y_sum += part
+    y = _finish(layer, inp, y_sum, True)
+    rms = float(yf.square().mean().sqrt())
+    assert float((y - yf).abs().max()) <= SUM_ORDER_TOL * rms
