@@ -183,11 +183,14 @@ cudaError_t launch_ep_finish(const Resolved& r, int64_t T, const float* y_sum, c
   const unsigned grid = (unsigned)std::min<int64_t>((n4 + 255) / 256, (int64_t)num_sms * 8);
   const float4* ys = reinterpret_cast<const float4*>(y_sum);
   if (r.act_bf16 && !r.y_fp32)
-    (void)launch_pdl(ep_finish_kernel<true, false>, dim3(grid), dim3(256), 0, st, n4, r.add_residual, ys, x, y);
+    (void)launch_pdl(ep_finish_kernel<true, false>, dim3(grid), dim3(256), 0, st, n4,
+                     r.add_residual, ys, x, y);
   else if (r.act_bf16)
-    (void)launch_pdl(ep_finish_kernel<true, true>, dim3(grid), dim3(256), 0, st, n4, r.add_residual, ys, x, y);
+    (void)launch_pdl(ep_finish_kernel<true, true>, dim3(grid), dim3(256), 0, st, n4,
+                     r.add_residual, ys, x, y);
   else
-    (void)launch_pdl(ep_finish_kernel<false, true>, dim3(grid), dim3(256), 0, st, n4, r.add_residual, ys, x, y);
+    (void)launch_pdl(ep_finish_kernel<false, true>, dim3(grid), dim3(256), 0, st, n4,
+                     r.add_residual, ys, x, y);
   return cudaGetLastError();
 }
 
@@ -195,15 +198,16 @@ cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* 
                            void* y, cudaStream_t st) {
   const int32_t* row_of = reinterpret_cast<const int32_t*>(ws + L.row_of);
   const float* eo = reinterpret_cast<const float*>(ws + L.expert_out);
+  const dim3 grid = combine_grid(T, r.d);
   if (r.act_bf16 && !r.y_fp32)
-    (void)launch_pdl(combine_kernel<true, false>, dim3(combine_grid(T, r.d)), dim3(128), 0, st, (int)T, r.k, r.S, r.d, r.add_residual,
-                                                             row_of, eo, x, y);
+    (void)launch_pdl(combine_kernel<true, false>, grid, dim3(128), 0, st, (int)T, r.k, r.S, r.d,
+                     r.add_residual, row_of, eo, x, y);
   else if (r.act_bf16)
-    (void)launch_pdl(combine_kernel<true, true>, dim3(combine_grid(T, r.d)), dim3(128), 0, st, (int)T, r.k, r.S, r.d, r.add_residual,
-                                                            row_of, eo, x, y);
+    (void)launch_pdl(combine_kernel<true, true>, grid, dim3(128), 0, st, (int)T, r.k, r.S, r.d,
+                     r.add_residual, row_of, eo, x, y);
   else
-    (void)launch_pdl(combine_kernel<false, true>, dim3(combine_grid(T, r.d)), dim3(128), 0, st, (int)T, r.k, r.S, r.d, r.add_residual,
-                                                             row_of, eo, x, y);
+    (void)launch_pdl(combine_kernel<false, true>, grid, dim3(128), 0, st, (int)T, r.k, r.S, r.d,
+                     r.add_residual, row_of, eo, x, y);
   return cudaGetLastError();
 }
 

@@ -431,23 +431,26 @@ cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, cons
     const int vn = bf16 ? 8 : 4;
     const int kc = ((r.d + kSplitK - 1) / kSplitK + vn - 1) / vn * vn;
     const dim3 grid((unsigned)((r.E + 31) / 32), kSplitK);
+    const dim3 block(kSmallWarps * 32);
     if (bf16)
-      (void)launch_pdl(gate_logits_splitk_kernel<__nv_bfloat16>, dim3(grid), dim3(kSmallWarps * 32), 0, st,
-          (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d, kc);
+      (void)launch_pdl(gate_logits_splitk_kernel<__nv_bfloat16>, grid, block, 0, st,
+                       (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T,
+                       r.E, r.d, kc);
     else
-      (void)launch_pdl(gate_logits_splitk_kernel<float>, dim3(grid), dim3(kSmallWarps * 32), 0, st,
-          (const float*)x, (const float*)w_gate, logits, (int)T, r.E, r.d, kc);
+      (void)launch_pdl(gate_logits_splitk_kernel<float>, grid, block, 0, st, (const float*)x,
+                       (const float*)w_gate, logits, (int)T, r.E, r.d, kc);
     return cudaGetLastError();
   }
   // Tensor-core logits write 16-byte chunks of fp32 rows of E entries.
   if (bf16 && r.E % 4 == 0) return launch_gate_logits_tc(r, T, x, w_gate, logits, err, num_sms, st);
   dim3 grid((r.E + kLE - 1) / kLE, (unsigned)((T + kLT - 1) / kLT));
   if (bf16)
-    (void)launch_pdl(gate_logits_kernel<__nv_bfloat16>, dim3(grid), dim3(kLThreads), 0, st,
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E, r.d);
+    (void)launch_pdl(gate_logits_kernel<__nv_bfloat16>, grid, dim3(kLThreads), 0, st,
+                     (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T, r.E,
+                     r.d);
   else
-    (void)launch_pdl(gate_logits_kernel<float>, dim3(grid), dim3(kLThreads), 0, st, (const float*)x, (const float*)w_gate,
-                                                          logits, (int)T, r.E, r.d);
+    (void)launch_pdl(gate_logits_kernel<float>, grid, dim3(kLThreads), 0, st, (const float*)x,
+                     (const float*)w_gate, logits, (int)T, r.E, r.d);
   return cudaGetLastError();
 }
 
@@ -457,9 +460,9 @@ cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits
   const unsigned grid = (unsigned)((T + kPermChunk - 1) / kPermChunk);
   const int ks = scores_in ? 1 : gate_logit_splits(r, T);
   const int np = (r.E + 31) / 32;
-#define KT_SELECT(NPV)                                                                        \
-  (void)launch_pdl(gate_select_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, ks, logits, scores_in, \
-                                                           bias, idx, w, chunk_counts)
+#define KT_SELECT(NPV)                                                                         \
+  (void)launch_pdl(gate_select_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, \
+                   ks, logits, scores_in, bias, idx, w, chunk_counts)
   if (np <= 1) KT_SELECT(1);
   else if (np <= 2) KT_SELECT(2);
   else if (np <= 4) KT_SELECT(4);
@@ -479,7 +482,8 @@ cudaError_t launch_gate_scores(const Resolved& r, int64_t T, const float* logits
   const int ks = gate_logit_splits(r, T);
   const int np = (r.E + 31) / 32;
 #define KT_SCORES(NPV) \
-  (void)launch_pdl(gate_scores_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, ks, logits, scores)
+  (void)launch_pdl(gate_scores_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, \
+                   ks, logits, scores)
   if (np <= 1) KT_SCORES(1);
   else if (np <= 2) KT_SCORES(2);
   else if (np <= 4) KT_SCORES(4);

@@ -303,35 +303,40 @@ cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, c
                            char* ws, const int32_t* idx, const float* w, const void* x,
                            cudaStream_t st) {
   auto I32 = [&](size_t off) { return reinterpret_cast<int32_t*>(ws + off); };
-  (void)launch_pdl(permute_scan_kernel, dim3(1), dim3(kScanThreads), 0, st,
-      r.E, r.S, (int)T, r.k, (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows, tab,
-      r.n_local, r.sb, r.se,
-      I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts), I32(L.offsets),
-      reinterpret_cast<Chunk*>(ws + L.chunks), reinterpret_cast<int2*>(ws + L.tiles_up),
-      reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0));
+  (void)launch_pdl(permute_scan_kernel, dim3(1), dim3(kScanThreads), 0, st, r.E, r.S, (int)T, r.k,
+                   (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows, tab,
+                   r.n_local, r.sb, r.se, I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts),
+                   I32(L.offsets), reinterpret_cast<Chunk*>(ws + L.chunks),
+                   reinterpret_cast<int2*>(ws + L.tiles_up),
+                   reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // Few chunks (a decode step): split each chunk's row copies over column
   // slices so that about two CTAs per SM copy.
-  const int slices = r.act_bf16 ? (int)std::max<int64_t>(1, std::min<int64_t>(16, (296 + L.nperm - 1) / L.nperm)) : 1;
+  const int64_t want = (296 + L.nperm - 1) / L.nperm;
+  const int slices = r.act_bf16 ? (int)std::max<int64_t>(1, std::min<int64_t>(16, want)) : 1;
   const dim3 grid((unsigned)L.nperm, (unsigned)slices);
   float* rw = reinterpret_cast<float*>(ws + L.row_weight);
   const int32_t* base = I32(L.chunk_base);
   if (r.fp8)
-    (void)launch_pdl(permute_scatter_kernel<kCopyF8>, dim3(grid), dim3(256), 0, st,
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
-        I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(ws + L.xq),
-        reinterpret_cast<uint4*>(ws + L.xperm), reinterpret_cast<const uint8_t*>(ws + L.xs),
-        reinterpret_cast<uint8_t*>(ws + L.tok_sf));
+    (void)launch_pdl(permute_scatter_kernel<kCopyF8>, grid, dim3(256), 0, st, r.E, r.S, (int)T,
+                     r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
+                     I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw,
+                     reinterpret_cast<const uint4*>(ws + L.xq),
+                     reinterpret_cast<uint4*>(ws + L.xperm),
+                     reinterpret_cast<const uint8_t*>(ws + L.xs),
+                     reinterpret_cast<uint8_t*>(ws + L.tok_sf));
   else if (r.dtype == KT_DTYPE_BF16)
-    (void)launch_pdl(permute_scatter_kernel<kCopyBf16>, dim3(grid), dim3(256), 0, st,
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
-        I32(L.row_of), I32(L.tok_of), rw, reinterpret_cast<const uint4*>(x),
-        reinterpret_cast<uint4*>(ws + L.xperm), nullptr, nullptr);
+    (void)launch_pdl(permute_scatter_kernel<kCopyBf16>, grid, dim3(256), 0, st, r.E, r.S, (int)T,
+                     r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
+                     I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw,
+                     reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(ws + L.xperm),
+                     nullptr, nullptr);
   else
-    (void)launch_pdl(permute_scatter_kernel<kNoCopy>, dim3(grid), dim3(256), 0, st,
-        r.E, r.S, (int)T, r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets), I32(L.gchunk0),
-        I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr, nullptr);
+    (void)launch_pdl(permute_scatter_kernel<kNoCopy>, grid, dim3(256), 0, st, r.E, r.S, (int)T,
+                     r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
+                     I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr,
+                     nullptr);
   return cudaGetLastError();
 }
 
