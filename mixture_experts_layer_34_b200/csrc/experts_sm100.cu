@@ -764,13 +764,16 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
               // K = 32 MMAs, each reading its K block's scale byte.
               const uint32_t sS = smem_u32(sf_base + stage * kScaleStageBytes);
               const uint32_t sB = sS + kSlabsLight * kSfaSlabBytes + j * kSfbSlabBytes;
-              sf_copy_pair(tmem_base + kSfaCol, sS + j * kSfaSlabBytes);
-              sf_copy_pair(tmem_base + kSfbCol, sB);
-              sf_copy_pair(tmem_base + kSfbCol + 4, sB + kSfbSlabBytes / 2);
+              // Token rows 128 and up (second half of the slab's token scales)
+              // exist only in tiles of more than 128 columns.
+              const uint32_t sfa = tmem_base + kSfaCol, sfb = tmem_base + kSfbCol;
+              sf_copy_pair(sfa, sS + j * kSfaSlabBytes);
+              sf_copy_pair(sfb, sB);
+              if (n > 128) sf_copy_pair(sfb + 4, sB + kSfbSlabBytes / 2);
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                mma_pair_mxf8(d0, da + 2 * ks, db + 2 * ks, idesc_mxf8(256, n, ks),
-                              tmem_base + kSfaCol, tmem_base + kSfbCol, (kb | j | ks) != 0);
+                mma_pair_mxf8(d0, da + 2 * ks, db + 2 * ks, idesc_mxf8(256, n, ks), sfa, sfb,
+                              (kb | j | ks) != 0);
             } else {
 #pragma unroll
               for (int ks = 0; ks < kBK / 16; ++ks)
