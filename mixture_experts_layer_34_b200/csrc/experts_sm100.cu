@@ -836,6 +836,18 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
       }
       if (ch.group < 0) break;
       const int n = pair_cols(ch.nrows);
+      // Down: the routing weights of the tile's rows (lane l holds rows l + 32 i;
+      // shared-expert rows weigh 1), loaded before the accumulator wait so their
+      // latency overlaps it instead of stalling every 16-column block.
+      constexpr bool kDown = kKind == kKindDown || kKind == kKindDownF8;
+      float rw[kDown ? 8 : 1];
+      if (kDown) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = lane + 32 * i, row = ch.row0 + r;
+          rw[i] = (r < ch.nrows && row < args.n_routed_rows) ? args.row_weight[row] : 1.0f;
+        }
+      }
       const bool ready = mbar_wait(&tfull_bar[buf], bphase, err, 4 + 8 * kKind);
       if (!uniform_ok<kUp>(ready, 1 + pr)) break;
       tc_fence_after();
@@ -858,14 +870,15 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           float* xc = xchg + (pr * 2 + xb) * 16 * 32;
           const int mine0 = gate_warp ? 0 : 8, other0 = 8 - mine0;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) xc[(other0 + i) * 32 + lane] = v[other0 + i];
+          for (int i = 0; i < 8; ++i) xc[(other0 + i) * 32 + lane] = gate_warp ? v[8 + i] : v[i];
           asm volatile("bar.sync %0, 64;" ::"r"(1 + pr) : "memory");
           xb ^= 1;
           uint8_t* s8 = stg;
           uint8_t my_scale = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float mv = v[mine0 + i], ov = xc[(mine0 + i) * 32 + lane];
+            // (static indices into v: the selects keep it in registers)
+            const float mv = gate_warp ? v[i] : v[8 + i], ov = xc[(mine0 + i) * 32 + lane];
             const float h = gate_warp ? silu(mv) * ov : silu(ov) * mv;
             const uint32_t amax =
                 __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7fffffffu);
@@ -905,11 +918,15 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
               sb[i * 32 + lane] = __float2bfloat16_rn(silu(v[i]) * xc[i * 32 + lane]);
           }
         } else {
-          if (kKind == kKindDown || kKind == kKindDownF8) {
+          if (kDown) {
+            // Column c0 + i is row c0 + i of the tile: lane (c0 + i) % 32 holds
+            // its weight in rw[0] (c0 is a multiple of 16; rw moves down one
+            // register after every 32 columns, so all indices stay static).
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int row = ch.row0 + c0 + i;
-              v[i] *= row < args.n_routed_rows ? args.row_weight[row] : 1.0f;
+            for (int i = 0; i < 16; ++i) v[i] *= __shfl_sync(0xffffffffu, rw[0], (c0 & 16) + i);
+            if (c0 & 16) {
+#pragma unroll
+              for (int k = 0; k + 1 < (kDown ? 8 : 1); ++k) rw[k] = rw[k + 1];
             }
           }
           float* sf = reinterpret_cast<float*>(stg);
