@@ -68,6 +68,9 @@ def parse_args(argv=None):
     ap.add_argument("--parallel", choices=("dp", "ep"), default="dp",
                     help="N>1: dp = replicas on their own tokens (default); ep = experts "
                          "split over the ranks, one all-reduce per step")
+    ap.add_argument("--ep-placement", choices=("contiguous", "balanced"), default="balanced",
+                    help="--parallel ep: experts in contiguous ranges, or placed by the load "
+                         "of another seeded batch")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -283,14 +286,7 @@ def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
         torch.cuda.synchronize()
         return t0.elapsed_time(t1) / steps
 
-    # Expected load: the routing of another seeded batch (rank 1's tokens).
-    g = torch.Generator(device="cpu").manual_seed(rank_tokens_seed(layer, 1))
-    x2 = torch.randn(inp["x"].shape, generator=g).to(inp["x"].dtype).to(dev)
-    idx2 = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
-    w2_ = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
-    K.kt_moe_gate(cfg, T, x2, inp["w_gate"], inp["bias"], None, idx2, w2_, ws)
-    load2 = np.bincount(idx2.cpu().numpy().ravel(), minlength=E)
-    del x2
+    load2 = expected_load(layer, inp, dev)
     placements = {"contiguous": ep.contiguous_placement(E, ranks),
                   "balanced": ep.balanced_placement(load2, ranks)}
     out = {}
@@ -335,15 +331,34 @@ def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
     return res
 
 
-def time_ep_layer(layer, dev, rank, world, steps, warmup):
+def expected_load(layer, inp, dev) -> np.ndarray:
+    """Per-expert token counts of another seeded batch of the same workload (the
+    tokens of rank 1 of a data-parallel run), routed by kt_moe_gate."""
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    cfg = K.config_for(layer)
+    T = layer.T
+    g = torch.Generator(device="cpu").manual_seed(rank_tokens_seed(layer, 1))
+    x2 = torch.randn(inp["x"].shape, generator=g).to(inp["x"].dtype).to(dev)
+    ws = K.alloc_workspace(cfg, T, dev)
+    idx = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
+    w = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
+    K.kt_moe_gate(cfg, T, x2, inp["w_gate"], inp["bias"], None, idx, w, ws)
+    return np.bincount(idx.cpu().numpy().ravel(), minlength=layer.n_experts)
+
+
+def time_ep_layer(layer, dev, rank, world, steps, warmup, placement_kind="balanced"):
     """N > 1, --parallel ep: the expert-parallel layer over the process group
-    (NCCL all-reduce of the fp32 partials); the same T tokens on every rank."""
+    (NCCL all-reduce of the fp32 partials); the same T tokens on every rank.
+    Every rank computes the same placement from the same seeded batch."""
     from mixture_experts_layer_34_b200 import ep
     from mixture_experts_layer_34_b200 import ktmoe as K
     inp = W.make_layer(layer, dev)
     cfg = K.config_for(layer)
+    placement = None
+    if placement_kind == "balanced":
+        placement = ep.balanced_placement(expected_load(layer, inp, dev), world)
     m = ep.ExpertParallelMoE(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
-                             rank, world)
+                             rank, world, placement=placement)
     inp["w1"] = inp["w3"] = inp["w2"] = None
     torch.cuda.empty_cache()
     y = torch.empty((layer.T, layer.dim), dtype=inp["x"].dtype, device=dev)
@@ -719,7 +734,7 @@ def run_ep(a, layer, dev, rank, world, local, peaks):
     """--parallel ep with N > 1: one JSON line for the expert-parallel layer."""
     clocks = ClockSampler(local)
     clocks.start()
-    ms = time_ep_layer(layer, dev, rank, world, a.steps, a.warmup)
+    ms = time_ep_layer(layer, dev, rank, world, a.steps, a.warmup, a.ep_placement)
     clk = clocks.stop()
     if rank == 0:
         T = layer.T
@@ -732,6 +747,7 @@ def run_ep(a, layer, dev, rank, world, local, peaks):
             "impl": "ours",
             "config": {"workload": layer.name, "T": T, "parallelism": f"ep{world} "
                        "(experts split, fp32 partials all-reduced over NCCL)",
+                       "placement": a.ep_placement,
                        "l2": "inputs larger than L2"},
             "gpu_launches": (LAUNCHES_PER_FORWARD + 1) * a.steps,
             "clocks": clk,
