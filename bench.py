@@ -186,7 +186,8 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-# Algorithmic work (per launch), stated in the design doc
+# Algorithmic work per launch: the bytes the method must move and the FLOPs it
+# must do (activated experts only; no padding, no implementation buffers)
 # ---------------------------------------------------------------------------
 def algorithmic(layer, idx: np.ndarray) -> dict:
     T, d, I, k, S, E = layer.T, layer.dim, layer.inter, layer.topk, layer.n_shared, layer.n_experts

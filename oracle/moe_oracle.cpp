@@ -23,7 +23,7 @@
 // written below, so that a GPU gate fed the same fp32 scores can be compared
 // index for index.
 //
-// Readings where the pages are silent (each listed in the design doc):
+// Readings where the pages are silent:
 //  - ties in both top-k's go to the lower index (groups and experts);
 //  - idx is returned in descending key order;
 //  - renormalisation is a config switch (on for sigmoid, off for softmax);

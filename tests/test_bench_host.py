@@ -1,0 +1,63 @@
+"""bench.py's host-side arithmetic and inputs (CPU only).
+
+The algorithmic FLOPs and bytes behind every roofline line, against their
+closed forms for a layer small enough to count by hand; the DRAM-traffic table
+and the measured peaks the roofline reads; the flags of the multi-GPU and
+expert-parallel runs.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import bench
+from mixture_experts_layer_34_b200 import workloads as W
+
+
+def test_algorithmic_counts_match_closed_forms():
+    layer = W.BY_NAME["small_sig_bias"]          # T 300, d 512, E 32, k 4, S 1, I 256, bf16
+    T, d, E, k, S, I = 300, 512, 32, 4, 1, 256
+    idx = np.tile(np.arange(k, dtype=np.int32), (T, 1))     # every token -> experts 0..3
+    w = bench.algorithmic(layer, idx)
+    R = T * (k + S)
+    assert w["rows"] == R
+    assert w["active_experts"] == k + S                      # 4 routed hit + 1 shared
+    assert w["flops_up"] == 4 * d * I * R
+    assert w["flops_down"] == 2 * d * I * R
+    assert w["flops_layer"] == W.flops_per_token(layer) * T
+    assert W.flops_per_token(layer) == 6 * d * I * (k + S) + 2 * d * E
+    # bf16: weights 2 B per element; W_gate, x and y once
+    assert w["bytes_layer"] == (k + S) * 3 * d * I * 2 + E * d * 2 + 2 * T * d * 2
+    assert w["bytes_up"] == (k + S) * 2 * d * I * 2 + R * d * 2 + R * I * 2
+
+
+def test_algorithmic_mxfp8_weight_bytes():
+    layer = W.BY_NAME["small_sig_bias_mxfp8"]
+    idx = np.tile(np.arange(4, dtype=np.int32), (layer.T, 1))
+    w = bench.algorithmic(layer, idx)
+    # one code byte per weight plus one scale byte per 32
+    per_expert = 3 * layer.dim * layer.inter * (1 + 1 / 32)
+    tok = layer.n_experts * layer.dim * 2 + 2 * layer.T * layer.dim * 2
+    assert w["bytes_layer"] == pytest.approx(5 * per_expert + tok)
+
+
+def test_traffic_table_is_read_per_kernel_and_workload():
+    assert bench.traffic("up", "v3_prefill_T8192_zipf") > 1.5e10
+    assert bench.traffic("down", "v3_decode_T8") > 1e9
+    assert bench.traffic("up", "no_such_workload") is None
+
+
+def test_peaks_come_from_the_measured_file():
+    p = bench.load_peaks()
+    assert p["source"] in ("measured", "fallback")
+    assert p["hbm_gbs"] > 1000 and p["bf16_tflops"] > 100
+    assert p["bf16_tflops_sustained"] <= p["bf16_tflops"]
+
+
+def test_flags():
+    a = bench.parse_args([])
+    assert (a.gpus, a.parallel, a.ep_placement, a.ep_ranks) == (1, "dp", "balanced", 8)
+    a = bench.parse_args(["--gpus", "4", "--parallel", "ep", "--ep-placement", "contiguous"])
+    assert (a.gpus, a.parallel, a.ep_placement) == (4, "ep", "contiguous")
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--parallel", "tp"])
