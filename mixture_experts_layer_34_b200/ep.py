@@ -187,3 +187,29 @@ class ExpertParallelMoE:
         self.reduce(part)
         self.finish(part, x, y)
         return y
+
+    def graph(self, x, y, topk_idx=None, topk_w=None) -> "EpGraph":
+        """The whole step (local forward, all-reduce, finish) captured once as a
+        CUDA graph on these buffers; ``replay()`` reruns it (x is read in place,
+        so a decode loop rewrites x between replays). NCCL's all-reduce is
+        captured with the kernels when the group has more than one rank."""
+        T = x.shape[0]
+        self.buffers(T, x.device)
+        # One eager step first: the library's one-time host setup (kernel
+        # attributes) stays out of the capture, and NCCL's communicator exists.
+        self.forward(x, y, topk_idx, topk_w)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            self.forward(x, y, topk_idx, topk_w)
+        return EpGraph(g, (x, y, topk_idx, topk_w))
+
+
+class EpGraph:
+    """A captured expert-parallel step; holds the tensors bound into it."""
+
+    def __init__(self, g, keep):
+        self._g, self._keep = g, keep
+
+    def replay(self):
+        self._g.replay()

@@ -315,3 +315,25 @@ def test_mxfp8_placed_ranks_sum_to_the_forward():
     y = _finish(layer, inp, y_sum, True)
     rms = float(yf.square().mean().sqrt())
     assert float((y - yf).abs().max()) <= SUM_ORDER_TOL * rms
+
+
+@pytest.mark.parametrize("name", ["small_sig_bias", "small_sig_bias_mxfp8"])
+def test_graph_replay_is_the_eager_step(name):
+    """The captured step (local forward + finish; one rank, so no all-reduce)
+    replays to the eager step's output bit for bit, and follows new x."""
+    layer = W.BY_NAME[name]
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer)
+    placement = _shuffled_placement(layer.n_experts, 1)
+    m = ep.ExpertParallelMoE(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                             0, 1, placement=placement)
+    x = inp["x"].clone()
+    y = torch.empty((layer.T, layer.dim), dtype=torch.bfloat16, device="cuda")
+    g = m.graph(x, y)
+    ref = torch.empty_like(y)
+    for step in range(3):
+        x.copy_(inp["x"] * (1.0 + 0.25 * step))
+        g.replay()
+        m.forward(x, ref)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref), step
