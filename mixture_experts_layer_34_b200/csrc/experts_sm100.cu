@@ -38,10 +38,14 @@
 //   - The tile list (chunk, feature tile) is built on the device: within an
 //     expert, blocks of 8 token chunks run feature-tile-major, so that tiles
 //     reading one weight tile are neighbours in the list. Pairs take tiles from
-//     a device counter (the even CTA's producer fetches and publishes each tile
-//     to both CTAs through a 4-slot ring of mbarrier-guarded slots), so tiles
-//     start in list order and neighbours run together and share the weight
-//     tile through L2, however long earlier tiles took.
+//     a device counter (the even CTA's producer claims the next tile halfway
+//     through the current one and publishes it to both CTAs through a 4-slot
+//     ring of mbarrier-guarded slots), so tiles start in list order and
+//     neighbours run together and share the weight tile through L2, however
+//     long earlier tiles took.
+//   - Launched with programmatic dependent launch: the barrier and TMEM setup
+//     overlaps the previous kernel's tail; global memory is touched only after
+//     griddepcontrol.wait.
 // No TMA multicast is used.
 //
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the
