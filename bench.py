@@ -71,6 +71,9 @@ def parse_args(argv=None):
     ap.add_argument("--ep-placement", choices=("contiguous", "balanced"), default="balanced",
                     help="--parallel ep: experts in contiguous ranges, or placed by the load "
                          "of another seeded batch")
+    ap.add_argument("--ep-output", choices=("full", "sharded"), default="full",
+                    help="--parallel ep: every rank gets all T output rows (all-reduce), or "
+                         "its token share (reduce-scatter; T divisible by N)")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -316,15 +319,21 @@ def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
         raise RuntimeError(f"device error in the expert-parallel steps: {K.strerror(rc)}")
     msg = T * layer.dim * 4
     ar_ms = 2 * (ranks - 1) / ranks * msg / (ALLREDUCE_BUS_GBS * 1e9) * 1e3
+    rs_ms = ar_ms / 2          # a reduce-scatter moves half an all-reduce's bytes
     torch.cuda.empty_cache()
     res = {"ranks": ranks, "workload": layer.name, "finish_ms": round(finish_ms, 4),
-           "allreduce_bytes": msg, "allreduce_ms_projected": round(ar_ms, 4), "unit": "tokens/s"}
+           "allreduce_bytes": msg, "allreduce_ms_projected": round(ar_ms, 4),
+           "reduce_scatter_ms_projected": round(rs_ms, 4), "unit": "tokens/s"}
     for name, rank_ms in out.items():
         step_ms = max(rank_ms) + ar_ms + finish_ms
+        # token-sharded output: reduce-scatter, and the finish on 1/ranks of the rows
+        shard_ms = max(rank_ms) + rs_ms + finish_ms / ranks
         res[name] = {"rank_local_ms": [round(v, 4) for v in rank_ms],
                      "max_rank_local_ms": round(max(rank_ms), 4),
                      "step_ms_projected": round(step_ms, 4),
-                     "value_projected": round(T / (step_ms / 1e3), 1)}
+                     "value_projected": round(T / (step_ms / 1e3), 1),
+                     "sharded_step_ms_projected": round(shard_ms, 4),
+                     "sharded_value_projected": round(T / (shard_ms / 1e3), 1)}
     res["note"] = ("local steps and finish measured here, one rank after another on this GPU; "
                    "the fp32 all-reduce is projected at the measured 8-GPU NCCL bus bandwidth "
                    f"({ALLREDUCE_BUS_GBS:.0f} GB/s), not measured (one GPU); the balanced "
@@ -347,7 +356,8 @@ def expected_load(layer, inp, dev) -> np.ndarray:
     return np.bincount(idx.cpu().numpy().ravel(), minlength=layer.n_experts)
 
 
-def time_ep_layer(layer, dev, rank, world, steps, warmup, placement_kind="balanced"):
+def time_ep_layer(layer, dev, rank, world, steps, warmup, placement_kind="balanced",
+                  output="full"):
     """N > 1, --parallel ep: the expert-parallel layer over the process group
     (NCCL all-reduce of the fp32 partials); the same T tokens on every rank.
     Every rank computes the same placement from the same seeded batch."""
@@ -362,16 +372,20 @@ def time_ep_layer(layer, dev, rank, world, steps, warmup, placement_kind="balanc
                              rank, world, placement=placement)
     inp["w1"] = inp["w3"] = inp["w2"] = None
     torch.cuda.empty_cache()
-    y = torch.empty((layer.T, layer.dim), dtype=inp["x"].dtype, device=dev)
+    sb, se = m.shared_range(layer.T)
+    rows = layer.T if output == "full" else se - sb
+    y = torch.empty((rows, layer.dim), dtype=inp["x"].dtype, device=dev)
+    step = (lambda: m.forward(inp["x"], y)) if output == "full" else \
+        (lambda: m.forward_shard(inp["x"], y))
     for _ in range(warmup):
-        m.forward(inp["x"], y)
+        step()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0.record()
     for _ in range(steps):
-        m.forward(inp["x"], y)
+        step()
     t1.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -735,7 +749,7 @@ def run_ep(a, layer, dev, rank, world, local, peaks):
     """--parallel ep with N > 1: one JSON line for the expert-parallel layer."""
     clocks = ClockSampler(local)
     clocks.start()
-    ms = time_ep_layer(layer, dev, rank, world, a.steps, a.warmup, a.ep_placement)
+    ms = time_ep_layer(layer, dev, rank, world, a.steps, a.warmup, a.ep_placement, a.ep_output)
     clk = clocks.stop()
     if rank == 0:
         T = layer.T
@@ -748,7 +762,7 @@ def run_ep(a, layer, dev, rank, world, local, peaks):
             "impl": "ours",
             "config": {"workload": layer.name, "T": T, "parallelism": f"ep{world} "
                        "(experts split, fp32 partials all-reduced over NCCL)",
-                       "placement": a.ep_placement,
+                       "placement": a.ep_placement, "output": a.ep_output,
                        "l2": "inputs larger than L2"},
             "gpu_launches": (LAUNCHES_PER_FORWARD + 1) * a.steps,
             "clocks": clk,

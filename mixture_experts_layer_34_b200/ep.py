@@ -15,7 +15,9 @@ Per rank:
     local experts on their tokens, and the shared experts on this rank's share
     of the tokens (``token_range``), summed in fp32 by ``kt_moe_forward_local``;
   * one all-reduce of that fp32 [T, dim] partial (NCCL over NVLink/NVSwitch on
-    GPUs), which sums routed outputs and z in one message;
+    GPUs), which sums routed outputs and z in one message; or, for a next layer
+    that takes its tokens sharded over the same ranks, a reduce-scatter that
+    leaves each rank the sum for its own share of the tokens (half the bytes);
   * ``kt_moe_ep_finish``: the residual and the rounding to y's type.
 
 Every arithmetic step runs in libktmoe.so's kernels; this module holds the
@@ -140,6 +142,7 @@ class ExpertParallelMoE:
             self.w1, self.w3, self.w2 = w1, w3, w2
         self._ws: dict[int, torch.Tensor] = {}
         self._part: dict[int, torch.Tensor] = {}
+        self._shard: dict[int, torch.Tensor] = {}
 
     def shared_range(self, T: int) -> tuple[int, int]:
         return token_range(T, self.world, self.rank)
@@ -187,6 +190,30 @@ class ExpertParallelMoE:
         self.reduce(part)
         self.finish(part, x, y)
         return y
+
+    def forward_shard(self, x, y_shard, topk_idx=None, topk_w=None):
+        """The output rows of this rank's token share only (``token_range``;
+        T must be a multiple of the world size): one reduce-scatter instead of
+        the all-reduce. y_shard is [T / world, dim]."""
+        T = x.shape[0]
+        if T % self.world:
+            raise ValueError(f"reduce-scatter needs T ({T}) divisible by the world size")
+        _, part = self.buffers(T, x.device)
+        self.local(x, part, topk_idx, topk_w)
+        sb, se = self.shared_range(T)
+        if self.world > 1:
+            if T not in self._shard:
+                self._shard[T] = torch.empty((se - sb, self.cfg.dim), dtype=part.dtype,
+                                             device=x.device)
+            shard = self._shard[T]
+            dist.reduce_scatter_tensor(shard, part, op=dist.ReduceOp.SUM, group=self.group)
+        else:
+            shard = part
+        self.finish_rows(shard, x[sb:se], y_shard)
+        return y_shard
+
+    def finish_rows(self, part, x_rows, y_rows):
+        K.kt_moe_ep_finish(self.cfg, x_rows.shape[0], part, x_rows, y_rows)
 
     def graph(self, x, y, topk_idx=None, topk_w=None) -> "EpGraph":
         """The whole step (local forward, all-reduce, finish) captured once as a

@@ -120,7 +120,7 @@ def _ep_layer():
     return layer, W.make_layer(layer, "cpu")
 
 
-def _ep_worker(rank, world, port, q, placed=False):
+def _ep_worker(rank, world, port, q, placed=False, sharded=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
     import numpy as np
@@ -168,6 +168,9 @@ def _ep_worker(rank, world, port, q, placed=False):
             def finish(self, part, x, y):
                 y.copy_(part + (x.to(torch.float64) if layer.add_residual else 0))
 
+            def finish_rows(self, part, x_rows, y_rows):
+                self.finish(part, x_rows, y_rows)
+
         cfg = K.config_for(layer)
         placement = None
         if placed:   # a seeded shuffle of the experts, the same on every rank
@@ -175,11 +178,20 @@ def _ep_worker(rank, world, port, q, placed=False):
             placement = [sorted(perm[r::world]) for r in range(world)]
         m = OracleRank(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], rank,
                        world, placement=placement)
-        y = torch.empty(x.shape[0], layer.dim, dtype=torch.float64)
-        m.forward(x, y)
-        dist.destroy_process_group()
         ref = O.forward(fields, x, idx, w, inp["w1"], inp["w3"], inp["w2"], range(x.shape[0]),
                         True)
+        if sharded:
+            # each rank's token share, gathered here only to compare
+            sb, se = m.shared_range(x.shape[0])
+            ys = torch.empty(se - sb, layer.dim, dtype=torch.float64)
+            m.forward_shard(x, ys)
+            parts = [torch.empty_like(ys) for _ in range(world)]
+            dist.all_gather(parts, ys)
+            y = torch.cat(parts)
+        else:
+            y = torch.empty(x.shape[0], layer.dim, dtype=torch.float64)
+            m.forward(x, y)
+        dist.destroy_process_group()
         err = float(np.abs(y.numpy() - ref).max() / np.abs(ref).max())
         q.put((rank, (m.experts[0], m.experts[-1] + 1) if not placed else len(m.experts), err))
     except Exception as e:  # pragma: no cover - reported to the parent
@@ -203,6 +215,19 @@ def test_expert_parallel_with_a_placement_gloo():
     out = _run(2, _ep_worker_placed)
     assert [r[1] for r in out] == [16, 16], out
     for rank, n, err in out:
+        assert isinstance(err, float), err
+        assert err < 1e-12, (rank, err)
+
+
+def _ep_worker_sharded(rank, world, port, q):
+    _ep_worker(rank, world, port, q, sharded=True)
+
+
+def test_expert_parallel_reduce_scatter_gloo():
+    """forward_shard: one reduce-scatter, each rank finishes its token share;
+    the shares put together are the oracle's forward."""
+    out = _run(2, _ep_worker_sharded)
+    for rank, rng, err in out:
         assert isinstance(err, float), err
         assert err < 1e-12, (rank, err)
 

@@ -337,3 +337,36 @@ def test_graph_replay_is_the_eager_step(name):
         m.forward(x, ref)
         torch.cuda.synchronize()
         assert torch.equal(y, ref), step
+
+
+def test_sharded_finish_is_the_full_finish_on_each_share():
+    """forward_shard with one rank equals forward; with the partials of 4 ranks
+    summed, finishing each rank's token share (x offset into its rows) gives
+    the rows of the full finish, bit for bit."""
+    layer = W.BY_NAME["small_odd_dims"]           # residual on: the finish reads x rows
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer)
+    T = 76                                          # a multiple of 4 (the layer has 77)
+    x = inp["x"][:T].contiguous()
+    m = ep.ExpertParallelMoE(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                             0, 1)
+    y = torch.empty((T, layer.dim), dtype=torch.bfloat16, device="cuda")
+    ys = torch.empty_like(y)
+    m.forward(x, y)
+    m.forward_shard(x, ys)
+    assert torch.equal(y, ys)
+    world = 4
+    y_sum = torch.zeros((T, layer.dim), device="cuda")
+    for rank in range(world):
+        r = ep.ExpertParallelMoE(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"],
+                                 inp["w2"], rank, world)
+        _, part = r.buffers(T, x.device)
+        r.local(x, part)
+        y_sum += part
+    full = torch.empty_like(y)
+    K.kt_moe_ep_finish(cfg, T, y_sum, x, full)
+    for rank in range(world):
+        sb, se = ep.token_range(T, world, rank)
+        shard = torch.empty((se - sb, layer.dim), dtype=torch.bfloat16, device="cuda")
+        m.finish_rows(y_sum[sb:se].contiguous(), x[sb:se], shard)
+        assert torch.equal(shard, full[sb:se]), rank
