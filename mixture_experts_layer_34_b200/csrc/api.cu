@@ -86,6 +86,7 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
   r->n_local = E;
   r->sb = 0;
   r->se = (int)T;
+  r->num_sms = 0;
   r->add_residual = c->add_residual;
   r->y_fp32 = c->dtype == KT_DTYPE_F32 ? 1 : c->y_fp32;
   r->has_bias = has_bias ? 1 : 0;
@@ -332,16 +333,18 @@ SlotTable identity_table(const Resolved& r) {
   return t;
 }
 
-int run_forward(const Resolved& r, const SlotTable& tab, int64_t T, const void* x,
+int run_forward(const Resolved& r_in, const SlotTable& tab, int64_t T, const void* x,
                 const void* w_gate,
                 const float* bias, const void* wa, const void* wb, const void* wc,
                 const uint8_t* sf_up, const uint8_t* sf_down, void* y, bool partial,
                 int32_t* topk_idx_out, float* topk_w_out, void* workspace, void* stream,
                 void* const* stage_events) {
-  const Layout L = make_layout(r, T);
   int sms = 0;
   int rc = device_info(&sms);
   if (rc != KT_OK) return rc;
+  Resolved r = r_in;
+  r.num_sms = sms;
+  const Layout L = make_layout(r, T);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   int* err = reinterpret_cast<int*>(ws + L.err);

@@ -164,14 +164,15 @@ ep_finish_kernel(int64_t n4, int add_residual, const float4* __restrict__ y_sum,
 
 // Column slices per token: one CTA per token when there are many, several when
 // few (a decode step), each slice at least 128 columns of 16-byte vectors.
-dim3 combine_grid(int64_t T, int d) {
+dim3 combine_grid(int64_t T, int d, int num_sms) {
   const int64_t most = std::max<int64_t>(1, d / (128 * 8));
-  return dim3((unsigned)T, (unsigned)std::max<int64_t>(1, std::min<int64_t>(most, 296 / T)));
+  const int64_t target = 2 * (num_sms > 0 ? num_sms : 148);
+  return dim3((unsigned)T, (unsigned)std::max<int64_t>(1, std::min<int64_t>(most, target / T)));
 }
 
 cudaError_t launch_combine_partial(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                    float* y_part, cudaStream_t st) {
-  (void)launch_pdl(combine_partial_kernel, dim3(combine_grid(T, r.d)), dim3(128), 0, st,
+  (void)launch_pdl(combine_partial_kernel, combine_grid(T, r.d, r.num_sms), dim3(128), 0, st,
       (int)T, r.k, r.S, r.d, r.sb, r.se, reinterpret_cast<const int32_t*>(ws + L.row_of),
       reinterpret_cast<const float*>(ws + L.expert_out), reinterpret_cast<float4*>(y_part));
   return cudaGetLastError();
@@ -198,7 +199,7 @@ cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* 
                            void* y, cudaStream_t st) {
   const int32_t* row_of = reinterpret_cast<const int32_t*>(ws + L.row_of);
   const float* eo = reinterpret_cast<const float*>(ws + L.expert_out);
-  const dim3 grid = combine_grid(T, r.d);
+  const dim3 grid = combine_grid(T, r.d, r.num_sms);
   if (r.act_bf16 && !r.y_fp32)
     (void)launch_pdl(combine_kernel<true, false>, grid, dim3(128), 0, st, (int)T, r.k, r.S, r.d,
                      r.add_residual, row_of, eo, x, y);

@@ -56,6 +56,7 @@ struct Resolved {
   int n_local;      // routed experts computed here (all: E); their weights are the first
                     // n_local slots of w1/w3/w2 (placed by a SlotTable), the shared ones follow
   int sb, se;       // tokens the shared experts run on here: [sb, se) (all: [0, T))
+  int num_sms;      // SMs of the device (set by the forward before its launches)
   int add_residual;
   int y_fp32;       // y in fp32 (else in dtype)
   int has_bias;

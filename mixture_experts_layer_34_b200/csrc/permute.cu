@@ -313,7 +313,8 @@ cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, c
   if (e != cudaSuccess) return e;
   // Few chunks (a decode step): split each chunk's row copies over column
   // slices so that about two CTAs per SM copy.
-  const int64_t want = (296 + L.nperm - 1) / L.nperm;
+  const int64_t target = 2 * (r.num_sms > 0 ? r.num_sms : 148);
+  const int64_t want = (target + L.nperm - 1) / L.nperm;
   const int slices = r.act_bf16 ? (int)std::max<int64_t>(1, std::min<int64_t>(16, want)) : 1;
   const dim3 grid((unsigned)L.nperm, (unsigned)slices);
   float* rw = reinterpret_cast<float*>(ws + L.row_weight);
