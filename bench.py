@@ -11,18 +11,24 @@ tokens, no collective on the data path): weak scaling, timed on the device as
 the max over ranks.
 
 Rank 0 prints one JSON line. `value` is tokens/s of the whole job; `e2e` is the
-same metric with host buffers (pinned x copied in and y copied out every step);
-`roofline` is the dominant kernel (the gate/up expert GEMM) against the measured
-bf16 tensor peak; `cpu_baseline` is the CPU oracle timed on a sample of the
-same workload on this host's cores. `--impl reference` times the oracle alone
-(rank 0 only) in the same JSON form.
+same metric with host buffers (pinned x copied in and y copied out every step,
+serial with the compute), `e2e_pipelined` the same copies overlapped with the
+neighbouring steps' compute on two copy streams; `roofline` is the dominant
+kernel (the gate/up expert GEMM) against the measured bf16 tensor peak
+(sustained: the GEMM runs inside back-to-back steps at the power cap);
+`routing` is the expert-load histogram summary and the near-tie count;
+`cpu_baseline` is the CPU oracle timed on a sample of the same workload on this
+host's cores; "mxfp8" repeats prefill and decode with MXFP8 expert weights.
+`--impl reference` times the oracle alone (rank 0 only) in the same JSON form.
 
 "expert_parallel" (N = 1) times each rank's local step of the expert-parallel
 layer over --ep-ranks ranks (its experts, all tokens through the gate, its
-share of the shared experts' tokens) one rank after another on this GPU, plus
-the finish kernel; the all-reduce between them is projected, not measured.
-With N > 1, `--parallel ep` runs that layer for real over NCCL (the same T
-tokens on every rank, strong scaling).
+share of the shared experts' tokens) one rank after another on this GPU, for
+contiguous expert ranges and for a placement balanced on another batch's load,
+plus the finish kernel; the all-reduce (or, for a token-sharded output, the
+reduce-scatter) between them is projected, not measured. With N > 1,
+`--parallel ep` runs that layer for real over NCCL (the same T tokens on every
+rank, strong scaling; --ep-placement, --ep-output).
 """
 from __future__ import annotations
 
