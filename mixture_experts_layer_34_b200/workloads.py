@@ -187,6 +187,14 @@ LIMITS = [
                 topk_groups=8, topk=32, n_shared=8, inter=128, score_func=SIGMOID,
                 route_scale=2.5, norm_topk=-1, group_score=GROUP_AUTO, dtype="f32",
                 bias="normal", seed=2405, init="fan_in"),
+    # Degenerate routing: every expert selected (k = E), and a single routed
+    # expert with no shared one (the layer is one dense SwiGLU FFN).
+    LayerConfig("limits_k_equals_E", T=40, dim=128, n_experts=8, n_groups=1, topk_groups=1,
+                topk=8, n_shared=1, inter=128, score_func=SIGMOID, route_scale=1.0,
+                norm_topk=-1, group_score=GROUP_AUTO, dtype="bf16", bias="normal", seed=2407),
+    LayerConfig("limits_one_expert", T=70, dim=256, n_experts=1, n_groups=1, topk_groups=1,
+                topk=1, n_shared=0, inter=128, score_func=SOFTMAX, route_scale=1.0,
+                norm_topk=0, group_score=GROUP_AUTO, dtype="bf16", bias="none", seed=2408),
     LayerConfig("limits_E512_k32_S8_mxfp8", T=67, dim=256, n_experts=512, n_groups=32,
                 topk_groups=8, topk=32, n_shared=8, inter=128, score_func=SIGMOID,
                 route_scale=2.5, norm_topk=-1, group_score=GROUP_AUTO, dtype="mxfp8",

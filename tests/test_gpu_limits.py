@@ -2,7 +2,8 @@
 
 Configs at the largest expert count, group count, top-k and shared-expert count
 the boundary accepts (E = 512, G = 32, k = 32, S = 8) in bf16, fp32 and MXFP8;
-a single token; top-1 over 512 experts; and 65,536 tokens (589,824 hidden rows).
+a single token; top-1 over 512 experts; every expert selected (k = E); one
+routed expert and no shared one; and 65,536 tokens (589,824 hidden rows).
 Same bounds as the other parity tests: max|dy| <= 2e-2 * RMS(y_ref) (bf16,
 MXFP8; on the fp32 output) and 1e-4 * RMS(y_ref) (fp32), routing differences
 only at near ties.
@@ -37,7 +38,8 @@ def _check(layer, toks):
 
 
 @pytest.mark.parametrize("name", ["limits_E512_k32_S8", "limits_T1", "limits_E512_k1_softmax",
-                                  "limits_E512_k32_S8_f32"])
+                                  "limits_E512_k32_S8_f32", "limits_k_equals_E",
+                                  "limits_one_expert"])
 def test_limit_layers_every_token(name):
     layer = W.BY_NAME[name]
     inp, out = _check(layer, list(range(layer.T)))
