@@ -141,8 +141,8 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
   const int tid = threadIdx.x;
   const int NG = E + S;
   // Per-expert totals over the chunks; shared experts hold tokens [sb, se) (all
-  // T unless the caller splits them); routed experts outside [eb, ee) are
-  // computed elsewhere (slot -1) hold none.
+  // T unless the caller splits them); routed experts computed elsewhere (slot
+  // -1) hold none.
   if (tid < NG) {
     int run = 0;
     if (tid >= E)
