@@ -194,6 +194,16 @@ int kt_moe_forward_static(const kt_moe_config* cfg, int64_t T, const void* x,
 void* kt_moe_static_scratch(void);
 
 /*
+ * Diagnostic of the device-side failure path: one kernel thread waits, through
+ * the same bounded wait as the GEMM kernels, on an mbarrier that nothing
+ * arrives on; after limit_ns (0 < limit_ns <= 1e9) it records the timeout in
+ * the workspace error word and exits. kt_moe_check(workspace, stream) then
+ * returns KT_ERR_TIMEOUT; the context stays usable (the next forward on the
+ * workspace resets the word). workspace: device, 256-B aligned, at least 8 B.
+ */
+int kt_moe_selftest_timeout(void* workspace, int64_t limit_ns, void* stream);
+
+/*
  * The layer forward as a replayable CUDA graph, for decode steps where the
  * launch gaps of the eight stream operations are a visible share of a step of
  * well under a millisecond. There is no counterpart on the pages (their engine

@@ -698,6 +698,19 @@ int kt_moe_mxfp8_pack_local(const kt_moe_config* cfg, int expert_begin, int expe
 
 void* kt_moe_static_scratch(void) { return static_scratch_ptr(); }
 
+int kt_moe_selftest_timeout(void* workspace, int64_t limit_ns, void* stream) {
+  if (!workspace) return KT_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return KT_ERR_ALIGN;
+  if (limit_ns <= 0 || limit_ns > 1000000000LL) return KT_ERR_INVALID_CONFIG;
+  int sms = 0;
+  int rc = device_info(&sms);
+  if (rc != KT_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* err = static_cast<int*>(workspace);
+  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  return launch_wait_selftest(err, (uint64_t)limit_ns, st) == cudaSuccess ? KT_OK : KT_ERR_CUDA;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

@@ -221,13 +221,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait. Returns false (after recording the timeout) if the phase did not
 // complete within kWaitLimitNs, or if another CTA already recorded an error.
 // Slow path of mbar_wait, out of line so the issuing loops stay short.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int* err, int where) {
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int* err, int where,
+                                            uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*reinterpret_cast<volatile int*>(err) != 0) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         set_error(err, kDevErrTimeout, where);
         return false;
       }
@@ -1124,7 +1125,22 @@ int pair_grid(int num_sms, int max_pairs) {
   return 2 * (pairs > 0 ? pairs : 1);
 }
 
+// Diagnostic of the bounded wait: one thread waits, through the same slow path
+// as the GEMM kernels, on a barrier that nothing ever arrives on.
+__global__ void wait_selftest_kernel(int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  mbar_wait_slow(&bar, 0, err, 99, limit_ns);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(err, limit_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t prepare_grouped_gemm() {
   cudaError_t e = ensure_smem_attr<kKindUp>();

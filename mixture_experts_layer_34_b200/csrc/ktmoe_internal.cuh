@@ -155,6 +155,9 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
 // encoder), done before a stream capture so that the capture holds only
 // stream work.
 cudaError_t prepare_grouped_gemm();
+// One bounded wait on a barrier that never completes (limit_ns), recording the
+// timeout in the error word like the GEMM kernels' waits.
+cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, char* ws,
                                const void* x, const void* w1, const void* w3, const void* w2,
                                int num_sms, cudaStream_t st, bool up);

@@ -32,7 +32,7 @@ EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_fo
            "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8", "kt_moe_graph_create_mxfp8",
            "kt_moe_forward_local", "kt_moe_forward_local_mxfp8", "kt_moe_ep_finish",
            "kt_moe_mxfp8_scale_bytes_local", "kt_moe_mxfp8_pack_local", "kt_moe_forward_placed",
-           "kt_moe_forward_placed_mxfp8")
+           "kt_moe_forward_placed_mxfp8", "kt_moe_selftest_timeout")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -142,6 +142,8 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_mxfp8_scale_bytes_local.restype = ctypes.c_size_t
             L.kt_moe_mxfp8_pack_local.argtypes = [CP, C, C, P, P, P, P, P, P, P, P, P]
             L.kt_moe_mxfp8_pack_local.restype = ctypes.c_int
+            L.kt_moe_selftest_timeout.argtypes = [P, I64, P]
+            L.kt_moe_selftest_timeout.restype = ctypes.c_int
             L.kt_moe_version.argtypes = []
             L.kt_moe_version.restype = ctypes.c_int
             _lib = L
@@ -480,6 +482,14 @@ def kt_moe_static_scratch() -> int:
 def kt_moe_check(workspace, stream=None) -> int:
     """Synchronise the stream and read the workspace's device error word."""
     return lib().kt_moe_check(_ptr(workspace), _stream(stream))
+
+
+def kt_moe_selftest_timeout(workspace, limit_ns: int, stream=None):
+    """Run the bounded-wait diagnostic (see include/ktmoe.h); kt_moe_check then
+    reports KT_ERR_TIMEOUT."""
+    rc = lib().kt_moe_selftest_timeout(_ptr(workspace), int(limit_ns), _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_selftest_timeout", rc)
 
 
 def kt_moe_version() -> int:

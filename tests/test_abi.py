@@ -286,6 +286,15 @@ def test_placed_table_host_side_errors():
     assert placed(None) == K.KT_ERR_NULL
 
 
+def test_selftest_host_side_errors():
+    L = K.lib()
+    V = ctypes.c_void_p
+    assert L.kt_moe_selftest_timeout(None, 1000, None) == K.KT_ERR_WORKSPACE
+    assert L.kt_moe_selftest_timeout(V(0x7000080), 1000, None) == K.KT_ERR_ALIGN
+    for bad in (0, -5, 2_000_000_000):
+        assert L.kt_moe_selftest_timeout(V(0x7000000), bad, None) == K.KT_ERR_INVALID_CONFIG
+
+
 def test_strerror_covers_codes():
     for code in range(-8, 1):
         assert K.strerror(code) and K.strerror(code) != "unknown error code"
