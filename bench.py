@@ -21,6 +21,14 @@ kernel (the gate/up expert GEMM) against the measured bf16 tensor peak
 host's cores; "mxfp8" repeats prefill and decode with MXFP8 expert weights.
 `--impl reference` times the oracle alone (rank 0 only) in the same JSON form.
 
+`--dump DIR` saves each timed step's inputs and outputs as .npy files under
+DIR/<workload>_rank<r>/, also when a device error stops the run (before it
+raises): x, w_gate, bias, the routing (idx, w), y, a probe of the expert
+weights and meta.json. The expert weights themselves are not written: they are
+redrawn from the workload's seed. `python bench.py --replay DIR/<dumped step>`
+redraws them, checks the probe, reruns the forward on the dumped tokens and
+compares the routing and y bit for bit.
+
 "expert_parallel" (N = 1) times each rank's local step of the expert-parallel
 layer over --ep-ranks ranks (its experts, all tokens through the gate, its
 share of the shared experts' tokens) one rank after another on this GPU, for
@@ -80,6 +88,10 @@ def parse_args(argv=None):
     ap.add_argument("--ep-output", choices=("full", "sharded"), default="full",
                     help="--parallel ep: every rank gets all T output rows (all-reduce), or "
                          "its token share (reduce-scatter; T divisible by N)")
+    ap.add_argument("--dump", default=None,
+                    help="save each step's inputs and outputs (.npy) under this directory")
+    ap.add_argument("--replay", default=None,
+                    help="rerun a step saved by --dump and compare bit for bit, then exit")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -399,12 +411,13 @@ def time_ep_layer(layer, dev, rank, world, steps, warmup, placement_kind="balanc
     if rc != K.KT_OK:
         raise RuntimeError(f"device error in the expert-parallel steps: {K.strerror(rc)}")
     return max_over_ranks(t0.elapsed_time(t1), world, dev)
-def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
+def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False, dump=None):
     from mixture_experts_layer_34_b200 import ktmoe as K
     inp = W.make_layer(layer, dev)
     if rank > 0:
         g = torch.Generator(device="cpu").manual_seed(rank_tokens_seed(layer, rank))
         inp["x"] = torch.randn(inp["x"].shape, generator=g).to(inp["x"].dtype).to(dev)
+    probe = weight_probe(layer, inp) if dump else None
     cfg = K.config_for(layer)
     T = layer.T
     ws = K.alloc_workspace(cfg, T, dev)
@@ -431,10 +444,16 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
         else:
             K.kt_moe_forward(cfg, T, x, *args[3:8], yo, *args[9:])
 
+    def save(rc):
+        if dump:
+            dump_step(os.path.join(dump, f"{layer.name}_rank{rank}"), layer, inp, idx, w, y,
+                      probe, rc, rank)
+
     for _ in range(warmup):
         fwd(inp["x"])
     rc = K.kt_moe_check(ws)
     if rc != K.KT_OK:
+        save(rc)
         raise RuntimeError(f"device error after warm-up: {K.strerror(rc)}")
 
     # Stage events, created (recorded once) before the timed region.
@@ -455,6 +474,7 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
     barrier(world)
     ms = t0.elapsed_time(t1)
     rc = K.kt_moe_check(ws)
+    save(rc)
     if rc != K.KT_OK:
         raise RuntimeError(f"device error in the timed region: {K.strerror(rc)}")
     stage_ms = {name: statistics.fmean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps))
@@ -560,6 +580,89 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False):
     return out
 
 
+# ---------------------------------------------------------------------------
+# Dump and replay of one step
+# ---------------------------------------------------------------------------
+def _np_of(t: torch.Tensor) -> np.ndarray:
+    """A tensor as numpy; bf16 as its raw 16-bit patterns (numpy has no bf16)."""
+    t = t.detach()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def _tensor_of(a: np.ndarray, dtype: str, dev) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype == "bf16":
+        t = t.view(torch.int16).view(torch.bfloat16)
+    return t.to(dev)
+
+
+def weight_probe(layer, inp) -> np.ndarray:
+    """A few rows of the expert weights (first, middle and last slot), as fp32:
+    enough to tell whether a redraw from the seed gave the same weights."""
+    n = layer.n_experts + layer.n_shared
+    rows = [inp["w1"][0, 0], inp["w3"][n // 2, -1], inp["w2"][n - 1, layer.dim // 2]]
+    return np.concatenate([r.float().cpu().numpy() for r in rows])
+
+
+def dump_step(path, layer, inp, idx, w, y, probe, rc, rank):
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    os.makedirs(path, exist_ok=True)
+    torch.cuda.synchronize()
+    arrays = {"x": inp["x"], "w_gate": inp["w_gate"], "idx": idx, "w": w, "y": y}
+    if inp["bias"] is not None:
+        arrays["bias"] = inp["bias"]
+    dtypes = {}
+    for name, t in arrays.items():
+        np.save(os.path.join(path, name + ".npy"), _np_of(t))
+        dtypes[name] = "bf16" if t.dtype == torch.bfloat16 else str(t.dtype).replace("torch.", "")
+    np.save(os.path.join(path, "w_probe.npy"), probe)
+    meta = {"workload": layer.name, "T": layer.T, "rank": rank, "weight_seed": layer.seed,
+            "check": K.strerror(rc), "library_version": K.kt_moe_version(),
+            "checked_build": K.kt_moe_checked_build(), "dtypes": dtypes,
+            "device": torch.cuda.get_device_name(), "torch": torch.__version__}
+    with open(os.path.join(path, "meta.json"), "w") as f:
+        json.dump(meta, f, indent=1)
+
+
+def replay_step(path) -> dict:
+    """Rerun a dumped step: same weights (redrawn and probed), the dumped x,
+    w_gate and bias; the routing and y must come out identical."""
+    from mixture_experts_layer_34_b200 import ktmoe as K
+    meta = json.load(open(os.path.join(path, "meta.json")))
+    layer = W.BY_NAME[meta["workload"]]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    load = lambda n: _tensor_of(np.load(os.path.join(path, n + ".npy")), meta["dtypes"][n], dev)
+    inp = W.make_layer(layer, dev)
+    probe_ok = bool(np.array_equal(weight_probe(layer, inp),
+                                   np.load(os.path.join(path, "w_probe.npy"))))
+    inp["x"], inp["w_gate"] = load("x"), load("w_gate")
+    inp["bias"] = load("bias") if "bias" in meta["dtypes"] else None
+    cfg = K.config_for(layer)
+    T = layer.T
+    ws = K.alloc_workspace(cfg, T, dev)
+    y = torch.empty_like(load("y"))
+    idx = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
+    w = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
+    if layer.dtype == "mxfp8":
+        q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+        K.kt_moe_forward_mxfp8(cfg, T, inp["x"], inp["w_gate"], inp["bias"], q["w1q"], q["w3q"],
+                               q["w2q"], q["sf_up"], q["sf_down"], y, idx, w, ws)
+    else:
+        K.kt_moe_forward(cfg, T, inp["x"], inp["w_gate"], inp["bias"], inp["w1"], inp["w3"],
+                         inp["w2"], y, idx, w, ws)
+    rc = K.kt_moe_check(ws)
+    y_ref = load("y")
+    same = {"idx": torch.equal(idx, load("idx")), "w": torch.equal(w, load("w")),
+            "y": torch.equal(y, y_ref)}
+    dy = float((y.float() - y_ref.float()).abs().max()) if not same["y"] else 0.0
+    return {"replay": meta["workload"], "dumped_check": meta["check"], "check": K.strerror(rc),
+            "weights_redrawn_identically": probe_ok, "identical": same, "max_abs_dy": dy,
+            "match": probe_ok and rc == K.KT_OK and all(same.values())}
+
+
 def cpu_oracle_sample(layer, inp, idx_all, target_s: float) -> dict:
     """Time the CPU oracle (gate + literal expert loop) on the first n tokens."""
     import oracle.oracle as O
@@ -610,7 +713,7 @@ def run_ours(a):
         return run_ep(a, layer, dev, rank, world, local, peaks)
     clocks = ClockSampler(local)
     clocks.start()
-    pre = time_layer(layer, dev, rank, world, a.steps, a.warmup, a.e2e_steps)
+    pre = time_layer(layer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, dump=a.dump)
     epr = None
     if world == 1 and a.ep_ranks > 1:
         epr = time_ep_ranks(layer, pre["inp"], dev, a.ep_ranks, a.steps, a.warmup)
@@ -618,7 +721,8 @@ def run_ours(a):
     dec = None
     if a.decode_workload != "none":
         dlayer = W.BY_NAME[a.decode_workload]
-        dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, graph=True)
+        dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, graph=True,
+                         dump=a.dump)
         dec["routing"] = routing_stats(dlayer, dec["inp"], dec["idx"], dev)
     # The same layers with MXFP8 expert weights (same shapes, seeds and tokens).
     f8 = {}
@@ -628,7 +732,7 @@ def run_ours(a):
             if name in W.BY_NAME:
                 f8[key] = (W.BY_NAME[name], time_layer(W.BY_NAME[name], dev, rank, world, a.steps,
                                                        a.warmup, a.e2e_steps,
-                                                       graph=key == "decode"))
+                                                       graph=key == "decode", dump=a.dump))
                 f8[key][1].pop("inp")
     clk = clocks.stop()
 
@@ -829,6 +933,10 @@ def run_reference(a):
 
 def main(argv=None):
     a = parse_args(argv)
+    if a.replay:
+        r = replay_step(a.replay)
+        print(json.dumps(r))
+        sys.exit(0 if r["match"] else 1)
     if a.impl == "reference":
         run_reference(a)
     else:

@@ -62,7 +62,8 @@ enum {
   KT_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed               */
   KT_ERR_TIMEOUT = -6,        /* a bounded device-side wait gave up (kt_moe_check)  */
   KT_ERR_UNSUPPORTED = -7,    /* no sm_100 device, or a size beyond a kernel limit  */
-  KT_ERR_SCRATCH_LIMIT = -8   /* call needs more than the static scratch holds       */
+  KT_ERR_SCRATCH_LIMIT = -8,  /* call needs more than the static scratch holds       */
+  KT_ERR_BOUNDS = -9          /* checked build: an index check failed (kt_moe_check) */
 };
 
 /*
@@ -425,8 +426,10 @@ int kt_moe_balance_stats(const kt_moe_config* cfg, int64_t T, const float* score
                          float* loss_out, void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then read the device error word the last call on this
- * workspace left (a bounded wait inside a kernel that gave up sets it).
- * Returns KT_OK, KT_ERR_TIMEOUT, or KT_ERR_CUDA if the stream reports an error. */
+ * workspace left (a bounded wait inside a kernel that gave up sets it; in the
+ * checked build, so does an index check that failed).
+ * Returns KT_OK, KT_ERR_TIMEOUT, KT_ERR_BOUNDS (checked build only), or
+ * KT_ERR_CUDA if the stream reports an error. */
 int kt_moe_check(const void* workspace, void* stream);
 
 /* Byte offsets of the internal buffers inside the workspace, for tests and
@@ -475,6 +478,14 @@ const char* kt_moe_strerror(int code);
 
 /* Library version: (major << 16) | minor. */
 int kt_moe_version(void);
+
+/* 1 for the checked build (libktmoe_checked.so, compiled with -DKT_CHECKED),
+ * 0 for the release build. The checked build range-checks, where it is used,
+ * every index one kernel takes from another kernel's output (expert ids, the
+ * row maps row_of / tok_of, the GEMM chunk and tile lists, chunk counts): a
+ * failed check skips the access and records KT_ERR_BOUNDS for kt_moe_check.
+ * Same entry points, same results; it is a debugging aid, not a fast path. */
+int kt_moe_checked_build(void);
 
 #ifdef __cplusplus
 }

@@ -3,7 +3,9 @@
     python -m mixture_experts_layer_34_b200.build [--force] [-v]
 
 Each .cu under csrc/ is compiled to an object in _build/ (in parallel), then
-linked into one shared library beside this file. The CUDA runtime is linked
+linked into one shared library beside this file: libktmoe.so (release) and
+libktmoe_checked.so (-DKT_CHECKED: index checks on every value one kernel
+takes from another's output; loaded when KTMOE_LIB=checked). The CUDA runtime is linked
 statically; the driver entry point for tensor-map encoding is looked up at run
 time, so the library loads on a machine without a GPU (every call then returns
 an error code).
@@ -22,6 +24,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libktmoe.so")
+LIB_CHECKED = os.path.join(HERE, "libktmoe_checked.so")
 
 SOURCES = ["api.cu", "gate.cu", "permute.cu", "experts_sm100.cu", "experts_f32.cu", "combine.cu",
            "balance.cu", "mxfp8.cu"]
@@ -42,10 +45,10 @@ def _deps() -> list[str]:
     return deps + [os.path.join(INCLUDE, "ktmoe.h"), os.path.abspath(__file__)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
@@ -82,10 +85,24 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
     return lib
 
 
+def build_checked(force: bool = False) -> str:
+    """The checked build (libktmoe_checked.so), rebuilt when a source changed."""
+    if not force and up_to_date(LIB_CHECKED):
+        return LIB_CHECKED
+    return build(force=True, out=LIB_CHECKED, defines=("KT_CHECKED",))
+
+
+def build_all(force: bool = False) -> list[str]:
+    return [build(force=force), build_checked(force=force)]
+
+
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print registers/spills/smem")
+    ap.add_argument("--checked", action="store_true", help="also build libktmoe_checked.so")
     a = ap.parse_args()
     print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info))
+    if a.checked:
+        print(build_checked(force=a.force))

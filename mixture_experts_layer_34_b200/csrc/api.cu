@@ -211,7 +211,7 @@ int kt_moe_gate(const kt_moe_config* cfg, int64_t T, const void* x, const void* 
   if (!scores_in && launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess)
     return KT_ERR_CUDA;
   if (launch_gate_select(r, T, logits, scores_in, bias, topk_idx, topk_w,
-                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), st) != cudaSuccess)
+                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), err, st) != cudaSuccess)
     return KT_ERR_CUDA;
   return KT_OK;
 }
@@ -360,7 +360,7 @@ int run_forward(const Resolved& r_in, const SlotTable& tab, int64_t T, const voi
   if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
   if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
   if (launch_gate_select(r, T, logits, nullptr, bias, idx, w,
-                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), st) != cudaSuccess)
+                         reinterpret_cast<int32_t*>(ws + L.chunk_counts), err, st) != cudaSuccess)
     return KT_ERR_CUDA;
   if (!mark(1)) return KT_ERR_CUDA;
   // MXFP8: tokens to codes and scales first; the permutation copies the codes
@@ -831,7 +831,8 @@ int kt_moe_check(const void* workspace, void* stream) {
   int err[2] = {0, 0};
   if (cudaMemcpy(err, workspace, sizeof err, cudaMemcpyDeviceToHost) != cudaSuccess)
     return KT_ERR_CUDA;
-  return err[0] == 0 ? KT_OK : KT_ERR_TIMEOUT;
+  if (err[0] == 0) return KT_OK;
+  return err[0] == kDevErrBounds ? KT_ERR_BOUNDS : KT_ERR_TIMEOUT;
 }
 
 const char* kt_moe_strerror(int code) {
@@ -846,10 +847,13 @@ const char* kt_moe_strerror(int code) {
     case KT_ERR_UNSUPPORTED: return "unsupported device (needs compute capability 10.0, sm_100a)";
     case KT_ERR_SCRATCH_LIMIT:
       return "kt_moe_forward_static: the call needs more scratch than the 32 MiB static array";
+    case KT_ERR_BOUNDS: return "an index check of the checked build failed (an access was skipped)";
     default: return "unknown error code";
   }
 }
 
 int kt_moe_version(void) { return (0 << 16) | 1; }
+
+int kt_moe_checked_build(void) { return kChecked ? 1 : 0; }
 
 }  // extern "C"

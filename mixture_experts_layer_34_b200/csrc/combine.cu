@@ -21,13 +21,16 @@ template <bool kBF16, bool kF32Out>
 __global__ void __launch_bounds__(128)
 combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __restrict__ row_of,
                const float* __restrict__ expert_out, const void* __restrict__ x,
-               void* __restrict__ y) {
+               void* __restrict__ y, int* __restrict__ err) {
   pdl_wait();
   constexpr int V = kBF16 ? 8 : 4;
   __shared__ int rows[kMaxShared + kMaxTopk];
   const int t = blockIdx.x;
   if (threadIdx.x < S) rows[threadIdx.x] = T_ * k + threadIdx.x * T_ + t;
-  if (threadIdx.x < k) rows[S + threadIdx.x] = row_of[(int64_t)t * k + threadIdx.x];
+  if (threadIdx.x < k) {
+    const int row = row_of[(int64_t)t * k + threadIdx.x];
+    rows[S + threadIdx.x] = in_range(row, 0, (int64_t)T_ * k, err, 121) ? row : -1;
+  }
   __syncthreads();
   const int nrow = S + k;
   const int nq = d / V;
@@ -39,6 +42,7 @@ combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __r
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
     for (int j = 0; j < nrow; ++j) {
+      if (kChecked && rows[j] < 0) continue;
       const float4* src = reinterpret_cast<const float4*>(expert_out + (int64_t)rows[j] * d) + q * (V / 4);
 #pragma unroll
       for (int h = 0; h < V / 4; ++h) {
@@ -92,7 +96,7 @@ combine_kernel(int T_, int k, int S, int d, int add_residual, const int32_t* __r
 __global__ void __launch_bounds__(128)
 combine_partial_kernel(int T_, int k, int S, int d, int sb, int se,
                        const int32_t* __restrict__ row_of, const float* __restrict__ expert_out,
-                       float4* __restrict__ y) {
+                       float4* __restrict__ y, int* __restrict__ err) {
   pdl_wait();
   __shared__ int rows[kMaxShared + kMaxTopk];
   __shared__ int nrow;
@@ -103,7 +107,7 @@ combine_partial_kernel(int T_, int k, int S, int d, int sb, int se,
       for (int s = 0; s < S; ++s) rows[n++] = T_ * k + s * T_ + t;
     for (int j = 0; j < k; ++j) {
       const int row = row_of[(int64_t)t * k + j];
-      if (row >= 0) rows[n++] = row;
+      if (row >= 0 && in_range(row, 0, (int64_t)T_ * k, err, 122)) rows[n++] = row;
     }
     nrow = n;
   }
@@ -174,7 +178,8 @@ cudaError_t launch_combine_partial(const Resolved& r, int64_t T, const Layout& L
                                    float* y_part, cudaStream_t st) {
   (void)launch_pdl(combine_partial_kernel, combine_grid(T, r.d, r.num_sms), dim3(128), 0, st,
       (int)T, r.k, r.S, r.d, r.sb, r.se, reinterpret_cast<const int32_t*>(ws + L.row_of),
-      reinterpret_cast<const float*>(ws + L.expert_out), reinterpret_cast<float4*>(y_part));
+      reinterpret_cast<const float*>(ws + L.expert_out), reinterpret_cast<float4*>(y_part),
+      reinterpret_cast<int*>(ws + L.err));
   return cudaGetLastError();
 }
 
@@ -200,15 +205,16 @@ cudaError_t launch_combine(const Resolved& r, int64_t T, const Layout& L, char* 
   const int32_t* row_of = reinterpret_cast<const int32_t*>(ws + L.row_of);
   const float* eo = reinterpret_cast<const float*>(ws + L.expert_out);
   const dim3 grid = combine_grid(T, r.d, r.num_sms);
+  int* err = reinterpret_cast<int*>(ws + L.err);
   if (r.act_bf16 && !r.y_fp32)
     (void)launch_pdl(combine_kernel<true, false>, grid, dim3(128), 0, st, (int)T, r.k, r.S, r.d,
-                     r.add_residual, row_of, eo, x, y);
+                     r.add_residual, row_of, eo, x, y, err);
   else if (r.act_bf16)
     (void)launch_pdl(combine_kernel<true, true>, grid, dim3(128), 0, st, (int)T, r.k, r.S, r.d,
-                     r.add_residual, row_of, eo, x, y);
+                     r.add_residual, row_of, eo, x, y, err);
   else
     (void)launch_pdl(combine_kernel<false, true>, grid, dim3(128), 0, st, (int)T, r.k, r.S, r.d,
-                     r.add_residual, row_of, eo, x, y);
+                     r.add_residual, row_of, eo, x, y, err);
   return cudaGetLastError();
 }
 

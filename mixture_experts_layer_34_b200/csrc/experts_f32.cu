@@ -23,13 +23,15 @@ __global__ void __launch_bounds__(256)
 up_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_chunks_p, int E,
               int d, int I, const float* __restrict__ x, const float* __restrict__ w1,
               const float* __restrict__ w3, const int32_t* __restrict__ tok_of,
-              float* __restrict__ hidden) {
+              float* __restrict__ hidden, int T_, int n_routed_rows, int n_groups,
+              int64_t n_rows, int max_chunks, int* __restrict__ err) {
   pdl_wait();
   __shared__ float xs[kTB][kTK + 1];
   __shared__ float as[kTB][kTK + 1];
   __shared__ float bs[kTB][kTK + 1];
   __shared__ int tok[kTB];
-  const int n_chunks = *n_chunks_p;
+  int n_chunks = *n_chunks_p;
+  if (!in_range(n_chunks, 0, max_chunks + 1, err, 141)) n_chunks = 0;
   const int rblocks = kChunkRows / kTB;
   const int fblocks = (I + kTB - 1) / kTB;
   const int ntiles = n_chunks * rblocks * fblocks;
@@ -39,6 +41,7 @@ up_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_ch
     const int rb = (tile / fblocks) % rblocks;
     const int fb = tile % fblocks;
     const Chunk ch = chunks[ci];
+    if (!chunk_in_range(ch, n_groups, n_rows, kChunkRows, err, 142)) continue;
     const int r0 = rb * kTB;
     if (r0 >= ch.nrows) continue;   // uniform across the CTA
     const int f0 = fb * kTB;
@@ -48,7 +51,15 @@ up_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_ch
     if (threadIdx.x < kTB) {
       const int rr = r0 + threadIdx.x;
       int t = -1;
-      if (rr < ch.nrows) t = ch.group < E ? tok_of[ch.src_row0 + rr] : ch.src_row0 + rr;
+      if (rr < ch.nrows) {
+        if (ch.group >= E) {
+          t = ch.src_row0 + rr;
+        } else {
+          const int sr = ch.src_row0 + rr;
+          t = in_range(sr, 0, n_routed_rows, err, 146) ? tok_of[sr] : -1;
+        }
+        if (t >= 0 && !in_range(t, 0, T_, err, 147)) t = -1;
+      }
       tok[threadIdx.x] = t;
     }
     float g[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
@@ -88,11 +99,13 @@ __global__ void __launch_bounds__(256)
 down_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_chunks_p, int d,
                 int I, int n_routed_rows, const float* __restrict__ hidden,
                 const float* __restrict__ w2, const float* __restrict__ row_weight,
-                float* __restrict__ out) {
+                float* __restrict__ out, int n_groups, int64_t n_rows, int max_chunks,
+                int* __restrict__ err) {
   pdl_wait();
   __shared__ float hs[kTB][kTK + 1];
   __shared__ float ws[kTB][kTK + 1];
-  const int n_chunks = *n_chunks_p;
+  int n_chunks = *n_chunks_p;
+  if (!in_range(n_chunks, 0, max_chunks + 1, err, 151)) n_chunks = 0;
   const int rblocks = kChunkRows / kTB;
   const int oblocks = (d + kTB - 1) / kTB;
   const int ntiles = n_chunks * rblocks * oblocks;
@@ -102,6 +115,7 @@ down_f32_kernel(const Chunk* __restrict__ chunks, const int32_t* __restrict__ n_
     const int rb = (tile / oblocks) % rblocks;
     const int ob = tile % oblocks;
     const Chunk ch = chunks[ci];
+    if (!chunk_in_range(ch, n_groups, n_rows, kChunkRows, err, 152)) continue;
     const int r0 = rb * kTB;
     if (r0 >= ch.nrows) continue;
     const int o0 = ob * kTB;
@@ -144,18 +158,22 @@ cudaError_t launch_experts_f32(const Resolved& r, int64_t T, const Layout& L, ch
                                int num_sms, cudaStream_t st, bool up) {
   const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.meta);
   const int grid = num_sms * 4;
+  const int64_t n_rows = T * (r.k + r.S);
+  int* err = reinterpret_cast<int*>(ws + L.err);
   if (up) {
     (void)launch_pdl(up_f32_kernel, dim3(grid), dim3(256), 0, st,
         reinterpret_cast<const Chunk*>(ws + L.chunks), meta + 0, routed_slots(r), r.d, r.I,
         static_cast<const float*>(x), static_cast<const float*>(w1), static_cast<const float*>(w3),
-        reinterpret_cast<const int32_t*>(ws + L.tok_of), reinterpret_cast<float*>(ws + L.hidden));
+        reinterpret_cast<const int32_t*>(ws + L.tok_of), reinterpret_cast<float*>(ws + L.hidden),
+        (int)T, (int)(T * r.k), weight_slots(r), n_rows, (int)L.max_chunks, err);
     return cudaGetLastError();
   }
   (void)launch_pdl(down_f32_kernel, dim3(grid), dim3(256), 0, st,
       reinterpret_cast<const Chunk*>(ws + L.chunks), meta + 0, r.d, r.I, (int)(T * r.k),
       reinterpret_cast<const float*>(ws + L.hidden), static_cast<const float*>(w2),
       reinterpret_cast<const float*>(ws + L.row_weight),
-      reinterpret_cast<float*>(ws + L.expert_out));
+      reinterpret_cast<float*>(ws + L.expert_out), weight_slots(r), n_rows, (int)L.max_chunks,
+      err);
   return cudaGetLastError();
 }
 

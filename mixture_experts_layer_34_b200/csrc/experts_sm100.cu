@@ -142,6 +142,11 @@ struct GemmArgs {
   const float* row_weight;   // down: weight of routed rows
   int n_routed_rows;         // T * k
   int* err;
+  // Bounds of the chunk and tile lists (the checked build verifies each tile):
+  int n_groups;              // weight slots
+  int64_t n_rows;            // hidden rows T * (k + S)
+  int max_chunks;            // chunk list capacity
+  int max_chunk_rows;        // rows per chunk at most
   int tma3d;                 // 1: one box per stage from the 3-D/4-D maps (K % 64 == 0)
   int gate_hi;               // up, 3-D maps: W3 precedes W1 in memory, so the upper 64
                              // rows of each CTA's weight tile are W1 (gate)
@@ -436,8 +441,15 @@ __device__ __forceinline__ void get_tile(const GemmArgs& a, int t, Chunk& ch, in
   } else {
     const int2 e = a.tiles[t];
     ci = e.x;
-    ch = a.chunks[e.x];
     ft = e.y;
+    // (Checked build) a tile naming a chunk, feature tile, weight slot or rows
+    // outside the lists ends this pair's schedule like the end marker.
+    if (!in_range(e.x, 0, a.max_chunks, a.err, 131) || !in_range(e.y, 0, a.n_ftiles, a.err, 132)) {
+      ch = Chunk{-1, 0, 0, 0};
+      return;
+    }
+    ch = a.chunks[e.x];
+    if (!chunk_in_range(ch, a.n_groups, a.n_rows, a.max_chunk_rows, a.err, 133)) ch = Chunk{-1, 0, 0, 0};
   }
 }
 
@@ -1165,6 +1177,10 @@ cudaError_t launch_experts_bf16(const Resolved& r, int64_t T, const Layout& L, c
   a.n_routed_rows = (int)Rr;
   a.err = reinterpret_cast<int*>(ws + L.err);
   a.E = routed_slots(r);
+  a.n_groups = NG;
+  a.n_rows = R;
+  a.max_chunks = (int)L.max_chunks;
+  a.max_chunk_rows = kChunkRows;
   const int grid = pair_grid(num_sms, 0);
   TmaMaps M;
   memset(&M, 0, sizeof(M));
@@ -1226,6 +1242,10 @@ cudaError_t launch_experts_mxfp8(const Resolved& r, int64_t T, const Layout& L, 
   a.n_routed_rows = (int)Rr;
   a.err = reinterpret_cast<int*>(ws + L.err);
   a.E = routed_slots(r);
+  a.n_groups = NG;
+  a.n_rows = R;
+  a.max_chunks = (int)L.max_chunks;
+  a.max_chunk_rows = kChunkRowsF8;
   a.tma3d = 1;
   const int grid = pair_grid(num_sms, 0);
   TmaMaps M;

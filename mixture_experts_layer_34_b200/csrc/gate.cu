@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kSelWarps * 32)
 gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ logits,
                    const float* __restrict__ scores_in, const float* __restrict__ bias,
                    int32_t* __restrict__ out_idx, float* __restrict__ out_w,
-                   int32_t* __restrict__ chunk_counts) {
+                   int32_t* __restrict__ chunk_counts, int* __restrict__ err) {
   pdl_wait();
   __shared__ int scount[kMaxExperts];
   __shared__ float skey[kSelWarps][kMaxExperts];
@@ -389,7 +389,7 @@ gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
       wv = __fmul_rn(wv, r.route_scale);
       out_idx[(int64_t)t * k + lane] = my_e;
       out_w[(int64_t)t * k + lane] = wv;
-      atomicAdd(&scount[my_e], 1);
+      if (in_range(my_e, 0, E, err, 161)) atomicAdd(&scount[my_e], 1);
     }
   }
   __syncthreads();
@@ -456,13 +456,13 @@ cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, cons
 
 cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits,
                                const float* scores_in, const float* bias, int32_t* idx, float* w,
-                               int32_t* chunk_counts, cudaStream_t st) {
+                               int32_t* chunk_counts, int* err, cudaStream_t st) {
   const unsigned grid = (unsigned)((T + kPermChunk - 1) / kPermChunk);
   const int ks = scores_in ? 1 : gate_logit_splits(r, T);
   const int np = (r.E + 31) / 32;
 #define KT_SELECT(NPV)                                                                         \
   (void)launch_pdl(gate_select_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, \
-                   ks, logits, scores_in, bias, idx, w, chunk_counts)
+                   ks, logits, scores_in, bias, idx, w, chunk_counts, err)
   if (np <= 1) KT_SELECT(1);
   else if (np <= 2) KT_SELECT(2);
   else if (np <= 4) KT_SELECT(4);

@@ -39,6 +39,7 @@ constexpr int kGateSplitK = 16;     // ... into this many partial sums
 
 // Device error word codes (workspace offset 0). The second int holds a detail.
 constexpr int kDevErrTimeout = 1;
+constexpr int kDevErrBounds = 2;   // checked build only: an index check failed
 
 // ---------------------------------------------------------------------------
 // Config with every automatic choice resolved
@@ -130,7 +131,7 @@ cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, c
                                   float* logits, int* err, int num_sms, cudaStream_t st);
 cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits,
                                const float* scores_in, const float* bias, int32_t* idx,
-                               float* w, int32_t* chunk_counts, cudaStream_t st);
+                               float* w, int32_t* chunk_counts, int* err, cudaStream_t st);
 // Scores s [T, E] fp32 from the logits region (gate step 1's score function).
 cudaError_t launch_gate_scores(const Resolved& r, int64_t T, const float* logits, float* scores,
                                cudaStream_t st);
@@ -214,6 +215,34 @@ __device__ __forceinline__ int64_t chunk_scale_offset(int64_t chunk, int nslab, 
 // Device-side helpers used by several kernels.
 __device__ __forceinline__ void set_error(int* err, int code, int detail) {
   if (atomicCAS(err, 0, code) == 0) err[1] = detail;
+}
+
+// Index checks of the checked build (compiled with -DKT_CHECKED into
+// libktmoe_checked.so). Every index one kernel takes from another kernel's
+// output (expert ids, row maps, GEMM chunk and tile lists, token ids, chunk
+// counts) is range-checked where it is used: a failed check records
+// kDevErrBounds and the site in the error word and the access is skipped, so
+// kt_moe_check reports KT_ERR_BOUNDS instead of the kernel touching memory it
+// does not own. In release builds in_range is constant true and the checks
+// compile away.
+#ifdef KT_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+__device__ __forceinline__ bool in_range(int64_t v, int64_t lo, int64_t hi, int* err, int site) {
+  if (!kChecked || (v >= lo && v < hi)) return true;
+  set_error(err, kDevErrBounds, site);
+  return false;
+}
+// A GEMM chunk: weight slot in [0, n_groups), 1..max_rows rows inside the
+// n_rows hidden rows, a non-negative first activation row.
+__device__ __forceinline__ bool chunk_in_range(const Chunk& c, int n_groups, int64_t n_rows,
+                                               int max_rows, int* err, int site) {
+  return in_range(c.group, 0, n_groups, err, site) &&
+         in_range(c.nrows, 1, max_rows + 1, err, site + 1) &&
+         in_range(c.row0, 0, n_rows - c.nrows + 1, err, site + 2) &&
+         in_range(c.src_row0, 0, INT32_MAX, err, site + 3);
 }
 
 // Programmatic dependent launch: the forward's kernels are launched so that the

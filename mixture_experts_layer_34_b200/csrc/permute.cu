@@ -96,7 +96,7 @@ __device__ __forceinline__ int merged_pos_l(int j, int nh, int nl) {
 // ordered per group by tile_of, and the two are merged proportionally so that
 // the pairs running at any moment mix both kinds.
 __device__ void fill_tiles(int2* __restrict__ tiles, int F, int NG, const int* cb, int* hb,
-                           int* lb, const int* tot) {
+                           int* lb, const int* tot, int* err) {
   const int tid = threadIdx.x;
   if (tid < NG) {
     const int nt = (cb[tid + 1] - cb[tid]) * F;
@@ -114,11 +114,15 @@ __device__ void fill_tiles(int2* __restrict__ tiles, int F, int NG, const int* c
   __syncthreads();
   for (int i = tid; i < nh; i += blockDim.x) {
     const int g = find_group(hb, NG, i);
-    tiles[merged_pos_h(i, nh, nl)] = tile_of(i - hb[g], cb[g + 1] - cb[g], F, cb[g]);
+    const int pos = merged_pos_h(i, nh, nl);
+    if (in_range(pos, 0, nh + nl, err, 104))
+      tiles[pos] = tile_of(i - hb[g], cb[g + 1] - cb[g], F, cb[g]);
   }
   for (int j = tid; j < nl; j += blockDim.x) {
     const int g = find_group(lb, NG, j);
-    tiles[merged_pos_l(j, nh, nl)] = tile_of(j - lb[g], cb[g + 1] - cb[g], F, cb[g]);
+    const int pos = merged_pos_l(j, nh, nl);
+    if (in_range(pos, 0, nh + nl, err, 104))
+      tiles[pos] = tile_of(j - lb[g], cb[g + 1] - cb[g], F, cb[g]);
   }
   __syncthreads();
 }
@@ -130,7 +134,7 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                     Chunk* __restrict__ chunks, int2* __restrict__ tiles_up,
                     int2* __restrict__ tiles_dn, int32_t* __restrict__ meta,
-                    int32_t* __restrict__ gchunk0) {
+                    int32_t* __restrict__ gchunk0, int max_chunks, int* __restrict__ err) {
   pdl_wait();
   constexpr int NGMAX = kMaxExperts + kMaxShared;
   __shared__ int tot[NGMAX];
@@ -155,7 +159,7 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
   }
   __syncthreads();
   // Routed experts: rows [0, T*k); shared expert s: rows T*k + s*T + t.
-  block_exclusive_scan(rows0, E);
+  const int routed_rows = block_exclusive_scan(rows0, E);
   if (tid >= E && tid < NG) rows0[tid] = T_ * k + (tid - E) * T_;
   __syncthreads();
   if (tid < NG) offsets[tid] = rows0[tid];
@@ -172,16 +176,21 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
   if (tid < NG) cb[tid] = (tot[tid] + chunk_rows - 1) / chunk_rows;
   __syncthreads();
   const int n_chunks = block_exclusive_scan(cb, NG);
+  // (Checked build) more routed rows or chunks than the workspace holds: no
+  // GEMM work is scheduled.
+  const bool fits = in_range(routed_rows, 0, (int64_t)T_ * k + 1, err, 101) &&
+                    in_range(n_chunks, 0, max_chunks + 1, err, 102);
   if (tid < NG) gchunk0[tid] = cb[tid];
   if (tid == 0) {
     cb[NG] = n_chunks;
-    meta[0] = n_chunks;
-    meta[1] = n_chunks * Fu;
-    meta[2] = n_chunks * Fd;
+    meta[0] = fits ? n_chunks : 0;
+    meta[1] = fits ? n_chunks * Fu : 0;
+    meta[2] = fits ? n_chunks * Fd : 0;
     meta[3] = 0;   // gate/up GEMM tile counter
     meta[4] = 0;   // down GEMM tile counter
   }
   __syncthreads();
+  if (!fits) return;
   // The chunks name weight slots: routed expert g in slot tab.slot[g], shared
   // expert E + s in slot n_local + s.
   for (int i = tid; i < n_chunks; i += blockDim.x) {
@@ -192,8 +201,8 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
     const int src0 = g < E ? rows0[g] : sb;
     chunks[i] = Chunk{slot, row0 + r, min(chunk_rows, tot[g] - r), src0 + r};
   }
-  fill_tiles(tiles_up, Fu, NG, cb, hb, lb, tot);
-  fill_tiles(tiles_dn, Fd, NG, cb, hb, lb, tot);
+  fill_tiles(tiles_up, Fu, NG, cb, hb, lb, tot, err);
+  fill_tiles(tiles_dn, Fd, NG, cb, hb, lb, tot, err);
 }
 
 // Copy modes of the scatter.
@@ -209,7 +218,8 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
                        const int32_t* __restrict__ gchunk0, int32_t* __restrict__ row_of,
                        int32_t* __restrict__ tok_of, float* __restrict__ row_weight,
                        const uint4* __restrict__ x, uint4* __restrict__ xperm,
-                       const uint8_t* __restrict__ xs, uint8_t* __restrict__ tok_sf) {
+                       const uint8_t* __restrict__ xs, uint8_t* __restrict__ tok_sf,
+                       int max_chunks, int* __restrict__ err) {
   pdl_wait();
   __shared__ uint32_t mask[kMaxExperts];
   __shared__ int srow[kPermChunk * kMaxTopk];
@@ -222,7 +232,7 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
   for (int q = threadIdx.x; q < nent; q += blockDim.x) {
     const int tl = q / k;
     const int e = idx[(int64_t)t0 * k + q];
-    atomicOr(&mask[e], 1u << tl);
+    if (in_range(e, 0, E, err, 111)) atomicOr(&mask[e], 1u << tl);
   }
   __syncthreads();
   // blockIdx.y: a column slice of the copies (few tokens: several CTAs share a
@@ -231,13 +241,19 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
   for (int q = threadIdx.x; q < nent; q += blockDim.x) {
     const int tl = q / k;
     const int e = idx[(int64_t)t0 * k + q];
-    if (tab.slot[e] < 0) {   // an expert computed elsewhere: no row here
+    // An expert computed elsewhere (or, checked build, an id out of range): no row here.
+    if ((kChecked && (e < 0 || e >= E)) || tab.slot[e] < 0) {
       if (lead) row_of[(int64_t)t0 * k + q] = -1;
       srow[q] = -1;
       continue;
     }
     const int rank = __popc(mask[e] & ((1u << tl) - 1u));
     const int row = chunk_base[(int64_t)c * E + e] + rank;
+    if (!in_range(row, 0, (int64_t)T_ * k, err, 112)) {
+      if (lead) row_of[(int64_t)t0 * k + q] = -1;
+      srow[q] = -1;
+      continue;
+    }
     if (lead) {
       row_of[(int64_t)t0 * k + q] = row;
       tok_of[row] = t0 + tl;
@@ -289,6 +305,8 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
       rel = t0 + tl - sb;
     }
     const int64_t chunk = gchunk0[g] + rel / chunk_rows;
+    if (!in_range(rel, 0, INT32_MAX, err, 113) || !in_range(chunk, 0, max_chunks, err, 114))
+      continue;
     const int m = rel % chunk_rows;
     const uint32_t* srcs = reinterpret_cast<const uint32_t*>(xs + (int64_t)(t0 + tl) * (d / 32));
     for (int s4 = lane; s4 < nslab; s4 += 32)
@@ -308,7 +326,8 @@ cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, c
                    r.n_local, r.sb, r.se, I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts),
                    I32(L.offsets), reinterpret_cast<Chunk*>(ws + L.chunks),
                    reinterpret_cast<int2*>(ws + L.tiles_up),
-                   reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0));
+                   reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0),
+                   (int)L.max_chunks, I32(L.err));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // Few chunks (a decode step): split each chunk's row copies over column
@@ -326,18 +345,18 @@ cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, c
                      reinterpret_cast<const uint4*>(ws + L.xq),
                      reinterpret_cast<uint4*>(ws + L.xperm),
                      reinterpret_cast<const uint8_t*>(ws + L.xs),
-                     reinterpret_cast<uint8_t*>(ws + L.tok_sf));
+                     reinterpret_cast<uint8_t*>(ws + L.tok_sf), (int)L.max_chunks, I32(L.err));
   else if (r.dtype == KT_DTYPE_BF16)
     (void)launch_pdl(permute_scatter_kernel<kCopyBf16>, grid, dim3(256), 0, st, r.E, r.S, (int)T,
                      r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
                      I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw,
                      reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(ws + L.xperm),
-                     nullptr, nullptr);
+                     nullptr, nullptr, (int)L.max_chunks, I32(L.err));
   else
     (void)launch_pdl(permute_scatter_kernel<kNoCopy>, grid, dim3(256), 0, st, r.E, r.S, (int)T,
                      r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
                      I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr,
-                     nullptr);
+                     nullptr, (int)L.max_chunks, I32(L.err));
   return cudaGetLastError();
 }
 

@@ -12,13 +12,18 @@ import os
 import threading
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libktmoe.so")
+# KTMOE_LIB=checked loads the checked build (libktmoe_checked.so: every index
+# a kernel takes from another kernel's output is range-checked; same entry
+# points and results); anything else, or unset, the release build.
+LIB_NAMES = {"release": "libktmoe.so", "checked": "libktmoe_checked.so"}
+LIB_PATH = os.path.join(HERE, LIB_NAMES.get(os.environ.get("KTMOE_LIB", "release"), "libktmoe.so"))
 
 KT_SCORE_SIGMOID, KT_SCORE_SOFTMAX = 0, 1
 KT_GROUP_AUTO, KT_GROUP_AMAX, KT_GROUP_TOP2SUM = 0, 1, 2
 KT_OK = 0
 KT_ERR_INVALID_CONFIG, KT_ERR_NULL, KT_ERR_WORKSPACE, KT_ERR_ALIGN = -1, -2, -3, -4
 KT_ERR_CUDA, KT_ERR_TIMEOUT, KT_ERR_UNSUPPORTED, KT_ERR_SCRATCH_LIMIT = -5, -6, -7, -8
+KT_ERR_BOUNDS = -9
 KT_STATIC_SCRATCH_BYTES = 32 << 20
 KT_DTYPE_F32, KT_DTYPE_BF16, KT_DTYPE_MXFP8 = 0, 1, 2
 
@@ -32,7 +37,7 @@ EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_fo
            "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8", "kt_moe_graph_create_mxfp8",
            "kt_moe_forward_local", "kt_moe_forward_local_mxfp8", "kt_moe_ep_finish",
            "kt_moe_mxfp8_scale_bytes_local", "kt_moe_mxfp8_pack_local", "kt_moe_forward_placed",
-           "kt_moe_forward_placed_mxfp8", "kt_moe_selftest_timeout")
+           "kt_moe_forward_placed_mxfp8", "kt_moe_selftest_timeout", "kt_moe_checked_build")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -146,6 +151,8 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_selftest_timeout.restype = ctypes.c_int
             L.kt_moe_version.argtypes = []
             L.kt_moe_version.restype = ctypes.c_int
+            L.kt_moe_checked_build.argtypes = []
+            L.kt_moe_checked_build.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -494,6 +501,10 @@ def kt_moe_selftest_timeout(workspace, limit_ns: int, stream=None):
 
 def kt_moe_version() -> int:
     return lib().kt_moe_version()
+
+
+def kt_moe_checked_build() -> bool:
+    return bool(lib().kt_moe_checked_build())
 
 
 def config_for(layer, y_fp32: bool = False) -> kt_moe_config:

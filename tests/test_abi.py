@@ -30,6 +30,23 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
 
 
+def test_checked_library_exports_every_declared_symbol():
+    """The checked build (-DKT_CHECKED) has the same ABI and says which it is;
+    loaded in a fresh process, as the binding picks one library per process."""
+    import subprocess
+    import sys
+    code = ("from mixture_experts_layer_34_b200 import ktmoe as K; "
+            "L = K.lib(); assert K.LIB_PATH.endswith('libktmoe_checked.so'), K.LIB_PATH; "
+            "missing = [n for n in K.EXPORTS if not hasattr(L, n)]; assert not missing, missing; "
+            "assert K.kt_moe_checked_build(); print('ok')")
+    env = dict(os.environ, KTMOE_LIB="checked")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT,
+                       env=env, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+    if os.environ.get("KTMOE_LIB", "release") != "checked":
+        assert not K.kt_moe_checked_build()
+
+
 def test_library_links_no_torch():
     # The library is plain C ABI: it must not need libtorch / libc10 to load.
     import subprocess
@@ -296,7 +313,7 @@ def test_selftest_host_side_errors():
 
 
 def test_strerror_covers_codes():
-    for code in range(-8, 1):
+    for code in range(-9, 1):
         assert K.strerror(code) and K.strerror(code) != "unknown error code"
     assert K.strerror(-99) == "unknown error code"
 

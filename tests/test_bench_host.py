@@ -61,3 +61,24 @@ def test_flags():
     assert (a.gpus, a.parallel, a.ep_placement) == (4, "ep", "contiguous")
     with pytest.raises(SystemExit):
         bench.parse_args(["--parallel", "tp"])
+
+
+def test_dump_arrays_round_trip_bit_for_bit():
+    """--dump writes bf16 as its 16-bit patterns; reading back gives the same bits."""
+    import torch
+    g = torch.Generator().manual_seed(3)
+    for t in (torch.randn(5, 7, generator=g).to(torch.bfloat16), torch.randn(4, 3, generator=g),
+              torch.randint(-5, 9, (6, 2), generator=g, dtype=torch.int32)):
+        a = bench._np_of(t)
+        tag = "bf16" if t.dtype == torch.bfloat16 else str(t.dtype)
+        back = bench._tensor_of(a, tag, "cpu")
+        assert back.dtype == t.dtype and torch.equal(back, t)
+    special = torch.tensor([float("inf"), -0.0, 1e-40, 3.0], dtype=torch.bfloat16)
+    assert bench._np_of(special).tolist() == [0x7F80, 0x8000, special[2].view(torch.int16).item(),
+                                              0x4040]
+
+
+def test_dump_and_replay_flags():
+    a = bench.parse_args(["--dump", "/tmp/d"])
+    assert a.dump == "/tmp/d" and a.replay is None
+    assert bench.parse_args(["--replay", "/tmp/d/x"]).replay == "/tmp/d/x"
