@@ -593,3 +593,110 @@ int oracle_forward_mxfp8(const oracle_cfg* c, int64_t T, const void* x, const in
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// MXFP4 expert weights (the 4-bit form of the layer).
+//
+// Format: MX FP4 E2M1. Blocks of 32 consecutive elements along K share one
+// power-of-two scale 2^e (8-bit biased exponent e + 127, as for MXFP8); each
+// element is FP4 E2M1: 1 sign bit, 2 exponent bits with bias 1, 1 mantissa
+// bit, a subnormal at exponent 0, no infinities or NaN. Its magnitudes are
+// 0, 0.5, 1, 1.5, 2, 3, 4 and 6. The KTransformers DeepSeek page ("DeepSeek
+// V4-Flash", its training notes) runs routed experts held natively in MXFP4;
+// the pages give no quantisation rule, and the one taken mirrors the MXFP8
+// rule above:
+//   scale  : e = the smallest integer with amax <= 6 * 2^e (no element
+//            saturates); for amax = m * 2^E with m in [1, 2) that is
+//            e = E - 2 + (m > 1.5); amax = 0 gives e = -127; clamped to
+//            [-127, 127];
+//   element: code = E2M1 round-to-nearest-even of v / 2^e (ties go to the
+//            code whose mantissa bit is 0).
+// Codes here are one per byte (0..15, sign in bit 3); the library packs two
+// per byte. Tokens and SwiGLU hidden vectors stay MXFP8 (E4M3), so the 4-bit
+// forward is the FP8 forward on weights whose every element is an E2M1 value
+// times its block scale (each of those is exactly an E4M3 value times the same
+// scale, which is how oracle.py evaluates it).
+// ===========================================================================
+namespace {
+
+double e2m1_to_double(uint8_t c) {
+  const int ex = (c >> 1) & 3, man = c & 1;
+  const double mag = ex == 0 ? 0.5 * man : std::ldexp(1.0 + 0.5 * man, ex - 1);
+  return (c & 8) ? -mag : mag;
+}
+
+uint8_t e2m1_from_double(double v) {
+  const uint8_t sign = std::signbit(v) ? 8 : 0;
+  const double a = std::fabs(v);
+  // Above the largest magnitude the code saturates at 6 (decided before the
+  // distance search, whose differences lose 6 - 4 for huge values).
+  if (a >= 6.0) return (uint8_t)(sign | 7);
+  // The nearest of the eight magnitudes; on a tie the even code (mantissa 0).
+  uint8_t best = 0;
+  double best_err = a;
+  for (uint8_t c = 1; c < 8; ++c) {
+    const double err = std::fabs(a - e2m1_to_double(c));
+    if (err < best_err || (err == best_err && (c & 1) == 0)) {
+      best = c;
+      best_err = err;
+    }
+  }
+  return (uint8_t)(sign | best);
+}
+
+int mx4_exponent(double amax) {
+  if (!(amax > 0.0)) return -127;
+  int E = 0;
+  const double f = std::frexp(amax, &E);   // amax = (2f) * 2^(E-1), 2f in [1, 2)
+  int e = (E - 1) - 2 + (2.0 * f > 1.5 ? 1 : 0);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+}  // namespace
+
+extern "C" {
+
+// E2M1 round-to-nearest-even of n doubles (saturating at +-6) and back.
+int oracle_e2m1_encode(int64_t n, const double* v, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e2m1_from_double(v[i]);
+  return 0;
+}
+int oracle_e2m1_decode(int64_t n, const uint8_t* c, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e2m1_to_double(c[i]);
+  return 0;
+}
+
+// MXFP4 quantisation of a row-major [rows, K] matrix (K a multiple of 32) held
+// as fp32 (dtype 0), bf16 (1) or double (2): codes [rows, K] (one per byte),
+// scales [rows, K/32] (biased exponents). Returns -1 if K % 32 != 0.
+int oracle_mx4_quantize(int64_t rows, int64_t K, int dtype, const void* src, uint8_t* codes,
+                        uint8_t* scales) {
+  if (K % 32 != 0) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < K / 32; ++b) {
+      double v[32], amax = 0.0;
+      for (int i = 0; i < 32; ++i) {
+        v[i] = load_any(src, dtype, r * K + b * 32 + i);
+        amax = std::max(amax, std::fabs(v[i]));
+      }
+      const int e = mx4_exponent(amax);
+      scales[r * (K / 32) + b] = (uint8_t)(e + 127);
+      for (int i = 0; i < 32; ++i) codes[r * K + b * 32 + i] = e2m1_from_double(std::ldexp(v[i], -e));
+    }
+  }
+  return 0;
+}
+
+// codes * 2^(scale - 127), double [rows, K].
+int oracle_mx4_dequantize(int64_t rows, int64_t K, const uint8_t* codes, const uint8_t* scales,
+                          double* out) {
+  if (K % 32 != 0) return -1;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t i = 0; i < K; ++i)
+      out[r * K + i] = std::ldexp(e2m1_to_double(codes[r * K + i]),
+                                  (int)scales[r * (K / 32) + i / 32] - 127);
+  return 0;
+}
+
+}  // extern "C"

@@ -68,6 +68,10 @@ def _load():
             lib.oracle_e4m3_decode.argtypes = [I64, P, P]
             lib.oracle_mx_quantize.argtypes = [I64, I64, ctypes.c_int, P, P, P]
             lib.oracle_mx_dequantize.argtypes = [I64, I64, P, P, P]
+            lib.oracle_e2m1_encode.argtypes = [I64, P, P]
+            lib.oracle_e2m1_decode.argtypes = [I64, P, P]
+            lib.oracle_mx4_quantize.argtypes = [I64, I64, ctypes.c_int, P, P, P]
+            lib.oracle_mx4_dequantize.argtypes = [I64, I64, P, P, P]
             lib.oracle_forward_mxfp8.argtypes = [CP, I64, P, P, P, P, P, P, P, P, P, ctypes.c_int,
                                                  I64, P, P]
             lib.oracle_forward_part.argtypes = [CP, I64, ctypes.c_int, P, P, P, P, P, P,
@@ -344,6 +348,65 @@ def forward_mxfp8(cfg: dict, x, idx, w, w1, w3, w2, tok_ids, has_bias: bool,
     if code != 0:
         raise ValueError("oracle_forward_mxfp8: bad token id, missing weights or dims not multiples of 32")
     return y
+
+
+# ----------------------------------------------------------------------------
+# MXFP4 (E2M1 elements, one power-of-two scale per 32 along K)
+# ----------------------------------------------------------------------------
+def e2m1_encode(v) -> np.ndarray:
+    """E2M1 codes (uint8 0..15, sign in bit 3) of float64 values, round to
+    nearest even, saturating at 6."""
+    v = np.ascontiguousarray(np.asarray(v, np.float64))
+    out = np.empty(v.shape, np.uint8)
+    _load().oracle_e2m1_encode(v.size, _ptr(v), _ptr(out))
+    return out
+
+
+def e2m1_decode(c) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(c, np.uint8))
+    out = np.empty(c.shape, np.float64)
+    _load().oracle_e2m1_decode(c.size, _ptr(c), _ptr(out))
+    return out
+
+
+def mx4_quantize(a) -> tuple[np.ndarray, np.ndarray]:
+    """[rows, K] (fp32, bf16 tensor or float64) -> (codes [rows, K] uint8, one
+    E2M1 code per byte; biased scale exponents [rows, K/32] uint8)."""
+    if isinstance(a, np.ndarray) and a.dtype == np.float64:
+        raw, dt = np.ascontiguousarray(a), 2
+    else:
+        raw, dt = _as_raw(a)
+    rows, K = raw.shape
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, K // 32), np.uint8)
+    if _load().oracle_mx4_quantize(rows, K, dt, _ptr(raw), _ptr(codes), _ptr(scales)) != 0:
+        raise ValueError("mx4_quantize: K must be a multiple of 32")
+    return codes, scales
+
+
+def mx4_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, K = codes.shape
+    out = np.empty((rows, K), np.float64)
+    _load().oracle_mx4_dequantize(rows, K, _ptr(codes), _ptr(scales), _ptr(out))
+    return out
+
+
+def e2m1_as_e4m3(codes: np.ndarray) -> np.ndarray:
+    """The E4M3 code of each E2M1 code's value (every E2M1 value is an E4M3
+    value, so this loses nothing)."""
+    table = e4m3_encode(e2m1_decode(np.arange(16, dtype=np.uint8)))
+    return table[np.asarray(codes, np.uint8)]
+
+
+def forward_mxfp4(cfg: dict, x, idx, w, w1, w3, w2, tok_ids, has_bias: bool) -> np.ndarray:
+    """The literal loop with MXFP4 expert weights (tokens and hidden vectors in
+    MXFP8, as in the 8-bit form). w1/w3/w2: sequences of E+S (E2M1 codes, scales)
+    pairs (None where unused). The weights' values are those of E4M3 codes with
+    the same scales, so this is forward_mxfp8 on the re-encoded codes."""
+    conv = lambda ws: [None if q is None else (e2m1_as_e4m3(q[0]), q[1]) for q in ws]
+    return forward_mxfp8(cfg, x, idx, w, conv(w1), conv(w3), conv(w2), tok_ids, has_bias)
 
 
 def forward_part(cfg: dict, x, idx, w, w1, w3, w2, tok_ids, has_bias: bool, expert_begin: int,
