@@ -18,7 +18,8 @@ kernel (the gate/up expert GEMM) against the measured bf16 tensor peak
 (sustained: the GEMM runs inside back-to-back steps at the power cap);
 `routing` is the expert-load histogram summary and the near-tie count;
 `cpu_baseline` is the CPU oracle timed on a sample of the same workload on this
-host's cores; "mxfp8" repeats prefill and decode with MXFP8 expert weights.
+host's cores; "mxfp8" and "mxfp4" repeat prefill and decode with MXFP8 and
+MXFP4 expert weights.
 `--impl reference` times the oracle alone (rank 0 only) in the same JSON form.
 
 `--dump DIR` saves each timed step's inputs and outputs as .npy files under
@@ -76,6 +77,7 @@ def parse_args(argv=None):
                     help="target wall time of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true", help="skip the MXFP8-weight lines")
+    ap.add_argument("--no-mxfp4", action="store_true", help="skip the MXFP4-weight lines")
     ap.add_argument("--ep-ranks", type=int, default=8,
                     help="N=1: time each rank's local step of the expert-parallel layer over "
                          "this many ranks, one after another (0 to skip)")
@@ -213,8 +215,9 @@ class ClockSampler:
 def algorithmic(layer, idx: np.ndarray) -> dict:
     T, d, I, k, S, E = layer.T, layer.dim, layer.inter, layer.topk, layer.n_shared, layer.n_experts
     es = 4 if layer.dtype == "f32" else 2
-    # expert-weight bytes per element (MXFP8: one byte plus one scale byte per 32)
-    ew = 1 + 1 / 32 if layer.dtype == "mxfp8" else es
+    # expert-weight bytes per element (MXFP8: one byte plus one scale byte per 32;
+    # MXFP4: half a byte plus one scale byte per 32)
+    ew = {"mxfp8": 1 + 1 / 32, "mxfp4": 0.5 + 1 / 32}.get(layer.dtype, es)
     R = T * (k + S)
     active = int((np.bincount(idx.ravel(), minlength=E) > 0).sum()) + S
     return {
@@ -424,7 +427,7 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False, d
     y = torch.empty((T, layer.dim), dtype=inp["x"].dtype, device=dev)
     idx = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
     w = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
-    fp8 = layer.dtype == "mxfp8"
+    fp8 = layer.dtype in ("mxfp8", "mxfp4")   # block-scaled expert weights
     if fp8:
         # MXFP8 form: pack the seeded bf16 expert weights once, then drop them.
         q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
@@ -646,7 +649,7 @@ def replay_step(path) -> dict:
     y = torch.empty_like(load("y"))
     idx = torch.empty((T, layer.topk), dtype=torch.int32, device=dev)
     w = torch.empty((T, layer.topk), dtype=torch.float32, device=dev)
-    if layer.dtype == "mxfp8":
+    if layer.dtype in ("mxfp8", "mxfp4"):
         q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
         K.kt_moe_forward_mxfp8(cfg, T, inp["x"], inp["w_gate"], inp["bias"], q["w1q"], q["w3q"],
                                q["w2q"], q["sf_up"], q["sf_down"], y, idx, w, ws)
@@ -724,16 +727,19 @@ def run_ours(a):
         dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, graph=True,
                          dump=a.dump)
         dec["routing"] = routing_stats(dlayer, dec["inp"], dec["idx"], dev)
-    # The same layers with MXFP8 expert weights (same shapes, seeds and tokens).
-    f8 = {}
-    if not a.no_mxfp8:
+    # The same layers with MXFP8 and MXFP4 expert weights (same shapes, seeds and
+    # tokens).
+    mx = {}
+    for fmt, skip in (("mxfp8", a.no_mxfp8), ("mxfp4", a.no_mxfp4)):
+        if skip:
+            continue
         for key, base in (("prefill", layer.name), ("decode", a.decode_workload)):
-            name = base + "_mxfp8"
+            name = base + "_" + fmt
             if name in W.BY_NAME:
-                f8[key] = (W.BY_NAME[name], time_layer(W.BY_NAME[name], dev, rank, world, a.steps,
-                                                       a.warmup, a.e2e_steps,
-                                                       graph=key == "decode", dump=a.dump))
-                f8[key][1].pop("inp")
+                res = time_layer(W.BY_NAME[name], dev, rank, world, a.steps, a.warmup,
+                                 a.e2e_steps, graph=key == "decode", dump=a.dump)
+                res.pop("inp")
+                mx.setdefault(fmt, {})[key] = (W.BY_NAME[name], res)
     clk = clocks.stop()
 
     cpu = None
@@ -812,11 +818,17 @@ def run_ours(a):
                           "value": round(world * dl.T * a.steps / (dec["graph_ms"] / 1e3), 1),
                           "unit": "tokens/s"},
             }
-        if f8:
-            line["mxfp8"] = {"note": "MXFP8 expert weights (E4M3, power-of-two scale per 32 "
-                                     "along K); bf16 tokens, gate and output"}
-            f8_peak = 2 * peaks["bf16_tflops_sustained"]
-            for key, (fl, res) in f8.items():
+        notes = {"mxfp8": "MXFP8 expert weights (E4M3, power-of-two scale per 32 along K); "
+                          "bf16 tokens, gate and output",
+                 "mxfp4": "MXFP4 expert weights (E2M1 codes two per byte, power-of-two scale "
+                          "per 32 along K) against MXFP8 (E4M3) tokens and hidden rows; bf16 "
+                          "gate and output"}
+        # Both block-scaled forms run tcgen05 kind::mxf8f6f4, whose dense rate is
+        # the FP8 one (E2M1 operands there do not run faster).
+        mx_peak = 2 * peaks["bf16_tflops_sustained"]
+        for fmt, runs in mx.items():
+            line[fmt] = {"note": notes[fmt]}
+            for key, (fl, res) in runs.items():
                 ms = res["ms"] / K_
                 ent = {"workload": fl.name, "value": round(world * fl.T / (ms / 1e3), 1),
                        "unit": "tokens/s", "ms_per_step": round(ms, 4),
@@ -824,12 +836,13 @@ def run_ours(a):
                        "e2e": {"value": round(world * fl.T * a.e2e_steps / (res["e2e_ms"] / 1e3), 1),
                                "unit": "tokens/s"}}
                 up_s = res["stage_ms"]["up_gemm"] / 1e3
+                kern = ("grouped gate/up GEMM (tcgen05 kind::mxf8f6f4"
+                        + (", E2M1 x E4M3)" if fmt == "mxfp4" else ")"))
                 if key == "prefill":
                     ach = res["work"]["flops_up"] / up_s / 1e12
-                    ent["roofline"] = {"kernel": "grouped gate/up GEMM (tcgen05 kind::mxf8f6f4)",
-                                       "bound": "tensor", "achieved": round(ach, 1),
-                                       "peak": f8_peak, "unit": "TFLOP/s",
-                                       "frac": round(ach / f8_peak, 4),
+                    ent["roofline"] = {"kernel": kern, "bound": "tensor", "achieved": round(ach, 1),
+                                       "peak": mx_peak, "unit": "TFLOP/s",
+                                       "frac": round(ach / mx_peak, 4),
                                        "traffic": traffic("up", fl.name),
                                        "peak_source": peaks["source"] + " bf16 (sustained) x 2, "
                                                       "the nominal fp8 / bf16 ratio"}
@@ -838,8 +851,7 @@ def run_ours(a):
                     lgbs = res["work"]["bytes_layer"] / (ms / 1e3) / 1e9
                     ent["layer_hbm_gbs"] = round(lgbs, 1)
                     ent["layer_hbm_frac"] = round(lgbs / peaks["hbm_gbs"], 4)
-                    ent["roofline"] = {"kernel": "grouped gate/up GEMM (tcgen05 kind::mxf8f6f4)",
-                                       "bound": "hbm", "achieved": round(gbs, 1),
+                    ent["roofline"] = {"kernel": kern, "bound": "hbm", "achieved": round(gbs, 1),
                                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                        "frac": round(gbs / peaks["hbm_gbs"], 4),
                                        "traffic": traffic("up", fl.name)}
@@ -847,7 +859,7 @@ def run_ours(a):
                     ent["graph"] = {"ms_per_step": round(res["graph_ms"] / K_, 4),
                                     "value": round(world * fl.T * K_ / (res["graph_ms"] / 1e3), 1),
                                     "unit": "tokens/s"}
-                line["mxfp8"][key] = ent
+                line[fmt][key] = ent
         if epr:
             line["expert_parallel"] = epr
         print(json.dumps(line), flush=True)

@@ -50,8 +50,10 @@ enum { KT_SCORE_SIGMOID = 0, KT_SCORE_SOFTMAX = 1 };
 /* Group score of gate step 2. AUTO = TOP2SUM when a bias is given, else AMAX. */
 enum { KT_GROUP_AUTO = 0, KT_GROUP_AMAX = 1, KT_GROUP_TOP2SUM = 2 };
 /* Activation / expert-weight dtype. KT_DTYPE_MXFP8: bf16 tokens, gate weights
- * and output (as KT_DTYPE_BF16); expert weights in MXFP8 (kt_moe_forward_mxfp8). */
-enum { KT_DTYPE_F32 = 0, KT_DTYPE_BF16 = 1, KT_DTYPE_MXFP8 = 2 };
+ * and output (as KT_DTYPE_BF16); expert weights in MXFP8 (kt_moe_forward_mxfp8).
+ * KT_DTYPE_MXFP4: the same with expert weights in MXFP4 (4-bit E2M1 elements;
+ * also through kt_moe_forward_mxfp8 and the other MXFP8 entry points). */
+enum { KT_DTYPE_F32 = 0, KT_DTYPE_BF16 = 1, KT_DTYPE_MXFP8 = 2, KT_DTYPE_MXFP4 = 3 };
 
 enum {
   KT_OK = 0,
@@ -77,7 +79,7 @@ enum {
  * implies topk_groups == 1; TOP2SUM needs >= 2 experts per group;
  * 0 <= n_shared <= 8; route_scale finite and > 0; dim, inter >= 8 and
  * multiples of 8 (bf16) or 4 (fp32), so rows are 16-byte multiples; for
- * KT_DTYPE_MXFP8 multiples of 128 (one 128-byte K slab of FP8).
+ * KT_DTYPE_MXFP8 and KT_DTYPE_MXFP4 multiples of 128 (one 128-element K slab).
  */
 typedef struct {
   int32_t n_experts;    /* E: routed experts                                      */
@@ -289,6 +291,33 @@ int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, con
                          const uint8_t* w2q, const uint8_t* sf_up, const uint8_t* sf_down,
                          void* y, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                          size_t ws_bytes, void* stream, void* const* stage_events);
+
+/*
+ * MXFP4 expert weights: the 4-bit form of the layer (cfg->dtype =
+ * KT_DTYPE_MXFP4). The KTransformers DeepSeek page runs routed experts held
+ * natively in MXFP4 ("DeepSeek V4-Flash", its training notes) and gives no
+ * quantisation rule. Format: E2M1 elements (1 sign bit, 2 exponent bits with
+ * bias 1, 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one
+ * power-of-two scale 2^e per 32 consecutive elements along K, stored as the
+ * byte e + 127. Rule (the MXFP8 rule with 6 for 448): e is the smallest integer
+ * with amax <= 6 * 2^e (0 gives e = -127), each element the E2M1
+ * round-to-nearest-even of v * 2^-e. Codes are packed two per byte, element 2i
+ * in the low nibble of byte i, the sign in bit 3 of its nibble.
+ *
+ * kt_moe_mxfp4_quantize: row-major [rows, K] bf16 (K % 32 == 0) -> packed codes
+ *   [rows, K/2] bytes and scale bytes [rows, K/32]; 16-B aligned src and codes.
+ *
+ * The MXFP8 entry points take MXFP4 configs unchanged: kt_moe_mxfp8_pack writes
+ *   packed codes (w1q, w3q [E+S, inter, dim/2], w2q [E+S, dim, inter/2] bytes)
+ *   and the scales in the layout above (kt_moe_mxfp8_scale_bytes, the same
+ *   sizes); kt_moe_forward_mxfp8, kt_moe_graph_create_mxfp8 and the
+ *   expert-parallel *_mxfp8 forms run the 4-bit layer. The code pointers must be
+ *   32-byte aligned and w3q - w1q a multiple of 32 bytes (KT_ERR_ALIGN). Tokens
+ *   and SwiGLU hidden rows stay MXFP8 (E4M3); the GEMMs run the block-scaled
+ *   tensor-core MMA with E2M1 weights and E4M3 tokens, fp32 accumulation.
+ */
+int kt_moe_mxfp4_quantize(int64_t rows, int64_t K, const void* src, uint8_t* codes,
+                          uint8_t* scales, void* stream);
 
 /*
  * Expert-parallel form: the multi-card steps of "MoE 前向四步" in the DeepSeek-V3

@@ -56,9 +56,11 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
   if (!std::isfinite(c->route_scale) || !(c->route_scale > 0.f)) return KT_ERR_INVALID_CONFIG;
   if (c->score_func != KT_SCORE_SIGMOID && c->score_func != KT_SCORE_SOFTMAX)
     return KT_ERR_INVALID_CONFIG;
-  if (c->dtype != KT_DTYPE_F32 && c->dtype != KT_DTYPE_BF16 && c->dtype != KT_DTYPE_MXFP8)
+  if (c->dtype != KT_DTYPE_F32 && c->dtype != KT_DTYPE_BF16 && c->dtype != KT_DTYPE_MXFP8 &&
+      c->dtype != KT_DTYPE_MXFP4)
     return KT_ERR_INVALID_CONFIG;
-  const int align = c->dtype == KT_DTYPE_MXFP8 ? 128 : (c->dtype == KT_DTYPE_BF16 ? 8 : 4);
+  const bool block_scaled = c->dtype == KT_DTYPE_MXFP8 || c->dtype == KT_DTYPE_MXFP4;
+  const int align = block_scaled ? 128 : (c->dtype == KT_DTYPE_BF16 ? 8 : 4);
   if (c->dim < 8 || c->inter < 8 || c->dim % align || c->inter % align) return KT_ERR_INVALID_CONFIG;
   if (c->dim > (1 << 16) || c->inter > (1 << 16)) return KT_ERR_INVALID_CONFIG;
   if (c->norm_topk < -1 || c->norm_topk > 1) return KT_ERR_INVALID_CONFIG;
@@ -81,7 +83,8 @@ int resolve(const kt_moe_config* c, int64_t T, int has_bias, Resolved* r) {
   if (G > 1 && r->group_score == KT_GROUP_TOP2SUM && gs < 2) return KT_ERR_INVALID_CONFIG;
   r->dtype = c->dtype;
   r->act_bf16 = c->dtype != KT_DTYPE_F32;
-  r->fp8 = c->dtype == KT_DTYPE_MXFP8;
+  r->fp8 = block_scaled ? 1 : 0;
+  r->w4 = c->dtype == KT_DTYPE_MXFP4 ? 1 : 0;
   r->chunk_rows = r->fp8 ? kChunkRowsF8 : kChunkRows;
   r->n_local = E;
   r->sb = 0;
@@ -471,6 +474,20 @@ int kt_moe_mxfp8_quantize(int64_t rows, int64_t K, const void* src, uint8_t* cod
              : KT_ERR_CUDA;
 }
 
+int kt_moe_mxfp4_quantize(int64_t rows, int64_t K, const void* src, uint8_t* codes,
+                          uint8_t* scales, void* stream) {
+  if (rows < 0 || K <= 0 || K % 32 != 0) return KT_ERR_INVALID_CONFIG;
+  if (!src || !codes || !scales) return KT_ERR_NULL;
+  if (!aligned(src, 16) || !aligned(codes, 16)) return KT_ERR_ALIGN;
+  int sms = 0;
+  const int rc = device_info(&sms);
+  if (rc != KT_OK) return rc;
+  return launch_mx4_quantize(src, rows, K, codes, scales, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? KT_OK
+             : KT_ERR_CUDA;
+}
+
 size_t kt_moe_mxfp8_scale_bytes(const kt_moe_config* cfg, int down) {
   Resolved r;
   if (resolve(cfg, 1, 0, &r) != KT_OK || !r.fp8) return 0;
@@ -496,6 +513,12 @@ int kt_moe_mxfp8_pack(const kt_moe_config* cfg, const void* w1, const void* w3, 
              : KT_ERR_CUDA;
 }
 
+// Checks of the block-scaled weight arguments (MXFP8 and MXFP4 configs). The
+// packed gate/up scales list W1's rows before W3's and the kernel loads the
+// codes of both in one box in address order, so W1's must come first.
+static int mxfp8_weight_args(const Resolved& r, const uint8_t* w1q, const uint8_t* w3q,
+                             const uint8_t* w2q, const uint8_t* sf_up, const uint8_t* sf_down);
+
 int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, const void* w_gate,
                          const float* bias, const uint8_t* w1q, const uint8_t* w3q,
                          const uint8_t* w2q, const uint8_t* sf_up, const uint8_t* sf_down,
@@ -505,13 +528,7 @@ int kt_moe_forward_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x, con
   int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y, topk_idx_out,
                               topk_w_out, workspace, ws_bytes, &r);
   if (rc != KT_OK) return rc;
-  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
-  if (!sf_up || !sf_down) return KT_ERR_NULL;
-  // The packed gate/up scales list W1's rows before W3's; the kernel loads the
-  // codes of both in one box in address order, so W1's must come first.
-  if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
-    return KT_ERR_INVALID_CONFIG;
-  if (!aligned(sf_up, 16) || !aligned(sf_down, 16)) return KT_ERR_ALIGN;
+  if ((rc = mxfp8_weight_args(r, w1q, w3q, w2q, sf_up, sf_down)) != KT_OK) return rc;
   return run_forward(r, identity_table(r), T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y,
                      false, topk_idx_out,
                      topk_w_out, workspace, stream, stage_events);
@@ -565,12 +582,16 @@ static int placed_table(Resolved* r, const int32_t* expert_slot, SlotTable* tab)
 }
 
 static int mxfp8_weight_args(const Resolved& r, const uint8_t* w1q, const uint8_t* w3q,
-                             const uint8_t* sf_up, const uint8_t* sf_down) {
+                             const uint8_t* w2q, const uint8_t* sf_up, const uint8_t* sf_down) {
   if (!r.fp8) return KT_ERR_INVALID_CONFIG;
   if (!sf_up || !sf_down) return KT_ERR_NULL;
   if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
     return KT_ERR_INVALID_CONFIG;
   if (!aligned(sf_up, 16) || !aligned(sf_down, 16)) return KT_ERR_ALIGN;
+  // Packed 4-bit codes are read through 32-byte aligned tensor maps.
+  if (r.w4 && (!aligned(w1q, 32) || !aligned(w3q, 32) || !aligned(w2q, 32) ||
+               (reinterpret_cast<uintptr_t>(w3q) - reinterpret_cast<uintptr_t>(w1q)) % 32 != 0))
+    return KT_ERR_ALIGN;
   return KT_OK;
 }
 
@@ -603,7 +624,7 @@ int kt_moe_forward_local_mxfp8(const kt_moe_config* cfg, int64_t T, const void* 
   int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y_part, topk_idx_out,
                               topk_w_out, workspace, ws_bytes, &r, /*y_partial=*/true);
   if (rc != KT_OK) return rc;
-  if ((rc = mxfp8_weight_args(r, w1q, w3q, sf_up, sf_down)) != KT_OK) return rc;
+  if ((rc = mxfp8_weight_args(r, w1q, w3q, w2q, sf_up, sf_down)) != KT_OK) return rc;
   if ((rc = range_table(&r, expert_begin, expert_end, &tab)) != KT_OK) return rc;
   if ((rc = set_shared_range(&r, T, shared_begin, shared_end)) != KT_OK) return rc;
   return run_forward(r, tab, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y_part, true,
@@ -639,7 +660,7 @@ int kt_moe_forward_placed_mxfp8(const kt_moe_config* cfg, int64_t T, const void*
   int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y_part, topk_idx_out,
                               topk_w_out, workspace, ws_bytes, &r, /*y_partial=*/true);
   if (rc != KT_OK) return rc;
-  if ((rc = mxfp8_weight_args(r, w1q, w3q, sf_up, sf_down)) != KT_OK) return rc;
+  if ((rc = mxfp8_weight_args(r, w1q, w3q, w2q, sf_up, sf_down)) != KT_OK) return rc;
   if ((rc = placed_table(&r, expert_slot, &tab)) != KT_OK) return rc;
   if ((rc = set_shared_range(&r, T, shared_begin, shared_end)) != KT_OK) return rc;
   return run_forward(r, tab, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y_part, true,
@@ -799,10 +820,7 @@ int kt_moe_graph_create_mxfp8(const kt_moe_config* cfg, int64_t T, const void* x
   int rc = check_forward_args(cfg, T, x, w_gate, bias, w1q, w3q, w2q, y, topk_idx_out,
                               topk_w_out, workspace, ws_bytes, &r);
   if (rc != KT_OK) return rc;
-  if (!r.fp8) return KT_ERR_INVALID_CONFIG;
-  if (!sf_up || !sf_down) return KT_ERR_NULL;
-  if (reinterpret_cast<uintptr_t>(w3q) <= reinterpret_cast<uintptr_t>(w1q))
-    return KT_ERR_INVALID_CONFIG;
+  if ((rc = mxfp8_weight_args(r, w1q, w3q, w2q, sf_up, sf_down)) != KT_OK) return rc;
   return capture_graph(
       [&](cudaStream_t cs) {
         return kt_moe_forward_mxfp8(cfg, T, x, w_gate, bias, w1q, w3q, w2q, sf_up, sf_down, y,

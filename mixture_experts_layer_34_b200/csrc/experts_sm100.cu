@@ -147,6 +147,7 @@ struct GemmArgs {
   int64_t n_rows;            // hidden rows T * (k + S)
   int max_chunks;            // chunk list capacity
   int max_chunk_rows;        // rows per chunk at most
+  int a_fp4;                 // MXFP8 kinds: weights as packed E2M1 codes (MXFP4), else E4M3
   int tma3d;                 // 1: one box per stage from the 3-D/4-D maps (K % 64 == 0)
   int gate_hi;               // up, 3-D maps: W3 precedes W1 in memory, so the upper 64
                              // rows of each CTA's weight tile are W1 (gate)
@@ -325,11 +326,13 @@ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
 }
 // MXFP8: E4M3 A and B, E8M0 block scales (one per 32 along K) read from TMEM;
 // the scale byte used by this K = 32 MMA is selected by sf_id (bits 29-30 for A,
-// 4-5 for B). Accumulation is fp32.
-__device__ __forceinline__ uint32_t idesc_mxf8(int M, int N, int sf_id) {
-  return (static_cast<uint32_t>(sf_id) << 4) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) |
-         (static_cast<uint32_t>(sf_id) << 29);
+// 4-5 for B). a_fmt (bits 7-9) is A's element format: 0 E4M3, 5 E2M1 (MXFP4
+// weights; B stays E4M3). Accumulation is fp32.
+constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
+__device__ __forceinline__ uint32_t idesc_mxf8(int M, int N, int sf_id, uint32_t a_fmt) {
+  return (static_cast<uint32_t>(sf_id) << 4) | (a_fmt << 7) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(sf_id) << 29);
 }
 __device__ __forceinline__ void mma_pair_mxf8(uint32_t d_tmem, uint64_t a, uint64_t b,
                                               uint32_t idesc, uint32_t sfa_tmem,
@@ -656,10 +659,12 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           uint8_t* sB = sA + slabs * kATileBytes;
           if (args.tma3d) {
             // Two boxes for the whole stage; slabs past K are filled with zeros
-            // and counted in the transaction bytes.
+            // and counted in the transaction bytes. Packed 4-bit weight codes
+            // count their global bytes, half the weight tile's shared bytes.
             const uint32_t sf_bytes = KD::kF8 ? slabs * (kSfaSlabBytes + kSfbSlabBytes) : 0;
+            const uint32_t a_tx = (KD::kF8 && args.a_fp4) ? kATileBytes / 2 : kATileBytes;
             if (leader)
-              mbar_arrive_expect_tx(&full_bar[stage], 2u * (slabs * (kATileBytes + b_slab) + sf_bytes));
+              mbar_arrive_expect_tx(&full_bar[stage], 2u * (slabs * (a_tx + b_slab) + sf_bytes));
             if (kUp)
               tma_load4_pair(sA, a3, fbar, 0, a_row, 0, s0, pol_a);
             else
@@ -730,6 +735,7 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer (even CTA, for the pair) ----------------
       const uint64_t desc_a0 = sw128_desc(smem_u32(stage_base));
+      const uint32_t a_fmt = args.a_fp4 ? kFmtE2M1 : kFmtE4M3;
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
@@ -789,8 +795,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
               if (n > 128) sf_copy_pair(sfb + 4, sB + kSfbSlabBytes / 2);
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                mma_pair_mxf8(d0, da + 2 * ks, db + 2 * ks, idesc_mxf8(256, n, ks), sfa, sfb,
-                              (kb | j | ks) != 0);
+                mma_pair_mxf8(d0, da + 2 * ks, db + 2 * ks, idesc_mxf8(256, n, ks, a_fmt), sfa,
+                              sfb, (kb | j | ks) != 0);
             } else {
 #pragma unroll
               for (int ks = 0; ks < kBK / 16; ++ks)
@@ -1030,16 +1036,30 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 // 3-D view [cols / slab][rows][slab] of a row-major [rows, cols] matrix of bf16
 // (slab 64) or one-byte E4M3 codes (u8: slab 128) with cols a multiple of the
 // slab; box = box_slabs x box_rows x slab (128 bytes wide), landing slab-major.
+// Element kinds of the K-slab maps: bf16 (64 per 128-byte slab), bytes (E4M3
+// codes, 128 per slab), and packed E2M1 codes (128 per slab: 64 bytes in
+// global memory, which the copy spreads to 128 bytes in shared memory, each 8
+// bytes of codes followed by an 8-byte gap, the layout the block-scaled MMA
+// reads 4-bit operands in; its transaction count is the 64 global bytes).
+enum { kElemBf16 = 0, kElemU8 = 1, kElemFp4 = 2 };
+
+CUtensorMapDataType elem_type(int elem) {
+  return elem == kElemFp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B
+                          : (elem == kElemU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                             : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
 bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
-               uint32_t box_slabs, bool u8 = false) {
+               uint32_t box_slabs, int elem = kElemBf16) {
   EncodeTiledFn enc = get_encode_fn();
-  const uint64_t es = u8 ? 1 : 2, slab = 128 / es;
+  // Elements per slab and global bytes per slab row.
+  const uint64_t slab = elem == kElemBf16 ? 64 : 128, slab_bytes = elem == kElemFp4 ? 64 : 128;
   if (!enc || cols % slab != 0) return false;
   const cuuint64_t dims[3] = {slab, rows, cols / slab};
-  const cuuint64_t strides[2] = {cols * es, 128};
+  const cuuint64_t strides[2] = {cols / slab * slab_bytes, slab_bytes};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(slab), box_rows, box_slabs};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+  return enc(m, elem_type(elem), 3,
              const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
@@ -1052,19 +1072,20 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
 // per slab [box_rows rows of the first | the same rows of the second].
 // *q_first tells whether q is the first.
 bool make_map4_pair(CUtensorMap* m, const void* p, const void* q, uint64_t rows, uint64_t cols,
-                    uint32_t box_rows, uint32_t box_slabs, bool* q_first, bool u8 = false) {
+                    uint32_t box_rows, uint32_t box_slabs, bool* q_first, int elem = kElemBf16) {
   EncodeTiledFn enc = get_encode_fn();
   const uint64_t up = reinterpret_cast<uint64_t>(p), uq = reinterpret_cast<uint64_t>(q);
   const uint64_t lo = up < uq ? up : uq, hi = up < uq ? uq : up;
-  const uint64_t es = u8 ? 1 : 2, slab = 128 / es;
+  const uint64_t slab = elem == kElemBf16 ? 64 : 128, slab_bytes = elem == kElemFp4 ? 64 : 128;
+  const uint64_t align = elem == kElemFp4 ? 32 : 16;   // packed 4-bit maps: 32-byte strides
   *q_first = uq < up;
-  if (!enc || cols % slab != 0 || hi == lo || (hi - lo) % 16 != 0 || (hi - lo) >= (1ull << 40))
+  if (!enc || cols % slab != 0 || hi == lo || (hi - lo) % align != 0 || (hi - lo) >= (1ull << 40))
     return false;
   const cuuint64_t dims[4] = {slab, rows, 2, cols / slab};
-  const cuuint64_t strides[3] = {cols * es, hi - lo, 128};
+  const cuuint64_t strides[3] = {cols / slab * slab_bytes, hi - lo, slab_bytes};
   const cuuint32_t box[4] = {static_cast<cuuint32_t>(slab), box_rows, 2, box_slabs};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+  return enc(m, elem_type(elem), 4,
              reinterpret_cast<void*>(lo), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
@@ -1090,9 +1111,9 @@ bool make_map_rows256(CUtensorMap* m, const void* base, uint64_t n_rows, uint32_
 // E4M3 token-row maps of one source (3-D only).
 bool make_token_maps_u8(TmaMaps* M, int src, const void* base, uint64_t rows, uint64_t cols) {
   for (int hb = 1; hb <= 4; ++hb)
-    if (!make_map3(&M->b3[src][hb - 1], base, rows, cols, hb * kBoxRows, kSlabs, true))
+    if (!make_map3(&M->b3[src][hb - 1], base, rows, cols, hb * kBoxRows, kSlabs, kElemU8))
       return false;
-  return make_map3(&M->b3[src][4], base, rows, cols, kBoxRows, kSlabsLight, true);
+  return make_map3(&M->b3[src][4], base, rows, cols, kBoxRows, kSlabsLight, kElemU8);
 }
 
 bool make_token_maps(TmaMaps* M, int src, const void* base, uint64_t rows, uint64_t cols,
@@ -1247,6 +1268,8 @@ cudaError_t launch_experts_mxfp8(const Resolved& r, int64_t T, const Layout& L, 
   a.max_chunks = (int)L.max_chunks;
   a.max_chunk_rows = kChunkRowsF8;
   a.tma3d = 1;
+  a.a_fp4 = r.w4;
+  const int welem = r.w4 ? kElemFp4 : kElemU8;   // weight codes: E2M1 pairs or E4M3 bytes
   const int grid = pair_grid(num_sms, 0);
   TmaMaps M;
   memset(&M, 0, sizeof(M));
@@ -1254,8 +1277,8 @@ cudaError_t launch_experts_mxfp8(const Resolved& r, int64_t T, const Layout& L, 
     const uint64_t rows = (uint64_t)NG * r.I;
     const uint64_t sfb_rows = (uint64_t)L.max_chunks * (r.d / 128) * 4;
     bool w3_first = false;
-    if (!make_map4_pair(&M.a3[0], wa, wb, rows, r.d, 64, kSlabs, &w3_first, true) ||
-        !make_map4_pair(&M.a3[1], wa, wb, rows, r.d, 64, kSlabsLight, &w3_first, true) ||
+    if (!make_map4_pair(&M.a3[0], wa, wb, rows, r.d, 64, kSlabs, &w3_first, welem) ||
+        !make_map4_pair(&M.a3[1], wa, wb, rows, r.d, 64, kSlabsLight, &w3_first, welem) ||
         !make_token_maps_u8(&M, 0, ws + L.xperm, Rr, r.d) ||
         !make_token_maps_u8(&M, 1, ws + L.xq, T, r.d) ||
         !make_map_rows256(&M.sfa[0], sf, mx_packed_bytes(r, false) / 256, 2 * kSlabs) ||
@@ -1282,8 +1305,8 @@ cudaError_t launch_experts_mxfp8(const Resolved& r, int64_t T, const Layout& L, 
   }
   const uint64_t rows = (uint64_t)NG * r.d;
   const uint64_t sfb_rows = (uint64_t)L.max_chunks * (r.I / 128) * 4;
-  if (!make_map3(&M.a3[0], wa, rows, r.I, kARowsCta, kSlabs, true) ||
-      !make_map3(&M.a3[1], wa, rows, r.I, kARowsCta, kSlabsLight, true) ||
+  if (!make_map3(&M.a3[0], wa, rows, r.I, kARowsCta, kSlabs, welem) ||
+      !make_map3(&M.a3[1], wa, rows, r.I, kARowsCta, kSlabsLight, welem) ||
       !make_token_maps_u8(&M, 0, ws + L.hidden, R, r.I) ||
       !make_map_rows256(&M.sfa[0], sf, mx_packed_bytes(r, true) / 256, 2 * kSlabs) ||
       !make_map_rows256(&M.sfa[1], sf, mx_packed_bytes(r, true) / 256, 2 * kSlabsLight) ||

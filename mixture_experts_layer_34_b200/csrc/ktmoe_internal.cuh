@@ -52,7 +52,8 @@ struct Resolved {
   int group_score;  // KT_GROUP_AMAX / KT_GROUP_TOP2SUM (G == 1: unused)
   int dtype;        // KT_DTYPE_*
   int act_bf16;     // tokens, gate weights and output in bf16 (KT_DTYPE_BF16 / MXFP8)
-  int fp8;          // expert weights in MXFP8
+  int fp8;          // block-scaled expert weights (MXFP8 or MXFP4): tokens and hidden rows in MXFP8
+  int w4;           // expert weights in MXFP4 (E2M1 codes, two per byte)
   int chunk_rows;   // token rows per GEMM chunk: kChunkRows, or kChunkRowsF8 for MXFP8
   int n_local;      // routed experts computed here (all: E); their weights are the first
                     // n_local slots of w1/w3/w2 (placed by a SlotTable), the shared ones follow
@@ -174,6 +175,9 @@ cudaError_t launch_ep_finish(const Resolved& r, int64_t T, const float* y_sum, c
 // MXFP8 (mxfp8.cu).
 cudaError_t launch_mx_quantize(const void* src, int64_t rows, int64_t K, uint8_t* codes,
                                uint8_t* scales, cudaStream_t st);
+// MXFP4: packed E2M1 codes [rows, K/2] (element 2i in the low nibble of byte i).
+cudaError_t launch_mx4_quantize(const void* src, int64_t rows, int64_t K, uint8_t* codes,
+                                uint8_t* scales, cudaStream_t st);
 size_t mx_packed_bytes(const Resolved& r, bool down);
 cudaError_t launch_mx_pack(const Resolved& r, const void* w1, const void* w3, const void* w2,
                            uint8_t* w1q, uint8_t* w3q, uint8_t* w2q, uint8_t* sf_up,
@@ -201,6 +205,26 @@ __device__ __forceinline__ float mx_inv_scale(int e) {
 // E4M3 code of v * inv, round to nearest even (|v * inv| <= 448 by the scale rule).
 __device__ __forceinline__ uint8_t mx_code(float v, float inv) {
   return (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(v, inv), __NV_SATFINITE, __NV_E4M3);
+}
+// MXFP4 scale exponent: the smallest e with amax <= 6 * 2^e (amax = m * 2^E,
+// m in [1, 2): e = E - 2 + (m > 1.5)); 0 or subnormal amax gives -127.
+__device__ __forceinline__ int mx4_scale_exp(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ef = (int)((b >> 23) & 0xFF);
+  if (ef == 0) return -127;
+  const int e = ef - 127 - 2 + ((b & 0x7FFFFFu) > 0x400000u ? 1 : 0);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+// E2M1 code (0..15, sign in bit 3) of v: round to nearest of the magnitudes
+// 0, 0.5, 1, 1.5, 2, 3, 4, 6, ties to the even code (mantissa bit 0), values
+// above 6 to 6. The code is the number of decision points at or below |v|;
+// each tie point counts toward the even neighbour (a strict or a non-strict
+// comparison).
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  const float a = fabsf(v);
+  const uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+                     (a >= 3.5f) + (a > 5.0f);
+  return c | ((__float_as_uint(v) >> 28) & 8u);
 }
 
 // Byte offset of the scale of (row m of a GEMM chunk, K block b) in the chunk

@@ -14,6 +14,11 @@
 //                        and the packed scale blocks the grouped GEMM loads
 //                        (mx_packed_offset_*: the layout kt_moe_mxfp8_pack
 //                        documents).
+//
+// MXFP4 (kW4 = true; the 4-bit form): the same blocks with E2M1 elements and
+// the rule e = the smallest integer with amax <= 6 * 2^e (mx4_scale_exp,
+// e2m1_code); 32 codes pack into 16 bytes, element 2i in the low nibble of
+// byte i. The scale layout is the same.
 #include <cuda_bf16.h>
 
 #include "ktmoe_internal.cuh"
@@ -53,13 +58,45 @@ __device__ __forceinline__ uint8_t mx_block_bf16(const uint4* __restrict__ src,
   return (uint8_t)(e + 127);
 }
 
+// 32 bf16 values (64 bytes) to 32 E2M1 codes (16 bytes); returns the scale byte.
+__device__ __forceinline__ uint8_t mx4_block_bf16(const uint4* __restrict__ src,
+                                                  uint4* __restrict__ dst) {
+  float v[32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = src[q];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
+      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int e = mx4_scale_exp(amax);
+  const float inv = mx_inv_scale(e);
+  uint32_t packed[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t p = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p |= e2m1_code(__fmul_rn(v[8 * q + i], inv)) << (4 * i);
+    packed[q] = p;
+  }
+  dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  return (uint8_t)(e + 127);
+}
+
+template <bool kW4>
 __global__ void __launch_bounds__(256)
 mx_quantize_kernel(const uint4* __restrict__ src, int64_t nblocks, uint4* __restrict__ codes,
                    uint8_t* __restrict__ scales) {
   pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nblocks) return;
-  scales[i] = mx_block_bf16(src + i * 4, codes + i * 2);
+  scales[i] = kW4 ? mx4_block_bf16(src + i * 4, codes + i) : mx_block_bf16(src + i * 4, codes + i * 2);
 }
 
 // Packed scale offsets (bytes). Gate/up: a 512-byte block per (group, feature
@@ -81,12 +118,14 @@ __device__ __forceinline__ int64_t mx_packed_offset_down(int64_t g, int o, int b
 }
 
 // which: 0 W1, 1 W3 (rows NG*I, K = d), 2 W2 (rows NG*d, K = I).
+template <bool kW4>
 __global__ void __launch_bounds__(256)
 mx_pack_kernel(const uint4* __restrict__ src, int64_t nblocks, int which, int d, int I,
                uint4* __restrict__ codes, uint8_t* __restrict__ sf) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nblocks) return;
-  const uint8_t s = mx_block_bf16(src + i * 4, codes + i * 2);
+  const uint8_t s =
+      kW4 ? mx4_block_bf16(src + i * 4, codes + i) : mx_block_bf16(src + i * 4, codes + i * 2);
   const int K = which == 2 ? I : d;
   const int64_t row = i / (K / 32);
   const int b = (int)(i % (K / 32));
@@ -102,7 +141,16 @@ cudaError_t launch_mx_quantize(const void* src, int64_t rows, int64_t K, uint8_t
                                uint8_t* scales, cudaStream_t st) {
   const int64_t nb = rows * (K / 32);
   if (nb == 0) return cudaSuccess;
-  (void)launch_pdl(mx_quantize_kernel, dim3((unsigned)((nb + 255) / 256)), dim3(256), 0, st,
+  (void)launch_pdl(mx_quantize_kernel<false>, dim3((unsigned)((nb + 255) / 256)), dim3(256), 0, st,
+      static_cast<const uint4*>(src), nb, reinterpret_cast<uint4*>(codes), scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx4_quantize(const void* src, int64_t rows, int64_t K, uint8_t* codes,
+                                uint8_t* scales, cudaStream_t st) {
+  const int64_t nb = rows * (K / 32);
+  if (nb == 0) return cudaSuccess;
+  (void)launch_pdl(mx_quantize_kernel<true>, dim3((unsigned)((nb + 255) / 256)), dim3(256), 0, st,
       static_cast<const uint4*>(src), nb, reinterpret_cast<uint4*>(codes), scales);
   return cudaGetLastError();
 }
@@ -122,12 +170,13 @@ cudaError_t launch_mx_pack(const Resolved& r, const void* w1, const void* w3, co
   if (e != cudaSuccess) return e;
   const int64_t nb_up = NG * r.I * (r.d / 32), nb_dn = NG * r.d * (r.I / 32);
   const unsigned gu = (unsigned)((nb_up + 255) / 256), gd = (unsigned)((nb_dn + 255) / 256);
-  mx_pack_kernel<<<gu, 256, 0, st>>>(static_cast<const uint4*>(w1), nb_up, 0, r.d, r.I,
-                                     reinterpret_cast<uint4*>(w1q), sf_up);
-  mx_pack_kernel<<<gu, 256, 0, st>>>(static_cast<const uint4*>(w3), nb_up, 1, r.d, r.I,
-                                     reinterpret_cast<uint4*>(w3q), sf_up);
-  mx_pack_kernel<<<gd, 256, 0, st>>>(static_cast<const uint4*>(w2), nb_dn, 2, r.d, r.I,
-                                     reinterpret_cast<uint4*>(w2q), sf_down);
+  auto pack = r.w4 ? mx_pack_kernel<true> : mx_pack_kernel<false>;
+  pack<<<gu, 256, 0, st>>>(static_cast<const uint4*>(w1), nb_up, 0, r.d, r.I,
+                           reinterpret_cast<uint4*>(w1q), sf_up);
+  pack<<<gu, 256, 0, st>>>(static_cast<const uint4*>(w3), nb_up, 1, r.d, r.I,
+                           reinterpret_cast<uint4*>(w3q), sf_up);
+  pack<<<gd, 256, 0, st>>>(static_cast<const uint4*>(w2), nb_dn, 2, r.d, r.I,
+                           reinterpret_cast<uint4*>(w2q), sf_down);
   return cudaGetLastError();
 }
 

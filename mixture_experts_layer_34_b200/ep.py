@@ -133,7 +133,7 @@ class ExpertParallelMoE:
             if w.shape[0] != n_slots:
                 raise ValueError(f"local stack has {w.shape[0]} slots, expected {n_slots}")
         self.w_gate, self.bias = w_gate, bias
-        self.mxfp8 = cfg.dtype == K.KT_DTYPE_MXFP8
+        self.mxfp8 = cfg.dtype in (K.KT_DTYPE_MXFP8, K.KT_DTYPE_MXFP4)   # block-scaled weights
         if self.mxfp8:
             self.q = K.pack_mxfp8_local(cfg, 0, n_local, w1, w3, w2)
             self.w1 = self.w3 = self.w2 = None

@@ -25,7 +25,7 @@ KT_ERR_INVALID_CONFIG, KT_ERR_NULL, KT_ERR_WORKSPACE, KT_ERR_ALIGN = -1, -2, -3,
 KT_ERR_CUDA, KT_ERR_TIMEOUT, KT_ERR_UNSUPPORTED, KT_ERR_SCRATCH_LIMIT = -5, -6, -7, -8
 KT_ERR_BOUNDS = -9
 KT_STATIC_SCRATCH_BYTES = 32 << 20
-KT_DTYPE_F32, KT_DTYPE_BF16, KT_DTYPE_MXFP8 = 0, 1, 2
+KT_DTYPE_F32, KT_DTYPE_BF16, KT_DTYPE_MXFP8, KT_DTYPE_MXFP4 = 0, 1, 2, 3
 
 # Every symbol include/ktmoe.h declares.
 EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_forward",
@@ -37,7 +37,8 @@ EXPORTS = ("kt_moe_validate", "kt_moe_workspace_size", "kt_moe_gate", "kt_moe_fo
            "kt_moe_mxfp8_pack", "kt_moe_forward_mxfp8", "kt_moe_graph_create_mxfp8",
            "kt_moe_forward_local", "kt_moe_forward_local_mxfp8", "kt_moe_ep_finish",
            "kt_moe_mxfp8_scale_bytes_local", "kt_moe_mxfp8_pack_local", "kt_moe_forward_placed",
-           "kt_moe_forward_placed_mxfp8", "kt_moe_selftest_timeout", "kt_moe_checked_build")
+           "kt_moe_forward_placed_mxfp8", "kt_moe_selftest_timeout", "kt_moe_checked_build",
+           "kt_moe_mxfp4_quantize")
 
 
 class kt_moe_config(ctypes.Structure):
@@ -121,6 +122,8 @@ def lib() -> ctypes.CDLL:
             L.kt_moe_graph_destroy.restype = None
             L.kt_moe_mxfp8_quantize.argtypes = [I64, I64, P, P, P, P]
             L.kt_moe_mxfp8_quantize.restype = ctypes.c_int
+            L.kt_moe_mxfp4_quantize.argtypes = [I64, I64, P, P, P, P]
+            L.kt_moe_mxfp4_quantize.restype = ctypes.c_int
             L.kt_moe_mxfp8_scale_bytes.argtypes = [CP, ctypes.c_int]
             L.kt_moe_mxfp8_scale_bytes.restype = ctypes.c_size_t
             L.kt_moe_mxfp8_pack.argtypes = [CP, P, P, P, P, P, P, P, P, P]
@@ -312,6 +315,21 @@ def kt_moe_mxfp8_quantize(rows, K, src, codes, scales, stream=None):
         raise KtMoeError("kt_moe_mxfp8_quantize", rc)
 
 
+def kt_moe_mxfp4_quantize(rows, K, src, codes, scales, stream=None):
+    """bf16 [rows, K] -> packed E2M1 codes [rows, K/2] and scale bytes [rows, K/32]."""
+    rc = lib().kt_moe_mxfp4_quantize(int(rows), int(K), _ptr(src), _ptr(codes), _ptr(scales),
+                                     _stream(stream))
+    if rc != KT_OK:
+        raise KtMoeError("kt_moe_mxfp4_quantize", rc)
+
+
+def _code_shape(cfg, shape) -> tuple:
+    """Shape of the weight codes: one byte per element (MXFP8), or two 4-bit
+    codes per byte along K (MXFP4)."""
+    shape = tuple(shape)
+    return shape[:-1] + (shape[-1] // 2,) if cfg.dtype == KT_DTYPE_MXFP4 else shape
+
+
 def kt_moe_mxfp8_scale_bytes(cfg: kt_moe_config, down: bool) -> int:
     return int(lib().kt_moe_mxfp8_scale_bytes(ctypes.byref(cfg), int(bool(down))))
 
@@ -324,12 +342,13 @@ def kt_moe_mxfp8_pack(cfg, w1, w3, w2, w1q, w3q, w2q, sf_up, sf_down, stream=Non
 
 
 def pack_mxfp8(cfg, w1, w3, w2, stream=None) -> dict:
-    """Allocate the MXFP8 codes (W1 and W3 as the two halves of one buffer) and
-    the packed scales for bf16 weights, and pack them."""
+    """Allocate the MXFP8 (or, for an MXFP4 config, packed 4-bit) codes (W1 and
+    W3 as the two halves of one buffer) and the packed scales for bf16 weights,
+    and pack them."""
     import torch
-    w13 = torch.empty((2,) + tuple(w1.shape), dtype=torch.uint8, device=w1.device)
+    w13 = torch.empty((2,) + _code_shape(cfg, w1.shape), dtype=torch.uint8, device=w1.device)
     out = dict(w1q=w13[0], w3q=w13[1],      # W1's codes below W3's, as the forward needs
-               w2q=torch.empty(w2.shape, dtype=torch.uint8, device=w2.device),
+               w2q=torch.empty(_code_shape(cfg, w2.shape), dtype=torch.uint8, device=w2.device),
                sf_up=torch.empty(kt_moe_mxfp8_scale_bytes(cfg, False), dtype=torch.uint8,
                                  device=w1.device),
                sf_down=torch.empty(kt_moe_mxfp8_scale_bytes(cfg, True), dtype=torch.uint8,
@@ -439,10 +458,10 @@ def pack_mxfp8_local(cfg, expert_begin, expert_end, w1, w3, w2, stream=None) -> 
     """pack_mxfp8 for one rank's local stacks (routed experts [expert_begin,
     expert_end), then the shared ones)."""
     import torch
-    w13 = torch.empty((2,) + tuple(w1.shape), dtype=torch.uint8, device=w1.device)
+    w13 = torch.empty((2,) + _code_shape(cfg, w1.shape), dtype=torch.uint8, device=w1.device)
     sb = lambda down: kt_moe_mxfp8_scale_bytes_local(cfg, expert_begin, expert_end, down)
     out = dict(w1q=w13[0], w3q=w13[1],
-               w2q=torch.empty(w2.shape, dtype=torch.uint8, device=w2.device),
+               w2q=torch.empty(_code_shape(cfg, w2.shape), dtype=torch.uint8, device=w2.device),
                sf_up=torch.empty(sb(False), dtype=torch.uint8, device=w1.device),
                sf_down=torch.empty(sb(True), dtype=torch.uint8, device=w1.device))
     kt_moe_mxfp8_pack_local(cfg, expert_begin, expert_end, w1, w3, w2, out["w1q"], out["w3q"],
@@ -509,7 +528,8 @@ def kt_moe_checked_build() -> bool:
 
 def config_for(layer, y_fp32: bool = False) -> kt_moe_config:
     """kt_moe_config of a workloads.LayerConfig."""
-    dt = {"f32": KT_DTYPE_F32, "bf16": KT_DTYPE_BF16, "mxfp8": KT_DTYPE_MXFP8}[layer.dtype]
+    dt = {"f32": KT_DTYPE_F32, "bf16": KT_DTYPE_BF16, "mxfp8": KT_DTYPE_MXFP8,
+          "mxfp4": KT_DTYPE_MXFP4}[layer.dtype]
     return make_config(dtype=dt, y_fp32=int(y_fp32), **layer.kernel_fields())
 
 

@@ -59,7 +59,8 @@ class LayerConfig:
     route_scale: float
     norm_topk: int          # -1 auto (renormalise iff sigmoid), 0, 1
     group_score: int        # 0 auto, 1 amax, 2 top-2 sum
-    dtype: str              # "f32", "bf16" or "mxfp8" (bf16 tokens, MXFP8 expert weights)
+    dtype: str              # "f32", "bf16", "mxfp8" or "mxfp4" (bf16 tokens, MXFP8 / MXFP4
+                            # expert weights)
     bias: str               # "none", "normal", "zipf"
     seed: int
     init: str = "std002"    # "std002" or "fan_in"
@@ -201,6 +202,13 @@ LIMITS = [
                 bias="normal", seed=2406),
 ]
 BY_NAME.update({c.name: c for c in LIMITS})
+
+# MXFP4-expert forms: every MXFP8 layer above with its expert weights packed to
+# MXFP4 instead (E2M1 codes, two per byte, and a scale per 32), from the same
+# seeded bf16 weights; tokens and hidden rows stay MXFP8.
+MXFP4 = [c.with_(name=c.name.replace("_mxfp8", "_mxfp4"), dtype="mxfp4")
+         for c in MXFP8 + [BY_NAME["limits_E512_k32_S8_mxfp8"]]]
+BY_NAME.update({c.name: c for c in MXFP4})
 
 
 def torch_dtype(cfg: LayerConfig) -> torch.dtype:

@@ -79,7 +79,8 @@ BAD = [
     dict(topk_groups=5), dict(n_groups=1, topk_groups=2), dict(topk=0),
     dict(topk=9),                                                         # > TG * E/G = 8
     dict(n_shared=-1), dict(n_shared=9), dict(route_scale=0.0), dict(route_scale=float("inf")),
-    dict(route_scale=float("nan")), dict(score_func=2), dict(dtype=3), dict(dim=12),
+    dict(route_scale=float("nan")), dict(score_func=2), dict(dtype=4), dict(dim=12),
+    dict(dtype=2, dim=192), dict(dtype=3, inter=64),                     # MX: multiples of 128
     dict(inter=4), dict(norm_topk=2), dict(group_score=3), dict(add_residual=2), dict(y_fp32=2),
     dict(n_experts=16, n_groups=16, topk_groups=4, topk=4, group_score=2),  # top-2 of 1 expert
 ]
@@ -330,3 +331,45 @@ def test_no_device_reports_cuda_error():
     ptrs = [x.data_ptr()] * 6 + [y.data_ptr()] + [0, 0]
     rc = _call_forward(cfg, 64, ptrs, ws_ptr, n)
     assert rc in (K.KT_ERR_CUDA, K.KT_ERR_UNSUPPORTED)
+
+
+def test_mxfp4_host_side_errors():
+    """MXFP4 configs: dims must be multiples of 128; the packed 4-bit codes need
+    32-byte alignment (their tensor maps); the quantize entry checks K, NULLs
+    and alignment. Fake pointers, rejected on the host."""
+    cfg4 = K.config_for(W.BY_NAME["small_sig_bias_mxfp4"])
+    assert cfg4.dtype == K.KT_DTYPE_MXFP4
+    assert K.kt_moe_validate(cfg4, 300, True) == K.KT_OK
+    fields = {f: getattr(cfg4, f) for f, _ in K.kt_moe_config._fields_}
+    assert K.kt_moe_validate(K.make_config(**{**fields, "dim": 448}), 300, True) == \
+        K.KT_ERR_INVALID_CONFIG
+    assert K.kt_moe_validate(K.make_config(**{**fields, "dtype": 4}), 300, True) == \
+        K.KT_ERR_INVALID_CONFIG
+    # Scale sizes are the MXFP8 ones (same layout).
+    cfg8 = K.config_for(W.BY_NAME["small_sig_bias_mxfp8"])
+    for down in (False, True):
+        assert K.kt_moe_mxfp8_scale_bytes(cfg4, down) == K.kt_moe_mxfp8_scale_bytes(cfg8, down) > 0
+    L = K.lib()
+    T = 300
+    need = K.kt_moe_workspace_size(cfg4, T)
+    V = ctypes.c_void_p
+    x, wg, bias, y = 0x100000, 0x200000, 0x300000, 0x400000
+    w1q, w3q, w2q, sfu, sfd = 0x1000000, 0x1800000, 0x2000000, 0x2800000, 0x3000000
+    ws = 0x7000000
+
+    def fwd(c, a1, a3, a2):
+        return L.kt_moe_forward_mxfp8(ctypes.byref(c), T, V(x), V(wg), V(bias), V(a1), V(a3),
+                                      V(a2), V(sfu), V(sfd), V(y), None, None, V(ws), need, None,
+                                      None)
+    assert fwd(cfg4, w1q + 16, w3q + 16, w2q) == K.KT_ERR_ALIGN     # 16 but not 32 bytes
+    assert fwd(cfg4, w1q, w3q + 16, w2q) == K.KT_ERR_ALIGN
+    assert fwd(cfg4, w1q, w3q, w2q + 16) == K.KT_ERR_ALIGN
+    assert fwd(cfg4, w3q, w1q, w2q) == K.KT_ERR_INVALID_CONFIG      # W3's codes below W1's
+    # The same offsets pass the 8-bit checks (16-byte alignment suffices there);
+    # without a GPU the call then fails at the first CUDA call instead.
+    if not torch.cuda.is_available():
+        assert fwd(cfg8, w1q + 16, w3q + 16, w2q) in (K.KT_ERR_CUDA, K.KT_ERR_UNSUPPORTED)
+    q = L.kt_moe_mxfp4_quantize
+    assert q(4, 48, V(x), V(w1q), V(sfu), None) == K.KT_ERR_INVALID_CONFIG
+    assert q(4, 64, None, V(w1q), V(sfu), None) == K.KT_ERR_NULL
+    assert q(4, 64, V(x + 8), V(w1q), V(sfu), None) == K.KT_ERR_ALIGN

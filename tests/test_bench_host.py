@@ -82,3 +82,14 @@ def test_dump_and_replay_flags():
     a = bench.parse_args(["--dump", "/tmp/d"])
     assert a.dump == "/tmp/d" and a.replay is None
     assert bench.parse_args(["--replay", "/tmp/d/x"]).replay == "/tmp/d/x"
+
+
+def test_algorithmic_mxfp4_weight_bytes():
+    layer = W.BY_NAME["small_sig_bias_mxfp4"]
+    idx = np.tile(np.arange(4, dtype=np.int32), (layer.T, 1))
+    w = bench.algorithmic(layer, idx)
+    # half a byte per weight (two E2M1 codes per byte) plus one scale byte per 32
+    per_expert = 3 * layer.dim * layer.inter * (0.5 + 1 / 32)
+    tok = layer.n_experts * layer.dim * 2 + 2 * layer.T * layer.dim * 2
+    assert w["bytes_layer"] == pytest.approx(5 * per_expert + tok)
+    assert bench.parse_args(["--no-mxfp4"]).no_mxfp4

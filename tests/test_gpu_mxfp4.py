@@ -1,0 +1,225 @@
+"""MXFP4 expert weights on the GPU, through the C ABI, against the oracle.
+
+Quantisation (kt_moe_mxfp4_quantize, and kt_moe_mxfp8_pack with an MXFP4
+config) is integer work decided by the same rule on both sides from the same
+bf16 inputs: codes (unpacked from their nibbles, element 2i in the low nibble of
+byte i) and scales must be bit-exact, the scales in the packed layout the header
+documents (the MXFP8 layout).
+
+The forward is compared with the oracle's 4-bit forward, which quantises the
+same bf16 weights by the same rule (identical codes) and runs the MXFP8 literal
+loop on them in double (tokens and hidden rows in E4M3, as on the GPU). What
+differs is what differs in the 8-bit form: fp32 accumulation on the tensor
+cores, and hidden codes that can sit one E4M3 step apart at a rounding
+boundary. The bound is the same: max|dy| <= 2e-2 * RMS(y_ref) on the fp32
+output, with the bf16 output exactly its rounding.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.oracle as O
+from mixture_experts_layer_34_b200 import ep
+from mixture_experts_layer_34_b200 import ktmoe as K
+from mixture_experts_layer_34_b200 import workloads as W
+
+from parity import oracle_gate, routing_agreement
+from test_gpu_mxfp8 import _unpack_scales
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+def _unpack_codes(packed: np.ndarray) -> np.ndarray:
+    """[..., K/2] bytes -> [..., K] codes, element 2i from the low nibble."""
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = packed & 0xF
+    out[..., 1::2] = packed >> 4
+    return out
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (37, 256), (300, 7168), (2048, 2048)])
+def test_quantize_is_bit_exact(rows, cols):
+    g = torch.Generator().manual_seed(rows * cols + 4)
+    a = torch.randn(rows, cols, generator=g) * torch.exp2(torch.randint(-20, 20, (rows, 1),
+                                                                        generator=g).float())
+    a[0, :32] = 0.0                       # an all-zero block
+    if rows > 1:
+        a[1, :16] = 6.0                   # a block whose maximum is exactly representable
+        a[1, 32:64] = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -5.0] * 4)  # ties
+    a = a.to(torch.bfloat16)
+    codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(rows, cols // 32, dtype=torch.uint8, device="cuda")
+    K.kt_moe_mxfp4_quantize(rows, cols, a.cuda(), codes, scales)
+    torch.cuda.synchronize()
+    oc, os_ = O.mx4_quantize(a)
+    assert np.array_equal(_unpack_codes(codes.cpu().numpy()), oc)
+    assert np.array_equal(scales.cpu().numpy(), os_)
+
+
+@pytest.mark.parametrize("name", ["small_sig_bias_mxfp4", "small_softmax_mxfp4"])
+def test_pack_is_bit_exact_in_the_documented_layout(name):
+    layer = W.BY_NAME[name]
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer)
+    q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+    torch.cuda.synchronize()
+    assert q["w1q"].shape[-1] == layer.dim // 2 and q["w2q"].shape[-1] == layer.inter // 2
+    up = _unpack_scales(q["sf_up"], layer, False)
+    dn = _unpack_scales(q["sf_down"], layer, True)
+    for e in range(layer.n_experts + layer.n_shared):
+        for which, key in ((0, "w1"), (1, "w3")):
+            oc, os_ = O.mx4_quantize(inp[key][e].cpu())
+            assert np.array_equal(_unpack_codes(q[key + "q"][e].cpu().numpy()), oc), (e, key)
+            assert np.array_equal(up[which, e], os_), (e, key)
+        oc, os_ = O.mx4_quantize(inp["w2"][e].cpu())
+        assert np.array_equal(_unpack_codes(q["w2q"][e].cpu().numpy()), oc), e
+        assert np.array_equal(dn[e], os_), e
+
+
+def _forward(layer, inp, q, y_fp32, ws=None):
+    T = layer.T
+    cfg = K.config_for(layer, y_fp32=y_fp32)
+    ws = K.alloc_workspace(cfg, T) if ws is None else ws
+    y = torch.full((T, layer.dim), float("nan"), device="cuda",
+                   dtype=torch.float32 if y_fp32 else torch.bfloat16)
+    idx = torch.empty((T, layer.topk), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, layer.topk), dtype=torch.float32, device="cuda")
+    K.kt_moe_forward_mxfp8(cfg, T, inp["x"], inp["w_gate"], inp["bias"], q["w1q"], q["w3q"],
+                           q["w2q"], q["sf_up"], q["sf_down"], y, idx, w, ws)
+    assert K.kt_moe_check(ws) == K.KT_OK
+    return y, idx, w
+
+
+def _oracle_y(layer, inp, og, toks):
+    E, S = layer.n_experts, layer.n_shared
+    need = set(range(E, E + S))
+    for t in toks:
+        need.update(int(e) for e in og["idx"][t])
+    qw = {e: tuple(O.mx4_quantize(inp[k][e].cpu()) for k in ("w1", "w3", "w2")) for e in need}
+    pick = lambda j: [qw[e][j] if e in qw else None for e in range(E + S)]
+    return O.forward_mxfp4(layer.kernel_fields(), inp["x"].cpu(), og["idx"], og["w"], pick(0),
+                           pick(1), pick(2), toks, inp["bias"] is not None)
+
+
+def _check(layer, toks):
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer)
+    q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+    y32, idx, w = _forward(layer, inp, q, True)
+    y16, idx16, _ = _forward(layer, inp, q, False)
+    assert torch.equal(idx, idx16)
+    assert torch.equal(y16, y32.to(torch.bfloat16)), "bf16 y is not round(fp32 y)"
+    og = oracle_gate(layer, inp)
+    diff, near = routing_agreement(layer, og, idx.cpu().numpy())
+    assert near[diff].all(), f"routing differs away from near ties: {diff[~near[diff]]}"
+    keep = [t for t in toks if t not in set(diff.tolist())]
+    y_ref = _oracle_y(layer, inp, og, keep)
+    yg = y32[torch.as_tensor(keep, device="cuda")].cpu().numpy()
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    err = float(np.abs(yg - y_ref).max())
+    print(f"{layer.name}: max|dy| / RMS = {err / rms:.3e} over {len(keep)} tokens")
+    assert err <= TOL * rms
+    return inp, q, y32
+
+
+@pytest.mark.parametrize("name", ["small_sig_bias_mxfp4", "small_softmax_mxfp4"])
+def test_small_layers_every_token(name):
+    layer = W.BY_NAME[name]
+    _check(layer, list(range(layer.T)))
+
+
+def test_limits_every_token():
+    layer = W.BY_NAME["limits_E512_k32_S8_mxfp4"]
+    _check(layer, list(range(layer.T)))
+
+
+def test_v3_decode_every_token():
+    layer = W.BY_NAME["v3_decode_T8_mxfp4"]
+    _check(layer, list(range(layer.T)))
+
+
+def test_v3_prefill_sampled_tokens():
+    layer = W.BY_NAME["v3_prefill_T8192_zipf_mxfp4"]
+    rng = np.random.default_rng(18)
+    toks = sorted(rng.choice(layer.T, 6, replace=False).tolist())
+    _check(layer, toks)
+
+
+def test_forward_is_deterministic_and_graph_equals_stream():
+    layer = W.BY_NAME["small_sig_bias_mxfp4"]
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer, y_fp32=True)
+    q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+    ws = K.alloc_workspace(cfg, layer.T)
+    a, idx, w = _forward(layer, inp, q, True, ws)
+    b, _, _ = _forward(layer, inp, q, True, ws)
+    assert torch.equal(a, b)
+    y = torch.full_like(a, float("nan"))
+    gr = K.KtMoeGraph.mxfp8(cfg, layer.T, inp["x"], inp["w_gate"], inp["bias"], q, y, idx, w, ws)
+    gr.launch()
+    gr.launch()
+    torch.cuda.synchronize()
+    gr.destroy()
+    assert K.kt_moe_check(ws) == K.KT_OK
+    assert torch.equal(y, a)
+
+
+def test_output_does_not_depend_on_workspace_contents():
+    layer = W.BY_NAME["small_softmax_mxfp4"]
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer, y_fp32=True)
+    q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+    outs = []
+    for fill in (0x00, 0xFF):
+        ws = K.alloc_workspace(cfg, layer.T)
+        ws.fill_(fill)
+        y, _, _ = _forward(layer, inp, q, True, ws)
+        outs.append(y)
+    assert not torch.isnan(outs[1]).any()
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_tokens_with_distinct_scales():
+    layer = W.BY_NAME["small_softmax_mxfp4"]
+    inp = W.make_layer(layer, "cuda")
+    sc = torch.exp2((torch.arange(layer.T) % 7 - 3).float()).cuda()
+    inp["x"] = (inp["x"].float() * sc[:, None]).to(torch.bfloat16)
+    q = K.pack_mxfp8(K.config_for(layer), inp["w1"], inp["w3"], inp["w2"])
+    y32, idx, _ = _forward(layer, inp, q, True)
+    og = oracle_gate(layer, inp)
+    diff, near = routing_agreement(layer, og, idx.cpu().numpy())
+    assert near[diff].all()
+    toks = [t for t in range(0, layer.T, 3) if t not in set(diff.tolist())]
+    y_ref = _oracle_y(layer, inp, og, toks)
+    yg = y32[torch.as_tensor(toks, device="cuda")].cpu().numpy()
+    for i, t in enumerate(toks):
+        rms = float(np.sqrt(np.mean(y_ref[i] ** 2)))
+        assert np.abs(yg[i] - y_ref[i]).max() <= TOL * rms, t
+
+
+def test_expert_parallel_ranks_sum_to_the_full_forward():
+    """Two ranks (contiguous experts, halves of the shared tokens), one after
+    the other on this GPU: the fp32 partials summed and finished equal the
+    single-GPU forward within 1e-4 of its RMS (only the fp32 sum order differs)."""
+    layer = W.BY_NAME["small_sig_bias_mxfp4"]
+    inp = W.make_layer(layer, "cuda")
+    cfg = K.config_for(layer, y_fp32=True)
+    q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+    full, _, _ = _forward(layer, inp, q, True)
+    total = torch.zeros((layer.T, layer.dim), device="cuda")
+    for rank in range(2):
+        m = ep.ExpertParallelMoE(cfg, inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"],
+                                 rank, 2)
+        part = torch.full((layer.T, layer.dim), float("nan"), device="cuda")
+        m.local(inp["x"], part)
+        ws, _ = m.buffers(layer.T, inp["x"].device)
+        assert K.kt_moe_check(ws) == K.KT_OK
+        total += part
+    y = torch.empty_like(full)
+    K.kt_moe_ep_finish(cfg, layer.T, total, inp["x"], y)
+    rms = float(full.pow(2).mean().sqrt())
+    assert float((y - full).abs().max()) <= 1e-4 * rms

@@ -1,7 +1,7 @@
 """bench.py --dump / --replay on the GPU: a dumped step reruns bit for bit.
 
-A short bench run on a small layer (bf16 and its MXFP8 form) dumps each step's
-inputs and outputs; --replay redraws the expert weights from the seed, checks
+A short bench run on a small layer (bf16, MXFP8 and MXFP4 forms) dumps each
+step's inputs and outputs; --replay redraws the expert weights from the seed, checks
 the weight probe, reruns the forward on the dumped tokens and must reproduce
 the routing and y exactly (the forward is deterministic: fixed sum orders, no
 atomics in the arithmetic).
@@ -33,7 +33,8 @@ def test_dump_then_replay_is_bit_exact(tmp_path):
               "--dump", d])
     assert r.returncode == 0, r.stderr[-4000:]
     steps = sorted(os.listdir(d))
-    assert steps == ["small_sig_bias_mxfp8_rank0", "small_sig_bias_rank0"], steps
+    assert steps == ["small_sig_bias_mxfp4_rank0", "small_sig_bias_mxfp8_rank0",
+                     "small_sig_bias_rank0"], steps
     for s in steps:
         files = set(os.listdir(os.path.join(d, s)))
         assert {"x.npy", "w_gate.npy", "bias.npy", "idx.npy", "w.npy", "y.npy", "w_probe.npy",
