@@ -31,7 +31,7 @@ CASES = ["small_sig_bias", "small_softmax_ragged", "small_odd_dims", "small_amax
          "small_fp32_groups", "small_sig_bias_mxfp8", "limits_E512_k32_S8", "limits_T1",
          "limits_k_equals_E", "limits_one_expert", "limits_E512_k32_S8_f32",
          "limits_E512_k32_S8_mxfp8", "v3_shape_T2048_E32_profile",
-         "v3_shape_T2048_E32_profile_mxfp8"]
+         "v3_shape_T2048_E32_profile_mxfp8", "small_sig_bias_mxfp4", "limits_E512_k32_S8_mxfp4"]
 EP_CASES = ["small_sig_bias", "limits_E512_k32_S8"]
 
 
@@ -80,7 +80,7 @@ def run_cases() -> dict:
         layer = W.BY_NAME[name]
         inp = W.make_layer(layer, "cuda")
         q = None
-        if layer.dtype == "mxfp8":
+        if layer.dtype in ("mxfp8", "mxfp4"):
             q = K.pack_mxfp8(K.config_for(layer), inp["w1"], inp["w3"], inp["w2"])
         for y_fp32 in (True, False):
             for key, v in _forward(layer, inp, q, y_fp32).items():
