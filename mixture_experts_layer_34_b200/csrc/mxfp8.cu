@@ -96,7 +96,8 @@ mx_quantize_kernel(const uint4* __restrict__ src, int64_t nblocks, uint4* __rest
   pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nblocks) return;
-  scales[i] = kW4 ? mx4_block_bf16(src + i * 4, codes + i) : mx_block_bf16(src + i * 4, codes + i * 2);
+  scales[i] =
+      kW4 ? mx4_block_bf16(src + i * 4, codes + i) : mx_block_bf16(src + i * 4, codes + i * 2);
 }
 
 // Packed scale offsets (bytes). Gate/up: a 512-byte block per (group, feature

@@ -107,7 +107,8 @@ def test_checked_build_matches_release_bit_for_bit(tmp_path):
     for key, v in release.items():
         if key.endswith("rc"):
             assert int(v) == K.KT_OK, (key, K.strerror(int(v)))
-            assert int(checked[key]) == K.KT_OK, (key, "checked build:", K.strerror(int(checked[key])))
+            rc = int(checked[key])
+            assert rc == K.KT_OK, (key, "checked build:", K.strerror(rc))
         else:
             assert torch.equal(checked[key], v), key
 
