@@ -771,6 +771,13 @@ def run_ours(a):
             "stage_ms": {k: round(v, 4) for k, v in pre["stage_ms"].items()},
             "routing": pre["routing"],
             "layer_tflops": round(pre["work"]["flops_layer"] / (pre["ms"] / K_ / 1e3) / 1e12, 1),
+            # The whole layer against both roofs (its algorithmic bytes over the HBM
+            # copy peak, its FLOPs over the sustained bf16 peak): the HBM-bound
+            # layers (few tokens per expert) are judged by the first.
+            "layer_hbm_frac": round(pre["work"]["bytes_layer"] / (pre["ms"] / K_ / 1e3) / 1e9
+                                    / peaks["hbm_gbs"], 4),
+            "layer_tensor_frac": round(pre["work"]["flops_layer"] / (pre["ms"] / K_ / 1e3) / 1e12
+                                       / peaks["bf16_tflops_sustained"], 4),
             # The gate/up GEMM runs inside back-to-back steps under the 1 kW power
             # cap, so its denominator is the sustained bf16 figure; the burst
             # fraction is given beside it.
