@@ -93,3 +93,25 @@ def test_algorithmic_mxfp4_weight_bytes():
     tok = layer.n_experts * layer.dim * 2 + 2 * layer.T * layer.dim * 2
     assert w["bytes_layer"] == pytest.approx(5 * per_expert + tok)
     assert bench.parse_args(["--no-mxfp4"]).no_mxfp4
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    """--impl reference on rank 0: one JSON line with the contract's keys, the
+    oracle timed on a sample of the workload (here a small layer, on the CPU)."""
+    import json
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    a = bench.parse_args(["--impl", "reference", "--workload", "small_sig_bias", "--steps", "1",
+                          "--warmup", "3"])
+    bench.run_reference(a)
+    lines = [x for x in capsys.readouterr().out.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "impl",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
+    assert d["config"]["workload"] == "small_sig_bias"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]

@@ -32,6 +32,16 @@ def test_dump_then_replay_is_bit_exact(tmp_path):
               "--no-cpu-baseline", "--steps", "2", "--warmup", "3", "--e2e-steps", "2",
               "--dump", d])
     assert r.returncode == 0, r.stderr[-4000:]
+    # The run's one JSON line carries the contract's keys.
+    line = json.loads([x for x in r.stdout.splitlines() if x.startswith("{")][-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "roofline", "e2e", "gpu_launches", "clocks", "layer_hbm_frac", "mxfp8", "mxfp4"):
+        assert key in line, key
+    assert line["value"] > 0 and line["config"]["workload"] == "small_sig_bias"
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in line["roofline"], key
+    assert line["e2e"]["h2d_bytes_per_step"] == 300 * 512 * 2
     steps = sorted(os.listdir(d))
     assert steps == ["small_sig_bias_mxfp4_rank0", "small_sig_bias_mxfp8_rank0",
                      "small_sig_bias_rank0"], steps
