@@ -131,7 +131,8 @@ struct GemmArgs {
   const int32_t* n_tiles;    // device count of tiles
   int* counter;              // device tile counter (zeroed before the launch), or null:
                              // then pair p takes tiles p, p + pairs, ...
-  int implicit_rows;         // > 0: logits; chunks of kChunkRows over this many token rows
+  int implicit_rows;         // > 0: logits; chunks of implicit_chunk over this many token rows
+  int implicit_chunk;        // logits: token rows per chunk (a multiple of 32, <= kChunkRows)
   int n_ftiles;              // feature tiles per group
   int rows_per_group;        // weight rows per group (I for up, d for down, E for logits)
   int K;                     // reduction length
@@ -437,10 +438,10 @@ __device__ __forceinline__ bool uniform_ok(bool v, int bar_id) {
 
 __device__ __forceinline__ void get_tile(const GemmArgs& a, int t, Chunk& ch, int& ft, int& ci) {
   if (a.implicit_rows > 0) {
+    const int c = a.implicit_chunk;
     ci = t / a.n_ftiles;
     ft = t % a.n_ftiles;
-    ch = Chunk{0, ci * kChunkRows, min(kChunkRows, a.implicit_rows - ci * kChunkRows),
-               ci * kChunkRows};
+    ch = Chunk{0, ci * c, min(c, a.implicit_rows - ci * c), ci * c};
   } else {
     const int2 e = a.tiles[t];
     ci = e.x;
@@ -534,9 +535,10 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
   // kernel parameters; the previous kernel's outputs are read after this.
   pdl_wait();
 
-  const int n_tiles = args.implicit_rows > 0
-                          ? ((args.implicit_rows + kChunkRows - 1) / kChunkRows) * args.n_ftiles
-                          : *args.n_tiles;
+  const int n_tiles =
+      args.implicit_rows > 0
+          ? ((args.implicit_rows + args.implicit_chunk - 1) / args.implicit_chunk) * args.n_ftiles
+          : *args.n_tiles;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;   // static schedule only
   // K slabs per tile (the last may run past K: TMA fills those columns with zeros).
   const int n_slabs = (args.K + KD::kSlabK - 1) / KD::kSlabK;
@@ -1357,7 +1359,14 @@ cudaError_t launch_gate_logits_tc(const Resolved& r, int64_t T, const void* x, c
   a.row_weight = nullptr;
   a.n_routed_rows = 0;
   a.err = err;
-  const int tiles = (int)((T + kChunkRows - 1) / kChunkRows) * a.n_ftiles;
+  // Token chunks of 256 rows, halved (down to 64) while twice the tiles still
+  // fit in one wave of CTA pairs: W_g is small and stays in L2, so narrower
+  // tiles cost little more traffic and spread the logits over more of the GPU.
+  const int64_t n_pairs = num_sms / 2;
+  int chunk = kChunkRows;
+  while (chunk > 64 && 2 * ((T + chunk - 1) / chunk) * a.n_ftiles <= n_pairs) chunk /= 2;
+  a.implicit_chunk = chunk;
+  const int tiles = (int)((T + chunk - 1) / chunk) * a.n_ftiles;
   return launch<kKindLogits>(M, a, pair_grid(num_sms, tiles), st);
 }
 
