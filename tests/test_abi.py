@@ -1,5 +1,5 @@
 """The C-ABI library: loads, exports what include/ktmoe.h declares, and rejects bad
-calls on the host before any CUDA call (CPU; safe on a GPU machine too)."""
+calls on the host before any CUDA call (CPU; also safe where a GPU is present)."""
 from __future__ import annotations
 
 import ctypes
