@@ -223,3 +223,11 @@ def test_expert_parallel_ranks_sum_to_the_full_forward():
     K.kt_moe_ep_finish(cfg, layer.T, total, inp["x"], y)
     rms = float(full.pow(2).mean().sqrt())
     assert float((y - full).abs().max()) <= 1e-4 * rms
+
+
+@pytest.mark.parametrize("T", [1, 17, 64, 65, 225])
+def test_token_counts_every_token(T):
+    """Token counts around the gate's split-K / tensor-core switch (64) and the
+    224-row MXFP8 chunk, each token against the oracle."""
+    layer = W.BY_NAME["small_sig_bias_mxfp4"].with_(name=f"small_sig_bias_mxfp4_T{T}", T=T)
+    _check(layer, list(range(T)))
