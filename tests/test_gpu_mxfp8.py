@@ -218,3 +218,11 @@ def test_tokens_with_distinct_scales():
     for i, t in enumerate(toks):
         rms = float(np.sqrt(np.mean(y_ref[i] ** 2)))
         assert np.abs(yg[i] - y_ref[i]).max() <= TOL * rms, t
+
+
+@pytest.mark.parametrize("T", [1, 17, 64, 65, 225])
+def test_token_counts_every_token(T):
+    """Token counts around the gate's split-K / tensor-core switch (64) and the
+    224-row MXFP8 chunk, each token against the oracle."""
+    layer = W.BY_NAME["small_sig_bias_mxfp8"].with_(name=f"small_sig_bias_mxfp8_T{T}", T=T)
+    _check(layer, list(range(T)))
