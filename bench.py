@@ -10,16 +10,25 @@ GPUs every rank runs its own replica on its own tokens (data parallel over
 tokens, no collective on the data path): weak scaling, timed on the device as
 the max over ranks.
 
-Rank 0 prints one JSON line. `value` is tokens/s of the whole job; `e2e` is the
+Rank 0 prints one JSON line. `value` is tokens/s of the whole job, timed over
+the forwards alone (stage times come from a separate pass of the same steps with
+events at the stage boundaries: `stage_ms`, `staged_ms_per_step`); `e2e` is the
 same metric with host buffers (pinned x copied in and y copied out every step,
 serial with the compute), `e2e_pipelined` the same copies overlapped with the
 neighbouring steps' compute on two copy streams; `roofline` is the dominant
-kernel (the gate/up expert GEMM) against the measured bf16 tensor peak
-(sustained: the GEMM runs inside back-to-back steps at the power cap);
-`routing` is the expert-load histogram summary and the near-tie count;
-`cpu_baseline` is the CPU oracle timed on a sample of the same workload on this
-host's cores; "mxfp8" and "mxfp4" repeat prefill and decode with MXFP8 and
-MXFP4 expert weights.
+kernel (the gate/up expert GEMM) and `roofline_down` the down GEMM, each against
+the measured bf16 burst peak matched to the median SM clock of the timed region
+(the burst figure when that median is within 5% of the maximum clock, else
+scaled by median / maximum; `peak_clock_mhz` is the clock used); `routing` is
+the expert-load summary and, from the CPU oracle's gate over all T tokens, how
+many tokens the GPU routed differently (and how many of those away from the
+oracle's near ties) and the oracle's own near-tie count; `parity` compares the
+outputs of the CPU leg's tokens with the oracle's (fp32 form and bf16 output);
+`cpu_baseline` is the CPU oracle timed on this host's cores (its gate on all T
+tokens plus its expert loop on a sample, extrapolated to T; the decode layer in
+full); "v2lite_T512" and "v2_T4096" time the V2-shaped layers the same way;
+"mxfp8" and "mxfp4" repeat prefill and decode with MXFP8 and MXFP4 expert
+weights.
 `--impl reference` times the oracle alone (rank 0 only) in the same JSON form.
 
 `--dump DIR` saves each timed step's inputs and outputs as .npy files under
@@ -72,6 +81,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=W.V3_PREFILL.name)
     ap.add_argument("--decode-workload", default=W.V3_DECODE.name, help="'none' to skip")
+    ap.add_argument("--extra-workloads", default="auto",
+                    help="comma-separated layers also timed (no graph, no CPU leg); 'auto' = "
+                         "the V2-Lite and V2 layers when --workload is the V3 prefill; 'none'")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall time of the CPU-oracle sample")
@@ -161,15 +173,27 @@ def load_peaks() -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples every 100 ms while the timed work runs."""
+    """nvidia-smi clock/throttle samples every 50 ms while the timed work runs.
+    mark(name) / unmark(name) bracket a timed region on the host clock; stop()
+    gives the run's summary and the median SM clock inside each region."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+             "timestamp")
+    PERIOD_MS = 50
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.windows = {}
+
+    def mark(self, name: str):
+        self.windows[name] = [time.time(), None]
+
+    def unmark(self, name: str):
+        if name in self.windows:
+            self.windows[name][1] = time.time()
 
     def start(self):
         try:
@@ -177,7 +201,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -204,8 +228,38 @@ class ClockSampler:
         loaded = [s for s, p in zip(sm, power) if p > 0.3 * max(power)] or sm
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": float(rows[0][2]),
-                "reasons": reasons, "samples": len(rows)}
+        out = {"sm_mhz": statistics.median(loaded), "sm_max_mhz": float(rows[0][2]),
+               "reasons": reasons, "samples": len(rows)}
+        stamps = [_smi_time(r[9]) if len(r) > 9 else None for r in rows]
+        regions = {}
+        for name, (t0, t1) in self.windows.items():
+            if t1 is None:
+                continue
+            # samples taken inside the region, widened by one sampling period
+            pad = self.PERIOD_MS / 1e3
+            inside = [f for f, ts in zip(sm, stamps) if ts is not None and t0 - pad <= ts <= t1 + pad]
+            regions[name] = {"sm_mhz": statistics.median(inside) if inside else None,
+                             "samples": len(inside), "seconds": round(t1 - t0, 3)}
+        if regions:
+            out["regions"] = regions
+        return out
+
+
+def _smi_time(field: str):
+    """nvidia-smi's timestamp ("2026/12/02 16:43:10.123") as host epoch seconds."""
+    try:
+        return datetime.datetime.strptime(field.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+    except ValueError:
+        return None
+
+
+def clock_scaled_peak(burst: float, sm_mhz, sm_max_mhz) -> tuple[float, str]:
+    """The tensor peak that matches the SM clock a kernel ran at: the measured
+    burst figure when the median clock of its timed region is within 5% of the
+    maximum, else the burst figure scaled by median / maximum."""
+    if not sm_mhz or not sm_max_mhz or sm_mhz >= 0.95 * sm_max_mhz:
+        return burst, "burst (median SM clock within 5% of max)"
+    return burst * sm_mhz / sm_max_mhz, f"burst x {sm_mhz:.0f} / {sm_max_mhz:.0f} MHz"
 
 
 # ---------------------------------------------------------------------------
@@ -242,46 +296,13 @@ def algorithmic(layer, idx: np.ndarray) -> dict:
 ALLREDUCE_BUS_GBS = 725.0
 
 
-def routing_stats(layer, inp, idx: np.ndarray, dev) -> dict:
-    """Expert-load histogram summary of the timed routing, and the number of
-    near-tie tokens: those whose k-th and (k+1)-th selection keys, or TG-th and
-    (TG+1)-th group scores, differ by at most 1e-5 (from the library's scores,
-    kt_moe_scores, plus the bias, on the host)."""
-    from mixture_experts_layer_34_b200 import ktmoe as K
-    T, E, G, TG, k = layer.T, layer.n_experts, layer.n_groups, layer.topk_groups, layer.topk
-    cfg = K.config_for(layer)
-    ws = K.alloc_workspace(cfg, T, dev)
-    sc = torch.empty((T, E), dtype=torch.float32, device=dev)
-    K.kt_moe_scores(cfg, T, inp["x"], inp["w_gate"], sc, ws)
-    key = sc.cpu().numpy()
-    has_bias = inp["bias"] is not None
-    if has_bias:
-        key = (key + inp["bias"].float().cpu().numpy()[None, :]).astype(np.float32)
-    margin_g = np.full(T, np.inf, np.float32)
-    if G > 1:
-        gk = key.reshape(T, G, E // G)
-        top2 = layer.group_score == W.GROUP_TOP2SUM or (layer.group_score == W.GROUP_AUTO
-                                                       and has_bias)
-        if top2:
-            two = -np.sort(-gk, axis=2)[:, :, :2]
-            gsc = (two[:, :, 0] + two[:, :, 1]).astype(np.float32)
-        else:
-            gsc = gk.max(axis=2)
-        order = np.argsort(-gsc, axis=1, kind="stable")
-        gs_sorted = np.take_along_axis(gsc, order, axis=1)
-        margin_g = gs_sorted[:, TG - 1] - gs_sorted[:, TG]
-        keep = np.zeros((T, G), bool)
-        np.put_along_axis(keep, order[:, :TG], True, axis=1)
-        key = np.where(np.repeat(keep, E // G, axis=1), key, -np.inf)
-    ks = -np.sort(-key, axis=1)
-    margin_k = np.where(np.isfinite(ks[:, k]), ks[:, k - 1] - ks[:, k], np.inf)
-    near = (margin_k <= 1e-5) | (margin_g <= 1e-5)
-    load = np.bincount(idx.ravel(), minlength=E)
+def load_stats(layer, idx: np.ndarray) -> dict:
+    """Expert-load summary of the routing the timed forward produced."""
+    load = np.bincount(idx.ravel(), minlength=layer.n_experts)
     return {"load_max": int(load.max()), "load_mean": round(float(load.mean()), 2),
             "max_over_mean": round(float(load.max() / load.mean()), 2),
             "active_experts": int((load > 0).sum()), "zero_load_experts": int((load == 0).sum()),
-            "load_top8": np.sort(load)[::-1][:8].tolist(),
-            "near_tie_tokens": int(near.sum()), "near_tie_threshold": 1e-5}
+            "load_top8": np.sort(load)[::-1][:8].tolist()}
 
 
 def time_ep_ranks(layer, inp, dev, ranks, steps, warmup):
@@ -414,7 +435,14 @@ def time_ep_layer(layer, dev, rank, world, steps, warmup, placement_kind="balanc
     if rc != K.KT_OK:
         raise RuntimeError(f"device error in the expert-parallel steps: {K.strerror(rc)}")
     return max_over_ranks(t0.elapsed_time(t1), world, dev)
-def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False, dump=None):
+def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False, dump=None,
+               clocks=None, keep_y32=False):
+    """Time one layer: the plain forward (the headline loop: nothing but the
+    forwards between its two events), then a separate pass of the same steps
+    with stage events (stage_ms), optionally a CUDA-graph replay, and the
+    end-to-end loops with host buffers. keep_y32: also run one forward with an
+    fp32 output (the sum before its bf16 rounding) and return it with the bf16
+    output of the timed loop, for the comparison with the oracle."""
     from mixture_experts_layer_34_b200 import ktmoe as K
     inp = W.make_layer(layer, dev)
     if rank > 0:
@@ -436,16 +464,17 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False, d
         torch.cuda.empty_cache()
     args = (cfg, T, inp["x"], inp["w_gate"], inp["bias"], inp["w1"], inp["w3"], inp["w2"], y, idx, w, ws)
 
-    def fwd(x, events=None, y_out=None):
+    def fwd(x, events=None, y_out=None, c=None):
         yo = y if y_out is None else y_out
+        c = cfg if c is None else c
         if fp8:
-            K.kt_moe_forward_mxfp8(cfg, T, x, inp["w_gate"], inp["bias"], q["w1q"], q["w3q"],
+            K.kt_moe_forward_mxfp8(c, T, x, inp["w_gate"], inp["bias"], q["w1q"], q["w3q"],
                                    q["w2q"], q["sf_up"], q["sf_down"], yo, idx, w, ws,
                                    stage_events=events)
         elif events is not None:
-            K.kt_moe_forward_profiled(cfg, T, x, *args[3:8], yo, *args[9:], events)
+            K.kt_moe_forward_profiled(c, T, x, *args[3:8], yo, *args[9:], events)
         else:
-            K.kt_moe_forward(cfg, T, x, *args[3:8], yo, *args[9:])
+            K.kt_moe_forward(c, T, x, *args[3:8], yo, *args[9:])
 
     def save(rc):
         if dump:
@@ -459,30 +488,60 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False, d
         save(rc)
         raise RuntimeError(f"device error after warm-up: {K.strerror(rc)}")
 
-    # Stage events, created (recorded once) before the timed region.
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(K.KT_STAGE_EVENTS)]
-          for _ in range(steps)]
-    for row in ev:
-        for e in row:
-            e.record()
+    # The timed loop: the forwards alone, back to back on the launch stream.
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
+    if clocks:
+        clocks.mark(layer.name)
     t0.record()
     for s in range(steps):
-        fwd(inp["x"], ev[s])
+        fwd(inp["x"])
     t1.record()
     torch.cuda.synchronize()
+    if clocks:
+        clocks.unmark(layer.name)
     barrier(world)
     ms = t0.elapsed_time(t1)
     rc = K.kt_moe_check(ws)
     save(rc)
     if rc != K.KT_OK:
         raise RuntimeError(f"device error in the timed region: {K.strerror(rc)}")
+    ms_max = max_over_ranks(ms, world, dev)
+
+    # Stage times: the same number of steps again, right after, with events
+    # recorded on the launch stream at the stage boundaries (created and
+    # recorded once beforehand). Its total is reported beside the plain loop's.
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(K.KT_STAGE_EVENTS)]
+          for _ in range(steps)]
+    for row in ev:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark(layer.name + "/stages")
+    for s in range(steps):
+        fwd(inp["x"], ev[s])
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.unmark(layer.name + "/stages")
+    rc = K.kt_moe_check(ws)
+    if rc != K.KT_OK:
+        raise RuntimeError(f"device error in the stage pass: {K.strerror(rc)}")
     stage_ms = {name: statistics.fmean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps))
                 for i, name in enumerate(K.STAGES)}
-    ms_max = max_over_ranks(ms, world, dev)
+    staged_ms = statistics.fmean(ev[s][0].elapsed_time(ev[s][-1]) for s in range(steps))
+
+    # fp32-output forward (outside every timed region) for the oracle comparison.
+    y32 = y16 = None
+    if keep_y32:
+        y16 = y.clone()
+        y32 = torch.empty(y.shape, dtype=torch.float32, device=dev)
+        fwd(inp["x"], y_out=y32, c=K.config_for(layer, y_fp32=True))
+        rc = K.kt_moe_check(ws)
+        if rc != K.KT_OK:
+            raise RuntimeError(f"device error in the fp32-output forward: {K.strerror(rc)}")
 
     # The same forward replayed as one CUDA graph (kt_moe_graph_*), same buffers.
     graph_ms = None
@@ -575,10 +634,10 @@ def time_layer(layer, dev, rank, world, steps, warmup, e2e_steps, graph=False, d
         raise RuntimeError("pipelined forward differs from the plain one")
 
     work = algorithmic(layer, idx.cpu().numpy())
-    out = dict(inp=inp, idx=idx.cpu().numpy(), ms=ms_max, stage_ms=stage_ms, e2e_ms=e2e_ms,
-               e2e_pipe_ms=e2e_pipe_ms, graph_ms=graph_ms,
+    out = dict(inp=inp, idx=idx.cpu().numpy(), ms=ms_max, stage_ms=stage_ms, staged_ms=staged_ms,
+               e2e_ms=e2e_ms, e2e_pipe_ms=e2e_pipe_ms, graph_ms=graph_ms,
                work=work, h2d=inp["x"].numel() * inp["x"].element_size(),
-               d2h=y.numel() * y.element_size())
+               d2h=y.numel() * y.element_size(), y32=y32, y16=y16)
     del ws, y
     return out
 
@@ -666,38 +725,130 @@ def replay_step(path) -> dict:
             "match": probe_ok and rc == K.KT_OK and all(same.values())}
 
 
-def cpu_oracle_sample(layer, inp, idx_all, target_s: float) -> dict:
-    """Time the CPU oracle (gate + literal expert loop) on the first n tokens."""
+NEAR_TIE = 1e-5   # routing may differ from the oracle's only where its margins are this small
+
+
+def cpu_baseline_leg(layer, inp, res, target_s: float, full: bool = False) -> dict:
+    """The CPU oracle on this host's cores, on the timed workload's own inputs
+    (copied to the host outside every GPU timing), and what its results say
+    about the timed GPU run.
+
+    Timed: the oracle's gate on all T tokens, then its literal expert loop on
+    the first n tokens (n sized for about target_s seconds; all T if `full`).
+    value = T / (gate time + loop time x T / n): the whole layer at the two
+    measured rates (exactly the measured time when n = T).
+
+    Checked against the GPU run, from those oracle results: the routing of all
+    T tokens (how many differ from the oracle's, how many of those are not at
+    the oracle's near ties, and the oracle's own near-tie count: k-th and
+    (k+1)-th keys, or TG-th and (TG+1)-th group scores, within 1e-5), and the
+    outputs of the n tokens routed alike, as max|dy| / RMS(y_oracle) of the fp32
+    form and of the bf16 output."""
     import oracle.oracle as O
     kf = layer.kernel_fields()
     threads = O.num_threads()
+    T, E, S = layer.T, layer.n_experts, layer.n_shared
     x_h = inp["x"].cpu()
     wg_h = inp["w_gate"].cpu()
     bias = None if inp["bias"] is None else inp["bias"].float().cpu().numpy()
-    E, S = layer.n_experts, layer.n_shared
+    t = time.perf_counter()
+    g = O.gate(kf, x_h, wg_h, bias)
+    gate_s = time.perf_counter() - t
     host_w = {}
 
-    def run(n):
-        need = set(range(E, E + S)) | set(int(e) for e in idx_all[:n].ravel())
+    def loop(n):
+        need = set(range(E, E + S)) | set(int(e) for e in g["idx"][:n].ravel())
         for e in need - set(host_w):
             host_w[e] = (inp["w1"][e].cpu(), inp["w3"][e].cpu(), inp["w2"][e].cpu())
-        w1 = [host_w[e][0] if e in host_w else None for e in range(E + S)]
-        w3 = [host_w[e][1] if e in host_w else None for e in range(E + S)]
-        w2 = [host_w[e][2] if e in host_w else None for e in range(E + S)]
-        xs = x_h[:n].contiguous()
+        pick = lambda j: [host_w[e][j] if e in host_w else None for e in range(E + S)]
         t = time.perf_counter()
-        g = O.gate(kf, xs, wg_h, bias)
-        O.forward(kf, xs, g["idx"], g["w"], w1, w3, w2, range(n), bias is not None)
-        return time.perf_counter() - t
+        y = O.forward(kf, x_h, g["idx"], g["w"], pick(0), pick(1), pick(2), range(n),
+                      bias is not None)
+        return y, time.perf_counter() - t
 
-    n = max(1, min(layer.T, threads))
-    dt = run(n)
-    if dt < 0.5 * target_s and n < layer.T:
-        n = int(min(layer.T, max(n + 1, n * target_s / max(dt, 1e-3)), 64 * threads))
-        dt = run(n)
-    return {"value": n / dt, "unit": "tokens/s", "cores": min(threads, n), "kind": "oracle",
-            "sample": f"first {n} tokens of {layer.name}: fp64 gate + literal expert loop "
-                      f"({dt:.1f} s)"}
+    n = T if full else max(1, min(T, threads))
+    y_ref, loop_s = loop(n)
+    if not full and loop_s < 0.5 * target_s and n < T:
+        n = int(min(T, max(n + 1, n * target_s / max(loop_s, 1e-3)), 64 * threads))
+        y_ref, loop_s = loop(n)
+    total_s = gate_s + loop_s * T / n
+    what = (f"all {T} tokens" if n == T else
+            f"gate on all {T} tokens ({gate_s:.2f} s) + expert loop on the first {n} "
+            f"({loop_s:.2f} s), extrapolated to T")
+    cpu = {"value": T / total_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"{layer.name}: {what}; fp64 oracle", "gate_s": round(gate_s, 3),
+           "loop_tokens": n, "loop_s": round(loop_s, 3)}
+
+    idx_gpu = res["idx"]
+    diff = np.where((g["idx"] != idx_gpu).any(1))[0]
+    near = (g["kth_margin"] <= NEAR_TIE) | (g["grp_margin"] <= NEAR_TIE)
+    routing = {"tokens": T, "differ_from_oracle": int(len(diff)),
+               "differ_away_from_near_ties": int((~near[diff]).sum()),
+               "oracle_near_tie_tokens": int(near.sum()), "near_tie_threshold": NEAR_TIE}
+    parity = None
+    if res.get("y32") is not None:
+        keep = np.setdiff1d(np.arange(n), diff)
+        rms = float(np.sqrt(np.mean(y_ref[keep] ** 2)))
+        sel = torch.as_tensor(keep, device=res["y32"].device)
+        d32 = float(np.abs(res["y32"][sel].cpu().numpy() - y_ref[keep]).max())
+        d16 = float(np.abs(res["y16"][sel].float().cpu().numpy() - y_ref[keep]).max())
+        parity = {"tokens": int(len(keep)), "max_abs_dy_over_rms_fp32": round(d32 / rms, 6),
+                  "max_abs_dy_over_rms_bf16_output": round(d16 / rms, 6),
+                  "bound": 1e-4 if layer.dtype == "f32" else 2e-2,
+                  "note": "first tokens of the timed workload routed alike, against the fp64 "
+                          "oracle; fp32 form = the sum before its bf16 rounding"}
+    return {"cpu_baseline": cpu, "routing": routing, "parity": parity}
+
+
+def layer_fracs(layer, res, steps, peaks, clk_mhz, clk_max) -> dict:
+    """A layer's throughput against both roofs: its algorithmic bytes over the
+    HBM copy peak and its FLOPs over the clock-matched bf16 tensor peak."""
+    ms = res["ms"] / steps
+    tpk, _ = clock_scaled_peak(peaks["bf16_tflops"], clk_mhz, clk_max)
+    return {"layer_tflops": round(res["work"]["flops_layer"] / (ms / 1e3) / 1e12, 1),
+            "layer_hbm_gbs": round(res["work"]["bytes_layer"] / (ms / 1e3) / 1e9, 1),
+            "layer_hbm_frac": round(res["work"]["bytes_layer"] / (ms / 1e3) / 1e9
+                                    / peaks["hbm_gbs"], 4),
+            "layer_tensor_frac": round(res["work"]["flops_layer"] / (ms / 1e3) / 1e12 / tpk, 4)}
+
+
+def region_clock(clk: dict, name: str):
+    """Median SM clock inside a timed region, else of the whole run."""
+    reg = (clk.get("regions") or {}).get(name) or {}
+    return reg.get("sm_mhz") or clk.get("sm_mhz"), clk.get("sm_max_mhz")
+
+
+def tensor_roofline(kernel, flops, ms, peaks, clk, region, mult=1.0, traffic_bytes=None,
+                    dtype_note="bf16") -> dict:
+    """Roofline entry of a tensor-bound kernel: its algorithmic FLOPs over its
+    mean event-timed duration, against the measured burst peak (x mult for
+    another dtype) matched to the median SM clock of its timed region."""
+    f, fmax = region_clock(clk, region)
+    peak, rule = clock_scaled_peak(peaks["bf16_tflops"] * mult, f, fmax)
+    ach = flops / (ms / 1e3) / 1e12
+    return {"kernel": kernel, "bound": "tensor", "achieved": round(ach, 1),
+            "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+            "traffic": traffic_bytes,
+            "peak_source": f"{peaks['source']} {dtype_note} burst"
+                           + (f" x {mult:g} (nominal dtype ratio)" if mult != 1.0 else "")
+                           + f"; {rule}",
+            "peak_clock_mhz": f, "sm_max_mhz": fmax,
+            "frac_of_sustained": round(ach / (peaks["bf16_tflops_sustained"] * mult), 4)}
+
+
+def hbm_roofline(kernel, nbytes, ms, peaks, traffic_bytes=None) -> dict:
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"kernel": kernel, "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic_bytes,
+            "peak_source": peaks["source"] + " HBM copy"}
+
+
+def extra_workloads(a) -> list:
+    if a.extra_workloads == "none":
+        return []
+    if a.extra_workloads == "auto":
+        return [W.V2_LITE.name, W.V2.name] if a.workload == W.V3_PREFILL.name else []
+    return [n for n in a.extra_workloads.split(",") if n]
 
 
 def run_ours(a):
@@ -714,19 +865,27 @@ def run_ours(a):
 
     if world > 1 and a.parallel == "ep":
         return run_ep(a, layer, dev, rank, world, local, peaks)
+    cpu_leg = rank == 0 and world == 1 and not a.no_cpu_baseline
     clocks = ClockSampler(local)
     clocks.start()
-    pre = time_layer(layer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, dump=a.dump)
+    pre = time_layer(layer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, dump=a.dump,
+                     clocks=clocks, keep_y32=cpu_leg)
     epr = None
     if world == 1 and a.ep_ranks > 1:
         epr = time_ep_ranks(layer, pre["inp"], dev, a.ep_ranks, a.steps, a.warmup)
-    pre["routing"] = routing_stats(layer, pre["inp"], pre["idx"], dev)
     dec = None
     if a.decode_workload != "none":
         dlayer = W.BY_NAME[a.decode_workload]
         dec = time_layer(dlayer, dev, rank, world, a.steps, a.warmup, a.e2e_steps, graph=True,
-                         dump=a.dump)
-        dec["routing"] = routing_stats(dlayer, dec["inp"], dec["idx"], dev)
+                         dump=a.dump, clocks=clocks, keep_y32=cpu_leg)
+    # The other named layers (V2-Lite one prefill chunk, V2), timed the same way.
+    extra = {}
+    for name in extra_workloads(a):
+        res = time_layer(W.BY_NAME[name], dev, rank, world, a.steps, a.warmup, a.e2e_steps,
+                         dump=a.dump, clocks=clocks)
+        res.pop("inp")
+        torch.cuda.empty_cache()
+        extra[name] = res
     # The same layers with MXFP8 and MXFP4 expert weights (same shapes, seeds and
     # tokens).
     mx = {}
@@ -737,14 +896,19 @@ def run_ours(a):
             name = base + "_" + fmt
             if name in W.BY_NAME:
                 res = time_layer(W.BY_NAME[name], dev, rank, world, a.steps, a.warmup,
-                                 a.e2e_steps, graph=key == "decode", dump=a.dump)
+                                 a.e2e_steps, graph=key == "decode", dump=a.dump, clocks=clocks)
                 res.pop("inp")
                 mx.setdefault(fmt, {})[key] = (W.BY_NAME[name], res)
     clk = clocks.stop()
 
-    cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = cpu_oracle_sample(layer, pre["inp"], pre["idx"], a.cpu_seconds)
+    # CPU baseline leg: the oracle on the host (rank 0, one GPU), after every GPU
+    # timing; its results also check the timed runs' routing and outputs.
+    leg = dleg = None
+    if cpu_leg:
+        leg = cpu_baseline_leg(layer, pre["inp"], pre, a.cpu_seconds)
+        if dec:
+            dleg = cpu_baseline_leg(W.BY_NAME[a.decode_workload], dec["inp"], dec, a.cpu_seconds,
+                                    full=True)
     pre.pop("inp")
     if dec:
         dec.pop("inp")
@@ -754,8 +918,11 @@ def run_ours(a):
         T, K_ = layer.T, a.steps
         tokens = world * T * K_
         value = tokens / (pre["ms"] / 1e3)
+        fl = layer_fracs(layer, pre, K_, peaks, *region_clock(clk, layer.name))
         up_ms = pre["stage_ms"]["up_gemm"]
-        achieved = pre["work"]["flops_up"] / (up_ms / 1e3) / 1e12
+        routing = load_stats(layer, pre["idx"])
+        if leg:
+            routing["oracle"] = leg["routing"]
         line = {
             "metric": "MoE layer tokens/s (prefill T=8192, decode T=8) + % of HBM/tensor roofline",
             "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K_,
@@ -766,28 +933,18 @@ def run_ours(a):
             "config": {"workload": layer.name, "T": T, "dim": layer.dim, "experts": layer.n_experts,
                        "groups": f"{layer.n_groups}/{layer.topk_groups}", "topk": layer.topk,
                        "shared": layer.n_shared, "inter": layer.inter,
-                       "load": "Zipf(1.1)", "parallelism": f"dp{world} (replicas, no collective)",
+                       "load": "Zipf(1.1)" if layer.bias == "zipf" else "seeded gate",
+                       "parallelism": f"dp{world} (replicas, no collective)",
                        "l2": "inputs larger than L2: ~22 GB of expert weights read per step"},
+            # stage_ms: a separate pass of the same steps with stage events;
+            # staged_ms_per_step is that pass's step time.
             "stage_ms": {k: round(v, 4) for k, v in pre["stage_ms"].items()},
-            "routing": pre["routing"],
-            "layer_tflops": round(pre["work"]["flops_layer"] / (pre["ms"] / K_ / 1e3) / 1e12, 1),
-            # The whole layer against both roofs (its algorithmic bytes over the HBM
-            # copy peak, its FLOPs over the sustained bf16 peak): the HBM-bound
-            # layers (few tokens per expert) are judged by the first.
-            "layer_hbm_frac": round(pre["work"]["bytes_layer"] / (pre["ms"] / K_ / 1e3) / 1e9
-                                    / peaks["hbm_gbs"], 4),
-            "layer_tensor_frac": round(pre["work"]["flops_layer"] / (pre["ms"] / K_ / 1e3) / 1e12
-                                       / peaks["bf16_tflops_sustained"], 4),
-            # The gate/up GEMM runs inside back-to-back steps under the 1 kW power
-            # cap, so its denominator is the sustained bf16 figure; the burst
-            # fraction is given beside it.
-            "roofline": {"kernel": "grouped gate/up GEMM (tcgen05)", "bound": "tensor",
-                         "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
-                         "unit": "TFLOP/s",
-                         "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
-                         "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
-                         "traffic": traffic("up", layer.name),
-                         "peak_source": peaks["source"] + " (sustained)"},
+            "staged_ms_per_step": round(pre["staged_ms"], 4),
+            "routing": routing,
+            **fl,
+            "roofline": tensor_roofline("grouped gate/up GEMM (tcgen05)",
+                                        pre["work"]["flops_up"], up_ms, peaks, clk, layer.name,
+                                        traffic_bytes=traffic("up", layer.name)),
             "e2e": {"value": round(world * T * a.e2e_steps / (pre["e2e_ms"] / 1e3), 1),
                     "unit": "tokens/s", "h2d_bytes_per_step": pre["h2d"],
                     "d2h_bytes_per_step": pre["d2h"]},
@@ -797,74 +954,92 @@ def run_ours(a):
                               "unit": "tokens/s", "h2d_bytes_per_step": pre["h2d"],
                               "d2h_bytes_per_step": pre["d2h"]},
             "gpu_launches": LAUNCHES_PER_FORWARD * K_,
-            "cpu_baseline": cpu,
+            "cpu_baseline": leg["cpu_baseline"] if leg else None,
+            "parity": leg["parity"] if leg else None,
             "clocks": clk,
         }
+        line["roofline_down"] = tensor_roofline("grouped down GEMM (tcgen05)",
+                                                pre["work"]["flops_down"],
+                                                pre["stage_ms"]["down_gemm"], peaks, clk,
+                                                layer.name,
+                                                traffic_bytes=traffic("down", layer.name))
         if dec:
             dl = W.BY_NAME[a.decode_workload]
             dms = dec["ms"] / a.steps
-            up_bytes = dec["work"]["bytes_up"]
-            up_gbs = up_bytes / (dec["stage_ms"]["up_gemm"] / 1e3) / 1e9
-            layer_gbs = dec["work"]["bytes_layer"] / (dms / 1e3) / 1e9
+            droute = load_stats(dl, dec["idx"])
+            if dleg:
+                droute["oracle"] = dleg["routing"]
             line["decode"] = {
                 "workload": dl.name, "value": round(world * dl.T / (dms / 1e3), 1),
                 "unit": "tokens/s", "ms_per_step": round(dms, 4),
                 "active_experts": dec["work"]["active_experts"],
-                "routing": dec["routing"],
+                "routing": droute,
                 "stage_ms": {k: round(v, 4) for k, v in dec["stage_ms"].items()},
-                "layer_hbm_gbs": round(layer_gbs, 1),
-                "layer_hbm_frac": round(layer_gbs / peaks["hbm_gbs"], 4),
-                "roofline": {"kernel": "grouped gate/up GEMM (tcgen05)", "bound": "hbm",
-                             "achieved": round(up_gbs, 1), "peak": peaks["hbm_gbs"],
-                             "unit": "GB/s", "frac": round(up_gbs / peaks["hbm_gbs"], 4),
-                             "traffic": traffic("up", dl.name)},
+                **layer_fracs(dl, dec, a.steps, peaks, *region_clock(clk, dl.name)),
+                "roofline": hbm_roofline("grouped gate/up GEMM (tcgen05)", dec["work"]["bytes_up"],
+                                         dec["stage_ms"]["up_gemm"], peaks,
+                                         traffic("up", dl.name)),
                 "e2e": {"value": round(world * dl.T * a.e2e_steps / (dec["e2e_ms"] / 1e3), 1),
-                        "unit": "tokens/s"},
+                        "unit": "tokens/s", "h2d_bytes_per_step": dec["h2d"],
+                        "d2h_bytes_per_step": dec["d2h"]},
                 # the same steps replayed as one CUDA graph per step (kt_moe_graph_launch)
                 "graph": {"ms_per_step": round(dec["graph_ms"] / a.steps, 4),
                           "value": round(world * dl.T * a.steps / (dec["graph_ms"] / 1e3), 1),
                           "unit": "tokens/s"},
+                "cpu_baseline": dleg["cpu_baseline"] if dleg else None,
+                "parity": dleg["parity"] if dleg else None,
+            }
+        for name, res in extra.items():
+            xl = W.BY_NAME[name]
+            ms = res["ms"] / K_
+            f = layer_fracs(xl, res, K_, peaks, *region_clock(clk, name))
+            line[name] = {
+                "workload": name, "T": xl.T, "value": round(world * xl.T / (ms / 1e3), 1),
+                "unit": "tokens/s", "ms_per_step": round(ms, 4),
+                "stage_ms": {k: round(v, 4) for k, v in res["stage_ms"].items()},
+                **f,
+                "roofline": hbm_roofline("grouped gate/up GEMM (tcgen05)", res["work"]["bytes_up"],
+                                         res["stage_ms"]["up_gemm"], peaks, traffic("up", name)),
+                "roofline_tensor": tensor_roofline("grouped gate/up GEMM (tcgen05)",
+                                                   res["work"]["flops_up"],
+                                                   res["stage_ms"]["up_gemm"], peaks, clk, name),
+                "e2e": {"value": round(world * xl.T * a.e2e_steps / (res["e2e_ms"] / 1e3), 1),
+                        "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
+                        "d2h_bytes_per_step": res["d2h"]},
             }
         notes = {"mxfp8": "MXFP8 expert weights (E4M3, power-of-two scale per 32 along K); "
                           "bf16 tokens, gate and output",
                  "mxfp4": "MXFP4 expert weights (E2M1 codes two per byte, power-of-two scale "
                           "per 32 along K) against MXFP8 (E4M3) tokens and hidden rows; bf16 "
                           "gate and output"}
-        # Both block-scaled forms run tcgen05 kind::mxf8f6f4, whose dense rate is
-        # the FP8 one (E2M1 operands there do not run faster).
-        mx_peak = 2 * peaks["bf16_tflops_sustained"]
         for fmt, runs in mx.items():
             line[fmt] = {"note": notes[fmt]}
-            for key, (fl, res) in runs.items():
+            for key, (fl_, res) in runs.items():
                 ms = res["ms"] / K_
-                ent = {"workload": fl.name, "value": round(world * fl.T / (ms / 1e3), 1),
+                ent = {"workload": fl_.name, "value": round(world * fl_.T / (ms / 1e3), 1),
                        "unit": "tokens/s", "ms_per_step": round(ms, 4),
                        "stage_ms": {k: round(v, 4) for k, v in res["stage_ms"].items()},
-                       "e2e": {"value": round(world * fl.T * a.e2e_steps / (res["e2e_ms"] / 1e3), 1),
+                       "e2e": {"value": round(world * fl_.T * a.e2e_steps / (res["e2e_ms"] / 1e3), 1),
                                "unit": "tokens/s"}}
-                up_s = res["stage_ms"]["up_gemm"] / 1e3
+                up_ms_ = res["stage_ms"]["up_gemm"]
                 kern = ("grouped gate/up GEMM (tcgen05 kind::mxf8f6f4"
                         + (", E2M1 x E4M3)" if fmt == "mxfp4" else ")"))
                 if key == "prefill":
-                    ach = res["work"]["flops_up"] / up_s / 1e12
-                    ent["roofline"] = {"kernel": kern, "bound": "tensor", "achieved": round(ach, 1),
-                                       "peak": mx_peak, "unit": "TFLOP/s",
-                                       "frac": round(ach / mx_peak, 4),
-                                       "traffic": traffic("up", fl.name),
-                                       "peak_source": peaks["source"] + " bf16 (sustained) x 2, "
-                                                      "the nominal fp8 / bf16 ratio"}
+                    # Both block-scaled forms run tcgen05 kind::mxf8f6f4, whose
+                    # dense rate is the FP8 one (2x bf16; E2M1 operands there do
+                    # not run faster).
+                    ent["roofline"] = tensor_roofline(kern, res["work"]["flops_up"], up_ms_, peaks,
+                                                      clk, fl_.name, mult=2.0,
+                                                      traffic_bytes=traffic("up", fl_.name))
                 else:
-                    gbs = res["work"]["bytes_up"] / up_s / 1e9
                     lgbs = res["work"]["bytes_layer"] / (ms / 1e3) / 1e9
                     ent["layer_hbm_gbs"] = round(lgbs, 1)
                     ent["layer_hbm_frac"] = round(lgbs / peaks["hbm_gbs"], 4)
-                    ent["roofline"] = {"kernel": kern, "bound": "hbm", "achieved": round(gbs, 1),
-                                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                       "frac": round(gbs / peaks["hbm_gbs"], 4),
-                                       "traffic": traffic("up", fl.name)}
+                    ent["roofline"] = hbm_roofline(kern, res["work"]["bytes_up"], up_ms_, peaks,
+                                                   traffic("up", fl_.name))
                 if res.get("graph_ms") is not None:
                     ent["graph"] = {"ms_per_step": round(res["graph_ms"] / K_, 4),
-                                    "value": round(world * fl.T * K_ / (res["graph_ms"] / 1e3), 1),
+                                    "value": round(world * fl_.T * K_ / (res["graph_ms"] / 1e3), 1),
                                     "unit": "tokens/s"}
                 line[fmt][key] = ent
         if epr:

@@ -166,23 +166,29 @@ int kt_moe_forward_profiled(const kt_moe_config* cfg, int64_t T, const void* x,
  * counterpart on the pages: this entry point exists for the calling code, not
  * for the method.
  *
- * Some callers cannot call cudaMalloc or any allocator: code that runs while a
- * stream is being captured into a CUDA graph (an allocation there breaks the
- * capture), engines whose device memory is entirely owned by their own pool,
- * and plugin hosts that hand out no workspace. They pass only inputs and
- * outputs; the scratch comes from a fixed 32 MiB device array inside this
+ * Some callers cannot call cudaMalloc or any allocator: engines whose device
+ * memory is entirely owned by their own pool (an allocation behind the pool's
+ * back can fail once the pool holds the memory, or breaks its accounting),
+ * latency-critical loops where cudaMalloc and cudaFree would synchronise the
+ * device, and plugin hosts that hand out no workspace. They pass only inputs
+ * and outputs; the scratch comes from a fixed 32 MiB device array inside this
  * library (KT_STATIC_SCRATCH_BYTES), reserved on every GPU that loads the
  * library until the process exits. A call whose scratch need
  * (kt_moe_workspace_size) exceeds that returns KT_ERR_SCRATCH_LIMIT before
  * anything is enqueued — about 78 tokens of a DeepSeek-V3-shaped layer, so
- * decode-sized batches.
+ * decode-sized batches. This entry point allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
  *
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture. Every call on a device shares the one array, which keeps
- * the previous call's contents (each call resets what must start at zero);
- * calls whose work overlaps on the GPU — concurrent streams, or host threads
- * without ordering — race on it and must be serialised by the caller.
+ * Set-up: the first call on each device, with that device current, looks up
+ * the array's device address (cudaGetSymbolAddress) and does the library's
+ * other one-time host set-up for that device (the expert GEMMs' shared-memory
+ * limits, the tensor-map encoder); later calls only read the kept address. The
+ * address is kept for the life of the process: after a cudaDeviceReset of that
+ * device it is no longer valid, and this entry point must not be used again in
+ * that process. Every call on a device shares the one array, which keeps the
+ * previous call's contents (each call resets what must start at zero); calls
+ * whose work overlaps on the GPU — concurrent streams, or host threads without
+ * ordering — race on it and must be serialised by the caller.
  * Arguments, layouts, results and errors are otherwise those of
  * kt_moe_forward; kt_moe_check takes kt_moe_static_scratch() as its workspace.
  */

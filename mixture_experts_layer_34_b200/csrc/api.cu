@@ -429,6 +429,9 @@ std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the current device's scratch, looked up once per device.
+// The same first lookup also does the grouped GEMMs' one-time host set-up
+// (shared-memory limits of every kernel kind, the tensor-map encoder), so a
+// later call makes no such host call whatever its token count.
 void* static_scratch_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -436,6 +439,7 @@ void* static_scratch_ptr() {
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+    if (prepare_grouped_gemm() != cudaSuccess) return nullptr;
     g_scratch_ptr[dev] = p;
   }
   return g_scratch_ptr[dev];

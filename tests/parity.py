@@ -14,7 +14,49 @@ TOL_F32 = 1e-4      # same form, fp32 layers
 
 
 def tolerance(layer) -> float:
+    """The output bound by dtype. Block-scaled (MXFP8 / MXFP4) layers get the
+    bf16 form's bound here, for the tests that compare one output array only;
+    their main parity tests (mx_parity.check_forward) hold the hidden rows to
+    the oracle's codes and the outputs to 2e-4 of the RMS plus the effect of
+    the hidden codes that sit on a rounding boundary."""
     return TOL_F32 if layer.dtype == "f32" else TOL_BF16
+
+
+def coverage_tokens(idx: np.ndarray, n_experts: int, n_shared: int, chunk_rows: int,
+                    total: int = 512, n_heavy: int = 8, n_light: int = 8,
+                    seed: int = 0) -> list[int]:
+    """Tokens whose outputs reach every GEMM chunk position of the heavy experts.
+
+    The expert GEMMs take each expert's rows (its tokens in ascending order) in
+    chunks of `chunk_rows`. From the routing `idx` (the oracle's), pick one
+    random token from every chunk of the `n_heavy` most loaded experts and of the
+    shared experts (all T tokens in order), plus the last token of each of those
+    experts' final (partial) chunks, one token of each of the `n_light` least
+    loaded experts that have a token (all of those with at most four tokens), and
+    random tokens up to `total`."""
+    rng = np.random.default_rng(seed)
+    T = idx.shape[0]
+    load = np.bincount(idx.ravel(), minlength=n_experts)
+    pick: set[int] = set()
+
+    def cover(toks):
+        for c0 in range(0, len(toks), chunk_rows):
+            part = toks[c0:c0 + chunk_rows]
+            pick.add(int(part[rng.integers(len(part))]))
+        if len(toks):
+            pick.add(int(toks[-1]))
+
+    for e in np.argsort(-load, kind="stable")[:n_heavy]:
+        cover(np.where((idx == e).any(1))[0])
+    if n_shared:
+        cover(np.arange(T))
+    used = [e for e in np.argsort(load, kind="stable") if load[e] > 0]
+    for e in set(used[:n_light]) | {e for e in used if load[e] <= 4}:
+        pick.add(int(np.where((idx == e).any(1))[0][0]))
+    rest = np.setdiff1d(np.arange(T), np.fromiter(pick, np.int64))
+    need = max(0, min(total, T) - len(pick))
+    pick.update(int(t) for t in rng.choice(rest, min(need, len(rest)), replace=False))
+    return sorted(pick)
 
 
 def run_forward(layer, inp, T=None, ws=None, y_fp32=False):

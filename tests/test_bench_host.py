@@ -7,6 +7,7 @@ expert-parallel runs.
 """
 from __future__ import annotations
 
+import os
 import numpy as np
 import pytest
 
@@ -115,3 +116,77 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     assert d["config"]["workload"] == "small_sig_bias"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_clock_scaled_peak():
+    assert bench.clock_scaled_peak(1666.8, 1965.0, 1965.0)[0] == 1666.8
+    assert bench.clock_scaled_peak(1666.8, 1900.0, 1965.0)[0] == 1666.8     # within 5%
+    p, rule = bench.clock_scaled_peak(1666.8, 1335.0, 1965.0)
+    assert p == pytest.approx(1666.8 * 1335 / 1965) and "1335" in rule
+    assert bench.clock_scaled_peak(100.0, None, None)[0] == 100.0
+
+
+def test_smi_timestamps_parse_to_host_time():
+    import datetime
+    t = bench._smi_time("2026/12/02 16:43:10.250")
+    assert t == pytest.approx(datetime.datetime(2026, 12, 2, 16, 43, 10, 250000).timestamp())
+    assert bench._smi_time("[N/A]") is None
+
+
+def test_extra_workloads_flag():
+    assert bench.extra_workloads(bench.parse_args([])) == ["v2lite_T512", "v2_T4096"]
+    assert bench.extra_workloads(bench.parse_args(["--workload", "small_sig_bias"])) == []
+    assert bench.extra_workloads(bench.parse_args(["--extra-workloads", "none"])) == []
+    assert bench.extra_workloads(bench.parse_args(["--extra-workloads", "v2_T4096"])) == \
+        ["v2_T4096"]
+
+
+def test_cpu_leg_reports_routing_and_output_agreement():
+    """The CPU baseline leg's checks on a tiny layer, fed a 'GPU run' made from
+    the oracle itself with one token's routing changed and one output element
+    moved: exactly that token differs, and the moved element sets max|dy|."""
+    import torch
+    import oracle.oracle as O
+    layer = W.TINY
+    inp = W.make_layer(layer, "cpu")
+    kf = layer.kernel_fields()
+    g = O.gate(kf, inp["x"], inp["w_gate"], inp["bias"].numpy())
+    n = layer.n_experts + layer.n_shared
+    y = O.forward(kf, inp["x"], g["idx"], g["w"], [inp["w1"][e] for e in range(n)],
+                  [inp["w3"][e] for e in range(n)], [inp["w2"][e] for e in range(n)],
+                  range(layer.T), True)
+    idx = g["idx"].copy()
+    idx[5] = idx[5][::-1]                       # token 5 routed differently
+    y32 = torch.tensor(y, dtype=torch.float32)
+    rms = float(np.sqrt(np.mean(y ** 2)))
+    y32[7, 3] += 0.01 * rms
+    res = {"idx": idx, "y32": y32, "y16": y32.to(torch.bfloat16)}
+    out = bench.cpu_baseline_leg(layer, inp, res, target_s=0.1, full=True)
+    r = out["routing"]
+    assert r["tokens"] == layer.T and r["differ_from_oracle"] == 1
+    near5 = g["kth_margin"][5] <= 1e-5 or g["grp_margin"][5] <= 1e-5
+    assert r["differ_away_from_near_ties"] == (0 if near5 else 1)
+    p = out["parity"]
+    assert p["tokens"] == layer.T - 1
+    rms_keep = float(np.sqrt(np.mean(np.delete(y, 5, axis=0) ** 2)))
+    assert p["max_abs_dy_over_rms_fp32"] == pytest.approx(0.01 * rms / rms_keep, rel=1e-3)
+    cb = out["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["loop_tokens"] == layer.T and cb["value"] > 0
+
+
+def test_coverage_tokens_reach_every_chunk():
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    from parity import coverage_tokens
+    rng = np.random.default_rng(0)
+    T, E, k = 2000, 16, 2
+    # expert 0 in every token, expert 1 in 600, the rest random
+    idx = np.stack([np.zeros(T, np.int32), rng.integers(2, E, T).astype(np.int32)], 1)
+    idx[:600, 1] = 1
+    toks = coverage_tokens(idx, E, 1, 256, total=100, n_heavy=2, seed=3)
+    assert len(toks) == 100 and len(set(toks)) == 100
+    for e in (0, 1):
+        mine = np.where((idx == e).any(1))[0]
+        for c0 in range(0, len(mine), 256):
+            assert set(mine[c0:c0 + 256]) & set(toks), (e, c0)
+        assert mine[-1] in toks

@@ -1,10 +1,10 @@
 """kt_moe_forward_static: the layer forward without any caller allocation.
 
-Some callers cannot allocate device memory at all: code running while a stream
-is captured into a CUDA graph (an allocation would break the capture), engines
-whose device memory is entirely owned by their own pool, and plugin hosts that
-hand out no workspace. kt_moe_forward_static serves them with scratch from a
-fixed 32 MiB device array inside the library. These tests call it through the
+Some callers cannot allocate device memory at all: engines whose device memory
+is entirely owned by their own pool, latency-critical loops in which cudaMalloc
+and cudaFree would synchronise the device, and plugin hosts that hand out no
+workspace. kt_moe_forward_static serves them with scratch from a fixed 32 MiB
+device array inside the library. These tests call it through the
 C ABI and compare it with kt_moe_forward (caller workspace) on the same inputs,
 on two calls in a row, since the shared scratch keeps the previous call's
 contents; and they check that oversized calls are refused before any work.
