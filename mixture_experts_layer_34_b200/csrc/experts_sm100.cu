@@ -647,8 +647,10 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
         const int slabs = stage_slabs(hb);
         const int nk = (n_slabs + slabs - 1) / slabs;
         const uint32_t b_slab = hb * kBoxBytes;   // token-tile bytes of one slab
-        const CUtensorMap* a3 = &maps.a3[slabs == kSlabsLight ? 1 : 0];
-        const CUtensorMap* b3 = &maps.b3[src][slabs == kSlabsLight ? 4 : hb - 1];
+        // Maps of this tile's stage shape: 3-slab stages for one 32-row token
+        // block per CTA (hb == 1), else 2-slab stages of hb blocks.
+        const CUtensorMap* a3 = &maps.a3[hb == 1 ? 1 : 0];
+        const CUtensorMap* b3 = &maps.b3[src][hb == 1 ? 4 : hb - 1];
         for (int kb = 0; kb < nk; ++kb) {
           const int s0 = kb * slabs;
           const int valid = min(slabs, n_slabs - s0);
@@ -677,7 +679,7 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
               // token rows of the pair tile (1 KB per slab of the chunk's blocks),
               // as rows of 256 bytes.
               uint8_t* sS = sf_base + stage * kScaleStageBytes;
-              const int li = slabs == kSlabsLight ? 1 : 0;
+              const int li = hb == 1 ? 1 : 0;
               const int64_t ablk =
                   ((int64_t)(ch.group * args.n_ftiles_sf + ft) * 2 + rank) * args.n_kslabs + s0;
               tma_load_pair(sS, &maps.sfa[li], fbar, 0, (int)(2 * ablk), pol_a);

@@ -519,17 +519,21 @@ int oracle_mx_quantize(int64_t rows, int64_t K, int dtype, const void* src, uint
 int oracle_mx_dequantize(int64_t rows, int64_t K, const uint8_t* codes, const uint8_t* scales,
                          double* out) {
   if (K % 32 != 0) return -1;
+#pragma omp parallel for schedule(static)
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t i = 0; i < K; ++i) out[r * K + i] = mx_value(codes + r * K, scales + r * (K / 32), i);
   return 0;
 }
 
-// The literal forward ("MoE 前向四步") with MXFP8 expert weights: per token, u
-// is quantised (blocks of 32 along d); every expert computes, in double on the
-// dequantised values, h = silu(W1 u) * W3 u, quantises h (blocks of 32 along I;
-// skipped if quantize_hidden == 0) and returns W2 h. x is bf16 [T, d]. w1q/w3q
-// are per-expert code arrays [I, d] with scales [I, d/32]; w2q codes [d, I]
-// with scales [d, I/32]; E+S entries each (NULL where unused). y [n_tok, d].
+// The literal forward ("MoE 前向四步") with MXFP8 expert weights, in the page's
+// loop order: expert by expert (routed experts 0..E-1, then the shared ones),
+// each over the tokens that use it, y[token] += weight * expert(u). Per token, u
+// is quantised (blocks of 32 along d); an expert's weights are decoded once to
+// double, and each of its tokens computes h = silu(W1 u) * W3 u in double on the
+// dequantised values, quantises h (blocks of 32 along I; skipped if
+// quantize_hidden == 0) and adds weight * W2 h. x is bf16 [T, d]. w1q/w3q are
+// per-expert code arrays [I, d] with scales [I, d/32]; w2q codes [d, I] with
+// scales [d, I/32]; E+S entries each (NULL where unused). y [n_tok, d].
 int oracle_forward_mxfp8(const oracle_cfg* c, int64_t T, const void* x, const int32_t* idx,
                          const float* w, const uint8_t* const* w1q, const uint8_t* const* w1s,
                          const uint8_t* const* w3q, const uint8_t* const* w3s,
@@ -537,30 +541,55 @@ int oracle_forward_mxfp8(const oracle_cfg* c, int64_t T, const void* x, const in
                          int quantize_hidden, int64_t n_tok, const int64_t* tok_ids, double* y) {
   const int d = c->dim, I = c->inter, k = c->topk, E = c->n_experts, S = c->n_shared;
   if (d % 32 != 0 || I % 32 != 0) return -1;
-  int bad = 0;
-#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  // The users of each expert: (position in tok_ids, routing weight); the shared
+  // experts take every token with weight 1.
+  std::vector<std::vector<std::pair<int64_t, double>>> users(E + S);
   for (int64_t n = 0; n < n_tok; ++n) {
     const int64_t t = tok_ids[n];
-    if (t < 0 || t >= T) {
-      bad |= 1;
-      continue;
+    if (t < 0 || t >= T) return -1;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[t * k + j];
+      if (e < 0 || e >= E) return -1;
+      // (an expert named twice by one token contributes with both weights)
+      if (!users[e].empty() && users[e].back().first == n)
+        users[e].back().second += (double)w[t * k + j];
+      else
+        users[e].push_back({n, (double)w[t * k + j]});
     }
-    std::vector<double> u(d), uq(d), acc(d, 0.0), h(I), hq(I);
-    std::vector<uint8_t> cu(d), su(d / 32), ch(I), sh(I / 32);
-    for (int i = 0; i < d; ++i) u[i] = load_elem(x, 1, t * d + i);
-    mx_quantize_row(u.data(), d, cu.data(), su.data());
-    for (int i = 0; i < d; ++i) uq[i] = mx_value(cu.data(), su.data(), i);
-    auto run_expert = [&](int e, double weight) {
-      if (!w1q[e] || !w1s[e] || !w3q[e] || !w3s[e] || !w2q[e] || !w2s[e]) {
-        bad |= 1;
-        return;
-      }
+    for (int s = 0; s < S; ++s) users[E + s].push_back({n, 1.0});
+  }
+  // Quantised tokens.
+  std::vector<double> u((size_t)n_tok * d), uq((size_t)n_tok * d);
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < n_tok; ++n) {
+    std::vector<uint8_t> cu(d), su(d / 32);
+    for (int i = 0; i < d; ++i) u[n * d + i] = load_elem(x, 1, tok_ids[n] * d + i);
+    mx_quantize_row(&u[n * d], d, cu.data(), su.data());
+    for (int i = 0; i < d; ++i) uq[n * d + i] = mx_value(cu.data(), su.data(), i);
+  }
+  std::vector<double> acc((size_t)n_tok * d, 0.0);
+  std::vector<double> w1d((size_t)I * d), w3d((size_t)I * d), w2d((size_t)d * I);
+  for (int e = 0; e < E + S; ++e) {
+    if (users[e].empty()) continue;
+    if (!w1q[e] || !w1s[e] || !w3q[e] || !w3s[e] || !w2q[e] || !w2s[e]) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < (int64_t)I * d; ++j) {
+      w1d[j] = mx_value(w1q[e], w1s[e], j);
+      w3d[j] = mx_value(w3q[e], w3s[e], j);
+      w2d[j] = mx_value(w2q[e], w2s[e], j);
+    }
+    const auto& us = users[e];
+#pragma omp parallel for schedule(dynamic, 1)
+    for (size_t q = 0; q < us.size(); ++q) {
+      const int64_t n = us[q].first;
+      const double* un = &uq[n * d];
+      std::vector<double> h(I), hq(I);
+      std::vector<uint8_t> ch(I), sh(I / 32);
       for (int f = 0; f < I; ++f) {
         double g = 0.0, v = 0.0;
         for (int i = 0; i < d; ++i) {
-          const int64_t j = (int64_t)f * d + i;
-          g += mx_value(w1q[e], w1s[e], j) * uq[i];
-          v += mx_value(w3q[e], w3s[e], j) * uq[i];
+          g += w1d[(int64_t)f * d + i] * un[i];
+          v += w3d[(int64_t)f * d + i] * un[i];
         }
         h[f] = g / (1.0 + std::exp(-g)) * v;
       }
@@ -570,26 +599,20 @@ int oracle_forward_mxfp8(const oracle_cfg* c, int64_t T, const void* x, const in
       } else {
         hq = h;
       }
+      double* an = &acc[n * d];
       for (int o = 0; o < d; ++o) {
-        double s = 0.0;
-        for (int f = 0; f < I; ++f) s += mx_value(w2q[e], w2s[e], (int64_t)o * I + f) * hq[f];
-        acc[o] += weight * s;
+        double sum = 0.0;
+        for (int f = 0; f < I; ++f) sum += w2d[(int64_t)o * I + f] * hq[f];
+        an[o] += us[q].second * sum;
       }
-    };
-    for (int s = 0; s < S; ++s) run_expert(E + s, 1.0);
-    for (int j = 0; j < k; ++j) {
-      const int e = idx[t * k + j];
-      if (e < 0 || e >= E) {
-        bad |= 1;
-        continue;
-      }
-      run_expert(e, (double)w[t * k + j]);
     }
-    if (c->add_residual)
-      for (int i = 0; i < d; ++i) acc[i] += u[i];
-    std::copy(acc.begin(), acc.end(), y + n * d);
   }
-  return bad ? -1 : 0;
+  for (int64_t n = 0; n < n_tok; ++n) {
+    if (c->add_residual)
+      for (int i = 0; i < d; ++i) acc[n * d + i] += u[n * d + i];
+    std::copy(acc.begin() + n * d, acc.begin() + (n + 1) * d, y + n * d);
+  }
+  return 0;
 }
 
 }  // extern "C"
@@ -692,6 +715,7 @@ int oracle_mx4_quantize(int64_t rows, int64_t K, int dtype, const void* src, uin
 int oracle_mx4_dequantize(int64_t rows, int64_t K, const uint8_t* codes, const uint8_t* scales,
                           double* out) {
   if (K % 32 != 0) return -1;
+#pragma omp parallel for schedule(static)
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t i = 0; i < K; ++i)
       out[r * K + i] = std::ldexp(e2m1_to_double(codes[r * K + i]),

@@ -11,8 +11,9 @@ same bf16 weights by the same rule (identical codes) and runs the MXFP8 literal
 loop on them in double (tokens and hidden rows in E4M3, as on the GPU). What
 differs is what differs in the 8-bit form: fp32 accumulation on the tensor
 cores, and hidden codes that can sit one E4M3 step apart at a rounding
-boundary. The bound is the same: max|dy| <= 2e-2 * RMS(y_ref) on the fp32
-output, with the bf16 output exactly its rounding.
+boundary. The bound is the same as the 8-bit form's, set from those two
+differences with a margin: max|dy| <= 2e-3 * RMS(y_ref) on the fp32 output, with
+the bf16 output exactly its rounding.
 """
 from __future__ import annotations
 
@@ -25,12 +26,12 @@ from mixture_experts_layer_34_b200 import ep
 from mixture_experts_layer_34_b200 import ktmoe as K
 from mixture_experts_layer_34_b200 import workloads as W
 
-from parity import oracle_gate, routing_agreement
+import mx_parity as MX
+from parity import coverage_tokens, oracle_gate, routing_agreement
 from test_gpu_mxfp8 import _unpack_scales
 
 pytestmark = pytest.mark.gpu
 
-TOL = 2e-2
 
 
 def _unpack_codes(packed: np.ndarray) -> np.ndarray:
@@ -94,12 +95,19 @@ def _forward(layer, inp, q, y_fp32, ws=None):
     return y, idx, w
 
 
-def _oracle_y(layer, inp, og, toks):
+def _oracle_weights(layer, inp, og, toks):
+    """The oracle's MXFP4 (codes one per byte, scales) of W1, W3, W2 of every
+    expert the tokens use."""
     E, S = layer.n_experts, layer.n_shared
     need = set(range(E, E + S))
     for t in toks:
         need.update(int(e) for e in og["idx"][t])
-    qw = {e: tuple(O.mx4_quantize(inp[k][e].cpu()) for k in ("w1", "w3", "w2")) for e in need}
+    return {e: tuple(O.mx4_quantize(inp[k][e].cpu()) for k in ("w1", "w3", "w2")) for e in need}
+
+
+def _oracle_y(layer, inp, og, toks, qw=None):
+    E, S = layer.n_experts, layer.n_shared
+    qw = _oracle_weights(layer, inp, og, toks) if qw is None else qw
     pick = lambda j: [qw[e][j] if e in qw else None for e in range(E + S)]
     return O.forward_mxfp4(layer.kernel_fields(), inp["x"].cpu(), og["idx"], og["w"], pick(0),
                            pick(1), pick(2), toks, inp["bias"] is not None)
@@ -109,7 +117,9 @@ def _check(layer, toks):
     inp = W.make_layer(layer, "cuda")
     cfg = K.config_for(layer)
     q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
-    y32, idx, w = _forward(layer, inp, q, True)
+    cfg32 = K.config_for(layer, y_fp32=True)
+    ws = K.alloc_workspace(cfg32, layer.T)
+    y32, idx, w = _forward(layer, inp, q, True, ws)
     y16, idx16, _ = _forward(layer, inp, q, False)
     assert torch.equal(idx, idx16)
     assert torch.equal(y16, y32.to(torch.bfloat16)), "bf16 y is not round(fp32 y)"
@@ -117,12 +127,17 @@ def _check(layer, toks):
     diff, near = routing_agreement(layer, og, idx.cpu().numpy())
     assert near[diff].all(), f"routing differs away from near ties: {diff[~near[diff]]}"
     keep = [t for t in toks if t not in set(diff.tolist())]
-    y_ref = _oracle_y(layer, inp, og, keep)
-    yg = y32[torch.as_tensor(keep, device="cuda")].cpu().numpy()
+    qw = _oracle_weights(layer, inp, og, keep)
+    y_ref = _oracle_y(layer, inp, og, keep, qw)
+    st = MX.check_forward(layer, inp, y32, ws, og, keep, y_ref, qw, cfg32)
     rms = float(np.sqrt(np.mean(y_ref ** 2)))
-    err = float(np.abs(yg - y_ref).max())
-    print(f"{layer.name}: max|dy| / RMS = {err / rms:.3e} over {len(keep)} tokens")
-    assert err <= TOL * rms
+    err16 = float(np.abs(y16[torch.as_tensor(keep, device="cuda")].float().cpu().numpy()
+                         - y_ref).max())
+    print(f"{layer.name}: max|dy| / RMS = {st['max_rel']:.3e} (fp32 output; "
+          f"{st['max_rel_unexplained']:.3e} beyond the flip allowance), {err16 / rms:.3e} (bf16 "
+          f"output) over {len(keep)} tokens; hidden: {st['hidden_flips']} flips, "
+          f"{st['hidden_near']} near a boundary of {st['hidden_checked']}, "
+          f"{st['tokens_with_flips']} tokens with flips")
     return inp, q, y32
 
 
@@ -142,10 +157,14 @@ def test_v3_decode_every_token():
     _check(layer, list(range(layer.T)))
 
 
-def test_v3_prefill_sampled_tokens():
+def test_v3_prefill_chunk_coverage():
+    """At least 512 tokens: one from every 224-row GEMM chunk of the 8 heaviest
+    experts and of the shared expert (about 180 chunks), the last row of their
+    partial chunks, the lightest experts' tokens and random ones."""
     layer = W.BY_NAME["v3_prefill_T8192_zipf_mxfp4"]
-    rng = np.random.default_rng(18)
-    toks = sorted(rng.choice(layer.T, 6, replace=False).tolist())
+    og = oracle_gate(layer, W.make_gate_inputs(layer))
+    toks = coverage_tokens(og["idx"], layer.n_experts, layer.n_shared, 224, total=512, seed=18)
+    assert len(toks) >= 512
     _check(layer, toks)
 
 
@@ -184,21 +203,27 @@ def test_output_does_not_depend_on_workspace_contents():
 
 
 def test_tokens_with_distinct_scales():
+    """x ~ N(0,1) gives almost every 32-block the same exponent, which would hide
+    a kernel reading another token's scale; scaling token t by 2^(t mod 7 - 3)
+    makes every token's scales distinct. Hidden rows against the oracle's codes,
+    outputs within the two-part bound."""
     layer = W.BY_NAME["small_softmax_mxfp4"]
     inp = W.make_layer(layer, "cuda")
     sc = torch.exp2((torch.arange(layer.T) % 7 - 3).float()).cuda()
     inp["x"] = (inp["x"].float() * sc[:, None]).to(torch.bfloat16)
-    q = K.pack_mxfp8(K.config_for(layer), inp["w1"], inp["w3"], inp["w2"])
-    y32, idx, _ = _forward(layer, inp, q, True)
+    cfg = K.config_for(layer)
+    q = K.pack_mxfp8(cfg, inp["w1"], inp["w3"], inp["w2"])
+    cfg32 = K.config_for(layer, y_fp32=True)
+    ws = K.alloc_workspace(cfg32, layer.T)
+    y32, idx, _ = _forward(layer, inp, q, True, ws=ws)
     og = oracle_gate(layer, inp)
     diff, near = routing_agreement(layer, og, idx.cpu().numpy())
     assert near[diff].all()
     toks = [t for t in range(0, layer.T, 3) if t not in set(diff.tolist())]
-    y_ref = _oracle_y(layer, inp, og, toks)
-    yg = y32[torch.as_tensor(toks, device="cuda")].cpu().numpy()
-    for i, t in enumerate(toks):
-        rms = float(np.sqrt(np.mean(y_ref[i] ** 2)))
-        assert np.abs(yg[i] - y_ref[i]).max() <= TOL * rms, t
+    qw = _oracle_weights(layer, inp, og, toks)
+    y_ref = _oracle_y(layer, inp, og, toks, qw)
+    st = MX.check_forward(layer, inp, y32, ws, og, toks, y_ref, qw, cfg32)
+    print(f"{layer.name} distinct scales: {st}")
 
 
 def test_expert_parallel_ranks_sum_to_the_full_forward():
