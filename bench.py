@@ -800,11 +800,18 @@ def cpu_baseline_leg(layer, inp, res, target_s: float, full: bool = False) -> di
     return {"cpu_baseline": cpu, "routing": routing, "parity": parity}
 
 
+def tensor_mult(layer) -> float:
+    """Dense tensor rate of the layer's expert GEMMs relative to bf16: the
+    block-scaled forms run tcgen05 kind::mxf8f6f4 at the FP8 rate (nominally 2x;
+    E2M1 operands there do not run faster)."""
+    return 2.0 if layer.dtype in ("mxfp8", "mxfp4") else 1.0
+
+
 def layer_fracs(layer, res, steps, peaks, clk_mhz, clk_max) -> dict:
     """A layer's throughput against both roofs: its algorithmic bytes over the
-    HBM copy peak and its FLOPs over the clock-matched bf16 tensor peak."""
+    HBM copy peak and its FLOPs over the clock-matched tensor peak of its dtype."""
     ms = res["ms"] / steps
-    tpk, _ = clock_scaled_peak(peaks["bf16_tflops"], clk_mhz, clk_max)
+    tpk, _ = clock_scaled_peak(peaks["bf16_tflops"] * tensor_mult(layer), clk_mhz, clk_max)
     return {"layer_tflops": round(res["work"]["flops_layer"] / (ms / 1e3) / 1e12, 1),
             "layer_hbm_gbs": round(res["work"]["bytes_layer"] / (ms / 1e3) / 1e9, 1),
             "layer_hbm_frac": round(res["work"]["bytes_layer"] / (ms / 1e3) / 1e9
@@ -927,7 +934,8 @@ def run_ours(a):
             "metric": "MoE layer tokens/s (prefill T=8192, decode T=8) + % of HBM/tensor roofline",
             "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K_,
             "warmup": a.warmup, "ms_per_step": round(pre["ms"] / K_, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if layer.dtype == "bf16" else layer.dtype,
             "data": "synthetic (seeded; random-init weights of the V3 layer shape)",
             "impl": "ours",
             "config": {"workload": layer.name, "T": T, "dim": layer.dim, "experts": layer.n_experts,
@@ -944,6 +952,7 @@ def run_ours(a):
             **fl,
             "roofline": tensor_roofline("grouped gate/up GEMM (tcgen05)",
                                         pre["work"]["flops_up"], up_ms, peaks, clk, layer.name,
+                                        mult=tensor_mult(layer),
                                         traffic_bytes=traffic("up", layer.name)),
             "e2e": {"value": round(world * T * a.e2e_steps / (pre["e2e_ms"] / 1e3), 1),
                     "unit": "tokens/s", "h2d_bytes_per_step": pre["h2d"],
@@ -961,7 +970,7 @@ def run_ours(a):
         line["roofline_down"] = tensor_roofline("grouped down GEMM (tcgen05)",
                                                 pre["work"]["flops_down"],
                                                 pre["stage_ms"]["down_gemm"], peaks, clk,
-                                                layer.name,
+                                                layer.name, mult=tensor_mult(layer),
                                                 traffic_bytes=traffic("down", layer.name))
         if dec:
             dl = W.BY_NAME[a.decode_workload]

@@ -404,7 +404,10 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the fast reciprocal division (within 2 ulp;
+// the result is rounded to bf16 or quantised to E4M3 right after). For very
+// negative g the denominator overflows and the result is 0 (silu -> 0 there).
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ void st_cluster_s32(uint32_t caddr, int v) {
   asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
