@@ -479,7 +479,9 @@ int kt_moe_check(const void* workspace, void* stream);
  * in schedule order (feature tiles of 128 / 256 rows). */
 typedef struct {
   int64_t error_word;
-  int64_t logits;         /* fp32 [logits_splits][T][E]: partial sums over K, added in order */
+  int64_t logits;         /* fp32 [T][E] gate logits after the call (for T <= 64 the region
+                             holds logits_splits [T][E] slots of partial sums over K; the
+                             first is overwritten with their sum, added in order) */
   int64_t logits_splits;
   int64_t counts;
   int64_t offsets;

@@ -210,7 +210,7 @@ int kt_moe_gate(const kt_moe_config* cfg, int64_t T, const void* x, const void* 
   char* ws = static_cast<char*>(workspace);
   int* err = reinterpret_cast<int*>(ws + L.err);
   float* logits = reinterpret_cast<float*>(ws + L.logits);
-  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, kCallWords * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
   if (!scores_in && launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess)
     return KT_ERR_CUDA;
   if (launch_gate_select(r, T, logits, scores_in, bias, topk_idx, topk_w,
@@ -238,7 +238,7 @@ int kt_moe_scores(const kt_moe_config* cfg, int64_t T, const void* x, const void
   char* ws = static_cast<char*>(workspace);
   int* err = reinterpret_cast<int*>(ws + L.err);
   float* logits = reinterpret_cast<float*>(ws + L.logits);
-  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, kCallWords * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
   if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
   if (launch_gate_scores(r, T, logits, scores_out, st) != cudaSuccess) return KT_ERR_CUDA;
   return KT_OK;
@@ -360,7 +360,7 @@ int run_forward(const Resolved& r_in, const SlotTable& tab, int64_t T, const voi
     return true;
   };
   if (!mark(0)) return KT_ERR_CUDA;
-  if (cudaMemsetAsync(err, 0, 2 * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, kCallWords * sizeof(int), st) != cudaSuccess) return KT_ERR_CUDA;
   if (launch_gate_logits(r, T, x, w_gate, logits, err, sms, st) != cudaSuccess) return KT_ERR_CUDA;
   if (launch_gate_select(r, T, logits, nullptr, bias, idx, w,
                          reinterpret_cast<int32_t*>(ws + L.chunk_counts), err, st) != cudaSuccess)

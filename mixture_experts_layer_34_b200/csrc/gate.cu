@@ -127,15 +127,19 @@ gate_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg, float* __r
 // Logits for few tokens (T <= 64), split over K: CTA (eb, ks) computes the
 // partial dot products of 32 experts over the ks-th K range for all tokens
 // (one warp per 4 experts computed together, 16-byte loads along K split over
-// the lanes, 8 tokens at a time) and writes them to part[ks][t][e]. The selection kernel adds the
-// kSplitK partials in ks order, so the result does not depend on scheduling.
+// the lanes, 8 tokens at a time) and writes them to part[ks][t][e]. The last of
+// an expert block's kSplitK CTAs to finish (a counter in the workspace, zeroed
+// at the start of every call) adds the partials in ks order and writes the sum
+// over part[0]: the result does not depend on scheduling, and the selection
+// reads one value per logit.
 // ---------------------------------------------------------------------------
 constexpr int kSmallWarps = 8, kSmallTok = 8, kSplitK = kGateSplitK;
 
 template <typename T>
 __global__ void __launch_bounds__(kSmallWarps * 32)
 gate_logits_splitk_kernel(const T* __restrict__ x, const T* __restrict__ wg,
-                          float* __restrict__ part, int T_, int E, int d, int kc) {
+                          float* __restrict__ part, int T_, int E, int d, int kc,
+                          int* __restrict__ block_done) {
   pdl_wait();
   constexpr int VN = Vec16<T>::n, EW = 4;  // experts per warp, computed together
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -143,8 +147,7 @@ gate_logits_splitk_kernel(const T* __restrict__ x, const T* __restrict__ wg,
   const int k0 = ks * kc, k1 = min(d, k0 + kc);
   const int nc = k1 > k0 ? (k1 - k0) / VN : 0;
   const int e0 = blockIdx.x * 32 + warp * EW;
-  if (e0 >= E) return;
-  for (int t0 = 0; t0 < T_; t0 += kSmallTok) {
+  for (int t0 = 0; e0 < E && t0 < T_; t0 += kSmallTok) {
     float acc[EW][kSmallTok];
 #pragma unroll
     for (int ei = 0; ei < EW; ++ei)
@@ -184,6 +187,22 @@ gate_logits_splitk_kernel(const T* __restrict__ x, const T* __restrict__ wg,
           part[((int64_t)ks * T_ + t0 + j) * E + e0 + ei] = acc[ei][j];
       }
   }
+  // The last CTA of this expert block sums the partials.
+  __shared__ int last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&block_done[blockIdx.x], 1) == (int)gridDim.y - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const int eb0 = blockIdx.x * 32;
+  for (int i = threadIdx.x; i < T_ * 32; i += blockDim.x) {
+    const int t = i / 32, e = eb0 + i % 32;
+    if (e >= E) continue;
+    float sum = __ldcg(&part[(int64_t)t * E + e]);
+    for (int q = 1; q < (int)gridDim.y; ++q) sum += __ldcg(&part[((int64_t)q * T_ + t) * E + e]);
+    part[(int64_t)t * E + e] = sum;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -215,12 +234,11 @@ __device__ __forceinline__ Best warp_argmax(Best b) {
 }
 
 // Gate step 1 and the score function for token t, one warp: lane l gets the
-// scores of experts i * 32 + l in s[i]. `logits` holds `ksplit` partial sums
-// [ksplit][T][E], added in ks order; if `scores_in` is given it is used as is.
-// Lanes past E hold -inf (scores_in), 0 (sigmoid of -inf) or 0 (softmax).
+// scores of experts i * 32 + l in s[i], from the logits (or, if `scores_in` is
+// given, those scores as they are). Lanes past E hold -inf (scores_in), 0
+// (sigmoid of -inf) or 0 (softmax).
 template <int NP>
-__device__ __forceinline__ void token_scores(const Resolved& r, int T_, int ksplit,
-                                             const float* __restrict__ logits,
+__device__ __forceinline__ void token_scores(const Resolved& r, const float* __restrict__ logits,
                                              const float* __restrict__ scores_in, int t, int lane,
                                              float (&s)[NP]) {
   const int E = r.E;
@@ -230,21 +248,6 @@ __device__ __forceinline__ void token_scores(const Resolved& r, int T_, int kspl
   for (int i = 0; i < NP; ++i) {
     const int e = i * 32 + lane;
     s[i] = e < E ? row[e] : NEG_INF;
-  }
-  if (!scores_in && ksplit > 1) {
-    // Unrolled so that all partial loads are in flight at once; the adds
-    // still run in ks order.
-#pragma unroll
-    for (int i = 0; i < NP; ++i) {
-      const int e = i * 32 + lane;
-      float p[kSplitK - 1];
-#pragma unroll
-      for (int q = 1; q < kSplitK; ++q)
-        p[q - 1] = (e < E && q < ksplit) ? logits[((int64_t)q * T_ + t) * E + e] : 0.f;
-#pragma unroll
-      for (int q = 1; q < kSplitK; ++q)
-        if (q < ksplit) s[i] += p[q - 1];
-    }
   }
   if (!scores_in) {
     if (r.score_func == KT_SCORE_SIGMOID) {
@@ -275,11 +278,10 @@ __device__ __forceinline__ void token_scores(const Resolved& r, int T_, int kspl
 }
 
 // NP = experts per lane (E <= 32 * NP), a compile-time bound so the per-lane
-// arrays stay in registers. ksplit > 1: `logits` holds ksplit partial sums
-// [ksplit][T][E], added here in order.
+// arrays stay in registers.
 template <int NP>
 __global__ void __launch_bounds__(kSelWarps * 32)
-gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ logits,
+gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
                    const float* __restrict__ scores_in, const float* __restrict__ bias,
                    int32_t* __restrict__ out_idx, float* __restrict__ out_w,
                    int32_t* __restrict__ chunk_counts, int* __restrict__ err) {
@@ -299,7 +301,7 @@ gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
     if (t >= T_) break;
     // Step 1: scores (kept raw for step 5).
     float s[NP], key[NP];
-    token_scores<NP>(r, T_, ksplit, logits, scores_in, t, lane, s);
+    token_scores<NP>(r, logits, scores_in, t, lane, s);
     // Step 2a: selection keys s + b (the bias takes part in the selection only).
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
@@ -403,7 +405,7 @@ gate_select_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
 // the selection's result bit for bit). Same token-to-warp mapping.
 template <int NP>
 __global__ void __launch_bounds__(kSelWarps * 32)
-gate_scores_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ logits,
+gate_scores_kernel(Resolved r, int T_, const float* __restrict__ logits,
                    float* __restrict__ out) {
   pdl_wait();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -411,7 +413,7 @@ gate_scores_kernel(Resolved r, int T_, int ksplit, const float* __restrict__ log
     const int t = blockIdx.x * kPermChunk + tt * kSelWarps + warp;
     if (t >= T_) break;
     float s[NP];
-    token_scores<NP>(r, T_, ksplit, logits, nullptr, t, lane, s);
+    token_scores<NP>(r, logits, nullptr, t, lane, s);
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
       const int e = i * 32 + lane;
@@ -432,13 +434,14 @@ cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, cons
     const int kc = ((r.d + kSplitK - 1) / kSplitK + vn - 1) / vn * vn;
     const dim3 grid((unsigned)((r.E + 31) / 32), kSplitK);
     const dim3 block(kSmallWarps * 32);
+    int* done = err + kGateDoneWord;   // per expert block, zeroed with the error word
     if (bf16)
       (void)launch_pdl(gate_logits_splitk_kernel<__nv_bfloat16>, grid, block, 0, st,
                        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_gate, logits, (int)T,
-                       r.E, r.d, kc);
+                       r.E, r.d, kc, done);
     else
       (void)launch_pdl(gate_logits_splitk_kernel<float>, grid, block, 0, st, (const float*)x,
-                       (const float*)w_gate, logits, (int)T, r.E, r.d, kc);
+                       (const float*)w_gate, logits, (int)T, r.E, r.d, kc, done);
     return cudaGetLastError();
   }
   // Tensor-core logits write 16-byte chunks of fp32 rows of E entries.
@@ -458,11 +461,10 @@ cudaError_t launch_gate_select(const Resolved& r, int64_t T, const float* logits
                                const float* scores_in, const float* bias, int32_t* idx, float* w,
                                int32_t* chunk_counts, int* err, cudaStream_t st) {
   const unsigned grid = (unsigned)((T + kPermChunk - 1) / kPermChunk);
-  const int ks = scores_in ? 1 : gate_logit_splits(r, T);
   const int np = (r.E + 31) / 32;
 #define KT_SELECT(NPV)                                                                         \
   (void)launch_pdl(gate_select_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, \
-                   ks, logits, scores_in, bias, idx, w, chunk_counts, err)
+                   logits, scores_in, bias, idx, w, chunk_counts, err)
   if (np <= 1) KT_SELECT(1);
   else if (np <= 2) KT_SELECT(2);
   else if (np <= 4) KT_SELECT(4);
@@ -479,11 +481,10 @@ namespace ktmoe {
 cudaError_t launch_gate_scores(const Resolved& r, int64_t T, const float* logits, float* scores,
                                cudaStream_t st) {
   const unsigned grid = (unsigned)((T + kPermChunk - 1) / kPermChunk);
-  const int ks = gate_logit_splits(r, T);
   const int np = (r.E + 31) / 32;
 #define KT_SCORES(NPV) \
   (void)launch_pdl(gate_scores_kernel<NPV>, dim3(grid), dim3(kSelWarps * 32), 0, st, r, (int)T, \
-                   ks, logits, scores)
+                   logits, scores)
   if (np <= 1) KT_SCORES(1);
   else if (np <= 2) KT_SCORES(2);
   else if (np <= 4) KT_SCORES(4);

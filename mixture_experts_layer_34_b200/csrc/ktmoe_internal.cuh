@@ -37,6 +37,12 @@ constexpr int kMaxShared = 8;
 constexpr int kSmallTokens = 64;    // up to this many tokens the gate logits are split over K
 constexpr int kGateSplitK = 16;     // ... into this many partial sums
 
+// Words at the start of the workspace that every call zeroes first: [0] the
+// device error word, [1] its detail, [kGateDoneWord, +16) the split-K logits'
+// per-expert-block completion counters.
+constexpr int kGateDoneWord = 8;
+constexpr int kCallWords = kGateDoneWord + kMaxExperts / 32;
+
 // Device error word codes (workspace offset 0). The second int holds a detail.
 constexpr int kDevErrTimeout = 1;
 constexpr int kDevErrBounds = 2;   // checked build only: an index check failed
@@ -87,10 +93,10 @@ struct SlotTable {
 
 // Byte offsets of the workspace's internal buffers.
 struct Layout {
-  size_t err;          // int32[2]
+  size_t err;          // int32[kCallWords], zeroed by every call (256 bytes)
   size_t meta;         // int32[16]: [0] chunks, [1] up tiles, [2] down tiles,
                        // [3] / [4] up / down GEMM tile counters
-  size_t logits;       // fp32 [T, E]
+  size_t logits;       // fp32 [splits][T, E]; the first slot ends as the logits
   size_t idx;          // int32 [T, k] (when the caller gives no output buffer)
   size_t w;            // fp32 [T, k]
   size_t chunk_counts; // int32 [nperm, E]
@@ -122,8 +128,9 @@ Layout make_layout(const Resolved& r, int64_t T);
 // ---------------------------------------------------------------------------
 // Kernel launchers (each returns the cudaError_t of its launch)
 // ---------------------------------------------------------------------------
-// Number of partial-sum blocks the logits region holds (1, or kGateSplitK for
-// calls of at most kSmallTokens tokens).
+// Number of [T, E] slots the logits region holds (1, or kGateSplitK split-K
+// partial sums for calls of at most kSmallTokens tokens; after the logits
+// kernel the first slot holds the logits in either case).
 int gate_logit_splits(const Resolved& r, int64_t T);
 cudaError_t launch_gate_logits(const Resolved& r, int64_t T, const void* x, const void* w_gate,
                                float* logits, int* err, int num_sms, cudaStream_t st);

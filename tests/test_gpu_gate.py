@@ -32,12 +32,9 @@ def _gpu_gate(layer, inp, scores_in=None):
     K.kt_moe_gate(cfg, T, inp["x"], inp["w_gate"], inp["bias"], scores_in, idx, w, ws)
     assert K.kt_moe_check(ws) == K.KT_OK
     lay = K.kt_moe_workspace_layout(cfg, T)
-    ns = lay["logits_splits"]          # partial sums over K, added in order
-    part = ws[lay["logits"]: lay["logits"] + ns * T * layer.n_experts * 4].view(torch.float32)
-    part = part.view(ns, T, layer.n_experts).cpu().numpy()
-    logits = part[0].copy()
-    for k in range(1, ns):
-        logits += part[k]
+    # the first [T, E] slot of the logits region holds the logits after the call
+    logits = ws[lay["logits"]: lay["logits"] + T * layer.n_experts * 4].view(torch.float32)
+    logits = logits.view(T, layer.n_experts).cpu().numpy()
     return idx.cpu().numpy(), w.cpu().numpy(), logits
 
 
