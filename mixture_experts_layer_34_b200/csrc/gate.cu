@@ -212,25 +212,24 @@ gate_logits_splitk_kernel(const T* __restrict__ x, const T* __restrict__ wg,
 constexpr int kSelWarps = 8;
 constexpr unsigned kFull = 0xffffffffu;
 
-struct Best {
-  float key;
-  int idx;
-};
-// Larger key wins; lower index wins a tie.
-__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
-  return ka > kb || (ka == kb && ia < ib);
+// Keys as order-preserving unsigned integers, so that a warp's maximum is one
+// redux.sync: ord(a) < ord(b) iff a < b for non-NaN fp32 a, b (-0 and +0 map
+// to the same value, as they compare equal). 0 lies below every key and marks
+// "no candidate" (an expert already taken).
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if ((b & 0x7fffffffu) == 0) b = 0;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
-__device__ __forceinline__ Best warp_argmax(Best b) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float ok = __shfl_xor_sync(kFull, b.key, off);
-    const int oi = __shfl_xor_sync(kFull, b.idx, off);
-    if (better(ok, oi, b.key, b.idx)) {
-      b.key = ok;
-      b.idx = oi;
-    }
-  }
-  return b;
+__device__ __forceinline__ float key_of(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+// Warp argmax over one (key, index) candidate per lane: the largest key, and
+// among equal keys the lowest index (the tie rule of both top-k's). Returns the
+// index; `best` gets the key.
+__device__ __forceinline__ int warp_argmax(uint32_t u, int idx, uint32_t& best) {
+  best = __reduce_max_sync(kFull, u);
+  return (int)__reduce_min_sync(kFull, u == best ? (unsigned)idx : 0xffffffffu);
 }
 
 // Gate step 1 and the score function for token t, one warp: lane l gets the
@@ -300,86 +299,110 @@ gate_select_kernel(Resolved r, int T_, const float* __restrict__ logits,
     const int t = blockIdx.x * kPermChunk + tt * kSelWarps + warp;
     if (t >= T_) break;
     // Step 1: scores (kept raw for step 5).
-    float s[NP], key[NP];
+    float s[NP];
     token_scores<NP>(r, logits, scores_in, t, lane, s);
-    // Step 2a: selection keys s + b (the bias takes part in the selection only).
+    // Step 2a: selection keys s + b (the bias takes part in the selection only),
+    // as ordered integers (NaN keys count as -inf: indices stay valid).
+    const uint32_t kNegInf = ord_key(NEG_INF);
+    uint32_t ku[NP];
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
       const int e = i * 32 + lane;
       if (e < E) {
-        key[i] = r.has_bias ? __fadd_rn(s[i], bias[e]) : s[i];
-        if (key[i] != key[i]) key[i] = NEG_INF;   // NaN input: keep indices valid
+        const float kv = r.has_bias ? __fadd_rn(s[i], bias[e]) : s[i];
+        ku[i] = kv != kv ? kNegInf : ord_key(kv);
       } else {
-        key[i] = NEG_INF;
+        ku[i] = 0;
       }
     }
     // Steps 2b-3: group scores, keep topk_groups groups, mask the rest.
     if (G > 1) {
-#pragma unroll
-      for (int i = 0; i < NP; ++i) {
-        const int e = i * 32 + lane;
-        if (e < E) skey[warp][e] = key[i];
-      }
-      __syncwarp();
+      // Group score of group g in lane g: the group max (no bias) or the sum
+      // of its two largest keys, larger first (bias).
       float gsc = NEG_INF;
-      if (lane < G) {
-        const float* kg = &skey[warp][lane * gs];
-        if (r.group_score == KT_GROUP_TOP2SUM) {
-          float b1 = NEG_INF, b2 = NEG_INF;
-          for (int i = 0; i < gs; ++i) {
-            const float v = kg[i];
-            if (v > b1) {
-              b2 = b1;
-              b1 = v;
-            } else if (v > b2) {
-              b2 = v;
-            }
+      const bool top2 = r.group_score == KT_GROUP_TOP2SUM;
+      if (gs == 32) {
+        // Group g is slot g of every lane: warp reductions.
+#pragma unroll
+        for (int g = 0; g < NP; ++g) {
+          if (g >= G) break;
+          const uint32_t m1 = __reduce_max_sync(kFull, ku[g]);
+          float v = key_of(m1);
+          if (top2) {
+            const bool dup = __popc(__ballot_sync(kFull, ku[g] == m1)) > 1;
+            const uint32_t m2 = dup ? m1 : __reduce_max_sync(kFull, ku[g] == m1 ? 0u : ku[g]);
+            v = __fadd_rn(v, key_of(m2));
           }
-          gsc = __fadd_rn(b1, b2);
-        } else {
-          for (int i = 0; i < gs; ++i) gsc = fmaxf(gsc, kg[i]);
+          if (lane == g) gsc = v;
         }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+          const int e = i * 32 + lane;
+          if (e < E) skey[warp][e] = key_of(ku[i]);
+        }
+        __syncwarp();
+        if (lane < G) {
+          const float* kg = &skey[warp][lane * gs];
+          if (top2) {
+            float b1 = NEG_INF, b2 = NEG_INF;
+            for (int i = 0; i < gs; ++i) {
+              const float v = kg[i];
+              if (v > b1) {
+                b2 = b1;
+                b1 = v;
+              } else if (v > b2) {
+                b2 = v;
+              }
+            }
+            gsc = __fadd_rn(b1, b2);
+          } else {
+            for (int i = 0; i < gs; ++i) gsc = fmaxf(gsc, kg[i]);
+          }
+        }
+        __syncwarp();
       }
-      __syncwarp();
       unsigned kept = 0;
-      bool taken = lane >= G;
+      uint32_t gu = lane < G ? ord_key(gsc != gsc ? NEG_INF : gsc) : 0u;
       for (int rr = 0; rr < r.TG; ++rr) {
-        Best b = warp_argmax(Best{taken ? NEG_INF : gsc, taken ? 0x7fffffff : lane});
-        kept |= 1u << b.idx;
-        if (lane == b.idx) taken = true;
+        uint32_t best;
+        const int g = warp_argmax(gu, lane, best);
+        kept |= 1u << g;
+        if (lane == g) gu = 0;
       }
 #pragma unroll
       for (int i = 0; i < NP; ++i) {
         const int e = i * 32 + lane;
-        if (e < E && !((kept >> (e / gs)) & 1u)) key[i] = NEG_INF;
+        if (e < E && !((kept >> (e / gs)) & 1u)) ku[i] = kNegInf;
       }
     }
     // Step 4: global top-k over the masked keys; lane j keeps slot j.
     int my_e = 0;
     float my_s = 0.f;
     for (int j = 0; j < k; ++j) {
-      Best lb{NEG_INF, 0x7fffffff};
+      // this lane's best key (strict > keeps the lowest index among equals)
+      uint32_t lu = 0;
+      int li = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < NP; ++i) {
-        const int e = i * 32 + lane;
-        if (e < E && better(key[i], e, lb.key, lb.idx)) {
-          lb.key = key[i];
-          lb.idx = e;
+      for (int i = 0; i < NP; ++i)
+        if (ku[i] > lu) {
+          lu = ku[i];
+          li = i * 32 + lane;
         }
-      }
-      const Best b = warp_argmax(lb);
+      uint32_t best;
+      const int b = warp_argmax(lu, li, best);
       float won_s = 0.f;
-      if (lane == (b.idx & 31)) {
+      if (lane == (b & 31)) {
 #pragma unroll
         for (int i = 0; i < NP; ++i)
-          if (i == (b.idx >> 5)) {
+          if (i == (b >> 5)) {
             won_s = s[i];
-            key[i] = __int_as_float(0x7fffffff);  // NaN: never wins again
+            ku[i] = 0;                  // taken: never wins again
           }
       }
-      won_s = __shfl_sync(kFull, won_s, b.idx & 31);
+      won_s = __shfl_sync(kFull, won_s, b & 31);
       if (lane == j) {
-        my_e = b.idx;
+        my_e = b;
         my_s = won_s;
       }
     }
