@@ -21,6 +21,8 @@ namespace ktmoe {
 namespace {
 
 constexpr int kScanThreads = 1024;
+// Scatter CTA: 16 warps over one 32-token chunk (two tokens' row copies per warp).
+constexpr int kScatterThreads = 512;
 
 // Exclusive scan over n <= kScanThreads ints in shared memory; returns total.
 __device__ int block_exclusive_scan(int* buf, int n) {
@@ -146,13 +148,42 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
   const int NG = E + S;
   // Per-expert totals over the chunks; shared experts hold tokens [sb, se) (all
   // T unless the caller splits them); routed experts computed elsewhere (slot
-  // -1) hold none.
+  // -1) hold none. The chunks of each routed expert are cut into P segments,
+  // one thread each (thread e + p*E takes segment p of expert e), so that a
+  // long prefill's count loads run P-wide; each thread keeps 8 loads in flight.
+  __shared__ int seg[kScanThreads];
+  constexpr int kBatch = 8;
+  const int P = E > 0 ? max(1, min(32, kScanThreads / E)) : 1;
+  const int seg_len = (nperm + P - 1) / P;
+  const int se_e = tid % max(E, 1), se_p = tid / max(E, 1);
+  const bool seg_thread = E > 0 && se_p < P;
+  const int c_lo = min(nperm, se_p * seg_len), c_hi = min(nperm, c_lo + seg_len);
+  if (seg_thread) {
+    int run = 0;
+    if (tab.slot[se_e] >= 0) {
+      for (int c0 = c_lo; c0 < c_hi; c0 += kBatch) {
+        int v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          v[u] = c0 + u < c_hi ? chunk_counts[(int64_t)(c0 + u) * E + se_e] : 0;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) run += v[u];
+      }
+    }
+    seg[tid] = run;
+  }
+  __syncthreads();
   if (tid < NG) {
     int run = 0;
-    if (tid >= E)
+    if (tid >= E) {
       run = se - sb;
-    else if (tab.slot[tid] >= 0)
-      for (int c = 0; c < nperm; ++c) run += chunk_counts[(int64_t)c * E + tid];
+    } else {
+      for (int q = 0; q < P; ++q) {   // segment sums -> exclusive prefix per segment
+        const int v = seg[q * E + tid];
+        seg[q * E + tid] = run;
+        run += v;
+      }
+    }
     tot[tid] = run;
     rows0[tid] = run;
     counts[tid] = run;
@@ -164,12 +195,20 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
   __syncthreads();
   if (tid < NG) offsets[tid] = rows0[tid];
   if (tid == 0) offsets[NG] = T_ * k + S * T_;
-  // Chunk bases (global row of each permutation chunk's first row per expert).
-  if (tid < E) {
-    int run = rows0[tid];
-    for (int c = 0; c < nperm; ++c) {
-      chunk_base[(int64_t)c * E + tid] = run;
-      run += chunk_counts[(int64_t)c * E + tid];
+  // Chunk bases (global row of each permutation chunk's first row per expert),
+  // by the same segments.
+  if (seg_thread) {
+    int run = rows0[se_e] + seg[tid];
+    for (int c0 = c_lo; c0 < c_hi; c0 += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        v[u] = c0 + u < c_hi ? chunk_counts[(int64_t)(c0 + u) * E + se_e] : 0;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (c0 + u < c_hi) chunk_base[(int64_t)(c0 + u) * E + se_e] = run;
+        run += v[u];
+      }
     }
   }
   // GEMM chunks of chunk_rows rows and the two tile lists.
@@ -209,7 +248,7 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
 enum { kNoCopy = 0, kCopyBf16 = 1, kCopyF8 = 2 };
 
 template <int kMode>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kScatterThreads)
 permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
                        const __grid_constant__ SlotTable tab,
                        int sb, int se,
@@ -339,7 +378,7 @@ cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, c
   float* rw = reinterpret_cast<float*>(ws + L.row_weight);
   const int32_t* base = I32(L.chunk_base);
   if (r.fp8)
-    (void)launch_pdl(permute_scatter_kernel<kCopyF8>, grid, dim3(256), 0, st, r.E, r.S, (int)T,
+    (void)launch_pdl(permute_scatter_kernel<kCopyF8>, grid, dim3(kScatterThreads), 0, st, r.E, r.S, (int)T,
                      r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
                      I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw,
                      reinterpret_cast<const uint4*>(ws + L.xq),
@@ -347,13 +386,13 @@ cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, c
                      reinterpret_cast<const uint8_t*>(ws + L.xs),
                      reinterpret_cast<uint8_t*>(ws + L.tok_sf), (int)L.max_chunks, I32(L.err));
   else if (r.dtype == KT_DTYPE_BF16)
-    (void)launch_pdl(permute_scatter_kernel<kCopyBf16>, grid, dim3(256), 0, st, r.E, r.S, (int)T,
+    (void)launch_pdl(permute_scatter_kernel<kCopyBf16>, grid, dim3(kScatterThreads), 0, st, r.E, r.S, (int)T,
                      r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
                      I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw,
                      reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(ws + L.xperm),
                      nullptr, nullptr, (int)L.max_chunks, I32(L.err));
   else
-    (void)launch_pdl(permute_scatter_kernel<kNoCopy>, grid, dim3(256), 0, st, r.E, r.S, (int)T,
+    (void)launch_pdl(permute_scatter_kernel<kNoCopy>, grid, dim3(kScatterThreads), 0, st, r.E, r.S, (int)T,
                      r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
                      I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr,
                      nullptr, (int)L.max_chunks, I32(L.err));
