@@ -214,6 +214,26 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
                : "memory");
 }
+// The same arrive without release semantics: it does not wait until this
+// thread's earlier memory operations are visible across the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t caddr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
+               : "memory");
+}
+// Arrive on this CTA's barrier, ordering this thread's earlier writes to its
+// own shared memory before the arrive (CTA scope).
+__device__ __forceinline__ void mbar_arrive_local(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// Arrive on a barrier at a shared::cluster address and raise its expected
+// transaction bytes by `bytes` (completed by st.async below).
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t caddr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+                   caddr),
+               "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -409,8 +429,22 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // negative g the denominator overflows and the result is 0 (silu -> 0 there).
 __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-__device__ __forceinline__ void st_cluster_s32(uint32_t caddr, int v) {
-  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
+// Asynchronous stores into a peer CTA's shared memory, each completing its
+// bytes on the peer's barrier `bar` (shared::cluster addresses; 16- and 8-byte
+// aligned).
+__device__ __forceinline__ void st_async_v4(uint32_t caddr, int a, int b, int c, int d,
+                                            uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.s32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(caddr),
+      "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t caddr, int a, int b, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.s32 [%0], {%1, %2}, [%3];" ::
+                   "r"(caddr),
+               "r"(a), "r"(b), "r"(bar)
+               : "memory");
 }
 
 __device__ __forceinline__ void read_slot(const int* slot, Chunk& ch, int& ft, int& ci) {
@@ -597,14 +631,15 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           slot[4] = f;
           slot[5] = cidx;
           const uint32_t peer_slot = map_to_cta(smem_u32(slot), 1);
-          st_cluster_s32(peer_slot, c.group);
-          st_cluster_s32(peer_slot + 4, c.row0);
-          st_cluster_s32(peer_slot + 8, c.nrows);
-          st_cluster_s32(peer_slot + 12, c.src_row0);
-          st_cluster_s32(peer_slot + 16, f);
-          st_cluster_s32(peer_slot + 20, cidx);
-          mbar_arrive_cluster(map_to_cta(smem_u32(&sched_full[sslot]), 0));
-          mbar_arrive_cluster(map_to_cta(smem_u32(&sched_full[sslot]), 1));
+          // The odd CTA's copy travels by st.async and completes its 24 bytes
+          // on that CTA's barrier, so no release (which would wait for this
+          // thread's copies and remote stores in flight) sits between the last
+          // stage of one tile and the first copies of the next.
+          const uint32_t peer_full = map_to_cta(smem_u32(&sched_full[sslot]), 1);
+          st_async_v4(peer_slot, c.group, c.row0, c.nrows, c.src_row0, peer_full);
+          st_async_v2(peer_slot + 16, f, cidx, peer_full);
+          mbar_arrive_expect_tx_cluster(peer_full, 24u);
+          mbar_arrive_local(&sched_full[sslot]);
         } else {
           if (!mbar_wait(&sched_full[sslot], sphase, err, 6 + 8 * kKind)) {
             ok = false;
@@ -614,7 +649,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
         Chunk ch;
         int ft, ci;
         read_slot(sched_info + 8 * sslot, ch, ft, ci);
-        if (!leader) mbar_arrive_cluster(map_to_cta(smem_u32(&sched_empty[sslot]), 0));
+        const uint32_t empty_leader = map_to_cta(smem_u32(&sched_empty[sslot]), 0);
+        if (!leader && ch.group < 0) mbar_arrive_cluster(empty_leader);
         if (++sslot == kSched) {
           sslot = 0;
           sphase ^= 1u;
@@ -716,6 +752,10 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
             if (kb == nk / 2) claim();
             if (kb == nk - 1) fetch();
           }
+          // The slot's values are in the copies just issued (their coordinates
+          // needed the loads), so the slot is free: a relaxed arrive, which
+          // does not wait for the copies themselves.
+          if (!leader && kb == 0) mbar_arrive_cluster_relaxed(empty_leader);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
@@ -756,7 +796,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
         Chunk ch;
         int ft, ci;
         read_slot(sched_info + 8 * sslot, ch, ft, ci);
-        mbar_arrive_cluster(smem_u32(&sched_empty[sslot]));
+        const uint32_t empty_own = smem_u32(&sched_empty[sslot]);
+        if (ch.group < 0) mbar_arrive_cluster(empty_own);
         if (++sslot == kSched) {
           sslot = 0;
           sphase ^= 1u;
@@ -812,6 +853,9 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
           }
           mma_commit_both(smem_u32(&empty_bar[stage]));
           issued_any = true;
+          // The slot's values are in the MMAs just issued: relaxed arrive (a
+          // release would wait for the MMAs in flight).
+          if (kb == 0) mbar_arrive_cluster_relaxed(empty_own);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
