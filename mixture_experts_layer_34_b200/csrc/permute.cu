@@ -5,12 +5,14 @@
 // Here those gathers become one deterministic counting sort:
 //   counts   per 32-token chunk and expert (written by the gate-select CTAs),
 //   scan     per expert over chunks, then over experts -> row offsets, plus the
-//            chunk lists the grouped GEMMs walk (shared experts appended as
-//            always-selected groups of all T tokens),
+//            GEMM chunks (shared experts appended as always-selected groups of
+//            all T tokens),
 //   scatter  rank of (t, j) inside its expert = number of earlier tokens of the
 //            same chunk that chose that expert (bit mask + popc), so rows of one
 //            expert are in ascending token order; bf16 layers also copy x into
-//            the permuted activation buffer.
+//            the permuted activation buffer. The scatter CTAs also fill the two
+//            grouped GEMMs' tile lists, which the one-CTA scan would take tens
+//            of microseconds to write for a long prefill.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -93,40 +95,29 @@ __device__ __forceinline__ int merged_pos_l(int j, int nh, int nl) {
   return j + (int)(c < nh ? c : nh);
 }
 
-// Fill one GEMM's tile list: experts with at least kHeavyRows rows (compute-
-// bound) form stream H, the others (weight-streaming) stream L; each stream is
-// ordered per group by tile_of, and the two are merged proportionally so that
-// the pairs running at any moment mix both kinds.
-__device__ void fill_tiles(int2* __restrict__ tiles, int F, int NG, const int* cb, int* hb,
-                           int* lb, const int* tot, int* err) {
-  const int tid = threadIdx.x;
-  if (tid < NG) {
-    const int nt = (cb[tid + 1] - cb[tid]) * F;
-    const bool heavy = tot[tid] >= kHeavyRows;
-    hb[tid] = heavy ? nt : 0;
-    lb[tid] = heavy ? 0 : nt;
-  }
-  __syncthreads();
-  const int nh = block_exclusive_scan(hb, NG);
-  const int nl = block_exclusive_scan(lb, NG);
-  if (tid == 0) {
-    hb[NG] = nh;
-    lb[NG] = nl;
-  }
-  __syncthreads();
-  for (int i = tid; i < nh; i += blockDim.x) {
-    const int g = find_group(hb, NG, i);
+// Fill one GEMM's tile list with all threads of the grid: groups with at least
+// kHeavyRows rows (compute-bound) form stream H, the others (weight-streaming)
+// stream L; each stream is ordered per group by tile_of, and the two are merged
+// proportionally so that the pairs running at any moment mix both kinds. cb is
+// the groups' first GEMM chunk (cb[NG] = all chunks), hcb / lcb the exclusive
+// prefix of their chunks in H / L; F feature tiles per chunk.
+__device__ void fill_tiles(int2* __restrict__ tiles, int F, int NG, const int* cb, const int* hcb,
+                           const int* lcb, int* err) {
+  const int nh = F * hcb[NG], nl = F * lcb[NG];
+  const int stride = gridDim.x * gridDim.y * blockDim.x;
+  const int t0 = (blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int i = t0; i < nh; i += stride) {
+    const int g = find_group(hcb, NG, i / F);
     const int pos = merged_pos_h(i, nh, nl);
     if (in_range(pos, 0, nh + nl, err, 104))
-      tiles[pos] = tile_of(i - hb[g], cb[g + 1] - cb[g], F, cb[g]);
+      tiles[pos] = tile_of(i - F * hcb[g], cb[g + 1] - cb[g], F, cb[g]);
   }
-  for (int j = tid; j < nl; j += blockDim.x) {
-    const int g = find_group(lb, NG, j);
+  for (int j = t0; j < nl; j += stride) {
+    const int g = find_group(lcb, NG, j / F);
     const int pos = merged_pos_l(j, nh, nl);
     if (in_range(pos, 0, nh + nl, err, 104))
-      tiles[pos] = tile_of(j - lb[g], cb[g + 1] - cb[g], F, cb[g]);
+      tiles[pos] = tile_of(j - F * lcb[g], cb[g + 1] - cb[g], F, cb[g]);
   }
-  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kScanThreads)
@@ -134,16 +125,13 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
                     const __grid_constant__ SlotTable tab, int n_local, int sb, int se,
                     const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_base,
                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                    Chunk* __restrict__ chunks, int2* __restrict__ tiles_up,
-                    int2* __restrict__ tiles_dn, int32_t* __restrict__ meta,
+                    Chunk* __restrict__ chunks, int32_t* __restrict__ meta,
                     int32_t* __restrict__ gchunk0, int max_chunks, int* __restrict__ err) {
   pdl_wait();
   constexpr int NGMAX = kMaxExperts + kMaxShared;
   __shared__ int tot[NGMAX];
   __shared__ int rows0[NGMAX];
   __shared__ int cb[NGMAX + 1];
-  __shared__ int hb[NGMAX + 1];
-  __shared__ int lb[NGMAX + 1];
   const int tid = threadIdx.x;
   const int NG = E + S;
   // Per-expert totals over the chunks; shared experts hold tokens [sb, se) (all
@@ -211,7 +199,7 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
       }
     }
   }
-  // GEMM chunks of chunk_rows rows and the two tile lists.
+  // GEMM chunks of chunk_rows rows (their tile lists are the scatter's).
   if (tid < NG) cb[tid] = (tot[tid] + chunk_rows - 1) / chunk_rows;
   __syncthreads();
   const int n_chunks = block_exclusive_scan(cb, NG);
@@ -240,8 +228,6 @@ permute_scan_kernel(int E, int S, int T_, int k, int nperm, int Fu, int Fd, int 
     const int src0 = g < E ? rows0[g] : sb;
     chunks[i] = Chunk{slot, row0 + r, min(chunk_rows, tot[g] - r), src0 + r};
   }
-  fill_tiles(tiles_up, Fu, NG, cb, hb, lb, tot, err);
-  fill_tiles(tiles_dn, Fd, NG, cb, hb, lb, tot, err);
 }
 
 // Copy modes of the scatter.
@@ -258,10 +244,62 @@ permute_scatter_kernel(int E, int S, int T_, int k, int d, int chunk_rows,
                        int32_t* __restrict__ tok_of, float* __restrict__ row_weight,
                        const uint4* __restrict__ x, uint4* __restrict__ xperm,
                        const uint8_t* __restrict__ xs, uint8_t* __restrict__ tok_sf,
-                       int max_chunks, int* __restrict__ err) {
+                       int max_chunks, const int32_t* __restrict__ counts,
+                       const int32_t* __restrict__ meta, int Fu, int Fd,
+                       int2* __restrict__ tiles_up, int2* __restrict__ tiles_dn,
+                       int* __restrict__ err) {
   pdl_wait();
   __shared__ uint32_t mask[kMaxExperts];
   __shared__ int srow[kPermChunk * kMaxTopk];
+  // The grouped GEMMs' tile lists (none when the scan found that the chunks do
+  // not fit the workspace): every CTA builds the groups' chunk prefixes in H and
+  // L from the scan's chunk starts and row counts, then fills its share.
+  {
+    constexpr int NGMAX = kMaxExperts + kMaxShared;
+    __shared__ int s_cb[NGMAX + 1], s_hcb[NGMAX + 1], s_lcb[NGMAX + 1];
+    const int NG = E + S;
+    if (meta[1] > 0) {
+      for (int g = threadIdx.x; g < NG; g += blockDim.x) s_cb[g] = gchunk0[g];
+      if (threadIdx.x == 0) s_cb[NG] = meta[0];
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        // Warp 0: lane l takes a run of consecutive groups; exclusive prefix of
+        // the heavy and light chunk counts over the runs.
+        const int lane = threadIdx.x;
+        const int per = (NG + 31) / 32;
+        const int g0 = min(NG, lane * per), g1 = min(NG, g0 + per);
+        int h = 0, l = 0;
+        for (int g = g0; g < g1; ++g) {
+          const int nc = s_cb[g + 1] - s_cb[g];
+          if (counts[g] >= kHeavyRows) h += nc; else l += nc;
+        }
+        int hi = h, li = l;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int ho = __shfl_up_sync(0xffffffffu, hi, off);
+          const int lo = __shfl_up_sync(0xffffffffu, li, off);
+          if (lane >= off) {
+            hi += ho;
+            li += lo;
+          }
+        }
+        int hrun = hi - h, lrun = li - l;
+        for (int g = g0; g < g1; ++g) {
+          const int nc = s_cb[g + 1] - s_cb[g];
+          s_hcb[g] = hrun;
+          s_lcb[g] = lrun;
+          if (counts[g] >= kHeavyRows) hrun += nc; else lrun += nc;
+        }
+        if (lane == 31) {
+          s_hcb[NG] = hi;
+          s_lcb[NG] = li;
+        }
+      }
+      __syncthreads();
+      fill_tiles(tiles_up, Fu, NG, s_cb, s_hcb, s_lcb, err);
+      fill_tiles(tiles_dn, Fd, NG, s_cb, s_hcb, s_lcb, err);
+    }
+  }
   const int c = blockIdx.x;
   const int t0 = c * kPermChunk;
   const int nt = min(kPermChunk, T_ - t0);
@@ -360,13 +398,12 @@ cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, c
                            char* ws, const int32_t* idx, const float* w, const void* x,
                            cudaStream_t st) {
   auto I32 = [&](size_t off) { return reinterpret_cast<int32_t*>(ws + off); };
+  const int Fu = (r.I + 127) / 128, Fd = (r.d + 255) / 256;   // feature tiles per chunk
   (void)launch_pdl(permute_scan_kernel, dim3(1), dim3(kScanThreads), 0, st, r.E, r.S, (int)T, r.k,
-                   (int)L.nperm, (r.I + 127) / 128, (r.d + 255) / 256, r.chunk_rows, tab,
+                   (int)L.nperm, Fu, Fd, r.chunk_rows, tab,
                    r.n_local, r.sb, r.se, I32(L.chunk_counts), I32(L.chunk_base), I32(L.counts),
-                   I32(L.offsets), reinterpret_cast<Chunk*>(ws + L.chunks),
-                   reinterpret_cast<int2*>(ws + L.tiles_up),
-                   reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.meta), I32(L.gchunk0),
-                   (int)L.max_chunks, I32(L.err));
+                   I32(L.offsets), reinterpret_cast<Chunk*>(ws + L.chunks), I32(L.meta),
+                   I32(L.gchunk0), (int)L.max_chunks, I32(L.err));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // Few chunks (a decode step): split each chunk's row copies over column
@@ -384,18 +421,24 @@ cudaError_t launch_permute(const Resolved& r, const SlotTable& tab, int64_t T, c
                      reinterpret_cast<const uint4*>(ws + L.xq),
                      reinterpret_cast<uint4*>(ws + L.xperm),
                      reinterpret_cast<const uint8_t*>(ws + L.xs),
-                     reinterpret_cast<uint8_t*>(ws + L.tok_sf), (int)L.max_chunks, I32(L.err));
+                     reinterpret_cast<uint8_t*>(ws + L.tok_sf), (int)L.max_chunks, I32(L.counts), I32(L.meta), Fu, Fd,
+                     reinterpret_cast<int2*>(ws + L.tiles_up),
+                     reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.err));
   else if (r.dtype == KT_DTYPE_BF16)
     (void)launch_pdl(permute_scatter_kernel<kCopyBf16>, grid, dim3(kScatterThreads), 0, st, r.E, r.S, (int)T,
                      r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
                      I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw,
                      reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(ws + L.xperm),
-                     nullptr, nullptr, (int)L.max_chunks, I32(L.err));
+                     nullptr, nullptr, (int)L.max_chunks, I32(L.counts), I32(L.meta), Fu, Fd,
+                     reinterpret_cast<int2*>(ws + L.tiles_up),
+                     reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.err));
   else
     (void)launch_pdl(permute_scatter_kernel<kNoCopy>, grid, dim3(kScatterThreads), 0, st, r.E, r.S, (int)T,
                      r.k, r.d, r.chunk_rows, tab, r.sb, r.se, idx, w, base, I32(L.offsets),
                      I32(L.gchunk0), I32(L.row_of), I32(L.tok_of), rw, nullptr, nullptr, nullptr,
-                     nullptr, (int)L.max_chunks, I32(L.err));
+                     nullptr, (int)L.max_chunks, I32(L.counts), I32(L.meta), Fu, Fd,
+                     reinterpret_cast<int2*>(ws + L.tiles_up),
+                     reinterpret_cast<int2*>(ws + L.tiles_down), I32(L.err));
   return cudaGetLastError();
 }
 
