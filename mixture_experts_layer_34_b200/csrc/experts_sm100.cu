@@ -542,7 +542,8 @@ grouped_gemm_kernel(const __grid_constant__ TmaMaps maps, const GemmArgs args) {
     }
     mbar_init(drain_bar, 1);
     for (int i = 0; i < kSched; ++i) {
-      mbar_init(&sched_full[i], 1);     // one arrival: the even CTA's producer
+      mbar_init(&sched_full[i], 1);     // one arrival: the even CTA's producer (on the
+                                        // odd CTA, plus the slot's 24 bytes as transactions)
       mbar_init(&sched_empty[i], kSchedConsumers);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
