@@ -190,3 +190,79 @@ def test_coverage_tokens_reach_every_chunk():
         for c0 in range(0, len(mine), 256):
             assert set(mine[c0:c0 + 256]) & set(toks), (e, c0)
         assert mine[-1] in toks
+
+
+PEAKS = {"bf16_tflops": 1666.8, "bf16_tflops_sustained": 1391.0, "hbm_gbs": 6551.0,
+         "source": "measured"}
+
+
+def test_tensor_roofline_takes_the_clock_of_its_own_region():
+    """achieved = FLOPs / event time; the peak is the burst figure scaled to the
+    median clock of the kernel's region (the run's median when the region has no
+    samples); the fraction can be recomputed from the entry alone."""
+    clk = {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "regions": {"pre": {"sm_mhz": 1300.0}}}
+    e = bench.tensor_roofline("up", 4.33e12, 4.5, PEAKS, clk, "pre")
+    assert e["achieved"] == pytest.approx(4.33e12 / 4.5e-3 / 1e12, abs=0.05)
+    assert e["peak"] == pytest.approx(1666.8 * 1300 / 1965, abs=0.05)
+    assert e["peak_clock_mhz"] == 1300.0 and e["sm_max_mhz"] == 1965.0
+    assert e["frac"] == pytest.approx(e["achieved"] / e["peak"], abs=1e-3)
+    assert e["frac_of_sustained"] == pytest.approx(e["achieved"] / 1391.0, abs=1e-3)
+    # no samples in the region: the run's median (within 5% of max: burst)
+    e = bench.tensor_roofline("up", 4.33e12, 4.5, PEAKS, clk, "other")
+    assert e["peak"] == pytest.approx(1666.8) and e["peak_clock_mhz"] == 1900.0
+    # another dtype: its nominal ratio times the measured bf16 figure
+    e = bench.tensor_roofline("up", 4.33e12, 4.5, PEAKS, clk, "other", mult=2.0)
+    assert e["peak"] == pytest.approx(2 * 1666.8) and "x 2" in e["peak_source"]
+
+
+def test_hbm_roofline_and_layer_fractions():
+    e = bench.hbm_roofline("up", 2.64e9, 0.4, PEAKS, traffic_bytes=2645930837)
+    assert e["achieved"] == pytest.approx(6600.0) and e["frac"] == pytest.approx(6600 / 6551, abs=1e-4)
+    assert e["traffic"] == 2645930837 and e["unit"] == "GB/s"
+    layer = W.BY_NAME["v3_prefill_T8192_zipf"]
+    res = {"ms": 16.0, "work": {"flops_layer": 6.524e12, "bytes_layer": 22.6e9}}
+    f = bench.layer_fracs(layer, res, 2, PEAKS, 1300.0, 1965.0)    # 8 ms per step
+    assert f["layer_tflops"] == pytest.approx(6.524e12 / 8e-3 / 1e12, abs=0.05)
+    assert f["layer_hbm_frac"] == pytest.approx(22.6e9 / 8e-3 / 1e9 / 6551, abs=1e-4)
+    assert f["layer_tensor_frac"] == pytest.approx(
+        6.524e12 / 8e-3 / 1e12 / (1666.8 * 1300 / 1965), abs=1e-4)
+    mx = W.BY_NAME["v3_prefill_T8192_zipf_mxfp8"]
+    g = bench.layer_fracs(mx, res, 2, PEAKS, 1965.0, 1965.0)
+    assert g["layer_tensor_frac"] == pytest.approx(6.524e12 / 8e-3 / 1e12 / (2 * 1666.8), abs=1e-4)
+
+
+class _DoneProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def test_clock_sampler_assigns_samples_to_regions(tmp_path, monkeypatch):
+    """stop() on a recorded nvidia-smi log: the median clock of the loaded
+    samples, the throttle reasons seen, and per marked region the median of the
+    samples stamped inside it (widened by one sampling period)."""
+    import datetime
+    monkeypatch.setattr(bench.time, "sleep", lambda s: None)
+    t0 = datetime.datetime(2026, 12, 2, 16, 0, 0)
+    rows = []
+    for i, (mhz, cap) in enumerate([(1965, "Not Active")] * 4 + [(1300, "Active")] * 5
+                                   + [(1965, "Not Active")] * 3):
+        ts = (t0 + datetime.timedelta(milliseconds=50 * i)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        rows.append(f"0, {mhz}, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, {cap}, {ts}")
+    path = tmp_path / "clk.csv"
+    path.write_text("\n".join(rows) + "\n")
+    cs = bench.ClockSampler(0)
+    cs.path, cs.proc = str(path), _DoneProc()
+    base = t0.timestamp()
+    cs.windows = {"capped": [base + 0.25, base + 0.40], "open": [base + 0.5, None]}
+    out = cs.stop()
+    assert out["sm_max_mhz"] == 1965.0 and out["samples"] == 12
+    assert out["reasons"] == ["sw_power_cap"]
+    assert out["sm_mhz"] == 1965.0              # 7 of 12 loaded samples at full clock
+    reg = out["regions"]
+    assert set(reg) == {"capped"}               # an unclosed window is dropped
+    # [0.25, 0.40] s widened to [0.20, 0.45]: the five capped samples and one at full clock
+    assert reg["capped"]["sm_mhz"] == 1300.0 and reg["capped"]["samples"] == 6
+    assert not path.exists()
